@@ -1,0 +1,24 @@
+"""Plain, slow CPU oracle of the fast-weight chunk scan — TEST INFRASTRUCTURE ONLY.
+
+This package is the reference the CUDA path is checked against. It is written from
+the pages' descriptions of the method, in float64 with numpy, step by step in the
+pages' order, with no blocking, fusion or reordering beyond the definitions:
+
+* :mod:`oracle.inplace` — In-Place TTT apply-then-update scan with the Hebbian,
+  LM-aligned update and the Conv1D + Wtarget target (In-Place Test-Time Training,
+  §2 "Wdown as fast weight", §3 "apply first, update later", §4 "predict the next
+  token", §6 "context parallelism").
+* :mod:`oracle.linear` — TTT-Linear mini-batch gradient scan (TTT layers page,
+  "hidden state is itself a model" and the DeltaNet remark).
+* :mod:`oracle.gate` — SR-TTT surprisal gate and residual cache (SR-TTT technical
+  summary, §2.1 "Surprisal Filter" and "Residual Cache").
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline leg may
+import it. The product path (the C-ABI library and its Python binding) never does;
+it shares no code, header or constant with this package.
+
+Every function here is pinned by ``tests/test_oracle_*.py`` to closed forms,
+hand-derived worked examples (``tests/golden/``), special cases and brute force.
+"""
+
+from . import gate, inplace, linear  # noqa: F401
