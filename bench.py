@@ -1,0 +1,452 @@
+#!/usr/bin/env python
+"""Benchmark of the fast-weight chunk scan on B200 (one JSON line on rank 0).
+
+Default workload: the TTT-Linear mini-batch scan, B=8 sequences x H=12 heads of width 64,
+T=2048, inner mini-batch 16 (TTT layers page). A step is one ttt_chunk_scan over the whole
+batch with inputs resident in HBM; the state is reset (ttt_state_reset, untimed) before
+each step so every step scans from W0. L2 is flushed (a 512 MB write) before each timed
+step. The other four workloads (In-Place fp32, In-Place 4B-class, In-Place 128k with fused
+target, SR-TTT gate) are measured the same way and reported under "workloads".
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--workload NAME]
+                  [--only-main]
+
+With N > 1 (launched by torch.distributed.run) every rank runs an independent replica of
+the workload (the (sequence, head) problems are independent; no collective on the data
+path): scaling is weak and value = all ranks' tokens / the slowest rank's time.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from gen import workloads as wl  # noqa: E402
+
+METRIC = "fast-weight scan tokens/s and TFLOP/s per layer on 1 B200; % of BF16/HBM roofline"
+MAIN = wl.LINEAR_GD.name
+
+
+def load_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "sm_max_mhz": d.get("sm_max_mhz", 1965.0), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0,
+            "source": "fallback"}
+
+
+# --------------------------------------------------------------------------------------------
+# algorithmic work per workload (flops, compulsory bytes)
+# --------------------------------------------------------------------------------------------
+
+def work(spec) -> dict:
+    if isinstance(spec, wl.LinearSpec):
+        n = spec.B * spec.H * spec.T * spec.D
+        io_b = 2
+        byts = (2 + spec.with_queries) * n * io_b  # K, V (, Q) read
+        byts += spec.with_queries * n * io_b       # O written
+        byts += 2 * spec.B * spec.H * spec.D * spec.D * 4  # W0 read, W written
+        if spec.gate:
+            byts += spec.B * spec.H * spec.T * 4     # losses written
+            byts += spec.B * spec.H * (256 * 3 + 2) * 4  # cache
+        return {"tokens": spec.B * spec.T, "flops": spec.flops, "bytes": byts, "bound": "hbm"}
+    io_b = 4 if spec.dtype == "f32" else 2
+    byts = spec.T * spec.f * io_b + spec.T * spec.d * io_b * 2 + 2 * spec.d * spec.f * 4
+    if spec.target:
+        byts += spec.d * spec.d * 2 + spec.d * 3 * 4
+    bound = "alu" if spec.dtype == "f32" else "tensor"
+    return {"tokens": spec.T, "flops": spec.flops, "bytes": byts, "bound": bound}
+
+
+def fp32_alu_peak_tflops(peaks) -> float:
+    """148 SMs x 128 fp32 lanes x 2 flops (FFMA) x max SM clock."""
+    return 148 * 128 * 2 * peaks["sm_max_mhz"] * 1e6 / 1e12
+
+
+# --------------------------------------------------------------------------------------------
+# GPU arm
+# --------------------------------------------------------------------------------------------
+
+class Runner:
+    """Builds the state and inputs of one workload and runs timed steps."""
+
+    def __init__(self, spec, device):
+        import chunked_weight_layers_b200 as cwl
+        self.spec = spec
+        self.cwl = cwl
+        self.device = device
+        if isinstance(spec, wl.LinearSpec):
+            x = wl.linear_inputs(spec, device=device)
+            cfg = cwl.config("linear", batch=spec.B, heads=spec.H, chunk=spec.b, eta=spec.eta,
+                             gate_enable=int(spec.gate))
+            self.state = cwl.FastWeightState(cfg, x["W0"])
+            self.args = dict(keys=x["K"], targets=x["V"], queries=x.get("Q"))
+            self.out = torch.empty_like(x["K"]) if spec.with_queries else None
+            self.loss = (torch.empty((spec.B, spec.H, spec.T), device=device, dtype=torch.float32)
+                         if spec.gate else None)
+        else:
+            x = wl.inplace_inputs(spec, device=device)
+            io = 0 if spec.dtype == "f32" else 1
+            cfg = cwl.config("inplace", io_dtype=io, d_key=spec.f, d_val=spec.d, chunk=spec.C, eta=spec.eta,
+                             target_mode=int(spec.target), conv_pad_mode=spec.conv_pad_mode)
+            self.state = cwl.FastWeightState(cfg, x["W0"], x.get("Wtarget"), x.get("convw"))
+            self.args = dict(keys=x["Z"], targets=x["X0"] if spec.target else x["Vhat"], queries=None)
+            self.out = torch.empty((spec.T, spec.d), device=device, dtype=x["Z"].dtype)
+            self.loss = None
+        self.inputs = x
+
+    def step(self):
+        self.state.chunk_scan(self.args["keys"], self.args["targets"], self.args["queries"], out=self.out,
+                              loss_out=self.loss, T=self.spec.T)
+
+    def host_buffers(self):
+        pin = lambda t: None if t is None else t.cpu().pin_memory()  # noqa: E731
+        h = {k: pin(v) for k, v in self.args.items()}
+        h["out"] = None if self.out is None else torch.empty(self.out.shape, dtype=self.out.dtype).pin_memory()
+        h["loss"] = None if self.loss is None else torch.empty(self.loss.shape, dtype=torch.float32).pin_memory()
+        return h
+
+
+def time_steps(runner, steps, warmup, flush):
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        runner.state.reset()
+        runner.step()
+    torch.cuda.synchronize()
+    runner.state.poll()
+    times = []
+    l0 = runner.state.launch_count()
+    launches = 0
+    for _ in range(steps):
+        runner.state.reset()
+        flush.fill_(1)  # evict L2 (untimed)
+        n0 = runner.state.launch_count()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        runner.step()
+        e1.record(stream)
+        launches += runner.state.launch_count() - n0
+        e1.synchronize()
+        times.append(e0.elapsed_time(e1))
+    torch.cuda.synchronize()
+    runner.state.poll()
+    del l0
+    return times, launches
+
+
+def time_e2e(runner, steps, warmup):
+    h = runner.host_buffers()
+    st = runner.state
+
+    def once():
+        st.reset()
+        st.chunk_scan_host(h["keys"], h["targets"], h["queries"], out=h["out"], loss_out=h["loss"], T=runner.spec.T)
+
+    for _ in range(max(1, warmup)):
+        once()
+    torch.cuda.synchronize()
+    t = []
+    for _ in range(steps):
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        once()
+        e1.record()
+        e1.synchronize()
+        t.append(e0.elapsed_time(e1))
+    h2d = sum(v.numel() * v.element_size() for k, v in h.items() if k in ("keys", "targets", "queries") and v is not None)
+    d2h = sum(v.numel() * v.element_size() for k, v in h.items() if k in ("out", "loss") and v is not None)
+    return statistics.mean(t), h2d, d2h
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples every 200 ms while the timed region runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self, max_mhz):
+        if self.proc is None or self.path is None:
+            return {"sm_mhz": None, "sm_max_mhz": max_mhz, "reasons": ["unsampled"]}
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": max_mhz, "reasons": ["unsampled"]}
+        mhz = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(mhz) if mhz else None,
+                "sm_max_mhz": float(rows[0][2]) if rows[0][2].replace(".", "").isdigit() else max_mhz,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def roofline(spec, w, ms, peaks, traffic=None):
+    if w["bound"] == "hbm":
+        achieved = w["bytes"] / (ms * 1e-3) / 1e9
+        return {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": traffic, "peak_source": peaks["source"]}
+    if w["bound"] == "tensor":
+        achieved = w["flops"] / (ms * 1e-3) / 1e12
+        return {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops"], "traffic": traffic, "peak_source": peaks["source"],
+                "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"]}
+    achieved = w["flops"] / (ms * 1e-3) / 1e12
+    peak = fp32_alu_peak_tflops(peaks)
+    return {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+            "traffic": traffic, "peak_source": "148 SMs x 128 FP32 lanes x 2 x max SM clock"}
+
+
+def cpu_baseline(spec, budget_s=12.0) -> dict:
+    """The oracle as it stands on this host's cores, on a bounded sample of the workload."""
+    import numpy as np  # noqa: F401
+    from oracle import gate as ogate
+    from oracle import inplace as oinp
+    from oracle import linear as olin
+    cores = torch.get_num_threads()
+    t0 = time.perf_counter()
+    if isinstance(spec, wl.LinearSpec):
+        x = wl.linear_inputs(spec)
+        done_heads = 0
+        BH = spec.B * spec.H
+        K = x["K"].reshape(BH, 1, spec.T, spec.D)
+        V = x["V"].reshape(BH, 1, spec.T, spec.D)
+        Q = x["Q"].reshape(BH, 1, spec.T, spec.D) if "Q" in x else None
+        W0 = x["W0"].reshape(BH, 1, spec.D, spec.D)
+        t0 = time.perf_counter()
+        while done_heads < BH and time.perf_counter() - t0 < budget_s:
+            h = done_heads
+            _, _, L = olin.ttt_linear_scan(K[h:h + 1], V[h:h + 1], None if Q is None else Q[h:h + 1],
+                                          W0[h:h + 1], spec.eta, spec.b)
+            if spec.gate:
+                ogate.surprisal_route(L.astype("float32"), ogate.GateState(1, 1))
+            done_heads += 1
+        dt = time.perf_counter() - t0
+        tokens = spec.T * done_heads / spec.H
+        sample = f"{done_heads} of {BH} (sequence, head) scans, one at a time"
+    else:
+        Cs = spec.C
+        x = wl.inplace_inputs(wl.scaled(spec, T=min(spec.T, Cs * 2)) if spec.dtype == "bf16" else spec)
+        t0 = time.perf_counter()
+        chunks = 0
+        W = x["W0"]
+        Vh = x.get("Vhat")
+        if Vh is None:
+            Vh = torch.from_numpy(oinp.target_values(x["X0"], x["convw"], x["Wtarget"], spec.C))
+        T = x["Z"].shape[0]
+        while time.perf_counter() - t0 < budget_s and chunks * Cs < T:
+            sl = slice(chunks * Cs, (chunks + 1) * Cs)
+            _, W = oinp.inplace_scan(x["Z"][sl], Vh[sl], W, spec.eta, Cs)
+            chunks += 1
+        dt = time.perf_counter() - t0
+        tokens = chunks * Cs
+        sample = f"{chunks} chunk(s) of {Cs} tokens"
+    return {"value": tokens / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample,
+            "seconds": dt}
+
+
+def measure(spec, steps, warmup, flush, peaks, device, with_e2e):
+    r = Runner(spec, device)
+    times, launches = time_steps(r, steps, warmup, flush)
+    ms = statistics.mean(times)
+    w = work(spec)
+    out = {"workload": spec.name, "ms_per_step": ms, "tokens_per_s": w["tokens"] / (ms * 1e-3),
+           "tflops": w["flops"] / (ms * 1e-3) / 1e12, "roofline": roofline(spec, w, ms, peaks),
+           "gpu_launches_per_step": launches / max(1, steps), "times_ms": times}
+    if with_e2e:
+        e2e_ms, h2d, d2h = time_e2e(r, max(3, steps // 2), 1)
+        out["e2e"] = {"value": w["tokens"] / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                      "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+    r.state.close()
+    del r
+    torch.cuda.empty_cache()
+    return out
+
+
+def spec_by_name(name):
+    for s in wl.WORKLOADS.values():
+        if s.name == name:
+            return s
+    raise SystemExit(f"unknown workload {name}; choose from {list(wl.WORKLOADS)}")
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--workload", default=MAIN)
+    ap.add_argument("--only-main", action="store_true", help="skip the other four workloads")
+    a = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    spec = spec_by_name(a.workload)
+    w = work(spec)
+    peaks = load_peaks()
+
+    if a.impl == "reference":
+        if rank != 0:
+            return
+        cb = cpu_baseline(spec)
+        val = cb["value"]
+        print(json.dumps({"impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s", "n_gpus": a.gpus,
+                          "steps": a.steps, "warmup": a.warmup, "higher_is_better": True, "scaling": "weak",
+                          "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                          "config": {"workload": spec.name}, "cpu_baseline": cb,
+                          "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                                  "d2h_bytes_per_step": 0}}))
+        return
+
+    if a.warmup < 3:
+        a.warmup = 3
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+        pg = dist
+    from chunked_weight_layers_b200 import build
+    if rank == 0:
+        build.build()
+    if pg is not None:
+        pg.barrier()
+    flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=device)
+
+    runner = Runner(spec, device)
+    for _ in range(a.warmup):
+        runner.state.reset()
+        runner.step()
+    torch.cuda.synchronize()
+    runner.state.poll()
+    stream = torch.cuda.current_stream()
+    times = []
+    launches = 0
+    if pg is not None:
+        pg.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for _ in range(a.steps):
+            runner.state.reset()
+            flush.fill_(1)
+            n0 = runner.state.launch_count()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            runner.step()
+            e1.record(stream)
+            launches += runner.state.launch_count() - n0
+            e1.synchronize()
+            times.append(e0.elapsed_time(e1))
+        torch.cuda.synchronize()
+    if pg is not None:
+        pg.barrier()
+    runner.state.poll()
+    total_ms = sum(times)
+    if pg is not None:
+        t = torch.tensor([total_ms], device=device)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms = total_ms / a.steps
+    value = world * w["tokens"] / (ms * 1e-3)
+    e2e_ms, h2d, d2h = None, 0, 0
+    runner_e2e = None
+    try:
+        e2e_ms, h2d, d2h = time_e2e(runner, max(3, a.steps // 2), 1)
+        if pg is not None:
+            t = torch.tensor([e2e_ms], device=device)
+            pg.all_reduce(t, op=pg.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        runner_e2e = world * w["tokens"] / (e2e_ms * 1e-3)
+    except Exception as ex:  # report, do not hide
+        runner_e2e = None
+        print(f"e2e measurement failed: {ex}", file=sys.stderr)
+    runner.state.close()
+    del runner
+    torch.cuda.empty_cache()
+
+    extra = {}
+    if not a.only_main and world == 1:
+        for s in wl.WORKLOADS.values():
+            if s.name == spec.name:
+                continue
+            try:
+                extra[s.name] = measure(s, max(5, min(a.steps, 10)), 3, flush, peaks, device, with_e2e=False)
+            except Exception as ex:
+                extra[s.name] = {"error": str(ex)}
+
+    if rank == 0:
+        rl = roofline(spec, w, ms, peaks)
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": a.steps,
+            "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": spec.name, "B": getattr(spec, "B", 1), "H": getattr(spec, "H", 1),
+                       "T": spec.T, "chunk": getattr(spec, "b", getattr(spec, "C", None)),
+                       "parallelism": f"replicas{world}" if world > 1 else "single",
+                       "l2": "flushed before every timed step (512 MB write)"},
+            "tflops": world * w["flops"] / (ms * 1e-3) / 1e12,
+            "roofline": rl,
+            "e2e": {"value": runner_e2e, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": e2e_ms},
+            "gpu_launches": launches,
+            "clocks": clk.summary(peaks["sm_max_mhz"]),
+        }
+        if world == 1:
+            line["cpu_baseline"] = cpu_baseline(spec)
+        if extra:
+            line["workloads"] = extra
+        print(json.dumps(line))
+    if pg is not None:
+        pg.barrier()
+        pg.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,114 @@
+// Host-side internals of libttt.so: the state object and the kernel launchers.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <string>
+
+#include "../../include/ttt.h"
+
+namespace ttt {
+
+// Records `msg` as the calling thread's last error and returns `s`.
+ttt_status fail(ttt_status s, const char* fmt, ...);
+// Maps a CUDA runtime error to TTT_ERR_CUDA with a message naming `what`.
+ttt_status cuda_fail(cudaError_t e, const char* what);
+
+#define TTT_CUDA(call)                                        \
+  do {                                                        \
+    cudaError_t e_ = (call);                                  \
+    if (e_ != cudaSuccess) return ::ttt::cuda_fail(e_, #call); \
+  } while (0)
+
+#define TTT_TRY(call)                      \
+  do {                                     \
+    ttt_status s_ = (call);                \
+    if (s_ != TTT_OK) return s_;           \
+  } while (0)
+
+// Device-visible status word (pinned, mapped host memory): kernels record the first
+// failure there with atomicCAS; the host reads it in ttt_state_poll().
+struct StatusWord {
+  int* host = nullptr;
+  int* dev = nullptr;
+};
+
+struct InplaceBuffers {
+  float* W = nullptr;            // fp32 master [d, f]
+  float* W0 = nullptr;           // pretrained copy [d, f]
+  __nv_bfloat16* Wsh[2] = {nullptr, nullptr};  // bf16 copies of W for the apply (BF16 path)
+  int cur = 0;                   // index of the bf16 copy that holds the current W
+  __nv_bfloat16* Wtarget = nullptr;  // [d, d]
+  float* convw = nullptr;        // [d, taps]
+  __nv_bfloat16* conv = nullptr; // conv(X0) of one chunk [C, d]
+  __nv_bfloat16* Vhat[2] = {nullptr, nullptr};  // targets of a chunk [C, d]
+};
+
+struct LinearBuffers {
+  float* W = nullptr;   // [B, H, D, D]
+  float* W0 = nullptr;  // [B, H, D, D]
+};
+
+struct GateBuffers {
+  float* tau = nullptr;       // [B, H]
+  int32_t* tau_set = nullptr; // [B, H]
+  int32_t* entries = nullptr; // [B, H, cap, 3]
+  int32_t* counts = nullptr;  // [B, H, 2]
+  int64_t t_offset = 0;       // tokens gated since the last reset (host-side counter)
+};
+
+struct HostStaging {
+  void* buf[5] = {nullptr, nullptr, nullptr, nullptr, nullptr};
+  size_t bytes[5] = {0, 0, 0, 0, 0};
+};
+
+}  // namespace ttt
+
+struct ttt_state {
+  ttt_config cfg;
+  int device = 0;
+  int num_sms = 0;
+  ttt::StatusWord status;
+  ttt::InplaceBuffers ip;
+  ttt::LinearBuffers lin;
+  ttt::GateBuffers gate;
+  ttt::HostStaging staging;
+  int64_t launches = 0;
+};
+
+namespace ttt {
+
+size_t io_size(int dtype);
+
+// ---- kernel launchers (each returns TTT_OK or TTT_ERR_CUDA after the launch) ----------
+
+// In-Place, fp32 SIMT: one chunk of the scan (apply with W, then W += η·V̂ᵀZ).
+ttt_status inplace_f32_chunk(ttt_state* st, const float* Z, const float* Vhat, float* O, int C,
+                             cudaStream_t s);
+
+// In-Place, bf16 tensor cores: the whole scan over T tokens.
+ttt_status inplace_bf16_scan(ttt_state* st, const __nv_bfloat16* Z, const __nv_bfloat16* targets,
+                             int64_t T, __nv_bfloat16* O, cudaStream_t s);
+
+// TTT-Linear mini-batch scan over T tokens of every (sequence, head).
+ttt_status linear_scan(ttt_state* st, const __nv_bfloat16* K, const __nv_bfloat16* V,
+                       const __nv_bfloat16* Q, int64_t T, __nv_bfloat16* O, float* loss,
+                       cudaStream_t s);
+
+// Surprisal gate over T losses of every (sequence, head).
+ttt_status gate_route(ttt_state* st, const float* loss, int64_t T, cudaStream_t s);
+
+// Small utility kernels.
+ttt_status f32_to_bf16(const float* src, __nv_bfloat16* dst, size_t n, cudaStream_t s,
+                       ttt_state* st);
+ttt_status fill_i32(int32_t* dst, int32_t v, size_t n, cudaStream_t s, ttt_state* st);
+
+// TMA descriptor encoding through the driver entry point (no -lcuda link needed).
+ttt_status encode_tmap(CUtensorMap* map, CUtensorMapDataType dtype, int rank, const void* base,
+                       const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
+                       CUtensorMapSwizzle swizzle);
+
+}  // namespace ttt

@@ -1,0 +1,340 @@
+// TTT-Linear mini-batch gradient scan ("テスト時学習（Test-Time Training）とは", the TTT layers
+// page: the hidden state is the weight W of a linear model and each update is one
+// self-supervised gradient step). Per (sequence, head) and inner mini-batch i of b tokens:
+//   O_i = Q_i·W_i,   R_i = K_i·W_i − V_i,   L_t = ‖R_i[t]‖²,   W_{i+1} = W_i − (η/b)·K_iᵀ·R_i.
+//
+// Design (B200):
+//  * one CTA per (sequence, head); the per-head state is 64x64 fp32 and never leaves the SM:
+//    it lives in mma accumulator registers of four compute warps. Column c of W only ever
+//    depends on column c of R (R[:, c] = K·W[:, c] − V[:, c]), so warp w owns the 16 columns
+//    [16w, 16w+16) and runs its chain with no cross-warp synchronisation inside a step.
+//  * everything is computed transposed, so each accumulator layout is directly the next
+//    mma's A operand (no shuffles): Pᵀ = Wᵀ·Kᵀ (+ −Vᵀ), Oᵀ = Wᵀ·Qᵀ, Wᵀ += (−η/b·R)ᵀ·K.
+//  * the fp32 W is fed to the tensor cores as a bf16 hi + lo pair (two mma per product) so
+//    the operand rounding is ~2^-17 instead of 2^-9; R is fed the same way for the update.
+//  * K, V, Q stream through a 4-stage ring of 64-token tiles loaded by TMA (128-byte
+//    swizzle, 3-D maps over [B·H, T, 64] so a head's last tile is clipped to its own T);
+//    outputs are staged in swizzled smem and written by TMA stores.
+//  * the chain per step is latency-bound and tiny (393 kFLOP), so it runs on the legacy
+//    warp-level mma.sync path: a tcgen05 round trip (issue, commit, mbarrier, tcgen05.ld)
+//    per dependent 16x64x64 product costs more than the product itself.
+#include "common.cuh"
+#include "internal.h"
+
+namespace ttt {
+
+namespace {
+
+constexpr int kStages = 4;        // ring depth (64-token tiles)
+constexpr int kTileTok = 64;      // tokens per tile
+constexpr int kTileBytes = kTileTok * 128;  // 64 tokens x 64 bf16
+constexpr int kComputeWarps = 4;
+constexpr int kThreads = (kComputeWarps + 1) * 32;
+
+struct __align__(1024) LinearSmem {
+  uint8_t K[kStages][kTileBytes];
+  uint8_t V[kStages][kTileBytes];
+  uint8_t Q[kStages][kTileBytes];
+  uint8_t O[2][kTileBytes];
+  float lossp[kComputeWarps][kTileTok];
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
+  int abort;       // set by the producer when one of its waits ran out
+  int cabort[2];   // set by a compute warp whose wait for tile s ran out (index s & 1)
+  int consumed;
+};
+
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void named_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kComputeWarps * 32)); }
+
+// Split two fp32 values into packed bf16 hi and lo words (x ≈ hi + lo to ~2^-17 relative).
+__device__ __forceinline__ void split2(float x, float y, uint32_t& hi, uint32_t& lo) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(x, y);
+  const float2 hf = __bfloat1622float2(h);
+  hi = *reinterpret_cast<uint32_t*>(&h);
+  lo = pack_bf16(x - hf.x, y - hf.y);
+}
+
+__device__ __forceinline__ float2 unpack_bf16(uint32_t v) {
+  return __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&v));
+}
+
+template <int B>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_linear_scan(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                  const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
+                  float* __restrict__ Wstate, float* __restrict__ loss, int T, float beta, int has_q,
+                  int* status) {
+  extern __shared__ uint8_t smem_raw[];
+  LinearSmem& sm = *reinterpret_cast<LinearSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bh = blockIdx.x;
+  const int nstages = (T + kTileTok - 1) / kTileTok;
+  const uint32_t stage_bytes = (has_q ? 3u : 2u) * kTileBytes;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&sm.full[i], 1);
+      mbar_init(&sm.empty[i], kComputeWarps);
+    }
+    sm.abort = 0;
+    sm.cabort[0] = sm.cabort[1] = 0;
+    sm.consumed = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  if (warp == kComputeWarps) {
+    // ---------------- producer: TMA loads of K, V, Q tiles ----------------
+    if (lane == 0) {
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      if (has_q) tma_prefetch_desc(&tmQ);
+      int issued = 0;
+      for (int s = 0; s < nstages; ++s) {
+        const int slot = s % kStages;
+        if (s >= kStages && !mbar_wait(&sm.empty[slot], ((s / kStages) - 1) & 1, status, &sm.abort)) break;
+        mbar_arrive_expect_tx(&sm.full[slot], stage_bytes);
+        tma_load_3d(sm.K[slot], &tmK, &sm.full[slot], 0, s * kTileTok, bh);
+        tma_load_3d(sm.V[slot], &tmV, &sm.full[slot], 0, s * kTileTok, bh);
+        if (has_q) tma_load_3d(sm.Q[slot], &tmQ, &sm.full[slot], 0, s * kTileTok, bh);
+        issued = s + 1;
+      }
+      // Nothing may still be landing in shared memory when the CTA exits: wait (bounded) for
+      // the newest issued phase of every slot. A phase that already completed returns at once.
+      for (int s = issued - kStages; s < issued; ++s) {
+        if (s < 0) continue;
+        mbar_wait(&sm.full[s % kStages], (s / kStages) & 1, status, nullptr);
+      }
+    }
+    __syncthreads();
+    return;
+  }
+
+  // ---------------- compute warps ----------------
+  const int g = lane >> 2, q = lane & 3;
+  const int col0 = 16 * warp;  // first W column owned by this warp
+  float* Wg = Wstate + (size_t)bh * 64 * 64;
+
+  // Wᵀ slice in accumulator layout: acc[nt][e] = W[8nt + 2q + (e&1)][col0 + g + 8(e>>1)].
+  float acc[8][4];
+#pragma unroll
+  for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[nt][e] = Wg[(8 * nt + 2 * q + (e & 1)) * 64 + col0 + g + 8 * (e >> 1)];
+
+  constexpr int NT = B / 8;   // token n-tiles per mini-batch
+  constexpr int KT = B / 16;  // token k-steps per mini-batch
+
+  for (int s = 0; s < nstages; ++s) {
+    const int slot = s % kStages;
+    // Every compute warp takes the same exit decision: the flag for tile s is only written
+    // before this barrier and only read after it (tile s+2 uses the same flag, but no warp can
+    // reach its wait before all warps passed the end-of-tile barriers of tile s+1).
+    if (!mbar_wait(&sm.full[slot], (s / kStages) & 1, status, nullptr)) sm.cabort[s & 1] = 1;
+    named_sync();
+    if (*reinterpret_cast<volatile int*>(&sm.cabort[s & 1])) break;
+    const int ntok = min(kTileTok, T - s * kTileTok);
+    const uint32_t kbase = smem_u32(sm.K[slot]);
+    const uint32_t vbase = smem_u32(sm.V[slot]);
+    const uint32_t qbase = smem_u32(sm.Q[slot]);
+    uint8_t* obuf = sm.O[s & 1];
+
+    for (int r0 = 0; r0 < ntok; r0 += B) {
+      // A fragments of Wᵀ (hi and lo) for the four 16-key k-steps.
+      uint32_t whi[4][4], wlo[4][4];
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks) {
+        split2(acc[2 * ks][0], acc[2 * ks][1], whi[ks][0], wlo[ks][0]);
+        split2(acc[2 * ks][2], acc[2 * ks][3], whi[ks][1], wlo[ks][1]);
+        split2(acc[2 * ks + 1][0], acc[2 * ks + 1][1], whi[ks][2], wlo[ks][2]);
+        split2(acc[2 * ks + 1][2], acc[2 * ks + 1][3], whi[ks][3], wlo[ks][3]);
+      }
+
+      // Pᵀ = −Vᵀ + Wᵀ·Kᵀ and Oᵀ = Wᵀ·Qᵀ for the B tokens of this mini-batch.
+      float p[NT][4], o[NT][4];
+#pragma unroll
+      for (int nt = 0; nt < NT; nt += 2) {
+        // −V[t][c] for tokens r0+8nt.. (two n-tiles) and this warp's 16 columns.
+        uint32_t v[4];
+        const int mi = lane >> 3, ri = lane & 7;
+        ldsm_x4_t(vbase + swz128_bf16(r0 + 8 * (nt + (mi >> 1)) + ri, col0 + 8 * (mi & 1)), v);
+        const float2 v0 = unpack_bf16(v[0]), v1 = unpack_bf16(v[1]), v2 = unpack_bf16(v[2]), v3 = unpack_bf16(v[3]);
+        p[nt][0] = -v0.x; p[nt][1] = -v0.y; p[nt][2] = -v1.x; p[nt][3] = -v1.y;
+        if (nt + 1 < NT) { p[nt + 1][0] = -v2.x; p[nt + 1][1] = -v2.y; p[nt + 1][2] = -v3.x; p[nt + 1][3] = -v3.y; }
+      }
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o[nt][e] = 0.f;
+        float p2[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int ks = 0; ks < 4; ks += 2) {
+          // B fragments of Kᵀ (and Qᵀ): rows = tokens r0+8nt.., keys 16ks .. 16ks+31.
+          const int mi = lane >> 3, ri = lane & 7;
+          const uint32_t off = swz128_bf16(r0 + 8 * nt + ri, 16 * ks + 8 * mi);
+          uint32_t kb[4];
+          ldsm_x4(kbase + off, kb);
+          mma16816(p[nt], whi[ks], kb[0], kb[1]);
+          mma16816(p2, wlo[ks], kb[0], kb[1]);
+          mma16816(p[nt], whi[ks + 1], kb[2], kb[3]);
+          mma16816(p2, wlo[ks + 1], kb[2], kb[3]);
+          if (has_q) {
+            uint32_t qb[4];
+            ldsm_x4(qbase + off, qb);
+            mma16816(o[nt], whi[ks], qb[0], qb[1]);
+            mma16816(o[nt], wlo[ks], qb[0], qb[1]);
+            mma16816(o[nt], whi[ks + 1], qb[2], qb[3]);
+            mma16816(o[nt], wlo[ks + 1], qb[2], qb[3]);
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) p[nt][e] += p2[e];
+      }
+
+      // Per-token loss: this thread holds R for tokens 8nt+2q, 8nt+2q+1 at columns g, g+8.
+      if (loss != nullptr) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          float l0 = p[nt][0] * p[nt][0] + p[nt][2] * p[nt][2];
+          float l1 = p[nt][1] * p[nt][1] + p[nt][3] * p[nt][3];
+#pragma unroll
+          for (int m = 4; m < 32; m <<= 1) {
+            l0 += __shfl_xor_sync(0xffffffffu, l0, m);
+            l1 += __shfl_xor_sync(0xffffffffu, l1, m);
+          }
+          if (g == 0) {
+            sm.lossp[warp][r0 + 8 * nt + 2 * q] = l0;
+            sm.lossp[warp][r0 + 8 * nt + 2 * q + 1] = l1;
+          }
+        }
+      }
+
+      // Outputs into the swizzled staging tile (row = token in the tile, col = W column).
+      if (has_q) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int row = r0 + 8 * nt + 2 * q + (e & 1);
+            const int col = col0 + g + 8 * (e >> 1);
+            *reinterpret_cast<__nv_bfloat16*>(obuf + swz128_bf16(row, col)) = __float2bfloat16_rn(o[nt][e]);
+          }
+      }
+
+      // Wᵀ += Sᵀ·K with S = −(η/b)·R, S fed as bf16 hi + lo.
+      uint32_t shi[KT][4], slo[KT][4];
+#pragma unroll
+      for (int kt = 0; kt < KT; ++kt) {
+        split2(-beta * p[2 * kt][0], -beta * p[2 * kt][1], shi[kt][0], slo[kt][0]);
+        split2(-beta * p[2 * kt][2], -beta * p[2 * kt][3], shi[kt][1], slo[kt][1]);
+        split2(-beta * p[2 * kt + 1][0], -beta * p[2 * kt + 1][1], shi[kt][2], slo[kt][2]);
+        split2(-beta * p[2 * kt + 1][2], -beta * p[2 * kt + 1][3], shi[kt][3], slo[kt][3]);
+      }
+#pragma unroll
+      for (int kt = 0; kt < KT; ++kt) {
+#pragma unroll
+        for (int nt = 0; nt < 8; nt += 2) {
+          // B fragments of K[token][key]: tokens r0+16kt .. +15, keys 8nt .. 8nt+15 (transposed).
+          const int mi = lane >> 3, ri = lane & 7;
+          uint32_t kb[4];
+          ldsm_x4_t(kbase + swz128_bf16(r0 + 16 * kt + 8 * (mi & 1) + ri, 8 * nt + 8 * (mi >> 1)), kb);
+          mma16816(acc[nt], shi[kt], kb[0], kb[1]);
+          mma16816(acc[nt], slo[kt], kb[0], kb[1]);
+          mma16816(acc[nt + 1], shi[kt], kb[2], kb[3]);
+          mma16816(acc[nt + 1], slo[kt], kb[2], kb[3]);
+        }
+      }
+    }
+
+    // End of the tile: outputs and losses of 64 tokens are complete in shared memory.
+    if (has_q) fence_proxy_async_smem();
+    named_sync();
+    if (loss != nullptr && warp == 0) {
+      for (int i = lane; i < ntok; i += 32) {
+        const float l = (sm.lossp[0][i] + sm.lossp[1][i]) + (sm.lossp[2][i] + sm.lossp[3][i]);
+        loss[(size_t)bh * T + (size_t)s * kTileTok + i] = l;
+      }
+    }
+    if (threadIdx.x == 0) {
+      if (has_q) {
+        tma_store_3d(&tmO, obuf, 0, s * kTileTok, bh);
+        bulk_commit();
+        bulk_wait_read<1>();  // the other staging tile is free again
+      }
+      sm.consumed = s + 1;
+    }
+    named_sync();
+    if (lane == 0) mbar_arrive(&sm.empty[slot]);
+  }
+
+  if (threadIdx.x == 0 && has_q) bulk_wait<0>();
+  // Final state.
+#pragma unroll
+  for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) Wg[(8 * nt + 2 * q + (e & 1)) * 64 + col0 + g + 8 * (e >> 1)] = acc[nt][e];
+  __syncthreads();
+}
+
+template <int B>
+ttt_status launch(ttt_state* st, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
+                  const CUtensorMap& to, float* loss, int T, int has_q, cudaStream_t s) {
+  const size_t smem = sizeof(LinearSmem) + 1024;
+  TTT_CUDA(cudaFuncSetAttribute(k_linear_scan<B>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  const int grid = st->cfg.batch * st->cfg.heads;
+  const float beta = st->cfg.eta / (float)B;
+  k_linear_scan<B><<<grid, kThreads, smem, s>>>(tk, tv, tq, to, st->lin.W, loss, T, beta, has_q, st->status.dev);
+  st->launches++;
+  TTT_CUDA(cudaGetLastError());
+  return TTT_OK;
+}
+
+}  // namespace
+
+ttt_status linear_scan(ttt_state* st, const __nv_bfloat16* K, const __nv_bfloat16* V, const __nv_bfloat16* Q,
+                       int64_t T, __nv_bfloat16* O, float* loss, cudaStream_t s) {
+  const ttt_config& c = st->cfg;
+  const uint64_t BH = (uint64_t)c.batch * c.heads;
+  const uint64_t dims[3] = {64, (uint64_t)T, BH};
+  const uint64_t strides[2] = {128, (uint64_t)T * 128};
+  const uint32_t box[3] = {64, (uint32_t)kTileTok, 1};
+  CUtensorMap tk, tv, tq, to;
+  TTT_TRY(encode_tmap(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, K, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B));
+  TTT_TRY(encode_tmap(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, V, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B));
+  const int has_q = Q != nullptr;
+  if (has_q) {
+    TTT_TRY(encode_tmap(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, Q, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B));
+    TTT_TRY(encode_tmap(&to, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, O, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B));
+  } else {
+    tq = tk;
+    to = tk;
+  }
+  switch (c.chunk) {
+    case 16: return launch<16>(st, tk, tv, tq, to, loss, (int)T, has_q, s);
+    case 32: return launch<32>(st, tk, tv, tq, to, loss, (int)T, has_q, s);
+    case 64: return launch<64>(st, tk, tv, tq, to, loss, (int)T, has_q, s);
+    default: return fail(TTT_ERR_UNSUPPORTED, "TTT-Linear: mini-batch %d not built", c.chunk);
+  }
+}
+
+}  // namespace ttt

@@ -1,0 +1,450 @@
+// C ABI of libttt.so: argument validation, state memory, and dispatch to the kernels.
+// The semantics of every entry point are documented in include/ttt.h.
+#include <stdarg.h>
+#include <stdio.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include "internal.h"
+
+namespace ttt {
+
+static thread_local char g_last_error[512] = "";
+
+ttt_status fail(ttt_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+ttt_status cuda_fail(cudaError_t e, const char* what) {
+  cudaGetLastError();  // clear a sticky launch error so later calls can proceed
+  if (e == cudaErrorMemoryAllocation)
+    return fail(TTT_ERR_OOM, "%s: %s", what, cudaGetErrorString(e));
+  return fail(TTT_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+size_t io_size(int dtype) { return dtype == TTT_F32 ? 4 : 2; }
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Allocation that honours the fault-injection switch TTT_INJECT_OOM (tests only).
+static ttt_status dev_alloc(void** p, size_t bytes, const char* what) {
+  *p = nullptr;
+  const char* inj = getenv("TTT_INJECT_OOM");
+  if (inj != nullptr && inj[0] == '1') return fail(TTT_ERR_OOM, "%s: injected allocation failure", what);
+  if (bytes == 0) bytes = 16;
+  cudaError_t e = cudaMalloc(p, bytes);
+  if (e != cudaSuccess) {
+    *p = nullptr;
+    return cuda_fail(e, what);
+  }
+  return TTT_OK;
+}
+
+static void dev_free(void* p) {
+  if (p != nullptr) cudaFree(p);
+}
+
+static ttt_status validate(const ttt_config* c) {
+  if (c->rule == TTT_RULE_INPLACE_HEBBIAN) {
+    if (c->batch != 1 || c->heads != 1)
+      return fail(TTT_ERR_UNSUPPORTED, "In-Place scan: batch and heads must be 1 (one Wdown state)");
+    if (c->d_key < 1 || c->d_val < 1 || c->chunk < 1)
+      return fail(TTT_ERR_INVALID_ARG, "In-Place scan: d_key, d_val and chunk must be positive");
+    if (c->io_dtype == TTT_F32) {
+      if (c->target_mode != 0)
+        return fail(TTT_ERR_UNSUPPORTED, "In-Place fp32: fused target generation needs BF16 io");
+      return TTT_OK;
+    }
+    if (c->io_dtype != TTT_BF16) return fail(TTT_ERR_INVALID_ARG, "unknown io_dtype %d", c->io_dtype);
+    if (c->d_key % 8 != 0 || c->d_val % 8 != 0)
+      return fail(TTT_ERR_UNSUPPORTED, "In-Place BF16: d_key and d_val must be multiples of 8 (16-byte rows for TMA)");
+    if (c->chunk % 128 != 0)
+      return fail(TTT_ERR_UNSUPPORTED, "In-Place BF16: chunk must be a multiple of 128");
+    if (c->target_mode != 0 && c->target_mode != 1)
+      return fail(TTT_ERR_INVALID_ARG, "target_mode must be 0 or 1");
+    if (c->target_mode == 1) {
+      if (c->conv_taps < 1 || c->conv_taps > 8)
+        return fail(TTT_ERR_UNSUPPORTED, "conv_taps must lie in [1, 8]");
+      if (c->conv_pad_mode != 0 && c->conv_pad_mode != 1)
+        return fail(TTT_ERR_INVALID_ARG, "conv_pad_mode must be 0 or 1");
+    }
+    if (c->gate_enable) return fail(TTT_ERR_UNSUPPORTED, "the surprisal gate runs on TTT-Linear states");
+    return TTT_OK;
+  }
+  if (c->rule == TTT_RULE_LINEAR_GD) {
+    if (c->io_dtype != TTT_BF16) return fail(TTT_ERR_UNSUPPORTED, "TTT-Linear: io_dtype must be BF16");
+    if (c->batch < 1 || c->heads < 1) return fail(TTT_ERR_INVALID_ARG, "TTT-Linear: batch and heads must be positive");
+    if (c->d_key != 64 || c->d_val != 64)
+      return fail(TTT_ERR_UNSUPPORTED, "TTT-Linear: head width must be 64 (d_key = d_val = 64)");
+    if (c->chunk < 16 || c->chunk > 64 || c->chunk % 16 != 0)
+      return fail(TTT_ERR_UNSUPPORTED, "TTT-Linear: inner mini-batch must be 16, 32, 48 or 64");
+    if (c->target_mode != 0) return fail(TTT_ERR_INVALID_ARG, "target_mode applies to In-Place only");
+    if (c->gate_enable) {
+      if (c->gate_chunk != 64) return fail(TTT_ERR_UNSUPPORTED, "gate_chunk must be 64");
+      if (c->cache_capacity < 1) return fail(TTT_ERR_INVALID_ARG, "cache_capacity must be positive");
+      if (!(c->gate_pct > 0.f && c->gate_pct <= 1.f)) return fail(TTT_ERR_INVALID_ARG, "gate_pct must lie in (0, 1]");
+      if (c->gate_mean_num < 0 || c->gate_mean_den < 1)
+        return fail(TTT_ERR_INVALID_ARG, "gate mean fraction must be num >= 0, den >= 1");
+    }
+    return TTT_OK;
+  }
+  return fail(TTT_ERR_INVALID_ARG, "unknown rule %d", c->rule);
+}
+
+static size_t weight_elems(const ttt_config& c) {
+  if (c.rule == TTT_RULE_INPLACE_HEBBIAN) return (size_t)c.d_val * c.d_key;
+  return (size_t)c.batch * c.heads * c.d_key * c.d_key;
+}
+
+static void free_state(ttt_state* st) {
+  if (st == nullptr) return;
+  dev_free(st->ip.W);
+  dev_free(st->ip.W0);
+  dev_free(st->ip.Wsh[0]);
+  dev_free(st->ip.Wsh[1]);
+  dev_free(st->ip.Wtarget);
+  dev_free(st->ip.convw);
+  dev_free(st->ip.conv);
+  dev_free(st->ip.Vhat[0]);
+  dev_free(st->ip.Vhat[1]);
+  dev_free(st->lin.W);
+  dev_free(st->lin.W0);
+  dev_free(st->gate.tau);
+  dev_free(st->gate.tau_set);
+  dev_free(st->gate.entries);
+  dev_free(st->gate.counts);
+  for (int i = 0; i < 5; ++i) dev_free(st->staging.buf[i]);
+  if (st->status.host != nullptr) cudaFreeHost(st->status.host);
+  delete st;
+}
+
+static ttt_status gate_reset(ttt_state* st, cudaStream_t s) {
+  const ttt_config& c = st->cfg;
+  const size_t bh = (size_t)c.batch * c.heads;
+  TTT_CUDA(cudaMemsetAsync(st->gate.tau, 0, bh * sizeof(float), s));
+  TTT_CUDA(cudaMemsetAsync(st->gate.tau_set, 0, bh * sizeof(int32_t), s));
+  TTT_CUDA(cudaMemsetAsync(st->gate.counts, 0, bh * 2 * sizeof(int32_t), s));
+  TTT_TRY(fill_i32(st->gate.entries, -1, bh * (size_t)c.cache_capacity * 3, s, st));
+  st->gate.t_offset = 0;
+  return TTT_OK;
+}
+
+static ttt_status load_weights(ttt_state* st, const float* W, cudaStream_t s) {
+  const size_t n = weight_elems(st->cfg);
+  if (st->cfg.rule == TTT_RULE_INPLACE_HEBBIAN) {
+    TTT_CUDA(cudaMemcpyAsync(st->ip.W, W, n * sizeof(float), cudaMemcpyDeviceToDevice, s));
+    if (st->cfg.io_dtype == TTT_BF16) {
+      st->ip.cur = 0;
+      TTT_TRY(f32_to_bf16(st->ip.W, st->ip.Wsh[0], n, s, st));
+    }
+  } else {
+    TTT_CUDA(cudaMemcpyAsync(st->lin.W, W, n * sizeof(float), cudaMemcpyDeviceToDevice, s));
+  }
+  return TTT_OK;
+}
+
+static ttt_status create_impl(const ttt_config* cfg, const void* W0, const void* Wtarget,
+                              const float* convw, cudaStream_t s, ttt_state** out) {
+  TTT_TRY(validate(cfg));
+  const ttt_config& c = *cfg;
+  if (W0 == nullptr || !aligned16(W0)) return fail(TTT_ERR_INVALID_ARG, "W0 must be a 16-byte aligned device pointer");
+  const bool target = c.rule == TTT_RULE_INPLACE_HEBBIAN && c.target_mode == 1;
+  if (target) {
+    if (Wtarget == nullptr || convw == nullptr || !aligned16(Wtarget) || !aligned16(convw))
+      return fail(TTT_ERR_INVALID_ARG, "target_mode 1 needs 16-byte aligned Wtarget and convw");
+  } else if (Wtarget != nullptr || convw != nullptr) {
+    return fail(TTT_ERR_INVALID_ARG, "Wtarget and convw are only taken with target_mode 1");
+  }
+
+  ttt_state* st = new (std::nothrow) ttt_state();
+  if (st == nullptr) return fail(TTT_ERR_OOM, "host allocation of the state failed");
+  st->cfg = c;
+  ttt_status r = TTT_OK;
+  auto guard = [&](ttt_status x) {
+    if (x != TTT_OK && r == TTT_OK) r = x;
+    return r == TTT_OK;
+  };
+  cudaError_t e = cudaGetDevice(&st->device);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&st->num_sms, cudaDevAttrMultiProcessorCount, st->device);
+  if (e != cudaSuccess) {
+    free_state(st);
+    return cuda_fail(e, "cudaGetDevice");
+  }
+  e = cudaHostAlloc(reinterpret_cast<void**>(&st->status.host), sizeof(int), cudaHostAllocMapped);
+  if (e == cudaSuccess) e = cudaHostGetDevicePointer(reinterpret_cast<void**>(&st->status.dev), st->status.host, 0);
+  if (e != cudaSuccess) {
+    free_state(st);
+    return cuda_fail(e, "status word allocation");
+  }
+  *st->status.host = 0;
+
+  const size_t nW = weight_elems(c);
+  if (c.rule == TTT_RULE_INPLACE_HEBBIAN) {
+    guard(dev_alloc((void**)&st->ip.W, nW * 4, "W")) && guard(dev_alloc((void**)&st->ip.W0, nW * 4, "W0"));
+    if (r == TTT_OK && c.io_dtype == TTT_BF16) {
+      guard(dev_alloc((void**)&st->ip.Wsh[0], nW * 2, "W bf16 copy")) &&
+          guard(dev_alloc((void**)&st->ip.Wsh[1], nW * 2, "W bf16 copy"));
+    }
+    if (r == TTT_OK && target) {
+      const size_t dd = (size_t)c.d_val * c.d_val;
+      guard(dev_alloc((void**)&st->ip.Wtarget, dd * 2, "Wtarget")) &&
+          guard(dev_alloc((void**)&st->ip.convw, (size_t)c.d_val * c.conv_taps * 4, "convw")) &&
+          guard(dev_alloc((void**)&st->ip.conv, (size_t)c.chunk * c.d_val * 2, "conv buffer")) &&
+          guard(dev_alloc((void**)&st->ip.Vhat[0], (size_t)c.chunk * c.d_val * 2, "target buffer")) &&
+          guard(dev_alloc((void**)&st->ip.Vhat[1], (size_t)c.chunk * c.d_val * 2, "target buffer"));
+    }
+  } else {
+    guard(dev_alloc((void**)&st->lin.W, nW * 4, "W")) && guard(dev_alloc((void**)&st->lin.W0, nW * 4, "W0"));
+    const size_t bh = (size_t)c.batch * c.heads;
+    const int cap = c.gate_enable ? c.cache_capacity : 1;
+    st->cfg.cache_capacity = cap;
+    if (r == TTT_OK) {
+      guard(dev_alloc((void**)&st->gate.tau, bh * 4, "tau")) &&
+          guard(dev_alloc((void**)&st->gate.tau_set, bh * 4, "tau_set")) &&
+          guard(dev_alloc((void**)&st->gate.entries, bh * (size_t)cap * 3 * 4, "cache")) &&
+          guard(dev_alloc((void**)&st->gate.counts, bh * 2 * 4, "cache counts"));
+    }
+  }
+  if (r != TTT_OK) {
+    free_state(st);
+    return r;
+  }
+  float* W0dst = c.rule == TTT_RULE_INPLACE_HEBBIAN ? st->ip.W0 : st->lin.W0;
+  e = cudaMemcpyAsync(W0dst, W0, nW * 4, cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess && target) {
+    e = cudaMemcpyAsync(st->ip.Wtarget, Wtarget, (size_t)c.d_val * c.d_val * 2, cudaMemcpyDeviceToDevice, s);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(st->ip.convw, convw, (size_t)c.d_val * c.conv_taps * 4, cudaMemcpyDeviceToDevice, s);
+  }
+  if (e != cudaSuccess) {
+    free_state(st);
+    return cuda_fail(e, "copying the initial weights");
+  }
+  r = load_weights(st, W0dst, s);
+  if (r == TTT_OK && c.rule == TTT_RULE_LINEAR_GD) r = gate_reset(st, s);
+  if (r != TTT_OK) {
+    free_state(st);
+    return r;
+  }
+  *out = st;
+  return TTT_OK;
+}
+
+static ttt_status check_device(const ttt_state* st) {
+  int dev = -1;
+  TTT_CUDA(cudaGetDevice(&dev));
+  if (dev != st->device) return fail(TTT_ERR_INVALID_ARG, "current device %d is not the state's device %d", dev, st->device);
+  return TTT_OK;
+}
+
+static ttt_status scan_impl(ttt_state* st, const void* keys, const void* targets, const void* queries,
+                            int64_t T, void* out, float* loss, cudaStream_t s) {
+  const ttt_config& c = st->cfg;
+  if (T < 0) return fail(TTT_ERR_INVALID_ARG, "T must be non-negative");
+  if (T % c.chunk != 0) return fail(TTT_ERR_INVALID_ARG, "T=%lld is not a multiple of the chunk %d", (long long)T, c.chunk);
+  if (T > (int64_t)INT32_MAX / 2) return fail(TTT_ERR_UNSUPPORTED, "T too large");
+  if (T == 0) return TTT_OK;
+  TTT_TRY(check_device(st));
+  if (keys == nullptr || targets == nullptr || !aligned16(keys) || !aligned16(targets))
+    return fail(TTT_ERR_INVALID_ARG, "keys and targets must be 16-byte aligned device pointers");
+  if (c.rule == TTT_RULE_INPLACE_HEBBIAN) {
+    if (queries != nullptr || loss != nullptr)
+      return fail(TTT_ERR_INVALID_ARG, "In-Place scan takes no queries and no loss output");
+    if (out == nullptr || !aligned16(out)) return fail(TTT_ERR_INVALID_ARG, "out must be a 16-byte aligned device pointer");
+    if (c.io_dtype == TTT_F32) {
+      const float* Z = static_cast<const float*>(keys);
+      const float* V = static_cast<const float*>(targets);
+      float* O = static_cast<float*>(out);
+      for (int64_t t0 = 0; t0 < T; t0 += c.chunk)
+        TTT_TRY(inplace_f32_chunk(st, Z + t0 * c.d_key, V + t0 * c.d_val, O + t0 * c.d_val, c.chunk, s));
+      return TTT_OK;
+    }
+    return inplace_bf16_scan(st, static_cast<const __nv_bfloat16*>(keys),
+                             static_cast<const __nv_bfloat16*>(targets), T,
+                             static_cast<__nv_bfloat16*>(out), s);
+  }
+  if ((queries == nullptr) != (out == nullptr))
+    return fail(TTT_ERR_INVALID_ARG, "TTT-Linear: out must be given exactly when queries are");
+  if (queries != nullptr && (!aligned16(queries) || !aligned16(out)))
+    return fail(TTT_ERR_INVALID_ARG, "queries and out must be 16-byte aligned");
+  if (loss != nullptr && !aligned16(loss)) return fail(TTT_ERR_INVALID_ARG, "loss_out must be 16-byte aligned");
+  if (c.gate_enable) {
+    if (loss == nullptr) return fail(TTT_ERR_INVALID_ARG, "the gate needs loss_out");
+    if (T % c.gate_chunk != 0) return fail(TTT_ERR_INVALID_ARG, "T must be a multiple of gate_chunk with the gate on");
+  }
+  TTT_TRY(linear_scan(st, static_cast<const __nv_bfloat16*>(keys), static_cast<const __nv_bfloat16*>(targets),
+                      static_cast<const __nv_bfloat16*>(queries), T, static_cast<__nv_bfloat16*>(out), loss, s));
+  if (c.gate_enable) TTT_TRY(gate_route(st, loss, T, s));
+  return TTT_OK;
+}
+
+static ttt_status ensure_staging(ttt_state* st, int i, size_t bytes) {
+  if (st->staging.bytes[i] >= bytes) return TTT_OK;
+  dev_free(st->staging.buf[i]);
+  st->staging.buf[i] = nullptr;
+  st->staging.bytes[i] = 0;
+  TTT_TRY(dev_alloc(&st->staging.buf[i], bytes, "host-call staging buffer"));
+  st->staging.bytes[i] = bytes;
+  return TTT_OK;
+}
+
+}  // namespace ttt
+
+using namespace ttt;
+
+extern "C" {
+
+int32_t ttt_abi_version(void) { return 1; }
+
+const char* ttt_last_error_string(void) { return ttt::g_last_error; }
+
+ttt_status ttt_config_init(ttt_config* cfg, int32_t rule) {
+  if (cfg == nullptr) return fail(TTT_ERR_INVALID_ARG, "cfg is NULL");
+  if (rule != TTT_RULE_INPLACE_HEBBIAN && rule != TTT_RULE_LINEAR_GD) return fail(TTT_ERR_INVALID_ARG, "unknown rule %d", rule);
+  memset(cfg, 0, sizeof(*cfg));
+  cfg->rule = rule;
+  cfg->io_dtype = TTT_BF16;
+  cfg->batch = 1;
+  cfg->heads = 1;
+  cfg->d_key = 64;
+  cfg->d_val = 64;
+  cfg->chunk = rule == TTT_RULE_LINEAR_GD ? 16 : 1024;
+  cfg->eta = 1.0f;
+  cfg->conv_taps = 3;
+  cfg->gate_chunk = 64;
+  cfg->cache_capacity = 256;
+  cfg->gate_pct = 0.95f;
+  cfg->gate_ema_old = 0.9f;
+  cfg->gate_ema_new = 0.1f;
+  cfg->gate_mean_num = 4;
+  cfg->gate_mean_den = 5;
+  return TTT_OK;
+}
+
+ttt_status ttt_state_create(const ttt_config* cfg, const void* W0, const void* Wtarget, const float* convw,
+                            ttt_stream stream, ttt_state** out) {
+  if (out == nullptr) return fail(TTT_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  if (cfg == nullptr) return fail(TTT_ERR_INVALID_ARG, "cfg is NULL");
+  return create_impl(cfg, W0, Wtarget, convw, reinterpret_cast<cudaStream_t>(stream), out);
+}
+
+ttt_status ttt_chunk_scan(ttt_state* st, const void* keys, const void* targets, const void* queries, int64_t T,
+                          void* out, float* loss_out, ttt_stream stream) {
+  if (st == nullptr) return fail(TTT_ERR_INVALID_ARG, "state is NULL");
+  return scan_impl(st, keys, targets, queries, T, out, loss_out, reinterpret_cast<cudaStream_t>(stream));
+}
+
+ttt_status ttt_chunk_scan_host(ttt_state* st, const void* keys, const void* targets, const void* queries,
+                               int64_t T, void* out, float* loss_out, ttt_stream stream) {
+  if (st == nullptr) return fail(TTT_ERR_INVALID_ARG, "state is NULL");
+  const ttt_config& c = st->cfg;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (T < 0 || T % c.chunk != 0) return fail(TTT_ERR_INVALID_ARG, "T must be a non-negative multiple of the chunk");
+  if (T == 0) return TTT_OK;
+  if (keys == nullptr || targets == nullptr) return fail(TTT_ERR_INVALID_ARG, "keys and targets are required");
+  const size_t es = io_size(c.io_dtype);
+  const size_t bh = (size_t)c.batch * c.heads;
+  const size_t kb = bh * T * c.d_key * es;
+  const size_t vb = bh * T * c.d_val * es;
+  const size_t ob = c.rule == TTT_RULE_INPLACE_HEBBIAN ? T * c.d_val * es : bh * T * c.d_key * es;
+  const size_t lb = bh * T * sizeof(float);
+  TTT_TRY(check_device(st));
+  TTT_TRY(ensure_staging(st, 0, kb));
+  TTT_TRY(ensure_staging(st, 1, vb));
+  if (queries != nullptr) TTT_TRY(ensure_staging(st, 2, kb));
+  if (out != nullptr) TTT_TRY(ensure_staging(st, 3, ob));
+  if (loss_out != nullptr) TTT_TRY(ensure_staging(st, 4, lb));
+  TTT_CUDA(cudaMemcpyAsync(st->staging.buf[0], keys, kb, cudaMemcpyHostToDevice, s));
+  TTT_CUDA(cudaMemcpyAsync(st->staging.buf[1], targets, vb, cudaMemcpyHostToDevice, s));
+  if (queries != nullptr) TTT_CUDA(cudaMemcpyAsync(st->staging.buf[2], queries, kb, cudaMemcpyHostToDevice, s));
+  TTT_TRY(scan_impl(st, st->staging.buf[0], st->staging.buf[1], queries ? st->staging.buf[2] : nullptr, T,
+                    out ? st->staging.buf[3] : nullptr, loss_out ? static_cast<float*>(st->staging.buf[4]) : nullptr,
+                    s));
+  if (out != nullptr) TTT_CUDA(cudaMemcpyAsync(out, st->staging.buf[3], ob, cudaMemcpyDeviceToHost, s));
+  if (loss_out != nullptr) TTT_CUDA(cudaMemcpyAsync(loss_out, st->staging.buf[4], lb, cudaMemcpyDeviceToHost, s));
+  TTT_CUDA(cudaStreamSynchronize(s));
+  return TTT_OK;
+}
+
+ttt_status ttt_surprisal_route(ttt_state* st, const float* loss, int64_t T, ttt_stream stream) {
+  if (st == nullptr) return fail(TTT_ERR_INVALID_ARG, "state is NULL");
+  if (st->cfg.rule != TTT_RULE_LINEAR_GD) return fail(TTT_ERR_UNSUPPORTED, "the surprisal gate runs on TTT-Linear states");
+  if (!st->cfg.gate_enable) return fail(TTT_ERR_INVALID_ARG, "the state was created with gate_enable = 0");
+  if (T < 0 || T % st->cfg.gate_chunk != 0) return fail(TTT_ERR_INVALID_ARG, "T must be a non-negative multiple of gate_chunk");
+  if (T == 0) return TTT_OK;
+  if (loss == nullptr || !aligned16(loss)) return fail(TTT_ERR_INVALID_ARG, "loss must be a 16-byte aligned device pointer");
+  TTT_TRY(check_device(st));
+  return gate_route(st, loss, T, reinterpret_cast<cudaStream_t>(stream));
+}
+
+ttt_status ttt_state_reset(ttt_state* st, ttt_stream stream) {
+  if (st == nullptr) return fail(TTT_ERR_INVALID_ARG, "state is NULL");
+  TTT_TRY(check_device(st));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  TTT_TRY(load_weights(st, st->cfg.rule == TTT_RULE_INPLACE_HEBBIAN ? st->ip.W0 : st->lin.W0, s));
+  if (st->cfg.rule == TTT_RULE_LINEAR_GD) TTT_TRY(gate_reset(st, s));
+  return TTT_OK;
+}
+
+ttt_status ttt_state_get_weights(const ttt_state* st, float* W, ttt_stream stream) {
+  if (st == nullptr || W == nullptr) return fail(TTT_ERR_INVALID_ARG, "state and W are required");
+  const float* src = st->cfg.rule == TTT_RULE_INPLACE_HEBBIAN ? st->ip.W : st->lin.W;
+  TTT_CUDA(cudaMemcpyAsync(W, src, weight_elems(st->cfg) * 4, cudaMemcpyDeviceToDevice,
+                           reinterpret_cast<cudaStream_t>(stream)));
+  return TTT_OK;
+}
+
+ttt_status ttt_state_set_weights(ttt_state* st, const float* W, ttt_stream stream) {
+  if (st == nullptr || W == nullptr || !aligned16(W)) return fail(TTT_ERR_INVALID_ARG, "state and an aligned W are required");
+  TTT_TRY(check_device(st));
+  return load_weights(st, W, reinterpret_cast<cudaStream_t>(stream));
+}
+
+ttt_status ttt_cache_read(const ttt_state* st, int32_t* entries, int32_t* counts, ttt_stream stream) {
+  if (st == nullptr) return fail(TTT_ERR_INVALID_ARG, "state is NULL");
+  if (st->cfg.rule != TTT_RULE_LINEAR_GD) return fail(TTT_ERR_UNSUPPORTED, "In-Place states have no residual cache");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t bh = (size_t)st->cfg.batch * st->cfg.heads;
+  if (entries != nullptr)
+    TTT_CUDA(cudaMemcpyAsync(entries, st->gate.entries, bh * st->cfg.cache_capacity * 3 * 4, cudaMemcpyDeviceToDevice, s));
+  if (counts != nullptr) TTT_CUDA(cudaMemcpyAsync(counts, st->gate.counts, bh * 2 * 4, cudaMemcpyDeviceToDevice, s));
+  return TTT_OK;
+}
+
+ttt_status ttt_gate_read(const ttt_state* st, float* tau, int32_t* tau_set, ttt_stream stream) {
+  if (st == nullptr) return fail(TTT_ERR_INVALID_ARG, "state is NULL");
+  if (st->cfg.rule != TTT_RULE_LINEAR_GD) return fail(TTT_ERR_UNSUPPORTED, "In-Place states have no gate");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t bh = (size_t)st->cfg.batch * st->cfg.heads;
+  if (tau != nullptr) TTT_CUDA(cudaMemcpyAsync(tau, st->gate.tau, bh * 4, cudaMemcpyDeviceToDevice, s));
+  if (tau_set != nullptr) TTT_CUDA(cudaMemcpyAsync(tau_set, st->gate.tau_set, bh * 4, cudaMemcpyDeviceToDevice, s));
+  return TTT_OK;
+}
+
+ttt_status ttt_state_poll(ttt_state* st) {
+  if (st == nullptr) return fail(TTT_ERR_INVALID_ARG, "state is NULL");
+  TTT_CUDA(cudaDeviceSynchronize());
+  volatile int* w = st->status.host;
+  const int v = *w;
+  *w = 0;
+  if (v == 0) return TTT_OK;
+  if (v == TTT_ERR_TIMEOUT) return fail(TTT_ERR_TIMEOUT, "a bounded device-side wait ran out");
+  return fail(TTT_ERR_DEVICE, "a device-side check failed (code %d)", v);
+}
+
+int64_t ttt_state_launch_count(const ttt_state* st) { return st == nullptr ? 0 : st->launches; }
+
+ttt_status ttt_state_destroy(ttt_state* st) {
+  if (st == nullptr) return TTT_OK;
+  cudaError_t e = cudaDeviceSynchronize();
+  free_state(st);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize in destroy");
+  return TTT_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,177 @@
+/*
+ * ttt.h — C ABI of libttt.so, the fast-weight (test-time-training) chunk scan on one
+ * NVIDIA B200 (sm_100a).
+ *
+ * What the library computes (sources are the pages' titles and sections):
+ *
+ *  In-Place rule ("In-Place Test-Time Training", §2, §3, §4, §6). The fast weight is the
+ *  gated MLP's down projection Wdown [d_model x d_ff]. The sequence is cut into chunks of
+ *  C tokens. For chunk c, first O_c = Z_c · W_cᵀ with the weight from before this chunk
+ *  (chunk 0 uses the pretrained W0), then W_{c+1} = W_c + η · V̂_cᵀ · Z_c. The target is
+ *  either given (V̂) or produced as V̂ = Conv1D(X0) · Wtarget with depthwise taps at token
+ *  offsets 0, +1, +2 that read zero past the end of the token's chunk.
+ *
+ *  TTT-Linear rule ("テスト時学習（Test-Time Training）とは", the TTT layers page: the
+ *  hidden state is a linear model updated by one self-supervised gradient step). Per
+ *  (sequence, head), for each inner mini-batch i of b tokens: O_i = Q_i · W_i,
+ *  R_i = K_i · W_i − V_i, L_t = ‖R_i[t]‖², W_{i+1} = W_i − (η/b) · K_iᵀ · R_i.
+ *
+ *  Surprisal gate ("SR-TTT: Surprisal-Aware Residual Test-Time Training", §2.1). Per
+ *  (sequence, head) and chunk of 64 losses: p95 = 61st smallest; τ = p95 for the first
+ *  chunk, else τ = fl32(fl32(0.9·τ) + fl32(0.1·p95)); the chunk passes if
+ *  5·S ≥ 256·τ with S the double sum of its losses in index order; a token of a passing
+ *  chunk is routed if L_t > τ. Routed (sequence, head, t) triples are appended in
+ *  increasing t to that (sequence, head)'s cache until it is full; later ones are counted
+ *  as dropped.
+ *
+ * Conventions shared by every entry point:
+ *  - Every pointer argument marked "device" must point to memory of the CUDA device that
+ *    was current when the state was created, be 16-byte aligned and be densely packed in
+ *    the row-major layout stated for it. The caller owns all such buffers; the library
+ *    never frees or retains them beyond the call.
+ *  - All work is enqueued on `stream` (a cudaStream_t; NULL is the legacy default
+ *    stream). No call synchronises the device except ttt_state_poll(),
+ *    ttt_chunk_scan_host() and ttt_state_destroy().
+ *  - A call returns TTT_OK or an error status and never aborts the process. The message
+ *    of the last error on the calling thread is returned by ttt_last_error_string().
+ *  - Failures detected on the device (a bounded wait that ran out, a failed device-side
+ *    check) are recorded in the state's status word and returned by the next call of
+ *    ttt_state_poll().
+ */
+#ifndef TTT_H_
+#define TTT_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; declared here so this header needs no CUDA include. */
+typedef struct CUstream_st* ttt_stream;
+
+typedef enum {
+  TTT_OK = 0,
+  TTT_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size, T not a multiple of the chunk */
+  TTT_ERR_UNSUPPORTED = 2, /* a valid configuration this library does not implement */
+  TTT_ERR_OOM = 3,         /* device or pinned host allocation failed */
+  TTT_ERR_CUDA = 4,        /* a CUDA runtime or driver call failed */
+  TTT_ERR_TIMEOUT = 5,     /* a bounded device-side wait ran out (from ttt_state_poll) */
+  TTT_ERR_DEVICE = 6       /* a device-side consistency check failed (from ttt_state_poll) */
+} ttt_status;
+
+typedef enum { TTT_RULE_INPLACE_HEBBIAN = 0, TTT_RULE_LINEAR_GD = 1 } ttt_rule;
+typedef enum { TTT_F32 = 0, TTT_BF16 = 1 } ttt_dtype;
+
+typedef struct {
+  int32_t rule;           /* ttt_rule */
+  int32_t io_dtype;       /* ttt_dtype of keys, targets, queries and out. The weight state is
+                             always fp32. In-Place: F32 (SIMT FFMA) or BF16 (tensor cores).
+                             TTT-Linear: BF16. */
+  int32_t batch, heads;   /* TTT-Linear: sequences and heads per sequence. In-Place: 1 and 1. */
+  int32_t d_key;          /* In-Place: d_ff = f, columns of Wdown. TTT-Linear: head width (64). */
+  int32_t d_val;          /* In-Place: d_model = d, rows of Wdown. TTT-Linear: head width (64). */
+  int32_t chunk;          /* In-Place: chunk C. TTT-Linear: inner mini-batch b (multiple of 16,
+                             at most 64). */
+  float eta;              /* learning rate η */
+  int32_t target_mode;    /* In-Place only. 0: targets are V̂ [T, d]. 1: targets are X0 [T, d]
+                             and V̂ = Conv1D(X0)·Wtarget is produced inside the scan (BF16). */
+  int32_t conv_pad_mode;  /* 0: taps read zero past the token's chunk end (default).
+                             1: taps read zero past the end of the call's tokens only. */
+  int32_t conv_taps;      /* number of future taps (offsets 0 .. conv_taps-1); 3 */
+  int32_t gate_enable;    /* TTT-Linear only: run the surprisal gate on the scan's losses */
+  int32_t gate_chunk;     /* tokens per gate chunk; 64 */
+  int32_t cache_capacity; /* residual cache entries per (sequence, head); 256 */
+  float gate_pct;         /* percentile of the threshold (nearest rank); 0.95 */
+  float gate_ema_old;     /* weight on the previous τ; 0.9f */
+  float gate_ema_new;     /* weight on the chunk's percentile; 0.1f */
+  int32_t gate_mean_num;  /* the mean test is S/gate_chunk >= (num/den)·τ; 4 */
+  int32_t gate_mean_den;  /* 5 */
+} ttt_config;
+
+typedef struct ttt_state ttt_state; /* opaque; owns all of its device memory */
+
+/* ABI version of this header (incremented on any incompatible change). */
+int32_t ttt_abi_version(void);
+
+/* Fill *cfg with the defaults of `rule` (the values noted above, eta = 1, chunk 16 for
+ * TTT-Linear, 1024 for In-Place, BF16). INVALID_ARG if cfg is NULL or rule unknown. */
+ttt_status ttt_config_init(ttt_config* cfg, int32_t rule);
+
+/* Create a scan state on the current device and copy the initial weights into it.
+ *   W0       device. In-Place: fp32 [d_val, d_key] (Wdown, row-major).
+ *                    TTT-Linear: fp32 [batch, heads, d_key, d_key], applied as x·W.
+ *   Wtarget  device, In-Place with target_mode 1 only (else NULL): bf16 [d_val, d_val],
+ *            [in, out], V̂[t, j] = Σ_i conv[t, i]·Wtarget[i, j].
+ *   convw    device, target_mode 1 only (else NULL): fp32 [d_val, conv_taps].
+ * W0, Wtarget and convw are copied; the caller may free them after the call returns
+ * (stream-ordered). On success *out receives the state; on error *out is NULL and
+ * nothing is leaked. Errors: INVALID_ARG (bad sizes or pointers), UNSUPPORTED (shape or
+ * mode not implemented, see the message), OOM, CUDA. */
+ttt_status ttt_state_create(const ttt_config* cfg, const void* W0, const void* Wtarget,
+                            const float* convw, ttt_stream stream, ttt_state** out);
+
+/* Continue the scan over the next T tokens (successive calls form one scan).
+ *   In-Place:   keys = Z [T, d_key]; targets = V̂ [T, d_val] (target_mode 0) or X0 [T, d_val]
+ *               (target_mode 1); queries must be NULL; out = O [T, d_val] (required);
+ *               loss_out must be NULL. T must be a multiple of chunk.
+ *   TTT-Linear: keys = K, targets = V, queries = Q (or NULL), all [batch, heads, T, d_key];
+ *               out = O [batch, heads, T, d_key] (NULL iff queries is NULL);
+ *               loss_out = L [batch, heads, T] fp32 (or NULL; required when the gate is
+ *               enabled). T must be a multiple of chunk (and of gate_chunk with the gate).
+ * All inputs are read-only; outputs are written with the io dtype (loss fp32). Inputs and
+ * outputs must not overlap. T = 0 is a no-op. Errors: INVALID_ARG, UNSUPPORTED, CUDA. */
+ttt_status ttt_chunk_scan(ttt_state* st, const void* keys, const void* targets,
+                          const void* queries, int64_t T, void* out, float* loss_out,
+                          ttt_stream stream);
+
+/* ttt_chunk_scan with HOST buffers of the same shapes: copies the inputs to device
+ * staging buffers owned by the state (grown on demand), runs the scan, copies the outputs
+ * back and synchronises `stream`. Host buffers should be pinned for full speed. */
+ttt_status ttt_chunk_scan_host(ttt_state* st, const void* keys, const void* targets,
+                               const void* queries, int64_t T, void* out, float* loss_out,
+                               ttt_stream stream);
+
+/* Run the surprisal gate alone on a loss array `loss` (device, fp32 [batch, heads, T]),
+ * advancing the state's τ, cache and token position exactly as a gated scan would.
+ * TTT-Linear states only; T must be a multiple of gate_chunk. */
+ttt_status ttt_surprisal_route(ttt_state* st, const float* loss, int64_t T, ttt_stream stream);
+
+/* Document boundary: W ← W0, τ unset, cache emptied (entries -1, counts 0), token
+ * position 0. */
+ttt_status ttt_state_reset(ttt_state* st, ttt_stream stream);
+
+/* Copy the current fp32 weights out of / into the state (device buffers shaped like W0).
+ * set_weights also refreshes the In-Place bf16 copy used by the apply. */
+ttt_status ttt_state_get_weights(const ttt_state* st, float* W, ttt_stream stream);
+ttt_status ttt_state_set_weights(ttt_state* st, const float* W, ttt_stream stream);
+
+/* Copy out the residual cache: entries (device) int32 [batch, heads, cache_capacity, 3]
+ * holding (sequence, head, t) with t counted from the last reset, unused entries -1;
+ * counts (device) int32 [batch, heads, 2] = (tokens routed, routed tokens dropped).
+ * Either pointer may be NULL. */
+ttt_status ttt_cache_read(const ttt_state* st, int32_t* entries, int32_t* counts,
+                          ttt_stream stream);
+
+/* Copy out the gate thresholds: tau (device) fp32 [batch, heads]; tau_set (device) int32
+ * [batch, heads], 1 once a chunk has set τ. Either pointer may be NULL. */
+ttt_status ttt_gate_read(const ttt_state* st, float* tau, int32_t* tau_set, ttt_stream stream);
+
+/* Synchronise the device and return the first device-side failure recorded since the
+ * last poll (TTT_ERR_TIMEOUT or TTT_ERR_DEVICE), or TTT_OK; clears the record. */
+ttt_status ttt_state_poll(ttt_state* st);
+
+/* Number of kernels this state has launched since creation. */
+int64_t ttt_state_launch_count(const ttt_state* st);
+
+/* Synchronise the device and free everything the state owns. NULL is a no-op. */
+ttt_status ttt_state_destroy(ttt_state* st);
+
+/* Message of the last error returned on the calling thread ("" if none). */
+const char* ttt_last_error_string(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TTT_H_ */

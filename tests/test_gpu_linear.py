@@ -1,0 +1,121 @@
+"""GPU parity of the TTT-Linear mini-batch scan against the oracle."""
+
+import numpy as np
+import pytest
+import torch
+
+from gen import workloads
+from oracle import linear as ora
+from tests._util import rel_err
+
+pytestmark = pytest.mark.gpu
+
+TOL = 2e-2  # max|err| / max|ref| for bf16 inputs with fp32 accumulation
+
+
+@pytest.fixture(scope="module")
+def cwl():
+    from chunked_weight_layers_b200 import build
+    build.build()
+    import chunked_weight_layers_b200 as cwl
+    return cwl
+
+
+def run_linear(cwl, x, b, eta, with_q=True, loss=True):
+    K, V = x["K"], x["V"]
+    B, H, T, D = K.shape
+    cfg = cwl.config("linear", batch=B, heads=H, d_key=D, d_val=D, chunk=b, eta=eta)
+    st = cwl.FastWeightState(cfg, x["W0"])
+    Q = x.get("Q") if with_q else None
+    O = torch.empty_like(K) if Q is not None else None
+    L = torch.empty((B, H, T), device="cuda", dtype=torch.float32) if loss else None
+    st.chunk_scan(K, V, Q, out=O, loss_out=L)
+    W = torch.empty_like(x["W0"])
+    st.get_weights(W)
+    torch.cuda.synchronize()
+    st.poll()
+    return O, W, L, st
+
+
+def test_linear_workload_full_size(cwl):
+    spec = workloads.LINEAR_GD
+    x = workloads.linear_inputs(spec, device="cuda")
+    O, W, L, st = run_linear(cwl, x, spec.b, spec.eta)
+    Oref, Wref, Lref = ora.ttt_linear_scan(x["K"].cpu(), x["V"].cpu(), x["Q"].cpu(), x["W0"].cpu(), spec.eta, spec.b)
+    eo, ew, el = rel_err(O, Oref), rel_err(W, Wref), rel_err(L, Lref)
+    print(f"TTT-Linear workload: O {eo:.3e}  W {ew:.3e}  loss {el:.3e}")
+    assert eo <= TOL and ew <= TOL and el <= TOL
+    # Much tighter than the tolerance thanks to the hi/lo operand split; a regression to a
+    # single bf16 operand would show up here first.
+    assert max(eo, ew, el) <= 5e-3
+    assert st.launch_count() >= 1
+
+
+def test_identity_fixed_point_is_exact(cwl):
+    """W0 = I and V = K: every residual is exactly 0, W stays I, O = Q, losses 0."""
+    spec = workloads.scaled(workloads.LINEAR_GD, B=2, H=3, T=320)
+    x = workloads.linear_inputs(spec, device="cuda")
+    x["V"] = x["K"].clone()
+    O, W, L, _ = run_linear(cwl, x, 16, 1.0)
+    assert torch.equal(W, x["W0"])
+    assert torch.equal(O, x["Q"])
+    assert torch.count_nonzero(L).item() == 0
+
+
+@pytest.mark.parametrize("b,T", [(16, 208), (32, 224), (64, 192), (16, 64)])
+def test_small_shapes_and_ragged_tiles(cwl, b, T):
+    spec = workloads.scaled(workloads.LINEAR_GD, B=2, H=3, T=T, b=b, seed=77 + b)
+    x = workloads.linear_inputs(spec, device="cuda")
+    W0 = x["W0"].clone()
+    W0 += 0.05 * torch.randn(W0.shape, generator=torch.Generator().manual_seed(b)).cuda()
+    x["W0"] = W0
+    O, W, L, _ = run_linear(cwl, x, b, 0.5)
+    Oref, Wref, Lref = ora.ttt_linear_scan(x["K"].cpu(), x["V"].cpu(), x["Q"].cpu(), W0.cpu(), 0.5, b)
+    errs = rel_err(O, Oref), rel_err(W, Wref), rel_err(L, Lref)
+    assert max(errs) <= 5e-3, errs
+
+
+def test_without_queries_same_state_and_loss(cwl):
+    spec = workloads.scaled(workloads.LINEAR_GD, B=1, H=4, T=256)
+    x = workloads.linear_inputs(spec, device="cuda")
+    _, W1, L1, _ = run_linear(cwl, x, 16, 1.0)
+    _, W2, L2, _ = run_linear(cwl, x, 16, 1.0, with_q=False)
+    assert torch.equal(W1, W2) and torch.equal(L1, L2)
+
+
+def test_streaming_split_equals_one_call(cwl):
+    spec = workloads.scaled(workloads.LINEAR_GD, B=2, H=2, T=320)
+    x = workloads.linear_inputs(spec, device="cuda")
+    O1, W1, L1, _ = run_linear(cwl, x, 16, 1.0)
+    B, H, T, D = x["K"].shape
+    cfg = cwl.config("linear", batch=B, heads=H, chunk=16, eta=1.0)
+    st = cwl.FastWeightState(cfg, x["W0"])
+    outs, losses = [], []
+    for a, z in ((0, 112), (112, T)):
+        K, V, Q = (x[n][:, :, a:z].contiguous() for n in ("K", "V", "Q"))
+        O = torch.empty_like(K)
+        L = torch.empty((B, H, z - a), device="cuda")
+        st.chunk_scan(K, V, Q, out=O, loss_out=L)
+        outs.append(O)
+        losses.append(L)
+    W = torch.empty_like(x["W0"])
+    st.get_weights(W)
+    torch.cuda.synchronize()
+    assert torch.equal(torch.cat(outs, 2), O1) and torch.equal(torch.cat(losses, 2), L1)
+    assert torch.equal(W, W1)
+
+
+def test_rejects_bad_arguments(cwl):
+    from chunked_weight_layers_b200 import TTTError, abi
+    W0 = torch.eye(64, device="cuda").expand(1, 2, 64, 64).contiguous()
+    st = cwl.FastWeightState(cwl.config("linear", batch=1, heads=2, chunk=16), W0)
+    K = torch.zeros(1, 2, 40, 64, device="cuda", dtype=torch.bfloat16)
+    with pytest.raises(TTTError) as e:
+        st.chunk_scan(K, K, K, out=torch.empty_like(K))  # 40 is not a multiple of 16
+    assert e.value.status == abi.TTT_ERR_INVALID_ARG
+    with pytest.raises(TTTError) as e:
+        st.chunk_scan(K[:, :, :32].contiguous(), K[:, :, :32].contiguous(), K[:, :, :32].contiguous(), out=None)
+    assert e.value.status == abi.TTT_ERR_INVALID_ARG
+    with pytest.raises(TTTError) as e:
+        cwl.FastWeightState(cwl.config("linear", batch=1, heads=2, chunk=24), W0)
+    assert e.value.status == abi.TTT_ERR_UNSUPPORTED
