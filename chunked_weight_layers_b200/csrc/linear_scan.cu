@@ -78,6 +78,124 @@ __device__ __forceinline__ float2 unpack_bf16(uint32_t v) {
   return __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&v));
 }
 
+// One inner mini-batch of 16 tokens (tile rows r0 .. r0+15) for the warp owning W columns
+// [col0, col0+16). The work is ordered so that consecutive mma instructions are independent:
+// all operand fragments are loaded first, P is accumulated in four partial sums (one per
+// 16-key slice, hi then lo), the output product is issued between the two halves of P, and
+// the loss and output stores come after the weight update has been issued.
+//   Pᵀ = Wᵀ·Kᵀ with W as bf16 hi + lo (the chain's only operand that is not exact in bf16),
+//   Rᵀ = Pᵀ − Vᵀ, loss, Oᵀ = Wᵀ_hi·Qᵀ (the output is stored in bf16 anyway),
+//   Wᵀ += Sᵀ·K with S = −(η/b)·R rounded to bf16.
+__device__ __forceinline__ void step16(float (&acc)[8][4], uint32_t kbase, uint32_t vbase, uint32_t qbase,
+                                       uint8_t* obuf, float* lossp, int r0, int lane, int col0, float beta,
+                                       int has_q, bool want_loss) {
+  const int g = lane >> 2, q = lane & 3, mi = lane >> 3, ri = lane & 7;
+  uint32_t kb[2][2][4], kt[4][4], vf[4], qb[2][2][4];
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+    for (int kp = 0; kp < 2; ++kp) ldsm_x4(kbase + swz128_bf16(r0 + 8 * nt + ri, 32 * kp + 8 * mi), kb[nt][kp]);
+  ldsm_x4_t(vbase + swz128_bf16(r0 + 8 * (mi >> 1) + ri, col0 + 8 * (mi & 1)), vf);
+#pragma unroll
+  for (int np = 0; np < 4; ++np) ldsm_x4_t(kbase + swz128_bf16(r0 + 8 * (mi & 1) + ri, 16 * np + 8 * (mi >> 1)), kt[np]);
+  if (has_q) {
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int kp = 0; kp < 2; ++kp) ldsm_x4(qbase + swz128_bf16(r0 + 8 * nt + ri, 32 * kp + 8 * mi), qb[nt][kp]);
+  }
+
+  uint32_t whi[4][4], wlo[4][4];
+#pragma unroll
+  for (int ks = 0; ks < 4; ++ks) {
+    split2(acc[2 * ks][0], acc[2 * ks][1], whi[ks][0], wlo[ks][0]);
+    split2(acc[2 * ks][2], acc[2 * ks][3], whi[ks][1], wlo[ks][1]);
+    split2(acc[2 * ks + 1][0], acc[2 * ks + 1][1], whi[ks][2], wlo[ks][2]);
+    split2(acc[2 * ks + 1][2], acc[2 * ks + 1][3], whi[ks][3], wlo[ks][3]);
+  }
+
+  float pp[2][4][4], o[2][2][4];
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks) pp[nt][ks][e] = 0.f;
+      o[nt][0][e] = 0.f;
+      o[nt][1][e] = 0.f;
+    }
+#pragma unroll
+  for (int ks = 0; ks < 4; ++ks)
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+      mma16816(pp[nt][ks], whi[ks], kb[nt][ks >> 1][2 * (ks & 1)], kb[nt][ks >> 1][2 * (ks & 1) + 1]);
+  if (has_q) {
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks)
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+        mma16816(o[nt][ks & 1], whi[ks], qb[nt][ks >> 1][2 * (ks & 1)], qb[nt][ks >> 1][2 * (ks & 1) + 1]);
+  }
+#pragma unroll
+  for (int ks = 0; ks < 4; ++ks)
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+      mma16816(pp[nt][ks], wlo[ks], kb[nt][ks >> 1][2 * (ks & 1)], kb[nt][ks >> 1][2 * (ks & 1) + 1]);
+
+  // R = P − V: p[nt][e] is R[token 8nt + 2q + (e&1)][column col0 + g + 8(e>>1)].
+  float p[2][4];
+  {
+    const float2 v0 = unpack_bf16(vf[0]), v1 = unpack_bf16(vf[1]), v2 = unpack_bf16(vf[2]), v3 = unpack_bf16(vf[3]);
+    const float vv[2][4] = {{v0.x, v0.y, v1.x, v1.y}, {v2.x, v2.y, v3.x, v3.y}};
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        p[nt][e] = ((pp[nt][0][e] + pp[nt][1][e]) + (pp[nt][2][e] + pp[nt][3][e])) - vv[nt][e];
+  }
+
+  // Weight update Wᵀ += Sᵀ·K (eight independent n-tiles of keys).
+  uint32_t sa[4];
+  sa[0] = pack_bf16(-beta * p[0][0], -beta * p[0][1]);
+  sa[1] = pack_bf16(-beta * p[0][2], -beta * p[0][3]);
+  sa[2] = pack_bf16(-beta * p[1][0], -beta * p[1][1]);
+  sa[3] = pack_bf16(-beta * p[1][2], -beta * p[1][3]);
+#pragma unroll
+  for (int np = 0; np < 4; ++np) {
+    mma16816(acc[2 * np], sa, kt[np][0], kt[np][1]);
+    mma16816(acc[2 * np + 1], sa, kt[np][2], kt[np][3]);
+  }
+
+  // Off the critical path: per-token loss partials and the output tile.
+  if (want_loss) {
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      float l0 = p[nt][0] * p[nt][0] + p[nt][2] * p[nt][2];
+      float l1 = p[nt][1] * p[nt][1] + p[nt][3] * p[nt][3];
+#pragma unroll
+      for (int m = 4; m < 32; m <<= 1) {
+        l0 += __shfl_xor_sync(0xffffffffu, l0, m);
+        l1 += __shfl_xor_sync(0xffffffffu, l1, m);
+      }
+      if (g == 0) {
+        lossp[r0 + 8 * nt + 2 * q] = l0;
+        lossp[r0 + 8 * nt + 2 * q + 1] = l1;
+      }
+    }
+  }
+  if (has_q) {
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int row = r0 + 8 * nt + 2 * q + (e & 1);
+        const int col = col0 + g + 8 * (e >> 1);
+        *reinterpret_cast<__nv_bfloat16*>(obuf + swz128_bf16(row, col)) =
+            __float2bfloat16_rn(o[nt][0][e] + o[nt][1][e]);
+      }
+  }
+}
+
 template <int B>
 __global__ void __launch_bounds__(kThreads, 1)
     k_linear_scan(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -159,113 +277,117 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t qbase = smem_u32(sm.Q[slot]);
     uint8_t* obuf = sm.O[s & 1];
 
-    for (int r0 = 0; r0 < ntok; r0 += B) {
-      // A fragments of Wᵀ (hi and lo) for the four 16-key k-steps.
-      uint32_t whi[4][4], wlo[4][4];
-#pragma unroll
-      for (int ks = 0; ks < 4; ++ks) {
-        split2(acc[2 * ks][0], acc[2 * ks][1], whi[ks][0], wlo[ks][0]);
-        split2(acc[2 * ks][2], acc[2 * ks][3], whi[ks][1], wlo[ks][1]);
-        split2(acc[2 * ks + 1][0], acc[2 * ks + 1][1], whi[ks][2], wlo[ks][2]);
-        split2(acc[2 * ks + 1][2], acc[2 * ks + 1][3], whi[ks][3], wlo[ks][3]);
-      }
-
-      // Pᵀ = −Vᵀ + Wᵀ·Kᵀ and Oᵀ = Wᵀ·Qᵀ for the B tokens of this mini-batch.
-      float p[NT][4], o[NT][4];
-#pragma unroll
-      for (int nt = 0; nt < NT; nt += 2) {
-        // −V[t][c] for tokens r0+8nt.. (two n-tiles) and this warp's 16 columns.
-        uint32_t v[4];
-        const int mi = lane >> 3, ri = lane & 7;
-        ldsm_x4_t(vbase + swz128_bf16(r0 + 8 * (nt + (mi >> 1)) + ri, col0 + 8 * (mi & 1)), v);
-        const float2 v0 = unpack_bf16(v[0]), v1 = unpack_bf16(v[1]), v2 = unpack_bf16(v[2]), v3 = unpack_bf16(v[3]);
-        p[nt][0] = -v0.x; p[nt][1] = -v0.y; p[nt][2] = -v1.x; p[nt][3] = -v1.y;
-        if (nt + 1 < NT) { p[nt + 1][0] = -v2.x; p[nt + 1][1] = -v2.y; p[nt + 1][2] = -v3.x; p[nt + 1][3] = -v3.y; }
-      }
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) o[nt][e] = 0.f;
-        float p2[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int ks = 0; ks < 4; ks += 2) {
-          // B fragments of Kᵀ (and Qᵀ): rows = tokens r0+8nt.., keys 16ks .. 16ks+31.
-          const int mi = lane >> 3, ri = lane & 7;
-          const uint32_t off = swz128_bf16(r0 + 8 * nt + ri, 16 * ks + 8 * mi);
-          uint32_t kb[4];
-          ldsm_x4(kbase + off, kb);
-          mma16816(p[nt], whi[ks], kb[0], kb[1]);
-          mma16816(p2, wlo[ks], kb[0], kb[1]);
-          mma16816(p[nt], whi[ks + 1], kb[2], kb[3]);
-          mma16816(p2, wlo[ks + 1], kb[2], kb[3]);
-          if (has_q) {
-            uint32_t qb[4];
-            ldsm_x4(qbase + off, qb);
-            mma16816(o[nt], whi[ks], qb[0], qb[1]);
-            mma16816(o[nt], wlo[ks], qb[0], qb[1]);
-            mma16816(o[nt], whi[ks + 1], qb[2], qb[3]);
-            mma16816(o[nt], wlo[ks + 1], qb[2], qb[3]);
-          }
+    if constexpr (B == 16) {
+      for (int r0 = 0; r0 < ntok; r0 += 16)
+        step16(acc, kbase, vbase, qbase, obuf, sm.lossp[warp], r0, lane, col0, beta, has_q, loss != nullptr);
+    } else {
+      for (int r0 = 0; r0 < ntok; r0 += B) {
+        // A fragments of Wᵀ (hi and lo) for the four 16-key k-steps.
+        uint32_t whi[4][4], wlo[4][4];
+  #pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          split2(acc[2 * ks][0], acc[2 * ks][1], whi[ks][0], wlo[ks][0]);
+          split2(acc[2 * ks][2], acc[2 * ks][3], whi[ks][1], wlo[ks][1]);
+          split2(acc[2 * ks + 1][0], acc[2 * ks + 1][1], whi[ks][2], wlo[ks][2]);
+          split2(acc[2 * ks + 1][2], acc[2 * ks + 1][3], whi[ks][3], wlo[ks][3]);
         }
-#pragma unroll
-        for (int e = 0; e < 4; ++e) p[nt][e] += p2[e];
-      }
 
-      // Per-token loss: this thread holds R for tokens 8nt+2q, 8nt+2q+1 at columns g, g+8.
-      if (loss != nullptr) {
-#pragma unroll
+        // Pᵀ = −Vᵀ + Wᵀ·Kᵀ and Oᵀ = Wᵀ·Qᵀ for the B tokens of this mini-batch.
+        float p[NT][4], o[NT][4];
+  #pragma unroll
+        for (int nt = 0; nt < NT; nt += 2) {
+          // −V[t][c] for tokens r0+8nt.. (two n-tiles) and this warp's 16 columns.
+          uint32_t v[4];
+          const int mi = lane >> 3, ri = lane & 7;
+          ldsm_x4_t(vbase + swz128_bf16(r0 + 8 * (nt + (mi >> 1)) + ri, col0 + 8 * (mi & 1)), v);
+          const float2 v0 = unpack_bf16(v[0]), v1 = unpack_bf16(v[1]), v2 = unpack_bf16(v[2]), v3 = unpack_bf16(v[3]);
+          p[nt][0] = -v0.x; p[nt][1] = -v0.y; p[nt][2] = -v1.x; p[nt][3] = -v1.y;
+          if (nt + 1 < NT) { p[nt + 1][0] = -v2.x; p[nt + 1][1] = -v2.y; p[nt + 1][2] = -v3.x; p[nt + 1][3] = -v3.y; }
+        }
+  #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-          float l0 = p[nt][0] * p[nt][0] + p[nt][2] * p[nt][2];
-          float l1 = p[nt][1] * p[nt][1] + p[nt][3] * p[nt][3];
-#pragma unroll
-          for (int m = 4; m < 32; m <<= 1) {
-            l0 += __shfl_xor_sync(0xffffffffu, l0, m);
-            l1 += __shfl_xor_sync(0xffffffffu, l1, m);
+  #pragma unroll
+          for (int e = 0; e < 4; ++e) o[nt][e] = 0.f;
+          float p2[4] = {0.f, 0.f, 0.f, 0.f};
+  #pragma unroll
+          for (int ks = 0; ks < 4; ks += 2) {
+            // B fragments of Kᵀ (and Qᵀ): rows = tokens r0+8nt.., keys 16ks .. 16ks+31.
+            const int mi = lane >> 3, ri = lane & 7;
+            const uint32_t off = swz128_bf16(r0 + 8 * nt + ri, 16 * ks + 8 * mi);
+            uint32_t kb[4];
+            ldsm_x4(kbase + off, kb);
+            mma16816(p[nt], whi[ks], kb[0], kb[1]);
+            mma16816(p2, wlo[ks], kb[0], kb[1]);
+            mma16816(p[nt], whi[ks + 1], kb[2], kb[3]);
+            mma16816(p2, wlo[ks + 1], kb[2], kb[3]);
+            if (has_q) {
+              uint32_t qb[4];
+              ldsm_x4(qbase + off, qb);
+              mma16816(o[nt], whi[ks], qb[0], qb[1]);
+              mma16816(o[nt], wlo[ks], qb[0], qb[1]);
+              mma16816(o[nt], whi[ks + 1], qb[2], qb[3]);
+              mma16816(o[nt], wlo[ks + 1], qb[2], qb[3]);
+            }
           }
-          if (g == 0) {
-            sm.lossp[warp][r0 + 8 * nt + 2 * q] = l0;
-            sm.lossp[warp][r0 + 8 * nt + 2 * q + 1] = l1;
+  #pragma unroll
+          for (int e = 0; e < 4; ++e) p[nt][e] += p2[e];
+        }
+
+        // Per-token loss: this thread holds R for tokens 8nt+2q, 8nt+2q+1 at columns g, g+8.
+        if (loss != nullptr) {
+  #pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            float l0 = p[nt][0] * p[nt][0] + p[nt][2] * p[nt][2];
+            float l1 = p[nt][1] * p[nt][1] + p[nt][3] * p[nt][3];
+  #pragma unroll
+            for (int m = 4; m < 32; m <<= 1) {
+              l0 += __shfl_xor_sync(0xffffffffu, l0, m);
+              l1 += __shfl_xor_sync(0xffffffffu, l1, m);
+            }
+            if (g == 0) {
+              sm.lossp[warp][r0 + 8 * nt + 2 * q] = l0;
+              sm.lossp[warp][r0 + 8 * nt + 2 * q + 1] = l1;
+            }
           }
         }
-      }
 
-      // Outputs into the swizzled staging tile (row = token in the tile, col = W column).
-      if (has_q) {
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int row = r0 + 8 * nt + 2 * q + (e & 1);
-            const int col = col0 + g + 8 * (e >> 1);
-            *reinterpret_cast<__nv_bfloat16*>(obuf + swz128_bf16(row, col)) = __float2bfloat16_rn(o[nt][e]);
+        // Outputs into the swizzled staging tile (row = token in the tile, col = W column).
+        if (has_q) {
+  #pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+  #pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int row = r0 + 8 * nt + 2 * q + (e & 1);
+              const int col = col0 + g + 8 * (e >> 1);
+              *reinterpret_cast<__nv_bfloat16*>(obuf + swz128_bf16(row, col)) = __float2bfloat16_rn(o[nt][e]);
+            }
+        }
+
+        // Wᵀ += Sᵀ·K with S = −(η/b)·R, S fed as bf16 hi + lo.
+        uint32_t shi[KT][4], slo[KT][4];
+  #pragma unroll
+        for (int kt = 0; kt < KT; ++kt) {
+          split2(-beta * p[2 * kt][0], -beta * p[2 * kt][1], shi[kt][0], slo[kt][0]);
+          split2(-beta * p[2 * kt][2], -beta * p[2 * kt][3], shi[kt][1], slo[kt][1]);
+          split2(-beta * p[2 * kt + 1][0], -beta * p[2 * kt + 1][1], shi[kt][2], slo[kt][2]);
+          split2(-beta * p[2 * kt + 1][2], -beta * p[2 * kt + 1][3], shi[kt][3], slo[kt][3]);
+        }
+  #pragma unroll
+        for (int kt = 0; kt < KT; ++kt) {
+  #pragma unroll
+          for (int nt = 0; nt < 8; nt += 2) {
+            // B fragments of K[token][key]: tokens r0+16kt .. +15, keys 8nt .. 8nt+15 (transposed).
+            const int mi = lane >> 3, ri = lane & 7;
+            uint32_t kb[4];
+            ldsm_x4_t(kbase + swz128_bf16(r0 + 16 * kt + 8 * (mi & 1) + ri, 8 * nt + 8 * (mi >> 1)), kb);
+            mma16816(acc[nt], shi[kt], kb[0], kb[1]);
+            mma16816(acc[nt], slo[kt], kb[0], kb[1]);
+            mma16816(acc[nt + 1], shi[kt], kb[2], kb[3]);
+            mma16816(acc[nt + 1], slo[kt], kb[2], kb[3]);
           }
-      }
-
-      // Wᵀ += Sᵀ·K with S = −(η/b)·R, S fed as bf16 hi + lo.
-      uint32_t shi[KT][4], slo[KT][4];
-#pragma unroll
-      for (int kt = 0; kt < KT; ++kt) {
-        split2(-beta * p[2 * kt][0], -beta * p[2 * kt][1], shi[kt][0], slo[kt][0]);
-        split2(-beta * p[2 * kt][2], -beta * p[2 * kt][3], shi[kt][1], slo[kt][1]);
-        split2(-beta * p[2 * kt + 1][0], -beta * p[2 * kt + 1][1], shi[kt][2], slo[kt][2]);
-        split2(-beta * p[2 * kt + 1][2], -beta * p[2 * kt + 1][3], shi[kt][3], slo[kt][3]);
-      }
-#pragma unroll
-      for (int kt = 0; kt < KT; ++kt) {
-#pragma unroll
-        for (int nt = 0; nt < 8; nt += 2) {
-          // B fragments of K[token][key]: tokens r0+16kt .. +15, keys 8nt .. 8nt+15 (transposed).
-          const int mi = lane >> 3, ri = lane & 7;
-          uint32_t kb[4];
-          ldsm_x4_t(kbase + swz128_bf16(r0 + 16 * kt + 8 * (mi & 1) + ri, 8 * nt + 8 * (mi >> 1)), kb);
-          mma16816(acc[nt], shi[kt], kb[0], kb[1]);
-          mma16816(acc[nt], slo[kt], kb[0], kb[1]);
-          mma16816(acc[nt + 1], shi[kt], kb[2], kb[3]);
-          mma16816(acc[nt + 1], slo[kt], kb[2], kb[3]);
         }
       }
     }
-
     // End of the tile: outputs and losses of 64 tokens are complete in shared memory.
     if (has_q) fence_proxy_async_smem();
     named_sync();
