@@ -1,13 +1,550 @@
-// In-Place TTT scan on the tcgen05 tensor cores (bf16 in, fp32 accumulate).
+// In-Place TTT scan on the 5th-generation tensor cores (tcgen05, bf16 in, fp32 accumulate in
+// TMEM), for Wdown states too large to stay on chip (d_model 2560 x d_ff 9728 = 99.6 MB fp32).
+//
+// "In-Place Test-Time Training", §3: chunk c is first applied with the weight from before
+// the chunk, O_c = Z_c·W_cᵀ, then the weight is updated from the same chunk (§2),
+// W_{c+1} = W_c + η·V̂_cᵀ·Z_c; with fused target generation (§4) V̂ = Conv1D(X0)·Wtarget.
+//
+// Design (B200):
+//  * one persistent launch per chunk; its CTAs (one per SM) work through a static tile
+//    schedule computed on the host by longest-processing-time-first, mixing three GEMM
+//    tile types of 128x256 outputs:
+//      APPLY  O_c tile   = Z_c[128 tok, f] · W_cᵀ            A, B K-major        → bf16 O
+//      UPDATE ΔW tile    = V̂_c[:, 128 rows]ᵀ · Z_c[:, 256]   A, B MN-major (K = tokens)
+//                          epilogue W += η·ΔW (fp32 read-modify-write) and writes the bf16
+//                          copy of W_{c+1} used by the next chunk's APPLY tiles
+//      TARGET V̂_{c+1} tile = conv(X0)_{c+1}[128 tok, d] · Wtarget[:, 256]  A K-major, B MN-major
+//    APPLY reads the bf16 copy of W_c while UPDATE writes the other copy, so both run in the
+//    same launch without waiting for each other; the compute-bound APPLY tiles and the
+//    HBM-bound UPDATE epilogues overlap on different SMs.
+//  * per CTA: warp 0 issues TMA loads (128-byte swizzle) into a 4-stage shared-memory ring,
+//    warp 1 allocates 512 TMEM columns and one lane issues tcgen05.mma (M=128, N=256, K=16)
+//    into one of two TMEM accumulators, warps 2..9 drain the other accumulator
+//    (tcgen05.ld 32x32b) in the epilogue, two warps per TMEM lane quarter.
+//  * every wait is bounded (%globaltimer); a wait that runs out records TTT_ERR_TIMEOUT in the
+//    state's status word, the CTA drains its in-flight copies and MMAs (bounded), frees TMEM
+//    and returns.
+#include <algorithm>
+#include <vector>
+
 #include "common.cuh"
 #include "internal.h"
 
 namespace ttt {
 
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 64;
+constexpr int kSt = 4;
+constexpr int kABytes = BM * BK * 2;  // 16 KB
+constexpr int kBBytes = BN * BK * 2;  // 32 KB
+constexpr int kEpiWarps = 8;
+constexpr int kThreadsTC = (2 + kEpiWarps) * 32;
+constexpr int kTmemCols = 512;
+
+enum : int { APPLY = 0, UPDATE = 1, TARGET = 2 };
+
+__host__ __device__ constexpr int32_t tile_code(int type, int m, int n) { return (type << 28) | (m << 14) | n; }
+__device__ __forceinline__ int tile_type(int32_t t) { return (t >> 28) & 3; }
+__device__ __forceinline__ int tile_m(int32_t t) { return (t >> 14) & 0x3FFF; }
+__device__ __forceinline__ int tile_n(int32_t t) { return t & 0x3FFF; }
+
+struct __align__(1024) TCSmem {
+  uint8_t A[kSt][kABytes];
+  uint8_t B[kSt][kBBytes];
+  uint64_t full[kSt], empty[kSt];
+  uint64_t tfull[2], tempty[2];
+  uint32_t tmem_base;
+  int abort;
+};
+
+struct TCArgs {
+  const int32_t* sched;  // [grid + 1] CTA offsets followed by the tile codes
+  int chunk;             // chunk c of this launch (token offset c·C)
+  int target_chunk;      // chunk whose targets the TARGET tiles produce
+  int vrow0;             // first V̂ row of chunk c in the tensor map of V̂
+  int d, f, C;
+  float eta;
+  float* W;                    // fp32 master [d, f]
+  __nv_bfloat16* Wsh_next;     // bf16 copy of W_{c+1} [d, f]
+  __nv_bfloat16* O;            // outputs [T, d]
+  __nv_bfloat16* Vhat_out;     // targets of target_chunk [C, d]
+  int* status;
+};
+
+// ---- tcgen05 wrappers -----------------------------------------------------------------
+
+__device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;  // descriptor version for tcgen05
+  d |= (uint64_t)2 << 61;  // 128-byte swizzle
+  return d;
+}
+
+// kind::f16 instruction descriptor: D fp32, A and B bf16, M = 128, N = 256.
+__host__ __device__ constexpr uint32_t idesc_bf16(int a_mn, int b_mn) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
+         ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ int kblocks(int type, const TCArgs& a) {
+  if (type == APPLY) return (a.f + BK - 1) / BK;
+  if (type == UPDATE) return a.C / BK;
+  return (a.d + BK - 1) / BK;
+}
+
+// Stores 32 consecutive bf16 values of one row (cols col0 .. col0+31, clipped to ncols).
+__device__ __forceinline__ void store_row_bf16(__nv_bfloat16* row, int col0, int ncols, const float* v) {
+  if (col0 + 32 <= ncols) {
+    uint4* dst = reinterpret_cast<uint4*>(row + col0);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint4 w;
+      w.x = pack_bf16(v[8 * q + 0], v[8 * q + 1]);
+      w.y = pack_bf16(v[8 * q + 2], v[8 * q + 3]);
+      w.z = pack_bf16(v[8 * q + 4], v[8 * q + 5]);
+      w.w = pack_bf16(v[8 * q + 6], v[8 * q + 7]);
+      dst[q] = w;
+    }
+  } else {
+    for (int j = 0; j < 32 && col0 + j < ncols; ++j) row[col0 + j] = __float2bfloat16_rn(v[j]);
+  }
+}
+
+__global__ void __launch_bounds__(kThreadsTC, 1)
+    k_inplace_tc(const __grid_constant__ CUtensorMap tmZk, const __grid_constant__ CUtensorMap tmZm,
+                 const __grid_constant__ CUtensorMap tmVm, const __grid_constant__ CUtensorMap tmWk,
+                 const __grid_constant__ CUtensorMap tmConv, const __grid_constant__ CUtensorMap tmWt,
+                 const TCArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  TCSmem& sm = *reinterpret_cast<TCSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int32_t* tiles = args.sched + gridDim.x + 1;
+  const int t_begin = args.sched[blockIdx.x];
+  const int t_end = args.sched[blockIdx.x + 1];
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kSt; ++i) {
+      mbar_init(&sm.full[i], 1);
+      mbar_init(&sm.empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sm.tfull[i], 1);
+      mbar_init(&sm.tempty[i], kEpiWarps);
+    }
+    sm.abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&sm.tmem_base)),
+                 "r"(kTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  volatile int* abort = &sm.abort;
+
+  if (warp == 0) {
+    // ------------------------------- TMA producer -------------------------------
+    if (lane == 0) {
+      tma_prefetch_desc(&tmZk);
+      tma_prefetch_desc(&tmZm);
+      tma_prefetch_desc(&tmVm);
+      tma_prefetch_desc(&tmWk);
+      uint32_t it = 0;
+      for (int ti = t_begin; ti < t_end && !*abort; ++ti) {
+        const int32_t tc = tiles[ti];
+        const int type = tile_type(tc), m = tile_m(tc), n = tile_n(tc);
+        const int nk = kblocks(type, args);
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % kSt;
+          if (it >= kSt && !mbar_wait(&sm.empty[s], ((it / kSt) - 1) & 1, args.status, abort)) break;
+          mbar_arrive_expect_tx(&sm.full[s], kABytes + kBBytes);
+          if (type == APPLY) {
+            tma_load_2d(sm.A[s], &tmZk, &sm.full[s], kb * BK, args.chunk * args.C + m * BM);
+            tma_load_2d(sm.B[s], &tmWk, &sm.full[s], kb * BK, n * BN);
+          } else if (type == UPDATE) {
+            for (int j = 0; j < BM / 64; ++j)
+              tma_load_2d(sm.A[s] + j * 8192, &tmVm, &sm.full[s], m * BM + j * 64, args.vrow0 + kb * BK);
+            for (int j = 0; j < BN / 64; ++j)
+              tma_load_2d(sm.B[s] + j * 8192, &tmZm, &sm.full[s], n * BN + j * 64, args.chunk * args.C + kb * BK);
+          } else {
+            tma_load_2d(sm.A[s], &tmConv, &sm.full[s], kb * BK, args.target_chunk * args.C + m * BM);
+            for (int j = 0; j < BN / 64; ++j)
+              tma_load_2d(sm.B[s] + j * 8192, &tmWt, &sm.full[s], n * BN + j * 64, kb * BK);
+          }
+        }
+      }
+      // Drain: the newest phase issued on every stage must have landed before exit.
+      for (uint32_t k = (it > (uint32_t)kSt ? it - kSt : 0); k < it; ++k)
+        mbar_wait(&sm.full[k % kSt], (k / kSt) & 1, args.status, nullptr);
+    }
+  } else if (warp == 1) {
+    // ------------------------------- MMA issuer -------------------------------
+    if (lane == 0) {
+      uint32_t it = 0, tcount = 0;
+      bool ok = true;
+      for (int ti = t_begin; ti < t_end && ok; ++ti, ++tcount) {
+        const int32_t tc = tiles[ti];
+        const int type = tile_type(tc);
+        const int nk = kblocks(type, args);
+        const int acc = tcount & 1;
+        if (tcount >= 2 && !mbar_wait(&sm.tempty[acc], ((tcount >> 1) - 1) & 1, args.status, abort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + (uint32_t)(acc * BN);
+        const uint32_t idesc = type == APPLY ? idesc_bf16(0, 0) : (type == UPDATE ? idesc_bf16(1, 1) : idesc_bf16(0, 1));
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % kSt;
+          if (!mbar_wait(&sm.full[s], (it / kSt) & 1, args.status, abort)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sm.A[s]), b0 = smem_u32(sm.B[s]);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            uint64_t ad, bd;
+            if (type == UPDATE) {
+              ad = umma_desc(a0 + kk * 2048, 8192, 1024);
+              bd = umma_desc(b0 + kk * 2048, 8192, 1024);
+            } else {
+              ad = umma_desc(a0 + kk * 32, 16, 1024);
+              bd = type == APPLY ? umma_desc(b0 + kk * 32, 16, 1024) : umma_desc(b0 + kk * 2048, 8192, 1024);
+            }
+            umma(d_tmem, ad, bd, idesc, (kb | kk) != 0);
+          }
+          umma_commit(&sm.empty[s]);  // frees the stage once these MMAs have read it
+        }
+        if (!ok) break;
+        umma_commit(&sm.tfull[acc]);  // accumulator ready for the epilogue
+      }
+      // Drain: the last commit covers every MMA issued before it; wait for it before TMEM
+      // is freed. After a clean run that is the last accumulator's commit, after an abort
+      // the last stage-release commit.
+      if (ok && t_end > t_begin) {
+        const uint32_t last = (uint32_t)(t_end - t_begin - 1);
+        mbar_wait(&sm.tfull[last & 1], (last >> 1) & 1, args.status, nullptr);
+      } else if (!ok && it > 0) {
+        mbar_wait(&sm.empty[(it - 1) % kSt], ((it - 1) / kSt) & 1, args.status, nullptr);
+      }
+    }
+  } else {
+    // ------------------------------- epilogue (8 warps) -------------------------------
+    const int lq = warp & 3;              // TMEM lane quarter this warp may access
+    const int half = (warp - 2) >> 2;     // which 128 columns of the 256-wide tile
+    uint32_t tcount = 0;
+    for (int ti = t_begin; ti < t_end; ++ti, ++tcount) {
+      const int32_t tc = tiles[ti];
+      const int type = tile_type(tc), m = tile_m(tc), n = tile_n(tc);
+      const int acc = tcount & 1;
+      if (!mbar_wait(&sm.tfull[acc], (tcount >> 1) & 1, args.status, abort)) break;
+      tc_fence_after();
+      const int row = m * BM + lq * 32 + lane;  // token (APPLY/TARGET) or Wdown row (UPDATE)
+      const uint32_t tbase = tmem + ((uint32_t)(lq * 32) << 16) + (uint32_t)(acc * BN + half * 128);
+#pragma unroll 1
+      for (int jc = 0; jc < 4; ++jc) {
+        const int col0 = n * BN + half * 128 + jc * 32;
+        uint32_t r[32];
+        tmem_ld32(tbase + jc * 32, r);
+        if (type == UPDATE) {
+          // W[row, col0..col0+31] += η·ΔW, and the bf16 copy for the next chunk.
+          const bool in = row < args.d;
+          float w[32];
+          float* Wrow = args.W + (size_t)row * args.f;
+          const bool full = col0 + 32 <= args.f;
+          if (in && full) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const float4 v = *reinterpret_cast<const float4*>(Wrow + col0 + 4 * q);
+              w[4 * q] = v.x;
+              w[4 * q + 1] = v.y;
+              w[4 * q + 2] = v.z;
+              w[4 * q + 3] = v.w;
+            }
+          } else if (in) {
+            for (int j = 0; j < 32; ++j) w[j] = col0 + j < args.f ? Wrow[col0 + j] : 0.f;
+          }
+          tmem_wait_ld();
+          if (in) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) w[j] = fmaf(args.eta, __uint_as_float(r[j]), w[j]);
+            if (full) {
+#pragma unroll
+              for (int q = 0; q < 8; ++q)
+                *reinterpret_cast<float4*>(Wrow + col0 + 4 * q) = make_float4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+            } else {
+              for (int j = 0; j < 32 && col0 + j < args.f; ++j) Wrow[col0 + j] = w[j];
+            }
+            store_row_bf16(args.Wsh_next + (size_t)row * args.f, col0, args.f, w);
+          }
+        } else {
+          tmem_wait_ld();
+          float v[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+          if (type == APPLY) {
+            store_row_bf16(args.O + ((size_t)args.chunk * args.C + row) * args.d, col0, args.d, v);
+          } else {
+            store_row_bf16(args.Vhat_out + (size_t)row * args.d, col0, args.d, v);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.tempty[acc]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
+}
+
+// Depthwise future-tap convolution of X0 for the fused target:
+// conv[t, i] = Σ_k w[i, k]·X0[t + k, i] over taps whose source t + k lies before the end of t's
+// chunk (pad mode 0) or before T (pad mode 1); fp32 arithmetic, stored as bf16.
+__global__ void k_target_conv(const __nv_bfloat16* __restrict__ X0, const float* __restrict__ w, __nv_bfloat16* __restrict__ out,
+                              int T, int d, int C, int taps, int pad_mode) {
+  const int pairs = d / 2;
+  const size_t n = (size_t)T * pairs;
+  for (size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x; idx < n; idx += (size_t)gridDim.x * blockDim.x) {
+    const int t = (int)(idx / pairs);
+    const int i = (int)(idx % pairs) * 2;
+    const int end = pad_mode == 0 ? min(T, (t / C + 1) * C) : T;
+    float a0 = 0.f, a1 = 0.f;
+    for (int k = 0; k < taps && t + k < end; ++k) {
+      const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162*>(X0 + (size_t)(t + k) * d + i);
+      const float2 xf = __bfloat1622float2(x);
+      a0 = fmaf(w[i * taps + k], xf.x, a0);
+      a1 = fmaf(w[(i + 1) * taps + k], xf.y, a1);
+    }
+    *reinterpret_cast<uint32_t*>(out + (size_t)t * d + i) = pack_bf16(a0, a1);
+  }
+}
+
+// ---- host: schedules ------------------------------------------------------------------
+
+struct Plan {
+  std::vector<int32_t> host;  // [grid + 1] offsets, then tile codes
+  int grid = 0;
+};
+
+Plan make_plan(int num_sms, int d, int f, int C, bool apply_update, bool target) {
+  struct T {
+    int32_t code;
+    int cost;
+  };
+  std::vector<T> tl;
+  const int mt_tok = C / BM, nt_d = (d + BN - 1) / BN;
+  if (apply_update) {
+    const int cost_apply = (f + BK - 1) / BK + 2;
+    for (int m = 0; m < mt_tok; ++m)
+      for (int n = 0; n < nt_d; ++n) tl.push_back({tile_code(APPLY, m, n), cost_apply});
+  }
+  if (target) {
+    const int cost_t = (d + BK - 1) / BK + 2;
+    for (int m = 0; m < mt_tok; ++m)
+      for (int n = 0; n < nt_d; ++n) tl.push_back({tile_code(TARGET, m, n), cost_t});
+  }
+  if (apply_update) {
+    // The read-modify-write epilogue (fp32 W in and out, bf16 copy out: 320 KB per tile)
+    // costs more than the 16-deep mainloop; weigh it in.
+    const int cost_u = std::max(C / BK, 20);
+    for (int m = 0; m < (d + BM - 1) / BM; ++m)
+      for (int n = 0; n < (f + BN - 1) / BN; ++n) tl.push_back({tile_code(UPDATE, m, n), cost_u});
+  }
+  const int grid = std::max(1, std::min<int>(num_sms, (int)tl.size()));
+  std::stable_sort(tl.begin(), tl.end(), [](const T& a, const T& b) { return a.cost > b.cost; });
+  std::vector<std::vector<int32_t>> per(grid);
+  std::vector<long> load(grid, 0);
+  for (const T& t : tl) {
+    int best = 0;
+    for (int i = 1; i < grid; ++i)
+      if (load[i] < load[best]) best = i;
+    per[best].push_back(t.code);
+    load[best] += t.cost;
+  }
+  Plan p;
+  p.grid = grid;
+  p.host.resize(grid + 1);
+  int off = 0;
+  for (int i = 0; i < grid; ++i) {
+    p.host[i] = off;
+    off += (int)per[i].size();
+  }
+  p.host[grid] = off;
+  for (int i = 0; i < grid; ++i) p.host.insert(p.host.end(), per[i].begin(), per[i].end());
+  return p;
+}
+
+ttt_status upload_plan(const Plan& p, int32_t** dev) {
+  TTT_CUDA(cudaMalloc(reinterpret_cast<void**>(dev), p.host.size() * sizeof(int32_t)));
+  TTT_CUDA(cudaMemcpy(*dev, p.host.data(), p.host.size() * sizeof(int32_t), cudaMemcpyHostToDevice));
+  return TTT_OK;
+}
+
+ttt_status map2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint32_t box_in, uint32_t box_out) {
+  const uint64_t dims[2] = {inner, outer};
+  const uint64_t strides[1] = {inner * 2};
+  const uint32_t box[2] = {box_in, box_out};
+  return encode_tmap(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+}  // namespace
+
+// Per-state tensor-core resources (schedules, conv buffer), created on first use.
+struct TCResources {
+  int32_t* plan_dev[3] = {nullptr, nullptr, nullptr};  // 0: steady, 1: target only, 2: apply+update only
+  int grid[3] = {0, 0, 0};
+  __nv_bfloat16* conv = nullptr;
+  size_t conv_rows = 0;
+};
+
+static ttt_status ensure_tc(ttt_state* st) {
+  if (st->ip.tc != nullptr) return TTT_OK;
+  const ttt_config& c = st->cfg;
+  TCResources* r = new (std::nothrow) TCResources();
+  if (r == nullptr) return fail(TTT_ERR_OOM, "host allocation failed");
+  const bool target = c.target_mode == 1;
+  Plan p0 = make_plan(st->num_sms, c.d_val, c.d_key, c.chunk, true, target);
+  ttt_status s = upload_plan(p0, &r->plan_dev[0]);
+  r->grid[0] = p0.grid;
+  if (s == TTT_OK && target) {
+    Plan p1 = make_plan(st->num_sms, c.d_val, c.d_key, c.chunk, false, true);
+    Plan p2 = make_plan(st->num_sms, c.d_val, c.d_key, c.chunk, true, false);
+    s = upload_plan(p1, &r->plan_dev[1]);
+    if (s == TTT_OK) s = upload_plan(p2, &r->plan_dev[2]);
+    r->grid[1] = p1.grid;
+    r->grid[2] = p2.grid;
+  }
+  if (s != TTT_OK) {
+    for (int i = 0; i < 3; ++i)
+      if (r->plan_dev[i]) cudaFree(r->plan_dev[i]);
+    delete r;
+    return s;
+  }
+  st->ip.tc = r;
+  return TTT_OK;
+}
+
+void free_tc(ttt_state* st) {
+  TCResources* r = st->ip.tc;
+  if (r == nullptr) return;
+  for (int i = 0; i < 3; ++i)
+    if (r->plan_dev[i]) cudaFree(r->plan_dev[i]);
+  if (r->conv) cudaFree(r->conv);
+  delete r;
+  st->ip.tc = nullptr;
+}
+
 ttt_status inplace_bf16_scan(ttt_state* st, const __nv_bfloat16* Z, const __nv_bfloat16* targets, int64_t T,
                              __nv_bfloat16* O, cudaStream_t s) {
-  (void)st; (void)Z; (void)targets; (void)T; (void)O; (void)s;
-  return fail(TTT_ERR_UNSUPPORTED, "In-Place BF16 scan not built yet");
+  const ttt_config& c = st->cfg;
+  const int d = c.d_val, f = c.d_key, C = c.chunk;
+  const bool target = c.target_mode == 1;
+  TTT_TRY(ensure_tc(st));
+  TCResources* r = st->ip.tc;
+  const int nchunks = (int)(T / C);
+
+  CUtensorMap tmZk, tmZm, tmVm_in, tmVm_buf[2], tmWk[2], tmConv, tmWt;
+  TTT_TRY(map2d(&tmZk, Z, f, T, BK, BM));
+  TTT_TRY(map2d(&tmZm, Z, f, T, 64, BK));
+  TTT_TRY(map2d(&tmWk[0], st->ip.Wsh[0], f, d, BK, BN));
+  TTT_TRY(map2d(&tmWk[1], st->ip.Wsh[1], f, d, BK, BN));
+  if (target) {
+    if (r->conv_rows < (size_t)T) {
+      if (r->conv) cudaFree(r->conv);
+      r->conv = nullptr;
+      r->conv_rows = 0;
+      TTT_CUDA(cudaMalloc(reinterpret_cast<void**>(&r->conv), (size_t)T * d * 2));
+      r->conv_rows = (size_t)T;
+    }
+    TTT_TRY(map2d(&tmConv, r->conv, d, T, BK, BM));
+    TTT_TRY(map2d(&tmWt, st->ip.Wtarget, d, d, 64, BK));
+    TTT_TRY(map2d(&tmVm_buf[0], st->ip.Vhat[0], d, C, 64, BK));
+    TTT_TRY(map2d(&tmVm_buf[1], st->ip.Vhat[1], d, C, 64, BK));
+    const size_t pairs = (size_t)T * (d / 2);
+    const int blocks = (int)std::min<size_t>((pairs + 255) / 256, (size_t)st->num_sms * 16);
+    k_target_conv<<<blocks, 256, 0, s>>>(targets, st->ip.convw, r->conv, (int)T, d, C, c.conv_taps, c.conv_pad_mode);
+    st->launches++;
+    TTT_CUDA(cudaGetLastError());
+  } else {
+    TTT_TRY(map2d(&tmVm_in, targets, d, T, 64, BK));
+    tmConv = tmZk;
+    tmWt = tmZk;
+  }
+
+  const size_t smem = sizeof(TCSmem) + 1024;
+  TTT_CUDA(cudaFuncSetAttribute(k_inplace_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+
+  auto launch = [&](int plan, int chunk, int tchunk) -> ttt_status {
+    TCArgs a;
+    a.sched = r->plan_dev[plan];
+    a.chunk = chunk;
+    a.target_chunk = tchunk;
+    a.vrow0 = target ? 0 : chunk * C;
+    a.d = d;
+    a.f = f;
+    a.C = C;
+    a.eta = c.eta;
+    a.W = st->ip.W;
+    a.Wsh_next = st->ip.Wsh[st->ip.cur ^ 1];
+    a.O = O;
+    a.Vhat_out = target ? st->ip.Vhat[tchunk & 1] : nullptr;
+    a.status = st->status.dev;
+    const CUtensorMap& vm = target ? tmVm_buf[chunk & 1] : tmVm_in;
+    k_inplace_tc<<<r->grid[plan], kThreadsTC, smem, s>>>(tmZk, tmZm, vm, tmWk[st->ip.cur], tmConv, tmWt, a);
+    st->launches++;
+    TTT_CUDA(cudaGetLastError());
+    return TTT_OK;
+  };
+
+  if (target) TTT_TRY(launch(1, 0, 0));  // targets of chunk 0
+  for (int ch = 0; ch < nchunks; ++ch) {
+    const bool last = ch + 1 == nchunks;
+    const int plan = target ? (last ? 2 : 0) : 0;
+    TTT_TRY(launch(plan, ch, ch + 1));
+    st->ip.cur ^= 1;  // the bf16 copy written by this launch holds W_{c+1}
+  }
+  return TTT_OK;
 }
 
 }  // namespace ttt

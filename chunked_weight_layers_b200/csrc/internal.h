@@ -12,6 +12,8 @@
 
 namespace ttt {
 
+struct TCResources;
+
 // Records `msg` as the calling thread's last error and returns `s`.
 ttt_status fail(ttt_status s, const char* fmt, ...);
 // Maps a CUDA runtime error to TTT_ERR_CUDA with a message naming `what`.
@@ -43,8 +45,8 @@ struct InplaceBuffers {
   int cur = 0;                   // index of the bf16 copy that holds the current W
   __nv_bfloat16* Wtarget = nullptr;  // [d, d]
   float* convw = nullptr;        // [d, taps]
-  __nv_bfloat16* conv = nullptr; // conv(X0) of one chunk [C, d]
-  __nv_bfloat16* Vhat[2] = {nullptr, nullptr};  // targets of a chunk [C, d]
+  __nv_bfloat16* Vhat[2] = {nullptr, nullptr};  // targets of a chunk [C, d] (fused target)
+  TCResources* tc = nullptr;     // tensor-core schedules and conv(X0) buffer, built on first use
 };
 
 struct LinearBuffers {
@@ -92,6 +94,9 @@ ttt_status inplace_f32_chunk(ttt_state* st, const float* Z, const float* Vhat, f
 // In-Place, bf16 tensor cores: the whole scan over T tokens.
 ttt_status inplace_bf16_scan(ttt_state* st, const __nv_bfloat16* Z, const __nv_bfloat16* targets,
                              int64_t T, __nv_bfloat16* O, cudaStream_t s);
+
+// Frees the tensor-core resources of a state (no-op if none were built).
+void free_tc(ttt_state* st);
 
 // TTT-Linear mini-batch scan over T tokens of every (sequence, head).
 ttt_status linear_scan(ttt_state* st, const __nv_bfloat16* K, const __nv_bfloat16* V,

@@ -108,7 +108,7 @@ static void free_state(ttt_state* st) {
   dev_free(st->ip.Wsh[1]);
   dev_free(st->ip.Wtarget);
   dev_free(st->ip.convw);
-  dev_free(st->ip.conv);
+  free_tc(st);
   dev_free(st->ip.Vhat[0]);
   dev_free(st->ip.Vhat[1]);
   dev_free(st->lin.W);
@@ -193,7 +193,6 @@ static ttt_status create_impl(const ttt_config* cfg, const void* W0, const void*
       const size_t dd = (size_t)c.d_val * c.d_val;
       guard(dev_alloc((void**)&st->ip.Wtarget, dd * 2, "Wtarget")) &&
           guard(dev_alloc((void**)&st->ip.convw, (size_t)c.d_val * c.conv_taps * 4, "convw")) &&
-          guard(dev_alloc((void**)&st->ip.conv, (size_t)c.chunk * c.d_val * 2, "conv buffer")) &&
           guard(dev_alloc((void**)&st->ip.Vhat[0], (size_t)c.chunk * c.d_val * 2, "target buffer")) &&
           guard(dev_alloc((void**)&st->ip.Vhat[1], (size_t)c.chunk * c.d_val * 2, "target buffer"));
     }
