@@ -71,6 +71,8 @@ _SIGNATURES = {
     "ttt_state_launch_count": (ctypes.c_int64, [_vp]),
     "ttt_state_destroy": (_st, [_vp]),
     "ttt_last_error_string": (ctypes.c_char_p, []),
+    "ttt_target_values_noalloc": (_st, [_vp, _vp, _vp, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
+                                        ctypes.c_int32, ctypes.c_int32, _vp, _vp]),
 }
 
 _lib = None

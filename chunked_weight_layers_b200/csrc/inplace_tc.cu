@@ -547,4 +547,63 @@ ttt_status inplace_bf16_scan(ttt_state* st, const __nv_bfloat16* Z, const __nv_b
   return TTT_OK;
 }
 
+
+// ---- target generation into caller-provided scratch -----------------------------------
+
+namespace {
+
+// Round-robin schedule of the TARGET tiles of one block of rows: tile i goes to CTA i % grid.
+// Same layout as the host-built schedules: [grid + 1] offsets, then the tile codes.
+__global__ void k_target_plan(int32_t* plan, int grid, int mt, int nt) {
+  const int n = mt * nt, q = n / grid, r = n % grid;
+  for (int c = threadIdx.x; c <= grid; c += blockDim.x) plan[c] = c * q + min(c, r);
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const int c = i % grid, j = i / grid;
+    plan[grid + 1 + c * q + min(c, r) + j] = tile_code(TARGET, i / nt, i % nt);
+  }
+}
+
+}  // namespace
+
+int target_values_plan_ints(int T, int d, int num_sms) {
+  const int ntiles = (T / BM) * ((d + BN - 1) / BN);
+  const int grid = std::max(1, std::min(num_sms, ntiles));
+  return grid + 1 + ntiles;
+}
+
+ttt_status target_values_into(const __nv_bfloat16* X0, const float* convw, const __nv_bfloat16* Wtarget, int T, int d,
+                              int C, int taps, int pad_mode, __nv_bfloat16* conv_scratch, int32_t* plan_scratch,
+                              __nv_bfloat16* out, int num_sms, cudaStream_t s) {
+  const int mt = T / BM, nt = (d + BN - 1) / BN;
+  const int grid = std::max(1, std::min(num_sms, mt * nt));
+  const size_t pairs = (size_t)T * (d / 2);
+  const int blocks = (int)std::min<size_t>((pairs + 255) / 256, (size_t)num_sms * 16);
+  k_target_conv<<<blocks, 256, 0, s>>>(X0, convw, conv_scratch, T, d, C, taps, pad_mode);
+  TTT_CUDA(cudaGetLastError());
+  k_target_plan<<<1, 256, 0, s>>>(plan_scratch, grid, mt, nt);
+  TTT_CUDA(cudaGetLastError());
+  CUtensorMap tmConv, tmWt;
+  TTT_TRY(map2d(&tmConv, conv_scratch, d, T, BK, BM));
+  TTT_TRY(map2d(&tmWt, Wtarget, d, d, 64, BK));
+  TCArgs a;
+  a.sched = plan_scratch;
+  a.chunk = 0;
+  a.target_chunk = 0;
+  a.vrow0 = 0;
+  a.d = d;
+  a.f = d;
+  a.C = T;
+  a.eta = 0.f;
+  a.W = nullptr;
+  a.Wsh_next = nullptr;
+  a.O = nullptr;
+  a.Vhat_out = out;
+  a.status = nullptr;
+  const size_t smem = sizeof(TCSmem) + 1024;
+  TTT_CUDA(cudaFuncSetAttribute(k_inplace_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  k_inplace_tc<<<grid, kThreadsTC, smem, s>>>(tmConv, tmConv, tmConv, tmConv, tmConv, tmWt, a);
+  TTT_CUDA(cudaGetLastError());
+  return TTT_OK;
+}
+
 }  // namespace ttt

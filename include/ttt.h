@@ -157,6 +157,32 @@ ttt_status ttt_cache_read(const ttt_state* st, int32_t* entries, int32_t* counts
  * [batch, heads], 1 once a chunk has set τ. Either pointer may be NULL. */
 ttt_status ttt_gate_read(const ttt_state* st, float* tau, int32_t* tau_set, ttt_stream stream);
 
+/* Target generation V̂ = Conv1D(X0)·Wtarget for T tokens without allocating device memory.
+ * The pages have no counterpart of this entry point: it exists for callers that cannot call
+ * cudaMalloc where they need the work done — their device memory is owned by another
+ * allocator that has reserved the GPU, or they run a loop that must not allocate after
+ * start-up (cudaMalloc can block and synchronise the device). It computes the same values
+ * as the fused target of an In-Place state with target_mode 1 (same kernels), but keeps its
+ * scratch (the conv rows and the tile schedule) in one fixed array of device memory inside
+ * the library image (about 8.1 MB, held by every GPU that loads the library until exit)
+ * instead of state memory, and calls no cudaMalloc, cudaFree or allocating routine.
+ *   X0       device bf16 [T, d_model], the token embeddings.
+ *   convw    device fp32 [d_model, conv_taps], depthwise taps at token offsets 0..taps-1.
+ *   Wtarget  device bf16 [d_model, d_model], [in, out].
+ *   chunk    taps read zero past the end of each chunk of this many tokens (conv_pad_mode 0)
+ *            or past token T only (conv_pad_mode 1).
+ *   Vhat_out device bf16 [T, d_model], written.
+ * Limits: T a multiple of 128, d_model a multiple of 8, T·d_model ≤ 4,194,304; larger inputs
+ * are rejected with TTT_ERR_INVALID_ARG and a message naming the limit. The first call on
+ * each device looks up the device address of the fixed array (cudaGetSymbolAddress with
+ * that device current); make that first call before any stream capture. All calls share
+ * the array and it keeps the last call's contents: calls whose GPU work overlaps (other
+ * streams, other host threads) race on it. A bounded device-side wait that runs out is not
+ * reported by this entry point (there is no state to hold the status). */
+ttt_status ttt_target_values_noalloc(const void* X0, const float* convw, const void* Wtarget, int64_t T,
+                                     int32_t d_model, int32_t chunk, int32_t conv_taps, int32_t conv_pad_mode,
+                                     void* Vhat_out, ttt_stream stream);
+
 /* Synchronise the device and return the first device-side failure recorded since the
  * last poll (TTT_ERR_TIMEOUT or TTT_ERR_DEVICE), or TTT_OK; clears the record. */
 ttt_status ttt_state_poll(ttt_state* st);
