@@ -17,10 +17,14 @@
 //    APPLY reads the bf16 copy of W_c while UPDATE writes the other copy, so both run in the
 //    same launch without waiting for each other; the compute-bound APPLY tiles and the
 //    HBM-bound UPDATE epilogues overlap on different SMs.
-//  * per CTA: warp 0 issues TMA loads (128-byte swizzle) into a 4-stage shared-memory ring,
+//  * per CTA: warp 0 issues TMA loads (128-byte swizzle) into a 3-stage shared-memory ring,
 //    warp 1 allocates 512 TMEM columns and one lane issues tcgen05.mma (M=128, N=256, K=16)
 //    into one of two TMEM accumulators, warps 2..9 drain the other accumulator
-//    (tcgen05.ld 32x32b) in the epilogue, two warps per TMEM lane quarter.
+//    (tcgen05.ld 32x32b) in the epilogue, two warps per TMEM lane quarter, and warp 10
+//    streams the fp32 W of UPDATE tiles by TMA into a 4-slot ring of 128x32 sub-tiles while
+//    the mainloop runs. The epilogue adds η·ΔW in shared memory, writes the bf16 copy beside
+//    it, and two TMA stores per sub-tile write both back: the read-modify-write of the 99.6 MB
+//    state never goes through per-thread global loads.
 //  * every wait is bounded (%globaltimer); a wait that runs out records TTT_ERR_TIMEOUT in the
 //    state's status word, the CTA drains its in-flight copies and MMAs (bounded), frees TMEM
 //    and returns.
@@ -35,11 +39,16 @@ namespace ttt {
 namespace {
 
 constexpr int BM = 128, BN = 256, BK = 64;
-constexpr int kSt = 4;
-constexpr int kABytes = BM * BK * 2;  // 16 KB
-constexpr int kBBytes = BN * BK * 2;  // 32 KB
+constexpr int kSt = 3;                      // operand ring depth (k-blocks)
+constexpr int kABytes = BM * BK * 2;        // 16 KB
+constexpr int kBBytes = BN * BK * 2;        // 32 KB
+constexpr int kWCols = 32;                  // columns of one W sub-tile of an UPDATE tile
+constexpr int kWBytes = BM * kWCols * 4;    // 16 KB of fp32 W
+constexpr int kShBytes = BM * kWCols * 2;   // 8 KB of its bf16 copy
+constexpr int kWSlots = 4;                  // W sub-tile ring depth
 constexpr int kEpiWarps = 8;
-constexpr int kThreadsTC = (2 + kEpiWarps) * 32;
+constexpr int kWarpWload = 2 + kEpiWarps;   // the warp that streams W sub-tiles in
+constexpr int kThreadsTC = (3 + kEpiWarps) * 32;
 constexpr int kTmemCols = 512;
 
 enum : int { APPLY = 0, UPDATE = 1, TARGET = 2 };
@@ -52,10 +61,15 @@ __device__ __forceinline__ int tile_n(int32_t t) { return t & 0x3FFF; }
 struct __align__(1024) TCSmem {
   uint8_t A[kSt][kABytes];
   uint8_t B[kSt][kBBytes];
+  uint8_t Wr[kWSlots][kWBytes];  // fp32 W sub-tiles (128 rows x 32 columns, 128-byte swizzle)
+  uint8_t Sh[2][kShBytes];       // bf16 copy of an updated sub-tile, one per column half (64-byte swizzle)
   uint64_t full[kSt], empty[kSt];
   uint64_t tfull[2], tempty[2];
+  uint64_t wfull[kWSlots], wempty[kWSlots];
   uint32_t tmem_base;
   int abort;
+  int eflag[2][2];  // per column half: a wait of sub-tile e ran out (index e & 1)
+  int tflag[2][2];  // per column half: the accumulator wait of tile t ran out (index t & 1)
 };
 
 struct TCArgs {
@@ -65,8 +79,6 @@ struct TCArgs {
   int vrow0;             // first V̂ row of chunk c in the tensor map of V̂
   int d, f, C;
   float eta;
-  float* W;                    // fp32 master [d, f]
-  __nv_bfloat16* Wsh_next;     // bf16 copy of W_{c+1} [d, f]
   __nv_bfloat16* O;            // outputs [T, d]
   __nv_bfloat16* Vhat_out;     // targets of target_chunk [C, d]
   int* status;
@@ -143,10 +155,15 @@ __device__ __forceinline__ void store_row_bf16(__nv_bfloat16* row, int col0, int
   }
 }
 
+__device__ __forceinline__ void named_sync_half(int half) {
+  asm volatile("bar.sync %0, %1;" ::"r"(1 + half), "n"(4 * 32) : "memory");
+}
+
 __global__ void __launch_bounds__(kThreadsTC, 1)
     k_inplace_tc(const __grid_constant__ CUtensorMap tmZk, const __grid_constant__ CUtensorMap tmZm,
                  const __grid_constant__ CUtensorMap tmVm, const __grid_constant__ CUtensorMap tmWk,
                  const __grid_constant__ CUtensorMap tmConv, const __grid_constant__ CUtensorMap tmWt,
+                 const __grid_constant__ CUtensorMap tmWf, const __grid_constant__ CUtensorMap tmWs,
                  const TCArgs args) {
   extern __shared__ uint8_t smem_raw[];
   TCSmem& sm = *reinterpret_cast<TCSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -164,7 +181,13 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       mbar_init(&sm.tfull[i], 1);
       mbar_init(&sm.tempty[i], kEpiWarps);
     }
+    for (int i = 0; i < kWSlots; ++i) {
+      mbar_init(&sm.wfull[i], 1);
+      mbar_init(&sm.wempty[i], 1);
+    }
     sm.abort = 0;
+    sm.eflag[0][0] = sm.eflag[0][1] = sm.eflag[1][0] = sm.eflag[1][1] = 0;
+    sm.tflag[0][0] = sm.tflag[0][1] = sm.tflag[1][0] = sm.tflag[1][1] = 0;
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -212,6 +235,30 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       // Drain: the newest phase issued on every stage must have landed before exit.
       for (uint32_t k = (it > (uint32_t)kSt ? it - kSt : 0); k < it; ++k)
         mbar_wait(&sm.full[k % kSt], (k / kSt) & 1, args.status, nullptr);
+    }
+  } else if (warp == kWarpWload) {
+    // ---------------- W sub-tile loader (fp32 W of UPDATE tiles, 128 x 32) ----------------
+    if (lane == 0) {
+      tma_prefetch_desc(&tmWf);
+      uint32_t e = 0;
+      for (int ti = t_begin; ti < t_end && !*abort; ++ti) {
+        const int32_t tc = tiles[ti];
+        if (tile_type(tc) != UPDATE) continue;
+        const int m = tile_m(tc), n = tile_n(tc);
+        bool ok = true;
+        for (int k = 0; k < BN / kWCols; ++k, ++e) {
+          const int s = e % kWSlots;
+          if (e >= (uint32_t)kWSlots && !mbar_wait(&sm.wempty[s], ((e / kWSlots) - 1) & 1, args.status, abort)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&sm.wfull[s], kWBytes);
+          tma_load_2d(sm.Wr[s], &tmWf, &sm.wfull[s], n * BN + (k & 1) * 128 + (k >> 1) * kWCols, m * BM);
+        }
+        if (!ok) break;
+      }
+      for (uint32_t k = (e > (uint32_t)kWSlots ? e - kWSlots : 0); k < e; ++k)
+        mbar_wait(&sm.wfull[k % kWSlots], (k / kWSlots) & 1, args.status, nullptr);
     }
   } else if (warp == 1) {
     // ------------------------------- MMA issuer -------------------------------
@@ -269,67 +316,105 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     // ------------------------------- epilogue (8 warps) -------------------------------
     const int lq = warp & 3;              // TMEM lane quarter this warp may access
     const int half = (warp - 2) >> 2;     // which 128 columns of the 256-wide tile
-    uint32_t tcount = 0;
-    for (int ti = t_begin; ti < t_end; ++ti, ++tcount) {
+    const bool leader = lq == 0 && lane == 0;  // issues this half's TMA stores
+    uint32_t tcount = 0, ecount = 0;      // tiles seen; W sub-tiles consumed by this half
+    const int row_in_tile = lq * 32 + lane;
+    bool stop = false;
+    for (int ti = t_begin; ti < t_end && !stop; ++ti, ++tcount) {
       const int32_t tc = tiles[ti];
       const int type = tile_type(tc), m = tile_m(tc), n = tile_n(tc);
       const int acc = tcount & 1;
-      if (!mbar_wait(&sm.tfull[acc], (tcount >> 1) & 1, args.status, abort)) break;
+      bool ok = mbar_wait(&sm.tfull[acc], (tcount >> 1) & 1, args.status, nullptr);
+      ok = __all_sync(0xffffffffu, ok);
+      // The four warps of a column half share named barriers, so they leave together: the
+      // flag of tile t is written only before this barrier and read only after it.
+      if (!ok && lane == 0) sm.tflag[half][tcount & 1] = 1;
+      named_sync_half(half);
+      if (*reinterpret_cast<volatile int*>(&sm.tflag[half][tcount & 1])) break;
       tc_fence_after();
-      const int row = m * BM + lq * 32 + lane;  // token (APPLY/TARGET) or Wdown row (UPDATE)
       const uint32_t tbase = tmem + ((uint32_t)(lq * 32) << 16) + (uint32_t)(acc * BN + half * 128);
+      if (type == UPDATE) {
+        // W sub-tiles arrive in smem by TMA; W ← W + η·ΔW in place, the bf16 copy beside it,
+        // and both go back to global memory by TMA stores issued by the half's leader.
 #pragma unroll 1
-      for (int jc = 0; jc < 4; ++jc) {
-        const int col0 = n * BN + half * 128 + jc * 32;
-        uint32_t r[32];
-        tmem_ld32(tbase + jc * 32, r);
-        if (type == UPDATE) {
-          // W[row, col0..col0+31] += η·ΔW, and the bf16 copy for the next chunk.
-          const bool in = row < args.d;
-          float w[32];
-          float* Wrow = args.W + (size_t)row * args.f;
-          const bool full = col0 + 32 <= args.f;
-          if (in && full) {
+        for (int j = 0; j < 4; ++j, ++ecount) {
+          const uint32_t e = 8u * (ecount >> 2) + 2u * (uint32_t)j + (uint32_t)half;  // ring entry
+          const int slot = e % kWSlots;
+          bool okw = mbar_wait(&sm.wfull[slot], (e / kWSlots) & 1, args.status, nullptr);
+          okw = __all_sync(0xffffffffu, okw);
+          if (okw) {
+            uint32_t r[32];
+            tmem_ld32(tbase + j * kWCols, r);
+            tmem_wait_ld();
+            uint8_t* wrow = sm.Wr[slot] + row_in_tile * 128;
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              const float4 v = *reinterpret_cast<const float4*>(Wrow + col0 + 4 * q);
-              w[4 * q] = v.x;
-              w[4 * q + 1] = v.y;
-              w[4 * q + 2] = v.z;
-              w[4 * q + 3] = v.w;
+            for (int c = 0; c < 8; ++c) {
+              float4* p = reinterpret_cast<float4*>(wrow + ((c ^ (row_in_tile & 7)) << 4));
+              float4 w = *p;
+              w.x = fmaf(args.eta, __uint_as_float(r[4 * c + 0]), w.x);
+              w.y = fmaf(args.eta, __uint_as_float(r[4 * c + 1]), w.y);
+              w.z = fmaf(args.eta, __uint_as_float(r[4 * c + 2]), w.z);
+              w.w = fmaf(args.eta, __uint_as_float(r[4 * c + 3]), w.w);
+              *p = w;
+              r[4 * c + 0] = __float_as_uint(w.x);
+              r[4 * c + 1] = __float_as_uint(w.y);
+              r[4 * c + 2] = __float_as_uint(w.z);
+              r[4 * c + 3] = __float_as_uint(w.w);
             }
-          } else if (in) {
-            for (int j = 0; j < 32; ++j) w[j] = col0 + j < args.f ? Wrow[col0 + j] : 0.f;
-          }
-          tmem_wait_ld();
-          if (in) {
+            uint8_t* srow = sm.Sh[half] + row_in_tile * 64;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) w[j] = fmaf(args.eta, __uint_as_float(r[j]), w[j]);
-            if (full) {
-#pragma unroll
-              for (int q = 0; q < 8; ++q)
-                *reinterpret_cast<float4*>(Wrow + col0 + 4 * q) = make_float4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
-            } else {
-              for (int j = 0; j < 32 && col0 + j < args.f; ++j) Wrow[col0 + j] = w[j];
+            for (int c = 0; c < 4; ++c) {
+              uint4 v;
+              v.x = pack_bf16(__uint_as_float(r[8 * c + 0]), __uint_as_float(r[8 * c + 1]));
+              v.y = pack_bf16(__uint_as_float(r[8 * c + 2]), __uint_as_float(r[8 * c + 3]));
+              v.z = pack_bf16(__uint_as_float(r[8 * c + 4]), __uint_as_float(r[8 * c + 5]));
+              v.w = pack_bf16(__uint_as_float(r[8 * c + 6]), __uint_as_float(r[8 * c + 7]));
+              *reinterpret_cast<uint4*>(srow + ((c ^ ((row_in_tile >> 1) & 3)) << 4)) = v;
             }
-            store_row_bf16(args.Wsh_next + (size_t)row * args.f, col0, args.f, w);
+            fence_proxy_async_smem();
+          } else if (lane == 0) {
+            sm.eflag[half][ecount & 1] = 1;
           }
-        } else {
+          named_sync_half(half);
+          // Every warp of the half takes the same decision: the flag of this sub-tile is only
+          // written before the barrier above and only read after it.
+          if (*reinterpret_cast<volatile int*>(&sm.eflag[half][ecount & 1])) {
+            stop = true;
+            break;
+          }
+          if (leader) {
+            const int col = n * BN + half * 128 + j * kWCols;
+            tma_store_2d(&tmWf, sm.Wr[slot], col, m * BM);
+            tma_store_2d(&tmWs, sm.Sh[half], col, m * BM);
+            bulk_commit();
+            bulk_wait_read<0>();          // both stores have read shared memory
+            mbar_arrive(&sm.wempty[slot]);
+          }
+          named_sync_half(half);          // the bf16 staging tile is free again
+        }
+        if (stop) break;
+      } else {
+        const int row = m * BM + row_in_tile;  // token within the chunk
+#pragma unroll 1
+        for (int jc = 0; jc < 4; ++jc) {
+          const int col0 = n * BN + half * 128 + jc * 32;
+          uint32_t r[32];
+          tmem_ld32(tbase + jc * 32, r);
           tmem_wait_ld();
           float v[32];
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-          if (type == APPLY) {
+          if (type == APPLY)
             store_row_bf16(args.O + ((size_t)args.chunk * args.C + row) * args.d, col0, args.d, v);
-          } else {
+          else
             store_row_bf16(args.Vhat_out + (size_t)row * args.d, col0, args.d, v);
-          }
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.tempty[acc]);
     }
+    if (leader) bulk_wait<0>();
   }
 
   tc_fence_before();
@@ -421,12 +506,16 @@ ttt_status upload_plan(const Plan& p, int32_t** dev) {
   return TTT_OK;
 }
 
-ttt_status map2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint32_t box_in, uint32_t box_out) {
+ttt_status map2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint32_t box_in, uint32_t box_out,
+                 CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                 CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B) {
   const uint64_t dims[2] = {inner, outer};
-  const uint64_t strides[1] = {inner * 2};
+  const uint64_t strides[1] = {inner * (dt == CU_TENSOR_MAP_DATA_TYPE_FLOAT32 ? 4u : 2u)};
   const uint32_t box[2] = {box_in, box_out};
-  return encode_tmap(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+  return encode_tmap(m, dt, 2, base, dims, strides, box, sw);
 }
+
+static_assert(sizeof(TCSmem) + 1024 <= 232448, "k_inplace_tc exceeds the 227 KB of shared memory per block");
 
 }  // namespace
 
@@ -484,7 +573,10 @@ ttt_status inplace_bf16_scan(ttt_state* st, const __nv_bfloat16* Z, const __nv_b
   TCResources* r = st->ip.tc;
   const int nchunks = (int)(T / C);
 
-  CUtensorMap tmZk, tmZm, tmVm_in, tmVm_buf[2], tmWk[2], tmConv, tmWt;
+  CUtensorMap tmZk, tmZm, tmVm_in, tmVm_buf[2], tmWk[2], tmConv, tmWt, tmWf, tmWs[2];
+  TTT_TRY(map2d(&tmWf, st->ip.W, f, d, kWCols, BM, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, CU_TENSOR_MAP_SWIZZLE_128B));
+  TTT_TRY(map2d(&tmWs[0], st->ip.Wsh[0], f, d, kWCols, BM, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, CU_TENSOR_MAP_SWIZZLE_64B));
+  TTT_TRY(map2d(&tmWs[1], st->ip.Wsh[1], f, d, kWCols, BM, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, CU_TENSOR_MAP_SWIZZLE_64B));
   TTT_TRY(map2d(&tmZk, Z, f, T, BK, BM));
   TTT_TRY(map2d(&tmZm, Z, f, T, 64, BK));
   TTT_TRY(map2d(&tmWk[0], st->ip.Wsh[0], f, d, BK, BN));
@@ -525,13 +617,12 @@ ttt_status inplace_bf16_scan(ttt_state* st, const __nv_bfloat16* Z, const __nv_b
     a.f = f;
     a.C = C;
     a.eta = c.eta;
-    a.W = st->ip.W;
-    a.Wsh_next = st->ip.Wsh[st->ip.cur ^ 1];
     a.O = O;
     a.Vhat_out = target ? st->ip.Vhat[tchunk & 1] : nullptr;
     a.status = st->status.dev;
     const CUtensorMap& vm = target ? tmVm_buf[chunk & 1] : tmVm_in;
-    k_inplace_tc<<<r->grid[plan], kThreadsTC, smem, s>>>(tmZk, tmZm, vm, tmWk[st->ip.cur], tmConv, tmWt, a);
+    k_inplace_tc<<<r->grid[plan], kThreadsTC, smem, s>>>(tmZk, tmZm, vm, tmWk[st->ip.cur], tmConv, tmWt, tmWf,
+                                                         tmWs[st->ip.cur ^ 1], a);
     st->launches++;
     TTT_CUDA(cudaGetLastError());
     return TTT_OK;
@@ -594,14 +685,12 @@ ttt_status target_values_into(const __nv_bfloat16* X0, const float* convw, const
   a.f = d;
   a.C = T;
   a.eta = 0.f;
-  a.W = nullptr;
-  a.Wsh_next = nullptr;
   a.O = nullptr;
   a.Vhat_out = out;
   a.status = nullptr;
   const size_t smem = sizeof(TCSmem) + 1024;
   TTT_CUDA(cudaFuncSetAttribute(k_inplace_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-  k_inplace_tc<<<grid, kThreadsTC, smem, s>>>(tmConv, tmConv, tmConv, tmConv, tmConv, tmWt, a);
+  k_inplace_tc<<<grid, kThreadsTC, smem, s>>>(tmConv, tmConv, tmConv, tmConv, tmConv, tmWt, tmConv, tmConv, a);
   TTT_CUDA(cudaGetLastError());
   return TTT_OK;
 }

@@ -8,7 +8,7 @@
 
 #include <string>
 
-#include "../../include/ttt.h"
+#include "ttt.h"
 
 namespace ttt {
 

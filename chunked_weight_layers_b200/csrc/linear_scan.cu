@@ -10,8 +10,9 @@
 //    [16w, 16w+16) and runs its chain with no cross-warp synchronisation inside a step.
 //  * everything is computed transposed, so each accumulator layout is directly the next
 //    mma's A operand (no shuffles): Pᵀ = Wᵀ·Kᵀ (+ −Vᵀ), Oᵀ = Wᵀ·Qᵀ, Wᵀ += (−η/b·R)ᵀ·K.
-//  * the fp32 W is fed to the tensor cores as a bf16 hi + lo pair (two mma per product) so
-//    the operand rounding is ~2^-17 instead of 2^-9; R is fed the same way for the update.
+//  * the fp32 W stays in registers; the tensor cores see it rounded to bf16 each step (the
+//    kSplitW switch feeds it as a bf16 hi + lo pair instead); the update operand −(η/b)·R is
+//    rounded to bf16.
 //  * K, V, Q stream through a 4-stage ring of 64-token tiles loaded by TMA (128-byte
 //    swizzle, 3-D maps over [B·H, T, 64] so a head's last tile is clipped to its own T);
 //    outputs are staged in swizzled smem and written by TMA stores.
@@ -78,57 +79,97 @@ __device__ __forceinline__ float2 unpack_bf16(uint32_t v) {
   return __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&v));
 }
 
+// Per-lane shared-memory offsets of the fragments one 16-token step reads or writes. With
+// the 128-byte swizzle the XOR pattern depends only on the row's low three bits, so an
+// offset computed for rows 0..15 holds for any step starting at a multiple of 16 rows:
+// the step adds r0·128.
+struct StepOffsets {
+  uint32_t kb[2][2];  // Kᵀ (and Qᵀ) B fragments of the product with W: [token n-tile][key pair]
+  uint32_t kt[4];     // K B fragments of the update: key n-tile pairs
+  uint32_t v;         // −Vᵀ accumulator init for this warp's 16 columns
+  uint32_t o;         // output tile rows for stmatrix
+};
+
+__device__ __forceinline__ StepOffsets step_offsets(int lane, int col0) {
+  const int mi = lane >> 3, ri = lane & 7;
+  StepOffsets f;
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+    for (int kp = 0; kp < 2; ++kp) f.kb[nt][kp] = swz128_bf16(8 * nt + ri, 32 * kp + 8 * mi);
+#pragma unroll
+  for (int np = 0; np < 4; ++np) f.kt[np] = swz128_bf16(8 * (mi & 1) + ri, 16 * np + 8 * (mi >> 1));
+  f.v = swz128_bf16(8 * (mi >> 1) + ri, col0 + 8 * (mi & 1));
+  f.o = swz128_bf16(8 * (mi >> 1) + ri, col0 + 8 * (mi & 1));
+  return f;
+}
+
+__device__ __forceinline__ void stsm_x4_t(uint32_t addr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3) {
+  asm volatile("stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(r0), "r"(r1),
+               "r"(r2), "r"(r3)
+               : "memory");
+}
+
+// Whether the product with W feeds W to the tensor cores as bf16 hi + lo (two mma per
+// product, operand rounding ~2^-17) or as one bf16 value (rounding 2^-9). Measured on the
+// B=8 x H=12 x T=2048 workload: one value is 22% faster; the final W error stays ~1e-3
+// (it comes from rounding the update operand), the loss error grows from 1.2e-4 to 7e-4.
+constexpr bool kSplitW = false;
+
 // One inner mini-batch of 16 tokens (tile rows r0 .. r0+15) for the warp owning W columns
-// [col0, col0+16). The work is ordered so that consecutive mma instructions are independent:
-// all operand fragments are loaded first, P is accumulated in four partial sums (one per
-// 16-key slice, hi then lo), the output product is issued between the two halves of P, and
-// the loss and output stores come after the weight update has been issued.
-//   Pᵀ = Wᵀ·Kᵀ with W as bf16 hi + lo (the chain's only operand that is not exact in bf16),
-//   Rᵀ = Pᵀ − Vᵀ, loss, Oᵀ = Wᵀ_hi·Qᵀ (the output is stored in bf16 anyway),
-//   Wᵀ += Sᵀ·K with S = −(η/b)·R rounded to bf16.
+// [col0, col0+16). Operand fragments are loaded first; consecutive mma instructions are
+// independent (partial sums per 16-key slice); the loss and the output tile come after the
+// weight update has been issued.
+//   Pᵀ = Wᵀ·Kᵀ,  Rᵀ = Pᵀ − Vᵀ,  Oᵀ = Wᵀ·Qᵀ (W as bf16 hi),  Wᵀ += Sᵀ·K with S = −(η/b)·R in bf16.
 __device__ __forceinline__ void step16(float (&acc)[8][4], uint32_t kbase, uint32_t vbase, uint32_t qbase,
-                                       uint8_t* obuf, float* lossp, int r0, int lane, int col0, float beta,
-                                       int has_q, bool want_loss) {
-  const int g = lane >> 2, q = lane & 3, mi = lane >> 3, ri = lane & 7;
+                                       uint32_t obase, const StepOffsets& f, float* lossp, int r0, int lane,
+                                       float beta, int has_q, bool want_loss) {
+  const int g = lane >> 2, q = lane & 3;
+  const uint32_t rofs = (uint32_t)r0 * 128u;
   uint32_t kb[2][2][4], kt[4][4], vf[4], qb[2][2][4];
 #pragma unroll
   for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-    for (int kp = 0; kp < 2; ++kp) ldsm_x4(kbase + swz128_bf16(r0 + 8 * nt + ri, 32 * kp + 8 * mi), kb[nt][kp]);
-  ldsm_x4_t(vbase + swz128_bf16(r0 + 8 * (mi >> 1) + ri, col0 + 8 * (mi & 1)), vf);
+    for (int kp = 0; kp < 2; ++kp) ldsm_x4(kbase + rofs + f.kb[nt][kp], kb[nt][kp]);
+  ldsm_x4_t(vbase + rofs + f.v, vf);
 #pragma unroll
-  for (int np = 0; np < 4; ++np) ldsm_x4_t(kbase + swz128_bf16(r0 + 8 * (mi & 1) + ri, 16 * np + 8 * (mi >> 1)), kt[np]);
+  for (int np = 0; np < 4; ++np) ldsm_x4_t(kbase + rofs + f.kt[np], kt[np]);
   if (has_q) {
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-      for (int kp = 0; kp < 2; ++kp) ldsm_x4(qbase + swz128_bf16(r0 + 8 * nt + ri, 32 * kp + 8 * mi), qb[nt][kp]);
+      for (int kp = 0; kp < 2; ++kp) ldsm_x4(qbase + rofs + f.kb[nt][kp], qb[nt][kp]);
   }
 
   uint32_t whi[4][4], wlo[4][4];
 #pragma unroll
   for (int ks = 0; ks < 4; ++ks) {
-    split2(acc[2 * ks][0], acc[2 * ks][1], whi[ks][0], wlo[ks][0]);
-    split2(acc[2 * ks][2], acc[2 * ks][3], whi[ks][1], wlo[ks][1]);
-    split2(acc[2 * ks + 1][0], acc[2 * ks + 1][1], whi[ks][2], wlo[ks][2]);
-    split2(acc[2 * ks + 1][2], acc[2 * ks + 1][3], whi[ks][3], wlo[ks][3]);
+    if (kSplitW) {
+      split2(acc[2 * ks][0], acc[2 * ks][1], whi[ks][0], wlo[ks][0]);
+      split2(acc[2 * ks][2], acc[2 * ks][3], whi[ks][1], wlo[ks][1]);
+      split2(acc[2 * ks + 1][0], acc[2 * ks + 1][1], whi[ks][2], wlo[ks][2]);
+      split2(acc[2 * ks + 1][2], acc[2 * ks + 1][3], whi[ks][3], wlo[ks][3]);
+    } else {
+      whi[ks][0] = pack_bf16(acc[2 * ks][0], acc[2 * ks][1]);
+      whi[ks][1] = pack_bf16(acc[2 * ks][2], acc[2 * ks][3]);
+      whi[ks][2] = pack_bf16(acc[2 * ks + 1][0], acc[2 * ks + 1][1]);
+      whi[ks][3] = pack_bf16(acc[2 * ks + 1][2], acc[2 * ks + 1][3]);
+    }
   }
 
-  float pp[2][4][4], o[2][2][4];
+  float pp[2][2][4], o[2][2][4];
 #pragma unroll
   for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-#pragma unroll
-      for (int ks = 0; ks < 4; ++ks) pp[nt][ks][e] = 0.f;
-      o[nt][0][e] = 0.f;
-      o[nt][1][e] = 0.f;
+      pp[nt][0][e] = pp[nt][1][e] = 0.f;
+      o[nt][0][e] = o[nt][1][e] = 0.f;
     }
 #pragma unroll
   for (int ks = 0; ks < 4; ++ks)
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
-      mma16816(pp[nt][ks], whi[ks], kb[nt][ks >> 1][2 * (ks & 1)], kb[nt][ks >> 1][2 * (ks & 1) + 1]);
+      mma16816(pp[nt][ks & 1], whi[ks], kb[nt][ks >> 1][2 * (ks & 1)], kb[nt][ks >> 1][2 * (ks & 1) + 1]);
   if (has_q) {
 #pragma unroll
     for (int ks = 0; ks < 4; ++ks)
@@ -136,11 +177,13 @@ __device__ __forceinline__ void step16(float (&acc)[8][4], uint32_t kbase, uint3
       for (int nt = 0; nt < 2; ++nt)
         mma16816(o[nt][ks & 1], whi[ks], qb[nt][ks >> 1][2 * (ks & 1)], qb[nt][ks >> 1][2 * (ks & 1) + 1]);
   }
+  if (kSplitW) {
 #pragma unroll
-  for (int ks = 0; ks < 4; ++ks)
+    for (int ks = 0; ks < 4; ++ks)
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
-      mma16816(pp[nt][ks], wlo[ks], kb[nt][ks >> 1][2 * (ks & 1)], kb[nt][ks >> 1][2 * (ks & 1) + 1]);
+      for (int nt = 0; nt < 2; ++nt)
+        mma16816(pp[nt][ks & 1], wlo[ks], kb[nt][ks >> 1][2 * (ks & 1)], kb[nt][ks >> 1][2 * (ks & 1) + 1]);
+  }
 
   // R = P − V: p[nt][e] is R[token 8nt + 2q + (e&1)][column col0 + g + 8(e>>1)].
   float p[2][4];
@@ -150,8 +193,7 @@ __device__ __forceinline__ void step16(float (&acc)[8][4], uint32_t kbase, uint3
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-      for (int e = 0; e < 4; ++e)
-        p[nt][e] = ((pp[nt][0][e] + pp[nt][1][e]) + (pp[nt][2][e] + pp[nt][3][e])) - vv[nt][e];
+      for (int e = 0; e < 4; ++e) p[nt][e] = (pp[nt][0][e] + pp[nt][1][e]) - vv[nt][e];
   }
 
   // Weight update Wᵀ += Sᵀ·K (eight independent n-tiles of keys).
@@ -177,22 +219,14 @@ __device__ __forceinline__ void step16(float (&acc)[8][4], uint32_t kbase, uint3
         l0 += __shfl_xor_sync(0xffffffffu, l0, m);
         l1 += __shfl_xor_sync(0xffffffffu, l1, m);
       }
-      if (g == 0) {
-        lossp[r0 + 8 * nt + 2 * q] = l0;
-        lossp[r0 + 8 * nt + 2 * q + 1] = l1;
-      }
+      if (g == 0) *reinterpret_cast<float2*>(&lossp[r0 + 8 * nt + 2 * q]) = make_float2(l0, l1);
     }
   }
   if (has_q) {
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int row = r0 + 8 * nt + 2 * q + (e & 1);
-        const int col = col0 + g + 8 * (e >> 1);
-        *reinterpret_cast<__nv_bfloat16*>(obuf + swz128_bf16(row, col)) =
-            __float2bfloat16_rn(o[nt][0][e] + o[nt][1][e]);
-      }
+    stsm_x4_t(obase + rofs + f.o, pack_bf16(o[0][0][0] + o[0][1][0], o[0][0][1] + o[0][1][1]),
+              pack_bf16(o[0][0][2] + o[0][1][2], o[0][0][3] + o[0][1][3]),
+              pack_bf16(o[1][0][0] + o[1][1][0], o[1][0][1] + o[1][1][1]),
+              pack_bf16(o[1][0][2] + o[1][1][2], o[1][0][3] + o[1][1][3]));
   }
 }
 
@@ -260,6 +294,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
     for (int e = 0; e < 4; ++e) acc[nt][e] = Wg[(8 * nt + 2 * q + (e & 1)) * 64 + col0 + g + 8 * (e >> 1)];
 
+  const StepOffsets offs = step_offsets(lane, col0);
   constexpr int NT = B / 8;   // token n-tiles per mini-batch
   constexpr int KT = B / 16;  // token k-steps per mini-batch
 
@@ -279,7 +314,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if constexpr (B == 16) {
       for (int r0 = 0; r0 < ntok; r0 += 16)
-        step16(acc, kbase, vbase, qbase, obuf, sm.lossp[warp], r0, lane, col0, beta, has_q, loss != nullptr);
+        step16(acc, kbase, vbase, qbase, smem_u32(obuf), offs, sm.lossp[warp], r0, lane, beta, has_q, loss != nullptr);
     } else {
       for (int r0 = 0; r0 < ntok; r0 += B) {
         // A fragments of Wᵀ (hi and lo) for the four 16-key k-steps.
