@@ -224,6 +224,29 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
+def dominant_kernel(spec) -> str:
+    if isinstance(spec, wl.LinearSpec):
+        return "k_linear_scan"
+    return "k_sgemm" if spec.dtype == "f32" else "k_inplace_tc"
+
+
+def traffic_per_launch(spec):
+    """DRAM bytes per launch of the workload's dominant kernel from the committed ncu record,
+    or None when there is none or the kernel's source changed since the capture."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(p):
+        return None
+    rec = json.load(open(p)).get(f"{dominant_kernel(spec)}@{spec.name.split('@')[0]}")
+    if rec is None:
+        return None
+    src = os.path.join(ROOT, rec["source"])
+    if not os.path.exists(src):
+        return None
+    digest = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    return rec["bytes_per_launch"] if digest.startswith(rec["sha256_prefix"]) else None
+
+
 def roofline(spec, w, ms, peaks, traffic=None):
     if w["bound"] == "hbm":
         achieved = w["bytes"] / (ms * 1e-3) / 1e9
@@ -294,7 +317,8 @@ def measure(spec, steps, warmup, flush, peaks, device, with_e2e):
     ms = statistics.mean(times)
     w = work(spec)
     out = {"workload": spec.name, "ms_per_step": ms, "tokens_per_s": w["tokens"] / (ms * 1e-3),
-           "tflops": w["flops"] / (ms * 1e-3) / 1e12, "roofline": roofline(spec, w, ms, peaks),
+           "tflops": w["flops"] / (ms * 1e-3) / 1e12,
+           "roofline": roofline(spec, w, ms, peaks, traffic_per_launch(spec)),
            "gpu_launches_per_step": launches / max(1, steps), "times_ms": times}
     if with_e2e:
         e2e_ms, h2d, d2h = time_e2e(r, max(3, steps // 2), 1)
@@ -327,6 +351,9 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     spec = spec_by_name(a.workload)
+    if world > 1:
+        # Weak scaling: every rank scans its own batch of independent problems (its own seed).
+        spec = wl.scaled(spec, seed=spec.seed + 7919 * rank)
     w = work(spec)
     peaks = load_peaks()
 
@@ -388,21 +415,15 @@ def main():
     if pg is not None:
         pg.barrier()
     runner.state.poll()
-    total_ms = sum(times)
-    if pg is not None:
-        t = torch.tensor([total_ms], device=device)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        total_ms = float(t.item())
+    from chunked_weight_layers_b200.dist import max_over_ranks
+    total_ms = max_over_ranks(sum(times), device)
     ms = total_ms / a.steps
     value = world * w["tokens"] / (ms * 1e-3)
     e2e_ms, h2d, d2h = None, 0, 0
     runner_e2e = None
     try:
         e2e_ms, h2d, d2h = time_e2e(runner, max(3, a.steps // 2), 1)
-        if pg is not None:
-            t = torch.tensor([e2e_ms], device=device)
-            pg.all_reduce(t, op=pg.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = max_over_ranks(e2e_ms, device)
         runner_e2e = world * w["tokens"] / (e2e_ms * 1e-3)
     except Exception as ex:  # report, do not hide
         runner_e2e = None
@@ -422,7 +443,8 @@ def main():
                 extra[s.name] = {"error": str(ex)}
 
     if rank == 0:
-        rl = roofline(spec, w, ms, peaks)
+        rl = roofline(spec, w, ms, peaks, traffic_per_launch(spec))
+        rl["kernel"] = dominant_kernel(spec)
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": a.steps,
             "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
