@@ -4,21 +4,27 @@
 //   O_i = Q_i·W_i,   R_i = K_i·W_i − V_i,   L_t = ‖R_i[t]‖²,   W_{i+1} = W_i − (η/b)·K_iᵀ·R_i.
 //
 // Design (B200):
-//  * one CTA per (sequence, head); the per-head state is 64x64 fp32 and never leaves the SM:
-//    it lives in mma accumulator registers of four compute warps. Column c of W only ever
-//    depends on column c of R (R[:, c] = K·W[:, c] − V[:, c]), so warp w owns the 16 columns
-//    [16w, 16w+16) and runs its chain with no cross-warp synchronisation inside a step.
-//  * everything is computed transposed, so each accumulator layout is directly the next
-//    mma's A operand (no shuffles): Pᵀ = Wᵀ·Kᵀ (+ −Vᵀ), Oᵀ = Wᵀ·Qᵀ, Wᵀ += (−η/b·R)ᵀ·K.
-//  * the fp32 W stays in registers; the tensor cores see it rounded to bf16 each step (the
-//    kSplitW switch feeds it as a bf16 hi + lo pair instead); the update operand −(η/b)·R is
-//    rounded to bf16.
-//  * K, V, Q stream through a 4-stage ring of 64-token tiles loaded by TMA (128-byte
-//    swizzle, 3-D maps over [B·H, T, 64] so a head's last tile is clipped to its own T);
-//    outputs are staged in swizzled smem and written by TMA stores.
-//  * the chain per step is latency-bound and tiny (393 kFLOP), so it runs on the legacy
-//    warp-level mma.sync path: a tcgen05 round trip (issue, commit, mbarrier, tcgen05.ld)
-//    per dependent 16x64x64 product costs more than the product itself.
+//  * the per-head state is 64x64 fp32 and never leaves the SM: it lives in mma accumulator
+//    registers. Column c of W only ever depends on column c of R (R[:, c] = K·W[:, c] − V[:, c]),
+//    so columns are split across warps (and, for b = 16, a head's two column halves across
+//    two CTAs) with no communication inside a step.
+//  * k_linear_n8 (b = 16 when 2·B·H ≤ SM count): two CTAs per head, four warps per CTA, eight
+//    columns per warp, products in their natural orientation with movmatrix.trans turning
+//    accumulators into B operands; partial losses of the two halves are added into a zeroed
+//    output. Half the work per warp, so the serial chain of long scans runs faster.
+//  * k_linear_scan (otherwise, and for b = 32 or 64): one CTA per head, sixteen columns per
+//    warp, every product computed transposed so each accumulator layout is directly the next
+//    mma's A operand. Measured on the B=8 x H=12 workload (192 half-heads > 148 SMs) this is
+//    the faster form: 53 us against 57 us.
+//  * the tensor cores see W rounded to bf16 each step and the update operand −(η/b)·R rounded
+//    to bf16; W itself and every accumulation stay fp32.
+//  * K, V, Q stream through a 4-stage ring of 64-token tiles loaded by TMA (128-byte swizzle,
+//    3-D maps over [B·H, T, 64] so a head's last tile is clipped to its own T); outputs are
+//    staged in swizzled smem and written by TMA stores.
+//  * the chain per step is latency-bound and tiny (393 kFLOP per head), so it runs on the
+//    warp-level mma.sync path: a tcgen05 round trip (issue, commit, mbarrier, tcgen05.ld) per
+//    dependent 16x64x64 product costs more than the product itself. Measured on B200:
+//    mma.sync m16n8k16 latency ~21 cycles, at most one per ~8.2 cycles per SM sub-partition.
 #include "common.cuh"
 #include "internal.h"
 
@@ -229,6 +235,7 @@ __device__ __forceinline__ void step16(float (&acc)[8][4], uint32_t kbase, uint3
               pack_bf16(o[1][0][2] + o[1][1][2], o[1][0][3] + o[1][1][3]));
   }
 }
+
 
 template <int B>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -453,6 +460,229 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
 }
 
+
+// ---------------------------------------------------------------------------------------------
+// Inner mini-batch b = 16, eight columns per warp, each head split over two CTAs.
+//
+// Column c of W only depends on column c of R, so a head's 64 columns are split into two
+// halves on two CTAs (no communication) and each of a CTA's four warps owns 8 columns. The
+// products run in their natural orientation (m16n8k16 with N = 8 columns):
+//   P = K·W (A = K from ldmatrix, B = W from the accumulator via movmatrix.trans),
+//   R = P − V, loss, S = −(η/b)·R,
+//   W += Kᵀ·S (A = Kᵀ from ldmatrix.trans, B = S via movmatrix.trans),  O = Q·W.
+// Half the instructions per warp and step of the 16-columns-per-warp form, and the heads
+// reach every SM. The per-token loss is the sum of the two halves' partial sums: each CTA
+// adds its partial to a zeroed output (two terms onto zero: the result does not depend on
+// their order).
+// ---------------------------------------------------------------------------------------------
+
+struct N8Offsets {
+  uint32_t ka[4];  // K (or Q) A fragments: [16-key k-step]
+  uint32_t kt[4];  // Kᵀ A fragments of the update: [16-key m-tile]
+  uint32_t v;      // V fragment of this warp's 8 columns
+  uint32_t o;      // output staging rows (64-byte rows, 64-byte swizzle)
+};
+
+__device__ __forceinline__ N8Offsets n8_offsets(int lane, int vcol, int w) {
+  const int mi = lane >> 3, ri = lane & 7;
+  N8Offsets f;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    f.ka[k] = swz128_bf16(8 * (mi & 1) + ri, 16 * k + 8 * (mi >> 1));
+    f.kt[k] = swz128_bf16(8 * (mi >> 1) + ri, 16 * k + 8 * (mi & 1));
+  }
+  f.v = swz128_bf16(8 * (mi & 1) + ri, vcol);
+  const int orow = 8 * (mi & 1) + ri;
+  f.o = (uint32_t)(orow * 64 + ((w ^ ((orow >> 1) & 3)) << 4));
+  return f;
+}
+
+__device__ __forceinline__ uint32_t movm_t(uint32_t a) {
+  uint32_t d;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(a));
+  return d;
+}
+
+__device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t& r0, uint32_t& r1) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(addr));
+}
+
+__device__ __forceinline__ void stsm_x2(uint32_t addr, uint32_t r0, uint32_t r1) {
+  asm volatile("stmatrix.sync.aligned.m8n8.x2.shared.b16 [%0], {%1, %2};" ::"r"(addr), "r"(r0), "r"(r1) : "memory");
+}
+
+__device__ __forceinline__ void mma_n8(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// acc[mt][e] = W[16mt + g + 8(e>>1)][col0 + 2q + (e&1)] for this warp's 8 columns.
+__device__ __forceinline__ void step16_n8(float (&acc)[4][4], uint32_t kbase, uint32_t vbase, uint32_t qbase,
+                                          uint32_t obase, const N8Offsets& f, float* lossp, int r0, int lane,
+                                          float beta, int has_q, bool want_loss) {
+  const int g = lane >> 2;
+  const uint32_t rofs = (uint32_t)r0 * 128u;
+  uint32_t ka[4][4], kt[4][4], qa[4][4], v0, v1;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) ldsm_x4(kbase + rofs + f.ka[k], ka[k]);
+  ldsm_x2(vbase + rofs + f.v, v0, v1);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) ldsm_x4_t(kbase + rofs + f.kt[k], kt[k]);
+  if (has_q) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) ldsm_x4(qbase + rofs + f.ka[k], qa[k]);
+  }
+  // W as B fragments: movmatrix.trans turns the accumulator layout (key rows, column pairs)
+  // into (key pairs, column) per 8x8 block.
+  uint32_t wb[4][2];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    wb[k][0] = movm_t(pack_bf16(acc[k][0], acc[k][1]));
+    wb[k][1] = movm_t(pack_bf16(acc[k][2], acc[k][3]));
+  }
+  float pa[4] = {0.f, 0.f, 0.f, 0.f}, pb[4] = {0.f, 0.f, 0.f, 0.f}, o[4] = {0.f, 0.f, 0.f, 0.f};
+  mma_n8(pa, ka[0], wb[0][0], wb[0][1]);
+  mma_n8(pb, ka[1], wb[1][0], wb[1][1]);
+  mma_n8(pa, ka[2], wb[2][0], wb[2][1]);
+  mma_n8(pb, ka[3], wb[3][0], wb[3][1]);
+  if (has_q) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) mma_n8(o, qa[k], wb[k][0], wb[k][1]);
+  }
+  // R = P − V: p[e] = R[token g + 8(e>>1)][column 2q + (e&1)].
+  const float2 va = unpack_bf16(v0), vb = unpack_bf16(v1);
+  float p[4];
+  p[0] = (pa[0] + pb[0]) - va.x;
+  p[1] = (pa[1] + pb[1]) - va.y;
+  p[2] = (pa[2] + pb[2]) - vb.x;
+  p[3] = (pa[3] + pb[3]) - vb.y;
+  // S = −(η/b)·R as B fragments (token pairs, column).
+  const uint32_t sb0 = movm_t(pack_bf16(-beta * p[0], -beta * p[1]));
+  const uint32_t sb1 = movm_t(pack_bf16(-beta * p[2], -beta * p[3]));
+#pragma unroll
+  for (int k = 0; k < 4; ++k) mma_n8(acc[k], kt[k], sb0, sb1);
+
+  if (want_loss) {
+    float l0 = p[0] * p[0] + p[1] * p[1];
+    float l1 = p[2] * p[2] + p[3] * p[3];
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+    if ((lane & 3) == 0) {
+      lossp[r0 + g] = l0;
+      lossp[r0 + g + 8] = l1;
+    }
+  }
+  if (has_q) stsm_x2(obase + (uint32_t)r0 * 64u + f.o, pack_bf16(o[0], o[1]), pack_bf16(o[2], o[3]));
+}
+
+struct __align__(1024) N8Smem {
+  uint8_t K[kStages][kTileBytes];
+  uint8_t V[kStages][kTileBytes];
+  uint8_t Q[kStages][kTileBytes];
+  uint8_t O[2][kTileTok * 64];  // this CTA's 32 output columns of a tile (64-byte swizzle)
+  float lossp[kComputeWarps][kTileTok];
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
+  int abort;
+  int cabort[2];
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+    k_linear_n8(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
+                float* __restrict__ Wstate, float* __restrict__ loss, int T, float beta, int has_q, int* status) {
+  extern __shared__ uint8_t smem_raw[];
+  N8Smem& sm = *reinterpret_cast<N8Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bh = blockIdx.x >> 1, half = blockIdx.x & 1;
+  const int nstages = (T + kTileTok - 1) / kTileTok;
+  const uint32_t stage_bytes = (has_q ? 3u : 2u) * kTileBytes;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&sm.full[i], 1);
+      mbar_init(&sm.empty[i], kComputeWarps);
+    }
+    sm.abort = 0;
+    sm.cabort[0] = sm.cabort[1] = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  if (warp == kComputeWarps) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      if (has_q) tma_prefetch_desc(&tmQ);
+      int issued = 0;
+      for (int s = 0; s < nstages; ++s) {
+        const int slot = s % kStages;
+        if (s >= kStages && !mbar_wait(&sm.empty[slot], ((s / kStages) - 1) & 1, status, &sm.abort)) break;
+        mbar_arrive_expect_tx(&sm.full[slot], stage_bytes);
+        tma_load_3d(sm.K[slot], &tmK, &sm.full[slot], 0, s * kTileTok, bh);
+        tma_load_3d(sm.V[slot], &tmV, &sm.full[slot], 0, s * kTileTok, bh);
+        if (has_q) tma_load_3d(sm.Q[slot], &tmQ, &sm.full[slot], 0, s * kTileTok, bh);
+        issued = s + 1;
+      }
+      for (int s = issued - kStages; s < issued; ++s) {
+        if (s < 0) continue;
+        mbar_wait(&sm.full[s % kStages], (s / kStages) & 1, status, nullptr);
+      }
+    }
+    __syncthreads();
+    return;
+  }
+
+  const int g = lane >> 2, q = lane & 3;
+  const int col0 = 32 * half + 8 * warp;  // first W column owned by this warp
+  float* Wg = Wstate + (size_t)bh * 64 * 64;
+  float acc[4][4];
+#pragma unroll
+  for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[mt][e] = Wg[(16 * mt + g + 8 * (e >> 1)) * 64 + col0 + 2 * q + (e & 1)];
+  const N8Offsets offs = n8_offsets(lane, col0, warp);
+
+  for (int s = 0; s < nstages; ++s) {
+    const int slot = s % kStages;
+    // Every compute warp takes the same exit decision (see k_linear_scan).
+    if (!mbar_wait(&sm.full[slot], (s / kStages) & 1, status, nullptr)) sm.cabort[s & 1] = 1;
+    named_sync();
+    if (*reinterpret_cast<volatile int*>(&sm.cabort[s & 1])) break;
+    const int ntok = min(kTileTok, T - s * kTileTok);
+    const uint32_t kbase = smem_u32(sm.K[slot]), vbase = smem_u32(sm.V[slot]), qbase = smem_u32(sm.Q[slot]);
+    uint8_t* obuf = sm.O[s & 1];
+    for (int r0 = 0; r0 < ntok; r0 += 16)
+      step16_n8(acc, kbase, vbase, qbase, smem_u32(obuf), offs, sm.lossp[warp], r0, lane, beta, has_q,
+                loss != nullptr);
+    if (has_q) fence_proxy_async_smem();
+    named_sync();
+    if (loss != nullptr && warp == 0) {
+      for (int i = lane; i < ntok; i += 32) {
+        const float l = (sm.lossp[0][i] + sm.lossp[1][i]) + (sm.lossp[2][i] + sm.lossp[3][i]);
+        atomicAdd(&loss[(size_t)bh * T + (size_t)s * kTileTok + i], l);
+      }
+    }
+    if (threadIdx.x == 0 && has_q) {
+      tma_store_3d(&tmO, obuf, 32 * half, s * kTileTok, bh);
+      bulk_commit();
+      bulk_wait_read<1>();
+    }
+    named_sync();
+    if (lane == 0) mbar_arrive(&sm.empty[slot]);
+  }
+  if (threadIdx.x == 0 && has_q) bulk_wait<0>();
+#pragma unroll
+  for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) Wg[(16 * mt + g + 8 * (e >> 1)) * 64 + col0 + 2 * q + (e & 1)] = acc[mt][e];
+  __syncthreads();
+}
+
 template <int B>
 ttt_status launch(ttt_state* st, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
                   const CUtensorMap& to, float* loss, int T, int has_q, cudaStream_t s) {
@@ -466,6 +696,19 @@ ttt_status launch(ttt_state* st, const CUtensorMap& tk, const CUtensorMap& tv, c
   return TTT_OK;
 }
 
+
+ttt_status launch_n8(ttt_state* st, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
+                     const CUtensorMap& to, float* loss, int T, int has_q, cudaStream_t s) {
+  const size_t smem = sizeof(N8Smem) + 1024;
+  TTT_CUDA(cudaFuncSetAttribute(k_linear_n8, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  const int bh = st->cfg.batch * st->cfg.heads;
+  if (loss != nullptr) TTT_CUDA(cudaMemsetAsync(loss, 0, (size_t)bh * T * sizeof(float), s));
+  const float beta = st->cfg.eta / 16.0f;
+  k_linear_n8<<<2 * bh, kThreads, smem, s>>>(tk, tv, tq, to, st->lin.W, loss, T, beta, has_q, st->status.dev);
+  st->launches++;
+  TTT_CUDA(cudaGetLastError());
+  return TTT_OK;
+}
 }  // namespace
 
 ttt_status linear_scan(ttt_state* st, const __nv_bfloat16* K, const __nv_bfloat16* V, const __nv_bfloat16* Q,
@@ -476,18 +719,27 @@ ttt_status linear_scan(ttt_state* st, const __nv_bfloat16* K, const __nv_bfloat1
   const uint64_t strides[2] = {128, (uint64_t)T * 128};
   const uint32_t box[3] = {64, (uint32_t)kTileTok, 1};
   CUtensorMap tk, tv, tq, to;
+  // b = 16: eight columns per warp on two CTAs per head when every half-head gets its own SM;
+  // otherwise sixteen columns per warp on one CTA per head (fewer, fuller SMs win then).
+  const bool n8 = c.chunk == 16 && 2 * (int64_t)c.batch * c.heads <= st->num_sms;
   TTT_TRY(encode_tmap(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, K, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B));
   TTT_TRY(encode_tmap(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, V, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B));
   const int has_q = Q != nullptr;
   if (has_q) {
     TTT_TRY(encode_tmap(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, Q, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B));
-    TTT_TRY(encode_tmap(&to, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, O, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B));
+    if (n8) {
+      const uint32_t obox[3] = {32, (uint32_t)kTileTok, 1};
+      TTT_TRY(encode_tmap(&to, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, O, dims, strides, obox, CU_TENSOR_MAP_SWIZZLE_64B));
+    } else {
+      TTT_TRY(encode_tmap(&to, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, O, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B));
+    }
   } else {
     tq = tk;
     to = tk;
   }
   switch (c.chunk) {
-    case 16: return launch<16>(st, tk, tv, tq, to, loss, (int)T, has_q, s);
+    case 16: return n8 ? launch_n8(st, tk, tv, tq, to, loss, (int)T, has_q, s)
+                       : launch<16>(st, tk, tv, tq, to, loss, (int)T, has_q, s);
     case 32: return launch<32>(st, tk, tv, tq, to, loss, (int)T, has_q, s);
     case 64: return launch<64>(st, tk, tv, tq, to, loss, (int)T, has_q, s);
     default: return fail(TTT_ERR_UNSUPPORTED, "TTT-Linear: mini-batch %d not built", c.chunk);

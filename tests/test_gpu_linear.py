@@ -62,9 +62,12 @@ def test_identity_fixed_point_is_exact(cwl):
     assert torch.count_nonzero(L).item() == 0
 
 
-@pytest.mark.parametrize("b,T", [(16, 208), (32, 224), (64, 192), (16, 64)])
-def test_small_shapes_and_ragged_tiles(cwl, b, T):
-    spec = workloads.scaled(workloads.LINEAR_GD, B=2, H=3, T=T, b=b, seed=77 + b)
+@pytest.mark.parametrize("b,T,B,H", [(16, 208, 2, 3), (32, 224, 2, 3), (64, 192, 2, 3), (16, 64, 2, 3),
+                                     (16, 208, 1, 80)])
+def test_small_shapes_and_ragged_tiles(cwl, b, T, B, H):
+    """B*H = 6 takes the eight-columns-per-warp kernel at b = 16; B*H = 80 (160 half-heads,
+    more than the 148 SMs) takes the sixteen-columns-per-warp one."""
+    spec = workloads.scaled(workloads.LINEAR_GD, B=B, H=H, T=T, b=b, seed=77 + b + H)
     x = workloads.linear_inputs(spec, device="cuda")
     W0 = x["W0"].clone()
     W0 += 0.05 * torch.randn(W0.shape, generator=torch.Generator().manual_seed(b)).cuda()
