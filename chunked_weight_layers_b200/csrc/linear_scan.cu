@@ -8,19 +8,24 @@
 //    registers. Column c of W only ever depends on column c of R (R[:, c] = K·W[:, c] − V[:, c]),
 //    so columns are split across warps (and, for b = 16, a head's two column halves across
 //    two CTAs) with no communication inside a step.
+//  * k_linear_b16 (b = 16, one CTA per head): four compute warps own sixteen columns each and
+//    compute every product transposed, so each accumulator layout is directly the next mma's A
+//    operand. Operand fragments are loaded one step ahead; a 64-token tile is four
+//    straight-line steps with all waits at its top. A TMA producer warp fills the K/V/Q ring
+//    and a writer warp sums loss partials and stores the output tiles, so compute warps never
+//    meet at a barrier.
 //  * k_linear_n8 (b = 16 when 2·B·H ≤ SM count): two CTAs per head, four warps per CTA, eight
 //    columns per warp, products in their natural orientation with movmatrix.trans turning
 //    accumulators into B operands; partial losses of the two halves are added into a zeroed
-//    output. Half the work per warp, so the serial chain of long scans runs faster.
-//  * k_linear_scan (otherwise, and for b = 32 or 64): one CTA per head, sixteen columns per
-//    warp, every product computed transposed so each accumulator layout is directly the next
-//    mma's A operand. Measured on the B=8 x H=12 workload (192 half-heads > 148 SMs) this is
-//    the faster form: 53 us against 57 us.
-//  * the tensor cores see W rounded to bf16 each step and the update operand −(η/b)·R rounded
-//    to bf16; W itself and every accumulation stay fp32.
+//    output.
+//  * k_linear_scan (b = 32 or 64): one CTA per head, sixteen columns per warp, W and the update
+//    operand fed to the tensor cores as bf16 hi + lo pairs.
+//  * for b = 16 the tensor cores see W rounded to bf16 each step and the update operand
+//    −(η/b)·R rounded to bf16; W itself and every accumulation stay fp32.
 //  * K, V, Q stream through a 4-stage ring of 64-token tiles loaded by TMA (128-byte swizzle,
 //    3-D maps over [B·H, T, 64] so a head's last tile is clipped to its own T); outputs are
-//    staged in swizzled smem and written by TMA stores.
+//    staged in swizzled smem and written by TMA stores. Compute warps wait on a full slot for
+//    under 6% of the scan, and an 8-stage ring measured no faster.
 //  * the chain per step is latency-bound and tiny (393 kFLOP per head), so it runs on the
 //    warp-level mma.sync path: a tcgen05 round trip (issue, commit, mbarrier, tcgen05.ld) per
 //    dependent 16x64x64 product costs more than the product itself. Measured on B200:
@@ -32,7 +37,7 @@ namespace ttt {
 
 namespace {
 
-constexpr int kStages = 4;        // ring depth (64-token tiles)
+constexpr int kStages = 4;        // ring depth (64-token tiles): 96 KB of K/V/Q in flight per SM
 constexpr int kTileTok = 64;      // tokens per tile
 constexpr int kTileBytes = kTileTok * 128;  // 64 tokens x 64 bf16
 constexpr int kComputeWarps = 4;
@@ -116,93 +121,75 @@ __device__ __forceinline__ void stsm_x4_t(uint32_t addr, uint32_t r0, uint32_t r
                : "memory");
 }
 
-// Whether the product with W feeds W to the tensor cores as bf16 hi + lo (two mma per
-// product, operand rounding ~2^-17) or as one bf16 value (rounding 2^-9). Measured on the
-// B=8 x H=12 x T=2048 workload: one value is 22% faster; the final W error stays ~1e-3
-// (it comes from rounding the update operand), the loss error grows from 1.2e-4 to 7e-4.
-constexpr bool kSplitW = false;
+// Operand fragments of one 16-token inner mini-batch (tile rows r0 .. r0+15) for the warp
+// owning W columns [col0, col0+16). They are loaded one step ahead: while a step's dependent
+// chain runs, the shared-memory reads of the next step are already in flight.
+struct Frag16 {
+  uint32_t kb[2][2][4];  // Kᵀ B fragments of the product with W: [token n-tile][key pair]
+  uint32_t kt[4][4];     // K B fragments of the update: [key n-tile pair]
+  uint32_t vf[4];        // Vᵀ of this warp's columns
+  uint32_t qb[2][2][4];  // Qᵀ B fragments of the outputs
+};
 
-// One inner mini-batch of 16 tokens (tile rows r0 .. r0+15) for the warp owning W columns
-// [col0, col0+16). Operand fragments are loaded first; consecutive mma instructions are
-// independent (partial sums per 16-key slice); the loss and the output tile come after the
-// weight update has been issued.
-//   Pᵀ = Wᵀ·Kᵀ,  Rᵀ = Pᵀ − Vᵀ,  Oᵀ = Wᵀ·Qᵀ (W as bf16 hi),  Wᵀ += Sᵀ·K with S = −(η/b)·R in bf16.
-__device__ __forceinline__ void step16(float (&acc)[8][4], uint32_t kbase, uint32_t vbase, uint32_t qbase,
-                                       uint32_t obase, const StepOffsets& f, float* lossp, int r0, int lane,
-                                       float beta, int has_q, bool want_loss) {
-  const int g = lane >> 2, q = lane & 3;
+template <bool HAS_Q>
+__device__ __forceinline__ void load_frag16(Frag16& F, uint32_t kbase, uint32_t vbase, uint32_t qbase,
+                                            const StepOffsets& f, int r0) {
   const uint32_t rofs = (uint32_t)r0 * 128u;
-  uint32_t kb[2][2][4], kt[4][4], vf[4], qb[2][2][4];
 #pragma unroll
   for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-    for (int kp = 0; kp < 2; ++kp) ldsm_x4(kbase + rofs + f.kb[nt][kp], kb[nt][kp]);
-  ldsm_x4_t(vbase + rofs + f.v, vf);
+    for (int kp = 0; kp < 2; ++kp) ldsm_x4(kbase + rofs + f.kb[nt][kp], F.kb[nt][kp]);
+  ldsm_x4_t(vbase + rofs + f.v, F.vf);
 #pragma unroll
-  for (int np = 0; np < 4; ++np) ldsm_x4_t(kbase + rofs + f.kt[np], kt[np]);
-  if (has_q) {
+  for (int np = 0; np < 4; ++np) ldsm_x4_t(kbase + rofs + f.kt[np], F.kt[np]);
+  if (HAS_Q) {
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-      for (int kp = 0; kp < 2; ++kp) ldsm_x4(qbase + rofs + f.kb[nt][kp], qb[nt][kp]);
+      for (int kp = 0; kp < 2; ++kp) ldsm_x4(qbase + rofs + f.kb[nt][kp], F.qb[nt][kp]);
   }
+}
 
-  uint32_t whi[4][4], wlo[4][4];
+// One inner mini-batch from loaded fragments, everything transposed so that each accumulator
+// layout is directly the next mma's A operand:
+//   Pᵀ = Wᵀ·Kᵀ,  Rᵀ = Pᵀ − Vᵀ,  Wᵀ += Sᵀ·K with S = −(η/b)·R,  Oᵀ = Wᵀ_old·Qᵀ.
+// The tensor cores see W and S rounded to bf16; W and every accumulation stay fp32. The
+// output products are issued after the update so they do not delay the dependent chain.
+template <bool HAS_Q, bool LOSS>
+__device__ __forceinline__ void compute16(float (&acc)[8][4], const Frag16& F, uint32_t obase, uint32_t ofs_o,
+                                          float* lossp, int r0, int lane, float beta) {
+  const int g = lane >> 2, q = lane & 3;
+  uint32_t wa[4][4];
 #pragma unroll
   for (int ks = 0; ks < 4; ++ks) {
-    if (kSplitW) {
-      split2(acc[2 * ks][0], acc[2 * ks][1], whi[ks][0], wlo[ks][0]);
-      split2(acc[2 * ks][2], acc[2 * ks][3], whi[ks][1], wlo[ks][1]);
-      split2(acc[2 * ks + 1][0], acc[2 * ks + 1][1], whi[ks][2], wlo[ks][2]);
-      split2(acc[2 * ks + 1][2], acc[2 * ks + 1][3], whi[ks][3], wlo[ks][3]);
-    } else {
-      whi[ks][0] = pack_bf16(acc[2 * ks][0], acc[2 * ks][1]);
-      whi[ks][1] = pack_bf16(acc[2 * ks][2], acc[2 * ks][3]);
-      whi[ks][2] = pack_bf16(acc[2 * ks + 1][0], acc[2 * ks + 1][1]);
-      whi[ks][3] = pack_bf16(acc[2 * ks + 1][2], acc[2 * ks + 1][3]);
-    }
+    wa[ks][0] = pack_bf16(acc[2 * ks][0], acc[2 * ks][1]);
+    wa[ks][1] = pack_bf16(acc[2 * ks][2], acc[2 * ks][3]);
+    wa[ks][2] = pack_bf16(acc[2 * ks + 1][0], acc[2 * ks + 1][1]);
+    wa[ks][3] = pack_bf16(acc[2 * ks + 1][2], acc[2 * ks + 1][3]);
   }
-
-  float pp[2][2][4], o[2][2][4];
+  // Two partial sums per token n-tile (keys 0-15 + 32-47 and 16-31 + 48-63) halve the chain.
+  float pp[2][2][4];
 #pragma unroll
   for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      pp[nt][0][e] = pp[nt][1][e] = 0.f;
-      o[nt][0][e] = o[nt][1][e] = 0.f;
-    }
+    for (int e = 0; e < 4; ++e) pp[nt][0][e] = pp[nt][1][e] = 0.f;
 #pragma unroll
   for (int ks = 0; ks < 4; ++ks)
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
-      mma16816(pp[nt][ks & 1], whi[ks], kb[nt][ks >> 1][2 * (ks & 1)], kb[nt][ks >> 1][2 * (ks & 1) + 1]);
-  if (has_q) {
-#pragma unroll
-    for (int ks = 0; ks < 4; ++ks)
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
-        mma16816(o[nt][ks & 1], whi[ks], qb[nt][ks >> 1][2 * (ks & 1)], qb[nt][ks >> 1][2 * (ks & 1) + 1]);
-  }
-  if (kSplitW) {
-#pragma unroll
-    for (int ks = 0; ks < 4; ++ks)
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
-        mma16816(pp[nt][ks & 1], wlo[ks], kb[nt][ks >> 1][2 * (ks & 1)], kb[nt][ks >> 1][2 * (ks & 1) + 1]);
-  }
+      mma16816(pp[nt][ks & 1], wa[ks], F.kb[nt][ks >> 1][2 * (ks & 1)], F.kb[nt][ks >> 1][2 * (ks & 1) + 1]);
 
   // R = P − V: p[nt][e] is R[token 8nt + 2q + (e&1)][column col0 + g + 8(e>>1)].
   float p[2][4];
   {
-    const float2 v0 = unpack_bf16(vf[0]), v1 = unpack_bf16(vf[1]), v2 = unpack_bf16(vf[2]), v3 = unpack_bf16(vf[3]);
+    const float2 v0 = unpack_bf16(F.vf[0]), v1 = unpack_bf16(F.vf[1]), v2 = unpack_bf16(F.vf[2]),
+                 v3 = unpack_bf16(F.vf[3]);
     const float vv[2][4] = {{v0.x, v0.y, v1.x, v1.y}, {v2.x, v2.y, v3.x, v3.y}};
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) p[nt][e] = (pp[nt][0][e] + pp[nt][1][e]) - vv[nt][e];
   }
-
-  // Weight update Wᵀ += Sᵀ·K (eight independent n-tiles of keys).
   uint32_t sa[4];
   sa[0] = pack_bf16(-beta * p[0][0], -beta * p[0][1]);
   sa[1] = pack_bf16(-beta * p[0][2], -beta * p[0][3]);
@@ -210,12 +197,27 @@ __device__ __forceinline__ void step16(float (&acc)[8][4], uint32_t kbase, uint3
   sa[3] = pack_bf16(-beta * p[1][2], -beta * p[1][3]);
 #pragma unroll
   for (int np = 0; np < 4; ++np) {
-    mma16816(acc[2 * np], sa, kt[np][0], kt[np][1]);
-    mma16816(acc[2 * np + 1], sa, kt[np][2], kt[np][3]);
+    mma16816(acc[2 * np], sa, F.kt[np][0], F.kt[np][1]);
+    mma16816(acc[2 * np + 1], sa, F.kt[np][2], F.kt[np][3]);
   }
 
-  // Off the critical path: per-token loss partials and the output tile.
-  if (want_loss) {
+  if (HAS_Q) {
+    float o[2][2][4];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[nt][0][e] = o[nt][1][e] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks)
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+        mma16816(o[nt][ks & 1], wa[ks], F.qb[nt][ks >> 1][2 * (ks & 1)], F.qb[nt][ks >> 1][2 * (ks & 1) + 1]);
+    stsm_x4_t(obase + (uint32_t)r0 * 128u + ofs_o, pack_bf16(o[0][0][0] + o[0][1][0], o[0][0][1] + o[0][1][1]),
+              pack_bf16(o[0][0][2] + o[0][1][2], o[0][0][3] + o[0][1][3]),
+              pack_bf16(o[1][0][0] + o[1][1][0], o[1][0][1] + o[1][1][1]),
+              pack_bf16(o[1][0][2] + o[1][1][2], o[1][0][3] + o[1][1][3]));
+  }
+  if (LOSS) {
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
       float l0 = p[nt][0] * p[nt][0] + p[nt][2] * p[nt][2];
@@ -228,14 +230,181 @@ __device__ __forceinline__ void step16(float (&acc)[8][4], uint32_t kbase, uint3
       if (g == 0) *reinterpret_cast<float2*>(&lossp[r0 + 8 * nt + 2 * q]) = make_float2(l0, l1);
     }
   }
-  if (has_q) {
-    stsm_x4_t(obase + rofs + f.o, pack_bf16(o[0][0][0] + o[0][1][0], o[0][0][1] + o[0][1][1]),
-              pack_bf16(o[0][0][2] + o[0][1][2], o[0][0][3] + o[0][1][3]),
-              pack_bf16(o[1][0][0] + o[1][1][0], o[1][0][1] + o[1][1][1]),
-              pack_bf16(o[1][0][2] + o[1][1][2], o[1][0][3] + o[1][1][3]));
-  }
 }
 
+// ---------------------------------------------------------------------------------------------
+// Inner mini-batch b = 16, one CTA per head: four compute warps (sixteen columns each), one
+// TMA producer warp and one writer warp. The compute warps never wait on each other: tiles
+// arrive through full/empty mbarriers, and a finished 64-token tile (outputs in swizzled
+// staging, per-warp loss partials) is handed to the writer through an oready mbarrier; the
+// writer sums the loss partials, issues the TMA store of the outputs and returns the staging
+// buffer through ofree.
+// ---------------------------------------------------------------------------------------------
+
+constexpr int kB16Threads = (kComputeWarps + 2) * 32;
+
+struct __align__(1024) B16Smem {
+  uint8_t K[kStages][kTileBytes];
+  uint8_t V[kStages][kTileBytes];
+  uint8_t Q[kStages][kTileBytes];
+  uint8_t O[2][kTileBytes];
+  float lossp[2][kComputeWarps][kTileTok];
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
+  uint64_t oready[2];
+  uint64_t ofree[2];
+  int abort;  // set by whichever warp's wait ran out; every other wait then returns at once
+};
+
+// Warp-uniform bounded wait: false (with abort set) if the phase did not complete in time.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, int* status, int* abort) {
+  bool ok = mbar_wait(bar, parity, status, abort);
+  ok = __all_sync(0xffffffffu, ok);
+  if (!ok) *reinterpret_cast<volatile int*>(abort) = 1;
+  return ok;
+}
+
+template <bool HAS_Q, bool LOSS>
+__global__ void __launch_bounds__(kB16Threads, 1)
+    k_linear_b16(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                 const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
+                 float* __restrict__ Wstate, float* __restrict__ loss, int T, float beta, int* status) {
+  extern __shared__ uint8_t smem_raw[];
+  B16Smem& sm = *reinterpret_cast<B16Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bh = blockIdx.x;
+  const int ntiles = (T + kTileTok - 1) / kTileTok;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&sm.full[i], 1);
+      mbar_init(&sm.empty[i], kComputeWarps * 32);  // every compute lane arrives
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sm.oready[i], kComputeWarps * 32);
+      mbar_init(&sm.ofree[i], 1);
+    }
+    sm.abort = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  if (warp == kComputeWarps) {
+    // ---------------- producer: TMA loads of K, V (and Q) tiles ----------------
+    if (lane == 0) {
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      if (HAS_Q) tma_prefetch_desc(&tmQ);
+      const uint32_t stage_bytes = (HAS_Q ? 3u : 2u) * kTileBytes;
+      int issued = 0;
+      for (int t = 0; t < ntiles; ++t) {
+        const int slot = t % kStages;
+        if (t >= kStages && !mbar_wait(&sm.empty[slot], ((t / kStages) - 1) & 1, status, &sm.abort)) break;
+        mbar_arrive_expect_tx(&sm.full[slot], stage_bytes);
+        tma_load_3d(sm.K[slot], &tmK, &sm.full[slot], 0, t * kTileTok, bh);
+        tma_load_3d(sm.V[slot], &tmV, &sm.full[slot], 0, t * kTileTok, bh);
+        if (HAS_Q) tma_load_3d(sm.Q[slot], &tmQ, &sm.full[slot], 0, t * kTileTok, bh);
+        issued = t + 1;
+      }
+      // Nothing may still be landing in shared memory when the CTA exits.
+      for (int t = issued - kStages; t < issued; ++t) {
+        if (t < 0) continue;
+        mbar_wait(&sm.full[t % kStages], (t / kStages) & 1, status, nullptr);
+      }
+    }
+    return;
+  }
+
+  if (warp == kComputeWarps + 1) {
+    // ---------------- writer: loss sums and output stores per tile ----------------
+    for (int t = 0; t < ntiles; ++t) {
+      const int b = t & 1;
+      if (!warp_wait(&sm.oready[b], (t >> 1) & 1, status, &sm.abort)) break;
+      if (LOSS) {
+        const int ntok = min(kTileTok, T - t * kTileTok);
+        for (int i = lane; i < ntok; i += 32)
+          loss[(size_t)bh * T + (size_t)t * kTileTok + i] =
+              (sm.lossp[b][0][i] + sm.lossp[b][1][i]) + (sm.lossp[b][2][i] + sm.lossp[b][3][i]);
+      }
+      if (HAS_Q && lane == 0) {
+        tma_store_3d(&tmO, sm.O[b], 0, t * kTileTok, bh);
+        bulk_commit();
+        bulk_wait_read<0>();
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.ofree[b]);
+    }
+    if (HAS_Q && lane == 0) bulk_wait<0>();
+    return;
+  }
+
+  // ---------------- compute warps ----------------
+  const int g = lane >> 2, q = lane & 3;
+  const int col0 = 16 * warp;
+  float* Wg = Wstate + (size_t)bh * 64 * 64;
+  // Wᵀ slice in accumulator layout: acc[nt][e] = W[8nt + 2q + (e&1)][col0 + g + 8(e>>1)].
+  float acc[8][4];
+#pragma unroll
+  for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[nt][e] = Wg[(8 * nt + 2 * q + (e & 1)) * 64 + col0 + g + 8 * (e >> 1)];
+  const StepOffsets offs = step_offsets(lane, col0);
+
+  // Fragments of step s (rows 16s .. 16s+15) of tile t are loaded one step before they are
+  // used. A 64-token tile is four straight-line steps: every wait of the tile sits at its top
+  // and the end-of-tile arrivals are made by all lanes, so the steps themselves contain no
+  // branch (a branch costs a warp its in-flight mma results: measured on B200, a per-step
+  // conditional structure ran 540 cycles a step against 313 for straight-line steps).
+  auto load = [&](Frag16& F, int t, int s) {
+    const int slot = t % kStages;
+    load_frag16<HAS_Q>(F, smem_u32(sm.K[slot]), smem_u32(sm.V[slot]), smem_u32(sm.Q[slot]), offs, 16 * s);
+  };
+  auto comp = [&](const Frag16& F, int t, int s) {
+    compute16<HAS_Q, LOSS>(acc, F, smem_u32(sm.O[t & 1]), offs.o, sm.lossp[t & 1][warp], 16 * s, lane, beta);
+  };
+
+  const int nfull = T / kTileTok, rem = (T % kTileTok) / 16;
+  Frag16 F0, F1;
+  bool ok = ntiles > 0 && warp_wait(&sm.full[0], 0, status, &sm.abort);
+  if (ok) load(F0, 0, 0);
+  int t = 0;
+  for (; ok && t < nfull; ++t) {
+    // The staging buffer of tile t was last used by tile t − 2; tile t+1's inputs are needed
+    // by the last step of this tile.
+    if (t >= 2 && !warp_wait(&sm.ofree[t & 1], ((t >> 1) - 1) & 1, status, &sm.abort)) ok = false;
+    if (ok && t + 1 < ntiles && !warp_wait(&sm.full[(t + 1) % kStages], ((t + 1) / kStages) & 1, status, &sm.abort))
+      ok = false;
+    if (!ok) break;
+    load(F1, t, 1);
+    comp(F0, t, 0);
+    load(F0, t, 2);
+    comp(F1, t, 1);
+    load(F1, t, 3);
+    comp(F0, t, 2);
+    mbar_arrive(&sm.empty[t % kStages]);  // every fragment of tile t has been read
+    load(F0, t + 1, 0);                   // past the last tile this reads a stale slot, unused
+    comp(F1, t, 3);
+    if (HAS_Q) fence_proxy_async_smem();
+    mbar_arrive(&sm.oready[t & 1]);
+  }
+  // A last tile of fewer than 64 tokens (its first fragments are already in F0).
+  if (ok && rem > 0) {
+    if (t < 2 || warp_wait(&sm.ofree[t & 1], ((t >> 1) - 1) & 1, status, &sm.abort)) {
+      comp(F0, t, 0);
+      for (int s = 1; s < rem; ++s) {
+        load(F1, t, s);
+        comp(F1, t, s);
+      }
+      mbar_arrive(&sm.empty[t % kStages]);
+      if (HAS_Q) fence_proxy_async_smem();
+      mbar_arrive(&sm.oready[t & 1]);
+    }
+  }
+#pragma unroll
+  for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) Wg[(8 * nt + 2 * q + (e & 1)) * 64 + col0 + g + 8 * (e >> 1)] = acc[nt][e];
+}
 
 template <int B>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -319,10 +488,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t qbase = smem_u32(sm.Q[slot]);
     uint8_t* obuf = sm.O[s & 1];
 
-    if constexpr (B == 16) {
-      for (int r0 = 0; r0 < ntok; r0 += 16)
-        step16(acc, kbase, vbase, qbase, smem_u32(obuf), offs, sm.lossp[warp], r0, lane, beta, has_q, loss != nullptr);
-    } else {
+    {
       for (int r0 = 0; r0 < ntok; r0 += B) {
         // A fragments of Wᵀ (hi and lo) for the four 16-key k-steps.
         uint32_t whi[4][4], wlo[4][4];
@@ -696,6 +862,26 @@ ttt_status launch(ttt_state* st, const CUtensorMap& tk, const CUtensorMap& tv, c
   return TTT_OK;
 }
 
+template <bool HAS_Q, bool LOSS>
+ttt_status launch_b16_impl(ttt_state* st, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
+                           const CUtensorMap& to, float* loss, int T, cudaStream_t s) {
+  const size_t smem = sizeof(B16Smem) + 1024;
+  TTT_CUDA(cudaFuncSetAttribute(k_linear_b16<HAS_Q, LOSS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  const int grid = st->cfg.batch * st->cfg.heads;
+  const float beta = st->cfg.eta / 16.0f;
+  k_linear_b16<HAS_Q, LOSS><<<grid, kB16Threads, smem, s>>>(tk, tv, tq, to, st->lin.W, loss, T, beta, st->status.dev);
+  st->launches++;
+  TTT_CUDA(cudaGetLastError());
+  return TTT_OK;
+}
+
+ttt_status launch_b16(ttt_state* st, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
+                      const CUtensorMap& to, float* loss, int T, int has_q, cudaStream_t s) {
+  if (has_q) return loss ? launch_b16_impl<true, true>(st, tk, tv, tq, to, loss, T, s)
+                         : launch_b16_impl<true, false>(st, tk, tv, tq, to, loss, T, s);
+  return loss ? launch_b16_impl<false, true>(st, tk, tv, tq, to, loss, T, s)
+              : launch_b16_impl<false, false>(st, tk, tv, tq, to, loss, T, s);
+}
 
 ttt_status launch_n8(ttt_state* st, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
                      const CUtensorMap& to, float* loss, int T, int has_q, cudaStream_t s) {
@@ -739,7 +925,7 @@ ttt_status linear_scan(ttt_state* st, const __nv_bfloat16* K, const __nv_bfloat1
   }
   switch (c.chunk) {
     case 16: return n8 ? launch_n8(st, tk, tv, tq, to, loss, (int)T, has_q, s)
-                       : launch<16>(st, tk, tv, tq, to, loss, (int)T, has_q, s);
+                       : launch_b16(st, tk, tv, tq, to, loss, (int)T, has_q, s);
     case 32: return launch<32>(st, tk, tv, tq, to, loss, (int)T, has_q, s);
     case 64: return launch<64>(st, tk, tv, tq, to, loss, (int)T, has_q, s);
     default: return fail(TTT_ERR_UNSUPPORTED, "TTT-Linear: mini-batch %d not built", c.chunk);

@@ -75,7 +75,9 @@ def test_small_shapes_and_ragged_tiles(cwl, b, T, B, H):
     O, W, L, _ = run_linear(cwl, x, b, 0.5)
     Oref, Wref, Lref = ora.ttt_linear_scan(x["K"].cpu(), x["V"].cpu(), x["Q"].cpu(), W0.cpu(), 0.5, b)
     errs = rel_err(O, Oref), rel_err(W, Wref), rel_err(L, Lref)
-    assert max(errs) <= 5e-3, errs
+    # O is stored in bf16 (rounding up to 2^-9 of an element) and computed from W rounded to
+    # bf16; W and the losses stay far tighter.
+    assert errs[0] <= 1e-2 and max(errs[1:]) <= 5e-3, errs
 
 
 def test_without_queries_same_state_and_loss(cwl):
@@ -122,3 +124,28 @@ def test_rejects_bad_arguments(cwl):
     with pytest.raises(TTTError) as e:
         cwl.FastWeightState(cwl.config("linear", batch=1, heads=2, chunk=24), W0)
     assert e.value.status == abi.TTT_ERR_UNSUPPORTED
+
+
+def test_streaming_paired_kernel_split_at_32(cwl):
+    """B*H = 80 takes the sixteen-columns-per-warp kernel, which processes mini-batches in
+    pairs: calls split at a multiple of 32 tokens reproduce one call bit for bit."""
+    spec = workloads.scaled(workloads.LINEAR_GD, B=1, H=80, T=192, seed=123)
+    x = workloads.linear_inputs(spec, device="cuda")
+    O1, W1, L1, _ = run_linear(cwl, x, 16, 1.0)
+    B, H, T, D = x["K"].shape
+    st = cwl.FastWeightState(cwl.config("linear", batch=B, heads=H, chunk=16, eta=1.0), x["W0"])
+    outs, losses = [], []
+    for a, z in ((0, 96), (96, T)):
+        K, V, Q = (x[n][:, :, a:z].contiguous() for n in ("K", "V", "Q"))
+        O = torch.empty_like(K)
+        L = torch.empty((B, H, z - a), device="cuda")
+        st.chunk_scan(K, V, Q, out=O, loss_out=L)
+        outs.append(O)
+        losses.append(L)
+    W = torch.empty_like(x["W0"])
+    st.get_weights(W)
+    torch.cuda.synchronize()
+    assert torch.equal(torch.cat(outs, 2), O1) and torch.equal(torch.cat(losses, 2), L1)
+    assert torch.equal(W, W1)
+    Oref, Wref, Lref = ora.ttt_linear_scan(x["K"].cpu(), x["V"].cpu(), x["Q"].cpu(), x["W0"].cpu(), 1.0, 16)
+    assert rel_err(O1, Oref) <= 1e-2 and rel_err(W1, Wref) <= 5e-3 and rel_err(L1, Lref) <= 5e-3
