@@ -370,11 +370,21 @@ __global__ void __launch_bounds__(kB16Threads, 1)
   int t = 0;
   for (; ok && t < nfull; ++t) {
     // The staging buffer of tile t was last used by tile t − 2; tile t+1's inputs are needed
-    // by the last step of this tile.
-    if (t >= 2 && !warp_wait(&sm.ofree[t & 1], ((t >> 1) - 1) & 1, status, &sm.abort)) ok = false;
-    if (ok && t + 1 < ntiles && !warp_wait(&sm.full[(t + 1) % kStages], ((t + 1) / kStages) & 1, status, &sm.abort))
-      ok = false;
-    if (!ok) break;
+    // by the last step of this tile. Both are tested without a branch (a phase that has nothing
+    // to wait for is given the parity of its completed predecessor: for t < 2 that is the phase
+    // before a fresh barrier's first, which counts as complete); only if either is still open
+    // does the warp take the bounded waits. A branch here costs the warp its in-flight mma
+    // results, so there is one per tile (a two-tile loop body measured slower: its code no
+    // longer fits the instruction cache).
+    const int t1 = t + 1;
+    const uint32_t pfree = ((t >> 1) + 1) & 1;
+    const uint32_t pfull = ((t1 / kStages) + (t1 < ntiles ? 0 : 1)) & 1;
+    const bool ready = mbar_try_wait(&sm.ofree[t & 1], pfree) & mbar_try_wait(&sm.full[t1 % kStages], pfull);
+    if (!__all_sync(0xffffffffu, ready)) {
+      ok = warp_wait(&sm.ofree[t & 1], pfree, status, &sm.abort) &&
+           warp_wait(&sm.full[t1 % kStages], pfull, status, &sm.abort);
+      if (!ok) break;
+    }
     load(F1, t, 1);
     comp(F0, t, 0);
     load(F0, t, 2);
