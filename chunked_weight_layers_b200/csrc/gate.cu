@@ -12,12 +12,15 @@
 // until it holds `capacity` entries; later routed tokens are counted as dropped.
 //
 // Only τ is sequential across chunks, so the kernel splits the work by dependency:
-//   1. every warp selects p95 and sums S for its chunks in parallel (a stable rank of each
-//      of the 64 values, two per lane, by 64 shuffled comparisons);
+//   1. every warp takes p95 and S of its chunks (chunk_stats: counting selection and an
+//      exactness-checked tree sum);
 //   2. one thread runs the scalar τ recurrence over the block of chunks;
 //   3. all threads flag routed tokens and compact them in order with a block-wide scan.
 // One CTA per (sequence, head); losses are processed in blocks of 64 chunks (4096 tokens).
+// This kernel serves the standalone routing call; the b = 16 TTT-Linear scan runs the same
+// gate in its writer warp, tile by tile.
 #include "common.cuh"
+#include "gate_chunk.cuh"
 #include "internal.h"
 
 namespace ttt {
@@ -30,7 +33,7 @@ constexpr int kBlockChunks = 64;
 constexpr int kBlockTok = kChunk * kBlockChunks;
 constexpr int kTokPerThread = kBlockTok / kGateThreads;  // 16
 
-struct GateSmem {
+struct __align__(16) GateSmem {
   float x[kBlockTok];
   double S[kBlockChunks];
   float p[kBlockChunks];
@@ -66,29 +69,12 @@ __global__ void __launch_bounds__(kGateThreads)
 
     // 1. percentile and sum of every chunk (warp per chunk).
     for (int g = warp; g < nch; g += kGateThreads / 32) {
-      const float v0 = sm.x[g * kChunk + lane];
-      const float v1 = sm.x[g * kChunk + 32 + lane];
-      int r0 = 0, r1 = 0;  // stable ranks of v0 (index lane) and v1 (index lane + 32)
-      for (int j = 0; j < 32; ++j) {
-        const float u0 = __shfl_sync(0xffffffffu, v0, j);  // index j
-        const float u1 = __shfl_sync(0xffffffffu, v1, j);  // index j + 32
-        r0 += (u0 < v0) || (u0 == v0 && j < lane);
-        r0 += (u1 < v0);
-        r1 += (u0 < v1) || (u0 == v1);
-        r1 += (u1 < v1) || (u1 == v1 && j < lane);
-      }
-      const unsigned m0 = __ballot_sync(0xffffffffu, r0 == rank - 1);
-      const unsigned m1 = __ballot_sync(0xffffffffu, r1 == rank - 1);
       float pv;
-      if (m0 != 0u)
-        pv = __shfl_sync(0xffffffffu, v0, __ffs(m0) - 1);
-      else
-        pv = __shfl_sync(0xffffffffu, v1, __ffs(m1) - 1);
+      double S;
+      chunk_stats(&sm.x[g * kChunk], lane, rank, pv, S);
       if (lane == 0) {
-        double S = 0.0;
-        for (int j = 0; j < kChunk; ++j) S += (double)sm.x[g * kChunk + j];
-        sm.S[g] = S;
         sm.p[g] = pv;
+        sm.S[g] = S;
       }
     }
     __syncthreads();
@@ -98,7 +84,7 @@ __global__ void __launch_bounds__(kGateThreads)
       float tau = sm.tau_carry;
       int set = sm.tau_set;
       for (int g = 0; g < nch; ++g) {
-        tau = set ? __fadd_rn(__fmul_rn(ema_old, tau), __fmul_rn(ema_new, sm.p[g])) : sm.p[g];
+        tau = tau_next(tau, set, sm.p[g], ema_old, ema_new);
         set = 1;
         sm.tau[g] = tau;
         sm.pass[g] = lhs_scale * sm.S[g] >= rhs_scale * (double)tau;
@@ -160,14 +146,19 @@ __global__ void __launch_bounds__(kGateThreads)
 
 }  // namespace
 
-ttt_status gate_route(ttt_state* st, const float* loss, int64_t T, cudaStream_t s) {
-  const ttt_config& c = st->cfg;
+int gate_rank(const ttt_config& c) {
   // Nearest rank ceil(pct·n), computed in double like the definition.
   const double x = (double)c.gate_pct * kChunk;
   int rank = (int)x;
   if ((double)rank < x - 1e-9) ++rank;
   if (rank < 1) rank = 1;
   if (rank > kChunk) rank = kChunk;
+  return rank;
+}
+
+ttt_status gate_route(ttt_state* st, const float* loss, int64_t T, cudaStream_t s) {
+  const ttt_config& c = st->cfg;
+  const int rank = gate_rank(c);
   const double lhs = (double)c.gate_mean_den;
   const double rhs = (double)c.gate_mean_num * kChunk;
   k_gate<<<c.batch * c.heads, kGateThreads, 0, s>>>(loss, (int)T, c.heads, rank, c.gate_ema_old, c.gate_ema_new, lhs,

@@ -105,6 +105,8 @@ ttt_status linear_scan(ttt_state* st, const __nv_bfloat16* K, const __nv_bfloat1
 
 // Surprisal gate over T losses of every (sequence, head).
 ttt_status gate_route(ttt_state* st, const float* loss, int64_t T, cudaStream_t s);
+// Nearest rank ceil(gate_pct·64) of the gate's percentile (1-based).
+int gate_rank(const ttt_config& c);
 
 // Small utility kernels.
 ttt_status f32_to_bf16(const float* src, __nv_bfloat16* dst, size_t n, cudaStream_t s,

@@ -6,18 +6,15 @@
 // Design (B200):
 //  * the per-head state is 64x64 fp32 and never leaves the SM: it lives in mma accumulator
 //    registers. Column c of W only ever depends on column c of R (R[:, c] = K·W[:, c] − V[:, c]),
-//    so columns are split across warps (and, for b = 16, a head's two column halves across
-//    two CTAs) with no communication inside a step.
+//    so columns are split across warps with no communication inside a step.
 //  * k_linear_b16 (b = 16, one CTA per head): four compute warps own sixteen columns each and
 //    compute every product transposed, so each accumulator layout is directly the next mma's A
 //    operand. Operand fragments are loaded one step ahead; a 64-token tile is four
 //    straight-line steps with all waits at its top. A TMA producer warp fills the K/V/Q ring
 //    and a writer warp sums loss partials and stores the output tiles, so compute warps never
-//    meet at a barrier.
-//  * k_linear_n8 (b = 16 when 2·B·H ≤ SM count): two CTAs per head, four warps per CTA, eight
-//    columns per warp, products in their natural orientation with movmatrix.trans turning
-//    accumulators into B operands; partial losses of the two halves are added into a zeroed
-//    output.
+//    meet at a barrier. Measured on B200 it is faster than splitting a head's columns over two
+//    CTAs (eight columns per warp, movmatrix for the B operands) even when SMs are idle: 104
+//    against 173 us for B=4 x H=16 x T=8192, 32 against 41 us for a single head.
 //  * k_linear_scan (b = 32 or 64): one CTA per head, sixteen columns per warp, W and the update
 //    operand fed to the tensor cores as bf16 hi + lo pairs.
 //  * for b = 16 the tensor cores see W rounded to bf16 each step and the update operand
@@ -31,6 +28,7 @@
 //    dependent 16x64x64 product costs more than the product itself. Measured on B200:
 //    mma.sync m16n8k16 latency ~21 cycles, at most one per ~8.2 cycles per SM sub-partition.
 #include "common.cuh"
+#include "gate_chunk.cuh"
 #include "internal.h"
 
 namespace ttt {
@@ -241,7 +239,10 @@ __device__ __forceinline__ void compute16(float (&acc)[8][4], const Frag16& F, u
 // buffer through ofree.
 // ---------------------------------------------------------------------------------------------
 
-constexpr int kB16Threads = (kComputeWarps + 2) * 32;
+constexpr int kGateWarps = 2;  // alternate tiles: each has two tiles' time for one chunk's statistics
+constexpr int kGateRing = 4;   // tiles of losses in flight from the writer to the gate warps
+template <bool GATE>
+constexpr int b16_threads() { return (kComputeWarps + 2 + (GATE ? kGateWarps : 0)) * 32; }
 
 struct __align__(1024) B16Smem {
   uint8_t K[kStages][kTileBytes];
@@ -249,11 +250,32 @@ struct __align__(1024) B16Smem {
   uint8_t Q[kStages][kTileBytes];
   uint8_t O[2][kTileBytes];
   float lossp[2][kComputeWarps][kTileTok];
+  float gl[kGateRing][kTileTok];  // tiles' losses handed from the writer to the gate warps
   uint64_t full[kStages];
   uint64_t empty[kStages];
   uint64_t oready[2];
   uint64_t ofree[2];
+  uint64_t gready[kGateRing];
+  uint64_t gfree[kGateRing];
   int abort;  // set by whichever warp's wait ran out; every other wait then returns at once
+  // The gate's sequential state, passed between the gate warps in tile order: gate_turn is the
+  // tile whose threshold update and routing may run next.
+  float g_tau;
+  int g_tau_set;
+  int g_routed;
+  int gate_turn;
+};
+
+// The surprisal gate's state and constants for the scan that runs it in its own warps.
+struct GateArgs {
+  float* tau;         // [B·H] threshold carried between calls
+  int32_t* tau_set;   // [B·H] whether τ has been set since reset
+  int32_t* entries;   // [B·H, capacity, 3] (sequence, head, token) of routed tokens
+  int32_t* counts;    // [B·H, 2] routed since reset, dropped because the cache was full
+  int capacity, rank, heads;
+  float ema_old, ema_new;
+  double lhs, rhs;    // pass ⇔ lhs·S ≥ rhs·τ
+  int64_t t_offset;   // tokens gated since reset before this call
 };
 
 // Warp-uniform bounded wait: false (with abort set) if the phase did not complete in time.
@@ -264,11 +286,30 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, int* s
   return ok;
 }
 
-template <bool HAS_Q, bool LOSS>
-__global__ void __launch_bounds__(kB16Threads, 1)
+// Bounded wait until *turn == want (a shared-memory counter advanced by another warp).
+__device__ __forceinline__ bool wait_turn(const int* turn, int want, int* status, int* abort) {
+  const volatile int* tv = turn;
+  const volatile int* av = abort;
+  if (*tv == want) return true;
+  const uint64_t t0 = globaltimer();
+  while (*tv != want) {
+    if (*av) return false;
+    if (globaltimer() - t0 > kWaitBudgetNs) {
+      record_status(status, kDevTimeout);
+      *const_cast<volatile int*>(av) = 1;
+      return false;
+    }
+  }
+  return true;
+}
+
+template <bool HAS_Q, bool LOSS, bool GATE>
+__global__ void __launch_bounds__(b16_threads<true>(), 1)
     k_linear_b16(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                  const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
-                 float* __restrict__ Wstate, float* __restrict__ loss, int T, float beta, int* status) {
+                 float* __restrict__ Wstate, float* __restrict__ loss, int T, float beta, int* status,
+                 const GateArgs ga) {
+  static_assert(!GATE || LOSS, "the gate reads the losses");
   extern __shared__ uint8_t smem_raw[];
   B16Smem& sm = *reinterpret_cast<B16Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -284,7 +325,17 @@ __global__ void __launch_bounds__(kB16Threads, 1)
       mbar_init(&sm.oready[i], kComputeWarps * 32);
       mbar_init(&sm.ofree[i], 1);
     }
+    for (int i = 0; i < kGateRing; ++i) {
+      mbar_init(&sm.gready[i], 1);
+      mbar_init(&sm.gfree[i], 1);
+    }
     sm.abort = 0;
+    if (GATE) {
+      sm.g_tau = ga.tau[bh];
+      sm.g_tau_set = ga.tau_set[bh];
+      sm.g_routed = ga.counts[2 * bh];
+      sm.gate_turn = 0;
+    }
     fence_barrier_init();
   }
   __syncthreads();
@@ -316,15 +367,23 @@ __global__ void __launch_bounds__(kB16Threads, 1)
   }
 
   if (warp == kComputeWarps + 1) {
-    // ---------------- writer: loss sums and output stores per tile ----------------
+    // ---------------- writer: losses and output stores per tile ----------------
     for (int t = 0; t < ntiles; ++t) {
       const int b = t & 1;
       if (!warp_wait(&sm.oready[b], (t >> 1) & 1, status, &sm.abort)) break;
+      float v0 = 0.f, v1 = 0.f;  // losses of tokens lane and lane + 32 of the tile
       if (LOSS) {
         const int ntok = min(kTileTok, T - t * kTileTok);
-        for (int i = lane; i < ntok; i += 32)
-          loss[(size_t)bh * T + (size_t)t * kTileTok + i] =
-              (sm.lossp[b][0][i] + sm.lossp[b][1][i]) + (sm.lossp[b][2][i] + sm.lossp[b][3][i]);
+        float* Lt = loss + (size_t)bh * T + (size_t)t * kTileTok;
+        if (lane < ntok) {
+          v0 = (sm.lossp[b][0][lane] + sm.lossp[b][1][lane]) + (sm.lossp[b][2][lane] + sm.lossp[b][3][lane]);
+          Lt[lane] = v0;
+        }
+        if (lane + 32 < ntok) {
+          const int i = lane + 32;
+          v1 = (sm.lossp[b][0][i] + sm.lossp[b][1][i]) + (sm.lossp[b][2][i] + sm.lossp[b][3][i]);
+          Lt[i] = v1;
+        }
       }
       if (HAS_Q && lane == 0) {
         tma_store_3d(&tmO, sm.O[b], 0, t * kTileTok, bh);
@@ -333,8 +392,80 @@ __global__ void __launch_bounds__(kB16Threads, 1)
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.ofree[b]);
+      if (GATE) {
+        // Hand the tile's losses to the gate warps (slot t % kGateRing, last read for tile
+        // t − kGateRing; a fresh barrier's phase before its first counts as complete).
+        const int r = t % kGateRing;
+        if (!warp_wait(&sm.gfree[r], ((t / kGateRing) + 1) & 1, status, &sm.abort)) break;
+        sm.gl[r][lane] = v0;
+        sm.gl[r][lane + 32] = v1;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.gready[r]);
+      }
     }
     if (HAS_Q && lane == 0) bulk_wait<0>();
+    return;
+  }
+
+  if (GATE && warp >= kComputeWarps + 2) {
+    // ---------------- gate warps: the surprisal gate, one 64-token chunk per tile ----------------
+    // With the gate on T is a multiple of 64, so every tile is one gate chunk. Gate warp w takes
+    // the tiles t ≡ w (mod kGateWarps): the chunk's percentile and sum are independent of the
+    // other chunks; the threshold update and the routing then run in tile order, passed from
+    // warp to warp through gate_turn.
+    const int w = warp - (kComputeWarps + 2);
+    const int seq = bh / ga.heads, head = bh % ga.heads;
+    int32_t* E = ga.entries + (size_t)bh * ga.capacity * 3;
+    for (int t = w; t < ntiles; t += kGateWarps) {
+      const int r = t % kGateRing;
+      if (!warp_wait(&sm.gready[r], (t / kGateRing) & 1, status, &sm.abort)) break;
+      const float v0 = sm.gl[r][lane], v1 = sm.gl[r][lane + 32];
+      float p;
+      double S;
+      chunk_stats(sm.gl[r], lane, ga.rank, p, S);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.gfree[r]);
+      if (!__all_sync(0xffffffffu, wait_turn(&sm.gate_turn, t, status, &sm.abort))) break;
+      __threadfence_block();
+      float tau = *reinterpret_cast<volatile float*>(&sm.g_tau);
+      const bool set = *reinterpret_cast<volatile int*>(&sm.g_tau_set) != 0;
+      const int routed = *reinterpret_cast<volatile int*>(&sm.g_routed);
+      tau = tau_next(tau, set, p, ga.ema_old, ga.ema_new);
+      const bool pass = ga.lhs * S >= ga.rhs * (double)tau;
+      const bool f0 = pass && v0 > tau, f1 = pass && v1 > tau;
+      const unsigned m0 = __ballot_sync(0xffffffffu, f0), m1 = __ballot_sync(0xffffffffu, f1);
+      const unsigned below = (1u << lane) - 1u;
+      const int pos0 = routed + __popc(m0 & below), pos1 = routed + __popc(m0) + __popc(m1 & below);
+      const int tok = (int)(ga.t_offset + (int64_t)t * kTileTok) + lane;
+      if (f0 && pos0 < ga.capacity) {
+        E[3 * pos0 + 0] = seq;
+        E[3 * pos0 + 1] = head;
+        E[3 * pos0 + 2] = tok;
+      }
+      if (f1 && pos1 < ga.capacity) {
+        E[3 * pos1 + 0] = seq;
+        E[3 * pos1 + 1] = head;
+        E[3 * pos1 + 2] = tok + 32;
+      }
+      __syncwarp();
+      if (lane == 0) {
+        *reinterpret_cast<volatile float*>(&sm.g_tau) = tau;
+        *reinterpret_cast<volatile int*>(&sm.g_tau_set) = 1;
+        *reinterpret_cast<volatile int*>(&sm.g_routed) = routed + __popc(m0) + __popc(m1);
+        __threadfence_block();
+        *reinterpret_cast<volatile int*>(&sm.gate_turn) = t + 1;
+      }
+    }
+    // The warp that ran the last tile writes the state back.
+    if (ntiles > 0 && w == (ntiles - 1) % kGateWarps && lane == 0 &&
+        *reinterpret_cast<volatile int*>(&sm.gate_turn) == ntiles) {
+      __threadfence_block();
+      const int routed = sm.g_routed;
+      ga.tau[bh] = sm.g_tau;
+      ga.tau_set[bh] = sm.g_tau_set;
+      ga.counts[2 * bh + 0] = routed;
+      ga.counts[2 * bh + 1] = routed > ga.capacity ? routed - ga.capacity : 0;
+    }
     return;
   }
 
@@ -637,228 +768,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 
-// ---------------------------------------------------------------------------------------------
-// Inner mini-batch b = 16, eight columns per warp, each head split over two CTAs.
-//
-// Column c of W only depends on column c of R, so a head's 64 columns are split into two
-// halves on two CTAs (no communication) and each of a CTA's four warps owns 8 columns. The
-// products run in their natural orientation (m16n8k16 with N = 8 columns):
-//   P = K·W (A = K from ldmatrix, B = W from the accumulator via movmatrix.trans),
-//   R = P − V, loss, S = −(η/b)·R,
-//   W += Kᵀ·S (A = Kᵀ from ldmatrix.trans, B = S via movmatrix.trans),  O = Q·W.
-// Half the instructions per warp and step of the 16-columns-per-warp form, and the heads
-// reach every SM. The per-token loss is the sum of the two halves' partial sums: each CTA
-// adds its partial to a zeroed output (two terms onto zero: the result does not depend on
-// their order).
-// ---------------------------------------------------------------------------------------------
-
-struct N8Offsets {
-  uint32_t ka[4];  // K (or Q) A fragments: [16-key k-step]
-  uint32_t kt[4];  // Kᵀ A fragments of the update: [16-key m-tile]
-  uint32_t v;      // V fragment of this warp's 8 columns
-  uint32_t o;      // output staging rows (64-byte rows, 64-byte swizzle)
-};
-
-__device__ __forceinline__ N8Offsets n8_offsets(int lane, int vcol, int w) {
-  const int mi = lane >> 3, ri = lane & 7;
-  N8Offsets f;
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    f.ka[k] = swz128_bf16(8 * (mi & 1) + ri, 16 * k + 8 * (mi >> 1));
-    f.kt[k] = swz128_bf16(8 * (mi >> 1) + ri, 16 * k + 8 * (mi & 1));
-  }
-  f.v = swz128_bf16(8 * (mi & 1) + ri, vcol);
-  const int orow = 8 * (mi & 1) + ri;
-  f.o = (uint32_t)(orow * 64 + ((w ^ ((orow >> 1) & 3)) << 4));
-  return f;
-}
-
-__device__ __forceinline__ uint32_t movm_t(uint32_t a) {
-  uint32_t d;
-  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(a));
-  return d;
-}
-
-__device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t& r0, uint32_t& r1) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(addr));
-}
-
-__device__ __forceinline__ void stsm_x2(uint32_t addr, uint32_t r0, uint32_t r1) {
-  asm volatile("stmatrix.sync.aligned.m8n8.x2.shared.b16 [%0], {%1, %2};" ::"r"(addr), "r"(r0), "r"(r1) : "memory");
-}
-
-__device__ __forceinline__ void mma_n8(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-// acc[mt][e] = W[16mt + g + 8(e>>1)][col0 + 2q + (e&1)] for this warp's 8 columns.
-__device__ __forceinline__ void step16_n8(float (&acc)[4][4], uint32_t kbase, uint32_t vbase, uint32_t qbase,
-                                          uint32_t obase, const N8Offsets& f, float* lossp, int r0, int lane,
-                                          float beta, int has_q, bool want_loss) {
-  const int g = lane >> 2;
-  const uint32_t rofs = (uint32_t)r0 * 128u;
-  uint32_t ka[4][4], kt[4][4], qa[4][4], v0, v1;
-#pragma unroll
-  for (int k = 0; k < 4; ++k) ldsm_x4(kbase + rofs + f.ka[k], ka[k]);
-  ldsm_x2(vbase + rofs + f.v, v0, v1);
-#pragma unroll
-  for (int k = 0; k < 4; ++k) ldsm_x4_t(kbase + rofs + f.kt[k], kt[k]);
-  if (has_q) {
-#pragma unroll
-    for (int k = 0; k < 4; ++k) ldsm_x4(qbase + rofs + f.ka[k], qa[k]);
-  }
-  // W as B fragments: movmatrix.trans turns the accumulator layout (key rows, column pairs)
-  // into (key pairs, column) per 8x8 block.
-  uint32_t wb[4][2];
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    wb[k][0] = movm_t(pack_bf16(acc[k][0], acc[k][1]));
-    wb[k][1] = movm_t(pack_bf16(acc[k][2], acc[k][3]));
-  }
-  float pa[4] = {0.f, 0.f, 0.f, 0.f}, pb[4] = {0.f, 0.f, 0.f, 0.f}, o[4] = {0.f, 0.f, 0.f, 0.f};
-  mma_n8(pa, ka[0], wb[0][0], wb[0][1]);
-  mma_n8(pb, ka[1], wb[1][0], wb[1][1]);
-  mma_n8(pa, ka[2], wb[2][0], wb[2][1]);
-  mma_n8(pb, ka[3], wb[3][0], wb[3][1]);
-  if (has_q) {
-#pragma unroll
-    for (int k = 0; k < 4; ++k) mma_n8(o, qa[k], wb[k][0], wb[k][1]);
-  }
-  // R = P − V: p[e] = R[token g + 8(e>>1)][column 2q + (e&1)].
-  const float2 va = unpack_bf16(v0), vb = unpack_bf16(v1);
-  float p[4];
-  p[0] = (pa[0] + pb[0]) - va.x;
-  p[1] = (pa[1] + pb[1]) - va.y;
-  p[2] = (pa[2] + pb[2]) - vb.x;
-  p[3] = (pa[3] + pb[3]) - vb.y;
-  // S = −(η/b)·R as B fragments (token pairs, column).
-  const uint32_t sb0 = movm_t(pack_bf16(-beta * p[0], -beta * p[1]));
-  const uint32_t sb1 = movm_t(pack_bf16(-beta * p[2], -beta * p[3]));
-#pragma unroll
-  for (int k = 0; k < 4; ++k) mma_n8(acc[k], kt[k], sb0, sb1);
-
-  if (want_loss) {
-    float l0 = p[0] * p[0] + p[1] * p[1];
-    float l1 = p[2] * p[2] + p[3] * p[3];
-    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-    if ((lane & 3) == 0) {
-      lossp[r0 + g] = l0;
-      lossp[r0 + g + 8] = l1;
-    }
-  }
-  if (has_q) stsm_x2(obase + (uint32_t)r0 * 64u + f.o, pack_bf16(o[0], o[1]), pack_bf16(o[2], o[3]));
-}
-
-struct __align__(1024) N8Smem {
-  uint8_t K[kStages][kTileBytes];
-  uint8_t V[kStages][kTileBytes];
-  uint8_t Q[kStages][kTileBytes];
-  uint8_t O[2][kTileTok * 64];  // this CTA's 32 output columns of a tile (64-byte swizzle)
-  float lossp[kComputeWarps][kTileTok];
-  uint64_t full[kStages];
-  uint64_t empty[kStages];
-  int abort;
-  int cabort[2];
-};
-
-__global__ void __launch_bounds__(kThreads, 1)
-    k_linear_n8(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
-                float* __restrict__ Wstate, float* __restrict__ loss, int T, float beta, int has_q, int* status) {
-  extern __shared__ uint8_t smem_raw[];
-  N8Smem& sm = *reinterpret_cast<N8Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bh = blockIdx.x >> 1, half = blockIdx.x & 1;
-  const int nstages = (T + kTileTok - 1) / kTileTok;
-  const uint32_t stage_bytes = (has_q ? 3u : 2u) * kTileBytes;
-
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < kStages; ++i) {
-      mbar_init(&sm.full[i], 1);
-      mbar_init(&sm.empty[i], kComputeWarps);
-    }
-    sm.abort = 0;
-    sm.cabort[0] = sm.cabort[1] = 0;
-    fence_barrier_init();
-  }
-  __syncthreads();
-
-  if (warp == kComputeWarps) {
-    if (lane == 0) {
-      tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
-      if (has_q) tma_prefetch_desc(&tmQ);
-      int issued = 0;
-      for (int s = 0; s < nstages; ++s) {
-        const int slot = s % kStages;
-        if (s >= kStages && !mbar_wait(&sm.empty[slot], ((s / kStages) - 1) & 1, status, &sm.abort)) break;
-        mbar_arrive_expect_tx(&sm.full[slot], stage_bytes);
-        tma_load_3d(sm.K[slot], &tmK, &sm.full[slot], 0, s * kTileTok, bh);
-        tma_load_3d(sm.V[slot], &tmV, &sm.full[slot], 0, s * kTileTok, bh);
-        if (has_q) tma_load_3d(sm.Q[slot], &tmQ, &sm.full[slot], 0, s * kTileTok, bh);
-        issued = s + 1;
-      }
-      for (int s = issued - kStages; s < issued; ++s) {
-        if (s < 0) continue;
-        mbar_wait(&sm.full[s % kStages], (s / kStages) & 1, status, nullptr);
-      }
-    }
-    __syncthreads();
-    return;
-  }
-
-  const int g = lane >> 2, q = lane & 3;
-  const int col0 = 32 * half + 8 * warp;  // first W column owned by this warp
-  float* Wg = Wstate + (size_t)bh * 64 * 64;
-  float acc[4][4];
-#pragma unroll
-  for (int mt = 0; mt < 4; ++mt)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) acc[mt][e] = Wg[(16 * mt + g + 8 * (e >> 1)) * 64 + col0 + 2 * q + (e & 1)];
-  const N8Offsets offs = n8_offsets(lane, col0, warp);
-
-  for (int s = 0; s < nstages; ++s) {
-    const int slot = s % kStages;
-    // Every compute warp takes the same exit decision (see k_linear_scan).
-    if (!mbar_wait(&sm.full[slot], (s / kStages) & 1, status, nullptr)) sm.cabort[s & 1] = 1;
-    named_sync();
-    if (*reinterpret_cast<volatile int*>(&sm.cabort[s & 1])) break;
-    const int ntok = min(kTileTok, T - s * kTileTok);
-    const uint32_t kbase = smem_u32(sm.K[slot]), vbase = smem_u32(sm.V[slot]), qbase = smem_u32(sm.Q[slot]);
-    uint8_t* obuf = sm.O[s & 1];
-    for (int r0 = 0; r0 < ntok; r0 += 16)
-      step16_n8(acc, kbase, vbase, qbase, smem_u32(obuf), offs, sm.lossp[warp], r0, lane, beta, has_q,
-                loss != nullptr);
-    if (has_q) fence_proxy_async_smem();
-    named_sync();
-    if (loss != nullptr && warp == 0) {
-      for (int i = lane; i < ntok; i += 32) {
-        const float l = (sm.lossp[0][i] + sm.lossp[1][i]) + (sm.lossp[2][i] + sm.lossp[3][i]);
-        atomicAdd(&loss[(size_t)bh * T + (size_t)s * kTileTok + i], l);
-      }
-    }
-    if (threadIdx.x == 0 && has_q) {
-      tma_store_3d(&tmO, obuf, 32 * half, s * kTileTok, bh);
-      bulk_commit();
-      bulk_wait_read<1>();
-    }
-    named_sync();
-    if (lane == 0) mbar_arrive(&sm.empty[slot]);
-  }
-  if (threadIdx.x == 0 && has_q) bulk_wait<0>();
-#pragma unroll
-  for (int mt = 0; mt < 4; ++mt)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) Wg[(16 * mt + g + 8 * (e >> 1)) * 64 + col0 + 2 * q + (e & 1)] = acc[mt][e];
-  __syncthreads();
-}
-
 template <int B>
 ttt_status launch(ttt_state* st, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
                   const CUtensorMap& to, float* loss, int T, int has_q, cudaStream_t s) {
@@ -872,14 +781,16 @@ ttt_status launch(ttt_state* st, const CUtensorMap& tk, const CUtensorMap& tv, c
   return TTT_OK;
 }
 
-template <bool HAS_Q, bool LOSS>
+template <bool HAS_Q, bool LOSS, bool GATE>
 ttt_status launch_b16_impl(ttt_state* st, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
-                           const CUtensorMap& to, float* loss, int T, cudaStream_t s) {
+                           const CUtensorMap& to, float* loss, int T, const GateArgs& ga, cudaStream_t s) {
   const size_t smem = sizeof(B16Smem) + 1024;
-  TTT_CUDA(cudaFuncSetAttribute(k_linear_b16<HAS_Q, LOSS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  TTT_CUDA(cudaFuncSetAttribute(k_linear_b16<HAS_Q, LOSS, GATE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)smem));
   const int grid = st->cfg.batch * st->cfg.heads;
   const float beta = st->cfg.eta / 16.0f;
-  k_linear_b16<HAS_Q, LOSS><<<grid, kB16Threads, smem, s>>>(tk, tv, tq, to, st->lin.W, loss, T, beta, st->status.dev);
+  k_linear_b16<HAS_Q, LOSS, GATE>
+      <<<grid, b16_threads<GATE>(), smem, s>>>(tk, tv, tq, to, st->lin.W, loss, T, beta, st->status.dev, ga);
   st->launches++;
   TTT_CUDA(cudaGetLastError());
   return TTT_OK;
@@ -887,24 +798,24 @@ ttt_status launch_b16_impl(ttt_state* st, const CUtensorMap& tk, const CUtensorM
 
 ttt_status launch_b16(ttt_state* st, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
                       const CUtensorMap& to, float* loss, int T, int has_q, cudaStream_t s) {
-  if (has_q) return loss ? launch_b16_impl<true, true>(st, tk, tv, tq, to, loss, T, s)
-                         : launch_b16_impl<true, false>(st, tk, tv, tq, to, loss, T, s);
-  return loss ? launch_b16_impl<false, true>(st, tk, tv, tq, to, loss, T, s)
-              : launch_b16_impl<false, false>(st, tk, tv, tq, to, loss, T, s);
+  const ttt_config& c = st->cfg;
+  GateArgs ga{};
+  if (c.gate_enable) {
+    ga = GateArgs{st->gate.tau, st->gate.tau_set, st->gate.entries, st->gate.counts, c.cache_capacity,
+                  gate_rank(c), c.heads, c.gate_ema_old, c.gate_ema_new, (double)c.gate_mean_den,
+                  (double)c.gate_mean_num * kTileTok, st->gate.t_offset};
+    const ttt_status r = has_q ? launch_b16_impl<true, true, true>(st, tk, tv, tq, to, loss, T, ga, s)
+                               : launch_b16_impl<false, true, true>(st, tk, tv, tq, to, loss, T, ga, s);
+    if (r != TTT_OK) return r;
+    st->gate.t_offset += T;
+    return TTT_OK;
+  }
+  if (has_q) return loss ? launch_b16_impl<true, true, false>(st, tk, tv, tq, to, loss, T, ga, s)
+                         : launch_b16_impl<true, false, false>(st, tk, tv, tq, to, loss, T, ga, s);
+  return loss ? launch_b16_impl<false, true, false>(st, tk, tv, tq, to, loss, T, ga, s)
+              : launch_b16_impl<false, false, false>(st, tk, tv, tq, to, loss, T, ga, s);
 }
 
-ttt_status launch_n8(ttt_state* st, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
-                     const CUtensorMap& to, float* loss, int T, int has_q, cudaStream_t s) {
-  const size_t smem = sizeof(N8Smem) + 1024;
-  TTT_CUDA(cudaFuncSetAttribute(k_linear_n8, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-  const int bh = st->cfg.batch * st->cfg.heads;
-  if (loss != nullptr) TTT_CUDA(cudaMemsetAsync(loss, 0, (size_t)bh * T * sizeof(float), s));
-  const float beta = st->cfg.eta / 16.0f;
-  k_linear_n8<<<2 * bh, kThreads, smem, s>>>(tk, tv, tq, to, st->lin.W, loss, T, beta, has_q, st->status.dev);
-  st->launches++;
-  TTT_CUDA(cudaGetLastError());
-  return TTT_OK;
-}
 }  // namespace
 
 ttt_status linear_scan(ttt_state* st, const __nv_bfloat16* K, const __nv_bfloat16* V, const __nv_bfloat16* Q,
@@ -915,27 +826,18 @@ ttt_status linear_scan(ttt_state* st, const __nv_bfloat16* K, const __nv_bfloat1
   const uint64_t strides[2] = {128, (uint64_t)T * 128};
   const uint32_t box[3] = {64, (uint32_t)kTileTok, 1};
   CUtensorMap tk, tv, tq, to;
-  // b = 16: eight columns per warp on two CTAs per head when every half-head gets its own SM;
-  // otherwise sixteen columns per warp on one CTA per head (fewer, fuller SMs win then).
-  const bool n8 = c.chunk == 16 && 2 * (int64_t)c.batch * c.heads <= st->num_sms;
   TTT_TRY(encode_tmap(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, K, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B));
   TTT_TRY(encode_tmap(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, V, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B));
   const int has_q = Q != nullptr;
   if (has_q) {
     TTT_TRY(encode_tmap(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, Q, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B));
-    if (n8) {
-      const uint32_t obox[3] = {32, (uint32_t)kTileTok, 1};
-      TTT_TRY(encode_tmap(&to, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, O, dims, strides, obox, CU_TENSOR_MAP_SWIZZLE_64B));
-    } else {
-      TTT_TRY(encode_tmap(&to, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, O, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B));
-    }
+    TTT_TRY(encode_tmap(&to, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, O, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B));
   } else {
     tq = tk;
     to = tk;
   }
   switch (c.chunk) {
-    case 16: return n8 ? launch_n8(st, tk, tv, tq, to, loss, (int)T, has_q, s)
-                       : launch_b16(st, tk, tv, tq, to, loss, (int)T, has_q, s);
+    case 16: return launch_b16(st, tk, tv, tq, to, loss, (int)T, has_q, s);
     case 32: return launch<32>(st, tk, tv, tq, to, loss, (int)T, has_q, s);
     case 64: return launch<64>(st, tk, tv, tq, to, loss, (int)T, has_q, s);
     default: return fail(TTT_ERR_UNSUPPORTED, "TTT-Linear: mini-batch %d not built", c.chunk);

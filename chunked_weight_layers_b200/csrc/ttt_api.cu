@@ -277,7 +277,9 @@ static ttt_status scan_impl(ttt_state* st, const void* keys, const void* targets
   }
   TTT_TRY(linear_scan(st, static_cast<const __nv_bfloat16*>(keys), static_cast<const __nv_bfloat16*>(targets),
                       static_cast<const __nv_bfloat16*>(queries), T, static_cast<__nv_bfloat16*>(out), loss, s));
-  if (c.gate_enable) TTT_TRY(gate_route(st, loss, T, s));
+  // The b = 16 scan runs the gate itself, tile by tile; the other mini-batch sizes hand the
+  // losses to the standalone gate kernel.
+  if (c.gate_enable && c.chunk != 16) TTT_TRY(gate_route(st, loss, T, s));
   return TTT_OK;
 }
 

@@ -65,8 +65,8 @@ def test_identity_fixed_point_is_exact(cwl):
 @pytest.mark.parametrize("b,T,B,H", [(16, 208, 2, 3), (32, 224, 2, 3), (64, 192, 2, 3), (16, 64, 2, 3),
                                      (16, 208, 1, 80)])
 def test_small_shapes_and_ragged_tiles(cwl, b, T, B, H):
-    """B*H = 6 takes the eight-columns-per-warp kernel at b = 16; B*H = 80 (160 half-heads,
-    more than the 148 SMs) takes the sixteen-columns-per-warp one."""
+    """Ragged last tiles (T = 208 and 224 are not multiples of the 64-token tile), each inner
+    mini-batch size, and more heads than fit one wave at a time."""
     spec = workloads.scaled(workloads.LINEAR_GD, B=B, H=H, T=T, b=b, seed=77 + b + H)
     x = workloads.linear_inputs(spec, device="cuda")
     W0 = x["W0"].clone()
@@ -126,16 +126,17 @@ def test_rejects_bad_arguments(cwl):
     assert e.value.status == abi.TTT_ERR_UNSUPPORTED
 
 
-def test_streaming_paired_kernel_split_at_32(cwl):
-    """B*H = 80 takes the sixteen-columns-per-warp kernel, which processes mini-batches in
-    pairs: calls split at a multiple of 32 tokens reproduce one call bit for bit."""
-    spec = workloads.scaled(workloads.LINEAR_GD, B=1, H=80, T=192, seed=123)
+def test_streaming_split_inside_tiles(cwl):
+    """Calls split at 48 and 176 tokens (inside 64-token tiles, so each call has a ragged last
+    tile and the next starts a fresh tile mid-sequence) reproduce one call bit for bit: every
+    16-token step runs the same arithmetic wherever the tile boundaries fall."""
+    spec = workloads.scaled(workloads.LINEAR_GD, B=1, H=80, T=256, seed=123)
     x = workloads.linear_inputs(spec, device="cuda")
     O1, W1, L1, _ = run_linear(cwl, x, 16, 1.0)
     B, H, T, D = x["K"].shape
     st = cwl.FastWeightState(cwl.config("linear", batch=B, heads=H, chunk=16, eta=1.0), x["W0"])
     outs, losses = [], []
-    for a, z in ((0, 96), (96, T)):
+    for a, z in ((0, 48), (48, 176), (176, T)):
         K, V, Q = (x[n][:, :, a:z].contiguous() for n in ("K", "V", "Q"))
         O = torch.empty_like(K)
         L = torch.empty((B, H, z - a), device="cuda")
