@@ -226,7 +226,7 @@ class ClockSampler:
 
 def dominant_kernel(spec) -> str:
     if isinstance(spec, wl.LinearSpec):
-        return "k_linear_scan"
+        return "k_linear_b16" if spec.b == 16 else "k_linear_scan"
     return "k_sgemm" if spec.dtype == "f32" else "k_inplace_tc"
 
 
