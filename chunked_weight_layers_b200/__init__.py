@@ -20,17 +20,31 @@ __all__ = ["FastWeightState", "TTTError", "config", "abi"]
 def _ptr(t) -> int | None:
     if t is None:
         return None
-    if not t.is_cuda:
-        raise ValueError("expected a CUDA tensor")
-    if not t.is_contiguous():
-        raise ValueError("expected a contiguous tensor")
+    if not (t.is_cuda and t.is_contiguous()):
+        raise ValueError("expected a contiguous CUDA tensor")
     return t.data_ptr()
 
 
-def _stream(stream) -> int | None:
+def _current_raw_stream():
+    """A function returning torch's current CUDA stream handle of the current device: torch's
+    direct accessor when present (a fraction of a microsecond a call), else the public API."""
     import torch
+    raw = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+    cur_dev = getattr(torch._C, "_cuda_getDevice", None)
+    if raw is not None and cur_dev is not None:
+        return lambda: raw(cur_dev())
+    return lambda: torch.cuda.current_stream().cuda_stream
+
+
+_raw_stream = None
+
+
+def _stream(stream) -> int | None:
+    global _raw_stream
     if stream is None:
-        stream = torch.cuda.current_stream()
+        if _raw_stream is None:
+            _raw_stream = _current_raw_stream()
+        return _raw_stream() or None
     return stream.cuda_stream or None
 
 

@@ -52,6 +52,13 @@ struct InplaceBuffers {
 struct LinearBuffers {
   float* W = nullptr;   // [B, H, D, D]
   float* W0 = nullptr;  // [B, H, D, D]
+  // Tensor maps of the last scan's K, V, Q, O (re-encoded only when a pointer or T changes:
+  // encoding costs microseconds of host time per call) and the kernels whose shared-memory
+  // size has been raised for this state's device.
+  const void* map_key[4] = {nullptr, nullptr, nullptr, nullptr};
+  int64_t map_T = -1;
+  CUtensorMap maps[4];
+  uint32_t smem_set = 0;
 };
 
 struct GateBuffers {

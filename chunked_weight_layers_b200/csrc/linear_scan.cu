@@ -772,7 +772,11 @@ template <int B>
 ttt_status launch(ttt_state* st, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
                   const CUtensorMap& to, float* loss, int T, int has_q, cudaStream_t s) {
   const size_t smem = sizeof(LinearSmem) + 1024;
-  TTT_CUDA(cudaFuncSetAttribute(k_linear_scan<B>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  const uint32_t bit = 1u << (8 + B / 32);
+  if (!(st->lin.smem_set & bit)) {
+    TTT_CUDA(cudaFuncSetAttribute(k_linear_scan<B>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    st->lin.smem_set |= bit;
+  }
   const int grid = st->cfg.batch * st->cfg.heads;
   const float beta = st->cfg.eta / (float)B;
   k_linear_scan<B><<<grid, kThreads, smem, s>>>(tk, tv, tq, to, st->lin.W, loss, T, beta, has_q, st->status.dev);
@@ -785,8 +789,12 @@ template <bool HAS_Q, bool LOSS, bool GATE>
 ttt_status launch_b16_impl(ttt_state* st, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
                            const CUtensorMap& to, float* loss, int T, const GateArgs& ga, cudaStream_t s) {
   const size_t smem = sizeof(B16Smem) + 1024;
-  TTT_CUDA(cudaFuncSetAttribute(k_linear_b16<HAS_Q, LOSS, GATE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)smem));
+  const uint32_t bit = 1u << (4 * GATE + 2 * HAS_Q + LOSS);
+  if (!(st->lin.smem_set & bit)) {
+    TTT_CUDA(cudaFuncSetAttribute(k_linear_b16<HAS_Q, LOSS, GATE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)smem));
+    st->lin.smem_set |= bit;
+  }
   const int grid = st->cfg.batch * st->cfg.heads;
   const float beta = st->cfg.eta / 16.0f;
   k_linear_b16<HAS_Q, LOSS, GATE>
@@ -825,17 +833,25 @@ ttt_status linear_scan(ttt_state* st, const __nv_bfloat16* K, const __nv_bfloat1
   const uint64_t dims[3] = {64, (uint64_t)T, BH};
   const uint64_t strides[2] = {128, (uint64_t)T * 128};
   const uint32_t box[3] = {64, (uint32_t)kTileTok, 1};
-  CUtensorMap tk, tv, tq, to;
-  TTT_TRY(encode_tmap(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, K, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B));
-  TTT_TRY(encode_tmap(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, V, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B));
-  const int has_q = Q != nullptr;
-  if (has_q) {
-    TTT_TRY(encode_tmap(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, Q, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B));
-    TTT_TRY(encode_tmap(&to, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, O, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B));
-  } else {
-    tq = tk;
-    to = tk;
+  LinearBuffers& lb = st->lin;
+  const bool has_q = Q != nullptr;
+  const void* key[4] = {K, V, Q, O};
+  if (lb.map_T != T || lb.map_key[0] != key[0] || lb.map_key[1] != key[1] || lb.map_key[2] != key[2] ||
+      lb.map_key[3] != key[3]) {
+    lb.map_T = -1;  // invalid until all four are encoded
+    TTT_TRY(encode_tmap(&lb.maps[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, K, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B));
+    TTT_TRY(encode_tmap(&lb.maps[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, V, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B));
+    if (has_q) {
+      TTT_TRY(encode_tmap(&lb.maps[2], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, Q, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B));
+      TTT_TRY(encode_tmap(&lb.maps[3], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, O, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B));
+    } else {
+      lb.maps[2] = lb.maps[0];
+      lb.maps[3] = lb.maps[0];
+    }
+    for (int i = 0; i < 4; ++i) lb.map_key[i] = key[i];
+    lb.map_T = T;
   }
+  const CUtensorMap &tk = lb.maps[0], &tv = lb.maps[1], &tq = lb.maps[2], &to = lb.maps[3];
   switch (c.chunk) {
     case 16: return launch_b16(st, tk, tv, tq, to, loss, (int)T, has_q, s);
     case 32: return launch<32>(st, tk, tv, tq, to, loss, (int)T, has_q, s);

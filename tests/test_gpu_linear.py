@@ -150,3 +150,18 @@ def test_streaming_split_inside_tiles(cwl):
     assert torch.equal(W, W1)
     Oref, Wref, Lref = ora.ttt_linear_scan(x["K"].cpu(), x["V"].cpu(), x["Q"].cpu(), x["W0"].cpu(), 1.0, 16)
     assert rel_err(O1, Oref) <= 1e-2 and rel_err(W1, Wref) <= 5e-3 and rel_err(L1, Lref) <= 5e-3
+
+
+@pytest.mark.parametrize("T,B,H", [(16, 1, 3), (48, 2, 2), (112, 1, 1), (1024, 2, 160)])
+def test_edge_lengths_and_more_heads_than_sms(cwl, T, B, H):
+    """One 16-token step, a single ragged tile (48 tokens), a full tile plus a ragged one
+    (112), and 320 heads (more CTAs than SMs: they run in waves): each against the oracle,
+    with and without queries, and the loss."""
+    spec = workloads.scaled(workloads.LINEAR_GD, B=B, H=H, T=T, seed=500 + T + H)
+    x = workloads.linear_inputs(spec, device="cuda")
+    O, W, L, _ = run_linear(cwl, x, 16, 1.0)
+    Oref, Wref, Lref = ora.ttt_linear_scan(x["K"].cpu(), x["V"].cpu(), x["Q"].cpu(), x["W0"].cpu(), 1.0, 16)
+    errs = rel_err(O, Oref), rel_err(W, Wref), rel_err(L, Lref)
+    assert errs[0] <= 1e-2 and max(errs[1:]) <= 5e-3, errs
+    _, W2, L2, _ = run_linear(cwl, x, 16, 1.0, with_q=False)
+    assert torch.equal(W2, W) and torch.equal(L2, L)
