@@ -487,6 +487,14 @@ Plan make_plan(int num_sms, int d, int f, int C, bool apply_update, bool target)
     per[best].push_back(t.code);
     load[best] += t.cost;
   }
+  // Within each CTA, UPDATE tiles first and the long APPLY/TARGET tile last: the launch then
+  // ends on an epilogue that only stores outputs rather than on a W read-modify-write, and
+  // the CTAs holding an APPLY tile stream W while the others do too (measured on B200:
+  // 3.59 against 3.68 ms on the T=32768 workload).
+  for (auto& v : per)
+    std::stable_sort(v.begin(), v.end(), [](int32_t a, int32_t b) {
+      return (((a >> 28) & 3) == UPDATE) > (((b >> 28) & 3) == UPDATE);
+    });
   Plan p;
   p.grid = grid;
   p.host.resize(grid + 1);
