@@ -50,6 +50,7 @@ constexpr int kEpiWarps = 8;
 constexpr int kWarpWload = 2 + kEpiWarps;   // the warp that streams W sub-tiles in
 constexpr int kThreadsTC = (3 + kEpiWarps) * 32;
 constexpr int kTmemCols = 512;
+constexpr int kRotate = 61;                 // list rotation between rounds (coprime to 148)
 
 enum : int { APPLY = 0, UPDATE = 1, TARGET = 2 };
 
@@ -82,6 +83,18 @@ struct TCArgs {
   __nv_bfloat16* O;            // outputs [T, d]
   __nv_bfloat16* Vhat_out;     // targets of target_chunk [C, d]
   int* status;
+  // Several chunks in one launch: every CTA runs its tile list once per chunk (chunk index
+  // chunk + r in round r). The bf16 copy of W rotates through three buffers: round r applies
+  // with buffer (cur0 + r) % 3 and its UPDATE tiles write buffer (cur0 + r + 1) % 3, the one
+  // round r − 2 applied with. upd_done[r·nbd + b] / app_done[r·nbd + b] count the finished
+  // UPDATE / APPLY work of round r on 256-row block b of W; an APPLY tile of round r waits for
+  // round r − 1's UPDATE tiles of its block, an UPDATE tile of round r for round r − 2's APPLY
+  // tiles of its block. Null counters: one round, no waits.
+  int rounds;
+  int cur0;
+  int nbd;
+  int* upd_done;
+  int* app_done;
 };
 
 // ---- tcgen05 wrappers -----------------------------------------------------------------
@@ -155,22 +168,73 @@ __device__ __forceinline__ void store_row_bf16(__nv_bfloat16* row, int col0, int
   }
 }
 
+__device__ __forceinline__ const CUtensorMap* pick3(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& c,
+                                                    int i) {
+  return i == 0 ? &a : (i == 1 ? &b : &c);
+}
+
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Bounded wait until *ctr ≥ want (a counter other CTAs raise); then the async proxy (TMA) may
+// read what they published.
+__device__ __forceinline__ bool wait_counter(const int* ctr, int want, int* status, volatile int* abort) {
+  const volatile int* c = ctr;
+  if (*c < want) {
+    const uint64_t t0 = globaltimer();
+    while (*c < want) {
+      if (*abort) return false;
+      if (globaltimer() - t0 > kWaitBudgetNs) {
+        record_status(status, kDevTimeout);
+        *abort = 1;
+        return false;
+      }
+      __nanosleep(128);
+    }
+  }
+  __threadfence();
+  fence_proxy_async_global();
+  return true;
+}
+
+// Work expected on 256-row block b of W per round: UPDATE halves (two 128-row tiles per block,
+// fewer at the edge, times the f tiles, two column halves each) and APPLY tiles (C/128).
+__device__ __forceinline__ int upd_expect(const TCArgs& a, int b) {
+  const int mt = (a.d + BM - 1) / BM, nf = (a.f + BN - 1) / BN;
+  return (min(2 * b + 2, mt) - 2 * b) * nf * 2;
+}
+
 __device__ __forceinline__ void named_sync_half(int half) {
   asm volatile("bar.sync %0, %1;" ::"r"(1 + half), "n"(4 * 32) : "memory");
 }
 
 __global__ void __launch_bounds__(kThreadsTC, 1)
     k_inplace_tc(const __grid_constant__ CUtensorMap tmZk, const __grid_constant__ CUtensorMap tmZm,
-                 const __grid_constant__ CUtensorMap tmVm, const __grid_constant__ CUtensorMap tmWk,
+                 const __grid_constant__ CUtensorMap tmVm, const __grid_constant__ CUtensorMap tmWk0,
+                 const __grid_constant__ CUtensorMap tmWk1, const __grid_constant__ CUtensorMap tmWk2,
                  const __grid_constant__ CUtensorMap tmConv, const __grid_constant__ CUtensorMap tmWt,
-                 const __grid_constant__ CUtensorMap tmWf, const __grid_constant__ CUtensorMap tmWs,
+                 const __grid_constant__ CUtensorMap tmWf, const __grid_constant__ CUtensorMap tmWs0,
+                 const __grid_constant__ CUtensorMap tmWs1, const __grid_constant__ CUtensorMap tmWs2,
                  const TCArgs args) {
   extern __shared__ uint8_t smem_raw[];
   TCSmem& sm = *reinterpret_cast<TCSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int32_t* tiles = args.sched + gridDim.x + 1;
-  const int t_begin = args.sched[blockIdx.x];
-  const int t_end = args.sched[blockIdx.x + 1];
+  // In round r the CTA runs tile list (blockIdx.x + r·kRotate) mod gridDim.x: over the rounds
+  // every CTA works through a mix of the lists, so their different loads even out instead of
+  // adding up round after round.
+  auto list_of = [&](int rnd) { return (int)(((long)blockIdx.x + (long)rnd * kRotate) % gridDim.x); };
+  int ntot = 0;  // tiles of this CTA over all rounds
+  for (int rnd = 0; rnd < args.rounds; ++rnd) ntot += args.sched[list_of(rnd) + 1] - args.sched[list_of(rnd)];
+  // Walks the CTA's tiles in order: calls f(round, tile code) until it returns false.
+  auto for_tiles = [&](auto&& f) {
+    for (int rnd = 0; rnd < args.rounds; ++rnd) {
+      const int li = list_of(rnd);
+      for (int ti = args.sched[li]; ti < args.sched[li + 1]; ++ti)
+        if (!f(rnd, tiles[ti])) return;
+    }
+  };
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kSt; ++i) {
@@ -207,31 +271,42 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       tma_prefetch_desc(&tmZk);
       tma_prefetch_desc(&tmZm);
       tma_prefetch_desc(&tmVm);
-      tma_prefetch_desc(&tmWk);
+      tma_prefetch_desc(&tmWk0);
       uint32_t it = 0;
-      for (int ti = t_begin; ti < t_end && !*abort; ++ti) {
-        const int32_t tc = tiles[ti];
+      for_tiles([&](int rnd, int32_t tc) -> bool {
+        if (*abort) return false;
         const int type = tile_type(tc), m = tile_m(tc), n = tile_n(tc);
         const int nk = kblocks(type, args);
+        const int chunk = args.chunk + rnd;
+        const CUtensorMap* wk = pick3(tmWk0, tmWk1, tmWk2, (args.cur0 + rnd) % 3);
+        if (args.upd_done != nullptr) {
+          if (type == APPLY && rnd >= 1 &&
+              !wait_counter(&args.upd_done[(rnd - 1) * args.nbd + n], upd_expect(args, n), args.status, abort))
+            return false;
+          if (type == UPDATE && rnd >= 2 &&
+              !wait_counter(&args.app_done[(rnd - 2) * args.nbd + m / 2], args.C / BM, args.status, abort))
+            return false;
+        }
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const int s = it % kSt;
-          if (it >= kSt && !mbar_wait(&sm.empty[s], ((it / kSt) - 1) & 1, args.status, abort)) break;
+          if (it >= kSt && !mbar_wait(&sm.empty[s], ((it / kSt) - 1) & 1, args.status, abort)) return false;
           mbar_arrive_expect_tx(&sm.full[s], kABytes + kBBytes);
           if (type == APPLY) {
-            tma_load_2d(sm.A[s], &tmZk, &sm.full[s], kb * BK, args.chunk * args.C + m * BM);
-            tma_load_2d(sm.B[s], &tmWk, &sm.full[s], kb * BK, n * BN);
+            tma_load_2d(sm.A[s], &tmZk, &sm.full[s], kb * BK, chunk * args.C + m * BM);
+            tma_load_2d(sm.B[s], wk, &sm.full[s], kb * BK, n * BN);
           } else if (type == UPDATE) {
             for (int j = 0; j < BM / 64; ++j)
-              tma_load_2d(sm.A[s] + j * 8192, &tmVm, &sm.full[s], m * BM + j * 64, args.vrow0 + kb * BK);
+              tma_load_2d(sm.A[s] + j * 8192, &tmVm, &sm.full[s], m * BM + j * 64, args.vrow0 + rnd * args.C + kb * BK);
             for (int j = 0; j < BN / 64; ++j)
-              tma_load_2d(sm.B[s] + j * 8192, &tmZm, &sm.full[s], n * BN + j * 64, args.chunk * args.C + kb * BK);
+              tma_load_2d(sm.B[s] + j * 8192, &tmZm, &sm.full[s], n * BN + j * 64, chunk * args.C + kb * BK);
           } else {
-            tma_load_2d(sm.A[s], &tmConv, &sm.full[s], kb * BK, args.target_chunk * args.C + m * BM);
+            tma_load_2d(sm.A[s], &tmConv, &sm.full[s], kb * BK, (args.target_chunk + rnd) * args.C + m * BM);
             for (int j = 0; j < BN / 64; ++j)
               tma_load_2d(sm.B[s] + j * 8192, &tmWt, &sm.full[s], n * BN + j * 64, kb * BK);
           }
         }
-      }
+        return true;
+      });
       // Drain: the newest phase issued on every stage must have landed before exit.
       for (uint32_t k = (it > (uint32_t)kSt ? it - kSt : 0); k < it; ++k)
         mbar_wait(&sm.full[k % kSt], (k / kSt) & 1, args.status, nullptr);
@@ -241,10 +316,14 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     if (lane == 0) {
       tma_prefetch_desc(&tmWf);
       uint32_t e = 0;
-      for (int ti = t_begin; ti < t_end && !*abort; ++ti) {
-        const int32_t tc = tiles[ti];
-        if (tile_type(tc) != UPDATE) continue;
+      for_tiles([&](int rnd, int32_t tc) -> bool {
+        if (*abort) return false;
+        if (tile_type(tc) != UPDATE) return true;
         const int m = tile_m(tc), n = tile_n(tc);
+        // The round before updated this W tile, possibly on another CTA.
+        if (args.upd_done != nullptr && rnd >= 1 &&
+            !wait_counter(&args.upd_done[(rnd - 1) * args.nbd + m / 2], upd_expect(args, m / 2), args.status, abort))
+          return false;
         bool ok = true;
         for (int k = 0; k < BN / kWCols; ++k, ++e) {
           const int s = e % kWSlots;
@@ -255,8 +334,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           mbar_arrive_expect_tx(&sm.wfull[s], kWBytes);
           tma_load_2d(sm.Wr[s], &tmWf, &sm.wfull[s], n * BN + (k & 1) * 128 + (k >> 1) * kWCols, m * BM);
         }
-        if (!ok) break;
-      }
+        return ok;
+      });
       for (uint32_t k = (e > (uint32_t)kWSlots ? e - kWSlots : 0); k < e; ++k)
         mbar_wait(&sm.wfull[k % kWSlots], (k / kWSlots) & 1, args.status, nullptr);
     }
@@ -265,14 +344,13 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     if (lane == 0) {
       uint32_t it = 0, tcount = 0;
       bool ok = true;
-      for (int ti = t_begin; ti < t_end && ok; ++ti, ++tcount) {
-        const int32_t tc = tiles[ti];
+      for_tiles([&](int, int32_t tc) -> bool {
         const int type = tile_type(tc);
         const int nk = kblocks(type, args);
         const int acc = tcount & 1;
         if (tcount >= 2 && !mbar_wait(&sm.tempty[acc], ((tcount >> 1) - 1) & 1, args.status, abort)) {
           ok = false;
-          break;
+          return false;
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem + (uint32_t)(acc * BN);
@@ -299,14 +377,16 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           }
           umma_commit(&sm.empty[s]);  // frees the stage once these MMAs have read it
         }
-        if (!ok) break;
+        if (!ok) return false;
         umma_commit(&sm.tfull[acc]);  // accumulator ready for the epilogue
-      }
+        ++tcount;
+        return true;
+      });
       // Drain: the last commit covers every MMA issued before it; wait for it before TMEM
       // is freed. After a clean run that is the last accumulator's commit, after an abort
       // the last stage-release commit.
-      if (ok && t_end > t_begin) {
-        const uint32_t last = (uint32_t)(t_end - t_begin - 1);
+      if (ok && ntot > 0) {
+        const uint32_t last = (uint32_t)(ntot - 1);
         mbar_wait(&sm.tfull[last & 1], (last >> 1) & 1, args.status, nullptr);
       } else if (!ok && it > 0) {
         mbar_wait(&sm.empty[(it - 1) % kSt], ((it - 1) / kSt) & 1, args.status, nullptr);
@@ -320,9 +400,9 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     uint32_t tcount = 0, ecount = 0;      // tiles seen; W sub-tiles consumed by this half
     const int row_in_tile = lq * 32 + lane;
     bool stop = false;
-    for (int ti = t_begin; ti < t_end && !stop; ++ti, ++tcount) {
-      const int32_t tc = tiles[ti];
+    for_tiles([&](int rnd, int32_t tc) -> bool {
       const int type = tile_type(tc), m = tile_m(tc), n = tile_n(tc);
+      const CUtensorMap* ws = pick3(tmWs0, tmWs1, tmWs2, (args.cur0 + rnd + 1) % 3);
       const int acc = tcount & 1;
       bool ok = mbar_wait(&sm.tfull[acc], (tcount >> 1) & 1, args.status, nullptr);
       ok = __all_sync(0xffffffffu, ok);
@@ -330,8 +410,14 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       // flag of tile t is written only before this barrier and read only after it.
       if (!ok && lane == 0) sm.tflag[half][tcount & 1] = 1;
       named_sync_half(half);
-      if (*reinterpret_cast<volatile int*>(&sm.tflag[half][tcount & 1])) break;
+      if (*reinterpret_cast<volatile int*>(&sm.tflag[half][tcount & 1])) return false;
       tc_fence_after();
+      // The accumulator is complete, so every operand of this tile has been read: an APPLY
+      // tile no longer needs its buffer of the bf16 copy of W.
+      if (type == APPLY && args.app_done != nullptr && warp == 2 && lane == 0) {
+        __threadfence();
+        atomicAdd(&args.app_done[rnd * args.nbd + n], 1);
+      }
       const uint32_t tbase = tmem + ((uint32_t)(lq * 32) << 16) + (uint32_t)(acc * BN + half * 128);
       if (type == UPDATE) {
         // W sub-tiles arrive in smem by TMA; W ← W + η·ΔW in place, the bf16 copy beside it,
@@ -385,14 +471,21 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           if (leader) {
             const int col = n * BN + half * 128 + j * kWCols;
             tma_store_2d(&tmWf, sm.Wr[slot], col, m * BM);
-            tma_store_2d(&tmWs, sm.Sh[half], col, m * BM);
+            tma_store_2d(ws, sm.Sh[half], col, m * BM);
             bulk_commit();
             bulk_wait_read<0>();          // both stores have read shared memory
             mbar_arrive(&sm.wempty[slot]);
           }
           named_sync_half(half);          // the bf16 staging tile is free again
         }
-        if (stop) break;
+        if (stop) return false;
+        // The stores of this half of the tile complete, then later rounds may read them.
+        if (leader && args.upd_done != nullptr) {
+          bulk_wait<0>();
+          fence_proxy_async_global();
+          __threadfence();
+          atomicAdd(&args.upd_done[rnd * args.nbd + m / 2], 1);
+        }
       } else {
         const int row = m * BM + row_in_tile;  // token within the chunk
 #pragma unroll 1
@@ -405,7 +498,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
           if (type == APPLY)
-            store_row_bf16(args.O + ((size_t)args.chunk * args.C + row) * args.d, col0, args.d, v);
+            store_row_bf16(args.O + ((size_t)(args.chunk + rnd) * args.C + row) * args.d, col0, args.d, v);
           else
             store_row_bf16(args.Vhat_out + (size_t)row * args.d, col0, args.d, v);
         }
@@ -413,7 +506,9 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.tempty[acc]);
-    }
+      ++tcount;
+      return true;
+    });
     if (leader) bulk_wait<0>();
   }
 
@@ -533,6 +628,8 @@ struct TCResources {
   int grid[3] = {0, 0, 0};
   __nv_bfloat16* conv = nullptr;
   size_t conv_rows = 0;
+  int* counters = nullptr;  // per-round progress counters of a multi-chunk launch
+  size_t counters_n = 0;
 };
 
 static ttt_status ensure_tc(ttt_state* st) {
@@ -568,6 +665,7 @@ void free_tc(ttt_state* st) {
   for (int i = 0; i < 3; ++i)
     if (r->plan_dev[i]) cudaFree(r->plan_dev[i]);
   if (r->conv) cudaFree(r->conv);
+  if (r->counters) cudaFree(r->counters);
   delete r;
   st->ip.tc = nullptr;
 }
@@ -581,14 +679,14 @@ ttt_status inplace_bf16_scan(ttt_state* st, const __nv_bfloat16* Z, const __nv_b
   TCResources* r = st->ip.tc;
   const int nchunks = (int)(T / C);
 
-  CUtensorMap tmZk, tmZm, tmVm_in, tmVm_buf[2], tmWk[2], tmConv, tmWt, tmWf, tmWs[2];
+  CUtensorMap tmZk, tmZm, tmVm_in, tmVm_buf[2], tmWk[3], tmConv, tmWt, tmWf, tmWs[3];
   TTT_TRY(map2d(&tmWf, st->ip.W, f, d, kWCols, BM, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, CU_TENSOR_MAP_SWIZZLE_128B));
-  TTT_TRY(map2d(&tmWs[0], st->ip.Wsh[0], f, d, kWCols, BM, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, CU_TENSOR_MAP_SWIZZLE_64B));
-  TTT_TRY(map2d(&tmWs[1], st->ip.Wsh[1], f, d, kWCols, BM, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, CU_TENSOR_MAP_SWIZZLE_64B));
+  for (int i = 0; i < 3; ++i) {
+    TTT_TRY(map2d(&tmWs[i], st->ip.Wsh[i], f, d, kWCols, BM, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, CU_TENSOR_MAP_SWIZZLE_64B));
+    TTT_TRY(map2d(&tmWk[i], st->ip.Wsh[i], f, d, BK, BN));
+  }
   TTT_TRY(map2d(&tmZk, Z, f, T, BK, BM));
   TTT_TRY(map2d(&tmZm, Z, f, T, 64, BK));
-  TTT_TRY(map2d(&tmWk[0], st->ip.Wsh[0], f, d, BK, BN));
-  TTT_TRY(map2d(&tmWk[1], st->ip.Wsh[1], f, d, BK, BN));
   if (target) {
     if (r->conv_rows < (size_t)T) {
       if (r->conv) cudaFree(r->conv);
@@ -615,7 +713,7 @@ ttt_status inplace_bf16_scan(ttt_state* st, const __nv_bfloat16* Z, const __nv_b
   const size_t smem = sizeof(TCSmem) + 1024;
   TTT_CUDA(cudaFuncSetAttribute(k_inplace_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
 
-  auto launch = [&](int plan, int chunk, int tchunk) -> ttt_status {
+  auto args_for = [&](int plan, int chunk, int tchunk, int rounds, int* counters) {
     TCArgs a;
     a.sched = r->plan_dev[plan];
     a.chunk = chunk;
@@ -628,20 +726,51 @@ ttt_status inplace_bf16_scan(ttt_state* st, const __nv_bfloat16* Z, const __nv_b
     a.O = O;
     a.Vhat_out = target ? st->ip.Vhat[tchunk & 1] : nullptr;
     a.status = st->status.dev;
-    const CUtensorMap& vm = target ? tmVm_buf[chunk & 1] : tmVm_in;
-    k_inplace_tc<<<r->grid[plan], kThreadsTC, smem, s>>>(tmZk, tmZm, vm, tmWk[st->ip.cur], tmConv, tmWt, tmWf,
-                                                         tmWs[st->ip.cur ^ 1], a);
+    a.rounds = rounds;
+    a.cur0 = st->ip.cur;
+    a.nbd = (d + BN - 1) / BN;
+    a.upd_done = counters;
+    a.app_done = counters ? counters + (size_t)rounds * a.nbd : nullptr;
+    return a;
+  };
+  auto launch = [&](int plan, const TCArgs& a, const CUtensorMap& vm) -> ttt_status {
+    k_inplace_tc<<<r->grid[plan], kThreadsTC, smem, s>>>(tmZk, tmZm, vm, tmWk[0], tmWk[1], tmWk[2], tmConv, tmWt,
+                                                         tmWf, tmWs[0], tmWs[1], tmWs[2], a);
     st->launches++;
     TTT_CUDA(cudaGetLastError());
     return TTT_OK;
   };
 
-  if (target) TTT_TRY(launch(1, 0, 0));  // targets of chunk 0
+  if (!target) {
+    // All chunks in one launch: each CTA runs its tile list once per chunk, waiting on
+    // progress counters only where a chunk needs another CTA's result of an earlier chunk,
+    // so a chunk's last tiles overlap the next chunk's first. The grid is one CTA per SM and
+    // is launched cooperatively, which guarantees that every CTA is resident.
+    const size_t need = 2 * (size_t)nchunks * ((d + BN - 1) / BN);
+    if (r->counters_n < need) {
+      if (r->counters) cudaFree(r->counters);
+      r->counters = nullptr;
+      r->counters_n = 0;
+      TTT_CUDA(cudaMalloc(reinterpret_cast<void**>(&r->counters), need * sizeof(int)));
+      r->counters_n = need;
+    }
+    TTT_CUDA(cudaMemsetAsync(r->counters, 0, need * sizeof(int), s));
+    TCArgs a = args_for(0, 0, 1, nchunks, r->counters);
+    void* params[] = {&tmZk, &tmZm, &tmVm_in, &tmWk[0], &tmWk[1], &tmWk[2], &tmConv, &tmWt, &tmWf,
+                      &tmWs[0], &tmWs[1], &tmWs[2], &a};
+    TTT_CUDA(cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(k_inplace_tc), dim3(r->grid[0]),
+                                         dim3(kThreadsTC), params, smem, s));
+    st->launches++;
+    st->ip.cur = (st->ip.cur + nchunks) % 3;
+    return TTT_OK;
+  }
+
+  TTT_TRY(launch(1, args_for(1, 0, 0, 1, nullptr), tmVm_buf[0]));  // targets of chunk 0
   for (int ch = 0; ch < nchunks; ++ch) {
     const bool last = ch + 1 == nchunks;
-    const int plan = target ? (last ? 2 : 0) : 0;
-    TTT_TRY(launch(plan, ch, ch + 1));
-    st->ip.cur ^= 1;  // the bf16 copy written by this launch holds W_{c+1}
+    const int plan = last ? 2 : 0;
+    TTT_TRY(launch(plan, args_for(plan, ch, ch + 1, 1, nullptr), tmVm_buf[ch & 1]));
+    st->ip.cur = (st->ip.cur + 1) % 3;  // the bf16 copy written by this launch holds W_{c+1}
   }
   return TTT_OK;
 }
@@ -696,9 +825,15 @@ ttt_status target_values_into(const __nv_bfloat16* X0, const float* convw, const
   a.O = nullptr;
   a.Vhat_out = out;
   a.status = nullptr;
+  a.rounds = 1;
+  a.cur0 = 0;
+  a.nbd = 0;
+  a.upd_done = nullptr;
+  a.app_done = nullptr;
   const size_t smem = sizeof(TCSmem) + 1024;
   TTT_CUDA(cudaFuncSetAttribute(k_inplace_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-  k_inplace_tc<<<grid, kThreadsTC, smem, s>>>(tmConv, tmConv, tmConv, tmConv, tmConv, tmWt, tmConv, tmConv, a);
+  k_inplace_tc<<<grid, kThreadsTC, smem, s>>>(tmConv, tmConv, tmConv, tmConv, tmConv, tmConv, tmConv, tmWt, tmConv,
+                                              tmConv, tmConv, tmConv, a);
   TTT_CUDA(cudaGetLastError());
   return TTT_OK;
 }

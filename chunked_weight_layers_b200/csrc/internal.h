@@ -41,7 +41,10 @@ struct StatusWord {
 struct InplaceBuffers {
   float* W = nullptr;            // fp32 master [d, f]
   float* W0 = nullptr;           // pretrained copy [d, f]
-  __nv_bfloat16* Wsh[2] = {nullptr, nullptr};  // bf16 copies of W for the apply (BF16 path)
+  // bf16 copies of W for the apply (BF16 path): chunk c applies with one while its update
+  // writes the next; three so that an update never overwrites the copy that the chunk
+  // before is still applying with when chunks overlap in one launch.
+  __nv_bfloat16* Wsh[3] = {nullptr, nullptr, nullptr};
   int cur = 0;                   // index of the bf16 copy that holds the current W
   __nv_bfloat16* Wtarget = nullptr;  // [d, d]
   float* convw = nullptr;        // [d, taps]

@@ -106,6 +106,7 @@ static void free_state(ttt_state* st) {
   dev_free(st->ip.W0);
   dev_free(st->ip.Wsh[0]);
   dev_free(st->ip.Wsh[1]);
+  dev_free(st->ip.Wsh[2]);
   dev_free(st->ip.Wtarget);
   dev_free(st->ip.convw);
   free_tc(st);
@@ -187,7 +188,8 @@ static ttt_status create_impl(const ttt_config* cfg, const void* W0, const void*
     guard(dev_alloc((void**)&st->ip.W, nW * 4, "W")) && guard(dev_alloc((void**)&st->ip.W0, nW * 4, "W0"));
     if (r == TTT_OK && c.io_dtype == TTT_BF16) {
       guard(dev_alloc((void**)&st->ip.Wsh[0], nW * 2, "W bf16 copy")) &&
-          guard(dev_alloc((void**)&st->ip.Wsh[1], nW * 2, "W bf16 copy"));
+          guard(dev_alloc((void**)&st->ip.Wsh[1], nW * 2, "W bf16 copy")) &&
+          guard(dev_alloc((void**)&st->ip.Wsh[2], nW * 2, "W bf16 copy"));
     }
     if (r == TTT_OK && target) {
       const size_t dd = (size_t)c.d_val * c.d_val;
