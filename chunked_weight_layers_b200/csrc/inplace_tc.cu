@@ -95,6 +95,13 @@ struct TCArgs {
   int nbd;
   int* upd_done;
   int* app_done;
+  // Fused target over several chunks: the last round runs sched_last (no TARGET tiles); the
+  // TARGET tiles of round r write V̂ of chunk chunk + r + 1 into vhat[(r + 1) & 1], which the
+  // UPDATE tiles of round r + 1 read; tgt_done[r·nbd + b] counts round r's TARGET work on
+  // 256-column block b of V̂ (one per epilogue warp and tile).
+  const int32_t* sched_last;
+  __nv_bfloat16* vhat[2];
+  int* tgt_done;
 };
 
 // ---- tcgen05 wrappers -----------------------------------------------------------------
@@ -211,7 +218,8 @@ __device__ __forceinline__ void named_sync_half(int half) {
 
 __global__ void __launch_bounds__(kThreadsTC, 1)
     k_inplace_tc(const __grid_constant__ CUtensorMap tmZk, const __grid_constant__ CUtensorMap tmZm,
-                 const __grid_constant__ CUtensorMap tmVm, const __grid_constant__ CUtensorMap tmWk0,
+                 const __grid_constant__ CUtensorMap tmVm, const __grid_constant__ CUtensorMap tmVm1,
+                 const __grid_constant__ CUtensorMap tmWk0,
                  const __grid_constant__ CUtensorMap tmWk1, const __grid_constant__ CUtensorMap tmWk2,
                  const __grid_constant__ CUtensorMap tmConv, const __grid_constant__ CUtensorMap tmWt,
                  const __grid_constant__ CUtensorMap tmWf, const __grid_constant__ CUtensorMap tmWs0,
@@ -220,19 +228,23 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   extern __shared__ uint8_t smem_raw[];
   TCSmem& sm = *reinterpret_cast<TCSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int32_t* tiles = args.sched + gridDim.x + 1;
   // In round r the CTA runs tile list (blockIdx.x + r·kRotate) mod gridDim.x: over the rounds
   // every CTA works through a mix of the lists, so their different loads even out instead of
   // adding up round after round.
   auto list_of = [&](int rnd) { return (int)(((long)blockIdx.x + (long)rnd * kRotate) % gridDim.x); };
+  auto sched_of = [&](int rnd) {
+    return (args.sched_last != nullptr && rnd == args.rounds - 1) ? args.sched_last : args.sched;
+  };
   int ntot = 0;  // tiles of this CTA over all rounds
-  for (int rnd = 0; rnd < args.rounds; ++rnd) ntot += args.sched[list_of(rnd) + 1] - args.sched[list_of(rnd)];
+  for (int rnd = 0; rnd < args.rounds; ++rnd) ntot += sched_of(rnd)[list_of(rnd) + 1] - sched_of(rnd)[list_of(rnd)];
   // Walks the CTA's tiles in order: calls f(round, tile code) until it returns false.
   auto for_tiles = [&](auto&& f) {
     for (int rnd = 0; rnd < args.rounds; ++rnd) {
+      const int32_t* sch = sched_of(rnd);
       const int li = list_of(rnd);
-      for (int ti = args.sched[li]; ti < args.sched[li + 1]; ++ti)
-        if (!f(rnd, tiles[ti])) return;
+      const int32_t* tl = sch + gridDim.x + 1;
+      for (int ti = sch[li]; ti < sch[li + 1]; ++ti)
+        if (!f(rnd, tl[ti])) return;
     }
   };
 
@@ -286,7 +298,19 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           if (type == UPDATE && rnd >= 2 &&
               !wait_counter(&args.app_done[(rnd - 2) * args.nbd + m / 2], args.C / BM, args.status, abort))
             return false;
+          if (args.tgt_done != nullptr) {
+            // V̂ of this round was produced by the previous round's TARGET tiles; a TARGET tile
+            // overwrites the V̂ buffer the previous round's UPDATE tiles of its block read.
+            if (type == UPDATE && rnd >= 1 &&
+                !wait_counter(&args.tgt_done[(rnd - 1) * args.nbd + m / 2], kEpiWarps * (args.C / BM), args.status,
+                              abort))
+              return false;
+            if (type == TARGET && rnd >= 1 &&
+                !wait_counter(&args.upd_done[(rnd - 1) * args.nbd + n], upd_expect(args, n), args.status, abort))
+              return false;
+          }
         }
+        const CUtensorMap* vm = (args.tgt_done != nullptr && (rnd & 1)) ? &tmVm1 : &tmVm;
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const int s = it % kSt;
           if (it >= kSt && !mbar_wait(&sm.empty[s], ((it / kSt) - 1) & 1, args.status, abort)) return false;
@@ -296,7 +320,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
             tma_load_2d(sm.B[s], wk, &sm.full[s], kb * BK, n * BN);
           } else if (type == UPDATE) {
             for (int j = 0; j < BM / 64; ++j)
-              tma_load_2d(sm.A[s] + j * 8192, &tmVm, &sm.full[s], m * BM + j * 64, args.vrow0 + rnd * args.C + kb * BK);
+              tma_load_2d(sm.A[s] + j * 8192, vm, &sm.full[s], m * BM + j * 64,
+                          args.vrow0 + (args.tgt_done != nullptr ? 0 : rnd * args.C) + kb * BK);
             for (int j = 0; j < BN / 64; ++j)
               tma_load_2d(sm.B[s] + j * 8192, &tmZm, &sm.full[s], n * BN + j * 64, chunk * args.C + kb * BK);
           } else {
@@ -500,7 +525,15 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           if (type == APPLY)
             store_row_bf16(args.O + ((size_t)(args.chunk + rnd) * args.C + row) * args.d, col0, args.d, v);
           else
-            store_row_bf16(args.Vhat_out + (size_t)row * args.d, col0, args.d, v);
+            store_row_bf16((args.tgt_done != nullptr ? args.vhat[(rnd + 1) & 1] : args.Vhat_out) + (size_t)row * args.d,
+                           col0, args.d, v);
+        }
+        if (type == TARGET && args.tgt_done != nullptr) {
+          __syncwarp();
+          if (lane == 0) {
+            __threadfence();
+            atomicAdd(&args.tgt_done[rnd * args.nbd + n], 1);
+          }
         }
       }
       tc_fence_before();
@@ -731,22 +764,34 @@ ttt_status inplace_bf16_scan(ttt_state* st, const __nv_bfloat16* Z, const __nv_b
     a.nbd = (d + BN - 1) / BN;
     a.upd_done = counters;
     a.app_done = counters ? counters + (size_t)rounds * a.nbd : nullptr;
+    a.sched_last = nullptr;
+    a.vhat[0] = a.vhat[1] = nullptr;
+    a.tgt_done = nullptr;
     return a;
   };
   auto launch = [&](int plan, const TCArgs& a, const CUtensorMap& vm) -> ttt_status {
-    k_inplace_tc<<<r->grid[plan], kThreadsTC, smem, s>>>(tmZk, tmZm, vm, tmWk[0], tmWk[1], tmWk[2], tmConv, tmWt,
+    k_inplace_tc<<<r->grid[plan], kThreadsTC, smem, s>>>(tmZk, tmZm, vm, vm, tmWk[0], tmWk[1], tmWk[2], tmConv, tmWt,
                                                          tmWf, tmWs[0], tmWs[1], tmWs[2], a);
     st->launches++;
     TTT_CUDA(cudaGetLastError());
     return TTT_OK;
   };
-
-  if (!target) {
-    // All chunks in one launch: each CTA runs its tile list once per chunk, waiting on
-    // progress counters only where a chunk needs another CTA's result of an earlier chunk,
-    // so a chunk's last tiles overlap the next chunk's first. The grid is one CTA per SM and
-    // is launched cooperatively, which guarantees that every CTA is resident.
-    const size_t need = 2 * (size_t)nchunks * ((d + BN - 1) / BN);
+  // All chunks in one launch: each CTA runs its tile list once per chunk, waiting on progress
+  // counters only where a chunk needs another CTA's result of an earlier chunk, so a chunk's
+  // last tiles overlap the next chunk's first. The grid is one CTA per SM and is launched
+  // cooperatively, which guarantees that every CTA is resident.
+  auto launch_rounds = [&](TCArgs& a, const CUtensorMap& vm0, const CUtensorMap& vm1) -> ttt_status {
+    const CUtensorMap* vm1p = &vm1;
+    void* params[] = {&tmZk, &tmZm, const_cast<CUtensorMap*>(&vm0), const_cast<CUtensorMap*>(vm1p), &tmWk[0], &tmWk[1],
+                      &tmWk[2], &tmConv, &tmWt, &tmWf, &tmWs[0], &tmWs[1], &tmWs[2], &a};
+    TTT_CUDA(cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(k_inplace_tc), dim3(r->grid[0]),
+                                         dim3(kThreadsTC), params, smem, s));
+    st->launches++;
+    st->ip.cur = (st->ip.cur + nchunks) % 3;
+    return TTT_OK;
+  };
+  const int nbd = (d + BN - 1) / BN;
+  auto counters = [&](size_t need) -> ttt_status {
     if (r->counters_n < need) {
       if (r->counters) cudaFree(r->counters);
       r->counters = nullptr;
@@ -755,17 +800,29 @@ ttt_status inplace_bf16_scan(ttt_state* st, const __nv_bfloat16* Z, const __nv_b
       r->counters_n = need;
     }
     TTT_CUDA(cudaMemsetAsync(r->counters, 0, need * sizeof(int), s));
-    TCArgs a = args_for(0, 0, 1, nchunks, r->counters);
-    void* params[] = {&tmZk, &tmZm, &tmVm_in, &tmWk[0], &tmWk[1], &tmWk[2], &tmConv, &tmWt, &tmWf,
-                      &tmWs[0], &tmWs[1], &tmWs[2], &a};
-    TTT_CUDA(cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(k_inplace_tc), dim3(r->grid[0]),
-                                         dim3(kThreadsTC), params, smem, s));
-    st->launches++;
-    st->ip.cur = (st->ip.cur + nchunks) % 3;
     return TTT_OK;
+  };
+
+  if (!target) {
+    TTT_TRY(counters(2 * (size_t)nchunks * nbd));
+    TCArgs a = args_for(0, 0, 1, nchunks, r->counters);
+    return launch_rounds(a, tmVm_in, tmVm_in);
   }
 
-  TTT_TRY(launch(1, args_for(1, 0, 0, 1, nullptr), tmVm_buf[0]));  // targets of chunk 0
+  // Fused target: the targets of the first chunk by their own launch, then every chunk in
+  // one launch whose rounds also produce the next chunk's targets (the last round runs the
+  // schedule without TARGET tiles).
+  TTT_TRY(launch(1, args_for(1, 0, 0, 1, nullptr), tmVm_buf[0]));
+  if (r->grid[2] == r->grid[0]) {
+    TTT_TRY(counters(3 * (size_t)nchunks * nbd));
+    TCArgs a = args_for(0, 0, 1, nchunks, r->counters);
+    a.sched_last = r->plan_dev[2];
+    a.vhat[0] = st->ip.Vhat[0];
+    a.vhat[1] = st->ip.Vhat[1];
+    a.tgt_done = r->counters + 2 * (size_t)nchunks * nbd;
+    a.Vhat_out = nullptr;
+    return launch_rounds(a, tmVm_buf[0], tmVm_buf[1]);
+  }
   for (int ch = 0; ch < nchunks; ++ch) {
     const bool last = ch + 1 == nchunks;
     const int plan = last ? 2 : 0;
@@ -830,10 +887,13 @@ ttt_status target_values_into(const __nv_bfloat16* X0, const float* convw, const
   a.nbd = 0;
   a.upd_done = nullptr;
   a.app_done = nullptr;
+  a.sched_last = nullptr;
+  a.vhat[0] = a.vhat[1] = nullptr;
+  a.tgt_done = nullptr;
   const size_t smem = sizeof(TCSmem) + 1024;
   TTT_CUDA(cudaFuncSetAttribute(k_inplace_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-  k_inplace_tc<<<grid, kThreadsTC, smem, s>>>(tmConv, tmConv, tmConv, tmConv, tmConv, tmConv, tmConv, tmWt, tmConv,
-                                              tmConv, tmConv, tmConv, a);
+  k_inplace_tc<<<grid, kThreadsTC, smem, s>>>(tmConv, tmConv, tmConv, tmConv, tmConv, tmConv, tmConv, tmConv, tmWt,
+                                              tmConv, tmConv, tmConv, tmConv, a);
   TTT_CUDA(cudaGetLastError());
   return TTT_OK;
 }
