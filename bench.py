@@ -345,12 +345,17 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--workload", default=MAIN)
     ap.add_argument("--only-main", action="store_true", help="skip the other four workloads")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="run the named workload with this many tokens instead (same widths and chunk; a smaller "
+                         "case for profilers, not a bench line)")
     a = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     spec = spec_by_name(a.workload)
+    if a.tokens is not None:
+        spec = wl.scaled(spec, T=a.tokens, name=f"{spec.name}@T{a.tokens}")
     if world > 1:
         # Weak scaling: every rank scans its own batch of independent problems (its own seed).
         spec = wl.scaled(spec, seed=spec.seed + 7919 * rank)
