@@ -6,17 +6,26 @@
 // W_{c+1} = W_c + η·V̂_cᵀ·Z_c; with fused target generation (§4) V̂ = Conv1D(X0)·Wtarget.
 //
 // Design (B200):
-//  * one persistent launch per chunk; its CTAs (one per SM) work through a static tile
-//    schedule computed on the host by longest-processing-time-first, mixing three GEMM
-//    tile types of 128x256 outputs:
+//  * one persistent, cooperative launch per scan call, one CTA per SM; every chunk is a round
+//    in which each CTA works through a tile list of a static schedule computed on the host
+//    by longest-processing-time-first, mixing three GEMM tile types of 128x256 outputs:
 //      APPLY  O_c tile   = Z_c[128 tok, f] · W_cᵀ            A, B K-major        → bf16 O
 //      UPDATE ΔW tile    = V̂_c[:, 128 rows]ᵀ · Z_c[:, 256]   A, B MN-major (K = tokens)
 //                          epilogue W += η·ΔW (fp32 read-modify-write) and writes the bf16
 //                          copy of W_{c+1} used by the next chunk's APPLY tiles
 //      TARGET V̂_{c+1} tile = conv(X0)_{c+1}[128 tok, d] · Wtarget[:, 256]  A K-major, B MN-major
-//    APPLY reads the bf16 copy of W_c while UPDATE writes the other copy, so both run in the
-//    same launch without waiting for each other; the compute-bound APPLY tiles and the
-//    HBM-bound UPDATE epilogues overlap on different SMs.
+//    The bf16 copy of W rotates through three buffers: chunk c applies with one, its update
+//    writes the next, and the third is what chunk c − 1 applied with, so APPLY and UPDATE
+//    tiles of neighbouring chunks overlap. Where a tile needs another CTA's work of an earlier
+//    chunk, it waits (bounded) on a progress counter per chunk and 256-row block of W: an APPLY
+//    tile on the previous chunk's UPDATE tiles of its block, an UPDATE tile on the APPLY
+//    tiles of two chunks back (their buffer is the one it overwrites), the W loader on the
+//    previous chunk's update of its tile, and with the fused target an UPDATE tile on the
+//    previous chunk's TARGET tiles and a TARGET tile on the UPDATE tiles that read the target
+//    buffer it overwrites. Every wait refers to an earlier chunk, so the CTA furthest behind
+//    can always proceed. In round r CTA i runs list (i + 61r) mod 148: the lists' different
+//    loads even out over the rounds. The compute-bound APPLY tiles and the HBM-bound UPDATE
+//    epilogues overlap on different SMs.
 //  * per CTA: warp 0 issues TMA loads (128-byte swizzle) into a 3-stage shared-memory ring,
 //    warp 1 allocates 512 TMEM columns and one lane issues tcgen05.mma (M=128, N=256, K=16)
 //    into one of two TMEM accumulators, warps 2..9 drain the other accumulator
