@@ -105,11 +105,12 @@ struct TCArgs {
   int* upd_done;
   int* app_done;
   // Fused target over several chunks: the last round runs sched_last (no TARGET tiles); the
-  // TARGET tiles of round r write V̂ of chunk chunk + r + 1 into vhat[(r + 1) & 1], which the
-  // UPDATE tiles of round r + 1 read; tgt_done[r·nbd + b] counts round r's TARGET work on
-  // 256-column block b of V̂ (one per epilogue warp and tile).
+  // TARGET tiles of round r write V̂ of chunk chunk + r + 1 into vhat[(r + 1) % 3], which the
+  // UPDATE tiles of round r + 1 read (the buffer they overwrite was read two rounds before);
+  // tgt_done[r·nbd + b] counts round r's TARGET work on 256-column block b of V̂ (one per
+  // epilogue warp and tile).
   const int32_t* sched_last;
-  __nv_bfloat16* vhat[2];
+  __nv_bfloat16* vhat[3];
   int* tgt_done;
 };
 
@@ -228,6 +229,7 @@ __device__ __forceinline__ void named_sync_half(int half) {
 __global__ void __launch_bounds__(kThreadsTC, 1)
     k_inplace_tc(const __grid_constant__ CUtensorMap tmZk, const __grid_constant__ CUtensorMap tmZm,
                  const __grid_constant__ CUtensorMap tmVm, const __grid_constant__ CUtensorMap tmVm1,
+                 const __grid_constant__ CUtensorMap tmVm2,
                  const __grid_constant__ CUtensorMap tmWk0,
                  const __grid_constant__ CUtensorMap tmWk1, const __grid_constant__ CUtensorMap tmWk2,
                  const __grid_constant__ CUtensorMap tmConv, const __grid_constant__ CUtensorMap tmWt,
@@ -314,12 +316,12 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
                 !wait_counter(&args.tgt_done[(rnd - 1) * args.nbd + m / 2], kEpiWarps * (args.C / BM), args.status,
                               abort))
               return false;
-            if (type == TARGET && rnd >= 1 &&
-                !wait_counter(&args.upd_done[(rnd - 1) * args.nbd + n], upd_expect(args, n), args.status, abort))
+            if (type == TARGET && rnd >= 2 &&
+                !wait_counter(&args.upd_done[(rnd - 2) * args.nbd + n], upd_expect(args, n), args.status, abort))
               return false;
           }
         }
-        const CUtensorMap* vm = (args.tgt_done != nullptr && (rnd & 1)) ? &tmVm1 : &tmVm;
+        const CUtensorMap* vm = args.tgt_done != nullptr ? pick3(tmVm, tmVm1, tmVm2, rnd % 3) : &tmVm;
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const int s = it % kSt;
           if (it >= kSt && !mbar_wait(&sm.empty[s], ((it / kSt) - 1) & 1, args.status, abort)) return false;
@@ -534,7 +536,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           if (type == APPLY)
             store_row_bf16(args.O + ((size_t)(args.chunk + rnd) * args.C + row) * args.d, col0, args.d, v);
           else
-            store_row_bf16((args.tgt_done != nullptr ? args.vhat[(rnd + 1) & 1] : args.Vhat_out) + (size_t)row * args.d,
+            store_row_bf16((args.tgt_done != nullptr ? args.vhat[(rnd + 1) % 3] : args.Vhat_out) + (size_t)row * args.d,
                            col0, args.d, v);
         }
         if (type == TARGET && args.tgt_done != nullptr) {
@@ -628,10 +630,14 @@ Plan make_plan(int num_sms, int d, int f, int C, bool apply_update, bool target)
   // ends on an epilogue that only stores outputs rather than on a W read-modify-write, and
   // the CTAs holding an APPLY tile stream W while the others do too (measured on B200:
   // 3.59 against 3.68 ms on the T=32768 workload).
+  // With the fused target, TARGET tiles come first: the next chunk's UPDATE tiles, at the
+  // start of their round, need them.
+  auto rank = [](int32_t code) {
+    const int t = (code >> 28) & 3;
+    return t == TARGET ? 0 : (t == UPDATE ? 1 : 2);
+  };
   for (auto& v : per)
-    std::stable_sort(v.begin(), v.end(), [](int32_t a, int32_t b) {
-      return (((a >> 28) & 3) == UPDATE) > (((b >> 28) & 3) == UPDATE);
-    });
+    std::stable_sort(v.begin(), v.end(), [&](int32_t a, int32_t b) { return rank(a) < rank(b); });
   Plan p;
   p.grid = grid;
   p.host.resize(grid + 1);
@@ -721,7 +727,7 @@ ttt_status inplace_bf16_scan(ttt_state* st, const __nv_bfloat16* Z, const __nv_b
   TCResources* r = st->ip.tc;
   const int nchunks = (int)(T / C);
 
-  CUtensorMap tmZk, tmZm, tmVm_in, tmVm_buf[2], tmWk[3], tmConv, tmWt, tmWf, tmWs[3];
+  CUtensorMap tmZk, tmZm, tmVm_in, tmVm_buf[3], tmWk[3], tmConv, tmWt, tmWf, tmWs[3];
   TTT_TRY(map2d(&tmWf, st->ip.W, f, d, kWCols, BM, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, CU_TENSOR_MAP_SWIZZLE_128B));
   for (int i = 0; i < 3; ++i) {
     TTT_TRY(map2d(&tmWs[i], st->ip.Wsh[i], f, d, kWCols, BM, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, CU_TENSOR_MAP_SWIZZLE_64B));
@@ -739,8 +745,7 @@ ttt_status inplace_bf16_scan(ttt_state* st, const __nv_bfloat16* Z, const __nv_b
     }
     TTT_TRY(map2d(&tmConv, r->conv, d, T, BK, BM));
     TTT_TRY(map2d(&tmWt, st->ip.Wtarget, d, d, 64, BK));
-    TTT_TRY(map2d(&tmVm_buf[0], st->ip.Vhat[0], d, C, 64, BK));
-    TTT_TRY(map2d(&tmVm_buf[1], st->ip.Vhat[1], d, C, 64, BK));
+    for (int i = 0; i < 3; ++i) TTT_TRY(map2d(&tmVm_buf[i], st->ip.Vhat[i], d, C, 64, BK));
     const size_t pairs = (size_t)T * (d / 2);
     const int blocks = (int)std::min<size_t>((pairs + 255) / 256, (size_t)st->num_sms * 16);
     k_target_conv<<<blocks, 256, 0, s>>>(targets, st->ip.convw, r->conv, (int)T, d, C, c.conv_taps, c.conv_pad_mode);
@@ -766,7 +771,7 @@ ttt_status inplace_bf16_scan(ttt_state* st, const __nv_bfloat16* Z, const __nv_b
     a.C = C;
     a.eta = c.eta;
     a.O = O;
-    a.Vhat_out = target ? st->ip.Vhat[tchunk & 1] : nullptr;
+    a.Vhat_out = target ? st->ip.Vhat[tchunk % 3] : nullptr;
     a.status = st->status.dev;
     a.rounds = rounds;
     a.cur0 = st->ip.cur;
@@ -774,12 +779,12 @@ ttt_status inplace_bf16_scan(ttt_state* st, const __nv_bfloat16* Z, const __nv_b
     a.upd_done = counters;
     a.app_done = counters ? counters + (size_t)rounds * a.nbd : nullptr;
     a.sched_last = nullptr;
-    a.vhat[0] = a.vhat[1] = nullptr;
+    a.vhat[0] = a.vhat[1] = a.vhat[2] = nullptr;
     a.tgt_done = nullptr;
     return a;
   };
   auto launch = [&](int plan, const TCArgs& a, const CUtensorMap& vm) -> ttt_status {
-    k_inplace_tc<<<r->grid[plan], kThreadsTC, smem, s>>>(tmZk, tmZm, vm, vm, tmWk[0], tmWk[1], tmWk[2], tmConv, tmWt,
+    k_inplace_tc<<<r->grid[plan], kThreadsTC, smem, s>>>(tmZk, tmZm, vm, vm, vm, tmWk[0], tmWk[1], tmWk[2], tmConv, tmWt,
                                                          tmWf, tmWs[0], tmWs[1], tmWs[2], a);
     st->launches++;
     TTT_CUDA(cudaGetLastError());
@@ -789,10 +794,11 @@ ttt_status inplace_bf16_scan(ttt_state* st, const __nv_bfloat16* Z, const __nv_b
   // counters only where a chunk needs another CTA's result of an earlier chunk, so a chunk's
   // last tiles overlap the next chunk's first. The grid is one CTA per SM and is launched
   // cooperatively, which guarantees that every CTA is resident.
-  auto launch_rounds = [&](TCArgs& a, const CUtensorMap& vm0, const CUtensorMap& vm1) -> ttt_status {
-    const CUtensorMap* vm1p = &vm1;
-    void* params[] = {&tmZk, &tmZm, const_cast<CUtensorMap*>(&vm0), const_cast<CUtensorMap*>(vm1p), &tmWk[0], &tmWk[1],
-                      &tmWk[2], &tmConv, &tmWt, &tmWf, &tmWs[0], &tmWs[1], &tmWs[2], &a};
+  auto launch_rounds = [&](TCArgs& a, const CUtensorMap& vm0, const CUtensorMap& vm1,
+                           const CUtensorMap& vm2) -> ttt_status {
+    void* params[] = {&tmZk, &tmZm, const_cast<CUtensorMap*>(&vm0), const_cast<CUtensorMap*>(&vm1),
+                      const_cast<CUtensorMap*>(&vm2), &tmWk[0], &tmWk[1], &tmWk[2], &tmConv, &tmWt, &tmWf,
+                      &tmWs[0], &tmWs[1], &tmWs[2], &a};
     TTT_CUDA(cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(k_inplace_tc), dim3(r->grid[0]),
                                          dim3(kThreadsTC), params, smem, s));
     st->launches++;
@@ -815,7 +821,7 @@ ttt_status inplace_bf16_scan(ttt_state* st, const __nv_bfloat16* Z, const __nv_b
   if (!target) {
     TTT_TRY(counters(2 * (size_t)nchunks * nbd));
     TCArgs a = args_for(0, 0, 1, nchunks, r->counters);
-    return launch_rounds(a, tmVm_in, tmVm_in);
+    return launch_rounds(a, tmVm_in, tmVm_in, tmVm_in);
   }
 
   // Fused target: the targets of the first chunk by their own launch, then every chunk in
@@ -828,14 +834,15 @@ ttt_status inplace_bf16_scan(ttt_state* st, const __nv_bfloat16* Z, const __nv_b
     a.sched_last = r->plan_dev[2];
     a.vhat[0] = st->ip.Vhat[0];
     a.vhat[1] = st->ip.Vhat[1];
+    a.vhat[2] = st->ip.Vhat[2];
     a.tgt_done = r->counters + 2 * (size_t)nchunks * nbd;
     a.Vhat_out = nullptr;
-    return launch_rounds(a, tmVm_buf[0], tmVm_buf[1]);
+    return launch_rounds(a, tmVm_buf[0], tmVm_buf[1], tmVm_buf[2]);
   }
   for (int ch = 0; ch < nchunks; ++ch) {
     const bool last = ch + 1 == nchunks;
     const int plan = last ? 2 : 0;
-    TTT_TRY(launch(plan, args_for(plan, ch, ch + 1, 1, nullptr), tmVm_buf[ch & 1]));
+    TTT_TRY(launch(plan, args_for(plan, ch, ch + 1, 1, nullptr), tmVm_buf[ch % 3]));
     st->ip.cur = (st->ip.cur + 1) % 3;  // the bf16 copy written by this launch holds W_{c+1}
   }
   return TTT_OK;
@@ -897,11 +904,11 @@ ttt_status target_values_into(const __nv_bfloat16* X0, const float* convw, const
   a.upd_done = nullptr;
   a.app_done = nullptr;
   a.sched_last = nullptr;
-  a.vhat[0] = a.vhat[1] = nullptr;
+  a.vhat[0] = a.vhat[1] = a.vhat[2] = nullptr;
   a.tgt_done = nullptr;
   const size_t smem = sizeof(TCSmem) + 1024;
   TTT_CUDA(cudaFuncSetAttribute(k_inplace_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-  k_inplace_tc<<<grid, kThreadsTC, smem, s>>>(tmConv, tmConv, tmConv, tmConv, tmConv, tmConv, tmConv, tmConv, tmWt,
+  k_inplace_tc<<<grid, kThreadsTC, smem, s>>>(tmConv, tmConv, tmConv, tmConv, tmConv, tmConv, tmConv, tmConv, tmConv, tmWt,
                                               tmConv, tmConv, tmConv, tmConv, a);
   TTT_CUDA(cudaGetLastError());
   return TTT_OK;

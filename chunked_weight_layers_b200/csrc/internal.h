@@ -48,7 +48,9 @@ struct InplaceBuffers {
   int cur = 0;                   // index of the bf16 copy that holds the current W
   __nv_bfloat16* Wtarget = nullptr;  // [d, d]
   float* convw = nullptr;        // [d, taps]
-  __nv_bfloat16* Vhat[2] = {nullptr, nullptr};  // targets of a chunk [C, d] (fused target)
+  // Targets of a chunk [C, d] (fused target): chunk c's are produced while chunk c − 1 runs and
+  // read by chunk c's update; three buffers so the producer never waits for a reader.
+  __nv_bfloat16* Vhat[3] = {nullptr, nullptr, nullptr};
   TCResources* tc = nullptr;     // tensor-core schedules and conv(X0) buffer, built on first use
 };
 

@@ -112,6 +112,7 @@ static void free_state(ttt_state* st) {
   free_tc(st);
   dev_free(st->ip.Vhat[0]);
   dev_free(st->ip.Vhat[1]);
+  dev_free(st->ip.Vhat[2]);
   dev_free(st->lin.W);
   dev_free(st->lin.W0);
   dev_free(st->gate.tau);
@@ -196,7 +197,8 @@ static ttt_status create_impl(const ttt_config* cfg, const void* W0, const void*
       guard(dev_alloc((void**)&st->ip.Wtarget, dd * 2, "Wtarget")) &&
           guard(dev_alloc((void**)&st->ip.convw, (size_t)c.d_val * c.conv_taps * 4, "convw")) &&
           guard(dev_alloc((void**)&st->ip.Vhat[0], (size_t)c.chunk * c.d_val * 2, "target buffer")) &&
-          guard(dev_alloc((void**)&st->ip.Vhat[1], (size_t)c.chunk * c.d_val * 2, "target buffer"));
+          guard(dev_alloc((void**)&st->ip.Vhat[1], (size_t)c.chunk * c.d_val * 2, "target buffer")) &&
+          guard(dev_alloc((void**)&st->ip.Vhat[2], (size_t)c.chunk * c.d_val * 2, "target buffer"));
     }
   } else {
     guard(dev_alloc((void**)&st->lin.W, nW * 4, "W")) && guard(dev_alloc((void**)&st->lin.W0, nW * 4, "W0"));
