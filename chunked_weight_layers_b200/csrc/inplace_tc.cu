@@ -21,10 +21,11 @@
 //    tile on the previous chunk's UPDATE tiles of its block, an UPDATE tile on the APPLY
 //    tiles of two chunks back (their buffer is the one it overwrites), the W loader on the
 //    previous chunk's update of its tile, and with the fused target an UPDATE tile on the
-//    previous chunk's TARGET tiles and a TARGET tile on the UPDATE tiles that read the target
-//    buffer it overwrites. Every wait refers to an earlier chunk, so the CTA furthest behind
-//    can always proceed. In round r CTA i runs list (i + 73r) mod 148: the lists' different
-//    loads even out over the rounds. The compute-bound APPLY tiles and the HBM-bound UPDATE
+//    previous chunk's TARGET tiles and a TARGET tile on the UPDATE tiles of two chunks back,
+//    which read the target buffer it overwrites (targets rotate through three buffers, and
+//    TARGET tiles come first in each list). Every wait refers to an earlier chunk, so the CTA
+//    furthest behind can always proceed. In round r CTA i runs list (i + 73r) mod 148: the
+//    lists' different loads even out over the rounds. The compute-bound APPLY tiles and the HBM-bound UPDATE
 //    epilogues overlap on different SMs.
 //  * per CTA: warp 0 issues TMA loads (128-byte swizzle) into a 3-stage shared-memory ring,
 //    warp 1 allocates 512 TMEM columns and one lane issues tcgen05.mma (M=128, N=256, K=16)
