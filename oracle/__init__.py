@@ -8,8 +8,9 @@ pages' order, with no blocking, fusion or reordering beyond the definitions:
   LM-aligned update and the Conv1D + Wtarget target (In-Place Test-Time Training,
   §2 "Wdown as fast weight", §3 "apply first, update later", §4 "predict the next
   token", §6 "context parallelism").
-* :mod:`oracle.linear` — TTT-Linear mini-batch gradient scan (TTT layers page,
-  "hidden state is itself a model" and the DeltaNet remark).
+* :mod:`oracle.linear` — TTT-Linear mini-batch gradient scan (TTT layers page: the
+  recurrent state is an inner model's weight trained while the sequence is read; and its
+  DeltaNet remark).
 * :mod:`oracle.gate` — SR-TTT surprisal gate and residual cache (SR-TTT technical
   summary, §2.1 "Surprisal Filter" and "Residual Cache").
 
