@@ -2,9 +2,9 @@
 
 Source: "テスト時学習（Test-Time Training）とは" (TTT layers page, arXiv 2407.04620):
 
-* "hidden state is itself a model": the hidden state is the weight W of a linear inner
-  model and the update rule is one step of self-supervised learning on the sequence;
-  TTT-Linear is the instance with a linear inner model.
+* the layer's recurrent state is the weight W of an inner model, and the update rule is
+  one step of self-supervised learning on the sequence; TTT-Linear is the instance with a
+  linear inner model.
 * the related-work remark: DeltaNet is TTT-Linear with inner mini-batch 1 and without
   LayerNorm and the residual connection.
 
