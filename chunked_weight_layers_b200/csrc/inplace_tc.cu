@@ -627,12 +627,11 @@ Plan make_plan(int num_sms, int d, int f, int C, bool apply_update, bool target)
     per[best].push_back(t.code);
     load[best] += t.cost;
   }
-  // Within each CTA, UPDATE tiles first and the long APPLY/TARGET tile last: the launch then
-  // ends on an epilogue that only stores outputs rather than on a W read-modify-write, and
-  // the CTAs holding an APPLY tile stream W while the others do too (measured on B200:
-  // 3.59 against 3.68 ms on the T=32768 workload).
-  // With the fused target, TARGET tiles come first: the next chunk's UPDATE tiles, at the
-  // start of their round, need them.
+  // Within each CTA: TARGET tiles first (the next chunk's UPDATE tiles, at the start of their
+  // round, need them), then UPDATE tiles, and the long APPLY tile last: a round then ends on
+  // an epilogue that only stores outputs rather than on a W read-modify-write, and the CTAs
+  // holding an APPLY tile stream W while the others do too (measured on B200: 3.59 against
+  // 3.68 ms on the T=32768 workload).
   auto rank = [](int32_t code) {
     const int t = (code >> 28) & 3;
     return t == TARGET ? 0 : (t == UPDATE ? 1 : 2);
