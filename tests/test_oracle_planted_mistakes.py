@@ -1,0 +1,119 @@
+"""Planted mistakes: every plausible slip in the oracle fails at least one committed pin.
+
+For each mutation below, one oracle module's source is edited in one place (on the CPU;
+nothing here touches the CUDA path), loaded as a separate module, and the pin tests of
+tests/test_oracle_<module>.py are run with it in place of the real module. The unmutated
+oracle passes all of them; each mutant must fail at least one. This is the evidence that
+the pins constrain the oracle's arithmetic rather than restate it.
+"""
+
+from __future__ import annotations
+
+import importlib
+import inspect
+import os
+import types
+
+import pytest
+
+ORACLE = os.path.join(os.path.dirname(__file__), "..", "oracle")
+
+# (module, description, [(text, replacement), ...]); each text occurs exactly once.
+MUTANTS = [
+    ("inplace", "wrong sign of the update",
+     [("W = W + eta * (Vc.T @ Zc)", "W = W - eta * (Vc.T @ Zc)")]),
+    ("inplace", "step size dropped from the update",
+     [("W = W + eta * (Vc.T @ Zc)", "W = W + (Vc.T @ Zc)")]),
+    ("inplace", "update applied before the chunk's own output",
+     [("        O[rows] = Zc @ W.T                 # apply with W before this chunk's update (§3)\n"
+       "        W = W + eta * (Vc.T @ Zc)          # ΔW = η·V̂ᵀ·Z (§2)",
+       "        W = W + eta * (Vc.T @ Zc)\n"
+       "        O[rows] = Zc @ W.T")]),
+    ("inplace", "every chunk applied with the initial weight",
+     [("O[rows] = Zc @ W.T ", "O[rows] = Zc @ f64(W0).T ")]),
+    ("inplace", "convolution tap shifted by one token",
+     [("        src = t + k\n", "        src = t + k + 1\n")]),
+    ("inplace", "convolution ignores the chunk boundary",
+     [("end = (t // C + 1) * C if pad_mode == 0 else np.full(T, T)", "end = np.full(T, T)")]),
+    ("inplace", "convolution weights of the wrong tap",
+     [("out[ok] += X[src[ok]] * w[:, k]", "out[ok] += X[src[ok]] * w[:, taps - 1 - k]")]),
+    ("linear", "wrong sign of the gradient step",
+     [("W = W - (eta / b) * (np.swapaxes(Ki, 1, 2) @ R)", "W = W + (eta / b) * (np.swapaxes(Ki, 1, 2) @ R)")]),
+    ("linear", "step size not divided by the mini-batch",
+     [("W = W - (eta / b) * (np.swapaxes(Ki, 1, 2) @ R)", "W = W - eta * (np.swapaxes(Ki, 1, 2) @ R)")]),
+    ("linear", "residual with the wrong sign",
+     [("R = Ki @ W - Vi ", "R = Vi - Ki @ W ")]),
+    ("linear", "transposed gradient",
+     [("W = W - (eta / b) * (np.swapaxes(Ki, 1, 2) @ R)", "W = W - (eta / b) * (np.swapaxes(R, 1, 2) @ Ki)")]),
+    ("linear", "outputs from the weight after the mini-batch's update",
+     [("        if Qf is not None:\n"
+       "            O[:, s] = Qf[:, s] @ W                       # output with W_i (start of mini-batch)\n",
+       ""),
+      ("        W = W - (eta / b) * (np.swapaxes(Ki, 1, 2) @ R)  # one gradient step on ℓ_i\n",
+       "        W = W - (eta / b) * (np.swapaxes(Ki, 1, 2) @ R)\n"
+       "        if Qf is not None:\n"
+       "            O[:, s] = Qf[:, s] @ W\n")]),
+    ("linear", "loss not squared per element",
+     [("loss[:, s] = np.sum(R * R, axis=2)", "loss[:, s] = np.sum(R, axis=2) ** 2")]),
+    ("gate", "percentile one rank too high",
+     [("p = np.sort(x)[rank - 1]", "p = np.sort(x)[min(rank, len(x) - 1)]")]),
+    ("gate", "EMA weights swapped",
+     [("tau = np.float32(np.float32(ema_old * tau) + np.float32(ema_new * p))",
+       "tau = np.float32(np.float32(ema_new * tau) + np.float32(ema_old * p))")]),
+    ("gate", "threshold not carried from chunk to chunk",
+     [("                if state.tau_set[bi, hi]:\n", "                if False:\n")]),
+    ("gate", "comparison with the threshold not strict",
+     [("if x[j] > tau:", "if x[j] >= tau:")]),
+    ("gate", "mean test with numerator and denominator swapped",
+     [("passed = mean_den * S >= float(mean_num * gate_chunk) * float(tau)",
+       "passed = mean_num * S >= float(mean_den * gate_chunk) * float(tau)")]),
+    ("gate", "mean test skipped",
+     [("                if not passed:\n                    continue\n", "")]),
+    ("gate", "dropped tokens not counted",
+     [("                            state.dropped[bi, hi] += 1\n", "                            pass\n")]),
+    ("gate", "token index ignores the stream position",
+     [("(bi, hi, state.t_offset + g * gate_chunk + j)", "(bi, hi, g * gate_chunk + j)")]),
+]
+
+
+def _load(module: str, edits) -> types.ModuleType:
+    src = open(os.path.join(ORACLE, f"{module}.py"), encoding="utf-8").read()
+    for text, replacement in edits:
+        assert src.count(text) == 1, f"mutation text not found once in oracle/{module}.py: {text!r}"
+        src = src.replace(text, replacement)
+    mod = types.ModuleType(f"oracle.planted_{module}")
+    mod.__package__ = "oracle"
+    exec(compile(src, f"<oracle/{module}.py, planted>", "exec"), mod.__dict__)
+    return mod
+
+
+def _failing_pins(module: str, impl: types.ModuleType) -> list[str]:
+    """Names of the pin tests of ``module`` that fail with ``impl`` swapped in."""
+    pins = importlib.import_module(f"tests.test_oracle_{module}")
+    real = getattr(pins, module)
+    setattr(pins, module, impl)
+    failed = []
+    try:
+        for name, fn in inspect.getmembers(pins, inspect.isfunction):
+            if not name.startswith("test_") or fn.__module__ != pins.__name__:
+                continue
+            try:
+                fn()
+            except (KeyboardInterrupt, SystemExit):
+                raise
+            except BaseException:  # an assertion, a pytest failure, or an error the slip causes
+                failed.append(name)
+    finally:
+        setattr(pins, module, real)
+    return failed
+
+
+@pytest.mark.parametrize("module", ["inplace", "linear", "gate"])
+def test_unmutated_oracle_passes_every_pin(module):
+    assert _failing_pins(module, _load(module, [])) == []
+
+
+@pytest.mark.parametrize("module,description,edits", MUTANTS, ids=[f"{m}: {d}" for m, d, _ in MUTANTS])
+def test_planted_mistake_fails_a_pin(module, description, edits):
+    failed = _failing_pins(module, _load(module, edits))
+    assert failed, f"no pin of oracle/{module}.py catches: {description}"
