@@ -263,7 +263,7 @@ def roofline(spec, w, ms, peaks, traffic=None):
             "traffic": traffic, "peak_source": "148 SMs x 128 FP32 lanes x 2 x max SM clock"}
 
 
-def cpu_baseline(spec, budget_s=12.0) -> dict:
+def cpu_baseline(spec, limit_s=12.0) -> dict:
     """The oracle as it stands on this host's cores, on a bounded sample of the workload."""
     import numpy as np  # noqa: F401
     from oracle import gate as ogate
@@ -280,7 +280,7 @@ def cpu_baseline(spec, budget_s=12.0) -> dict:
         Q = x["Q"].reshape(BH, 1, spec.T, spec.D) if "Q" in x else None
         W0 = x["W0"].reshape(BH, 1, spec.D, spec.D)
         t0 = time.perf_counter()
-        while done_heads < BH and time.perf_counter() - t0 < budget_s:
+        while done_heads < BH and time.perf_counter() - t0 < limit_s:
             h = done_heads
             _, _, L = olin.ttt_linear_scan(K[h:h + 1], V[h:h + 1], None if Q is None else Q[h:h + 1],
                                           W0[h:h + 1], spec.eta, spec.b)
@@ -300,7 +300,7 @@ def cpu_baseline(spec, budget_s=12.0) -> dict:
         if Vh is None:
             Vh = torch.from_numpy(oinp.target_values(x["X0"], x["convw"], x["Wtarget"], spec.C))
         T = x["Z"].shape[0]
-        while time.perf_counter() - t0 < budget_s and chunks * Cs < T:
+        while time.perf_counter() - t0 < limit_s and chunks * Cs < T:
             sl = slice(chunks * Cs, (chunks + 1) * Cs)
             _, W = oinp.inplace_scan(x["Z"][sl], Vh[sl], W, spec.eta, Cs)
             chunks += 1

@@ -14,7 +14,7 @@ constexpr int kDevCheck = 6;
 
 // Every spin-wait in this library gives up after this many nanoseconds of %globaltimer,
 // records TTT_ERR_TIMEOUT in the state's status word and lets the kernel wind down.
-constexpr uint64_t kWaitBudgetNs = 2000000000ull;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 __device__ __forceinline__ void record_status(int* status, int code) {
   if (status != nullptr) atomicCAS(status, 0, code);
@@ -67,7 +67,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Waits for phase `parity` of `bar` to complete. Returns false (after recording a timeout)
-// if it has not completed within the wait budget, or at once if *abort is already set.
+// if it has not completed within the wait limit, or at once if *abort is already set.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status,
                                           volatile int* abort) {
   if (mbar_try_wait(bar, parity)) return true;
@@ -77,7 +77,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* s
     if (mbar_try_wait(bar, parity)) return true;
     if ((++spins & 63u) == 0) {
       if (abort != nullptr && *abort) return false;
-      if (globaltimer() - t0 > kWaitBudgetNs) {
+      if (globaltimer() - t0 > kWaitLimitNs) {
         record_status(status, kDevTimeout);
         if (abort != nullptr) *abort = 1;
         return false;

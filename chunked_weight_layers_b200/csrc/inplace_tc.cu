@@ -203,7 +203,7 @@ __device__ __forceinline__ bool wait_counter(const int* ctr, int want, int* stat
     const uint64_t t0 = globaltimer();
     while (*c < want) {
       if (*abort) return false;
-      if (globaltimer() - t0 > kWaitBudgetNs) {
+      if (globaltimer() - t0 > kWaitLimitNs) {
         record_status(status, kDevTimeout);
         *abort = 1;
         return false;

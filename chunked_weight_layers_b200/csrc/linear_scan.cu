@@ -294,7 +294,7 @@ __device__ __forceinline__ bool wait_turn(const int* turn, int want, int* status
   const uint64_t t0 = globaltimer();
   while (*tv != want) {
     if (*av) return false;
-    if (globaltimer() - t0 > kWaitBudgetNs) {
+    if (globaltimer() - t0 > kWaitLimitNs) {
       record_status(status, kDevTimeout);
       *const_cast<volatile int*>(av) = 1;
       return false;
