@@ -5,11 +5,20 @@ include/ttt.h). This module is its thin Python binding: :class:`FastWeightState`
 torch tensors into device pointers and the current CUDA stream and calls the C entry
 points of the same names. There is no CPU or PyTorch fallback: without the compiled
 library, or without a CUDA device, every call raises.
+
+The C ABI takes bare pointers, so it cannot see a buffer's size or element type. Before each
+call the binding checks what only it can see: every tensor has the element type and at
+least the element count the call reads or writes (from the state's configuration and T),
+is contiguous, and lives on the current CUDA device. A tensor that fails raises ValueError
+and nothing is launched; everything else (T against the chunk, which buffers a rule takes,
+alignment) is the library's to reject.
 """
 
 from __future__ import annotations
 
 import ctypes
+
+import torch
 
 from . import abi
 from .abi import TTTError, check  # noqa: F401
@@ -17,18 +26,28 @@ from .abi import TTTError, check  # noqa: F401
 __all__ = ["FastWeightState", "TTTError", "config", "abi"]
 
 
-def _ptr(t) -> int | None:
+# torch's current CUDA device of this thread (its direct accessor when present: it is called
+# on every scan).
+_current_device = getattr(torch._C, "_cuda_getDevice", None) or torch.cuda.current_device
+
+
+def _arg(t, name: str, dtype, numel: int, dev: int | None) -> int | None:
+    """Device (or, with ``dev`` None, host) address of ``t`` once it is known to hold at
+    least ``numel`` contiguous elements of ``dtype`` on device ``dev``."""
     if t is None:
         return None
-    if not (t.is_cuda and t.is_contiguous()):
-        raise ValueError("expected a contiguous CUDA tensor")
+    if (t.dtype is not dtype or t.numel() < numel or not t.is_contiguous()
+            or (t.get_device() != dev if dev is not None else t.is_cuda)):
+        where = "the host" if dev is None else f"cuda:{dev}"
+        raise ValueError(f"{name}: expected a contiguous {dtype} tensor of at least {numel} elements on "
+                         f"{where}, got {tuple(t.shape)} {t.dtype} on {t.device}"
+                         f"{'' if t.is_contiguous() else ' (not contiguous)'}")
     return t.data_ptr()
 
 
 def _current_raw_stream():
     """A function returning torch's current CUDA stream handle of the current device: torch's
     direct accessor when present (a fraction of a microsecond a call), else the public API."""
-    import torch
     raw = getattr(torch._C, "_cuda_getCurrentRawStream", None)
     cur_dev = getattr(torch._C, "_cuda_getDevice", None)
     if raw is not None and cur_dev is not None:
@@ -62,56 +81,87 @@ def config(rule: str, **fields) -> abi.ttt_config:
     return cfg
 
 
+def _layout(cfg: abi.ttt_config):
+    """(In-Place?, io element type, sequence-head pairs, d_key, d_val, weight elements, cache
+    entries per pair) of a state created with ``cfg``, as include/ttt.h lays its buffers out."""
+    inplace = cfg.rule == abi.TTT_RULE_INPLACE_HEBBIAN
+    io = torch.float32 if cfg.io_dtype == abi.TTT_F32 else torch.bfloat16
+    bh = 1 if inplace else cfg.batch * cfg.heads
+    nW = cfg.d_val * cfg.d_key if inplace else bh * cfg.d_key * cfg.d_key
+    cap = cfg.cache_capacity if (not inplace and cfg.gate_enable) else 1
+    return inplace, io, bh, cfg.d_key, cfg.d_val, nW, cap
+
+
 class FastWeightState:
     """Owner of one ttt_state (device weights, gate threshold and residual cache)."""
 
     def __init__(self, cfg: abi.ttt_config, W0, Wtarget=None, convw=None, stream=None):
         self._lib = abi.load()
         self.cfg = cfg
+        # Element counts the calls need, fixed at creation (the library keeps its own copy of cfg).
+        self._inplace, self._io, self._bh, self._dk, self._dv, self._nW, self._cap = _layout(cfg)
+        dev = _current_device()
         h = ctypes.c_void_p()
-        check(self._lib.ttt_state_create(ctypes.byref(cfg), _ptr(W0), _ptr(Wtarget), _ptr(convw),
-                                         _stream(stream), ctypes.byref(h)))
+        check(self._lib.ttt_state_create(
+            ctypes.byref(cfg), _arg(W0, "W0", torch.float32, self._nW, dev),
+            _arg(Wtarget, "Wtarget", torch.bfloat16, cfg.d_val * cfg.d_val, dev),
+            _arg(convw, "convw", torch.float32, cfg.d_val * cfg.conv_taps, dev),
+            _stream(stream), ctypes.byref(h)))
         self._h = h
 
     @property
     def handle(self) -> int:
         return self._h.value
 
+    def _scan_args(self, keys, targets, queries, out, loss_out, T, dev):
+        io, bh = self._io, self._bh
+        nk, nv = bh * T * self._dk, bh * T * self._dv
+        no = T * self._dv if self._inplace else nk
+        return (_arg(keys, "keys", io, nk, dev), _arg(targets, "targets", io, nv, dev),
+                _arg(queries, "queries", io, nk, dev), int(T), _arg(out, "out", io, no, dev),
+                _arg(loss_out, "loss_out", torch.float32, bh * T, dev))
+
     def chunk_scan(self, keys, targets, queries=None, out=None, loss_out=None, T=None, stream=None):
         """ttt_chunk_scan on device tensors; ``T`` defaults to the token dimension of keys."""
         if T is None:
             T = keys.shape[-2]
-        check(self._lib.ttt_chunk_scan(self._h, _ptr(keys), _ptr(targets), _ptr(queries), int(T),
-                                       _ptr(out), _ptr(loss_out), _stream(stream)))
+        check(self._lib.ttt_chunk_scan(self._h, *self._scan_args(keys, targets, queries, out, loss_out, T,
+                                                                 _current_device()), _stream(stream)))
 
     def chunk_scan_host(self, keys, targets, queries=None, out=None, loss_out=None, T=None, stream=None):
         """ttt_chunk_scan_host on CPU tensors (pinned for full speed); synchronises."""
         if T is None:
             T = keys.shape[-2]
-        p = lambda t: None if t is None else t.data_ptr()  # noqa: E731
-        check(self._lib.ttt_chunk_scan_host(self._h, p(keys), p(targets), p(queries), int(T), p(out),
-                                            p(loss_out), _stream(stream)))
+        check(self._lib.ttt_chunk_scan_host(self._h, *self._scan_args(keys, targets, queries, out, loss_out, T,
+                                                                      None), _stream(stream)))
 
     def surprisal_route(self, loss, T=None, stream=None):
         if T is None:
             T = loss.shape[-1]
-        check(self._lib.ttt_surprisal_route(self._h, _ptr(loss), int(T), _stream(stream)))
+        check(self._lib.ttt_surprisal_route(self._h, _arg(loss, "loss", torch.float32, self._bh * T, _current_device()),
+                                            int(T), _stream(stream)))
 
     def reset(self, stream=None):
         check(self._lib.ttt_state_reset(self._h, _stream(stream)))
 
     def get_weights(self, W, stream=None):
-        check(self._lib.ttt_state_get_weights(self._h, _ptr(W), _stream(stream)))
+        check(self._lib.ttt_state_get_weights(self._h, _arg(W, "W", torch.float32, self._nW, _current_device()),
+                                              _stream(stream)))
         return W
 
     def set_weights(self, W, stream=None):
-        check(self._lib.ttt_state_set_weights(self._h, _ptr(W), _stream(stream)))
+        check(self._lib.ttt_state_set_weights(self._h, _arg(W, "W", torch.float32, self._nW, _current_device()),
+                                              _stream(stream)))
 
     def cache_read(self, entries=None, counts=None, stream=None):
-        check(self._lib.ttt_cache_read(self._h, _ptr(entries), _ptr(counts), _stream(stream)))
+        dev = _current_device()
+        check(self._lib.ttt_cache_read(self._h, _arg(entries, "entries", torch.int32, self._bh * self._cap * 3, dev),
+                                       _arg(counts, "counts", torch.int32, self._bh * 2, dev), _stream(stream)))
 
     def gate_read(self, tau=None, tau_set=None, stream=None):
-        check(self._lib.ttt_gate_read(self._h, _ptr(tau), _ptr(tau_set), _stream(stream)))
+        dev = _current_device()
+        check(self._lib.ttt_gate_read(self._h, _arg(tau, "tau", torch.float32, self._bh, dev),
+                                      _arg(tau_set, "tau_set", torch.int32, self._bh, dev), _stream(stream)))
 
     def poll(self):
         check(self._lib.ttt_state_poll(self._h))
@@ -129,3 +179,4 @@ class FastWeightState:
             self.close()
         except Exception:
             pass
+

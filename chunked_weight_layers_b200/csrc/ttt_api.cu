@@ -398,6 +398,7 @@ ttt_status ttt_state_reset(ttt_state* st, ttt_stream stream) {
 
 ttt_status ttt_state_get_weights(const ttt_state* st, float* W, ttt_stream stream) {
   if (st == nullptr || W == nullptr) return fail(TTT_ERR_INVALID_ARG, "state and W are required");
+  TTT_TRY(check_device(st));
   const float* src = st->cfg.rule == TTT_RULE_INPLACE_HEBBIAN ? st->ip.W : st->lin.W;
   TTT_CUDA(cudaMemcpyAsync(W, src, weight_elems(st->cfg) * 4, cudaMemcpyDeviceToDevice,
                            reinterpret_cast<cudaStream_t>(stream)));
@@ -413,6 +414,7 @@ ttt_status ttt_state_set_weights(ttt_state* st, const float* W, ttt_stream strea
 ttt_status ttt_cache_read(const ttt_state* st, int32_t* entries, int32_t* counts, ttt_stream stream) {
   if (st == nullptr) return fail(TTT_ERR_INVALID_ARG, "state is NULL");
   if (st->cfg.rule != TTT_RULE_LINEAR_GD) return fail(TTT_ERR_UNSUPPORTED, "In-Place states have no residual cache");
+  TTT_TRY(check_device(st));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const size_t bh = (size_t)st->cfg.batch * st->cfg.heads;
   if (entries != nullptr)
@@ -424,6 +426,7 @@ ttt_status ttt_cache_read(const ttt_state* st, int32_t* entries, int32_t* counts
 ttt_status ttt_gate_read(const ttt_state* st, float* tau, int32_t* tau_set, ttt_stream stream) {
   if (st == nullptr) return fail(TTT_ERR_INVALID_ARG, "state is NULL");
   if (st->cfg.rule != TTT_RULE_LINEAR_GD) return fail(TTT_ERR_UNSUPPORTED, "In-Place states have no gate");
+  TTT_TRY(check_device(st));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const size_t bh = (size_t)st->cfg.batch * st->cfg.heads;
   if (tau != nullptr) TTT_CUDA(cudaMemcpyAsync(tau, st->gate.tau, bh * 4, cudaMemcpyDeviceToDevice, s));

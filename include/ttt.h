@@ -34,6 +34,9 @@
  *    ttt_chunk_scan_host() and ttt_state_destroy().
  *  - A call returns TTT_OK or an error status and never aborts the process. The message
  *    of the last error on the calling thread is returned by ttt_last_error_string().
+ *  - Every call that takes a state must be made with the state's device current
+ *    (else INVALID_ARG). Calls on one state must not run concurrently from several host
+ *    threads; different states are independent.
  *  - Failures detected on the device (a bounded wait that ran out, a failed device-side
  *    check) are recorded in the state's status word and returned by the next call of
  *    ttt_state_poll().

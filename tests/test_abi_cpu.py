@@ -79,3 +79,62 @@ def _load_fresh(path):
         return abi.load(path)
     finally:
         abi._lib = saved
+
+
+def test_binding_checks_buffers_before_any_call():
+    """The binding's per-tensor check (element type, element count, contiguity, device) runs
+    before the C call and names the offending argument; host tensors pass only where a host
+    buffer is expected."""
+    import torch
+    from chunked_weight_layers_b200 import _arg
+    t = torch.zeros(4, 16, dtype=torch.bfloat16)
+    assert _arg(None, "x", torch.bfloat16, 64, None) is None
+    assert _arg(t, "keys", torch.bfloat16, 64, None) == t.data_ptr()
+    assert _arg(t, "keys", torch.bfloat16, 32, None) == t.data_ptr()  # larger buffers are fine
+    with pytest.raises(ValueError, match="keys: .*at least 65 elements"):
+        _arg(t, "keys", torch.bfloat16, 65, None)
+    with pytest.raises(ValueError, match="targets: .*torch.float32"):
+        _arg(t, "targets", torch.float32, 64, None)
+    with pytest.raises(ValueError, match="not contiguous"):
+        _arg(t.t(), "out", torch.bfloat16, 64, None)
+    with pytest.raises(ValueError, match="on cuda:0, got .* on cpu"):
+        _arg(t, "keys", torch.bfloat16, 64, 0)
+
+
+def test_binding_element_counts_follow_the_config(monkeypatch):
+    """The counts the binding demands are those include/ttt.h states for each rule's buffers."""
+    import torch
+    import chunked_weight_layers_b200 as cwl
+    seen = {}
+
+    def fake_arg(t, name, dtype, numel, dev):
+        seen[name] = (dtype, numel)
+        return None
+
+    monkeypatch.setattr(cwl, "_arg", fake_arg)
+    cases = [
+        # TTT-Linear, B=2, H=3, gate on with 8 cache entries, T=64: [B,H,T,64] io, [B,H,T] loss.
+        (dict(rule=1, io_dtype=1, batch=2, heads=3, d_key=64, d_val=64, chunk=16, gate_enable=1,
+              cache_capacity=8), 64,
+         dict(keys=24576, targets=24576, queries=24576, out=24576, loss_out=384), 24576, 8),
+        # TTT-Linear without the gate: the library keeps a one-entry cache per pair.
+        (dict(rule=1, io_dtype=1, batch=1, heads=5, d_key=64, d_val=64, chunk=16, gate_enable=0,
+              cache_capacity=256), 32,
+         dict(keys=10240, targets=10240, queries=10240, out=10240, loss_out=160), 20480, 1),
+        # In-Place bf16, f=512, d=256, T=384: Z [T,f], V̂ or X0 [T,d], O [T,d], W [d,f].
+        (dict(rule=0, io_dtype=1, batch=1, heads=1, d_key=512, d_val=256, chunk=128), 384,
+         dict(keys=196608, targets=98304, out=98304), 131072, 1),
+        # In-Place fp32 with the same widths.
+        (dict(rule=0, io_dtype=0, batch=1, heads=1, d_key=512, d_val=256, chunk=128), 384,
+         dict(keys=196608, targets=98304, out=98304), 131072, 1),
+    ]
+    for fields, T, want, nW, cap in cases:
+        cfg = cwl.abi.ttt_config(**fields)
+        st = object.__new__(cwl.FastWeightState)
+        st._inplace, st._io, st._bh, st._dk, st._dv, st._nW, st._cap = cwl._layout(cfg)
+        assert (st._nW, st._cap) == (nW, cap)
+        seen.clear()
+        st._scan_args(None, None, None, None, None, T, 0)
+        io = torch.float32 if fields["io_dtype"] == 0 else torch.bfloat16
+        for name, n in want.items():
+            assert seen[name] == (torch.float32 if name == "loss_out" else io, n), (fields, name)
