@@ -4,8 +4,8 @@
 Default workload: the TTT-Linear mini-batch scan, B=8 sequences x H=12 heads of width 64,
 T=2048, inner mini-batch 16 (TTT layers page). A step is one ttt_chunk_scan over the whole
 batch with inputs resident in HBM; the state is reset (ttt_state_reset, untimed) before
-each step so every step scans from W0. L2 is flushed (a 512 MB write) before each timed
-step. The other four workloads (In-Place fp32, In-Place 4B-class, In-Place 128k with fused
+each step so every step scans from W0. L2 is flushed before each timed step (a 512 MB
+write, read back so the step does not pay for writing the flush's dirty lines to HBM). The other four workloads (In-Place fp32, In-Place 4B-class, In-Place 128k with fused
 target, SR-TTT gate) are measured the same way and reported under "workloads".
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--workload NAME]
@@ -121,6 +121,14 @@ class Runner:
         return h
 
 
+def evict_l2(flush):
+    """Untimed, before each timed step: write the 512 MB buffer (evicts every input line from
+    the 126 MB L2), then read it back, so the lines the L2 holds when the step starts are clean
+    and the step is not charged for writing the flush's own dirty lines back to HBM."""
+    flush.fill_(1)
+    torch.sum(flush)
+
+
 def time_steps(runner, steps, warmup, flush):
     stream = torch.cuda.current_stream()
     for _ in range(warmup):
@@ -133,7 +141,7 @@ def time_steps(runner, steps, warmup, flush):
     launches = 0
     for _ in range(steps):
         runner.state.reset()
-        flush.fill_(1)  # evict L2 (untimed)
+        evict_l2(flush)
         n0 = runner.state.launch_count()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
@@ -335,7 +343,7 @@ def bench_config(spec, world) -> dict:
     return {"workload": spec.name, "B": getattr(spec, "B", 1), "H": getattr(spec, "H", 1), "T": spec.T,
             "chunk": getattr(spec, "b", getattr(spec, "C", None)),
             "parallelism": f"replicas{world}" if world > 1 else "single",
-            "l2": "flushed before every timed step (512 MB write)"}
+            "l2": "flushed before every timed step (512 MB write, then read back so no dirty line remains)"}
 
 
 def spec_by_name(name):
@@ -425,7 +433,7 @@ def main():
     with ClockSampler(local) as clk:
         for _ in range(a.steps):
             runner.state.reset()
-            flush.fill_(1)
+            evict_l2(flush)
             n0 = runner.state.launch_count()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
