@@ -244,6 +244,14 @@ static ttt_status check_device(const ttt_state* st) {
   return TTT_OK;
 }
 
+// Cache entries hold the token position since the last reset as int32: a gated call must not
+// take it past INT32_MAX.
+static ttt_status check_token_position(const ttt_state* st, int64_t T) {
+  if (st->gate.t_offset + T > (int64_t)INT32_MAX)
+    return fail(TTT_ERR_UNSUPPORTED, "the gate's token position would pass 2^31 - 1 (reset the state first)");
+  return TTT_OK;
+}
+
 static ttt_status scan_impl(ttt_state* st, const void* keys, const void* targets, const void* queries,
                             int64_t T, void* out, float* loss, cudaStream_t s) {
   const ttt_config& c = st->cfg;
@@ -278,6 +286,7 @@ static ttt_status scan_impl(ttt_state* st, const void* keys, const void* targets
   if (c.gate_enable) {
     if (loss == nullptr) return fail(TTT_ERR_INVALID_ARG, "the gate needs loss_out");
     if (T % c.gate_chunk != 0) return fail(TTT_ERR_INVALID_ARG, "T must be a multiple of gate_chunk with the gate on");
+    TTT_TRY(check_token_position(st, T));
   }
   TTT_TRY(linear_scan(st, static_cast<const __nv_bfloat16*>(keys), static_cast<const __nv_bfloat16*>(targets),
                       static_cast<const __nv_bfloat16*>(queries), T, static_cast<__nv_bfloat16*>(out), loss, s));
@@ -383,6 +392,7 @@ ttt_status ttt_surprisal_route(ttt_state* st, const float* loss, int64_t T, ttt_
   if (T < 0 || T % st->cfg.gate_chunk != 0) return fail(TTT_ERR_INVALID_ARG, "T must be a non-negative multiple of gate_chunk");
   if (T == 0) return TTT_OK;
   if (loss == nullptr || !aligned16(loss)) return fail(TTT_ERR_INVALID_ARG, "loss must be a 16-byte aligned device pointer");
+  TTT_TRY(check_token_position(st, T));
   TTT_TRY(check_device(st));
   return gate_route(st, loss, T, reinterpret_cast<cudaStream_t>(stream));
 }

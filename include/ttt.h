@@ -137,7 +137,9 @@ ttt_status ttt_chunk_scan_host(ttt_state* st, const void* keys, const void* targ
 
 /* Run the surprisal gate alone on a loss array `loss` (device, fp32 [batch, heads, T]),
  * advancing the state's τ, cache and token position exactly as a gated scan would.
- * TTT-Linear states only; T must be a multiple of gate_chunk. */
+ * TTT-Linear states only; T must be a multiple of gate_chunk. The token position (stored
+ * in the cache as int32) may not pass 2^31 − 1 between resets: a gated call that would take
+ * it there (this one or ttt_chunk_scan with the gate on) returns UNSUPPORTED. */
 ttt_status ttt_surprisal_route(ttt_state* st, const float* loss, int64_t T, ttt_stream stream);
 
 /* Document boundary: W ← W0, τ unset, cache emptied (entries -1, counts 0), token
