@@ -30,8 +30,12 @@
  *    the row-major layout stated for it. The caller owns all such buffers; the library
  *    never frees or retains them beyond the call.
  *  - All work is enqueued on `stream` (a cudaStream_t; NULL is the legacy default
- *    stream). No call synchronises the device except ttt_state_poll(),
- *    ttt_chunk_scan_host() and ttt_state_destroy().
+ *    stream). Calls that synchronise: ttt_state_poll(), ttt_chunk_scan_host() and
+ *    ttt_state_destroy() always; ttt_state_create(), the first ttt_chunk_scan() of an
+ *    In-Place BF16 state (it builds and uploads its tile schedules) and a scan that must
+ *    grow a state-owned scratch buffer (longer T than before, or the first host call) may,
+ *    through cudaMalloc, cudaFree and cudaMemcpy. Steady-state scans of unchanged sizes
+ *    enqueue only.
  *  - A call returns TTT_OK or an error status and never aborts the process. The message
  *    of the last error on the calling thread is returned by ttt_last_error_string().
  *  - Every call that takes a state must be made with the state's device current
