@@ -80,8 +80,8 @@ static ttt_status validate(const ttt_config* c) {
     if (c->batch < 1 || c->heads < 1) return fail(TTT_ERR_INVALID_ARG, "TTT-Linear: batch and heads must be positive");
     if (c->d_key != 64 || c->d_val != 64)
       return fail(TTT_ERR_UNSUPPORTED, "TTT-Linear: head width must be 64 (d_key = d_val = 64)");
-    if (c->chunk < 16 || c->chunk > 64 || c->chunk % 16 != 0)
-      return fail(TTT_ERR_UNSUPPORTED, "TTT-Linear: inner mini-batch must be 16, 32, 48 or 64");
+    if (c->chunk != 16 && c->chunk != 32 && c->chunk != 64)
+      return fail(TTT_ERR_UNSUPPORTED, "TTT-Linear: inner mini-batch must be 16, 32 or 64");
     if (c->target_mode != 0) return fail(TTT_ERR_INVALID_ARG, "target_mode applies to In-Place only");
     if (c->gate_enable) {
       if (c->gate_chunk != 64) return fail(TTT_ERR_UNSUPPORTED, "gate_chunk must be 64");

@@ -78,8 +78,8 @@ typedef struct {
   int32_t batch, heads;   /* TTT-Linear: sequences and heads per sequence. In-Place: 1 and 1. */
   int32_t d_key;          /* In-Place: d_ff = f, columns of Wdown. TTT-Linear: head width (64). */
   int32_t d_val;          /* In-Place: d_model = d, rows of Wdown. TTT-Linear: head width (64). */
-  int32_t chunk;          /* In-Place: chunk C. TTT-Linear: inner mini-batch b (multiple of 16,
-                             at most 64). */
+  int32_t chunk;          /* In-Place: chunk C. TTT-Linear: inner mini-batch b (16, 32 or 64;
+                             other values are UNSUPPORTED at ttt_state_create). */
   float eta;              /* learning rate η */
   int32_t target_mode;    /* In-Place only. 0: targets are V̂ [T, d]. 1: targets are X0 [T, d]
                              and V̂ = Conv1D(X0)·Wtarget is produced inside the scan (BF16). */
