@@ -271,14 +271,29 @@ def roofline(spec, w, ms, peaks, traffic=None):
             "traffic": traffic, "peak_source": "148 SMs x 128 FP32 lanes x 2 x max SM clock"}
 
 
+def oracle_threads() -> int:
+    """Threads of the BLAS pool behind numpy's matmul, the oracle's only multi-threaded step."""
+    try:
+        import threadpoolctl
+        n = [i["num_threads"] for i in threadpoolctl.threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return max(n)
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
 def cpu_baseline(spec, limit_s=12.0) -> dict:
-    """The oracle as it stands on this host's cores, on a bounded sample of the workload."""
+    """The oracle as it stands on this host's cores, on a bounded sample of the workload.
+
+    ``cores`` is the BLAS pool the oracle's matmuls run on; ``busy_threads`` is the process's
+    CPU time over the sample's wall time, i.e. how many of them were busy on average."""
     import numpy as np  # noqa: F401
     from oracle import gate as ogate
     from oracle import inplace as oinp
     from oracle import linear as olin
-    cores = torch.get_num_threads()
-    t0 = time.perf_counter()
+    cores = oracle_threads()
+    t0, c0 = time.perf_counter(), time.process_time()
     if isinstance(spec, wl.LinearSpec):
         x = wl.linear_inputs(spec)
         done_heads = 0
@@ -287,7 +302,7 @@ def cpu_baseline(spec, limit_s=12.0) -> dict:
         V = x["V"].reshape(BH, 1, spec.T, spec.D)
         Q = x["Q"].reshape(BH, 1, spec.T, spec.D) if "Q" in x else None
         W0 = x["W0"].reshape(BH, 1, spec.D, spec.D)
-        t0 = time.perf_counter()
+        t0, c0 = time.perf_counter(), time.process_time()
         while done_heads < BH and time.perf_counter() - t0 < limit_s:
             h = done_heads
             _, _, L = olin.ttt_linear_scan(K[h:h + 1], V[h:h + 1], None if Q is None else Q[h:h + 1],
@@ -301,7 +316,7 @@ def cpu_baseline(spec, limit_s=12.0) -> dict:
     else:
         Cs = spec.C
         x = wl.inplace_inputs(wl.scaled(spec, T=min(spec.T, Cs * 2)) if spec.dtype == "bf16" else spec)
-        t0 = time.perf_counter()
+        t0, c0 = time.perf_counter(), time.process_time()
         chunks = 0
         W = x["W0"]
         Vh = x.get("Vhat")
@@ -315,8 +330,9 @@ def cpu_baseline(spec, limit_s=12.0) -> dict:
         dt = time.perf_counter() - t0
         tokens = chunks * Cs
         sample = f"{chunks} chunk(s) of {Cs} tokens"
-    return {"value": tokens / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample,
-            "seconds": dt}
+    busy = (time.process_time() - c0) / dt if dt > 0 else 0.0
+    return {"value": tokens / dt, "unit": "tokens/s", "cores": cores, "busy_threads": round(busy, 2),
+            "kind": "oracle", "sample": sample, "seconds": dt}
 
 
 def measure(spec, steps, warmup, flush, peaks, device, with_e2e):
