@@ -13,6 +13,9 @@ pages' order, with no blocking, fusion or reordering beyond the definitions:
   DeltaNet remark).
 * :mod:`oracle.gate` — SR-TTT surprisal gate and residual cache (SR-TTT technical
   summary, §2.1 "Surprisal Filter" and "Residual Cache").
+* :mod:`oracle.cache_attention` — the residual cache's read path, attention over the cached
+  keys and values fused into the TTT output through the clamped gate α (SR-TTT technical
+  summary, §2.1 "Residual Cache" and "Alpha Fusion").
 
 Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline leg may
 import it. The product path (the C-ABI library and its Python binding) never does;
@@ -22,4 +25,4 @@ Every function here is pinned by ``tests/test_oracle_*.py`` to closed forms,
 hand-derived worked examples (``tests/golden/``), special cases and brute force.
 """
 
-from . import gate, inplace, linear  # noqa: F401
+from . import cache_attention, gate, inplace, linear  # noqa: F401

@@ -73,6 +73,21 @@ MUTANTS = [
      [("                            state.dropped[bi, hi] += 1\n", "                            pass\n")]),
     ("gate", "token index ignores the stream position",
      [("(bi, hi, state.t_offset + g * gate_chunk + j)", "(bi, hi, g * gate_chunk + j)")]),
+    ("cache_attention", "entries of the query's own gate chunk visible",
+     [("visible = gc < t // gate_chunk", "visible = gc <= t // gate_chunk")]),
+    ("cache_attention", "scores not scaled by 1/sqrt(D)",
+     [("scale = 1.0 / np.sqrt(D)", "scale = 1.0")]),
+    ("cache_attention", "softmax weights not normalised",
+     [("A[bi, hi, t] = (w / w.sum()) @ vc[visible]", "A[bi, hi, t] = w @ vc[visible]")]),
+    ("cache_attention", "alpha not clamped",
+     [("a = np.clip(f64(alpha), 0.0, 1.0)", "a = f64(alpha)")]),
+    ("cache_attention", "every cache slot read, not the stored entries",
+     [("n = min(int(np.asarray(counts)[bi, hi, 0]), E.shape[2])", "n = E.shape[2]")]),
+    ("cache_attention", "keys and values swapped",
+     [("kc, vc, gc = Kd[bi, hi, ts], Vd[bi, hi, ts], ts // gate_chunk",
+       "kc, vc, gc = Vd[bi, hi, ts], Kd[bi, hi, ts], ts // gate_chunk")]),
+    ("cache_attention", "query of the previous token",
+     [("s = (kc[visible] @ Qd[bi, hi, t]) * scale", "s = (kc[visible] @ Qd[bi, hi, t - 1]) * scale")]),
 ]
 
 
@@ -108,7 +123,7 @@ def _failing_pins(module: str, impl: types.ModuleType) -> list[str]:
     return failed
 
 
-@pytest.mark.parametrize("module", ["inplace", "linear", "gate"])
+@pytest.mark.parametrize("module", ["inplace", "linear", "gate", "cache_attention"])
 def test_unmutated_oracle_passes_every_pin(module):
     assert _failing_pins(module, _load(module, [])) == []
 
