@@ -63,3 +63,48 @@ def test_two_gloo_ranks():
             p.join(timeout=120)
             assert p.exitcode == 0
         assert out[0] == (True, 2.5) and out[1] == (True, 2.5)
+
+
+def _inplace_worker(rank, world, port, out):
+    """Rank ``rank`` scans its contiguous share of Wdown's rows (W0[rows], V̂[:, rows]) on its
+    own, then the ranks all-gather their output columns; nothing else crosses ranks."""
+    import numpy as np
+    from oracle import inplace
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        rng = np.random.default_rng(7)
+        T, C, d, f, eta = 96, 32, 10, 12, 0.05
+        Z, V, W0 = rng.standard_normal((T, f)), rng.standard_normal((T, d)), 0.1 * rng.standard_normal((d, f))
+        a, b = shard_range(d, rank, world)
+        O_mine, W_mine = inplace.inplace_scan_rows(Z, V[:, a:b], W0[a:b], eta, C)
+        cols = [torch.zeros(T, n, dtype=torch.float64) for n in
+                (shard_range(d, r, world)[1] - shard_range(d, r, world)[0] for r in range(world))]
+        dist.all_gather(cols, torch.from_numpy(np.ascontiguousarray(O_mine)))
+        rows = [torch.zeros(n, f, dtype=torch.float64) for n in
+                (shard_range(d, r, world)[1] - shard_range(d, r, world)[0] for r in range(world))]
+        dist.all_gather(rows, torch.from_numpy(np.ascontiguousarray(W_mine)))
+        O = torch.cat(cols, 1).numpy()
+        W = torch.cat(rows, 0).numpy()
+        O_ref, W_ref = inplace.inplace_scan(Z, V, W0, eta, C)
+        out[rank] = bool(np.allclose(O, O_ref, rtol=0, atol=1e-12) and np.allclose(W, W_ref, rtol=0, atol=1e-12))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_inplace_rows_shard_across_two_gloo_ranks():
+    """The In-Place scan shards over Wdown's rows: two ranks with half the rows each reproduce
+    the single-process scan (to float64 rounding) after one all-gather of output columns."""
+    world = 2
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as m:
+        out = m.dict()
+        port = _free_port()
+        procs = [ctx.Process(target=_inplace_worker, args=(r, world, port, out)) for r in range(world)]
+        for p in procs:
+            p.start()
+        for p in procs:
+            p.join(timeout=120)
+            assert p.exitcode == 0
+        assert out[0] is True and out[1] is True
