@@ -16,6 +16,9 @@ pages' order, with no blocking, fusion or reordering beyond the definitions:
 * :mod:`oracle.cache_attention` — the residual cache's read path, attention over the cached
   keys and values fused into the TTT output through the clamped gate α (SR-TTT technical
   summary, §2.1 "Residual Cache" and "Alpha Fusion").
+* :mod:`oracle.packed` — packed sequences: the weight reset to its pretrained value at every
+  document start, and the update delta's Frobenius norm clipped (In-Place Test-Time
+  Training, §6 and its implementation notes).
 
 Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline leg may
 import it. The product path (the C-ABI library and its Python binding) never does;
@@ -25,4 +28,4 @@ Every function here is pinned by ``tests/test_oracle_*.py`` to closed forms,
 hand-derived worked examples (``tests/golden/``), special cases and brute force.
 """
 
-from . import cache_attention, gate, inplace, linear  # noqa: F401
+from . import cache_attention, gate, inplace, linear, packed  # noqa: F401

@@ -1,0 +1,93 @@
+"""Oracle of packed sequences: per-document resets and update-norm clipping (float64) — test
+infrastructure only.
+
+Source: "In-Place Test-Time Training" (blog summary of arXiv 2604.06169), §6 "context
+parallelism" and the implementation notes that follow it:
+
+* when an independent document ends, the fast weight goes back to its pretrained state, so
+  nothing leaks from one document into the next;
+* the Frobenius norm of the update delta is clipped (the page's threshold reads 1e-5), so a
+  long run of updates cannot flood the weight.
+
+The TTT layers page gives the same boundary for TTT-Linear: the recurrent state is the inner
+model's weight, restarted for a new sequence.
+
+Readings taken where the pages leave it open (a CUDA path must apply the same ones):
+
+* a packed sequence is documents laid end to end; ``doc_starts`` lists each document's first
+  token (the first is 0). Every document is scanned as if alone: the weight starts from W0,
+  chunks (In-Place) or inner mini-batches (TTT-Linear) are counted from the document's first
+  token, and a document's last chunk or mini-batch may be shorter;
+* a shorter last TTT-Linear mini-batch of b' tokens takes the gradient step of its own loss
+  1/(2b')·‖K·W − V‖², i.e. W ← W − (η/b')·Kᵀ(K·W − V);
+* clipping acts on each chunk's delta ΔW_c = η·V̂_cᵀ·Z_c on its own: if ‖ΔW_c‖_F exceeds the
+  threshold, ΔW_c is scaled to that norm; the threshold is a parameter (None: no clipping).
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+from ._util import f64
+
+
+def _documents(doc_starts, T: int):
+    starts = [int(s) for s in doc_starts]
+    if not starts or starts[0] != 0 or any(b <= a for a, b in zip(starts, starts[1:])) or starts[-1] >= T:
+        raise ValueError("doc_starts must start at 0, increase strictly and lie below T")
+    return list(zip(starts, starts[1:] + [T]))
+
+
+def clip_delta(dW, clip):
+    """ΔW scaled to Frobenius norm ``clip`` when it is larger (unchanged otherwise)."""
+    if clip is None:
+        return dW
+    n = float(np.sqrt(np.sum(dW * dW)))
+    return dW * (clip / n) if n > clip else dW
+
+
+def inplace_scan_docs(Z, Vhat, W0, eta: float, C: int, doc_starts, clip=None):
+    """Apply-then-update over each document of a packed sequence, W reset to W0 at each start.
+
+    Z [T, f], Vhat [T, d], W0 [d, f]. Returns (O [T, d], W after the last document [d, f])."""
+    Zd, Vd, W0d = f64(Z), f64(Vhat), f64(W0)
+    T = Zd.shape[0]
+    O = np.empty((T, W0d.shape[0]))
+    W = W0d
+    for a, e in _documents(doc_starts, T):
+        W = W0d.copy()                                   # document boundary: pretrained weight
+        for c0 in range(a, e, C):
+            rows = slice(c0, min(c0 + C, e))
+            O[rows] = Zd[rows] @ W.T                     # apply first
+            W = W + clip_delta(eta * (Vd[rows].T @ Zd[rows]), clip)   # then update
+    return O, W
+
+
+def ttt_linear_scan_docs(K, V, Q, W0, eta: float, b: int, doc_starts):
+    """TTT-Linear over packed sequences; ``doc_starts[s]`` lists sequence s's document starts.
+
+    K, V, Q [B, H, T, D] (Q may be None), W0 [B, H, D, D]. Returns (O or None, W after each
+    sequence's last document [B, H, D, D], loss [B, H, T])."""
+    Kd, Vd = f64(K), f64(V)
+    Qd = None if Q is None else f64(Q)
+    W0d = f64(W0)
+    B, H, T, D = Kd.shape
+    O = None if Qd is None else np.empty((B, H, T, D))
+    loss = np.empty((B, H, T))
+    Wout = np.empty((B, H, D, D))
+    for s in range(B):
+        docs = _documents(doc_starts[s], T)
+        for h in range(H):
+            W = W0d[s, h]
+            for a, e in docs:
+                W = W0d[s, h].copy()                     # document boundary: W ← W0
+                for i0 in range(a, e, b):
+                    r = slice(i0, min(i0 + b, e))
+                    n = r.stop - r.start                 # b, or fewer for the last mini-batch
+                    if Qd is not None:
+                        O[s, h, r] = Qd[s, h, r] @ W     # outputs with the mini-batch's start W
+                    R = Kd[s, h, r] @ W - Vd[s, h, r]
+                    loss[s, h, r] = np.sum(R * R, axis=1)
+                    W = W - (eta / n) * (Kd[s, h, r].T @ R)
+            Wout[s, h] = W
+    return O, Wout, loss

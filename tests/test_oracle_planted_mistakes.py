@@ -88,6 +88,15 @@ MUTANTS = [
        "kc, vc, gc = Vd[bi, hi, ts], Kd[bi, hi, ts], ts // gate_chunk")]),
     ("cache_attention", "query of the previous token",
      [("s = (kc[visible] @ Qd[bi, hi, t]) * scale", "s = (kc[visible] @ Qd[bi, hi, t - 1]) * scale")]),
+    ("packed", "In-Place weight not reset at a document start",
+     [("        W = W0d.copy()                                   # document boundary: pretrained weight\n",
+       "")]),
+    ("packed", "TTT-Linear weight not reset at a document start",
+     [("                W = W0d[s, h].copy()                     # document boundary: W ← W0\n", "")]),
+    ("packed", "clipping enlarges small deltas instead of shrinking large ones",
+     [("return dW * (clip / n) if n > clip else dW", "return dW * (clip / n) if n < clip else dW")]),
+    ("packed", "short last mini-batch divided by b instead of its own size",
+     [("W = W - (eta / n) * (Kd[s, h, r].T @ R)", "W = W - (eta / b) * (Kd[s, h, r].T @ R)")]),
 ]
 
 
@@ -123,7 +132,7 @@ def _failing_pins(module: str, impl: types.ModuleType) -> list[str]:
     return failed
 
 
-@pytest.mark.parametrize("module", ["inplace", "linear", "gate", "cache_attention"])
+@pytest.mark.parametrize("module", ["inplace", "linear", "gate", "cache_attention", "packed"])
 def test_unmutated_oracle_passes_every_pin(module):
     assert _failing_pins(module, _load(module, [])) == []
 
