@@ -52,3 +52,33 @@ def test_reference_arm_under_torchrun_prints_one_line():
     assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["scaling"] == "weak"
     assert line["config"]["parallelism"] == "replicas2"
     assert line["config"]["workload"] == "ttt_linear_B8_H12_T2048_b16"
+
+
+def test_algorithmic_work_per_workload():
+    """The flops and compulsory bytes the roofline divides by, per workload, from each
+    workload's definition: In-Place 4·T·d·f flops (+ 2·T·d² for the fused target), Z, V̂ (or
+    X0) read and O written once, W0 read and W written once in fp32; TTT-Linear 6·d²·T per
+    (sequence, head) with queries (4·d²·T without), K, V (, Q) read and O written once in bf16,
+    fp32 W0 and W, plus the losses and the cache with the gate."""
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    from gen import workloads as wl
+    MB = 1e6
+    want = {
+        "inplace_fp32_T2048_C512_d256_f512": (4 * 2048 * 256 * 512, 2048 * 512 * 4 + 2 * 2048 * 256 * 4 + 2 * 256 * 512 * 4),
+        "ttt_linear_B8_H12_T2048_b16": (6 * 64 * 64 * 2048 * 96, 4 * 96 * 2048 * 64 * 2 + 2 * 96 * 64 * 64 * 4),
+        "inplace_bf16_T32768_C1024_d2560_f9728": (4 * 32768 * 2560 * 9728,
+                                                  32768 * 9728 * 2 + 2 * 32768 * 2560 * 2 + 2 * 2560 * 9728 * 4),
+        "inplace_bf16_target_T131072_C1024_d2560_f9728": (
+            4 * 131072 * 2560 * 9728 + 2 * 131072 * 2560 * 2560,
+            131072 * 9728 * 2 + 2 * 131072 * 2560 * 2 + 2 * 2560 * 9728 * 4 + 2560 * 2560 * 2 + 2560 * 3 * 4),
+        "srttt_gate_B4_H16_T8192_b16": (4 * 64 * 64 * 8192 * 64,
+                                        2 * 64 * 8192 * 64 * 2 + 2 * 64 * 64 * 64 * 4 + 64 * 8192 * 4 + 64 * (256 * 3 + 2) * 4),
+    }
+    for name, (flops, byts) in want.items():
+        w = bench.work(wl.WORKLOADS[name])
+        assert w["flops"] == flops and w["bytes"] == byts, name
+    # The figures quoted for the workloads: 4.83 GFLOP / 103.8 MB and 3.264 TFLOP / 1.17 GB.
+    assert round(bench.work(wl.LINEAR_GD)["bytes"] / MB, 1) == 103.8
+    assert round(bench.work(wl.INPLACE_4B)["flops"] / 1e12, 3) == 3.264
