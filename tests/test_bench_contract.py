@@ -32,7 +32,7 @@ def test_reference_arm_line():
     assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
 
 
-def test_reference_arm_under_torchrun_prints_one_line():
+def test_reference_arm_under_torchrun_prints_one_line(tmp_path):
     """Launched as the driver launches N > 1 (torch.distributed.run, two ranks on 127.0.0.1):
     rank 0 alone runs the oracle and prints the line; the other rank exits 0 without work."""
     import socket
@@ -40,7 +40,7 @@ def test_reference_arm_under_torchrun_prints_one_line():
     s.bind(("127.0.0.1", 0))
     port = s.getsockname()[1]
     s.close()
-    env = dict(os.environ, OMP_NUM_THREADS="1")
+    env = dict(os.environ, OMP_NUM_THREADS="1", TMPDIR=str(tmp_path))  # the launcher's scratch stays in tmp_path
     out = subprocess.run([sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
                           "--master-addr", "127.0.0.1", "--master-port", str(port), "bench.py", "--impl", "reference",
                           "--gpus", "2", "--steps", "1", "--warmup", "0"],
