@@ -3,10 +3,12 @@
 
 Default workload: the TTT-Linear mini-batch scan, B=8 sequences x H=12 heads of width 64,
 T=2048, inner mini-batch 16 (TTT layers page). A step is one ttt_chunk_scan over the whole
-batch with inputs resident in HBM; the state is reset (ttt_state_reset, untimed) before
-each step so every step scans from W0. L2 is flushed before each timed step (a 512 MB
-write, read back so the step does not pay for writing the flush's dirty lines to HBM). The other four workloads (In-Place fp32, In-Place 4B-class, In-Place 128k with fused
-target, SR-TTT gate) are measured the same way and reported under "workloads".
+batch with inputs resident in HBM. The K timed steps run back to back between two CUDA
+events (the state is reset once before the warm-up; consecutive steps continue one scan, as
+successive calls do) and take their inputs from copies whose total is over three times the
+126 MB L2, so every step reads from HBM rather than from L2. The other four workloads
+(In-Place fp32, In-Place 4B-class, In-Place 128k with fused target, SR-TTT gate) are
+measured the same way and reported under "workloads".
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--workload NAME]
                   [--only-main]
@@ -81,8 +83,17 @@ def fp32_alu_peak_tflops(peaks) -> float:
 # GPU arm
 # --------------------------------------------------------------------------------------------
 
+L2_BYTES = 126 * 2**20
+
+
 class Runner:
-    """Builds the state and inputs of one workload and runs timed steps."""
+    """Builds the state and inputs of one workload and runs its steps.
+
+    A step is one ttt_chunk_scan over the whole batch. Consecutive steps continue one scan
+    (the state is not reset between them) and take their inputs and outputs from ``n_sets``
+    copies in turn, enough copies that together they are over three times the 126 MB L2:
+    by the time a copy comes round again, the steps in between have moved more than the L2
+    holds, so every step reads its inputs from HBM."""
 
     def __init__(self, spec, device):
         import chunked_weight_layers_b200 as cwl
@@ -94,24 +105,31 @@ class Runner:
             cfg = cwl.config("linear", batch=spec.B, heads=spec.H, chunk=spec.b, eta=spec.eta,
                              gate_enable=int(spec.gate))
             self.state = cwl.FastWeightState(cfg, x["W0"])
-            self.args = dict(keys=x["K"], targets=x["V"], queries=x.get("Q"))
-            self.out = torch.empty_like(x["K"]) if spec.with_queries else None
-            self.loss = (torch.empty((spec.B, spec.H, spec.T), device=device, dtype=torch.float32)
-                         if spec.gate else None)
+            args = dict(keys=x["K"], targets=x["V"], queries=x.get("Q"))
+            out = torch.empty_like(x["K"]) if spec.with_queries else None
+            loss = (torch.empty((spec.B, spec.H, spec.T), device=device, dtype=torch.float32)
+                    if spec.gate else None)
         else:
             x = wl.inplace_inputs(spec, device=device)
             io = 0 if spec.dtype == "f32" else 1
             cfg = cwl.config("inplace", io_dtype=io, d_key=spec.f, d_val=spec.d, chunk=spec.C, eta=spec.eta,
                              target_mode=int(spec.target), conv_pad_mode=spec.conv_pad_mode)
             self.state = cwl.FastWeightState(cfg, x["W0"], x.get("Wtarget"), x.get("convw"))
-            self.args = dict(keys=x["Z"], targets=x["X0"] if spec.target else x["Vhat"], queries=None)
-            self.out = torch.empty((spec.T, spec.d), device=device, dtype=x["Z"].dtype)
-            self.loss = None
+            args = dict(keys=x["Z"], targets=x["X0"] if spec.target else x["Vhat"], queries=None)
+            out = torch.empty((spec.T, spec.d), device=device, dtype=x["Z"].dtype)
+            loss = None
         self.inputs = x
+        step_bytes = work(spec)["bytes"]
+        self.n_sets = max(1, -(-3 * L2_BYTES // step_bytes))
+        clone = lambda t: None if t is None else t.clone()  # noqa: E731
+        self.sets = [(args, out, loss)] + [
+            ({k: clone(v) for k, v in args.items()}, clone(out), clone(loss)) for _ in range(self.n_sets - 1)]
+        self.args, self.out, self.loss = self.sets[0]
+        self.set_bytes = self.n_sets * step_bytes
 
-    def step(self):
-        self.state.chunk_scan(self.args["keys"], self.args["targets"], self.args["queries"], out=self.out,
-                              loss_out=self.loss, T=self.spec.T)
+    def step(self, i=0):
+        a, out, loss = self.sets[i % self.n_sets]
+        self.state.chunk_scan(a["keys"], a["targets"], a["queries"], out=out, loss_out=loss, T=self.spec.T)
 
     def host_buffers(self):
         pin = lambda t: None if t is None else t.cpu().pin_memory()  # noqa: E731
@@ -120,40 +138,48 @@ class Runner:
         h["loss"] = None if self.loss is None else torch.empty(self.loss.shape, dtype=torch.float32).pin_memory()
         return h
 
-
-def evict_l2(flush):
-    """Untimed, before each timed step: write the 512 MB buffer (evicts every input line from
-    the 126 MB L2), then read it back, so the lines the L2 holds when the step starts are clean
-    and the step is not charged for writing the flush's own dirty lines back to HBM."""
-    flush.fill_(1)
-    torch.sum(flush)
+    def l2_note(self):
+        return (f"inputs larger than L2: {self.n_sets} copies of the step's inputs and outputs "
+                f"({self.set_bytes / 2**20:.0f} MiB in all) taken in turn, so each step reads from HBM")
 
 
-def time_steps(runner, steps, warmup, flush):
+def timed_pass(runner, steps, stream):
+    """EXACTLY ``steps`` back-to-back steps between two CUDA events on the launching stream
+    (synchronised on both sides): total ms and library launches. A second pass with an event
+    between every two steps gives the per-step times (for the median); it is not the value."""
+    torch.cuda.synchronize()
+    n0 = runner.state.launch_count()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    h0 = time.perf_counter()
+    for k in range(steps):
+        runner.step(k)
+    runner.host_ms = (time.perf_counter() - h0) * 1e3 / max(1, steps)  # host time to enqueue one step
+    e1.record(stream)
+    e1.synchronize()
+    total = e0.elapsed_time(e1)
+    launches = runner.state.launch_count() - n0
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    ev[0].record(stream)
+    for k in range(steps):
+        runner.step(k)
+        ev[k + 1].record(stream)
+    ev[-1].synchronize()
+    per_step = [ev[k].elapsed_time(ev[k + 1]) for k in range(steps)]
+    torch.cuda.synchronize()
+    return total, launches, per_step
+
+
+def time_steps(runner, steps, warmup):
     stream = torch.cuda.current_stream()
-    for _ in range(warmup):
-        runner.state.reset()
-        runner.step()
+    runner.state.reset()
+    for k in range(warmup):
+        runner.step(k)
     torch.cuda.synchronize()
     runner.state.poll()
-    times = []
-    l0 = runner.state.launch_count()
-    launches = 0
-    for _ in range(steps):
-        runner.state.reset()
-        evict_l2(flush)
-        n0 = runner.state.launch_count()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        runner.step()
-        e1.record(stream)
-        launches += runner.state.launch_count() - n0
-        e1.synchronize()
-        times.append(e0.elapsed_time(e1))
-    torch.cuda.synchronize()
+    total, launches, per_step = timed_pass(runner, steps, stream)
     runner.state.poll()
-    del l0
-    return times, launches
+    return total, launches, per_step
 
 
 def time_e2e(runner, steps, warmup):
@@ -182,7 +208,8 @@ def time_e2e(runner, steps, warmup):
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples every 200 ms while the timed region runs."""
+    """nvidia-smi clock / throttle-reason samples every 50 ms from the start of the main timed
+    region until every workload has been measured."""
 
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -199,7 +226,7 @@ class ClockSampler:
             os.close(fd)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+                 "-lms", "50"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
             time.sleep(0.3)
         except Exception:
             self.proc = None
@@ -235,7 +262,7 @@ class ClockSampler:
 def dominant_kernel(spec) -> str:
     if isinstance(spec, wl.LinearSpec):
         return "k_linear_b16" if spec.b == 16 else "k_linear_scan"
-    return "k_sgemm" if spec.dtype == "f32" else "k_inplace_tc"
+    return "k_f32_chunk" if spec.dtype == "f32" else "k_inplace_tc"
 
 
 def traffic_per_launch(spec):
@@ -335,22 +362,32 @@ def cpu_baseline(spec, limit_s=12.0) -> dict:
             "kind": "oracle", "sample": sample, "seconds": dt}
 
 
-def measure(spec, steps, warmup, flush, peaks, device, with_e2e):
+def measure(spec, steps, warmup, peaks, device, with_e2e, cpu_limit_s=None):
+    """One workload measured like the main line: device time per scan (mean over the timed
+    steps, median beside it), its roofline, end-to-end time through the host-buffer call, and
+    (with ``cpu_limit_s``) the oracle on a bounded sample of it."""
     r = Runner(spec, device)
-    times, launches = time_steps(r, steps, warmup, flush)
-    ms = statistics.mean(times)
+    total, launches, times = time_steps(r, steps, warmup)
+    ms = total / steps
     w = work(spec)
-    out = {"workload": spec.name, "ms_per_step": ms, "tokens_per_s": w["tokens"] / (ms * 1e-3),
-           "tflops": w["flops"] / (ms * 1e-3) / 1e12,
-           "roofline": roofline(spec, w, ms, peaks, traffic_per_launch(spec)),
-           "gpu_launches_per_step": launches / max(1, steps), "times_ms": times}
+    rl = roofline(spec, w, ms, peaks, traffic_per_launch(spec))
+    rl["kernel"] = dominant_kernel(spec)
+    out = {"workload": spec.name, "ms_per_step": ms, "ms_median": statistics.median(times),
+           "tokens_per_s": w["tokens"] / (ms * 1e-3), "tflops": w["flops"] / (ms * 1e-3) / 1e12,
+           "roofline": rl, "gpu_launches_per_step": launches / max(1, steps), "times_ms": times,
+           "host_ms_per_step": r.host_ms, "l2": r.l2_note()}
     if with_e2e:
-        e2e_ms, h2d, d2h = time_e2e(r, max(3, steps // 2), 1)
-        out["e2e"] = {"value": w["tokens"] / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                      "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+        try:
+            e2e_ms, h2d, d2h = time_e2e(r, max(3, min(steps, 10) // 2), 1)
+            out["e2e"] = {"value": w["tokens"] / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                          "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+        except Exception as ex:  # report, do not hide
+            out["e2e"] = {"error": str(ex)}
     r.state.close()
     del r
     torch.cuda.empty_cache()
+    if cpu_limit_s is not None:
+        out["cpu_baseline"] = cpu_baseline(spec, cpu_limit_s)
     return out
 
 
@@ -359,7 +396,7 @@ def bench_config(spec, world) -> dict:
     return {"workload": spec.name, "B": getattr(spec, "B", 1), "H": getattr(spec, "H", 1), "T": spec.T,
             "chunk": getattr(spec, "b", getattr(spec, "C", None)),
             "parallelism": f"replicas{world}" if world > 1 else "single",
-            "l2": "flushed before every timed step (512 MB write, then read back so no dirty line remains)"}
+            "l2": "inputs larger than L2: copies of the step's inputs taken in turn (over 3x the 126 MB L2)"}
 
 
 def spec_by_name(name):
@@ -432,38 +469,26 @@ def main():
         build.build()
     if pg is not None:
         pg.barrier()
-    flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=device)
-
     runner = Runner(spec, device)
-    for _ in range(a.warmup):
-        runner.state.reset()
-        runner.step()
+    runner.state.reset()
+    for k in range(a.warmup):
+        runner.step(k)
     torch.cuda.synchronize()
     runner.state.poll()
     stream = torch.cuda.current_stream()
-    times = []
-    launches = 0
     if pg is not None:
         pg.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
-        for _ in range(a.steps):
-            runner.state.reset()
-            evict_l2(flush)
-            n0 = runner.state.launch_count()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            runner.step()
-            e1.record(stream)
-            launches += runner.state.launch_count() - n0
-            e1.synchronize()
-            times.append(e0.elapsed_time(e1))
-        torch.cuda.synchronize()
+    clk = ClockSampler(local)
+    clk.__enter__()
+    total, launches, times = timed_pass(runner, a.steps, stream)
     if pg is not None:
         pg.barrier()
     runner.state.poll()
+    l2_note = runner.l2_note()
+    host_ms = runner.host_ms
     from chunked_weight_layers_b200.dist import max_over_ranks
-    total_ms = max_over_ranks(sum(times), device)
+    total_ms = max_over_ranks(total, device)
     ms = total_ms / a.steps
     value = world * w["tokens"] / (ms * 1e-3)
     e2e_ms, h2d, d2h = None, 0, 0
@@ -479,29 +504,39 @@ def main():
     del runner
     torch.cuda.empty_cache()
 
+    # The other four workloads, each a full measurement of its own (device time, roofline,
+    # end-to-end through the host-buffer call, oracle baseline on a bounded sample). The clock
+    # sampler keeps running through them, so its samples cover the whole of the GPU's work.
     extra = {}
     if not a.only_main and world == 1:
         for s in wl.WORKLOADS.values():
             if s.name == spec.name:
                 continue
             try:
-                extra[s.name] = measure(s, max(5, min(a.steps, 10)), 3, flush, peaks, device, with_e2e=False)
+                extra[s.name] = measure(s, max(5, min(a.steps, 20)), 3, peaks, device, with_e2e=True)
             except Exception as ex:
                 extra[s.name] = {"error": str(ex)}
+    clk.__exit__(None, None, None)
+    # The oracle baselines run after the sampler stops (the GPU idles meanwhile).
+    for s in wl.WORKLOADS.values():
+        if s.name in extra and "error" not in extra[s.name]:
+            extra[s.name]["cpu_baseline"] = cpu_baseline(s, 6.0)
 
     if rank == 0:
         rl = roofline(spec, w, ms, peaks, traffic_per_launch(spec))
         rl["kernel"] = dominant_kernel(spec)
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": a.steps,
-            "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "warmup": a.warmup, "ms_per_step": ms, "ms_median": statistics.median(times),
+            "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": bench_config(spec, world),
+            "config": dict(bench_config(spec, world), l2=l2_note),
             "tflops": world * w["flops"] / (ms * 1e-3) / 1e12,
             "roofline": rl,
             "e2e": {"value": runner_e2e, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_ms},
             "gpu_launches": launches,
+            "host_ms_per_step": host_ms,
             "clocks": clk.summary(peaks["sm_max_mhz"]),
         }
         if world == 1:

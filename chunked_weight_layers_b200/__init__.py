@@ -163,6 +163,10 @@ class FastWeightState:
         check(self._lib.ttt_gate_read(self._h, _arg(tau, "tau", torch.float32, self._bh, dev),
                                       _arg(tau_set, "tau_set", torch.int32, self._bh, dev), _stream(stream)))
 
+    def set_option(self, option: int, value: int):
+        """ttt_state_set_option (e.g. ``abi.TTT_OPT_LINEAR_CHUNK``)."""
+        check(self._lib.ttt_state_set_option(self._h, int(option), int(value)))
+
     def poll(self):
         check(self._lib.ttt_state_poll(self._h))
 

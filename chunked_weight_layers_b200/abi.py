@@ -28,6 +28,10 @@ TTT_RULE_LINEAR_GD = 1
 TTT_F32 = 0
 TTT_BF16 = 1
 
+TTT_OPT_LINEAR_CHUNK = 1
+TTT_OPT_WAIT_LIMIT_NS = 2
+TTT_OPT_INJECT_STALL = 3
+
 
 class ttt_config(ctypes.Structure):
     _fields_ = [
@@ -67,12 +71,13 @@ _SIGNATURES = {
     "ttt_state_set_weights": (_st, [_vp, _vp, _vp]),
     "ttt_cache_read": (_st, [_vp, _vp, _vp, _vp]),
     "ttt_gate_read": (_st, [_vp, _vp, _vp, _vp]),
+    "ttt_state_set_option": (_st, [_vp, ctypes.c_int32, ctypes.c_int64]),
     "ttt_state_poll": (_st, [_vp]),
     "ttt_state_launch_count": (ctypes.c_int64, [_vp]),
     "ttt_state_destroy": (_st, [_vp]),
     "ttt_last_error_string": (ctypes.c_char_p, []),
     "ttt_target_values_noalloc": (_st, [_vp, _vp, _vp, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
-                                        ctypes.c_int32, ctypes.c_int32, _vp, _vp]),
+                                        ctypes.c_int32, ctypes.c_int32, _vp, _vp, _vp]),
 }
 
 _lib = None

@@ -12,13 +12,22 @@ namespace ttt {
 constexpr int kDevTimeout = 5;
 constexpr int kDevCheck = 6;
 
-// Every spin-wait in this library gives up after this many nanoseconds of %globaltimer,
-// records TTT_ERR_TIMEOUT in the state's status word and lets the kernel wind down.
+// Every spin-wait in this library gives up after a limit of %globaltimer nanoseconds (by
+// default this many; a state can set its own), records TTT_ERR_TIMEOUT in the state's status
+// word and lets the kernel wind down.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+// Where a kernel reports a failure, and how long each of its spin-waits may last.
+struct DevStatus {
+  int* word;          // status word (mapped host memory or device memory), or null
+  uint64_t limit_ns;  // wait limit in %globaltimer nanoseconds
+};
 
 __device__ __forceinline__ void record_status(int* status, int code) {
   if (status != nullptr) atomicCAS(status, 0, code);
 }
+
+__device__ __forceinline__ void record_status(const DevStatus& status, int code) { record_status(status.word, code); }
 
 __device__ __forceinline__ uint64_t globaltimer() {
   uint64_t t;
@@ -68,7 +77,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 
 // Waits for phase `parity` of `bar` to complete. Returns false (after recording a timeout)
 // if it has not completed within the wait limit, or at once if *abort is already set.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status,
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const DevStatus& status,
                                           volatile int* abort) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
@@ -77,7 +86,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* s
     if (mbar_try_wait(bar, parity)) return true;
     if ((++spins & 63u) == 0) {
       if (abort != nullptr && *abort) return false;
-      if (globaltimer() - t0 > kWaitLimitNs) {
+      if (globaltimer() - t0 > status.limit_ns) {
         record_status(status, kDevTimeout);
         if (abort != nullptr) *abort = 1;
         return false;

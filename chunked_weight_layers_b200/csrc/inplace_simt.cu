@@ -2,8 +2,9 @@
 // chunk 512). "In-Place Test-Time Training", §3: for each chunk, O_c = Z_c·W_cᵀ with the
 // weight from before the chunk, then W_{c+1} = W_c + η·V̂_cᵀ·Z_c (§2).
 //
-// Both steps are small GEMMs (0.13 GFLOP per chunk) run as two tiled launches per chunk:
-// 64x64 output tiles, 16-deep k slices staged in shared memory, 4x4 outputs per thread.
+// Both steps are small GEMMs (0.13 GFLOP per chunk each), independent of each other within a
+// chunk: one launch per chunk runs the tiles of both (the update writes a second weight
+// buffer, swapped after the launch).
 // Tensor cores are not used here: TF32 would miss the 1e-4 tolerance of this workload and
 // the exact-integer checks, and the work is far too small to be throughput-bound.
 #include "common.cuh"
@@ -13,83 +14,104 @@ namespace ttt {
 
 namespace {
 
-constexpr int BM = 64, BN = 64, BK = 16, NT = 256;
+// Output tiles of 32 x 64, k slices of 32, 256 threads with 2 x 4 outputs each: a chunk of the
+// fp32 workload (C = 512, d = 256, f = 512) is 64 APPLY tiles and 64 UPDATE tiles, run by one
+// launch on 128 SMs.
+constexpr int BM = 32, BN = 64, BK = 32, NT = 256;
 
-// C[M,N] (op)= A[M,K]·B[K,N] where A is stored K-contiguous (A_KC) or M-contiguous, and B is
-// stored K-contiguous (B_KC, i.e. as [N,K]) or N-contiguous (as [K,N]).
-// UPDATE = false: C = acc.  UPDATE = true: C = C + eta·acc (fused multiply-add).
+struct SgemmSmem {
+  float As[BK][BM + 4];
+  float Bs[BK][BN + 4];
+};
+
+// One tile of C[M,N] = A[M,K]·B[K,N] (UPDATE = false) or C = Cin + eta·A·B (UPDATE = true),
+// where A is stored K-contiguous (A_KC, as [M,K]) or M-contiguous (as [K,M]) and B is stored
+// K-contiguous (B_KC, as [N,K]) or N-contiguous (as [K,N]). Every output accumulates its
+// products in increasing k with fmaf, so results do not depend on the tiling.
 template <bool A_KC, bool B_KC, bool UPDATE>
-__global__ void __launch_bounds__(NT) k_sgemm(const float* __restrict__ A, const float* __restrict__ B,
-                                              float* __restrict__ Cmat, int M, int N, int K, int lda, int ldb,
-                                              int ldc, float eta) {
-  __shared__ float As[BK][BM + 4];
-  __shared__ float Bs[BK][BN + 4];
+__device__ __forceinline__ void sgemm_tile(SgemmSmem& sm, const float* __restrict__ A, const float* __restrict__ B,
+                                           const float* __restrict__ Cin, float* __restrict__ Cout, int M, int N,
+                                           int K, int lda, int ldb, int ldc, float eta, int m0, int n0) {
   const int tid = threadIdx.x;
   const int tx = tid % 16, ty = tid / 16;
-  const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
-  float acc[4][4] = {};
+  float acc[2][4] = {};
   for (int k0 = 0; k0 < K; k0 += BK) {
-    // Stage the A slice as As[k][m].
+    // Stage A as As[k][m] (32 x 32: four elements a thread).
     if (A_KC) {
-      const int r = tid / 4, kq = (tid % 4) * 4;
+      const int r = tid / 8, kq = (tid % 8) * 4;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int m = m0 + r, k = k0 + kq + j;
-        As[kq + j][r] = (m < M && k < K) ? A[(size_t)m * lda + k] : 0.f;
+        sm.As[kq + j][r] = (m < M && k < K) ? A[(size_t)m * lda + k] : 0.f;
       }
     } else {
-      const int kk = tid / 16, mq = (tid % 16) * 4;
+      const int kk = tid / 8, mq = (tid % 8) * 4;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int m = m0 + mq + j, k = k0 + kk;
-        As[kk][mq + j] = (m < M && k < K) ? A[(size_t)k * lda + m] : 0.f;
+        sm.As[kk][mq + j] = (m < M && k < K) ? A[(size_t)k * lda + m] : 0.f;
       }
     }
-    // Stage the B slice as Bs[k][n].
+    // Stage B as Bs[k][n] (32 x 64: eight elements a thread).
     if (B_KC) {
-      const int r = tid / 4, kq = (tid % 4) * 4;
+      const int r = tid / 4, kq = (tid % 4) * 8;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
+      for (int j = 0; j < 8; ++j) {
         const int n = n0 + r, k = k0 + kq + j;
-        Bs[kq + j][r] = (n < N && k < K) ? B[(size_t)n * ldb + k] : 0.f;
+        sm.Bs[kq + j][r] = (n < N && k < K) ? B[(size_t)n * ldb + k] : 0.f;
       }
     } else {
-      const int kk = tid / 16, nq = (tid % 16) * 4;
+      const int kk = tid / 8, nq = (tid % 8) * 8;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
+      for (int j = 0; j < 8; ++j) {
         const int n = n0 + nq + j, k = k0 + kk;
-        Bs[kk][nq + j] = (n < N && k < K) ? B[(size_t)k * ldb + n] : 0.f;
+        sm.Bs[kk][nq + j] = (n < N && k < K) ? B[(size_t)k * ldb + n] : 0.f;
       }
     }
     __syncthreads();
+    const int kend = min(BK, K - k0);
+    for (int k = 0; k < kend; ++k) {
+      const float2 a = *reinterpret_cast<const float2*>(&sm.As[k][ty * 2]);
+      const float4 b = *reinterpret_cast<const float4*>(&sm.Bs[k][tx * 4]);
+      const float av[2] = {a.x, a.y};
+      const float bv[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
-    for (int k = 0; k < BK; ++k) {
-      float a[4], b[4];
+      for (int i = 0; i < 2; ++i)
 #pragma unroll
-      for (int i = 0; i < 4; ++i) a[i] = As[k][ty * 4 + i];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) b[j] = Bs[k][tx * 4 + j];
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
     }
     __syncthreads();
   }
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int m = m0 + ty * 4 + i;
+  for (int i = 0; i < 2; ++i) {
+    const int m = m0 + ty * 2 + i;
     if (m >= M) continue;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int n = n0 + tx * 4 + j;
       if (n >= N) continue;
-      float* c = Cmat + (size_t)m * ldc + n;
-      if (UPDATE)
-        *c = fmaf(eta, acc[i][j], *c);
-      else
-        *c = acc[i][j];
+      const size_t o = (size_t)m * ldc + n;
+      Cout[o] = UPDATE ? fmaf(eta, acc[i][j], Cin[o]) : acc[i][j];
     }
+  }
+}
+
+// One chunk: blocks [0, n_apply) compute tiles of O[C, d] = Z[C, f]·W[d, f]ᵀ with the weight
+// from before the chunk; the others tiles of Wn[d, f] = W + η·V̂[C, d]ᵀ·Z[C, f]. The update
+// writes a second buffer, so both run in the same launch.
+__global__ void __launch_bounds__(NT) k_f32_chunk(const float* __restrict__ Z, const float* __restrict__ Vhat,
+                                                  const float* __restrict__ W, float* __restrict__ Wn,
+                                                  float* __restrict__ O, int C, int d, int f, float eta,
+                                                  int apply_tiles_n) {
+  __shared__ __align__(16) SgemmSmem sm;
+  const int n_apply = ((C + BM - 1) / BM) * apply_tiles_n;
+  const int b = blockIdx.x;
+  if (b < n_apply) {
+    sgemm_tile<true, true, false>(sm, Z, W, nullptr, O, C, d, f, f, f, d, 0.f, (b / apply_tiles_n) * BM,
+                                  (b % apply_tiles_n) * BN);
+  } else {
+    const int u = b - n_apply, ntn = (f + BN - 1) / BN;
+    sgemm_tile<false, false, true>(sm, Vhat, Z, W, Wn, d, f, C, d, f, f, eta, (u / ntn) * BM, (u % ntn) * BN);
   }
 }
 
@@ -97,16 +119,15 @@ __global__ void __launch_bounds__(NT) k_sgemm(const float* __restrict__ A, const
 
 ttt_status inplace_f32_chunk(ttt_state* st, const float* Z, const float* Vhat, float* O, int C, cudaStream_t s) {
   const int d = st->cfg.d_val, f = st->cfg.d_key;
-  // Apply: O[C, d] = Z[C, f] · W[d, f]ᵀ — A = Z (K-contiguous), B = W as [N=d, K=f].
-  dim3 ga((d + BN - 1) / BN, (C + BM - 1) / BM);
-  k_sgemm<true, true, false><<<ga, NT, 0, s>>>(Z, st->ip.W, O, C, d, f, f, f, d, 0.f);
+  const int apply_tn = (d + BN - 1) / BN;
+  const int tiles = ((C + BM - 1) / BM) * apply_tn + ((d + BM - 1) / BM) * ((f + BN - 1) / BN);
+  k_f32_chunk<<<tiles, NT, 0, s>>>(Z, Vhat, st->ip.W, st->ip.Wf32_next, O, C, d, f, st->cfg.eta, apply_tn);
   st->launches++;
   TTT_CUDA(cudaGetLastError());
-  // Update: W[d, f] += η · V̂[C, d]ᵀ · Z[C, f] — A = V̂ᵀ (M-contiguous), B = Z as [K=C, N=f].
-  dim3 gu((f + BN - 1) / BN, (d + BM - 1) / BM);
-  k_sgemm<false, false, true><<<gu, NT, 0, s>>>(Vhat, Z, st->ip.W, d, f, C, d, f, f, st->cfg.eta);
-  st->launches++;
-  TTT_CUDA(cudaGetLastError());
+  // The weight after this chunk is in the second buffer: swap the two.
+  float* w = st->ip.W;
+  st->ip.W = st->ip.Wf32_next;
+  st->ip.Wf32_next = w;
   return TTT_OK;
 }
 

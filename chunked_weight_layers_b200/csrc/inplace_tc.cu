@@ -92,7 +92,10 @@ struct TCArgs {
   float eta;
   __nv_bfloat16* O;            // outputs [T, d]
   __nv_bfloat16* Vhat_out;     // targets of target_chunk [C, d]
-  int* status;
+  DevStatus status;
+  // Fault injection (tests): the APPLY tiles of this round wait for one more UPDATE than will
+  // ever be counted, so that wait runs out; -1 = none.
+  int stall_round;
   // Several chunks in one launch: every CTA runs its tile list once per chunk (chunk index
   // chunk + r in round r). The bf16 copy of W rotates through three buffers: round r applies
   // with buffer (cur0 + r) % 3 and its UPDATE tiles write buffer (cur0 + r + 1) % 3, the one
@@ -197,13 +200,13 @@ __device__ __forceinline__ void fence_proxy_async_global() {
 
 // Bounded wait until *ctr ≥ want (a counter other CTAs raise); then the async proxy (TMA) may
 // read what they published.
-__device__ __forceinline__ bool wait_counter(const int* ctr, int want, int* status, volatile int* abort) {
+__device__ __forceinline__ bool wait_counter(const int* ctr, int want, const DevStatus& status, volatile int* abort) {
   const volatile int* c = ctr;
   if (*c < want) {
     const uint64_t t0 = globaltimer();
     while (*c < want) {
       if (*abort) return false;
-      if (globaltimer() - t0 > kWaitLimitNs) {
+      if (globaltimer() - t0 > status.limit_ns) {
         record_status(status, kDevTimeout);
         *abort = 1;
         return false;
@@ -305,7 +308,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         const CUtensorMap* wk = pick3(tmWk0, tmWk1, tmWk2, (args.cur0 + rnd) % 3);
         if (args.upd_done != nullptr) {
           if (type == APPLY && rnd >= 1 &&
-              !wait_counter(&args.upd_done[(rnd - 1) * args.nbd + n], upd_expect(args, n), args.status, abort))
+              !wait_counter(&args.upd_done[(rnd - 1) * args.nbd + n],
+                            upd_expect(args, n) + (rnd == args.stall_round ? 1 : 0), args.status, abort))
             return false;
           if (type == UPDATE && rnd >= 2 &&
               !wait_counter(&args.app_done[(rnd - 2) * args.nbd + m / 2], args.C / BM, args.status, abort))
@@ -772,7 +776,12 @@ ttt_status inplace_bf16_scan(ttt_state* st, const __nv_bfloat16* Z, const __nv_b
     a.eta = c.eta;
     a.O = O;
     a.Vhat_out = target ? st->ip.Vhat[tchunk % 3] : nullptr;
-    a.status = st->status.dev;
+    a.status = DevStatus{st->status.dev, st->wait_limit_ns};
+    a.stall_round = -1;
+    if (st->inject_stall && rounds >= 2 && counters != nullptr) {
+      a.stall_round = 1;
+      st->inject_stall = 0;
+    }
     a.rounds = rounds;
     a.cur0 = st->ip.cur;
     a.nbd = (d + BN - 1) / BN;
@@ -874,7 +883,7 @@ int target_values_plan_ints(int T, int d, int num_sms) {
 
 ttt_status target_values_into(const __nv_bfloat16* X0, const float* convw, const __nv_bfloat16* Wtarget, int T, int d,
                               int C, int taps, int pad_mode, __nv_bfloat16* conv_scratch, int32_t* plan_scratch,
-                              __nv_bfloat16* out, int num_sms, cudaStream_t s) {
+                              __nv_bfloat16* out, int32_t* status, int num_sms, cudaStream_t s) {
   const int mt = T / BM, nt = (d + BN - 1) / BN;
   const int grid = std::max(1, std::min(num_sms, mt * nt));
   const size_t pairs = (size_t)T * (d / 2);
@@ -897,7 +906,8 @@ ttt_status target_values_into(const __nv_bfloat16* X0, const float* convw, const
   a.eta = 0.f;
   a.O = nullptr;
   a.Vhat_out = out;
-  a.status = nullptr;
+  a.status = DevStatus{status, kWaitLimitNs};
+  a.stall_round = -1;
   a.rounds = 1;
   a.cur0 = 0;
   a.nbd = 0;

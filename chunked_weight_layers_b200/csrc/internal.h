@@ -41,6 +41,7 @@ struct StatusWord {
 struct InplaceBuffers {
   float* W = nullptr;            // fp32 master [d, f]
   float* W0 = nullptr;           // pretrained copy [d, f]
+  float* Wf32_next = nullptr;    // fp32 path: the next chunk's weight, written beside W (swapped)
   // bf16 copies of W for the apply (BF16 path): chunk c applies with one while its update
   // writes the next; three so that an update never overwrites the copy that the chunk
   // before is still applying with when chunks overlap in one launch.
@@ -54,16 +55,27 @@ struct InplaceBuffers {
   TCResources* tc = nullptr;     // tensor-core schedules and conv(X0) buffer, built on first use
 };
 
+// Tensor maps of one scan's K, V, Q, O (encoding them costs microseconds of host time, so the
+// maps of the last few buffer sets are kept: a caller that cycles through a few sets of buffers
+// encodes each set once).
+struct LinearMapSet {
+  const void* key[4] = {nullptr, nullptr, nullptr, nullptr};
+  int64_t T = -1;
+  uint64_t last_use = 0;
+  CUtensorMap maps[4];
+};
+
 struct LinearBuffers {
   float* W = nullptr;   // [B, H, D, D]
   float* W0 = nullptr;  // [B, H, D, D]
-  // Tensor maps of the last scan's K, V, Q, O (re-encoded only when a pointer or T changes:
-  // encoding costs microseconds of host time per call) and the kernels whose shared-memory
-  // size has been raised for this state's device.
-  const void* map_key[4] = {nullptr, nullptr, nullptr, nullptr};
-  int64_t map_T = -1;
-  CUtensorMap maps[4];
-  uint32_t smem_set = 0;
+  static constexpr int kMapSets = 8;
+  LinearMapSet map_sets[kMapSets];
+  uint64_t map_clock = 0;
+  // Kernels whose shared-memory size has been raised for this state's device.
+  uint64_t smem_set = 0;
+  // Inner mini-batches per chunk of the b = 16 scan (TTT_OPT_LINEAR_CHUNK): 1 = one step at a
+  // time, 2 or 4 = the chunked form; 0 = the library's choice (1).
+  int form = 0;
 };
 
 struct GateBuffers {
@@ -91,6 +103,11 @@ struct ttt_state {
   ttt::GateBuffers gate;
   ttt::HostStaging staging;
   int64_t launches = 0;
+  // Limit of every spin-wait of this state's kernels (TTT_OPT_WAIT_LIMIT_NS), in ns.
+  uint64_t wait_limit_ns = 2000000000ull;
+  // Fault injection (TTT_OPT_INJECT_STALL, tests): the next scan that can makes one of its
+  // bounded waits wait for something that never comes; cleared once used.
+  int inject_stall = 0;
 };
 
 namespace ttt {

@@ -39,6 +39,7 @@ constexpr int kStages = 4;        // ring depth (64-token tiles): 96 KB of K/V/Q
 constexpr int kTileTok = 64;      // tokens per tile
 constexpr int kTileBytes = kTileTok * 128;  // 64 tokens x 64 bf16
 constexpr int kComputeWarps = 4;
+constexpr int kLossStride = 68;   // floats per row of loss partials (64 tokens + 4: no bank conflicts)
 constexpr int kThreads = (kComputeWarps + 1) * 32;
 
 struct __align__(1024) LinearSmem {
@@ -216,16 +217,246 @@ __device__ __forceinline__ void compute16(float (&acc)[8][4], const Frag16& F, u
               pack_bf16(o[1][0][2] + o[1][1][2], o[1][0][3] + o[1][1][3]));
   }
   if (LOSS) {
+    // Squared residuals of this lane's two columns; the writer warp sums the 32 partials of a
+    // token (eight lane groups, four warps), so no reduction sits on the chain.
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
-      float l0 = p[nt][0] * p[nt][0] + p[nt][2] * p[nt][2];
-      float l1 = p[nt][1] * p[nt][1] + p[nt][3] * p[nt][3];
+      const float l0 = p[nt][0] * p[nt][0] + p[nt][2] * p[nt][2];
+      const float l1 = p[nt][1] * p[nt][1] + p[nt][3] * p[nt][3];
+      *reinterpret_cast<float2*>(&lossp[g * kLossStride + r0 + 8 * nt + 2 * q]) = make_float2(l0, l1);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
+// Chunked form of the b = 16 scan. A chunk holds NB inner mini-batches (16-token blocks
+// i = 0 .. NB−1) and starts from weight W. Unrolling the steps inside the chunk,
+//   W_i = W − β·Σ_{j<i} K_jᵀR_j,   so
+//   R_i = K_i·W − V_i − β·Σ_{j<i} (K_i·K_jᵀ)·R_j,
+//   O_i = Q_i·W     − β·Σ_{j<i} (Q_i·K_jᵀ)·R_j,
+//   W_next = W − β·Σ_i K_iᵀR_i.
+// This is the same arithmetic as NB sequential steps, regrouped: every product with W uses the
+// weight from the chunk's start, so the NB products P_i = K_i·W are independent and issue back
+// to back; what stays sequential is the short correction of each block by the residuals of
+// the blocks before it (a 16x16x16 product per pair and warp). The Gram blocks G_ij = K_i·K_jᵀ
+// and M_ij = Q_i·K_jᵀ do not depend on W: the four compute warps share them out one tile
+// ahead (each computes a quarter into shared memory while it runs the tile before).
+// ---------------------------------------------------------------------------------------------
+
+// Chunked form: the Gram blocks K_i·K_jᵀ (and Q_i·K_jᵀ) of the block pairs i > j of every chunk
+// of a tile, bf16, each 16x16 block as four 8x8 tiles of 128 bytes ([i half][j half]).
+constexpr int kMaxTilePairs = 6;   // a 64-token chunk of four 16-token blocks has six pairs
+constexpr int kPairBytes = 1024;   // G block then M block
+
+// Slot of pair (i, j), i > j, among a chunk's pairs: (1,0) (2,0) (2,1) (3,0) (3,1) (3,2).
+__host__ __device__ constexpr int pair_slot(int i, int j) { return i * (i - 1) / 2 + j; }
+
+// Per-lane offset of the x4 ldmatrix / stmatrix that reads or writes a Gram block (four 8x8
+// tiles of 128 bytes: [i 0-7, j 0-7], [i 0-7, j 8-15], [i 8-15, j 0-7], [i 8-15, j 8-15]).
+__device__ __forceinline__ uint32_t gram_lane_ofs(int lane) { return (uint32_t)(lane >> 3) * 128u + (uint32_t)(lane & 7) * 16u; }
+
+// One Gram unit: columns 8nt .. 8nt+7 (tokens of block bj) of X_bi·K_bjᵀ, for X = K (into the G
+// block of slot `dst`) and, with queries, X = Q (into its M block). Rows come from a tile in the
+// ring (128-byte swizzle), blocks bi, bj counted in 16-token rows of the tile. Every fragment is
+// loaded before the first mma so the loads' latencies overlap.
+template <bool HAS_Q>
+__device__ __forceinline__ void gram_unit(uint32_t kbase, uint32_t qbase, int bi, int bj, int nt, uint32_t dst,
+                                          const StepOffsets& f, int lane) {
+  constexpr int NX = HAS_Q ? 2 : 1;
+  // B fragments of K_bjᵀ for this n-tile: dk 32kp .. 32kp+31.
+  uint32_t kb[2][4];
 #pragma unroll
-      for (int m = 4; m < 32; m <<= 1) {
-        l0 += __shfl_xor_sync(0xffffffffu, l0, m);
-        l1 += __shfl_xor_sync(0xffffffffu, l1, m);
+  for (int kp = 0; kp < 2; ++kp) ldsm_x4(kbase + (uint32_t)(16 * bj) * 128u + f.kb[nt][kp], kb[kp]);
+  const int arow = (lane & 7) + 8 * ((lane >> 3) & 1);
+  uint32_t a[NX][4][4];
+#pragma unroll
+  for (int x = 0; x < NX; ++x)
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks)
+      ldsm_x4((x == 0 ? kbase : qbase) + (uint32_t)(16 * bi) * 128u + swz128_bf16(arow, 16 * ks + 8 * (lane >> 4)),
+              a[x][ks]);
+  float c[NX][2][4];
+#pragma unroll
+  for (int x = 0; x < NX; ++x)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) c[x][0][e] = c[x][1][e] = 0.f;
+#pragma unroll
+  for (int ks = 0; ks < 4; ++ks)
+#pragma unroll
+    for (int x = 0; x < NX; ++x)
+      mma16816(c[x][ks & 1], a[x][ks], kb[ks >> 1][2 * (ks & 1)], kb[ks >> 1][2 * (ks & 1) + 1]);
+#pragma unroll
+  for (int x = 0; x < NX; ++x) {
+    // stmatrix x2: matrix 0 = rows i 0-7 (tile nt), matrix 1 = rows i 8-15 (tile 2 + nt).
+    const uint32_t addr = dst + (uint32_t)x * 512u + (uint32_t)((lane >> 3) & 1) * 256u + (uint32_t)nt * 128u +
+                          (uint32_t)(lane & 7) * 16u;
+    const uint32_t r0 = pack_bf16(c[x][0][0] + c[x][1][0], c[x][0][1] + c[x][1][1]);
+    const uint32_t r1 = pack_bf16(c[x][0][2] + c[x][1][2], c[x][0][3] + c[x][1][3]);
+    asm volatile("stmatrix.sync.aligned.m8n8.x2.shared.b16 [%0], {%1, %2};" ::"r"(addr), "r"(r0), "r"(r1) : "memory");
+  }
+}
+
+// This warp's share of the Gram blocks of one tile (all its chunks of NB blocks).
+template <int NB, bool HAS_Q>
+__device__ __forceinline__ void gram_tile(uint32_t kbase, uint32_t qbase, uint32_t gmbase, const StepOffsets& f,
+                                          int warp, int lane) {
+  constexpr int kPPC = NB * (NB - 1) / 2;   // pairs per chunk
+  constexpr int kUnits = (64 / (16 * NB)) * kPPC * 2;  // (pair, n-tile) units per tile
+#pragma unroll
+  for (int u0 = 0; u0 < kUnits; u0 += kComputeWarps) {
+    const int u = u0 + warp;
+    if (kUnits % kComputeWarps != 0 && u >= kUnits) break;
+    const int p = u >> 1, nt = u & 1;
+    const int cc = p / kPPC, loc = p % kPPC;
+    // loc = i(i−1)/2 + j
+    const int i = loc < 1 ? 1 : (loc < 3 ? 2 : 3);
+    const int j = loc - pair_slot(i, 0);
+    gram_unit<HAS_Q>(kbase, qbase, cc * NB + i, cc * NB + j, nt, gmbase + (uint32_t)p * kPairBytes, f, lane);
+  }
+}
+
+// Fragments one block of a chunk needs after its product with W: Vᵀ of this warp's columns,
+// the K operand of the update, the Qᵀ operand of the outputs, the Gram blocks G(i2, i) that
+// carry its residuals into the later blocks i2 and the M(i, j) that carry the earlier blocks'
+// residuals into its outputs.
+template <int NBLK, bool HAS_Q>
+struct BlkFrag {
+  uint32_t vf[4];
+  uint32_t kt[4][4];
+  uint32_t qb[2][2][4];
+  uint32_t g[NBLK > 1 ? NBLK - 1 : 1][4];
+  uint32_t m[NBLK > 1 ? NBLK - 1 : 1][4];
+};
+
+template <int NBLK, bool HAS_Q>
+__device__ __forceinline__ void load_blk(BlkFrag<NBLK, HAS_Q>& B, int i, uint32_t kbase, uint32_t vbase, uint32_t qbase,
+                                         uint32_t gbase, const StepOffsets& f, uint32_t gl, int r0) {
+  const uint32_t rofs = (uint32_t)(r0 + 16 * i) * 128u;
+  ldsm_x4_t(vbase + rofs + f.v, B.vf);
+#pragma unroll
+  for (int i2 = i + 1; i2 < NBLK; ++i2) ldsm_x4(gbase + (uint32_t)pair_slot(i2, i) * kPairBytes + gl, B.g[i2 - i - 1]);
+#pragma unroll
+  for (int np = 0; np < 4; ++np) ldsm_x4_t(kbase + rofs + f.kt[np], B.kt[np]);
+  if (HAS_Q) {
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int kp = 0; kp < 2; ++kp) ldsm_x4(qbase + rofs + f.kb[nt][kp], B.qb[nt][kp]);
+#pragma unroll
+    for (int j = 0; j < i; ++j) ldsm_x4(gbase + (uint32_t)pair_slot(i, j) * kPairBytes + 512u + gl, B.m[j]);
+  }
+}
+
+__device__ __forceinline__ void load_kb(uint32_t (&kb)[2][2][4], uint32_t rb, const StepOffsets& f) {
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+    for (int kp = 0; kp < 2; ++kp) ldsm_x4(rb + f.kb[nt][kp], kb[nt][kp]);
+}
+
+// One chunk of NBLK blocks (tile rows r0 .. r0 + 16·NBLK − 1) for the warp owning W columns
+// [col0, col0+16). `gbase` is the chunk's first pair slot. Everything transposed as in compute16:
+// Pᵀ_i = Wᵀ·K_iᵀ, Rᵀ_i = Pᵀ_i − V_iᵀ + Σ_{j<i} Sᵀ_j·G_ijᵀ with S = −β·R (bf16), Wᵀ += Σ_i Sᵀ_i·K_i,
+// Oᵀ_i = Wᵀ·Qᵀ_i + Σ_{j<i} Sᵀ_j·M_ijᵀ. The tensor cores see W, S and the Gram blocks rounded to bf16;
+// W and every accumulation stay fp32.
+// Loads and mma keep their program order (both are volatile), so every fragment is loaded one
+// phase before its first use: the Kᵀ operand of block i+1 while the products of block i issue,
+// block 0's remaining fragments while the last product with W issues, and block i+1's while
+// block i's outputs issue.
+template <int NBLK, bool HAS_Q, bool LOSS>
+__device__ __forceinline__ void chunk_run(float (&acc)[8][4], uint32_t kbase, uint32_t vbase, uint32_t qbase,
+                                          uint32_t gbase, uint32_t obase, const StepOffsets& f, float* lossp,
+                                          int r0, int lane, float beta) {
+  const int g = lane >> 2, q = lane & 3;
+  const uint32_t gl = gram_lane_ofs(lane);
+  uint32_t kbuf[2][2][2][4];
+  load_kb(kbuf[0], kbase + (uint32_t)r0 * 128u, f);
+  uint32_t wa[4][4];
+#pragma unroll
+  for (int ks = 0; ks < 4; ++ks) {
+    wa[ks][0] = pack_bf16(acc[2 * ks][0], acc[2 * ks][1]);
+    wa[ks][1] = pack_bf16(acc[2 * ks][2], acc[2 * ks][3]);
+    wa[ks][2] = pack_bf16(acc[2 * ks + 1][0], acc[2 * ks + 1][1]);
+    wa[ks][3] = pack_bf16(acc[2 * ks + 1][2], acc[2 * ks + 1][3]);
+  }
+  // P_i for every block of the chunk, two partial sums per token n-tile.
+  float pp[NBLK][2][2][4];
+  BlkFrag<NBLK, HAS_Q> F[2];
+#pragma unroll
+  for (int i = 0; i < NBLK; ++i) {
+    if (i + 1 < NBLK) load_kb(kbuf[(i + 1) & 1], kbase + (uint32_t)(r0 + 16 * (i + 1)) * 128u, f);
+    else load_blk<NBLK, HAS_Q>(F[0], 0, kbase, vbase, qbase, gbase, f, gl, r0);
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) pp[i][nt][0][e] = pp[i][nt][1][e] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks)
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+        mma16816(pp[i][nt][ks & 1], wa[ks], kbuf[i & 1][nt][ks >> 1][2 * (ks & 1)],
+                 kbuf[i & 1][nt][ks >> 1][2 * (ks & 1) + 1]);
+  }
+
+  uint32_t sa[NBLK][4];
+#pragma unroll
+  for (int i = 0; i < NBLK; ++i) {
+    BlkFrag<NBLK, HAS_Q>& B = F[i & 1];
+    // R_i = P_i − V_i (+ the corrections already accumulated into pp[i][.][0]).
+    const float2 v0 = unpack_bf16(B.vf[0]), v1 = unpack_bf16(B.vf[1]), v2 = unpack_bf16(B.vf[2]),
+                 v3 = unpack_bf16(B.vf[3]);
+    const float vv[2][4] = {{v0.x, v0.y, v1.x, v1.y}, {v2.x, v2.y, v3.x, v3.y}};
+    float p[2][4];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) p[nt][e] = (pp[i][nt][0][e] + pp[i][nt][1][e]) - vv[nt][e];
+    sa[i][0] = pack_bf16(-beta * p[0][0], -beta * p[0][1]);
+    sa[i][1] = pack_bf16(-beta * p[0][2], -beta * p[0][3]);
+    sa[i][2] = pack_bf16(-beta * p[1][0], -beta * p[1][1]);
+    sa[i][3] = pack_bf16(-beta * p[1][2], -beta * p[1][3]);
+    // Corrections of the later blocks by this block's residuals (the chain's critical step).
+#pragma unroll
+    for (int i2 = i + 1; i2 < NBLK; ++i2) {
+      mma16816(pp[i2][0][0], sa[i], B.g[i2 - i - 1][0], B.g[i2 - i - 1][1]);
+      mma16816(pp[i2][1][0], sa[i], B.g[i2 - i - 1][2], B.g[i2 - i - 1][3]);
+    }
+    // Wᵀ += Sᵀ_i·K_i.
+#pragma unroll
+    for (int np = 0; np < 4; ++np) {
+      mma16816(acc[2 * np], sa[i], B.kt[np][0], B.kt[np][1]);
+      mma16816(acc[2 * np + 1], sa[i], B.kt[np][2], B.kt[np][3]);
+    }
+    if (i + 1 < NBLK) load_blk<NBLK, HAS_Q>(F[(i + 1) & 1], i + 1, kbase, vbase, qbase, gbase, f, gl, r0);
+    if (LOSS) {
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        const float l0 = p[nt][0] * p[nt][0] + p[nt][2] * p[nt][2];
+        const float l1 = p[nt][1] * p[nt][1] + p[nt][3] * p[nt][3];
+        *reinterpret_cast<float2*>(&lossp[g * kLossStride + r0 + 16 * i + 8 * nt + 2 * q]) = make_float2(l0, l1);
       }
-      if (g == 0) *reinterpret_cast<float2*>(&lossp[r0 + 8 * nt + 2 * q]) = make_float2(l0, l1);
+    }
+    if (HAS_Q) {
+      float o[2][2][4];
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o[nt][0][e] = o[nt][1][e] = 0.f;
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks)
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+          mma16816(o[nt][ks & 1], wa[ks], B.qb[nt][ks >> 1][2 * (ks & 1)], B.qb[nt][ks >> 1][2 * (ks & 1) + 1]);
+#pragma unroll
+      for (int j = 0; j < i; ++j) {
+        mma16816(o[0][0], sa[j], B.m[j][0], B.m[j][1]);
+        mma16816(o[1][0], sa[j], B.m[j][2], B.m[j][3]);
+      }
+      stsm_x4_t(obase + (uint32_t)(r0 + 16 * i) * 128u + f.o,
+                pack_bf16(o[0][0][0] + o[0][1][0], o[0][0][1] + o[0][1][1]),
+                pack_bf16(o[0][0][2] + o[0][1][2], o[0][0][3] + o[0][1][3]),
+                pack_bf16(o[1][0][0] + o[1][1][0], o[1][0][1] + o[1][1][1]),
+                pack_bf16(o[1][0][2] + o[1][1][2], o[1][0][3] + o[1][1][3]));
     }
   }
 }
@@ -249,12 +480,16 @@ struct __align__(1024) B16Smem {
   uint8_t V[kStages][kTileBytes];
   uint8_t Q[kStages][kTileBytes];
   uint8_t O[2][kTileBytes];
-  float lossp[2][kComputeWarps][kTileTok];
+  uint8_t gm[2][kMaxTilePairs][kPairBytes];  // chunked form: Gram blocks of tiles t (t & 1)
+  // Per-lane loss partials of tile t (t & 1): [compute warp][lane group g][token], each the sum
+  // of the squared residuals of the warp's two columns g, g+8; the writer adds them up.
+  float lossp[2][kComputeWarps][8][kLossStride];
   float gl[kGateRing][kTileTok];  // tiles' losses handed from the writer to the gate warps
   uint64_t full[kStages];
   uint64_t empty[kStages];
   uint64_t oready[2];
   uint64_t ofree[2];
+  uint64_t gmready[2];  // chunked form: the Gram blocks of a tile are complete (all compute lanes)
   uint64_t gready[kGateRing];
   uint64_t gfree[kGateRing];
   int abort;  // set by whichever warp's wait ran out; every other wait then returns at once
@@ -279,7 +514,7 @@ struct GateArgs {
 };
 
 // Warp-uniform bounded wait: false (with abort set) if the phase did not complete in time.
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, int* status, int* abort) {
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const DevStatus& status, int* abort) {
   bool ok = mbar_wait(bar, parity, status, abort);
   ok = __all_sync(0xffffffffu, ok);
   if (!ok) *reinterpret_cast<volatile int*>(abort) = 1;
@@ -287,14 +522,14 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, int* s
 }
 
 // Bounded wait until *turn == want (a shared-memory counter advanced by another warp).
-__device__ __forceinline__ bool wait_turn(const int* turn, int want, int* status, int* abort) {
+__device__ __forceinline__ bool wait_turn(const int* turn, int want, const DevStatus& status, int* abort) {
   const volatile int* tv = turn;
   const volatile int* av = abort;
   if (*tv == want) return true;
   const uint64_t t0 = globaltimer();
   while (*tv != want) {
     if (*av) return false;
-    if (globaltimer() - t0 > kWaitLimitNs) {
+    if (globaltimer() - t0 > status.limit_ns) {
       record_status(status, kDevTimeout);
       *const_cast<volatile int*>(av) = 1;
       return false;
@@ -303,19 +538,29 @@ __device__ __forceinline__ bool wait_turn(const int* turn, int want, int* status
   return true;
 }
 
-template <bool HAS_Q, bool LOSS, bool GATE>
+// NB = inner mini-batches per chunk: 1 runs the steps one by one (compute16), 2 or 4 the chunked
+// form (chunk_run) with the Gram blocks shared through shared memory one tile ahead.
+template <bool HAS_Q, bool LOSS, bool GATE, int NB>
 __global__ void __launch_bounds__(b16_threads<true>(), 1)
     k_linear_b16(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                  const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
-                 float* __restrict__ Wstate, float* __restrict__ loss, int T, float beta, int* status,
-                 const GateArgs ga) {
+                 float* __restrict__ Wstate, float* __restrict__ loss, int T, float beta, const DevStatus status,
+                 const GateArgs ga, int stall_tile) {
   static_assert(!GATE || LOSS, "the gate reads the losses");
   extern __shared__ uint8_t smem_raw[];
   B16Smem& sm = *reinterpret_cast<B16Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bh = blockIdx.x;
   const int ntiles = (T + kTileTok - 1) / kTileTok;
+  float* Wg = Wstate + (size_t)bh * 64 * 64;
 
+  // Set-up that reads nothing a kernel before this one in the stream may still be writing runs
+  // first: with programmatic dependent launch it overlaps the end of that kernel.
+  if (warp == kComputeWarps && lane == 0) {
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+    if (HAS_Q) tma_prefetch_desc(&tmQ);
+  }
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&sm.full[i], 1);
@@ -324,42 +569,56 @@ __global__ void __launch_bounds__(b16_threads<true>(), 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sm.oready[i], kComputeWarps * 32);
       mbar_init(&sm.ofree[i], 1);
+      mbar_init(&sm.gmready[i], kComputeWarps * 32);
     }
     for (int i = 0; i < kGateRing; ++i) {
       mbar_init(&sm.gready[i], 1);
       mbar_init(&sm.gfree[i], 1);
     }
     sm.abort = 0;
-    if (GATE) {
-      sm.g_tau = ga.tau[bh];
-      sm.g_tau_set = ga.tau_set[bh];
-      sm.g_routed = ga.counts[2 * bh];
-      sm.gate_turn = 0;
-    }
+    sm.gate_turn = 0;
     fence_barrier_init();
+  }
+  // Wait for the kernel before this one (a no-op without programmatic dependent launch), then
+  // let the next one start its own set-up: it waits in turn before reading what this one writes.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;");
+  // The compute warps' slice of W, in accumulator layout (warp w owns columns 16w .. 16w+15):
+  // acc[nt][e] = W[8nt + 2q + (e&1)][16w + g + 8(e>>1)].
+  float acc[8][4];
+  if (warp < kComputeWarps) {
+    const int g = lane >> 2, q = lane & 3, col0 = 16 * warp;
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[nt][e] = Wg[(8 * nt + 2 * q + (e & 1)) * 64 + col0 + g + 8 * (e >> 1)];
+  }
+  if (GATE && threadIdx.x == 0) {
+    sm.g_tau = ga.tau[bh];
+    sm.g_tau_set = ga.tau_set[bh];
+    sm.g_routed = ga.counts[2 * bh];
   }
   __syncthreads();
 
   if (warp == kComputeWarps) {
     // ---------------- producer: TMA loads of K, V (and Q) tiles ----------------
     if (lane == 0) {
-      tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
-      if (HAS_Q) tma_prefetch_desc(&tmQ);
       const uint32_t stage_bytes = (HAS_Q ? 3u : 2u) * kTileBytes;
       int issued = 0;
       for (int t = 0; t < ntiles; ++t) {
         const int slot = t % kStages;
         if (t >= kStages && !mbar_wait(&sm.empty[slot], ((t / kStages) - 1) & 1, status, &sm.abort)) break;
-        mbar_arrive_expect_tx(&sm.full[slot], stage_bytes);
-        tma_load_3d(sm.K[slot], &tmK, &sm.full[slot], 0, t * kTileTok, bh);
-        tma_load_3d(sm.V[slot], &tmV, &sm.full[slot], 0, t * kTileTok, bh);
-        if (HAS_Q) tma_load_3d(sm.Q[slot], &tmQ, &sm.full[slot], 0, t * kTileTok, bh);
+        if (t != stall_tile) {
+          mbar_arrive_expect_tx(&sm.full[slot], stage_bytes);
+          tma_load_3d(sm.K[slot], &tmK, &sm.full[slot], 0, t * kTileTok, bh);
+          tma_load_3d(sm.V[slot], &tmV, &sm.full[slot], 0, t * kTileTok, bh);
+          if (HAS_Q) tma_load_3d(sm.Q[slot], &tmQ, &sm.full[slot], 0, t * kTileTok, bh);
+        }
         issued = t + 1;
       }
       // Nothing may still be landing in shared memory when the CTA exits.
       for (int t = issued - kStages; t < issued; ++t) {
-        if (t < 0) continue;
+        if (t < 0 || t == stall_tile) continue;
         mbar_wait(&sm.full[t % kStages], (t / kStages) & 1, status, nullptr);
       }
     }
@@ -375,14 +634,24 @@ __global__ void __launch_bounds__(b16_threads<true>(), 1)
       if (LOSS) {
         const int ntok = min(kTileTok, T - t * kTileTok);
         float* Lt = loss + (size_t)bh * T + (size_t)t * kTileTok;
+        // Each warp's sixteen columns as a pairwise tree over the lane groups, then the warps.
+        auto token_loss = [&](int i) {
+          float w[kComputeWarps];
+#pragma unroll
+          for (int cw = 0; cw < kComputeWarps; ++cw) {
+            const float* x = &sm.lossp[b][cw][0][i];
+            w[cw] = ((x[0 * kLossStride] + x[1 * kLossStride]) + (x[2 * kLossStride] + x[3 * kLossStride])) +
+                    ((x[4 * kLossStride] + x[5 * kLossStride]) + (x[6 * kLossStride] + x[7 * kLossStride]));
+          }
+          return (w[0] + w[1]) + (w[2] + w[3]);
+        };
         if (lane < ntok) {
-          v0 = (sm.lossp[b][0][lane] + sm.lossp[b][1][lane]) + (sm.lossp[b][2][lane] + sm.lossp[b][3][lane]);
+          v0 = token_loss(lane);
           Lt[lane] = v0;
         }
         if (lane + 32 < ntok) {
-          const int i = lane + 32;
-          v1 = (sm.lossp[b][0][i] + sm.lossp[b][1][i]) + (sm.lossp[b][2][i] + sm.lossp[b][3][i]);
-          Lt[i] = v1;
+          v1 = token_loss(lane + 32);
+          Lt[lane + 32] = v1;
         }
       }
       if (HAS_Q && lane == 0) {
@@ -472,14 +741,84 @@ __global__ void __launch_bounds__(b16_threads<true>(), 1)
   // ---------------- compute warps ----------------
   const int g = lane >> 2, q = lane & 3;
   const int col0 = 16 * warp;
-  float* Wg = Wstate + (size_t)bh * 64 * 64;
-  // Wᵀ slice in accumulator layout: acc[nt][e] = W[8nt + 2q + (e&1)][col0 + g + 8(e>>1)].
-  float acc[8][4];
-#pragma unroll
-  for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) acc[nt][e] = Wg[(8 * nt + 2 * q + (e & 1)) * 64 + col0 + g + 8 * (e >> 1)];
   const StepOffsets offs = step_offsets(lane, col0);
+
+  if constexpr (NB > 1) {
+    // ---- chunked form: chunks of NB blocks, Gram blocks one tile ahead ----
+    constexpr int kCPT = 64 / (16 * NB);          // chunks per tile
+    constexpr int kPPC = NB * (NB - 1) / 2;       // pairs per chunk
+    const int nfull = T / kTileTok, rem = (T % kTileTok) / 16;
+    const uint32_t gm0 = smem_u32(sm.gm[0]), gm1 = smem_u32(sm.gm[1]);
+    auto gram = [&](int tt) {  // this warp's share of tile tt's Gram blocks (a stale slot past the end: unused)
+      const int slot = tt % kStages;
+      gram_tile<NB, HAS_Q>(smem_u32(sm.K[slot]), smem_u32(sm.Q[slot]), (tt & 1) ? gm1 : gm0, offs, warp, lane);
+    };
+    bool ok = ntiles > 0 && warp_wait(&sm.full[0], 0, status, &sm.abort);
+    if (ok) {
+      gram(0);
+      mbar_arrive(&sm.gmready[0]);
+    }
+    int t = 0;
+    for (; ok && t < nfull; ++t) {
+      // Waits of the tile, tested without a branch (as in the per-step form): the output staging
+      // (last used by tile t − 2), the inputs of tile t+1 (read by the Gram share of tile t+1)
+      // and the Gram blocks of tile t.
+      const int t1 = t + 1;
+      const uint32_t pfree = ((t >> 1) + 1) & 1;
+      const uint32_t pfull = ((t1 / kStages) + (t1 < ntiles ? 0 : 1)) & 1;
+      const uint32_t pgm = (t >> 1) & 1;
+      const bool ready = mbar_try_wait(&sm.ofree[t & 1], pfree) & mbar_try_wait(&sm.full[t1 % kStages], pfull) &
+                         mbar_try_wait(&sm.gmready[t & 1], pgm);
+      if (!__all_sync(0xffffffffu, ready)) {
+        ok = warp_wait(&sm.ofree[t & 1], pfree, status, &sm.abort) &&
+             warp_wait(&sm.full[t1 % kStages], pfull, status, &sm.abort) &&
+             warp_wait(&sm.gmready[t & 1], pgm, status, &sm.abort);
+        if (!ok) break;
+      }
+      const int slot = t % kStages;
+      const uint32_t kb = smem_u32(sm.K[slot]), vb = smem_u32(sm.V[slot]), qb = smem_u32(sm.Q[slot]);
+      const uint32_t gb = (t & 1) ? gm1 : gm0, ob = smem_u32(sm.O[t & 1]);
+#pragma unroll
+      for (int cc = 0; cc < kCPT; ++cc)
+        chunk_run<NB, HAS_Q, LOSS>(acc, kb, vb, qb, gb + (uint32_t)(cc * kPPC) * kPairBytes, ob, offs,
+                                   &sm.lossp[t & 1][warp][0][0], 16 * NB * cc, lane, beta);
+      mbar_arrive(&sm.empty[slot]);  // every fragment of tile t has been read
+      // Tile t's Gram blocks have all been read by this warp: its share of tile t+1's may go into
+      // the other buffer (every warp passed the top of tile t, so none still reads tile t − 1's).
+      gram(t1);
+      mbar_arrive(&sm.gmready[t1 & 1]);
+      if (HAS_Q) fence_proxy_async_smem();
+      mbar_arrive(&sm.oready[t & 1]);
+    }
+    // A last tile of fewer than 64 tokens (rem 16-token blocks; its Gram blocks were made with
+    // the tile before, or in the prologue; rows past T were read as zeros).
+    if (ok && rem > 0) {
+      const bool w_ok = (t < 2 || warp_wait(&sm.ofree[t & 1], ((t >> 1) - 1) & 1, status, &sm.abort)) &&
+                        warp_wait(&sm.gmready[t & 1], (t >> 1) & 1, status, &sm.abort);
+      if (w_ok) {
+        const int slot = t % kStages;
+        const uint32_t kb = smem_u32(sm.K[slot]), vb = smem_u32(sm.V[slot]), qb = smem_u32(sm.Q[slot]);
+        const uint32_t gb = (t & 1) ? gm1 : gm0, ob = smem_u32(sm.O[t & 1]);
+        float* lp = &sm.lossp[t & 1][warp][0][0];
+        if (NB == 2) {
+          if (rem >= 2) chunk_run<2, HAS_Q, LOSS>(acc, kb, vb, qb, gb, ob, offs, lp, 0, lane, beta);
+          if (rem != 2) chunk_run<1, HAS_Q, LOSS>(acc, kb, vb, qb, gb, ob, offs, lp, rem == 1 ? 0 : 32, lane, beta);
+        } else {
+          if (rem == 1) chunk_run<1, HAS_Q, LOSS>(acc, kb, vb, qb, gb, ob, offs, lp, 0, lane, beta);
+          if (rem == 2) chunk_run<2, HAS_Q, LOSS>(acc, kb, vb, qb, gb, ob, offs, lp, 0, lane, beta);
+          if (rem == 3) chunk_run<3, HAS_Q, LOSS>(acc, kb, vb, qb, gb, ob, offs, lp, 0, lane, beta);
+        }
+        mbar_arrive(&sm.empty[slot]);
+        if (HAS_Q) fence_proxy_async_smem();
+        mbar_arrive(&sm.oready[t & 1]);
+      }
+    }
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) Wg[(8 * nt + 2 * q + (e & 1)) * 64 + col0 + g + 8 * (e >> 1)] = acc[nt][e];
+    return;
+  }
 
   // Fragments of step s (rows 16s .. 16s+15) of tile t are loaded one step before they are
   // used. A 64-token tile is four straight-line steps: every wait of the tile sits at its top
@@ -491,7 +830,7 @@ __global__ void __launch_bounds__(b16_threads<true>(), 1)
     load_frag16<HAS_Q>(F, smem_u32(sm.K[slot]), smem_u32(sm.V[slot]), smem_u32(sm.Q[slot]), offs, 16 * s);
   };
   auto comp = [&](const Frag16& F, int t, int s) {
-    compute16<HAS_Q, LOSS>(acc, F, smem_u32(sm.O[t & 1]), offs.o, sm.lossp[t & 1][warp], 16 * s, lane, beta);
+    compute16<HAS_Q, LOSS>(acc, F, smem_u32(sm.O[t & 1]), offs.o, &sm.lossp[t & 1][warp][0][0], 16 * s, lane, beta);
   };
 
   const int nfull = T / kTileTok, rem = (T % kTileTok) / 16;
@@ -552,7 +891,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     k_linear_scan(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
                   float* __restrict__ Wstate, float* __restrict__ loss, int T, float beta, int has_q,
-                  int* status) {
+                  const DevStatus status) {
   extern __shared__ uint8_t smem_raw[];
   LinearSmem& sm = *reinterpret_cast<LinearSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -772,14 +1111,55 @@ template <int B>
 ttt_status launch(ttt_state* st, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
                   const CUtensorMap& to, float* loss, int T, int has_q, cudaStream_t s) {
   const size_t smem = sizeof(LinearSmem) + 1024;
-  const uint32_t bit = 1u << (8 + B / 32);
+  const uint64_t bit = 1ull << (8 + B / 32);
   if (!(st->lin.smem_set & bit)) {
     TTT_CUDA(cudaFuncSetAttribute(k_linear_scan<B>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
     st->lin.smem_set |= bit;
   }
   const int grid = st->cfg.batch * st->cfg.heads;
   const float beta = st->cfg.eta / (float)B;
-  k_linear_scan<B><<<grid, kThreads, smem, s>>>(tk, tv, tq, to, st->lin.W, loss, T, beta, has_q, st->status.dev);
+  k_linear_scan<B><<<grid, kThreads, smem, s>>>(tk, tv, tq, to, st->lin.W, loss, T, beta, has_q,
+                                                DevStatus{st->status.dev, st->wait_limit_ns});
+  st->launches++;
+  TTT_CUDA(cudaGetLastError());
+  return TTT_OK;
+}
+
+template <bool HAS_Q, bool LOSS, bool GATE, int NB>
+ttt_status launch_b16_nb(ttt_state* st, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
+                         const CUtensorMap& to, float* loss, int T, const GateArgs& ga, cudaStream_t s) {
+  const size_t smem = sizeof(B16Smem) + 1024;
+  // One bit per instantiation whose shared-memory limit has been raised on this state's device.
+  const uint64_t bit = 1ull << (16 + 8 * (NB == 1 ? 0 : NB == 2 ? 1 : 2) + 4 * GATE + 2 * HAS_Q + LOSS);
+  if (!(st->lin.smem_set & bit)) {
+    TTT_CUDA(cudaFuncSetAttribute(k_linear_b16<HAS_Q, LOSS, GATE, NB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)smem));
+    st->lin.smem_set |= bit;
+  }
+  const int grid = st->cfg.batch * st->cfg.heads;
+  const float beta = st->cfg.eta / 16.0f;
+  // Fault injection (tests): the producer never loads tile 1, so the compute warps' wait for it
+  // runs out.
+  int stall_tile = -1;
+  if (st->inject_stall && T > 64) {
+    stall_tile = 1;
+    st->inject_stall = 0;
+  }
+  // Programmatic dependent launch: the kernel's set-up may overlap the end of the kernel before
+  // it in the stream (typically the previous scan); it waits for that kernel before reading
+  // anything.
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3((unsigned)grid);
+  lc.blockDim = dim3((unsigned)b16_threads<GATE>());
+  lc.dynamicSmemBytes = smem;
+  lc.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = attr;
+  lc.numAttrs = 1;
+  TTT_CUDA(cudaLaunchKernelEx(&lc, k_linear_b16<HAS_Q, LOSS, GATE, NB>, tk, tv, tq, to, st->lin.W, loss, T, beta,
+                              DevStatus{st->status.dev, st->wait_limit_ns}, ga, stall_tile));
   st->launches++;
   TTT_CUDA(cudaGetLastError());
   return TTT_OK;
@@ -788,20 +1168,11 @@ ttt_status launch(ttt_state* st, const CUtensorMap& tk, const CUtensorMap& tv, c
 template <bool HAS_Q, bool LOSS, bool GATE>
 ttt_status launch_b16_impl(ttt_state* st, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
                            const CUtensorMap& to, float* loss, int T, const GateArgs& ga, cudaStream_t s) {
-  const size_t smem = sizeof(B16Smem) + 1024;
-  const uint32_t bit = 1u << (4 * GATE + 2 * HAS_Q + LOSS);
-  if (!(st->lin.smem_set & bit)) {
-    TTT_CUDA(cudaFuncSetAttribute(k_linear_b16<HAS_Q, LOSS, GATE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)smem));
-    st->lin.smem_set |= bit;
+  switch (st->lin.form) {
+    case 2: return launch_b16_nb<HAS_Q, LOSS, GATE, 2>(st, tk, tv, tq, to, loss, T, ga, s);
+    case 4: return launch_b16_nb<HAS_Q, LOSS, GATE, 4>(st, tk, tv, tq, to, loss, T, ga, s);
+    default: return launch_b16_nb<HAS_Q, LOSS, GATE, 1>(st, tk, tv, tq, to, loss, T, ga, s);
   }
-  const int grid = st->cfg.batch * st->cfg.heads;
-  const float beta = st->cfg.eta / 16.0f;
-  k_linear_b16<HAS_Q, LOSS, GATE>
-      <<<grid, b16_threads<GATE>(), smem, s>>>(tk, tv, tq, to, st->lin.W, loss, T, beta, st->status.dev, ga);
-  st->launches++;
-  TTT_CUDA(cudaGetLastError());
-  return TTT_OK;
 }
 
 ttt_status launch_b16(ttt_state* st, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
@@ -836,22 +1207,30 @@ ttt_status linear_scan(ttt_state* st, const __nv_bfloat16* K, const __nv_bfloat1
   LinearBuffers& lb = st->lin;
   const bool has_q = Q != nullptr;
   const void* key[4] = {K, V, Q, O};
-  if (lb.map_T != T || lb.map_key[0] != key[0] || lb.map_key[1] != key[1] || lb.map_key[2] != key[2] ||
-      lb.map_key[3] != key[3]) {
-    lb.map_T = -1;  // invalid until all four are encoded
-    TTT_TRY(encode_tmap(&lb.maps[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, K, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B));
-    TTT_TRY(encode_tmap(&lb.maps[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, V, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B));
+  // Look the buffer set up among the cached ones; otherwise encode it into the least recently
+  // used entry.
+  LinearMapSet* ms = nullptr;
+  for (LinearMapSet& m : lb.map_sets)
+    if (m.T == T && m.key[0] == key[0] && m.key[1] == key[1] && m.key[2] == key[2] && m.key[3] == key[3]) ms = &m;
+  if (ms == nullptr) {
+    ms = &lb.map_sets[0];
+    for (LinearMapSet& m : lb.map_sets)
+      if (m.last_use < ms->last_use) ms = &m;
+    ms->T = -1;  // invalid until all four are encoded
+    TTT_TRY(encode_tmap(&ms->maps[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, K, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B));
+    TTT_TRY(encode_tmap(&ms->maps[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, V, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B));
     if (has_q) {
-      TTT_TRY(encode_tmap(&lb.maps[2], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, Q, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B));
-      TTT_TRY(encode_tmap(&lb.maps[3], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, O, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B));
+      TTT_TRY(encode_tmap(&ms->maps[2], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, Q, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B));
+      TTT_TRY(encode_tmap(&ms->maps[3], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, O, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B));
     } else {
-      lb.maps[2] = lb.maps[0];
-      lb.maps[3] = lb.maps[0];
+      ms->maps[2] = ms->maps[0];
+      ms->maps[3] = ms->maps[0];
     }
-    for (int i = 0; i < 4; ++i) lb.map_key[i] = key[i];
-    lb.map_T = T;
+    for (int i = 0; i < 4; ++i) ms->key[i] = key[i];
+    ms->T = T;
   }
-  const CUtensorMap &tk = lb.maps[0], &tv = lb.maps[1], &tq = lb.maps[2], &to = lb.maps[3];
+  ms->last_use = ++lb.map_clock;
+  const CUtensorMap &tk = ms->maps[0], &tv = ms->maps[1], &tq = ms->maps[2], &to = ms->maps[3];
   switch (c.chunk) {
     case 16: return launch_b16(st, tk, tv, tq, to, loss, (int)T, has_q, s);
     case 32: return launch<32>(st, tk, tv, tq, to, loss, (int)T, has_q, s);

@@ -10,11 +10,18 @@
 // library image. It allocates nothing: no cudaMalloc, no cudaFree, no allocating library
 // routine. The caller passes the inputs and the output.
 //
-// The fixed array (kScratchBytes, about 8.1 MB) is held by every GPU that loads the library
-// until the process exits. Every call shares it and it keeps the last call's contents;
-// every call overwrites all of the scratch it reads, so nothing needs clearing, but calls
-// whose GPU work overlaps (on different streams, or from different host threads without
+// The fixed array (kScratchBytes, about 8.1 MB) is a module variable: the CUDA runtime
+// creates it on a device when the library's module is first loaded there, which with lazy
+// module loading (the default since CUDA 12.2) is the first call's cudaGetSymbolAddress, and
+// at library load with CUDA_MODULE_LOADING=EAGER. That first call on a device may therefore
+// need about 8 MB of free device memory and may synchronise; from then on the device holds
+// the array until the process exits. Every call shares it and it keeps the last call's
+// contents; every call overwrites all of the scratch it reads, so nothing needs clearing, but
+// calls whose GPU work overlaps (on different streams, or from different host threads without
 // ordering) race on it.
+//
+// A bounded device-side wait that runs out is reported through the caller's optional status
+// word (a device int32 the call zeroes first), since there is no state to hold it.
 #include <mutex>
 
 #include "common.cuh"
@@ -25,7 +32,7 @@ namespace ttt {
 int target_values_plan_ints(int T, int d, int num_sms);
 ttt_status target_values_into(const __nv_bfloat16* X0, const float* convw, const __nv_bfloat16* Wtarget, int T, int d,
                               int C, int taps, int pad_mode, __nv_bfloat16* conv_scratch, int32_t* plan_scratch,
-                              __nv_bfloat16* out, int num_sms, cudaStream_t s);
+                              __nv_bfloat16* out, int32_t* status, int num_sms, cudaStream_t s);
 
 namespace {
 
@@ -75,13 +82,16 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 extern "C" ttt_status ttt_target_values_noalloc(const void* X0, const float* convw, const void* Wtarget, int64_t T,
                                                 int32_t d_model, int32_t chunk, int32_t conv_taps,
-                                                int32_t conv_pad_mode, void* Vhat_out, ttt_stream stream) {
+                                                int32_t conv_pad_mode, void* Vhat_out, int32_t* status,
+                                                ttt_stream stream) {
   using namespace ttt;
   if (T < 0) return fail(TTT_ERR_INVALID_ARG, "T must be non-negative");
   if (T == 0) return TTT_OK;
   if (X0 == nullptr || convw == nullptr || Wtarget == nullptr || Vhat_out == nullptr || !aligned16(X0) ||
       !aligned16(convw) || !aligned16(Wtarget) || !aligned16(Vhat_out))
     return fail(TTT_ERR_INVALID_ARG, "X0, convw, Wtarget and Vhat_out must be 16-byte aligned device pointers");
+  if (status != nullptr && (reinterpret_cast<uintptr_t>(status) & 3u) != 0)
+    return fail(TTT_ERR_INVALID_ARG, "status must be a 4-byte aligned device pointer or NULL");
   if (d_model < 8 || d_model % 8 != 0) return fail(TTT_ERR_UNSUPPORTED, "d_model must be a positive multiple of 8");
   if (T % 128 != 0) return fail(TTT_ERR_UNSUPPORTED, "T must be a multiple of 128");
   if (chunk < 1) return fail(TTT_ERR_INVALID_ARG, "chunk must be positive");
@@ -97,8 +107,10 @@ extern "C" ttt_status ttt_target_values_noalloc(const void* X0, const float* con
   if ((size_t)target_values_plan_ints((int)T, d_model, ds.num_sms) > kMaxPlanInts)
     return fail(TTT_ERR_INVALID_ARG, "too many tiles for the fixed schedule scratch");
   uint8_t* base = static_cast<uint8_t*>(ds.addr);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (status != nullptr) TTT_CUDA(cudaMemsetAsync(status, 0, sizeof(int32_t), s));
   return target_values_into(static_cast<const __nv_bfloat16*>(X0), convw, static_cast<const __nv_bfloat16*>(Wtarget),
                             (int)T, d_model, chunk, conv_taps, conv_pad_mode, reinterpret_cast<__nv_bfloat16*>(base),
                             reinterpret_cast<int32_t*>(base + kConvBytes), static_cast<__nv_bfloat16*>(Vhat_out),
-                            ds.num_sms, reinterpret_cast<cudaStream_t>(stream));
+                            status, ds.num_sms, s);
 }

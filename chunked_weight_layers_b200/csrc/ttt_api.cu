@@ -104,6 +104,7 @@ static void free_state(ttt_state* st) {
   if (st == nullptr) return;
   dev_free(st->ip.W);
   dev_free(st->ip.W0);
+  dev_free(st->ip.Wf32_next);
   dev_free(st->ip.Wsh[0]);
   dev_free(st->ip.Wsh[1]);
   dev_free(st->ip.Wsh[2]);
@@ -187,6 +188,7 @@ static ttt_status create_impl(const ttt_config* cfg, const void* W0, const void*
   const size_t nW = weight_elems(c);
   if (c.rule == TTT_RULE_INPLACE_HEBBIAN) {
     guard(dev_alloc((void**)&st->ip.W, nW * 4, "W")) && guard(dev_alloc((void**)&st->ip.W0, nW * 4, "W0"));
+    if (r == TTT_OK && c.io_dtype == TTT_F32) guard(dev_alloc((void**)&st->ip.Wf32_next, nW * 4, "W (next chunk)"));
     if (r == TTT_OK && c.io_dtype == TTT_BF16) {
       guard(dev_alloc((void**)&st->ip.Wsh[0], nW * 2, "W bf16 copy")) &&
           guard(dev_alloc((void**)&st->ip.Wsh[1], nW * 2, "W bf16 copy")) &&
@@ -453,6 +455,28 @@ ttt_status ttt_state_poll(ttt_state* st) {
   if (v == 0) return TTT_OK;
   if (v == TTT_ERR_TIMEOUT) return fail(TTT_ERR_TIMEOUT, "a bounded device-side wait ran out");
   return fail(TTT_ERR_DEVICE, "a device-side check failed (code %d)", v);
+}
+
+ttt_status ttt_state_set_option(ttt_state* st, int32_t option, int64_t value) {
+  if (st == nullptr) return fail(TTT_ERR_INVALID_ARG, "state is NULL");
+  switch (option) {
+    case TTT_OPT_LINEAR_CHUNK:
+      if (value != 0 && value != 1 && value != 2 && value != 4)
+        return fail(TTT_ERR_INVALID_ARG, "TTT_OPT_LINEAR_CHUNK must be 0, 1, 2 or 4 (got %lld)", (long long)value);
+      st->lin.form = (int)value;
+      return TTT_OK;
+    case TTT_OPT_WAIT_LIMIT_NS:
+      if (value < 1000 || value > 60000000000ll)
+        return fail(TTT_ERR_INVALID_ARG, "TTT_OPT_WAIT_LIMIT_NS must lie in [1000, 6e10] (got %lld)", (long long)value);
+      st->wait_limit_ns = (uint64_t)value;
+      return TTT_OK;
+    case TTT_OPT_INJECT_STALL:
+      if (value != 0 && value != 1) return fail(TTT_ERR_INVALID_ARG, "TTT_OPT_INJECT_STALL must be 0 or 1");
+      st->inject_stall = (int)value;
+      return TTT_OK;
+    default:
+      return fail(TTT_ERR_INVALID_ARG, "unknown option %d", option);
+  }
 }
 
 int64_t ttt_state_launch_count(const ttt_state* st) { return st == nullptr ? 0 : st->launches; }

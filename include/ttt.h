@@ -114,7 +114,9 @@ ttt_status ttt_config_init(ttt_config* cfg, int32_t rule);
  * W0, Wtarget and convw are copied; the caller may free them after the call returns
  * (stream-ordered). On success *out receives the state; on error *out is NULL and
  * nothing is leaked. Errors: INVALID_ARG (bad sizes or pointers), UNSUPPORTED (shape or
- * mode not implemented, see the message), OOM, CUDA. */
+ * mode not implemented, see the message), OOM, CUDA. The state starts at the pretrained
+ * weight ("In-Place Test-Time Training", §2: the MLP's own Wdown is the fast weight; the TTT
+ * layers page: the inner model's weight is the hidden state). */
 ttt_status ttt_state_create(const ttt_config* cfg, const void* W0, const void* Wtarget,
                             const float* convw, ttt_stream stream, ttt_state** out);
 
@@ -127,7 +129,12 @@ ttt_status ttt_state_create(const ttt_config* cfg, const void* W0, const void* W
  *               loss_out = L [batch, heads, T] fp32 (or NULL; required when the gate is
  *               enabled). T must be a multiple of chunk (and of gate_chunk with the gate).
  * All inputs are read-only; outputs are written with the io dtype (loss fp32). Inputs and
- * outputs must not overlap. T = 0 is a no-op. Errors: INVALID_ARG, UNSUPPORTED, CUDA. */
+ * outputs must not overlap. T = 0 is a no-op. Errors: INVALID_ARG, UNSUPPORTED, CUDA.
+ * Defined by "In-Place Test-Time Training", §3 (each chunk is applied with the weight from
+ * before it, then the weight is updated from that chunk) and §4 (the next-token-aligned
+ * target Conv1D(X0)·Wtarget, with padding at chunk boundaries from §6), and by the TTT
+ * layers page (one self-supervised gradient step of the inner linear model per mini-batch;
+ * with b = 1 and no normalisation it is the delta rule). */
 ttt_status ttt_chunk_scan(ttt_state* st, const void* keys, const void* targets,
                           const void* queries, int64_t T, void* out, float* loss_out,
                           ttt_stream stream);
@@ -143,27 +150,41 @@ ttt_status ttt_chunk_scan_host(ttt_state* st, const void* keys, const void* targ
  * advancing the state's τ, cache and token position exactly as a gated scan would.
  * TTT-Linear states only; T must be a multiple of gate_chunk. The token position (stored
  * in the cache as int32) may not pass 2^31 − 1 between resets: a gated call that would take
- * it there (this one or ttt_chunk_scan with the gate on) returns UNSUPPORTED. */
+ * it there (this one or ttt_chunk_scan with the gate on) returns UNSUPPORTED. Defined by
+ * "SR-TTT: Surprisal-Aware Residual Test-Time Training", §2.1 (the loss gate's two
+ * conditions and the residual cache). */
 ttt_status ttt_surprisal_route(ttt_state* st, const float* loss, int64_t T, ttt_stream stream);
 
 /* Document boundary: W ← W0, τ unset, cache emptied (entries -1, counts 0), token
- * position 0. */
+ * position 0. Defined by "In-Place Test-Time Training", §6 (implementation notes: when an
+ * independent document ends, the fast weight goes back to its pretrained value so that no
+ * information leaks from one document into the next; §8 repeats that the fast weight lives
+ * only within a document). The gate's threshold and cache are per-document state of the
+ * same scan ("SR-TTT", §2.1), so they restart with it. */
 ttt_status ttt_state_reset(ttt_state* st, ttt_stream stream);
 
 /* Copy the current fp32 weights out of / into the state (device buffers shaped like W0).
- * set_weights also refreshes the In-Place bf16 copy used by the apply. */
+ * set_weights also refreshes the In-Place bf16 copy used by the apply. The weight is the
+ * scan's whole recurrent state (the TTT layers page: the hidden state is the inner model's
+ * weight; "In-Place Test-Time Training", §2: Wdown is that weight), so saving it and setting
+ * it back resumes a scan exactly at a chunk boundary. */
 ttt_status ttt_state_get_weights(const ttt_state* st, float* W, ttt_stream stream);
 ttt_status ttt_state_set_weights(ttt_state* st, const float* W, ttt_stream stream);
 
 /* Copy out the residual cache: entries (device) int32 [batch, heads, cache_capacity, 3]
  * holding (sequence, head, t) with t counted from the last reset, unused entries -1;
  * counts (device) int32 [batch, heads, 2] = (tokens routed, routed tokens dropped).
- * Either pointer may be NULL. */
+ * Either pointer may be NULL. The cache is the fixed-capacity store of the tokens the gate
+ * finds incompressible ("SR-TTT: Surprisal-Aware Residual Test-Time Training", §2.1,
+ * "Residual Cache"); this library keeps the first cache_capacity of them in token order and
+ * counts the rest as dropped. */
 ttt_status ttt_cache_read(const ttt_state* st, int32_t* entries, int32_t* counts,
                           ttt_stream stream);
 
 /* Copy out the gate thresholds: tau (device) fp32 [batch, heads]; tau_set (device) int32
- * [batch, heads], 1 once a chunk has set τ. Either pointer may be NULL. */
+ * [batch, heads], 1 once a chunk has set τ. Either pointer may be NULL. τ is the
+ * EMA-smoothed 95th percentile of the per-token losses ("SR-TTT", §2.1, the gate's first
+ * condition). */
 ttt_status ttt_gate_read(const ttt_state* st, float* tau, int32_t* tau_set, ttt_stream stream);
 
 /* Target generation V̂ = Conv1D(X0)·Wtarget for T tokens without allocating device memory.
@@ -173,24 +194,60 @@ ttt_status ttt_gate_read(const ttt_state* st, float* tau, int32_t* tau_set, ttt_
  * start-up (cudaMalloc can block and synchronise the device). It computes the same values
  * as the fused target of an In-Place state with target_mode 1 (same kernels), but keeps its
  * scratch (the conv rows and the tile schedule) in one fixed array of device memory inside
- * the library image (about 8.1 MB, held by every GPU that loads the library until exit)
- * instead of state memory, and calls no cudaMalloc, cudaFree or allocating routine.
+ * the library image (about 8.1 MB) instead of state memory, and calls no cudaMalloc, cudaFree
+ * or allocating routine.
  *   X0       device bf16 [T, d_model], the token embeddings.
  *   convw    device fp32 [d_model, conv_taps], depthwise taps at token offsets 0..taps-1.
  *   Wtarget  device bf16 [d_model, d_model], [in, out].
  *   chunk    taps read zero past the end of each chunk of this many tokens (conv_pad_mode 0)
  *            or past token T only (conv_pad_mode 1).
  *   Vhat_out device bf16 [T, d_model], written.
+ *   status   device int32 or NULL. If given, the call first sets it to 0 (stream-ordered)
+ *            and a bounded device-side wait that runs out sets it to TTT_ERR_TIMEOUT (then
+ *            Vhat_out is incomplete); read it after the stream's work has finished.
  * Limits: T a multiple of 128, d_model a multiple of 8, T·d_model ≤ 4,194,304; larger inputs
- * are rejected with TTT_ERR_INVALID_ARG and a message naming the limit. The first call on
- * each device looks up the device address of the fixed array (cudaGetSymbolAddress with
- * that device current); make that first call before any stream capture. All calls share
+ * are rejected with TTT_ERR_INVALID_ARG and a message naming the limit. The fixed array is
+ * created on a device when the library's module is first loaded there: with lazy module
+ * loading (the CUDA default) that is this entry point's first call on the device, with
+ * CUDA_MODULE_LOADING=EAGER it is library load; from then on the device holds it until the
+ * process exits. The first call on each device therefore may need about 8 MB of free device
+ * memory and may synchronise: it looks up the array's device address (cudaGetSymbolAddress
+ * with that device current). Make that first call before any stream capture. All calls share
  * the array and it keeps the last call's contents: calls whose GPU work overlaps (other
- * streams, other host threads) race on it. A bounded device-side wait that runs out is not
- * reported by this entry point (there is no state to hold the status). */
+ * streams, other host threads) race on it. */
 ttt_status ttt_target_values_noalloc(const void* X0, const float* convw, const void* Wtarget, int64_t T,
                                      int32_t d_model, int32_t chunk, int32_t conv_taps, int32_t conv_pad_mode,
-                                     void* Vhat_out, ttt_stream stream);
+                                     void* Vhat_out, int32_t* status, ttt_stream stream);
+
+/* Options of a state, set after creation (ttt_state_set_option). */
+typedef enum {
+  /* TTT-Linear with b = 16: how many inner mini-batches the scan groups into one chunk.
+   * 1 runs the mini-batch steps one after another. 2 or 4 run the chunked form: inside a
+   * chunk every product with W uses the weight from the chunk's start, and each mini-batch's
+   * residual is corrected by those of the mini-batches before it through the Gram blocks
+   * K_i·K_jᵀ (and Q_i·K_jᵀ for the outputs). That is the same sequence of weights and outputs
+   * as the step-by-step rule, regrouped (rounding differs); results are bit-identical between
+   * a single call and calls split at multiples of 16·value tokens. 0 selects the default (1,
+   * the fastest on B200: the chunked forms issue more tensor-core work per token and the
+   * step chain is not what bounds this kernel). Other rules and mini-batch sizes ignore it. */
+  TTT_OPT_LINEAR_CHUNK = 1,
+  /* Limit of every spin-wait of this state's kernels, in nanoseconds of the GPU's global
+   * timer: a wait that lasts longer records TTT_ERR_TIMEOUT (read by ttt_state_poll), the
+   * kernel drains its own copies and tensor-core work in flight (each with the same limit),
+   * releases its tensor memory and returns. Range [1000, 60e9]; default 2e9 (2 s). */
+  TTT_OPT_WAIT_LIMIT_NS = 2,
+  /* Fault injection for tests of the path above, value 1: the next scan that can (an In-Place
+   * BF16 scan of two or more chunks, or a TTT-Linear b = 16 scan longer than 64 tokens) makes
+   * one of its bounded waits wait for something that never comes — an In-Place APPLY tile of
+   * the second chunk waits for one more finished UPDATE tile than exists; the TTT-Linear scan
+   * never loads its second 64-token tile — so that the wait runs out. The outputs of that scan
+   * are incomplete. 0 cancels a pending injection. */
+  TTT_OPT_INJECT_STALL = 3
+} ttt_option;
+
+/* Set option `option` of state `st` to `value`. Takes effect from the next call that
+ * enqueues work. Errors: INVALID_ARG (unknown option or value out of range). */
+ttt_status ttt_state_set_option(ttt_state* st, int32_t option, int64_t value);
 
 /* Synchronise the device and return the first device-side failure recorded since the
  * last poll (TTT_ERR_TIMEOUT or TTT_ERR_DEVICE), or TTT_OK; clears the record. */

@@ -27,10 +27,13 @@ def cwl():
     return cwl
 
 
-def gate_state(cwl, B, H, cap=256):
+def gate_state(cwl, B, H, cap=256, form=None):
     W0 = torch.eye(64, device="cuda").expand(B, H, 64, 64).contiguous()
     cfg = cwl.config("linear", batch=B, heads=H, chunk=16, gate_enable=1, cache_capacity=cap)
-    return cwl.FastWeightState(cfg, W0)
+    st = cwl.FastWeightState(cfg, W0)
+    if form is not None:
+        st.set_option(cwl.abi.TTT_OPT_LINEAR_CHUNK, form)
+    return st
 
 
 def read_gate(st, B, H, cap):
@@ -114,20 +117,32 @@ def test_streaming_calls_and_reset(cwl):
     assert_same_as_oracle(*read_gate(st, B, H, 64), ref)
 
 
-def test_gated_scan_workload(cwl):
+@pytest.fixture(scope="module")
+def gate_workload_ref():
+    spec = workloads.SR_TTT_GATE
+    x = workloads.linear_inputs(spec, device="cpu")
+    _, Wref, Lref = olin.ttt_linear_scan(x["K"], x["V"], None, x["W0"], spec.eta, spec.b)
+    ref2 = ogate.GateState(spec.B, spec.H, 256)
+    ogate.surprisal_route(Lref.astype(np.float32), ref2)
+    return Wref, Lref, ref2
+
+
+@pytest.mark.parametrize("form", [1, 2, 4])
+def test_gated_scan_workload(cwl, gate_workload_ref, form):
     """The SR-TTT workload: losses within tolerance of the oracle's; the oracle's gate on
     the GPU's losses reproduces the GPU cache exactly; against the oracle's own losses,
-    routing may differ only for tokens or chunks within rounding of τ."""
+    routing may differ only for tokens or chunks within rounding of τ. For the step-by-step
+    form and both chunked forms of the scan."""
     spec = workloads.SR_TTT_GATE
     x = workloads.linear_inputs(spec, device="cuda")
     B, H, T = spec.B, spec.H, spec.T
-    st = gate_state(cwl, B, H)
+    st = gate_state(cwl, B, H, form=form)
     L = torch.empty((B, H, T), device="cuda")
     st.chunk_scan(x["K"], x["V"], None, out=None, loss_out=L)
     W = torch.empty_like(x["W0"])
     st.get_weights(W)
     E, C, tau, ts = read_gate(st, B, H, 256)
-    _, Wref, Lref = olin.ttt_linear_scan(x["K"].cpu(), x["V"].cpu(), None, x["W0"].cpu(), spec.eta, spec.b)
+    Wref, Lref, ref2 = gate_workload_ref
     el, ew = rel_err(L, Lref), rel_err(W, Wref)
     print(f"SR-TTT workload: loss {el:.3e}  W {ew:.3e}  routed {int(C[..., 0].sum())}")
     assert el <= 2e-2 and ew <= 2e-2
@@ -138,8 +153,6 @@ def test_gated_scan_workload(cwl):
     # Needles are what the gate catches.
     assert int(C[..., 0].sum()) > 0
     # Against the oracle's own losses: differences only at the rounding margin.
-    ref2 = ogate.GateState(B, H, 256)
-    ogate.surprisal_route(Lref.astype(np.float32), ref2)
     diff = 0
     for b in range(B):
         for h in range(H):
@@ -150,8 +163,9 @@ def test_gated_scan_workload(cwl):
     assert diff <= 0.02 * max(1, int(C[..., 0].sum()))
 
 
+@pytest.mark.parametrize("form", [1, 2, 4])
 @pytest.mark.parametrize("with_q", [False, True])
-def test_gate_inside_the_scan_streams_and_saturates(cwl, with_q):
+def test_gate_inside_the_scan_streams_and_saturates(cwl, with_q, form):
     """The b = 16 scan runs the gate in its own kernel, tile by tile. Two calls (tokens
     0..319 and 320..767) with a cache of 8 entries, so it fills up and drops: the cache,
     counts and τ equal the oracle's gate run over the GPU's losses of both calls, bit for
@@ -159,7 +173,7 @@ def test_gate_inside_the_scan_streams_and_saturates(cwl, with_q):
     spec = workloads.scaled(workloads.SR_TTT_GATE, B=2, H=3, T=768, seed=91)
     x = workloads.linear_inputs(spec, device="cuda")
     B, H, T, cap = spec.B, spec.H, spec.T, 8
-    st = gate_state(cwl, B, H, cap)
+    st = gate_state(cwl, B, H, cap, form=form)
     losses = []
     for a, z in ((0, 320), (320, T)):
         K, V = (x[n][:, :, a:z].contiguous() for n in ("K", "V"))

@@ -57,7 +57,7 @@ def test_fp32_workload_full_size(cwl):
     eo, ew = rel_err(O, Oref), rel_err(W, Wref)
     print(f"fp32 workload: O rel err {eo:.3e}, W rel err {ew:.3e}")
     assert eo <= 1e-4 and ew <= 1e-4
-    assert st.launch_count() >= 2 * (spec.T // spec.C)
+    assert st.launch_count() >= spec.T // spec.C  # one launch per chunk
 
 
 def test_ragged_shapes(cwl):
