@@ -266,8 +266,9 @@ def dominant_kernel(spec) -> str:
 
 
 def traffic_per_launch(spec):
-    """DRAM bytes per launch of the workload's dominant kernel from the committed ncu record,
-    or None when there is none or the kernel's source changed since the capture."""
+    """DRAM bytes per step of the workload's dominant kernel (its bytes per launch times its
+    launches per step) from the committed ncu record, or None when there is none or the
+    kernel's source changed since the capture."""
     import hashlib
     p = os.path.join(ROOT, "profiles", "dram_traffic.json")
     if not os.path.exists(p):
@@ -279,7 +280,9 @@ def traffic_per_launch(spec):
     if not os.path.exists(src):
         return None
     digest = hashlib.sha256(open(src, "rb").read()).hexdigest()
-    return rec["bytes_per_launch"] if digest.startswith(rec["sha256_prefix"]) else None
+    if not digest.startswith(rec["sha256_prefix"]):
+        return None
+    return rec["bytes_per_launch"] * rec.get("launches_per_step", 1)
 
 
 def roofline(spec, w, ms, peaks, traffic=None):
@@ -417,6 +420,9 @@ def main():
     ap.add_argument("--tokens", type=int, default=None,
                     help="run the named workload with this many tokens instead (same widths and chunk; a smaller "
                          "case for profilers, not a bench line)")
+    ap.add_argument("--profile", type=int, default=None, metavar="N",
+                    help="for profilers: build the named workload, run one warm-up step and N more steps, print "
+                         "nothing else (no timing, no end-to-end pass, no oracle)")
     a = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -452,6 +458,19 @@ def main():
                           "data": "synthetic", "config": bench_config(spec, world), "cpu_baseline": cb,
                           "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                                   "d2h_bytes_per_step": 0}}))
+        return
+
+    if a.profile is not None:
+        torch.cuda.set_device(local)
+        from chunked_weight_layers_b200 import build
+        build.build()
+        runner = Runner(spec, torch.device("cuda", local))
+        runner.state.reset()
+        for k in range(1 + a.profile):
+            runner.step(k)
+        torch.cuda.synchronize()
+        runner.state.poll()
+        print(f"profiled {spec.name}: 1 + {a.profile} steps, {runner.state.launch_count()} library launches")
         return
 
     if a.warmup < 3:
