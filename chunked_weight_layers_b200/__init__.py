@@ -141,6 +141,22 @@ class FastWeightState:
         check(self._lib.ttt_surprisal_route(self._h, _arg(loss, "loss", torch.float32, self._bh * T, _current_device()),
                                             int(T), _stream(stream)))
 
+    def cache_attention(self, queries, keys, values, o_ttt, alpha, out=None, T=None, stream=None):
+        """ttt_cache_attention: ``out`` (default: ``o_ttt``, updated in place) = o_ttt +
+        clamp(alpha, 0, 1) ⊙ the attention of each query over the cache entries it may see."""
+        if T is None:
+            T = keys.shape[-2]
+        if out is None:
+            out = o_ttt
+        dev = _current_device()
+        n = self._bh * T * self._dk
+        check(self._lib.ttt_cache_attention(
+            self._h, _arg(queries, "queries", torch.bfloat16, n, dev), _arg(keys, "keys", torch.bfloat16, n, dev),
+            _arg(values, "values", torch.bfloat16, n, dev), _arg(o_ttt, "o_ttt", torch.bfloat16, n, dev),
+            _arg(alpha, "alpha", torch.float32, self.cfg.heads * self._dk, dev), int(T),
+            _arg(out, "out", torch.bfloat16, n, dev), _stream(stream)))
+        return out
+
     def reset(self, stream=None):
         check(self._lib.ttt_state_reset(self._h, _stream(stream)))
 

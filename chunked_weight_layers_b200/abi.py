@@ -72,6 +72,7 @@ _SIGNATURES = {
     "ttt_cache_read": (_st, [_vp, _vp, _vp, _vp]),
     "ttt_gate_read": (_st, [_vp, _vp, _vp, _vp]),
     "ttt_state_set_option": (_st, [_vp, ctypes.c_int32, ctypes.c_int64]),
+    "ttt_cache_attention": (_st, [_vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_int64, _vp, _vp]),
     "ttt_state_poll": (_st, [_vp]),
     "ttt_state_launch_count": (ctypes.c_int64, [_vp]),
     "ttt_state_destroy": (_st, [_vp]),

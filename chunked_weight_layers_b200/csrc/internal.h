@@ -132,6 +132,11 @@ ttt_status linear_scan(ttt_state* st, const __nv_bfloat16* K, const __nv_bfloat1
                        const __nv_bfloat16* Q, int64_t T, __nv_bfloat16* O, float* loss,
                        cudaStream_t s);
 
+// Residual-cache read path: out = o_ttt + clamp(α, 0, 1) ⊙ (attention over the visible entries).
+ttt_status cache_attention(const ttt_state* st, const __nv_bfloat16* Q, const __nv_bfloat16* K,
+                           const __nv_bfloat16* V, const __nv_bfloat16* O_ttt, const float* alpha, int64_t T,
+                           __nv_bfloat16* out, cudaStream_t s);
+
 // Surprisal gate over T losses of every (sequence, head).
 ttt_status gate_route(ttt_state* st, const float* loss, int64_t T, cudaStream_t s);
 // Nearest rank ceil(gate_pct·64) of the gate's percentile (1-based).

@@ -399,6 +399,24 @@ ttt_status ttt_surprisal_route(ttt_state* st, const float* loss, int64_t T, ttt_
   return gate_route(st, loss, T, reinterpret_cast<cudaStream_t>(stream));
 }
 
+ttt_status ttt_cache_attention(const ttt_state* st, const void* queries, const void* keys, const void* values,
+                               const void* o_ttt, const float* alpha, int64_t T, void* out, ttt_stream stream) {
+  if (st == nullptr) return fail(TTT_ERR_INVALID_ARG, "state is NULL");
+  if (st->cfg.rule != TTT_RULE_LINEAR_GD || !st->cfg.gate_enable)
+    return fail(TTT_ERR_UNSUPPORTED, "the cache read path needs a TTT-Linear state with the gate enabled");
+  if (T <= 0 || T != st->gate.t_offset)
+    return fail(TTT_ERR_INVALID_ARG, "T=%lld must equal the tokens scanned since the last reset (%lld)",
+                (long long)T, (long long)st->gate.t_offset);
+  const void* p[6] = {queries, keys, values, o_ttt, alpha, out};
+  for (const void* x : p)
+    if (x == nullptr || !aligned16(x))
+      return fail(TTT_ERR_INVALID_ARG, "queries, keys, values, o_ttt, alpha and out must be 16-byte aligned device pointers");
+  TTT_TRY(check_device(st));
+  return cache_attention(st, static_cast<const __nv_bfloat16*>(queries), static_cast<const __nv_bfloat16*>(keys),
+                         static_cast<const __nv_bfloat16*>(values), static_cast<const __nv_bfloat16*>(o_ttt), alpha, T,
+                         static_cast<__nv_bfloat16*>(out), reinterpret_cast<cudaStream_t>(stream));
+}
+
 ttt_status ttt_state_reset(ttt_state* st, ttt_stream stream) {
   if (st == nullptr) return fail(TTT_ERR_INVALID_ARG, "state is NULL");
   TTT_TRY(check_device(st));

@@ -187,6 +187,24 @@ ttt_status ttt_cache_read(const ttt_state* st, int32_t* entries, int32_t* counts
  * condition). */
 ttt_status ttt_gate_read(const ttt_state* st, float* tau, int32_t* tau_set, ttt_stream stream);
 
+/* Read path of the residual cache ("SR-TTT: Surprisal-Aware Residual Test-Time Training", §2.1,
+ * "Residual Cache" and "Alpha Fusion"): the layer's output is the TTT output plus the cache's
+ * attention output weighted by the gate vector α, clamped to [0, 1]:
+ *   out[b,h,t] = o_ttt[b,h,t] + clamp(α[h], 0, 1) ⊙ Σ_j softmax_j(q_t·k_j / √64)·v_j
+ * over the cache entries j of (b, h) that token t may see: those whose 64-token gate chunk lies
+ * before t's (a token's routing is known once its gate chunk has been scanned). The keys and
+ * values of an entry are the scanned K and V rows of its token. A query that sees no entry adds
+ * nothing (out = o_ttt).
+ *   queries, keys, values, o_ttt  device bf16 [batch, heads, T, 64]: the Q, K and V of all T
+ *            tokens scanned since the last reset (T must equal that count) and the scan's
+ *            outputs.
+ *   alpha    device fp32 [heads, 64].
+ *   out      device bf16 [batch, heads, T, 64]; may be o_ttt itself (updated in place).
+ * TTT-Linear states with the gate, cache_capacity ≤ 256. The cache is read as the gate left it
+ * on the stream. Errors: INVALID_ARG (sizes, pointers, T), UNSUPPORTED, CUDA. */
+ttt_status ttt_cache_attention(const ttt_state* st, const void* queries, const void* keys, const void* values,
+                               const void* o_ttt, const float* alpha, int64_t T, void* out, ttt_stream stream);
+
 /* Target generation V̂ = Conv1D(X0)·Wtarget for T tokens without allocating device memory.
  * The pages have no counterpart of this entry point: it exists for callers that cannot call
  * cudaMalloc where they need the work done — their device memory is owned by another
