@@ -95,7 +95,7 @@ class Runner:
     by the time a copy comes round again, the steps in between have moved more than the L2
     holds, so every step reads its inputs from HBM."""
 
-    def __init__(self, spec, device):
+    def __init__(self, spec, device, prefix=False):
         import chunked_weight_layers_b200 as cwl
         self.spec = spec
         self.cwl = cwl
@@ -115,6 +115,8 @@ class Runner:
             cfg = cwl.config("inplace", io_dtype=io, d_key=spec.f, d_val=spec.d, chunk=spec.C, eta=spec.eta,
                              target_mode=int(spec.target), conv_pad_mode=spec.conv_pad_mode)
             self.state = cwl.FastWeightState(cfg, x["W0"], x.get("Wtarget"), x.get("convw"))
+            if prefix:
+                self.state.set_option(cwl.abi.TTT_OPT_INPLACE_PREFIX, 1)
             args = dict(keys=x["Z"], targets=x["X0"] if spec.target else x["Vhat"], queries=None)
             out = torch.empty((spec.T, spec.d), device=device, dtype=x["Z"].dtype)
             loss = None
@@ -313,7 +315,7 @@ def oracle_threads() -> int:
     return os.cpu_count() or 1
 
 
-def cpu_baseline(spec, limit_s=12.0) -> dict:
+def cpu_baseline(spec, limit_s=12.0, prefix=False) -> dict:
     """The oracle as it stands on this host's cores, on a bounded sample of the workload.
 
     ``cores`` is the BLAS pool the oracle's matmuls run on; ``busy_threads`` is the process's
@@ -353,9 +355,10 @@ def cpu_baseline(spec, limit_s=12.0) -> dict:
         if Vh is None:
             Vh = torch.from_numpy(oinp.target_values(x["X0"], x["convw"], x["Wtarget"], spec.C))
         T = x["Z"].shape[0]
+        scan_fn = oinp.inplace_scan_prefix if prefix else oinp.inplace_scan
         while time.perf_counter() - t0 < limit_s and chunks * Cs < T:
             sl = slice(chunks * Cs, (chunks + 1) * Cs)
-            _, W = oinp.inplace_scan(x["Z"][sl], Vh[sl], W, spec.eta, Cs)
+            _, W = scan_fn(x["Z"][sl], Vh[sl], W, spec.eta, Cs)
             chunks += 1
         dt = time.perf_counter() - t0
         tokens = chunks * Cs
@@ -365,17 +368,19 @@ def cpu_baseline(spec, limit_s=12.0) -> dict:
             "kind": "oracle", "sample": sample, "seconds": dt}
 
 
-def measure(spec, steps, warmup, peaks, device, with_e2e, cpu_limit_s=None):
+def measure(spec, steps, warmup, peaks, device, with_e2e, cpu_limit_s=None, prefix=False):
     """One workload measured like the main line: device time per scan (mean over the timed
     steps, median beside it), its roofline, end-to-end time through the host-buffer call, and
     (with ``cpu_limit_s``) the oracle on a bounded sample of it."""
-    r = Runner(spec, device)
+    r = Runner(spec, device, prefix=prefix)
     total, launches, times = time_steps(r, steps, warmup)
     ms = total / steps
     w = work(spec)
     rl = roofline(spec, w, ms, peaks, traffic_per_launch(spec))
-    rl["kernel"] = dominant_kernel(spec)
-    out = {"workload": spec.name, "ms_per_step": ms, "ms_median": statistics.median(times),
+    rl["kernel"] = "k_gemm_tc" if prefix else dominant_kernel(spec)
+    if prefix:
+        rl["traffic"] = None  # no ncu capture of this form is recorded
+    out = {"workload": spec.name + (" (context-parallel form)" if prefix else ""), "ms_per_step": ms, "ms_median": statistics.median(times),
            "tokens_per_s": w["tokens"] / (ms * 1e-3), "tflops": w["flops"] / (ms * 1e-3) / 1e12,
            "roofline": rl, "gpu_launches_per_step": launches / max(1, steps), "times_ms": times,
            "host_ms_per_step": r.host_ms, "l2": r.l2_note()}
@@ -392,6 +397,110 @@ def measure(spec, steps, warmup, peaks, device, with_e2e, cpu_limit_s=None):
     if cpu_limit_s is not None:
         out["cpu_baseline"] = cpu_baseline(spec, cpu_limit_s)
     return out
+
+
+CACHE_READ = "srttt_cache_read_B4_H16_T8192"
+
+
+def _cache_read_setup(device):
+    """A gated scan of the SR-TTT workload with queries drawn as well (its cache is what the read
+    path reads), and a gate vector α."""
+    import chunked_weight_layers_b200 as cwl
+    spec = wl.scaled(wl.SR_TTT_GATE, with_queries=True)
+    x = wl.linear_inputs(spec, device=device)
+    cfg = cwl.config("linear", batch=spec.B, heads=spec.H, chunk=spec.b, eta=spec.eta, gate_enable=1)
+    st = cwl.FastWeightState(cfg, x["W0"])
+    O = torch.empty_like(x["K"])
+    st.chunk_scan(x["K"], x["V"], x["Q"], out=O, loss_out=torch.empty((spec.B, spec.H, spec.T), device=device))
+    alpha = torch.full((spec.H, 64), 0.25, device=device)
+    return spec, x, st, O, alpha
+
+
+def cache_read_work(spec, counts, entries) -> dict:
+    """Bytes (Q and o_ttt read, out written, cached K and V rows gathered per query block) and
+    flops (4·64 per query and visible entry, for Q·Kᵀ and P·V) of one read-path call."""
+    n = spec.B * spec.H * spec.T * 64
+    flops, gathered = 0, 0
+    E = entries.cpu().numpy()
+    C = counts.cpu().numpy()
+    for b in range(spec.B):
+        for h in range(spec.H):
+            m = min(int(C[b, h, 0]), E.shape[2])
+            toks = E[b, h, :m, 2]
+            for g in range(spec.T // 64):
+                vis = int((toks < 64 * g).sum())
+                flops += 4 * 64 * 64 * vis
+                gathered += 2 * vis * 128
+    return {"tokens": spec.B * spec.T, "flops": flops, "bytes": 3 * n * 2 + gathered, "bound": "hbm"}
+
+
+def measure_cache_read(steps, warmup, peaks, device):
+    spec, x, st, O, alpha = _cache_read_setup(device)
+    E = torch.empty((spec.B, spec.H, 256, 3), device=device, dtype=torch.int32)
+    C = torch.empty((spec.B, spec.H, 2), device=device, dtype=torch.int32)
+    st.cache_read(E, C)
+    w = cache_read_work(spec, C, E)
+    n_sets = max(1, -(-3 * L2_BYTES // w["bytes"]))
+    sets = [(x["Q"], O, torch.empty_like(O))] + [(x["Q"].clone(), O.clone(), torch.empty_like(O))
+                                                 for _ in range(n_sets - 1)]
+    stream = torch.cuda.current_stream()
+    for k in range(warmup):
+        q, o, out = sets[k % n_sets]
+        st.cache_attention(q, x["K"], x["V"], o, alpha, out=out)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    h0 = time.perf_counter()
+    for k in range(steps):
+        q, o, out = sets[k % n_sets]
+        st.cache_attention(q, x["K"], x["V"], o, alpha, out=out)
+    host_ms = (time.perf_counter() - h0) * 1e3 / steps
+    e1.record(stream)
+    e1.synchronize()
+    st.poll()
+    ms = e0.elapsed_time(e1) / steps
+    achieved = w["bytes"] / (ms * 1e-3) / 1e9
+    out = {"workload": CACHE_READ, "ms_per_step": ms, "tokens_per_s": w["tokens"] / (ms * 1e-3),
+           "tflops": w["flops"] / (ms * 1e-3) / 1e12,
+           "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                        "frac": achieved / peaks["hbm_gbs"], "traffic": None, "peak_source": peaks["source"],
+                        "kernel": "k_cache_attn",
+                        "tensor_frac": w["flops"] / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"]},
+           "gpu_launches_per_step": 1.0, "host_ms_per_step": host_ms,
+           "l2": f"inputs larger than L2: {n_sets} copies of the call's queries and outputs taken in turn",
+           "e2e": None, "e2e_note": "the read path has no host-buffer entry point"}
+    st.close()
+    torch.cuda.empty_cache()
+    return out
+
+
+def cpu_baseline_cache_read(limit_s) -> dict:
+    """The oracle's read path (attention over the visible entries, α fusion) on (sequence, head)
+    pairs of the gate workload's cache, one at a time, within the time limit."""
+    from oracle import cache_attention as oca
+    from oracle import gate as ogate
+    from oracle import linear as olin
+    spec = wl.scaled(wl.SR_TTT_GATE, with_queries=True)
+    x = wl.linear_inputs(spec)
+    cores = oracle_threads()
+    t0, c0 = time.perf_counter(), time.process_time()
+    done = 0
+    for h in range(spec.H):
+        if time.perf_counter() - t0 >= limit_s:
+            break
+        sl = (slice(0, 1), slice(h, h + 1))
+        K, V, Q = x["K"][sl], x["V"][sl], x["Q"][sl]
+        O, _, L = olin.ttt_linear_scan(K, V, Q, x["W0"][sl], spec.eta, spec.b)
+        gs = ogate.GateState(1, 1)
+        ogate.surprisal_route(L.astype("float32"), gs)
+        A = oca.cache_attention(Q, K, V, gs.entries, gs.counts())
+        oca.alpha_fusion(O, A, torch.full((1, 64), 0.25).numpy())
+        done += 1
+    dt = time.perf_counter() - t0
+    busy = (time.process_time() - c0) / dt if dt > 0 else 0.0
+    return {"value": spec.T * done / spec.H / dt, "unit": "tokens/s", "cores": cores, "busy_threads": round(busy, 2),
+            "kind": "oracle", "sample": f"{done} of {spec.B * spec.H} (sequence, head) pairs: scan, gate and read path",
+            "seconds": dt}
 
 
 def bench_config(spec, world) -> dict:
@@ -535,11 +644,28 @@ def main():
                 extra[s.name] = measure(s, max(5, min(a.steps, 20)), 3, peaks, device, with_e2e=True)
             except Exception as ex:
                 extra[s.name] = {"error": str(ex)}
+        # The two further forms of the path: the context-parallel In-Place scan on the 4B-class
+        # workload, and the residual-cache read path on the gate workload's cache.
+        cp_name = wl.INPLACE_4B.name + " (context-parallel form)"
+        try:
+            extra[cp_name] = measure(wl.INPLACE_4B, max(5, min(a.steps, 20)), 3, peaks, device, with_e2e=True,
+                                     prefix=True)
+        except Exception as ex:
+            extra[cp_name] = {"error": str(ex)}
+        try:
+            extra[CACHE_READ] = measure_cache_read(max(5, min(a.steps, 20)), 3, peaks, device)
+        except Exception as ex:
+            extra[CACHE_READ] = {"error": str(ex)}
     clk.__exit__(None, None, None)
     # The oracle baselines run after the sampler stops (the GPU idles meanwhile).
     for s in wl.WORKLOADS.values():
         if s.name in extra and "error" not in extra[s.name]:
             extra[s.name]["cpu_baseline"] = cpu_baseline(s, 6.0)
+    if "error" not in extra.get(wl.INPLACE_4B.name + " (context-parallel form)", {"error": 1}):
+        extra[wl.INPLACE_4B.name + " (context-parallel form)"]["cpu_baseline"] = cpu_baseline(wl.INPLACE_4B, 6.0,
+                                                                                               prefix=True)
+    if "error" not in extra.get(CACHE_READ, {"error": 1}):
+        extra[CACHE_READ]["cpu_baseline"] = cpu_baseline_cache_read(6.0)
 
     if rank == 0:
         rl = roofline(spec, w, ms, peaks, traffic_per_launch(spec))

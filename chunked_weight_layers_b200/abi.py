@@ -31,6 +31,7 @@ TTT_BF16 = 1
 TTT_OPT_LINEAR_CHUNK = 1
 TTT_OPT_WAIT_LIMIT_NS = 2
 TTT_OPT_INJECT_STALL = 3
+TTT_OPT_INPLACE_PREFIX = 4
 
 
 class ttt_config(ctypes.Structure):

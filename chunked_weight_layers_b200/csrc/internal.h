@@ -53,6 +53,12 @@ struct InplaceBuffers {
   // read by chunk c's update; three buffers so the producer never waits for a reader.
   __nv_bfloat16* Vhat[3] = {nullptr, nullptr, nullptr};
   TCResources* tc = nullptr;     // tensor-core schedules and conv(X0) buffer, built on first use
+  // Context-parallel form (TTT_OPT_INPLACE_PREFIX): the chunks' fp32 deltas [n][d][f] and the bf16
+  // weights each chunk applies with [n][d][f], grown on demand.
+  int prefix_form = 0;
+  float* prefix_D = nullptr;
+  __nv_bfloat16* prefix_Wb = nullptr;
+  int prefix_chunks = 0;
 };
 
 // Tensor maps of one scan's K, V, Q, O (encoding them costs microseconds of host time, so the
@@ -123,6 +129,11 @@ ttt_status inplace_f32_chunk(ttt_state* st, const float* Z, const float* Vhat, f
 // In-Place, bf16 tensor cores: the whole scan over T tokens.
 ttt_status inplace_bf16_scan(ttt_state* st, const __nv_bfloat16* Z, const __nv_bfloat16* targets,
                              int64_t T, __nv_bfloat16* O, cudaStream_t s);
+
+// In-Place, bf16 tensor cores, context-parallel form: all chunk deltas, their exclusive prefix
+// sums, then all chunk outputs (three launches, no cross-chunk waits).
+ttt_status inplace_bf16_scan_prefix(ttt_state* st, const __nv_bfloat16* Z, const __nv_bfloat16* Vhat, int64_t T,
+                                    __nv_bfloat16* O, cudaStream_t s);
 
 // Frees the tensor-core resources of a state (no-op if none were built).
 void free_tc(ttt_state* st);

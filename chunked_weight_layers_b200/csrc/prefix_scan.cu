@@ -1,0 +1,273 @@
+// Context-parallel form of the In-Place scan ("In-Place Test-Time Training", §6: the chunk
+// updates are additive, so every chunk's ΔW_j is computed in parallel, an exclusive prefix sum
+// gives each chunk the cumulative update before it, and then every chunk's outputs are
+// computed in parallel with its effective weight W_c = W_0 + η·Σ_{j<c} ΔW_j).
+//
+// Three launches per scan call of n chunks, none of which waits on another chunk:
+//   1. k_gemm_tc, batched over the chunks: D_j = η·V̂_jᵀ·Z_j (fp32 [n][d][f]);
+//   2. k_prefix_w: W_j = W_0 + Σ_{i<j} D_i, stored as bf16 [n][d][f] (the weight chunk j
+//      applies with); the fp32 sum after the last chunk becomes the state's weight;
+//   3. k_gemm_tc, batched over the chunks: O_j = Z_j·W_jᵀ (bf16).
+// It computes the same outputs and final weight as the sequential scan (the sums are taken in
+// the same order; each η·ΔW_j is rounded to fp32 before it is added) and is the form that
+// shards the sequence over devices; on one device it moves more data (the n fp32 deltas and
+// the n bf16 weights go through HBM) in exchange for launches without cross-chunk waits.
+//
+// k_gemm_tc is a plain batched GEMM on the 5th-generation tensor cores: one CTA per 128x256
+// output tile, TMA loads (128-byte swizzle) into a 3-stage ring, one thread issuing
+// tcgen05.mma (M=128, N=256, K=16) into a TMEM accumulator, four epilogue warps (one per TMEM
+// lane quarter) scaling and storing rows. Operands are K-major or MN-major as stored.
+#include "internal.h"
+#include "tc_common.cuh"
+
+namespace ttt {
+
+namespace {
+
+constexpr int GM = 128, GN = 256, GK = 64, kGSt = 3;
+constexpr int kGA = GM * GK * 2;  // 16 KB of A per stage
+constexpr int kGB = GN * GK * 2;  // 32 KB of B per stage
+constexpr int kGThreads = 6 * 32;  // TMA producer, MMA issuer, 4 epilogue warps
+constexpr int kGTmemCols = 256;
+
+struct __align__(1024) GemmSmem {
+  uint8_t A[kGSt][kGA];
+  uint8_t B[kGSt][kGB];
+  uint64_t full[kGSt], empty[kGSt], tfull;
+  uint32_t tmem;
+  int abort;
+};
+
+struct GemmArgs {
+  int M, N, K;         // per batch item
+  int a_mn, b_mn;      // operand stored MN-major (its M or N index contiguous) rather than K-major
+  int a_outer, b_outer;  // outer tensor-map coordinate of batch item 1 (item b starts at b times it)
+  void* out;           // [batch][M][ldo], fp32 (out_f32) or bf16
+  int out_f32;
+  long long out_batch;  // elements between batch items of out
+  int ldo;
+  float scale;         // out = scale · A·B
+  DevStatus status;
+};
+
+__global__ void __launch_bounds__(kGThreads, 1)
+    k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const GemmArgs g) {
+  extern __shared__ uint8_t smem_raw[];
+  GemmSmem& sm = *reinterpret_cast<GemmSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tiles_n = (g.N + GN - 1) / GN;
+  const int tm = blockIdx.x / tiles_n, tn = blockIdx.x % tiles_n, b = blockIdx.y;
+  const int nk = (g.K + GK - 1) / GK;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kGSt; ++i) {
+      mbar_init(&sm.full[i], 1);
+      mbar_init(&sm.empty[i], 1);
+    }
+    mbar_init(&sm.tfull, 1);
+    sm.abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) tc::alloc(&sm.tmem, kGTmemCols);
+  tc::fence_before();
+  __syncthreads();
+  tc::fence_after();
+  const uint32_t tmem = sm.tmem;
+  volatile int* abort = &sm.abort;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tmA);
+      tma_prefetch_desc(&tmB);
+      int kb = 0;
+      for (; kb < nk; ++kb) {
+        const int s = kb % kGSt;
+        if (kb >= kGSt && !mbar_wait(&sm.empty[s], ((kb / kGSt) - 1) & 1, g.status, abort)) break;
+        mbar_arrive_expect_tx(&sm.full[s], kGA + kGB);
+        if (!g.a_mn) {
+          tma_load_2d(sm.A[s], &tmA, &sm.full[s], kb * GK, b * g.a_outer + tm * GM);
+        } else {
+          for (int j = 0; j < GM / 64; ++j)
+            tma_load_2d(sm.A[s] + j * 8192, &tmA, &sm.full[s], tm * GM + j * 64, b * g.a_outer + kb * GK);
+        }
+        if (!g.b_mn) {
+          tma_load_2d(sm.B[s], &tmB, &sm.full[s], kb * GK, b * g.b_outer + tn * GN);
+        } else {
+          for (int j = 0; j < GN / 64; ++j)
+            tma_load_2d(sm.B[s] + j * 8192, &tmB, &sm.full[s], tn * GN + j * 64, b * g.b_outer + kb * GK);
+        }
+      }
+      // Nothing may still be landing in shared memory when the CTA exits.
+      for (int k = kb > kGSt ? kb - kGSt : 0; k < kb; ++k) mbar_wait(&sm.full[k % kGSt], (k / kGSt) & 1, g.status, nullptr);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = tc::idesc_bf16(GM, GN, g.a_mn, g.b_mn);
+      int kb = 0;
+      bool ok = true;
+      for (; kb < nk; ++kb) {
+        const int s = kb % kGSt;
+        if (!mbar_wait(&sm.full[s], (kb / kGSt) & 1, g.status, abort)) {
+          ok = false;
+          break;
+        }
+        tc::fence_after();
+        const uint32_t a0 = smem_u32(sm.A[s]), b0 = smem_u32(sm.B[s]);
+#pragma unroll
+        for (int kk = 0; kk < GK / 16; ++kk) {
+          const uint64_t ad = g.a_mn ? tc::smem_desc(a0 + kk * 2048, 8192, 1024) : tc::smem_desc(a0 + kk * 32, 16, 1024);
+          const uint64_t bd = g.b_mn ? tc::smem_desc(b0 + kk * 2048, 8192, 1024) : tc::smem_desc(b0 + kk * 32, 16, 1024);
+          tc::mma(tmem, ad, bd, idesc, (kb | kk) != 0);
+        }
+        tc::commit(&sm.empty[s]);  // frees the stage once these MMAs have read it
+      }
+      if (ok) {
+        tc::commit(&sm.tfull);
+        // The epilogue's wait covers the MMAs; this thread waits too, so TMEM is not freed early.
+        mbar_wait(&sm.tfull, 0, g.status, nullptr);
+      } else if (kb > 0) {
+        mbar_wait(&sm.empty[(kb - 1) % kGSt], ((kb - 1) / kGSt) & 1, g.status, nullptr);
+      }
+    }
+  } else {
+    // Epilogue: warp w reads TMEM lane quarter w % 4, i.e. tile rows 32(w % 4) .. +31.
+    const int q = warp & 3;
+    bool ok = mbar_wait(&sm.tfull, 0, g.status, abort);
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok) {
+      tc::fence_after();
+      const int row = tm * GM + q * 32 + lane;
+      const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16);
+#pragma unroll 1
+      for (int jc = 0; jc < GN / 32; ++jc) {
+        uint32_t r[32];
+        tc::ld32(tbase + jc * 32, r);
+        tc::wait_ld();
+        const int col0 = tn * GN + jc * 32;
+        if (row >= g.M || col0 >= g.N) continue;
+        float v[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = g.scale * __uint_as_float(r[j]);
+        if (g.out_f32) {
+          float* dst = static_cast<float*>(g.out) + b * g.out_batch + (long long)row * g.ldo + col0;
+          if (col0 + 32 <= g.N) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              reinterpret_cast<float4*>(dst)[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+          } else {
+            for (int j = 0; j < 32 && col0 + j < g.N; ++j) dst[j] = v[j];
+          }
+        } else {
+          __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(g.out) + b * g.out_batch + (long long)row * g.ldo + col0;
+          if (col0 + 32 <= g.N) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              uint4 w;
+              w.x = pack_bf16(v[8 * j + 0], v[8 * j + 1]);
+              w.y = pack_bf16(v[8 * j + 2], v[8 * j + 3]);
+              w.z = pack_bf16(v[8 * j + 4], v[8 * j + 5]);
+              w.w = pack_bf16(v[8 * j + 6], v[8 * j + 7]);
+              reinterpret_cast<uint4*>(dst)[j] = w;
+            }
+          } else {
+            for (int j = 0; j < 32 && col0 + j < g.N; ++j) dst[j] = __float2bfloat16_rn(v[j]);
+          }
+        }
+      }
+    }
+  }
+
+  tc::fence_before();
+  __syncthreads();
+  tc::fence_after();
+  if (warp == 1) tc::dealloc(tmem, kGTmemCols);
+}
+
+// W_j (bf16) = W_0 + Σ_{i<j} D_i for j = 0 .. n−1, then W ← W_0 + Σ_i D_i (fp32) and its bf16
+// copy. Four consecutive elements a thread; the sum over the chunks runs in chunk order.
+__global__ void k_prefix_w(const float* W0, const float* __restrict__ D, __nv_bfloat16* __restrict__ Wb, float* Wout,
+                           __nv_bfloat16* __restrict__ Wcopy, long long nelem, int n) {
+  const long long n4 = nelem / 4;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (long long)gridDim.x * blockDim.x) {
+    float4 acc = reinterpret_cast<const float4*>(W0)[i];
+    for (int j = 0; j < n; ++j) {
+      uint2 w;
+      w.x = pack_bf16(acc.x, acc.y);
+      w.y = pack_bf16(acc.z, acc.w);
+      reinterpret_cast<uint2*>(Wb + (long long)j * nelem)[i] = w;
+      const float4 dj = reinterpret_cast<const float4*>(D + (long long)j * nelem)[i];
+      acc.x += dj.x;
+      acc.y += dj.y;
+      acc.z += dj.z;
+      acc.w += dj.w;
+    }
+    reinterpret_cast<float4*>(Wout)[i] = acc;
+    uint2 w;
+    w.x = pack_bf16(acc.x, acc.y);
+    w.y = pack_bf16(acc.z, acc.w);
+    reinterpret_cast<uint2*>(Wcopy)[i] = w;
+  }
+}
+
+ttt_status map_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint32_t box_in, uint32_t box_out) {
+  const uint64_t dims[2] = {inner, outer};
+  const uint64_t strides[1] = {inner * 2};
+  const uint32_t box[2] = {box_in, box_out};
+  return encode_tmap(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+ttt_status gemm(ttt_state* st, const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& g, int batch,
+                cudaStream_t s) {
+  const size_t smem = sizeof(GemmSmem) + 1024;
+  TTT_CUDA(cudaFuncSetAttribute(k_gemm_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  const dim3 grid((unsigned)(((g.M + GM - 1) / GM) * ((g.N + GN - 1) / GN)), (unsigned)batch);
+  k_gemm_tc<<<grid, kGThreads, smem, s>>>(ta, tb, g);
+  st->launches++;
+  TTT_CUDA(cudaGetLastError());
+  return TTT_OK;
+}
+
+}  // namespace
+
+ttt_status inplace_bf16_scan_prefix(ttt_state* st, const __nv_bfloat16* Z, const __nv_bfloat16* Vhat, int64_t T,
+                                    __nv_bfloat16* O, cudaStream_t s) {
+  const ttt_config& c = st->cfg;
+  const int d = c.d_val, f = c.d_key, C = c.chunk;
+  const int n = (int)(T / C);
+  const size_t nelem = (size_t)d * f;
+  InplaceBuffers& ip = st->ip;
+  if (ip.prefix_chunks < n) {
+    if (ip.prefix_D) cudaFree(ip.prefix_D);
+    if (ip.prefix_Wb) cudaFree(ip.prefix_Wb);
+    ip.prefix_D = nullptr;
+    ip.prefix_Wb = nullptr;
+    ip.prefix_chunks = 0;
+    TTT_CUDA(cudaMalloc(reinterpret_cast<void**>(&ip.prefix_D), (size_t)n * nelem * 4));
+    TTT_CUDA(cudaMalloc(reinterpret_cast<void**>(&ip.prefix_Wb), (size_t)n * nelem * 2));
+    ip.prefix_chunks = n;
+  }
+  const DevStatus ds{st->status.dev, st->wait_limit_ns};
+
+  // 1. D_j = η·V̂_jᵀ·Z_j: M = d, N = f, K = C; A = V̂ (MN-major), B = Z (MN-major), batch j at token jC.
+  CUtensorMap tV, tZm;
+  TTT_TRY(map_bf16(&tV, Vhat, d, T, 64, 64));
+  TTT_TRY(map_bf16(&tZm, Z, f, T, 64, 64));
+  GemmArgs ga{d, f, C, 1, 1, C, C, ip.prefix_D, 1, (long long)nelem, f, c.eta, ds};
+  TTT_TRY(gemm(st, tV, tZm, ga, n, s));
+
+  // 2. Exclusive prefix sums: the weight each chunk applies with, and the final weight.
+  const long long n4 = (long long)(nelem / 4);
+  const int blocks = (int)std::min<long long>((n4 + 255) / 256, (long long)st->num_sms * 8);
+  k_prefix_w<<<blocks, 256, 0, s>>>(ip.W, ip.prefix_D, ip.prefix_Wb, ip.W, ip.Wsh[ip.cur], (long long)nelem, n);
+  st->launches++;
+  TTT_CUDA(cudaGetLastError());
+
+  // 3. O_j = Z_j·W_jᵀ: M = C, N = d, K = f; A = Z (K-major), B = W_j (K-major, rows jd ..).
+  CUtensorMap tZk, tW;
+  TTT_TRY(map_bf16(&tZk, Z, f, T, 64, 128));
+  TTT_TRY(map_bf16(&tW, ip.prefix_Wb, f, (uint64_t)n * d, 64, 256));
+  GemmArgs gc{C, d, f, 0, 0, C, d, O, 0, (long long)C * d, d, 1.0f, ds};
+  return gemm(st, tZk, tW, gc, n, s);
+}
+
+}  // namespace ttt

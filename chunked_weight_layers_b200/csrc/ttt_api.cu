@@ -105,6 +105,8 @@ static void free_state(ttt_state* st) {
   dev_free(st->ip.W);
   dev_free(st->ip.W0);
   dev_free(st->ip.Wf32_next);
+  dev_free(st->ip.prefix_D);
+  dev_free(st->ip.prefix_Wb);
   dev_free(st->ip.Wsh[0]);
   dev_free(st->ip.Wsh[1]);
   dev_free(st->ip.Wsh[2]);
@@ -276,6 +278,9 @@ static ttt_status scan_impl(ttt_state* st, const void* keys, const void* targets
         TTT_TRY(inplace_f32_chunk(st, Z + t0 * c.d_key, V + t0 * c.d_val, O + t0 * c.d_val, c.chunk, s));
       return TTT_OK;
     }
+    if (st->ip.prefix_form)
+      return inplace_bf16_scan_prefix(st, static_cast<const __nv_bfloat16*>(keys),
+                                      static_cast<const __nv_bfloat16*>(targets), T, static_cast<__nv_bfloat16*>(out), s);
     return inplace_bf16_scan(st, static_cast<const __nv_bfloat16*>(keys),
                              static_cast<const __nv_bfloat16*>(targets), T,
                              static_cast<__nv_bfloat16*>(out), s);
@@ -487,6 +492,13 @@ ttt_status ttt_state_set_option(ttt_state* st, int32_t option, int64_t value) {
       if (value < 1000 || value > 60000000000ll)
         return fail(TTT_ERR_INVALID_ARG, "TTT_OPT_WAIT_LIMIT_NS must lie in [1000, 6e10] (got %lld)", (long long)value);
       st->wait_limit_ns = (uint64_t)value;
+      return TTT_OK;
+    case TTT_OPT_INPLACE_PREFIX:
+      if (value != 0 && value != 1) return fail(TTT_ERR_INVALID_ARG, "TTT_OPT_INPLACE_PREFIX must be 0 or 1");
+      if (value == 1 && (st->cfg.rule != TTT_RULE_INPLACE_HEBBIAN || st->cfg.io_dtype != TTT_BF16 ||
+                         st->cfg.target_mode != 0))
+        return fail(TTT_ERR_UNSUPPORTED, "the context-parallel form runs In-Place BF16 states with given targets");
+      st->ip.prefix_form = (int)value;
       return TTT_OK;
     case TTT_OPT_INJECT_STALL:
       if (value != 0 && value != 1) return fail(TTT_ERR_INVALID_ARG, "TTT_OPT_INJECT_STALL must be 0 or 1");

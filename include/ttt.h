@@ -260,7 +260,16 @@ typedef enum {
    * the second chunk waits for one more finished UPDATE tile than exists; the TTT-Linear scan
    * never loads its second 64-token tile — so that the wait runs out. The outputs of that scan
    * are incomplete. 0 cancels a pending injection. */
-  TTT_OPT_INJECT_STALL = 3
+  TTT_OPT_INJECT_STALL = 3,
+  /* In-Place BF16 states with given targets (target_mode 0), value 1: run each scan call in the
+   * context-parallel form ("In-Place Test-Time Training", §6: the chunk updates are additive, so
+   * every chunk's ΔW_j is computed in parallel, an exclusive prefix sum gives each chunk its
+   * cumulative update, and every chunk's outputs are computed in parallel with
+   * W_c = W_start + η·Σ_{j<c} ΔW_j). Same outputs and final weight as the sequential form, up
+   * to rounding (each η·ΔW_j is rounded to fp32 before it is added). The call keeps n fp32
+   * deltas and n bf16 weights of d_val x d_key in state-owned scratch (grown on demand, n =
+   * T / chunk). 0 returns to the sequential form. UNSUPPORTED for other states. */
+  TTT_OPT_INPLACE_PREFIX = 4
 } ttt_option;
 
 /* Set option `option` of state `st` to `value`. Takes effect from the next call that
