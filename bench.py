@@ -503,6 +503,88 @@ def cpu_baseline_cache_read(limit_s) -> dict:
             "seconds": dt}
 
 
+def run_row_sharded(spec, a, world, rank, local, peaks):
+    """One In-Place layer split over the ranks by Wdown rows (RowShardedInplace): every rank holds
+    the whole Z and V̂ (same seed) and its rows of W; a step is one scan of the T tokens on every
+    rank plus the all-gather of the output columns. Strong scaling: value = T / the slowest
+    rank's time per step."""
+    import datetime
+
+    import torch.distributed as dist
+    from chunked_weight_layers_b200 import build
+    from chunked_weight_layers_b200.dist import RowShardedInplace, max_over_ranks
+    if not isinstance(spec, wl.InplaceSpec) or spec.target or spec.dtype != "bf16":
+        raise SystemExit("--shard rows takes an In-Place bf16 workload with given targets")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+    if rank == 0:
+        build.build()
+    if world > 1:
+        dist.barrier()
+    import chunked_weight_layers_b200 as cwl
+    x = wl.inplace_inputs(spec, device=device)
+    cfg = cwl.config("inplace", io_dtype=1, d_key=spec.f, d_val=spec.d, chunk=spec.C, eta=spec.eta)
+    layer = RowShardedInplace(cfg, x["W0"])
+    for _ in range(a.warmup):
+        layer.scan(x["Z"], x["Vhat"])
+    torch.cuda.synchronize()
+    layer.state.poll()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    clk = ClockSampler(local)
+    clk.__enter__()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n0 = layer.state.launch_count()
+    e0.record(stream)
+    for _ in range(a.steps):
+        layer.scan(x["Z"], x["Vhat"])
+    e1.record(stream)
+    e1.synchronize()
+    launches = layer.state.launch_count() - n0
+    if world > 1:
+        dist.barrier()
+    clk.__exit__(None, None, None)
+    layer.state.poll()
+    ms = max_over_ranks(e0.elapsed_time(e1), device) / a.steps
+    w = work(spec)
+    # End to end: inputs copied from pinned host memory, the sharded scan, the gathered output read back.
+    hZ, hV = x["Z"].cpu().pin_memory(), x["Vhat"].cpu().pin_memory()
+    hO = torch.empty((spec.T, spec.d), dtype=torch.bfloat16).pin_memory()
+    t = []
+    for k in range(3):
+        torch.cuda.synchronize()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record()
+        layer.reset()
+        O = layer.scan(hZ.to(device, non_blocking=True), hV.to(device, non_blocking=True))
+        hO.copy_(O, non_blocking=True)
+        f1.record()
+        f1.synchronize()
+        t.append(f0.elapsed_time(f1))
+    e2e_ms = max_over_ranks(statistics.mean(t), device)
+    if rank == 0:
+        rl = roofline(spec, w, ms, peaks, None)
+        rl["kernel"] = dominant_kernel(spec)
+        print(json.dumps({
+            "metric": METRIC, "value": w["tokens"] / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world,
+            "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "strong",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": dict(bench_config(spec, world), parallelism=f"rows{world}",
+                           l2="inputs larger than L2 (one step moves over 1 GB)"),
+            "tflops": w["flops"] / (ms * 1e-3) / 1e12, "roofline": rl,
+            "e2e": {"value": w["tokens"] / (e2e_ms * 1e-3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": (hZ.numel() + hV.numel()) * 2, "d2h_bytes_per_step": hO.numel() * 2,
+                    "ms_per_step": e2e_ms},
+            "gpu_launches": launches, "clocks": clk.summary(peaks["sm_max_mhz"])}))
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def bench_config(spec, world) -> dict:
     """The workload description both arms report."""
     return {"workload": spec.name, "B": getattr(spec, "B", 1), "H": getattr(spec, "H", 1), "T": spec.T,
@@ -529,6 +611,10 @@ def main():
     ap.add_argument("--tokens", type=int, default=None,
                     help="run the named workload with this many tokens instead (same widths and chunk; a smaller "
                          "case for profilers, not a bench line)")
+    ap.add_argument("--shard", choices=["replicas", "rows"], default="replicas",
+                    help="with N ranks: 'replicas' (default) runs an independent copy of the workload per rank "
+                         "(weak scaling); 'rows' splits one In-Place layer's Wdown rows over the ranks and "
+                         "all-gathers the output columns each step (strong scaling; In-Place workloads)")
     ap.add_argument("--profile", type=int, default=None, metavar="N",
                     help="for profilers: build the named workload, run one warm-up step and N more steps, print "
                          "nothing else (no timing, no end-to-end pass, no oracle)")
@@ -540,7 +626,7 @@ def main():
     spec = spec_by_name(a.workload)
     if a.tokens is not None:
         spec = wl.scaled(spec, T=a.tokens, name=f"{spec.name}@T{a.tokens}")
-    if world > 1:
+    if world > 1 and a.shard == "replicas":
         # Weak scaling: every rank scans its own batch of independent problems (its own seed).
         spec = wl.scaled(spec, seed=spec.seed + 7919 * rank)
     w = work(spec)
@@ -584,6 +670,9 @@ def main():
 
     if a.warmup < 3:
         a.warmup = 3
+    if a.shard == "rows":
+        run_row_sharded(spec, a, world, rank, local, peaks)
+        return
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
     pg = None

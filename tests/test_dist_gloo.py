@@ -65,37 +65,68 @@ def test_two_gloo_ranks():
         assert out[0] == (True, 2.5) and out[1] == (True, 2.5)
 
 
+class _OracleState:
+    """Stand-in for the library's state in this CPU test: the oracle's scan of a row block,
+    behind the calls RowShardedInplace makes (chunk_scan, get_weights, reset)."""
+
+    device = torch.device("cpu")
+
+    def __init__(self, cfg, W0_rows):
+        self.cfg = cfg
+        self.W0 = W0_rows.clone()
+        self.W = W0_rows.clone()
+
+    def chunk_scan(self, Z, Vhat, out, T):
+        from oracle import inplace
+        O, W = inplace.inplace_scan_rows(Z[:T].numpy(), Vhat[:T].numpy(), self.W.numpy(), self.cfg.eta, self.cfg.chunk)
+        out.copy_(torch.from_numpy(O))
+        self.W = torch.from_numpy(W)
+
+    def get_weights(self, W):
+        W.copy_(self.W)
+
+    def reset(self):
+        self.W = self.W0.clone()
+
+
 def _inplace_worker(rank, world, port, out):
-    """Rank ``rank`` scans its contiguous share of Wdown's rows (W0[rows], V̂[:, rows]) on its
-    own, then the ranks all-gather their output columns; nothing else crosses ranks."""
+    """Each rank runs RowShardedInplace (the product's host logic: row shares, V̂ column slices,
+    padded all-gathers) over the oracle's row scan; the gathered O and W must equal the
+    single-process scan, over two calls in a row."""
     import numpy as np
+    import chunked_weight_layers_b200 as cwl
+    from chunked_weight_layers_b200.dist import RowShardedInplace
     from oracle import inplace
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
         rng = np.random.default_rng(7)
-        T, C, d, f, eta = 96, 32, 10, 12, 0.05
+        T, C, d, f, eta = 96, 32, 11, 12, 0.05
         Z, V, W0 = rng.standard_normal((T, f)), rng.standard_normal((T, d)), 0.1 * rng.standard_normal((d, f))
-        a, b = shard_range(d, rank, world)
-        O_mine, W_mine = inplace.inplace_scan_rows(Z, V[:, a:b], W0[a:b], eta, C)
-        cols = [torch.zeros(T, n, dtype=torch.float64) for n in
-                (shard_range(d, r, world)[1] - shard_range(d, r, world)[0] for r in range(world))]
-        dist.all_gather(cols, torch.from_numpy(np.ascontiguousarray(O_mine)))
-        rows = [torch.zeros(n, f, dtype=torch.float64) for n in
-                (shard_range(d, r, world)[1] - shard_range(d, r, world)[0] for r in range(world))]
-        dist.all_gather(rows, torch.from_numpy(np.ascontiguousarray(W_mine)))
-        O = torch.cat(cols, 1).numpy()
-        W = torch.cat(rows, 0).numpy()
-        O_ref, W_ref = inplace.inplace_scan(Z, V, W0, eta, C)
-        out[rank] = bool(np.allclose(O, O_ref, rtol=0, atol=1e-12) and np.allclose(W, W_ref, rtol=0, atol=1e-12))
+        cfg = cwl.abi.ttt_config()
+        cfg.rule, cfg.io_dtype, cfg.d_key, cfg.d_val, cfg.chunk, cfg.eta = 0, 0, f, d, C, eta
+        layer = RowShardedInplace(cfg, torch.from_numpy(W0), make_state=_OracleState)
+        Zt, Vt = torch.from_numpy(Z), torch.from_numpy(V)
+        O1 = layer.scan(Zt[:64], Vt[:64])
+        O2 = layer.scan(Zt[64:], Vt[64:])
+        W = layer.get_weights().numpy()
+        O = torch.cat([O1, O2]).numpy()
+        O_ref, W_ref = inplace.inplace_scan(Z, V, W0, cfg.eta, C)  # η as the config holds it (fp32)
+        # The weight is read back as fp32, like the library's state.
+        ok = np.allclose(O, O_ref, rtol=0, atol=1e-12) and np.array_equal(W, W_ref.astype(np.float32))
+        ok = ok and layer.rows == shard_range(d, rank, world) and layer.state.W.shape[0] == layer.rows[1] - layer.rows[0]
+        layer.reset()
+        ok = ok and np.array_equal(layer.get_weights().numpy(), W0.astype(np.float32))
+        out[rank] = bool(ok)
     finally:
         dist.destroy_process_group()
 
 
 def test_inplace_rows_shard_across_two_gloo_ranks():
-    """The In-Place scan shards over Wdown's rows: two ranks with half the rows each reproduce
-    the single-process scan (to float64 rounding) after one all-gather of output columns."""
+    """The In-Place scan shards over Wdown's rows: two ranks (11 rows: 6 and 5) each holding their
+    rows reproduce the single-process scan (to float64 rounding) after one all-gather of output
+    columns a call."""
     world = 2
     ctx = mp.get_context("spawn")
     with ctx.Manager() as m:
