@@ -287,15 +287,27 @@ def traffic_per_launch(spec):
     return rec["bytes_per_launch"] * rec.get("launches_per_step", 1)
 
 
-def roofline(spec, w, ms, peaks, traffic=None):
+SUSTAINED_MS = 50.0  # a timed region at least this long runs in the power-capped regime
+
+
+def roofline(spec, w, ms, peaks, traffic=None, timed_ms=0.0):
+    """Roofline object of the dominant kernel. A tensor-bound kernel is compared with the burst
+    bf16 peak when its timed region is short and with the sustained one (the same GEMM held for
+    seconds under the power cap) when the K back-to-back steps run for SUSTAINED_MS or longer;
+    both fractions are reported."""
     if w["bound"] == "hbm":
         achieved = w["bytes"] / (ms * 1e-3) / 1e9
         return {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"], "traffic": traffic, "peak_source": peaks["source"]}
     if w["bound"] == "tensor":
         achieved = w["flops"] / (ms * 1e-3) / 1e12
-        return {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": achieved / peaks["bf16_tflops"], "traffic": traffic, "peak_source": peaks["source"],
+        sustained = timed_ms >= SUSTAINED_MS
+        peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
+        return {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": traffic, "peak_source": peaks["source"],
+                "peak_kind": (f"sustained (the {timed_ms:.0f} ms timed region runs back to back under the power cap)"
+                              if sustained else f"burst (a {timed_ms:.1f} ms timed region)"),
+                "frac_of_burst": achieved / peaks["bf16_tflops"],
                 "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"]}
     achieved = w["flops"] / (ms * 1e-3) / 1e12
     peak = fp32_alu_peak_tflops(peaks)
@@ -376,7 +388,7 @@ def measure(spec, steps, warmup, peaks, device, with_e2e, cpu_limit_s=None, pref
     total, launches, times = time_steps(r, steps, warmup)
     ms = total / steps
     w = work(spec)
-    rl = roofline(spec, w, ms, peaks, traffic_per_launch(spec))
+    rl = roofline(spec, w, ms, peaks, traffic_per_launch(spec), timed_ms=total)
     rl["kernel"] = "k_gemm_tc" if prefix else dominant_kernel(spec)
     if prefix:
         rl["traffic"] = None  # no ncu capture of this form is recorded
@@ -567,7 +579,7 @@ def run_row_sharded(spec, a, world, rank, local, peaks):
         t.append(f0.elapsed_time(f1))
     e2e_ms = max_over_ranks(statistics.mean(t), device)
     if rank == 0:
-        rl = roofline(spec, w, ms, peaks, None)
+        rl = roofline(spec, w, ms, peaks, None, timed_ms=ms * a.steps)
         rl["kernel"] = dominant_kernel(spec)
         print(json.dumps({
             "metric": METRIC, "value": w["tokens"] / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world,
@@ -757,7 +769,7 @@ def main():
         extra[CACHE_READ]["cpu_baseline"] = cpu_baseline_cache_read(6.0)
 
     if rank == 0:
-        rl = roofline(spec, w, ms, peaks, traffic_per_launch(spec))
+        rl = roofline(spec, w, ms, peaks, traffic_per_launch(spec), timed_ms=total_ms)
         rl["kernel"] = dominant_kernel(spec)
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": a.steps,
