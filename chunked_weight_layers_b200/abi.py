@@ -32,6 +32,7 @@ TTT_OPT_LINEAR_CHUNK = 1
 TTT_OPT_WAIT_LIMIT_NS = 2
 TTT_OPT_INJECT_STALL = 3
 TTT_OPT_INPLACE_PREFIX = 4
+TTT_OPT_SM_PAIR = 5
 
 
 class ttt_config(ctypes.Structure):

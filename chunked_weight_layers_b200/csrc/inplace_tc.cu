@@ -35,6 +35,15 @@
 //    the mainloop runs. The epilogue adds η·ΔW in shared memory, writes the bf16 copy beside
 //    it, and two TMA stores per sub-tile write both back: the read-modify-write of the 99.6 MB
 //    state never goes through per-thread global loads.
+//  * SM pairs: where the chunk and d_model are multiples of 256 the kernel runs as clusters
+//    of two CTAs on neighbouring SMs, each tile 256 rows x 256 columns. Each CTA loads by TMA
+//    its own 128 rows of A and its own 128 columns of B (32 KB a k-block instead of 48 KB
+//    for the same MMA work per SM, in a 4-stage ring), a lane of the second CTA tells the
+//    first when its stage has landed, and one lane of the first issues tcgen05.mma with
+//    cta_group::2 (M = 256, N = 256), whose commits arrive on the barriers of both CTAs.
+//    Each CTA's TMEM holds its own 128 rows of the accumulator, so the epilogue is the same
+//    per CTA; the second CTA's epilogue warps release the accumulator on the first's barrier.
+//    No load is multicast: every CTA reads its own operands.
 //  * every wait is bounded (%globaltimer); a wait that runs out records TTT_ERR_TIMEOUT in the
 //    state's status word, the CTA drains its in-flight copies and MMAs (bounded), frees TMEM
 //    and returns.
@@ -52,6 +61,11 @@ constexpr int BM = 128, BN = 256, BK = 64;
 constexpr int kSt = 3;                      // operand ring depth (k-blocks)
 constexpr int kABytes = BM * BK * 2;        // 16 KB
 constexpr int kBBytes = BN * BK * 2;        // 32 KB
+constexpr int kRingBytes = kSt * (kABytes + kBBytes);
+constexpr int kTileP = 2 * BM;              // rows of an SM-pair tile
+constexpr int kStP = 4;                     // operand ring depth of an SM pair (32 KB stages)
+constexpr int kStMax = 4;
+static_assert(kStP * (kABytes + kBBytes / 2) <= kRingBytes, "SM-pair stages exceed the operand ring");
 constexpr int kWCols = 32;                  // columns of one W sub-tile of an UPDATE tile
 constexpr int kWBytes = BM * kWCols * 4;    // 16 KB of fp32 W
 constexpr int kShBytes = BM * kWCols * 2;   // 8 KB of its bf16 copy
@@ -60,7 +74,6 @@ constexpr int kEpiWarps = 8;
 constexpr int kWarpWload = 2 + kEpiWarps;   // the warp that streams W sub-tiles in
 constexpr int kThreadsTC = (3 + kEpiWarps) * 32;
 constexpr int kTmemCols = 512;
-constexpr int kRotate = 73;                 // list rotation between rounds (coprime to 148; measured best of 1, 61, 73)
 
 enum : int { APPLY = 0, UPDATE = 1, TARGET = 2 };
 
@@ -70,11 +83,12 @@ __device__ __forceinline__ int tile_m(int32_t t) { return (t >> 14) & 0x3FFF; }
 __device__ __forceinline__ int tile_n(int32_t t) { return t & 0x3FFF; }
 
 struct __align__(1024) TCSmem {
-  uint8_t A[kSt][kABytes];
-  uint8_t B[kSt][kBBytes];
+  // Operand stages, each A (16 KB) followed by B (32 KB; 16 KB, this CTA's half, in an SM pair).
+  uint8_t ring[kRingBytes];
   uint8_t Wr[kWSlots][kWBytes];  // fp32 W sub-tiles (128 rows x 32 columns, 128-byte swizzle)
   uint8_t Sh[2][kShBytes];       // bf16 copy of an updated sub-tile, one per column half (64-byte swizzle)
-  uint64_t full[kSt], empty[kSt];
+  uint64_t full[kStMax], empty[kStMax];
+  uint64_t peer_full[kStMax];    // SM pair, first CTA: the second CTA's stage s has landed
   uint64_t tfull[2], tempty[2];
   uint64_t wfull[kWSlots], wempty[kWSlots];
   uint32_t tmem_base;
@@ -96,6 +110,9 @@ struct TCArgs {
   // Fault injection (tests): the APPLY tiles of this round wait for one more UPDATE than will
   // ever be counted, so that wait runs out; -1 = none.
   int stall_round;
+  // Round r runs tile list (list + r·rotate) mod (number of lists); rotate is coprime to that
+  // number, so over the rounds every CTA works through a mix of the lists.
+  int rotate;
   // Several chunks in one launch: every CTA runs its tile list once per chunk (chunk index
   // chunk + r in round r). The bf16 copy of W rotates through three buffers: round r applies
   // with buffer (cur0 + r) % 3 and its UPDATE tiles write buffer (cur0 + r + 1) % 3, the one
@@ -130,23 +147,95 @@ __device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint
   return d;
 }
 
-// kind::f16 instruction descriptor: D fp32, A and B bf16, M = 128, N = 256.
-__host__ __device__ constexpr uint32_t idesc_bf16(int a_mn, int b_mn) {
+// kind::f16 instruction descriptor: D fp32, A and B bf16, M = m, N = 256.
+__host__ __device__ constexpr uint32_t idesc_bf16(int m, int a_mn, int b_mn) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
-         ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+         ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
 }
 
+// PAIR: issued by the first CTA of an SM pair for both (cta_group::2); A and B are read from
+// the same shared-memory offsets in both CTAs and D lands in both CTAs' TMEM.
+template <bool PAIR>
 __device__ __forceinline__ void umma(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
-      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
-      : "memory");
+  if constexpr (PAIR) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
+        "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
+        "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+        : "memory");
+  }
 }
 
+// The mbarrier at this offset arrives once the MMAs issued before have completed; PAIR: the
+// arrival goes to the barrier at the same offset in both CTAs of the pair (CTA mask 0b11).
+template <bool PAIR>
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-               : "memory");
+  if constexpr (PAIR) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            smem_u32(bar)),
+        "h"((uint16_t)3)
+        : "memory");
+  } else {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+  }
+}
+
+// TMEM allocation by one warp; PAIR: by one warp in each CTA of the pair, same columns in both.
+template <bool PAIR>
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t cols) {
+  if constexpr (PAIR) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst)), "r"(cols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+  } else {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst)), "r"(cols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+}
+
+template <bool PAIR>
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t cols) {
+  if constexpr (PAIR)
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(cols));
+  else
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(cols));
+}
+
+// ---- thread-block clusters (SM pairs) ----------------------------------------------------
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// Every thread of both CTAs; what each wrote before is visible to the other after it.
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Address of this CTA's shared-memory object `p` in the first CTA of the cluster.
+__device__ __forceinline__ uint32_t in_first_cta(const void* p) {
+  uint32_t a;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, 0;" : "=r"(a) : "r"(smem_u32(p)));
+  return a;
+}
+
+// Arrive on the mbarrier at shared::cluster address `addr` (in the other CTA of the pair),
+// relaxed: it orders nothing before it. Its two uses signal events that have completed before
+// it is issued (a TMA load observed on this CTA's barrier; tcgen05.ld reads of TMEM finished by
+// tcgen05.wait::ld), not writes made visible by it. A release at cluster scope here waits for
+// every memory operation this thread has in flight; measured on B200 that made each
+// stage-landed message ~1400 cycles, more than the k-block's 512 cycles of MMA.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t addr) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(addr) : "memory");
 }
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -230,6 +319,9 @@ __device__ __forceinline__ void named_sync_half(int half) {
   asm volatile("bar.sync %0, %1;" ::"r"(1 + half), "n"(4 * 32) : "memory");
 }
 
+// PAIR = false: one CTA per tile of 128 x 256 outputs. PAIR = true: clusters of two CTAs, one
+// tile of 256 x 256 outputs per cluster, 128 rows per CTA (see the file comment).
+template <bool PAIR>
 __global__ void __launch_bounds__(kThreadsTC, 1)
     k_inplace_tc(const __grid_constant__ CUtensorMap tmZk, const __grid_constant__ CUtensorMap tmZm,
                  const __grid_constant__ CUtensorMap tmVm, const __grid_constant__ CUtensorMap tmVm1,
@@ -240,16 +332,26 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
                  const __grid_constant__ CUtensorMap tmWf, const __grid_constant__ CUtensorMap tmWs0,
                  const __grid_constant__ CUtensorMap tmWs1, const __grid_constant__ CUtensorMap tmWs2,
                  const TCArgs args) {
+  constexpr int kStages = PAIR ? kStP : kSt;
+  constexpr int kBCols = PAIR ? BN / 2 : BN;         // B columns (N) this CTA loads
+  constexpr int kStage = kABytes + kBCols * BK * 2;  // bytes of one stage of this CTA
   extern __shared__ uint8_t smem_raw[];
   TCSmem& sm = *reinterpret_cast<TCSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // In round r the CTA runs tile list (blockIdx.x + r·kRotate) mod gridDim.x: over the rounds
+  const int rank = PAIR ? (int)cluster_rank() : 0;  // 0: the CTA that issues the MMAs
+  const int nlists = PAIR ? (int)gridDim.x / 2 : (int)gridDim.x;
+  const int list_id = PAIR ? (int)blockIdx.x / 2 : (int)blockIdx.x;
+  // In round r the CTA (pair) runs tile list (list_id + r·rotate) mod nlists: over the rounds
   // every CTA works through a mix of the lists, so their different loads even out instead of
   // adding up round after round.
-  auto list_of = [&](int rnd) { return (int)(((long)blockIdx.x + (long)rnd * kRotate) % gridDim.x); };
+  auto list_of = [&](int rnd) { return (int)(((long)list_id + (long)rnd * args.rotate) % nlists); };
   auto sched_of = [&](int rnd) {
     return (args.sched_last != nullptr && rnd == args.rounds - 1) ? args.sched_last : args.sched;
   };
+  // First row of this CTA's 128 rows of tile row-block m (tokens for APPLY and TARGET tiles,
+  // rows of W for UPDATE tiles), and the 256-row block of W that an UPDATE tile lies in.
+  auto row0_of = [&](int m) { return PAIR ? m * kTileP + rank * BM : m * BM; };
+  auto wblock_of = [&](int m) { return PAIR ? m : m / 2; };
   int ntot = 0;  // tiles of this CTA over all rounds
   for (int rnd = 0; rnd < args.rounds; ++rnd) ntot += sched_of(rnd)[list_of(rnd) + 1] - sched_of(rnd)[list_of(rnd)];
   // Walks the CTA's tiles in order: calls f(round, tile code) until it returns false.
@@ -257,20 +359,22 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     for (int rnd = 0; rnd < args.rounds; ++rnd) {
       const int32_t* sch = sched_of(rnd);
       const int li = list_of(rnd);
-      const int32_t* tl = sch + gridDim.x + 1;
+      const int32_t* tl = sch + nlists + 1;
       for (int ti = sch[li]; ti < sch[li + 1]; ++ti)
         if (!f(rnd, tl[ti])) return;
     }
   };
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kSt; ++i) {
+    for (int i = 0; i < kStages; ++i) {
       mbar_init(&sm.full[i], 1);
       mbar_init(&sm.empty[i], 1);
+      mbar_init(&sm.peer_full[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sm.tfull[i], 1);
-      mbar_init(&sm.tempty[i], kEpiWarps);
+      // PAIR: the epilogue warps of both CTAs release an accumulator on the first CTA's barrier.
+      mbar_init(&sm.tempty[i], PAIR ? 2 * kEpiWarps : kEpiWarps);
     }
     for (int i = 0; i < kWSlots; ++i) {
       mbar_init(&sm.wfull[i], 1);
@@ -281,13 +385,10 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     sm.tflag[0][0] = sm.tflag[0][1] = sm.tflag[1][0] = sm.tflag[1][1] = 0;
     fence_barrier_init();
   }
-  if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&sm.tmem_base)),
-                 "r"(kTmemCols));
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
-  }
+  if (warp == 1) tmem_alloc<PAIR>(&sm.tmem_base, kTmemCols);
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) cluster_sync();  // both CTAs' barriers exist before either arrives remotely
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
   volatile int* abort = &sm.abort;
@@ -305,6 +406,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         const int type = tile_type(tc), m = tile_m(tc), n = tile_n(tc);
         const int nk = kblocks(type, args);
         const int chunk = args.chunk + rnd;
+        const int r0 = row0_of(m), wb = wblock_of(m);
+        const int b0 = n * BN + rank * (BN / 2);  // first B column (N) this CTA loads
         const CUtensorMap* wk = pick3(tmWk0, tmWk1, tmWk2, (args.cur0 + rnd) % 3);
         if (args.upd_done != nullptr) {
           if (type == APPLY && rnd >= 1 &&
@@ -312,13 +415,13 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
                             upd_expect(args, n) + (rnd == args.stall_round ? 1 : 0), args.status, abort))
             return false;
           if (type == UPDATE && rnd >= 2 &&
-              !wait_counter(&args.app_done[(rnd - 2) * args.nbd + m / 2], args.C / BM, args.status, abort))
+              !wait_counter(&args.app_done[(rnd - 2) * args.nbd + wb], args.C / BM, args.status, abort))
             return false;
           if (args.tgt_done != nullptr) {
             // V̂ of this round was produced by the previous round's TARGET tiles; a TARGET tile
             // overwrites the V̂ buffer the previous round's UPDATE tiles of its block read.
             if (type == UPDATE && rnd >= 1 &&
-                !wait_counter(&args.tgt_done[(rnd - 1) * args.nbd + m / 2], kEpiWarps * (args.C / BM), args.status,
+                !wait_counter(&args.tgt_done[(rnd - 1) * args.nbd + wb], kEpiWarps * (args.C / BM), args.status,
                               abort))
               return false;
             if (type == TARGET && rnd >= 2 &&
@@ -328,29 +431,38 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         }
         const CUtensorMap* vm = args.tgt_done != nullptr ? pick3(tmVm, tmVm1, tmVm2, rnd % 3) : &tmVm;
         for (int kb = 0; kb < nk; ++kb, ++it) {
-          const int s = it % kSt;
-          if (it >= kSt && !mbar_wait(&sm.empty[s], ((it / kSt) - 1) & 1, args.status, abort)) return false;
-          mbar_arrive_expect_tx(&sm.full[s], kABytes + kBBytes);
+          const int s = it % kStages;
+          if (it >= (uint32_t)kStages && !mbar_wait(&sm.empty[s], ((it / kStages) - 1) & 1, args.status, abort))
+            return false;
+          uint8_t* sa = sm.ring + s * kStage;
+          uint8_t* sb = sa + kABytes;
+          mbar_arrive_expect_tx(&sm.full[s], kStage);
           if (type == APPLY) {
-            tma_load_2d(sm.A[s], &tmZk, &sm.full[s], kb * BK, chunk * args.C + m * BM);
-            tma_load_2d(sm.B[s], wk, &sm.full[s], kb * BK, n * BN);
+            tma_load_2d(sa, &tmZk, &sm.full[s], kb * BK, chunk * args.C + r0);
+            tma_load_2d(sb, wk, &sm.full[s], kb * BK, b0);
           } else if (type == UPDATE) {
             for (int j = 0; j < BM / 64; ++j)
-              tma_load_2d(sm.A[s] + j * 8192, vm, &sm.full[s], m * BM + j * 64,
+              tma_load_2d(sa + j * 8192, vm, &sm.full[s], r0 + j * 64,
                           args.vrow0 + (args.tgt_done != nullptr ? 0 : rnd * args.C) + kb * BK);
-            for (int j = 0; j < BN / 64; ++j)
-              tma_load_2d(sm.B[s] + j * 8192, &tmZm, &sm.full[s], n * BN + j * 64, chunk * args.C + kb * BK);
+            for (int j = 0; j < kBCols / 64; ++j)
+              tma_load_2d(sb + j * 8192, &tmZm, &sm.full[s], b0 + j * 64, chunk * args.C + kb * BK);
           } else {
-            tma_load_2d(sm.A[s], &tmConv, &sm.full[s], kb * BK, (args.target_chunk + rnd) * args.C + m * BM);
-            for (int j = 0; j < BN / 64; ++j)
-              tma_load_2d(sm.B[s] + j * 8192, &tmWt, &sm.full[s], n * BN + j * 64, kb * BK);
+            tma_load_2d(sa, &tmConv, &sm.full[s], kb * BK, (args.target_chunk + rnd) * args.C + r0);
+            for (int j = 0; j < kBCols / 64; ++j)
+              tma_load_2d(sb + j * 8192, &tmWt, &sm.full[s], b0 + j * 64, kb * BK);
           }
         }
         return true;
       });
       // Drain: the newest phase issued on every stage must have landed before exit.
-      for (uint32_t k = (it > (uint32_t)kSt ? it - kSt : 0); k < it; ++k)
-        mbar_wait(&sm.full[k % kSt], (k / kSt) & 1, args.status, nullptr);
+      const uint32_t first = it > (uint32_t)kStages ? it - kStages : 0;
+      for (uint32_t k = first; k < it; ++k) mbar_wait(&sm.full[k % kStages], (k / kStages) & 1, args.status, nullptr);
+      // PAIR: the first CTA's MMA lane releases every stage by a commit that arrives on both
+      // CTAs' barriers; after a clean run wait for the last of them, so that none arrives
+      // after this CTA has exited.
+      if (PAIR && !*abort)
+        for (uint32_t k = first; k < it; ++k)
+          mbar_wait(&sm.empty[k % kStages], (k / kStages) & 1, args.status, nullptr);
     }
   } else if (warp == kWarpWload) {
     // ---------------- W sub-tile loader (fp32 W of UPDATE tiles, 128 x 32) ----------------
@@ -361,9 +473,10 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         if (*abort) return false;
         if (tile_type(tc) != UPDATE) return true;
         const int m = tile_m(tc), n = tile_n(tc);
+        const int r0 = row0_of(m), wb = wblock_of(m);
         // The round before updated this W tile, possibly on another CTA.
         if (args.upd_done != nullptr && rnd >= 1 &&
-            !wait_counter(&args.upd_done[(rnd - 1) * args.nbd + m / 2], upd_expect(args, m / 2), args.status, abort))
+            !wait_counter(&args.upd_done[(rnd - 1) * args.nbd + wb], upd_expect(args, wb), args.status, abort))
           return false;
         bool ok = true;
         for (int k = 0; k < BN / kWCols; ++k, ++e) {
@@ -373,7 +486,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
             break;
           }
           mbar_arrive_expect_tx(&sm.wfull[s], kWBytes);
-          tma_load_2d(sm.Wr[s], &tmWf, &sm.wfull[s], n * BN + (k & 1) * 128 + (k >> 1) * kWCols, m * BM);
+          tma_load_2d(sm.Wr[s], &tmWf, &sm.wfull[s], n * BN + (k & 1) * 128 + (k >> 1) * kWCols, r0);
         }
         return ok;
       });
@@ -381,29 +494,47 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         mbar_wait(&sm.wfull[k % kWSlots], (k / kWSlots) & 1, args.status, nullptr);
     }
   } else if (warp == 1) {
-    // ------------------------------- MMA issuer -------------------------------
-    if (lane == 0) {
+    if (PAIR && rank != 0) {
+      // ---------------- second CTA of a pair: report landed stages to the first ----------------
+      if (lane == 0) {
+        uint32_t it = 0;
+        for_tiles([&](int, int32_t tc) -> bool {
+          const int nk = kblocks(tile_type(tc), args);
+          for (int kb = 0; kb < nk; ++kb, ++it) {
+            const int s = it % kStages;
+            if (!mbar_wait(&sm.full[s], (it / kStages) & 1, args.status, abort)) return false;
+            mbar_arrive_remote(in_first_cta(&sm.peer_full[s]));
+          }
+          return true;
+        });
+      }
+    } else if (lane == 0) {
+      // ------------------------------- MMA issuer -------------------------------
       uint32_t it = 0, tcount = 0;
       bool ok = true;
       for_tiles([&](int, int32_t tc) -> bool {
         const int type = tile_type(tc);
         const int nk = kblocks(type, args);
         const int acc = tcount & 1;
-        if (tcount >= 2 && !mbar_wait(&sm.tempty[acc], ((tcount >> 1) - 1) & 1, args.status, abort)) {
+        if (tcount >= 2 && !mbar_wait<PAIR>(&sm.tempty[acc], ((tcount >> 1) - 1) & 1, args.status, abort)) {
           ok = false;
           return false;
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem + (uint32_t)(acc * BN);
-        const uint32_t idesc = type == APPLY ? idesc_bf16(0, 0) : (type == UPDATE ? idesc_bf16(1, 1) : idesc_bf16(0, 1));
+        constexpr int kM = PAIR ? kTileP : BM;
+        const uint32_t idesc = type == APPLY    ? idesc_bf16(kM, 0, 0)
+                               : type == UPDATE ? idesc_bf16(kM, 1, 1)
+                                                : idesc_bf16(kM, 0, 1);
         for (int kb = 0; kb < nk; ++kb, ++it) {
-          const int s = it % kSt;
-          if (!mbar_wait(&sm.full[s], (it / kSt) & 1, args.status, abort)) {
+          const int s = it % kStages;
+          if (!mbar_wait(&sm.full[s], (it / kStages) & 1, args.status, abort) ||
+              (PAIR && !mbar_wait<true>(&sm.peer_full[s], (it / kStages) & 1, args.status, abort))) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a0 = smem_u32(sm.A[s]), b0 = smem_u32(sm.B[s]);
+          const uint32_t a0 = smem_u32(sm.ring + s * kStage), b0 = a0 + kABytes;
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
             uint64_t ad, bd;
@@ -414,12 +545,12 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
               ad = umma_desc(a0 + kk * 32, 16, 1024);
               bd = type == APPLY ? umma_desc(b0 + kk * 32, 16, 1024) : umma_desc(b0 + kk * 2048, 8192, 1024);
             }
-            umma(d_tmem, ad, bd, idesc, (kb | kk) != 0);
+            umma<PAIR>(d_tmem, ad, bd, idesc, (kb | kk) != 0);
           }
-          umma_commit(&sm.empty[s]);  // frees the stage once these MMAs have read it
+          umma_commit<PAIR>(&sm.empty[s]);  // frees the stage (of both CTAs) once these MMAs have read it
         }
         if (!ok) return false;
-        umma_commit(&sm.tfull[acc]);  // accumulator ready for the epilogue
+        umma_commit<PAIR>(&sm.tfull[acc]);  // accumulator ready for the epilogue (of both CTAs)
         ++tcount;
         return true;
       });
@@ -430,7 +561,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         const uint32_t last = (uint32_t)(ntot - 1);
         mbar_wait(&sm.tfull[last & 1], (last >> 1) & 1, args.status, nullptr);
       } else if (!ok && it > 0) {
-        mbar_wait(&sm.empty[(it - 1) % kSt], ((it - 1) / kSt) & 1, args.status, nullptr);
+        mbar_wait(&sm.empty[(it - 1) % kStages], ((it - 1) / kStages) & 1, args.status, nullptr);
       }
     }
   } else {
@@ -443,6 +574,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     bool stop = false;
     for_tiles([&](int rnd, int32_t tc) -> bool {
       const int type = tile_type(tc), m = tile_m(tc), n = tile_n(tc);
+      const int r0 = row0_of(m);
       const CUtensorMap* ws = pick3(tmWs0, tmWs1, tmWs2, (args.cur0 + rnd + 1) % 3);
       const int acc = tcount & 1;
       bool ok = mbar_wait(&sm.tfull[acc], (tcount >> 1) & 1, args.status, nullptr);
@@ -511,8 +643,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           }
           if (leader) {
             const int col = n * BN + half * 128 + j * kWCols;
-            tma_store_2d(&tmWf, sm.Wr[slot], col, m * BM);
-            tma_store_2d(ws, sm.Sh[half], col, m * BM);
+            tma_store_2d(&tmWf, sm.Wr[slot], col, r0);
+            tma_store_2d(ws, sm.Sh[half], col, r0);
             bulk_commit();
             bulk_wait_read<0>();          // both stores have read shared memory
             mbar_arrive(&sm.wempty[slot]);
@@ -525,10 +657,10 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           bulk_wait<0>();
           fence_proxy_async_global();
           __threadfence();
-          atomicAdd(&args.upd_done[rnd * args.nbd + m / 2], 1);
+          atomicAdd(&args.upd_done[rnd * args.nbd + wblock_of(m)], 1);
         }
       } else {
-        const int row = m * BM + row_in_tile;  // token within the chunk
+        const int row = r0 + row_in_tile;  // token within the chunk
 #pragma unroll 1
         for (int jc = 0; jc < 4; ++jc) {
           const int col0 = n * BN + half * 128 + jc * 32;
@@ -554,7 +686,12 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.tempty[acc]);
+      if (lane == 0) {
+        if (PAIR && rank != 0)
+          mbar_arrive_remote(in_first_cta(&sm.tempty[acc]));
+        else
+          mbar_arrive(&sm.tempty[acc]);
+      }
       ++tcount;
       return true;
     });
@@ -563,8 +700,11 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
 
   tc_fence_before();
   __syncthreads();
+  // PAIR: neither CTA exits (or frees TMEM) while the other may still arrive on its barriers
+  // or the MMAs may still write its TMEM.
+  if constexpr (PAIR) cluster_sync();
   tc_fence_after();
-  if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
+  if (warp == 1) tmem_dealloc<PAIR>(tmem, kTmemCols);
 }
 
 // Depthwise future-tap convolution of X0 for the fused target:
@@ -592,17 +732,18 @@ __global__ void k_target_conv(const __nv_bfloat16* __restrict__ X0, const float*
 // ---- host: schedules ------------------------------------------------------------------
 
 struct Plan {
-  std::vector<int32_t> host;  // [grid + 1] offsets, then tile codes
-  int grid = 0;
+  std::vector<int32_t> host;  // [lists + 1] offsets, then tile codes
+  int grid = 0;               // tile lists: CTAs, or SM pairs when tm = 256
 };
 
-Plan make_plan(int num_sms, int d, int f, int C, bool apply_update, bool target) {
+// Tile lists for up to `lists` CTAs (tm = 128) or SM pairs (tm = 256, tiles of 256 rows).
+Plan make_plan(int lists, int tm, int d, int f, int C, bool apply_update, bool target) {
   struct T {
     int32_t code;
     int cost;
   };
   std::vector<T> tl;
-  const int mt_tok = C / BM, nt_d = (d + BN - 1) / BN;
+  const int mt_tok = C / tm, nt_d = (d + BN - 1) / BN;
   if (apply_update) {
     const int cost_apply = (f + BK - 1) / BK + 2;
     for (int m = 0; m < mt_tok; ++m)
@@ -617,10 +758,10 @@ Plan make_plan(int num_sms, int d, int f, int C, bool apply_update, bool target)
     // The read-modify-write epilogue (fp32 W in and out, bf16 copy out: 320 KB per tile)
     // costs more than the 16-deep mainloop; weigh it in.
     const int cost_u = std::max(C / BK, 20);
-    for (int m = 0; m < (d + BM - 1) / BM; ++m)
+    for (int m = 0; m < (d + tm - 1) / tm; ++m)
       for (int n = 0; n < (f + BN - 1) / BN; ++n) tl.push_back({tile_code(UPDATE, m, n), cost_u});
   }
-  const int grid = std::max(1, std::min<int>(num_sms, (int)tl.size()));
+  const int grid = std::max(1, std::min<int>(lists, (int)tl.size()));
   std::stable_sort(tl.begin(), tl.end(), [](const T& a, const T& b) { return a.cost > b.cost; });
   std::vector<std::vector<int32_t>> per(grid);
   std::vector<long> load(grid, 0);
@@ -672,12 +813,58 @@ ttt_status map2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t oute
 
 static_assert(sizeof(TCSmem) + 1024 <= 232448, "k_inplace_tc exceeds the 227 KB of shared memory per block");
 
+constexpr size_t kSmemTC = sizeof(TCSmem) + 1024;
+
+// Rotation of the tile lists between rounds: the largest step up to half the list count that
+// is coprime to it (73 for 148 lists, 35 for 74), so a CTA meets every list and consecutive
+// rounds take lists far apart (measured on 148 lists: 73 against 1 and 61).
+int list_rotation(int lists) {
+  for (int r = lists / 2; r > 1; --r) {
+    int a = lists, b = r;
+    while (b) {
+      const int t = a % b;
+      a = b;
+      b = t;
+    }
+    if (a == 1) return r;
+  }
+  return 1;
+}
+
+// Launches k_inplace_tc<pair> on `grid` CTAs (clusters of two when pair). Cooperative launches
+// (several rounds whose CTAs wait on one another) check that every CTA is resident; a cluster
+// launch is checked against the occupancy query when its lists are planned.
+ttt_status launch_tc(bool pair, int grid, bool cooperative, void** params, cudaStream_t s) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreadsTC);
+  cfg.dynamicSmemBytes = kSmemTC;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  if (pair) {
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 2;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+  } else {
+    at[0].id = cudaLaunchAttributeCooperative;
+    at[0].val.cooperative = cooperative ? 1 : 0;
+  }
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  const void* fn = pair ? reinterpret_cast<const void*>(k_inplace_tc<true>) : reinterpret_cast<const void*>(k_inplace_tc<false>);
+  TTT_CUDA(cudaLaunchKernelExC(&cfg, fn, params));
+  return TTT_OK;
+}
+
 }  // namespace
 
 // Per-state tensor-core resources (schedules, conv buffer), created on first use.
 struct TCResources {
   int32_t* plan_dev[3] = {nullptr, nullptr, nullptr};  // 0: steady, 1: target only, 2: apply+update only
-  int grid[3] = {0, 0, 0};
+  int grid[3] = {0, 0, 0};   // CTAs of each plan's launch (two per list with SM pairs)
+  int lists[3] = {0, 0, 0};
+  bool pair = false;         // tiles of 256 rows on SM pairs
   __nv_bfloat16* conv = nullptr;
   size_t conv_rows = 0;
   int* counters = nullptr;  // per-round progress counters of a multi-chunk launch
@@ -690,17 +877,48 @@ static ttt_status ensure_tc(ttt_state* st) {
   TCResources* r = new (std::nothrow) TCResources();
   if (r == nullptr) return fail(TTT_ERR_OOM, "host allocation failed");
   const bool target = c.target_mode == 1;
-  Plan p0 = make_plan(st->num_sms, c.d_val, c.d_key, c.chunk, true, target);
-  ttt_status s = upload_plan(p0, &r->plan_dev[0]);
-  r->grid[0] = p0.grid;
+  ttt_status s = TTT_OK;
+  // SM pairs where every tile has two full 128-row halves: the chunk and d_val multiples of 256.
+  int lists = st->num_sms;
+  r->pair = st->ip.sm_pair != 0 && c.chunk % kTileP == 0 && c.d_val % kTileP == 0;
+  if (r->pair) {
+    // As many pairs as can be resident at once (an SM left without a partner in its GPC idles).
+    cudaError_t e = cudaFuncSetAttribute(k_inplace_tc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemTC);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * (st->num_sms / 2));
+    cfg.blockDim = dim3(kThreadsTC);
+    cfg.dynamicSmemBytes = kSmemTC;
+    cudaLaunchAttribute at;
+    at.id = cudaLaunchAttributeClusterDimension;
+    at.val.clusterDim.x = 2;
+    at.val.clusterDim.y = 1;
+    at.val.clusterDim.z = 1;
+    cfg.attrs = &at;
+    cfg.numAttrs = 1;
+    int clusters = 0;
+    if (e == cudaSuccess) e = cudaOccupancyMaxActiveClusters(&clusters, k_inplace_tc<true>, &cfg);
+    if (e != cudaSuccess) {
+      delete r;
+      return fail(TTT_ERR_CUDA, "SM-pair occupancy query failed: %s", cudaGetErrorString(e));
+    }
+    lists = std::min(st->num_sms / 2, clusters);
+    if (lists < 1) r->pair = false;
+  }
+  if (!r->pair) lists = st->num_sms;
+  const int tm = r->pair ? kTileP : BM;
+  const int per = r->pair ? 2 : 1;
+  Plan p0 = make_plan(lists, tm, c.d_val, c.d_key, c.chunk, true, target);
+  s = upload_plan(p0, &r->plan_dev[0]);
+  r->lists[0] = p0.grid;
   if (s == TTT_OK && target) {
-    Plan p1 = make_plan(st->num_sms, c.d_val, c.d_key, c.chunk, false, true);
-    Plan p2 = make_plan(st->num_sms, c.d_val, c.d_key, c.chunk, true, false);
+    Plan p1 = make_plan(lists, tm, c.d_val, c.d_key, c.chunk, false, true);
+    Plan p2 = make_plan(lists, tm, c.d_val, c.d_key, c.chunk, true, false);
     s = upload_plan(p1, &r->plan_dev[1]);
     if (s == TTT_OK) s = upload_plan(p2, &r->plan_dev[2]);
-    r->grid[1] = p1.grid;
-    r->grid[2] = p2.grid;
+    r->lists[1] = p1.grid;
+    r->lists[2] = p2.grid;
   }
+  for (int i = 0; i < 3; ++i) r->grid[i] = per * r->lists[i];
   if (s != TTT_OK) {
     for (int i = 0; i < 3; ++i)
       if (r->plan_dev[i]) cudaFree(r->plan_dev[i]);
@@ -735,7 +953,8 @@ ttt_status inplace_bf16_scan(ttt_state* st, const __nv_bfloat16* Z, const __nv_b
   TTT_TRY(map2d(&tmWf, st->ip.W, f, d, kWCols, BM, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, CU_TENSOR_MAP_SWIZZLE_128B));
   for (int i = 0; i < 3; ++i) {
     TTT_TRY(map2d(&tmWs[i], st->ip.Wsh[i], f, d, kWCols, BM, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, CU_TENSOR_MAP_SWIZZLE_64B));
-    TTT_TRY(map2d(&tmWk[i], st->ip.Wsh[i], f, d, BK, BN));
+    // APPLY B operand: 256 rows of the bf16 W per tile, 128 per CTA of an SM pair.
+    TTT_TRY(map2d(&tmWk[i], st->ip.Wsh[i], f, d, BK, r->pair ? BN / 2 : BN));
   }
   TTT_TRY(map2d(&tmZk, Z, f, T, BK, BM));
   TTT_TRY(map2d(&tmZm, Z, f, T, 64, BK));
@@ -761,8 +980,10 @@ ttt_status inplace_bf16_scan(ttt_state* st, const __nv_bfloat16* Z, const __nv_b
     tmWt = tmZk;
   }
 
-  const size_t smem = sizeof(TCSmem) + 1024;
-  TTT_CUDA(cudaFuncSetAttribute(k_inplace_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  if (r->pair)
+    TTT_CUDA(cudaFuncSetAttribute(k_inplace_tc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemTC));
+  else
+    TTT_CUDA(cudaFuncSetAttribute(k_inplace_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemTC));
 
   auto args_for = [&](int plan, int chunk, int tchunk, int rounds, int* counters) {
     TCArgs a;
@@ -782,6 +1003,7 @@ ttt_status inplace_bf16_scan(ttt_state* st, const __nv_bfloat16* Z, const __nv_b
       a.stall_round = 1;
       st->inject_stall = 0;
     }
+    a.rotate = list_rotation(r->lists[plan]);
     a.rounds = rounds;
     a.cur0 = st->ip.cur;
     a.nbd = (d + BN - 1) / BN;
@@ -792,24 +1014,25 @@ ttt_status inplace_bf16_scan(ttt_state* st, const __nv_bfloat16* Z, const __nv_b
     a.tgt_done = nullptr;
     return a;
   };
-  auto launch = [&](int plan, const TCArgs& a, const CUtensorMap& vm) -> ttt_status {
-    k_inplace_tc<<<r->grid[plan], kThreadsTC, smem, s>>>(tmZk, tmZm, vm, vm, vm, tmWk[0], tmWk[1], tmWk[2], tmConv, tmWt,
-                                                         tmWf, tmWs[0], tmWs[1], tmWs[2], a);
+  auto launch = [&](int plan, TCArgs a, const CUtensorMap& vm) -> ttt_status {
+    void* params[] = {&tmZk, &tmZm, const_cast<CUtensorMap*>(&vm), const_cast<CUtensorMap*>(&vm),
+                      const_cast<CUtensorMap*>(&vm), &tmWk[0], &tmWk[1], &tmWk[2], &tmConv, &tmWt, &tmWf,
+                      &tmWs[0], &tmWs[1], &tmWs[2], &a};
+    TTT_TRY(launch_tc(r->pair, r->grid[plan], false, params, s));
     st->launches++;
-    TTT_CUDA(cudaGetLastError());
     return TTT_OK;
   };
   // All chunks in one launch: each CTA runs its tile list once per chunk, waiting on progress
   // counters only where a chunk needs another CTA's result of an earlier chunk, so a chunk's
-  // last tiles overlap the next chunk's first. The grid is one CTA per SM and is launched
-  // cooperatively, which guarantees that every CTA is resident.
+  // last tiles overlap the next chunk's first. The grid is one CTA (or SM pair) per SM (pair)
+  // that can be resident at once: launched cooperatively, or as clusters sized by the
+  // occupancy query, so every CTA is resident.
   auto launch_rounds = [&](TCArgs& a, const CUtensorMap& vm0, const CUtensorMap& vm1,
                            const CUtensorMap& vm2) -> ttt_status {
     void* params[] = {&tmZk, &tmZm, const_cast<CUtensorMap*>(&vm0), const_cast<CUtensorMap*>(&vm1),
                       const_cast<CUtensorMap*>(&vm2), &tmWk[0], &tmWk[1], &tmWk[2], &tmConv, &tmWt, &tmWf,
                       &tmWs[0], &tmWs[1], &tmWs[2], &a};
-    TTT_CUDA(cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(k_inplace_tc), dim3(r->grid[0]),
-                                         dim3(kThreadsTC), params, smem, s));
+    TTT_TRY(launch_tc(r->pair, r->grid[0], true, params, s));
     st->launches++;
     st->ip.cur = (st->ip.cur + nchunks) % 3;
     return TTT_OK;
@@ -916,9 +1139,9 @@ ttt_status target_values_into(const __nv_bfloat16* X0, const float* convw, const
   a.sched_last = nullptr;
   a.vhat[0] = a.vhat[1] = a.vhat[2] = nullptr;
   a.tgt_done = nullptr;
-  const size_t smem = sizeof(TCSmem) + 1024;
-  TTT_CUDA(cudaFuncSetAttribute(k_inplace_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-  k_inplace_tc<<<grid, kThreadsTC, smem, s>>>(tmConv, tmConv, tmConv, tmConv, tmConv, tmConv, tmConv, tmConv, tmConv, tmWt,
+  a.rotate = 1;
+  TTT_CUDA(cudaFuncSetAttribute(k_inplace_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemTC));
+  k_inplace_tc<false><<<grid, kThreadsTC, kSmemTC, s>>>(tmConv, tmConv, tmConv, tmConv, tmConv, tmConv, tmConv, tmConv, tmConv, tmWt,
                                               tmConv, tmConv, tmConv, tmConv, a);
   TTT_CUDA(cudaGetLastError());
   return TTT_OK;

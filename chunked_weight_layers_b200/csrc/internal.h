@@ -56,6 +56,7 @@ struct InplaceBuffers {
   // Context-parallel form (TTT_OPT_INPLACE_PREFIX): the chunks' fp32 deltas [n][d][f] and the bf16
   // weights each chunk applies with [n][d][f], grown on demand.
   int prefix_form = 0;
+  int sm_pair = 1;               // TTT_OPT_SM_PAIR: tensor-core tiles on SM pairs where shapes allow
   float* prefix_D = nullptr;
   __nv_bfloat16* prefix_Wb = nullptr;
   int prefix_chunks = 0;

@@ -500,6 +500,13 @@ ttt_status ttt_state_set_option(ttt_state* st, int32_t option, int64_t value) {
         return fail(TTT_ERR_UNSUPPORTED, "the context-parallel form runs In-Place BF16 states with given targets");
       st->ip.prefix_form = (int)value;
       return TTT_OK;
+    case TTT_OPT_SM_PAIR:
+      if (value != 0 && value != 1) return fail(TTT_ERR_INVALID_ARG, "TTT_OPT_SM_PAIR must be 0 or 1");
+      if (st->ip.sm_pair != (int)value) {
+        st->ip.sm_pair = (int)value;
+        free_tc(st);  // schedules are built per tile shape; rebuilt on the next scan
+      }
+      return TTT_OK;
     case TTT_OPT_INJECT_STALL:
       if (value != 0 && value != 1) return fail(TTT_ERR_INVALID_ARG, "TTT_OPT_INJECT_STALL must be 0 or 1");
       st->inject_stall = (int)value;

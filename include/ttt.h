@@ -269,7 +269,14 @@ typedef enum {
    * to rounding (each η·ΔW_j is rounded to fp32 before it is added). The call keeps n fp32
    * deltas and n bf16 weights of d_val x d_key in state-owned scratch (grown on demand, n =
    * T / chunk). 0 returns to the sequential form. UNSUPPORTED for other states. */
-  TTT_OPT_INPLACE_PREFIX = 4
+  TTT_OPT_INPLACE_PREFIX = 4,
+  /* In-Place BF16 states, sequential form: 1 (default) runs the tensor-core scan on pairs of
+   * SMs (clusters of two CTAs, tcgen05 MMAs of 256 x 256 tiles issued for both) wherever the
+   * chunk and d_val are multiples of 256, and on single SMs (128 x 256 tiles) otherwise; 0
+   * always uses single SMs. Both give the same results up to the order of fp32 additions
+   * inside the tensor cores. Changing it rebuilds the state's tile schedules on the next scan
+   * (the call synchronises the device). Other states ignore it. */
+  TTT_OPT_SM_PAIR = 5
 } ttt_option;
 
 /* Set option `option` of state `st` to `value`. Takes effect from the next call that

@@ -72,11 +72,14 @@ def test_linear_scan_wait_runs_out(cwl, form):
     assert torch.equal(O2, O) and torch.equal(W2, W) and torch.equal(L2, L)
 
 
-def test_inplace_tensor_core_scan_wait_runs_out(cwl):
+@pytest.mark.parametrize("C", [128, 256])
+def test_inplace_tensor_core_scan_wait_runs_out(cwl, C):
+    """C = 128: one CTA per tile; C = 256 (d = 256): clusters of two CTAs per tile, where the
+    CTAs of a pair also wait on each other."""
     from chunked_weight_layers_b200 import abi
-    spec = workloads.scaled(workloads.INPLACE_4B, T=256, C=128, d=256, f=256, seed=405)
+    spec = workloads.scaled(workloads.INPLACE_4B, T=2 * C, C=C, d=256, f=256, seed=405)
     x = workloads.inplace_inputs(spec, device="cuda")
-    cfg = cwl.config("inplace", io_dtype=1, d_key=256, d_val=256, chunk=128, eta=spec.eta)
+    cfg = cwl.config("inplace", io_dtype=1, d_key=256, d_val=256, chunk=C, eta=spec.eta)
 
     def scan(st):
         O = torch.empty((spec.T, spec.d), device="cuda", dtype=torch.bfloat16)
@@ -91,7 +94,7 @@ def test_inplace_tensor_core_scan_wait_runs_out(cwl):
     scan(st)  # two chunks: one launch of two rounds; round 1's APPLY tiles wait in vain
     _expect_timeout(st)
 
-    Oref, Wref = oinp.inplace_scan(x["Z"].cpu(), x["Vhat"].cpu(), x["W0"].cpu(), spec.eta, 128)
+    Oref, Wref = oinp.inplace_scan(x["Z"].cpu(), x["Vhat"].cpu(), x["W0"].cpu(), spec.eta, C)
     st.reset()
     O, W = scan(st)
     st.poll()
@@ -107,7 +110,7 @@ def test_option_ranges(cwl):
     W0 = torch.eye(64, device="cuda").expand(1, 1, 64, 64).contiguous()
     st = cwl.FastWeightState(cwl.config("linear", batch=1, heads=1, chunk=16), W0)
     for opt, bad in ((abi.TTT_OPT_WAIT_LIMIT_NS, 999), (abi.TTT_OPT_WAIT_LIMIT_NS, 60_000_000_001),
-                     (abi.TTT_OPT_INJECT_STALL, 2)):
+                     (abi.TTT_OPT_INJECT_STALL, 2), (abi.TTT_OPT_SM_PAIR, 2)):
         with pytest.raises(TTTError) as e:
             st.set_option(opt, bad)
         assert e.value.status == abi.TTT_ERR_INVALID_ARG
