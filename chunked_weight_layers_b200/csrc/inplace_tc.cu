@@ -31,14 +31,14 @@
 //    warp 1 allocates 512 TMEM columns and one lane issues tcgen05.mma (M=128, N=256, K=16)
 //    into one of two TMEM accumulators, warps 2..9 drain the other accumulator
 //    (tcgen05.ld 32x32b) in the epilogue, two warps per TMEM lane quarter, and warp 10
-//    streams the fp32 W of UPDATE tiles by TMA into a 4-slot ring of 128x32 sub-tiles while
+//    streams the fp32 W of UPDATE tiles by TMA into a 3-slot ring of 128x32 sub-tiles while
 //    the mainloop runs. The epilogue adds η·ΔW in shared memory, writes the bf16 copy beside
 //    it, and two TMA stores per sub-tile write both back: the read-modify-write of the 99.6 MB
 //    state never goes through per-thread global loads.
 //  * SM pairs: where the chunk and d_model are multiples of 256 the kernel runs as clusters
 //    of two CTAs on neighbouring SMs, each tile 256 rows x 256 columns. Each CTA loads by TMA
 //    its own 128 rows of A and its own 128 columns of B (32 KB a k-block instead of 48 KB
-//    for the same MMA work per SM, in a 4-stage ring), a lane of the second CTA tells the
+//    for the same MMA work per SM, in a 5-stage ring), a lane of the second CTA tells the
 //    first when its stage has landed, and one lane of the first issues tcgen05.mma with
 //    cta_group::2 (M = 256, N = 256), whose commits arrive on the barriers of both CTAs.
 //    Each CTA's TMEM holds its own 128 rows of the accumulator, so the epilogue is the same
@@ -61,15 +61,15 @@ constexpr int BM = 128, BN = 256, BK = 64;
 constexpr int kSt = 3;                      // operand ring depth (k-blocks)
 constexpr int kABytes = BM * BK * 2;        // 16 KB
 constexpr int kBBytes = BN * BK * 2;        // 32 KB
-constexpr int kRingBytes = kSt * (kABytes + kBBytes);
 constexpr int kTileP = 2 * BM;              // rows of an SM-pair tile
-constexpr int kStP = 4;                     // operand ring depth of an SM pair (32 KB stages)
-constexpr int kStMax = 4;
-static_assert(kStP * (kABytes + kBBytes / 2) <= kRingBytes, "SM-pair stages exceed the operand ring");
+constexpr int kStP = 5;                     // operand ring depth of an SM pair (32 KB stages)
+constexpr int kStMax = 5;
+constexpr int kRingBytes = kStP * (kABytes + kBBytes / 2);
+static_assert(kSt * (kABytes + kBBytes) <= kRingBytes, "single-SM stages exceed the operand ring");
 constexpr int kWCols = 32;                  // columns of one W sub-tile of an UPDATE tile
 constexpr int kWBytes = BM * kWCols * 4;    // 16 KB of fp32 W
 constexpr int kShBytes = BM * kWCols * 2;   // 8 KB of its bf16 copy
-constexpr int kWSlots = 4;                  // W sub-tile ring depth
+constexpr int kWSlots = 3;                  // W sub-tile ring depth
 constexpr int kEpiWarps = 8;
 constexpr int kWarpWload = 2 + kEpiWarps;   // the warp that streams W sub-tiles in
 constexpr int kThreadsTC = (3 + kEpiWarps) * 32;
