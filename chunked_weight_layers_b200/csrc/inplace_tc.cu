@@ -38,9 +38,10 @@
 //  * SM pairs: where the chunk and d_model are multiples of 256 the kernel runs as clusters
 //    of two CTAs on neighbouring SMs, each tile 256 rows x 256 columns. Each CTA loads by TMA
 //    its own 128 rows of A and its own 128 columns of B (32 KB a k-block instead of 48 KB
-//    for the same MMA work per SM, in a 5-stage ring), a lane of the second CTA tells the
-//    first when its stage has landed, and one lane of the first issues tcgen05.mma with
-//    cta_group::2 (M = 256, N = 256), whose commits arrive on the barriers of both CTAs.
+//    for the same MMA work per SM, in a 5-stage ring); both CTAs' loads of a stage complete
+//    on the first CTA's barrier, which expects the bytes of both, and one lane of the first
+//    issues tcgen05.mma with cta_group::2 (M = 256, N = 256), whose commits arrive on the
+//    barriers of both CTAs.
 //    Each CTA's TMEM holds its own 128 rows of the accumulator, so the epilogue is the same
 //    per CTA; the second CTA's epilogue warps release the accumulator on the first's barrier.
 //    No load is multicast: every CTA reads its own operands.
@@ -88,7 +89,6 @@ struct __align__(1024) TCSmem {
   uint8_t Wr[kWSlots][kWBytes];  // fp32 W sub-tiles (128 rows x 32 columns, 128-byte swizzle)
   uint8_t Sh[2][kShBytes];       // bf16 copy of an updated sub-tile, one per column half (64-byte swizzle)
   uint64_t full[kStMax], empty[kStMax];
-  uint64_t peer_full[kStMax];    // SM pair, first CTA: the second CTA's stage s has landed
   uint64_t tfull[2], tempty[2];
   uint64_t wfull[kWSlots], wempty[kWSlots];
   uint32_t tmem_base;
@@ -229,11 +229,10 @@ __device__ __forceinline__ uint32_t in_first_cta(const void* p) {
 }
 
 // Arrive on the mbarrier at shared::cluster address `addr` (in the other CTA of the pair),
-// relaxed: it orders nothing before it. Its two uses signal events that have completed before
-// it is issued (a TMA load observed on this CTA's barrier; tcgen05.ld reads of TMEM finished by
-// tcgen05.wait::ld), not writes made visible by it. A release at cluster scope here waits for
-// every memory operation this thread has in flight; measured on B200 that made each
-// stage-landed message ~1400 cycles, more than the k-block's 512 cycles of MMA.
+// relaxed: it orders nothing before it. It signals that this thread's tcgen05.ld reads of TMEM
+// have finished (tcgen05.wait::ld before it), not writes made visible by it. A release at
+// cluster scope would wait for every memory operation the thread has in flight (its output
+// stores): measured on B200, a release arrive took ~1400 cycles.
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t addr) {
   asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(addr) : "memory");
 }
@@ -281,6 +280,25 @@ __device__ __forceinline__ void store_row_bf16(__nv_bfloat16* row, int col0, int
 __device__ __forceinline__ const CUtensorMap* pick3(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& c,
                                                     int i) {
   return i == 0 ? &a : (i == 1 ? &b : &c);
+}
+
+// TMA load of a box into this CTA's shared memory, completing on the mbarrier at shared::cluster
+// address `bar`; PAIR: the barrier may be in the other CTA of the pair (cta_group::2 form).
+template <bool PAIR>
+__device__ __forceinline__ void tma_load_2d_to(void* dst, const CUtensorMap* map, uint32_t bar, int32_t c0, int32_t c1) {
+  if constexpr (PAIR) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
+        : "memory");
+  } else {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
+        : "memory");
+  }
 }
 
 __device__ __forceinline__ void fence_proxy_async_global() {
@@ -369,7 +387,6 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&sm.full[i], 1);
       mbar_init(&sm.empty[i], 1);
-      mbar_init(&sm.peer_full[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sm.tfull[i], 1);
@@ -436,33 +453,45 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
             return false;
           uint8_t* sa = sm.ring + s * kStage;
           uint8_t* sb = sa + kABytes;
-          mbar_arrive_expect_tx(&sm.full[s], kStage);
+          // SM pair: the loads of both CTAs complete on the first CTA's barrier, which expects
+          // the bytes of both (a load may complete before the expectation is posted: the phase
+          // cannot end before it is).
+          if (rank == 0) mbar_arrive_expect_tx(&sm.full[s], PAIR ? 2 * kStage : kStage);
+          const uint32_t fb = PAIR ? in_first_cta(&sm.full[s]) : smem_u32(&sm.full[s]);
           if (type == APPLY) {
-            tma_load_2d(sa, &tmZk, &sm.full[s], kb * BK, chunk * args.C + r0);
-            tma_load_2d(sb, wk, &sm.full[s], kb * BK, b0);
+            tma_load_2d_to<PAIR>(sa, &tmZk, fb, kb * BK, chunk * args.C + r0);
+            tma_load_2d_to<PAIR>(sb, wk, fb, kb * BK, b0);
           } else if (type == UPDATE) {
             for (int j = 0; j < BM / 64; ++j)
-              tma_load_2d(sa + j * 8192, vm, &sm.full[s], r0 + j * 64,
-                          args.vrow0 + (args.tgt_done != nullptr ? 0 : rnd * args.C) + kb * BK);
+              tma_load_2d_to<PAIR>(sa + j * 8192, vm, fb, r0 + j * 64,
+                                   args.vrow0 + (args.tgt_done != nullptr ? 0 : rnd * args.C) + kb * BK);
             for (int j = 0; j < kBCols / 64; ++j)
-              tma_load_2d(sb + j * 8192, &tmZm, &sm.full[s], b0 + j * 64, chunk * args.C + kb * BK);
+              tma_load_2d_to<PAIR>(sb + j * 8192, &tmZm, fb, b0 + j * 64, chunk * args.C + kb * BK);
           } else {
-            tma_load_2d(sa, &tmConv, &sm.full[s], kb * BK, (args.target_chunk + rnd) * args.C + r0);
+            tma_load_2d_to<PAIR>(sa, &tmConv, fb, kb * BK, (args.target_chunk + rnd) * args.C + r0);
             for (int j = 0; j < kBCols / 64; ++j)
-              tma_load_2d(sb + j * 8192, &tmWt, &sm.full[s], b0 + j * 64, kb * BK);
+              tma_load_2d_to<PAIR>(sb + j * 8192, &tmWt, fb, b0 + j * 64, kb * BK);
           }
         }
         return true;
       });
-      // Drain: the newest phase issued on every stage must have landed before exit.
+      // Drain: nothing may still land in this CTA's shared memory when it exits.
       const uint32_t first = it > (uint32_t)kStages ? it - kStages : 0;
-      for (uint32_t k = first; k < it; ++k) mbar_wait(&sm.full[k % kStages], (k / kStages) & 1, args.status, nullptr);
-      // PAIR: the first CTA's MMA lane releases every stage by a commit that arrives on both
-      // CTAs' barriers; after a clean run wait for the last of them, so that none arrives
-      // after this CTA has exited.
-      if (PAIR && !*abort)
+      if constexpr (!PAIR) {
+        for (uint32_t k = first; k < it; ++k)
+          mbar_wait(&sm.full[k % kStages], (k / kStages) & 1, args.status, nullptr);
+      } else if (!*abort) {
+        // Every stage was consumed by MMAs that waited for both CTAs' bytes; the commits that
+        // released the last stages arrive on this CTA's barriers too: wait for them.
         for (uint32_t k = first; k < it; ++k)
           mbar_wait(&sm.empty[k % kStages], (k / kStages) & 1, args.status, nullptr);
+      } else {
+        // After an abort a stage may never complete on the first CTA's barrier (its partner's
+        // half missing), so no barrier tells when this CTA's last loads have landed: wait
+        // 50 us, far beyond the latency of a TMA load, before the CTA may exit.
+        const uint64_t t0 = globaltimer();
+        while (globaltimer() - t0 < 50000) __nanosleep(1000);
+      }
     }
   } else if (warp == kWarpWload) {
     // ---------------- W sub-tile loader (fp32 W of UPDATE tiles, 128 x 32) ----------------
@@ -494,21 +523,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         mbar_wait(&sm.wfull[k % kWSlots], (k / kWSlots) & 1, args.status, nullptr);
     }
   } else if (warp == 1) {
-    if (PAIR && rank != 0) {
-      // ---------------- second CTA of a pair: report landed stages to the first ----------------
-      if (lane == 0) {
-        uint32_t it = 0;
-        for_tiles([&](int, int32_t tc) -> bool {
-          const int nk = kblocks(tile_type(tc), args);
-          for (int kb = 0; kb < nk; ++kb, ++it) {
-            const int s = it % kStages;
-            if (!mbar_wait(&sm.full[s], (it / kStages) & 1, args.status, abort)) return false;
-            mbar_arrive_remote(in_first_cta(&sm.peer_full[s]));
-          }
-          return true;
-        });
-      }
-    } else if (lane == 0) {
+    if (lane == 0 && rank == 0) {
       // ------------------------------- MMA issuer -------------------------------
       uint32_t it = 0, tcount = 0;
       bool ok = true;
@@ -528,8 +543,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
                                                 : idesc_bf16(kM, 0, 1);
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const int s = it % kStages;
-          if (!mbar_wait(&sm.full[s], (it / kStages) & 1, args.status, abort) ||
-              (PAIR && !mbar_wait<true>(&sm.peer_full[s], (it / kStages) & 1, args.status, abort))) {
+          if (!mbar_wait<PAIR>(&sm.full[s], (it / kStages) & 1, args.status, abort)) {
             ok = false;
             break;
           }
