@@ -19,15 +19,23 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 // Where a kernel reports a failure, and how long each of its spin-waits may last.
 struct DevStatus {
-  int* word;          // status word (mapped host memory or device memory), or null
-  uint64_t limit_ns;  // wait limit in %globaltimer nanoseconds
+  int* word;             // status word (mapped host memory or device memory), or null
+  uint64_t limit_ns;     // wait limit in %globaltimer nanoseconds
+  int* site = nullptr;   // where the first failure happened (kSite* | detail), or null
 };
+
+// Sites of a wait that ran out: an mbarrier (detail: its shared-memory offset) or a progress
+// counter in global memory (detail: the low bits of its word address).
+constexpr int kSiteMbarrier = 0x10000;
+constexpr int kSiteCounter = 0x20000;
 
 __device__ __forceinline__ void record_status(int* status, int code) {
   if (status != nullptr) atomicCAS(status, 0, code);
 }
 
-__device__ __forceinline__ void record_status(const DevStatus& status, int code) { record_status(status.word, code); }
+__device__ __forceinline__ void record_status(const DevStatus& status, int code, int site = 0) {
+  if (status.word != nullptr && atomicCAS(status.word, 0, code) == 0 && status.site != nullptr) *status.site = site;
+}
 
 __device__ __forceinline__ uint64_t globaltimer() {
   uint64_t t;
@@ -101,7 +109,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
     if ((++spins & 63u) == 0) {
       if (abort != nullptr && *abort) return false;
       if (globaltimer() - t0 > status.limit_ns) {
-        record_status(status, kDevTimeout);
+        record_status(status, kDevTimeout, kSiteMbarrier | (int)(smem_u32(bar) & 0xFFFFu));
         if (abort != nullptr) *abort = 1;
         return false;
       }

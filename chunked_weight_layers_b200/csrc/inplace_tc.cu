@@ -314,7 +314,7 @@ __device__ __forceinline__ bool wait_counter(const int* ctr, int want, const Dev
     while (*c < want) {
       if (*abort) return false;
       if (globaltimer() - t0 > status.limit_ns) {
-        record_status(status, kDevTimeout);
+        record_status(status, kDevTimeout, kSiteCounter | (int)((reinterpret_cast<uintptr_t>(ctr) >> 2) & 0xFFFFu));
         *abort = 1;
         return false;
       }
@@ -1011,7 +1011,7 @@ ttt_status inplace_bf16_scan(ttt_state* st, const __nv_bfloat16* Z, const __nv_b
     a.eta = c.eta;
     a.O = O;
     a.Vhat_out = target ? st->ip.Vhat[tchunk % 3] : nullptr;
-    a.status = DevStatus{st->status.dev, st->wait_limit_ns};
+    a.status = DevStatus{st->status.dev, st->wait_limit_ns, st->status.dev + 1};
     a.stall_round = -1;
     if (st->inject_stall && rounds >= 2 && counters != nullptr) {
       a.stall_round = 1;

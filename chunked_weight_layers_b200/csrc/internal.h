@@ -31,8 +31,9 @@ ttt_status cuda_fail(cudaError_t e, const char* what);
     if (s_ != TTT_OK) return s_;           \
   } while (0)
 
-// Device-visible status word (pinned, mapped host memory): kernels record the first
-// failure there with atomicCAS; the host reads it in ttt_state_poll().
+// Device-visible status words (pinned, mapped host memory): kernels record the first
+// failure in host[0] with atomicCAS and where it happened in host[1]; the host reads both in
+// ttt_state_poll().
 struct StatusWord {
   int* host = nullptr;
   int* dev = nullptr;

@@ -530,7 +530,7 @@ __device__ __forceinline__ bool wait_turn(const int* turn, int want, const DevSt
   while (*tv != want) {
     if (*av) return false;
     if (globaltimer() - t0 > status.limit_ns) {
-      record_status(status, kDevTimeout);
+      record_status(status, kDevTimeout, kSiteCounter | (int)((reinterpret_cast<uintptr_t>(turn) >> 2) & 0xFFFFu));
       *const_cast<volatile int*>(av) = 1;
       return false;
     }
@@ -1119,7 +1119,7 @@ ttt_status launch(ttt_state* st, const CUtensorMap& tk, const CUtensorMap& tv, c
   const int grid = st->cfg.batch * st->cfg.heads;
   const float beta = st->cfg.eta / (float)B;
   k_linear_scan<B><<<grid, kThreads, smem, s>>>(tk, tv, tq, to, st->lin.W, loss, T, beta, has_q,
-                                                DevStatus{st->status.dev, st->wait_limit_ns});
+                                                DevStatus{st->status.dev, st->wait_limit_ns, st->status.dev + 1});
   st->launches++;
   TTT_CUDA(cudaGetLastError());
   return TTT_OK;
@@ -1159,7 +1159,7 @@ ttt_status launch_b16_nb(ttt_state* st, const CUtensorMap& tk, const CUtensorMap
   lc.attrs = attr;
   lc.numAttrs = 1;
   TTT_CUDA(cudaLaunchKernelEx(&lc, k_linear_b16<HAS_Q, LOSS, GATE, NB>, tk, tv, tq, to, st->lin.W, loss, T, beta,
-                              DevStatus{st->status.dev, st->wait_limit_ns}, ga, stall_tile));
+                              DevStatus{st->status.dev, st->wait_limit_ns, st->status.dev + 1}, ga, stall_tile));
   st->launches++;
   TTT_CUDA(cudaGetLastError());
   return TTT_OK;

@@ -246,7 +246,7 @@ ttt_status inplace_bf16_scan_prefix(ttt_state* st, const __nv_bfloat16* Z, const
     TTT_CUDA(cudaMalloc(reinterpret_cast<void**>(&ip.prefix_Wb), (size_t)n * nelem * 2));
     ip.prefix_chunks = n;
   }
-  const DevStatus ds{st->status.dev, st->wait_limit_ns};
+  const DevStatus ds{st->status.dev, st->wait_limit_ns, st->status.dev + 1};
 
   // 1. D_j = η·V̂_jᵀ·Z_j: M = d, N = f, K = C; A = V̂ (MN-major), B = Z (MN-major), batch j at token jC.
   CUtensorMap tV, tZm;

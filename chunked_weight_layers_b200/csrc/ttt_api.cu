@@ -179,13 +179,13 @@ static ttt_status create_impl(const ttt_config* cfg, const void* W0, const void*
     free_state(st);
     return cuda_fail(e, "cudaGetDevice");
   }
-  e = cudaHostAlloc(reinterpret_cast<void**>(&st->status.host), sizeof(int), cudaHostAllocMapped);
+  e = cudaHostAlloc(reinterpret_cast<void**>(&st->status.host), 2 * sizeof(int), cudaHostAllocMapped);
   if (e == cudaSuccess) e = cudaHostGetDevicePointer(reinterpret_cast<void**>(&st->status.dev), st->status.host, 0);
   if (e != cudaSuccess) {
     free_state(st);
     return cuda_fail(e, "status word allocation");
   }
-  *st->status.host = 0;
+  st->status.host[0] = st->status.host[1] = 0;
 
   const size_t nW = weight_elems(c);
   if (c.rule == TTT_RULE_INPLACE_HEBBIAN) {
@@ -473,10 +473,14 @@ ttt_status ttt_state_poll(ttt_state* st) {
   if (st == nullptr) return fail(TTT_ERR_INVALID_ARG, "state is NULL");
   TTT_CUDA(cudaDeviceSynchronize());
   volatile int* w = st->status.host;
-  const int v = *w;
-  *w = 0;
+  const int v = w[0], site = w[1];
+  w[0] = 0;
+  w[1] = 0;
   if (v == 0) return TTT_OK;
-  if (v == TTT_ERR_TIMEOUT) return fail(TTT_ERR_TIMEOUT, "a bounded device-side wait ran out");
+  if (v == TTT_ERR_TIMEOUT)
+    return fail(TTT_ERR_TIMEOUT, "a bounded device-side wait ran out (%s 0x%x)",
+                (site & 0x30000) == 0x20000 ? "progress counter at word" : "mbarrier at shared offset",
+                site & 0xFFFF);
   return fail(TTT_ERR_DEVICE, "a device-side check failed (code %d)", v);
 }
 

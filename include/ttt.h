@@ -284,7 +284,9 @@ typedef enum {
 ttt_status ttt_state_set_option(ttt_state* st, int32_t option, int64_t value);
 
 /* Synchronise the device and return the first device-side failure recorded since the
- * last poll (TTT_ERR_TIMEOUT or TTT_ERR_DEVICE), or TTT_OK; clears the record. */
+ * last poll (TTT_ERR_TIMEOUT or TTT_ERR_DEVICE), or TTT_OK; clears the record. For a timeout,
+ * ttt_last_error_string() names the wait that ran out: an mbarrier (by its shared-memory
+ * offset in the kernel's layout) or a progress counter (by the low bits of its address). */
 ttt_status ttt_state_poll(ttt_state* st);
 
 /* Number of kernels this state has launched since creation. */
