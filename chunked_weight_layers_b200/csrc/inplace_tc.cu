@@ -32,7 +32,9 @@
 //    into one of two TMEM accumulators, warps 2..9 drain the other accumulator
 //    (tcgen05.ld 32x32b) in the epilogue, two warps per TMEM lane quarter, and warp 10
 //    streams the fp32 W of UPDATE tiles by TMA into a 3-slot ring of 128x32 sub-tiles while
-//    the mainloop runs. The epilogue adds η·ΔW in shared memory, writes the bf16 copy beside
+//    the mainloop runs; warp 11 waits on the progress counters of the tiles ahead (up to
+//    four), so the loads of a tile whose inputs are ready start without a round trip to L2.
+//    The epilogue adds η·ΔW in shared memory, writes the bf16 copy beside
 //    it, and two TMA stores per sub-tile write both back: the read-modify-write of the 99.6 MB
 //    state never goes through per-thread global loads.
 //  * SM pairs: where the chunk and d_model are multiples of 256 the kernel runs as clusters
@@ -73,7 +75,9 @@ constexpr int kShBytes = BM * kWCols * 2;   // 8 KB of its bf16 copy
 constexpr int kWSlots = 3;                  // W sub-tile ring depth
 constexpr int kEpiWarps = 8;
 constexpr int kWarpWload = 2 + kEpiWarps;   // the warp that streams W sub-tiles in
-constexpr int kThreadsTC = (3 + kEpiWarps) * 32;
+constexpr int kWarpDeps = 3 + kEpiWarps;    // the warp that waits for other CTAs' progress
+constexpr int kThreadsTC = (4 + kEpiWarps) * 32;
+constexpr int kDepSlots = 4;                // tiles whose dependencies may be cleared ahead of the loads
 constexpr int kTmemCols = 512;
 
 enum : int { APPLY = 0, UPDATE = 1, TARGET = 2 };
@@ -91,6 +95,7 @@ struct __align__(1024) TCSmem {
   uint64_t full[kStMax], empty[kStMax];
   uint64_t tfull[2], tempty[2];
   uint64_t wfull[kWSlots], wempty[kWSlots];
+  uint64_t dep_ok[kDepSlots], dep_free[kDepSlots];
   uint32_t tmem_base;
   int abort;
   int eflag[2][2];  // per column half: a wait of sub-tile e ran out (index e & 1)
@@ -397,6 +402,10 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       mbar_init(&sm.wfull[i], 1);
       mbar_init(&sm.wempty[i], 1);
     }
+    for (int i = 0; i < kDepSlots; ++i) {
+      mbar_init(&sm.dep_ok[i], 1);
+      mbar_init(&sm.dep_free[i], 1);
+    }
     sm.abort = 0;
     sm.eflag[0][0] = sm.eflag[0][1] = sm.eflag[1][0] = sm.eflag[1][1] = 0;
     sm.tflag[0][0] = sm.tflag[0][1] = sm.tflag[1][0] = sm.tflag[1][1] = 0;
@@ -417,34 +426,22 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       tma_prefetch_desc(&tmZm);
       tma_prefetch_desc(&tmVm);
       tma_prefetch_desc(&tmWk0);
-      uint32_t it = 0;
+      uint32_t it = 0, dep_u = 0;
       for_tiles([&](int rnd, int32_t tc) -> bool {
         if (*abort) return false;
         const int type = tile_type(tc), m = tile_m(tc), n = tile_n(tc);
         const int nk = kblocks(type, args);
         const int chunk = args.chunk + rnd;
-        const int r0 = row0_of(m), wb = wblock_of(m);
+        const int r0 = row0_of(m);
         const int b0 = n * BN + rank * (BN / 2);  // first B column (N) this CTA loads
         const CUtensorMap* wk = pick3(tmWk0, tmWk1, tmWk2, (args.cur0 + rnd) % 3);
         if (args.upd_done != nullptr) {
-          if (type == APPLY && rnd >= 1 &&
-              !wait_counter(&args.upd_done[(rnd - 1) * args.nbd + n],
-                            upd_expect(args, n) + (rnd == args.stall_round ? 1 : 0), args.status, abort))
-            return false;
-          if (type == UPDATE && rnd >= 2 &&
-              !wait_counter(&args.app_done[(rnd - 2) * args.nbd + wb], args.C / BM, args.status, abort))
-            return false;
-          if (args.tgt_done != nullptr) {
-            // V̂ of this round was produced by the previous round's TARGET tiles; a TARGET tile
-            // overwrites the V̂ buffer the previous round's UPDATE tiles of its block read.
-            if (type == UPDATE && rnd >= 1 &&
-                !wait_counter(&args.tgt_done[(rnd - 1) * args.nbd + wb], kEpiWarps * (args.C / BM), args.status,
-                              abort))
-              return false;
-            if (type == TARGET && rnd >= 2 &&
-                !wait_counter(&args.upd_done[(rnd - 2) * args.nbd + n], upd_expect(args, n), args.status, abort))
-              return false;
-          }
+          // The dependency warp has seen this tile's inputs published by other CTAs.
+          const int slot = (int)(dep_u % kDepSlots);
+          if (!mbar_wait(&sm.dep_ok[slot], (dep_u / kDepSlots) & 1, args.status, abort)) return false;
+          fence_proxy_async_global();  // TMA reads after that point see what the counters published
+          mbar_arrive(&sm.dep_free[slot]);
+          ++dep_u;
         }
         const CUtensorMap* vm = args.tgt_done != nullptr ? pick3(tmVm, tmVm1, tmVm2, rnd % 3) : &tmVm;
         for (int kb = 0; kb < nk; ++kb, ++it) {
@@ -492,6 +489,45 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         const uint64_t t0 = globaltimer();
         while (globaltimer() - t0 < 50000) __nanosleep(1000);
       }
+    }
+  } else if (warp == kWarpDeps) {
+    // ------------- dependencies: waits on other CTAs' progress, ahead of the loads -------------
+    // A counter read is an L2 round trip and its fences more; measured on B200, taken in the
+    // producer's path they held up the first k-blocks of every UPDATE tile. Here they run up
+    // to kDepSlots tiles ahead, and the producer only waits on a shared-memory barrier.
+    if (lane == 0 && args.upd_done != nullptr) {
+      uint32_t u = 0;
+      for_tiles([&](int rnd, int32_t tc) -> bool {
+        if (*abort) return false;
+        const int type = tile_type(tc), m = tile_m(tc), n = tile_n(tc);
+        const int wb = wblock_of(m);
+        const int slot = (int)(u % kDepSlots);
+        if (u >= (uint32_t)kDepSlots && !mbar_wait(&sm.dep_free[slot], ((u / kDepSlots) - 1) & 1, args.status, abort))
+          return false;
+        {
+          if (type == APPLY && rnd >= 1 &&
+              !wait_counter(&args.upd_done[(rnd - 1) * args.nbd + n],
+                            upd_expect(args, n) + (rnd == args.stall_round ? 1 : 0), args.status, abort))
+            return false;
+          if (type == UPDATE && rnd >= 2 &&
+              !wait_counter(&args.app_done[(rnd - 2) * args.nbd + wb], args.C / BM, args.status, abort))
+            return false;
+          if (args.tgt_done != nullptr) {
+            // V̂ of this round was produced by the previous round's TARGET tiles; a TARGET tile
+            // overwrites the V̂ buffer the previous round's UPDATE tiles of its block read.
+            if (type == UPDATE && rnd >= 1 &&
+                !wait_counter(&args.tgt_done[(rnd - 1) * args.nbd + wb], kEpiWarps * (args.C / BM), args.status,
+                              abort))
+              return false;
+            if (type == TARGET && rnd >= 2 &&
+                !wait_counter(&args.upd_done[(rnd - 2) * args.nbd + n], upd_expect(args, n), args.status, abort))
+              return false;
+          }
+        }
+        mbar_arrive(&sm.dep_ok[slot]);
+        ++u;
+        return true;
+      });
     }
   } else if (warp == kWarpWload) {
     // ---------------- W sub-tile loader (fp32 W of UPDATE tiles, 128 x 32) ----------------
