@@ -475,18 +475,26 @@ constexpr int kGateRing = 4;   // tiles of losses in flight from the writer to t
 template <bool GATE>
 constexpr int b16_threads() { return (kComputeWarps + 2 + (GATE ? kGateWarps : 0)) * 32; }
 
+// Shared memory of one instantiation: arrays a variant does not use shrink to one element, and
+// the plain TTT-Linear instantiation (queries, no losses, no gate, one mini-batch a step) keeps
+// three input stages instead of four: at ~89 KB two CTAs fit on one SM, so with programmatic
+// dependent launch every CTA of the next scan is resident (waiting) before this one ends, not
+// only those that find an idle SM.
+template <bool HAS_Q, bool LOSS, bool GATE, int NB>
 struct __align__(1024) B16Smem {
-  uint8_t K[kStages][kTileBytes];
-  uint8_t V[kStages][kTileBytes];
-  uint8_t Q[kStages][kTileBytes];
+  static constexpr int kS = (HAS_Q && !LOSS && !GATE && NB == 1) ? 3 : kStages;  // input ring depth
+  static constexpr int kGm = NB > 1 ? 2 : 1;
+  uint8_t K[kS][kTileBytes];
+  uint8_t V[kS][kTileBytes];
+  uint8_t Q[kS][kTileBytes];
   uint8_t O[2][kTileBytes];
-  uint8_t gm[2][kMaxTilePairs][kPairBytes];  // chunked form: Gram blocks of tiles t (t & 1)
+  uint8_t gm[kGm][NB > 1 ? kMaxTilePairs : 1][kPairBytes];  // chunked form: Gram blocks of tiles t (t & 1)
   // Per-lane loss partials of tile t (t & 1): [compute warp][lane group g][token], each the sum
   // of the squared residuals of the warp's two columns g, g+8; the writer adds them up.
-  float lossp[2][kComputeWarps][8][kLossStride];
-  float gl[kGateRing][kTileTok];  // tiles' losses handed from the writer to the gate warps
-  uint64_t full[kStages];
-  uint64_t empty[kStages];
+  float lossp[LOSS ? 2 : 1][kComputeWarps][8][LOSS ? kLossStride : 1];
+  float gl[GATE ? kGateRing : 1][kTileTok];  // tiles' losses handed from the writer to the gate warps
+  uint64_t full[kS];
+  uint64_t empty[kS];
   uint64_t oready[2];
   uint64_t ofree[2];
   uint64_t gmready[2];  // chunked form: the Gram blocks of a tile are complete (all compute lanes)
@@ -548,7 +556,11 @@ __global__ void __launch_bounds__(b16_threads<true>(), 1)
                  const GateArgs ga, int stall_tile) {
   static_assert(!GATE || LOSS, "the gate reads the losses");
   extern __shared__ uint8_t smem_raw[];
-  B16Smem& sm = *reinterpret_cast<B16Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  using Smem = B16Smem<HAS_Q, LOSS, GATE, NB>;
+  constexpr int kStages = Smem::kS;  // shadows the file-wide depth inside this kernel
+  Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // Loss partials of tile t for this warp (null without losses: the helpers then never use it).
+  auto lossp_of = [&](int t, int w) -> float* { return LOSS ? &sm.lossp[t & 1][w][0][0] : nullptr; };
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bh = blockIdx.x;
   const int ntiles = (T + kTileTok - 1) / kTileTok;
@@ -579,26 +591,13 @@ __global__ void __launch_bounds__(b16_threads<true>(), 1)
     sm.gate_turn = 0;
     fence_barrier_init();
   }
+  __syncthreads();  // the barriers exist for every warp
   // Wait for the kernel before this one (a no-op without programmatic dependent launch), then
   // let the next one start its own set-up: it waits in turn before reading what this one writes.
+  // After the wait each role starts at once: the producer's first loads are in flight while the
+  // compute warps read their slice of W.
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;");
-  // The compute warps' slice of W, in accumulator layout (warp w owns columns 16w .. 16w+15):
-  // acc[nt][e] = W[8nt + 2q + (e&1)][16w + g + 8(e>>1)].
-  float acc[8][4];
-  if (warp < kComputeWarps) {
-    const int g = lane >> 2, q = lane & 3, col0 = 16 * warp;
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[nt][e] = Wg[(8 * nt + 2 * q + (e & 1)) * 64 + col0 + g + 8 * (e >> 1)];
-  }
-  if (GATE && threadIdx.x == 0) {
-    sm.g_tau = ga.tau[bh];
-    sm.g_tau_set = ga.tau_set[bh];
-    sm.g_routed = ga.counts[2 * bh];
-  }
-  __syncthreads();
 
   if (warp == kComputeWarps) {
     // ---------------- producer: TMA loads of K, V (and Q) tiles ----------------
@@ -639,7 +638,7 @@ __global__ void __launch_bounds__(b16_threads<true>(), 1)
           float w[kComputeWarps];
 #pragma unroll
           for (int cw = 0; cw < kComputeWarps; ++cw) {
-            const float* x = &sm.lossp[b][cw][0][i];
+            const float* x = lossp_of(b, cw) + i;
             w[cw] = ((x[0 * kLossStride] + x[1 * kLossStride]) + (x[2 * kLossStride] + x[3 * kLossStride])) +
                     ((x[4 * kLossStride] + x[5 * kLossStride]) + (x[6 * kLossStride] + x[7 * kLossStride]));
           }
@@ -685,6 +684,14 @@ __global__ void __launch_bounds__(b16_threads<true>(), 1)
     const int w = warp - (kComputeWarps + 2);
     const int seq = bh / ga.heads, head = bh % ga.heads;
     int32_t* E = ga.entries + (size_t)bh * ga.capacity * 3;
+    // The gate's carried state, read by gate warp 0 before its first tile; the other gate warps
+    // read it only after gate_turn has passed through warp 0 (which fences its writes).
+    if (w == 0 && lane == 0) {
+      sm.g_tau = ga.tau[bh];
+      sm.g_tau_set = ga.tau_set[bh];
+      sm.g_routed = ga.counts[2 * bh];
+    }
+    __syncwarp();
     for (int t = w; t < ntiles; t += kGateWarps) {
       const int r = t % kGateRing;
       if (!warp_wait(&sm.gready[r], (t / kGateRing) & 1, status, &sm.abort)) break;
@@ -742,6 +749,13 @@ __global__ void __launch_bounds__(b16_threads<true>(), 1)
   const int g = lane >> 2, q = lane & 3;
   const int col0 = 16 * warp;
   const StepOffsets offs = step_offsets(lane, col0);
+  // This warp's slice of W, in accumulator layout (warp w owns columns 16w .. 16w+15):
+  // acc[nt][e] = W[8nt + 2q + (e&1)][16w + g + 8(e>>1)].
+  float acc[8][4];
+#pragma unroll
+  for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[nt][e] = Wg[(8 * nt + 2 * q + (e & 1)) * 64 + col0 + g + 8 * (e >> 1)];
 
   if constexpr (NB > 1) {
     // ---- chunked form: chunks of NB blocks, Gram blocks one tile ahead ----
@@ -781,7 +795,7 @@ __global__ void __launch_bounds__(b16_threads<true>(), 1)
 #pragma unroll
       for (int cc = 0; cc < kCPT; ++cc)
         chunk_run<NB, HAS_Q, LOSS>(acc, kb, vb, qb, gb + (uint32_t)(cc * kPPC) * kPairBytes, ob, offs,
-                                   &sm.lossp[t & 1][warp][0][0], 16 * NB * cc, lane, beta);
+                                   lossp_of(t, warp), 16 * NB * cc, lane, beta);
       mbar_arrive(&sm.empty[slot]);  // every fragment of tile t has been read
       // Tile t's Gram blocks have all been read by this warp: its share of tile t+1's may go into
       // the other buffer (every warp passed the top of tile t, so none still reads tile t − 1's).
@@ -799,7 +813,7 @@ __global__ void __launch_bounds__(b16_threads<true>(), 1)
         const int slot = t % kStages;
         const uint32_t kb = smem_u32(sm.K[slot]), vb = smem_u32(sm.V[slot]), qb = smem_u32(sm.Q[slot]);
         const uint32_t gb = (t & 1) ? gm1 : gm0, ob = smem_u32(sm.O[t & 1]);
-        float* lp = &sm.lossp[t & 1][warp][0][0];
+        float* lp = lossp_of(t, warp);
         if (NB == 2) {
           if (rem >= 2) chunk_run<2, HAS_Q, LOSS>(acc, kb, vb, qb, gb, ob, offs, lp, 0, lane, beta);
           if (rem != 2) chunk_run<1, HAS_Q, LOSS>(acc, kb, vb, qb, gb, ob, offs, lp, rem == 1 ? 0 : 32, lane, beta);
@@ -830,7 +844,7 @@ __global__ void __launch_bounds__(b16_threads<true>(), 1)
     load_frag16<HAS_Q>(F, smem_u32(sm.K[slot]), smem_u32(sm.V[slot]), smem_u32(sm.Q[slot]), offs, 16 * s);
   };
   auto comp = [&](const Frag16& F, int t, int s) {
-    compute16<HAS_Q, LOSS>(acc, F, smem_u32(sm.O[t & 1]), offs.o, &sm.lossp[t & 1][warp][0][0], 16 * s, lane, beta);
+    compute16<HAS_Q, LOSS>(acc, F, smem_u32(sm.O[t & 1]), offs.o, lossp_of(t, warp), 16 * s, lane, beta);
   };
 
   const int nfull = T / kTileTok, rem = (T % kTileTok) / 16;
@@ -1128,12 +1142,16 @@ ttt_status launch(ttt_state* st, const CUtensorMap& tk, const CUtensorMap& tv, c
 template <bool HAS_Q, bool LOSS, bool GATE, int NB>
 ttt_status launch_b16_nb(ttt_state* st, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
                          const CUtensorMap& to, float* loss, int T, const GateArgs& ga, cudaStream_t s) {
-  const size_t smem = sizeof(B16Smem) + 1024;
+  const size_t smem = sizeof(B16Smem<HAS_Q, LOSS, GATE, NB>) + 1024;
   // One bit per instantiation whose shared-memory limit has been raised on this state's device.
   const uint64_t bit = 1ull << (16 + 8 * (NB == 1 ? 0 : NB == 2 ? 1 : 2) + 4 * GATE + 2 * HAS_Q + LOSS);
   if (!(st->lin.smem_set & bit)) {
     TTT_CUDA(cudaFuncSetAttribute(k_linear_b16<HAS_Q, LOSS, GATE, NB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)smem));
+    // All of the SM's unified L1/shared memory as shared memory, so that two CTAs of the small
+    // instantiation fit on one SM.
+    TTT_CUDA(cudaFuncSetAttribute(k_linear_b16<HAS_Q, LOSS, GATE, NB>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                  (int)cudaSharedmemCarveoutMaxShared));
     st->lin.smem_set |= bit;
   }
   const int grid = st->cfg.batch * st->cfg.heads;
