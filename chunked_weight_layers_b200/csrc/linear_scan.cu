@@ -476,13 +476,13 @@ template <bool GATE>
 constexpr int b16_threads() { return (kComputeWarps + 2 + (GATE ? kGateWarps : 0)) * 32; }
 
 // Shared memory of one instantiation: arrays a variant does not use shrink to one element, and
-// the plain TTT-Linear instantiation (queries, no losses, no gate, one mini-batch a step) keeps
+// the plain TTT-Linear instantiations (no losses, no gate, one mini-batch a step) keep
 // three input stages instead of four: at ~89 KB two CTAs fit on one SM, so with programmatic
 // dependent launch every CTA of the next scan is resident (waiting) before this one ends, not
 // only those that find an idle SM.
 template <bool HAS_Q, bool LOSS, bool GATE, int NB>
 struct __align__(1024) B16Smem {
-  static constexpr int kS = (HAS_Q && !LOSS && !GATE && NB == 1) ? 3 : kStages;  // input ring depth
+  static constexpr int kS = (!LOSS && !GATE && NB == 1) ? 3 : kStages;  // input ring depth
   static constexpr int kGm = NB > 1 ? 2 : 1;
   uint8_t K[kS][kTileBytes];
   uint8_t V[kS][kTileBytes];
