@@ -177,6 +177,20 @@ __device__ __forceinline__ void compute16(float (&acc)[8][4], const Frag16& F, u
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
       mma16816(pp[nt][ks & 1], wa[ks], F.kb[nt][ks >> 1][2 * (ks & 1)], F.kb[nt][ks >> 1][2 * (ks & 1) + 1]);
+  // The first half of the output products goes into the P products' latency; the second half
+  // follows the update, into its latency (both halves are off the dependent chain).
+  float o[2][2][4];
+  if (HAS_Q) {
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[nt][0][e] = o[nt][1][e] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < 2; ++ks)
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+        mma16816(o[nt][ks & 1], wa[ks], F.qb[nt][ks >> 1][2 * (ks & 1)], F.qb[nt][ks >> 1][2 * (ks & 1) + 1]);
+  }
 
   // R = P − V: p[nt][e] is R[token 8nt + 2q + (e&1)][column col0 + g + 8(e>>1)].
   float p[2][4];
@@ -201,13 +215,8 @@ __device__ __forceinline__ void compute16(float (&acc)[8][4], const Frag16& F, u
   }
 
   if (HAS_Q) {
-    float o[2][2][4];
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) o[nt][0][e] = o[nt][1][e] = 0.f;
-#pragma unroll
-    for (int ks = 0; ks < 4; ++ks)
+    for (int ks = 2; ks < 4; ++ks)
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt)
         mma16816(o[nt][ks & 1], wa[ks], F.qb[nt][ks >> 1][2 * (ks & 1)], F.qb[nt][ks >> 1][2 * (ks & 1) + 1]);
