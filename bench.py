@@ -486,6 +486,90 @@ def measure_cache_read(steps, warmup, peaks, device):
     return out
 
 
+DOCS = wl.INPLACE_4B.name + " packed (7 documents, clipped)"
+DOCS_SEED, DOCS_N, DOCS_CLIP = 1006, 7, 1.0
+
+
+def measure_docs(steps, warmup, peaks, device):
+    """ttt_chunk_scan_docs on the 4B-class widths: T=32768 tokens as seven documents of seeded
+    ragged lengths, every chunk delta clipped to Frobenius norm 1.0. Work counts the real tokens
+    only (the padding that fills each document's last chunk is overhead)."""
+    import chunked_weight_layers_b200 as cwl
+    spec = wl.INPLACE_4B
+    starts = wl.document_starts(spec.T, DOCS_N, DOCS_SEED)
+    x = wl.inplace_inputs(spec, device=device)
+    cfg = cwl.config("inplace", io_dtype=1, d_key=spec.f, d_val=spec.d, chunk=spec.C, eta=spec.eta)
+    st = cwl.FastWeightState(cfg, x["W0"])
+    O = torch.empty((spec.T, spec.d), device=device, dtype=torch.bfloat16)
+    w = work(spec)
+    for _ in range(warmup):
+        st.chunk_scan_docs(x["Z"], x["Vhat"], starts, clip=DOCS_CLIP, out=O)
+    torch.cuda.synchronize()
+    n0 = st.launch_count()
+    stream = torch.cuda.current_stream()
+    times = []
+    for _ in range(steps):  # the call synchronises (its layout goes up from host memory): time each
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        st.chunk_scan_docs(x["Z"], x["Vhat"], starts, clip=DOCS_CLIP, out=O)
+        e1.record(stream)
+        e1.synchronize()
+        times.append(e0.elapsed_time(e1))
+    st.poll()
+    launches = (st.launch_count() - n0) / steps
+    ms = sum(times) / steps
+    tf = w["flops"] / (ms * 1e-3) / 1e12
+    # End to end: the inputs from pinned host memory, the call, the outputs back.
+    hz, hv = x["Z"].cpu().pin_memory(), x["Vhat"].cpu().pin_memory()
+    ho = torch.empty((spec.T, spec.d), dtype=torch.bfloat16).pin_memory()
+    dz, dv = torch.empty_like(x["Z"]), torch.empty_like(x["Vhat"])
+    e2e = []
+    for k in range(3):
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        dz.copy_(hz, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        st.chunk_scan_docs(dz, dv, starts, clip=DOCS_CLIP, out=O)
+        ho.copy_(O, non_blocking=True)
+        torch.cuda.synchronize()
+        e2e.append((time.perf_counter() - t0) * 1e3)
+    e2e_ms = statistics.median(e2e)
+    out = {"workload": DOCS, "doc_starts": starts, "clip_norm": DOCS_CLIP, "ms_per_step": ms,
+           "ms_median": statistics.median(times), "tokens_per_s": w["tokens"] / (ms * 1e-3), "tflops": tf,
+           "roofline": {"bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                        "frac": tf / peaks["bf16_tflops"], "traffic": None, "peak_source": peaks["source"],
+                        "kernel": "k_gemm_tc",
+                        "peak_kind": "burst (each call timed alone: it synchronises to upload its layout)"},
+           "gpu_launches_per_step": launches, "times_ms": times,
+           "l2": "inputs larger than L2 (the 4B-class Z alone is 637 MB)",
+           "e2e": {"value": w["tokens"] / (e2e_ms * 1e-3), "unit": "tokens/s",
+                   "h2d_bytes_per_step": hz.numel() * 2 + hv.numel() * 2, "d2h_bytes_per_step": ho.numel() * 2,
+                   "ms_per_step": e2e_ms}}
+    st.close()
+    del x, O, dz, dv
+    torch.cuda.empty_cache()
+    return out
+
+
+def cpu_baseline_docs(limit_s) -> dict:
+    """The oracle's packed scan (resets and clipping) on the first chunks of the measured
+    layout's first document, within the time limit."""
+    from oracle import packed as opk
+    spec = wl.INPLACE_4B
+    x = wl.inplace_inputs(wl.scaled(spec, T=spec.C * 2))
+    cores = oracle_threads()
+    t0, c0 = time.perf_counter(), time.process_time()
+    chunks = 0
+    while time.perf_counter() - t0 < limit_s and chunks < 2:
+        sl = slice(chunks * spec.C, (chunks + 1) * spec.C)
+        opk.inplace_scan_docs(x["Z"][sl], x["Vhat"][sl], x["W0"], spec.eta, spec.C, [0], DOCS_CLIP)
+        chunks += 1
+    dt = time.perf_counter() - t0
+    busy = (time.process_time() - c0) / dt if dt > 0 else 0.0
+    return {"value": chunks * spec.C / dt, "unit": "tokens/s", "cores": cores, "busy_threads": round(busy, 2),
+            "kind": "oracle", "sample": f"{chunks} chunk(s) of {spec.C} tokens (one document, clipped)", "seconds": dt}
+
+
 def cpu_baseline_cache_read(limit_s) -> dict:
     """The oracle's read path (attention over the visible entries, α fusion) on (sequence, head)
     pairs of the gate workload's cache, one at a time, within the time limit."""
@@ -760,6 +844,10 @@ def main():
             extra[CACHE_READ] = measure_cache_read(max(5, min(a.steps, 20)), 3, peaks, device)
         except Exception as ex:
             extra[CACHE_READ] = {"error": str(ex)}
+        try:
+            extra[DOCS] = measure_docs(max(3, min(a.steps, 5)), 2, peaks, device)
+        except Exception as ex:
+            extra[DOCS] = {"error": str(ex)}
     clk.__exit__(None, None, None)
     # The oracle baselines run after the sampler stops (the GPU idles meanwhile).
     for s in wl.WORKLOADS.values():
@@ -770,6 +858,8 @@ def main():
                                                                                                prefix=True)
     if "error" not in extra.get(CACHE_READ, {"error": 1}):
         extra[CACHE_READ]["cpu_baseline"] = cpu_baseline_cache_read(6.0)
+    if "error" not in extra.get(DOCS, {"error": 1}):
+        extra[DOCS]["cpu_baseline"] = cpu_baseline_docs(6.0)
 
     if rank == 0:
         rl = roofline(spec, w, ms, peaks, traffic_per_launch(spec), timed_ms=total_ms)

@@ -135,6 +135,22 @@ class FastWeightState:
         check(self._lib.ttt_chunk_scan_host(self._h, *self._scan_args(keys, targets, queries, out, loss_out, T,
                                                                       None), _stream(stream)))
 
+    def chunk_scan_docs(self, keys, targets, doc_starts, clip=None, out=None, T=None, stream=None):
+        """ttt_chunk_scan_docs (In-Place BF16 states with given targets): documents laid end to
+        end, ``doc_starts`` their first tokens (a sequence of ints, 0 first), each scanned from
+        the pretrained weight; ``clip`` the Frobenius norm each chunk delta is clipped to (None:
+        no clipping). Synchronises the stream (the layout goes up from host memory)."""
+        import ctypes
+        if T is None:
+            T = keys.shape[-2]
+        starts = (ctypes.c_int64 * len(doc_starts))(*[int(a) for a in doc_starts])
+        dev = _current_device()
+        check(self._lib.ttt_chunk_scan_docs(self._h, _arg(keys, "keys", self._io, T * self._dk, dev),
+                                            _arg(targets, "targets", self._io, T * self._dv, dev), int(T),
+                                            _arg(out, "out", self._io, T * self._dv, dev),
+                                            ctypes.cast(starts, ctypes.c_void_p), len(doc_starts),
+                                            float(clip or 0.0), _stream(stream)))
+
     def surprisal_route(self, loss, T=None, stream=None):
         if T is None:
             T = loss.shape[-1]

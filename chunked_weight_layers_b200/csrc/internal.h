@@ -61,6 +61,17 @@ struct InplaceBuffers {
   float* prefix_D = nullptr;
   __nv_bfloat16* prefix_Wb = nullptr;
   int prefix_chunks = 0;
+  // Packed sequences (ttt_chunk_scan_docs): Z, V̂ and O with every document padded to whole
+  // chunks, the padded row → input row map (−1: padding), the first-chunk-of-a-document flags
+  // and the chunk deltas' squared Frobenius norms, grown on demand.
+  __nv_bfloat16* docs_Z = nullptr;
+  __nv_bfloat16* docs_V = nullptr;
+  __nv_bfloat16* docs_O = nullptr;
+  int32_t* docs_rows = nullptr;
+  int32_t* docs_reset = nullptr;
+  double* docs_sumsq = nullptr;
+  int64_t docs_rows_cap = 0;
+  int docs_chunks_cap = 0;
 };
 
 // Tensor maps of one scan's K, V, Q, O (encoding them costs microseconds of host time, so the
@@ -136,6 +147,13 @@ ttt_status inplace_bf16_scan(ttt_state* st, const __nv_bfloat16* Z, const __nv_b
 // sums, then all chunk outputs (three launches, no cross-chunk waits).
 ttt_status inplace_bf16_scan_prefix(ttt_state* st, const __nv_bfloat16* Z, const __nv_bfloat16* Vhat, int64_t T,
                                     __nv_bfloat16* O, cudaStream_t s);
+
+// In-Place, bf16, packed sequences: documents laid end to end, each scanned from the
+// pretrained weight with its own chunks (a shorter last one), each chunk's delta clipped to
+// Frobenius norm `clip` when clip > 0. Context-parallel machinery; doc_starts is host memory.
+ttt_status inplace_bf16_scan_docs(ttt_state* st, const __nv_bfloat16* Z, const __nv_bfloat16* Vhat, int64_t T,
+                                  const int64_t* doc_starts, int ndocs, float clip, __nv_bfloat16* O,
+                                  cudaStream_t s);
 
 // Frees the tensor-core resources of a state (no-op if none were built).
 void free_tc(ttt_state* st);

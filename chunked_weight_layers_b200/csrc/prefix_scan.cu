@@ -17,6 +17,8 @@
 // output tile, TMA loads (128-byte swizzle) into a 3-stage ring, one thread issuing
 // tcgen05.mma (M=128, N=256, K=16) into a TMEM accumulator, four epilogue warps (one per TMEM
 // lane quarter) scaling and storing rows. Operands are K-major or MN-major as stored.
+#include <vector>
+
 #include "internal.h"
 #include "tc_common.cuh"
 
@@ -183,29 +185,89 @@ __global__ void __launch_bounds__(kGThreads, 1)
   if (warp == 1) tc::dealloc(tmem, kGTmemCols);
 }
 
-// W_j (bf16) = W_0 + Σ_{i<j} D_i for j = 0 .. n−1, then W ← W_0 + Σ_i D_i (fp32) and its bf16
-// copy. Four consecutive elements a thread; the sum over the chunks runs in chunk order.
+// W_j (bf16) = W_0 + Σ_{i<j} s_i·D_i for j = 0 .. n−1, then W ← W_0 + Σ_i s_i·D_i (fp32) and
+// its bf16 copy. Four consecutive elements a thread; the sum over the chunks runs in chunk
+// order. Packed sequences: where reset[j] is set the sum restarts from Wreset (a document's
+// first chunk), and with sumsq given s_i = clip / ‖D_i‖_F when that norm exceeds clip (else
+// 1, as without sumsq: the plain form's sums are bit for bit those of W + D).
 __global__ void k_prefix_w(const float* W0, const float* __restrict__ D, __nv_bfloat16* __restrict__ Wb, float* Wout,
-                           __nv_bfloat16* __restrict__ Wcopy, long long nelem, int n) {
+                           __nv_bfloat16* __restrict__ Wcopy, long long nelem, int n, const int32_t* __restrict__ reset,
+                           const float* __restrict__ Wreset, const double* __restrict__ sumsq, float clip) {
   const long long n4 = nelem / 4;
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (long long)gridDim.x * blockDim.x) {
     float4 acc = reinterpret_cast<const float4*>(W0)[i];
     for (int j = 0; j < n; ++j) {
+      if (reset != nullptr && reset[j]) acc = reinterpret_cast<const float4*>(Wreset)[i];
       uint2 w;
       w.x = pack_bf16(acc.x, acc.y);
       w.y = pack_bf16(acc.z, acc.w);
       reinterpret_cast<uint2*>(Wb + (long long)j * nelem)[i] = w;
+      float sc = 1.0f;
+      if (sumsq != nullptr) {
+        const double nrm = sqrt(sumsq[j]);
+        if (nrm > (double)clip) sc = (float)((double)clip / nrm);
+      }
       const float4 dj = reinterpret_cast<const float4*>(D + (long long)j * nelem)[i];
-      acc.x += dj.x;
-      acc.y += dj.y;
-      acc.z += dj.z;
-      acc.w += dj.w;
+      acc.x = fmaf(sc, dj.x, acc.x);
+      acc.y = fmaf(sc, dj.y, acc.y);
+      acc.z = fmaf(sc, dj.z, acc.z);
+      acc.w = fmaf(sc, dj.w, acc.w);
     }
     reinterpret_cast<float4*>(Wout)[i] = acc;
     uint2 w;
     w.x = pack_bf16(acc.x, acc.y);
     w.y = pack_bf16(acc.z, acc.w);
     reinterpret_cast<uint2*>(Wcopy)[i] = w;
+  }
+}
+
+// Row r of the padded layout (`width` bf16 elements, a multiple of 8) ← row rows[r] of the input,
+// or zeros where rows[r] < 0 (the padding that fills a document's last chunk).
+__global__ void k_gather_rows(const __nv_bfloat16* __restrict__ src, __nv_bfloat16* __restrict__ dst,
+                              const int32_t* __restrict__ rows, long long nrows, int width) {
+  const int v = width / 8;  // 16-byte vectors a row
+  const long long n = nrows * v;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const long long r = i / v;
+    const int c = (int)(i % v);
+    const int32_t from = rows[r];
+    uint4 x = make_uint4(0u, 0u, 0u, 0u);
+    if (from >= 0) x = reinterpret_cast<const uint4*>(src + (long long)from * width)[c];
+    reinterpret_cast<uint4*>(dst + r * width)[c] = x;
+  }
+}
+
+// Row rows[r] of the output ← row r of the padded layout, for every r that is not padding.
+__global__ void k_scatter_rows(const __nv_bfloat16* __restrict__ src, __nv_bfloat16* __restrict__ dst,
+                               const int32_t* __restrict__ rows, long long nrows, int width) {
+  const int v = width / 8;
+  const long long n = nrows * v;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const long long r = i / v;
+    const int32_t to = rows[r];
+    if (to >= 0) reinterpret_cast<uint4*>(dst + (long long)to * width)[i % v] = reinterpret_cast<const uint4*>(src + r * width)[i % v];
+  }
+}
+
+// sumsq[j] += Σ D_j² over this block's share of chunk j (blockIdx.y), float partials per thread,
+// a double per block.
+__global__ void k_chunk_sumsq(const float* __restrict__ D, long long nelem, double* __restrict__ sumsq) {
+  const float4* d = reinterpret_cast<const float4*>(D + (long long)blockIdx.y * nelem);
+  const long long n4 = nelem / 4;
+  float acc = 0.f;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (long long)gridDim.x * blockDim.x) {
+    const float4 x = d[i];
+    acc = fmaf(x.x, x.x, fmaf(x.y, x.y, fmaf(x.z, x.z, fmaf(x.w, x.w, acc))));
+  }
+  __shared__ double part[32];
+  double v = acc;
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = v;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t += part[w];
+    atomicAdd(&sumsq[blockIdx.y], t);
   }
 }
 
@@ -258,7 +320,8 @@ ttt_status inplace_bf16_scan_prefix(ttt_state* st, const __nv_bfloat16* Z, const
   // 2. Exclusive prefix sums: the weight each chunk applies with, and the final weight.
   const long long n4 = (long long)(nelem / 4);
   const int blocks = (int)std::min<long long>((n4 + 255) / 256, (long long)st->num_sms * 8);
-  k_prefix_w<<<blocks, 256, 0, s>>>(ip.W, ip.prefix_D, ip.prefix_Wb, ip.W, ip.Wsh[ip.cur], (long long)nelem, n);
+  k_prefix_w<<<blocks, 256, 0, s>>>(ip.W, ip.prefix_D, ip.prefix_Wb, ip.W, ip.Wsh[ip.cur], (long long)nelem, n,
+                                    nullptr, nullptr, nullptr, 0.f);
   st->launches++;
   TTT_CUDA(cudaGetLastError());
 
@@ -268,6 +331,109 @@ ttt_status inplace_bf16_scan_prefix(ttt_state* st, const __nv_bfloat16* Z, const
   TTT_TRY(map_bf16(&tW, ip.prefix_Wb, f, (uint64_t)n * d, 64, 256));
   GemmArgs gc{C, d, f, 0, 0, C, d, O, 0, (long long)C * d, d, 1.0f, ds};
   return gemm(st, tZk, tW, gc, n, s);
+}
+
+namespace {
+
+template <class T>
+ttt_status grow(T** p, size_t count) {
+  if (*p) cudaFree(*p);
+  *p = nullptr;
+  TTT_CUDA(cudaMalloc(reinterpret_cast<void**>(p), count * sizeof(T)));
+  return TTT_OK;
+}
+
+}  // namespace
+
+ttt_status inplace_bf16_scan_docs(ttt_state* st, const __nv_bfloat16* Z, const __nv_bfloat16* Vhat, int64_t T,
+                                  const int64_t* doc_starts, int ndocs, float clip, __nv_bfloat16* O,
+                                  cudaStream_t s) {
+  const ttt_config& c = st->cfg;
+  const int d = c.d_val, f = c.d_key, C = c.chunk;
+  const size_t nelem = (size_t)d * f;
+  InplaceBuffers& ip = st->ip;
+  // Padded layout: every document starts a chunk and fills its last chunk with zero rows (a
+  // zero row of Z and V̂ adds nothing to the delta, and its output row is dropped).
+  std::vector<int32_t> rows, reset;
+  for (int k = 0; k < ndocs; ++k) {
+    const int64_t a = doc_starts[k], e = k + 1 < ndocs ? doc_starts[k + 1] : T;
+    const int64_t nch = (e - a + C - 1) / C;
+    for (int64_t j = 0; j < nch; ++j) {
+      reset.push_back(j == 0 ? 1 : 0);
+      for (int r = 0; r < C; ++r) {
+        const int64_t t = a + j * C + r;
+        rows.push_back(t < e ? (int32_t)t : -1);
+      }
+    }
+  }
+  const int n = (int)reset.size();
+  const int64_t Tp = (int64_t)n * C;
+  if (Tp > (int64_t)INT32_MAX / 2) return fail(TTT_ERR_UNSUPPORTED, "padded length too large");
+  if (ip.docs_rows_cap < Tp) {
+    TTT_TRY(grow(&ip.docs_Z, (size_t)Tp * f));
+    TTT_TRY(grow(&ip.docs_V, (size_t)Tp * d));
+    TTT_TRY(grow(&ip.docs_O, (size_t)Tp * d));
+    TTT_TRY(grow(&ip.docs_rows, (size_t)Tp));
+    ip.docs_rows_cap = Tp;
+  }
+  if (ip.docs_chunks_cap < n) {
+    TTT_TRY(grow(&ip.docs_reset, (size_t)n));
+    TTT_TRY(grow(&ip.docs_sumsq, (size_t)n));
+    ip.docs_chunks_cap = n;
+  }
+  if (ip.prefix_chunks < n) {
+    if (ip.prefix_D) cudaFree(ip.prefix_D);
+    if (ip.prefix_Wb) cudaFree(ip.prefix_Wb);
+    ip.prefix_D = nullptr;
+    ip.prefix_Wb = nullptr;
+    ip.prefix_chunks = 0;
+    TTT_CUDA(cudaMalloc(reinterpret_cast<void**>(&ip.prefix_D), (size_t)n * nelem * 4));
+    TTT_CUDA(cudaMalloc(reinterpret_cast<void**>(&ip.prefix_Wb), (size_t)n * nelem * 2));
+    ip.prefix_chunks = n;
+  }
+  // The maps go up with the stream's work (pageable copies: staged by the driver before return).
+  TTT_CUDA(cudaMemcpyAsync(ip.docs_rows, rows.data(), rows.size() * sizeof(int32_t), cudaMemcpyHostToDevice, s));
+  TTT_CUDA(cudaMemcpyAsync(ip.docs_reset, reset.data(), reset.size() * sizeof(int32_t), cudaMemcpyHostToDevice, s));
+  const DevStatus ds{st->status.dev, st->wait_limit_ns, st->status.dev + 1};
+  const int gblocks = st->num_sms * 8;
+  k_gather_rows<<<gblocks, 256, 0, s>>>(Z, ip.docs_Z, ip.docs_rows, (long long)Tp, f);
+  k_gather_rows<<<gblocks, 256, 0, s>>>(Vhat, ip.docs_V, ip.docs_rows, (long long)Tp, d);
+  st->launches += 2;
+  TTT_CUDA(cudaGetLastError());
+
+  // 1. D_j = η·V̂_jᵀ·Z_j over the padded chunks.
+  CUtensorMap tV, tZm;
+  TTT_TRY(map_bf16(&tV, ip.docs_V, d, Tp, 64, 64));
+  TTT_TRY(map_bf16(&tZm, ip.docs_Z, f, Tp, 64, 64));
+  GemmArgs ga{d, f, C, 1, 1, C, C, ip.prefix_D, 1, (long long)nelem, f, c.eta, ds};
+  TTT_TRY(gemm(st, tV, tZm, ga, n, s));
+
+  // 2. Norms of the deltas (clipping), then the sums restarting at each document's first chunk.
+  if (clip > 0.f) {
+    TTT_CUDA(cudaMemsetAsync(ip.docs_sumsq, 0, (size_t)n * sizeof(double), s));
+    const long long n4 = (long long)(nelem / 4);
+    const int bx = (int)std::max<long long>(1, std::min<long long>((n4 + 255) / 256, (st->num_sms * 8 + n - 1) / n));
+    k_chunk_sumsq<<<dim3(bx, n), 256, 0, s>>>(ip.prefix_D, (long long)nelem, ip.docs_sumsq);
+    st->launches++;
+    TTT_CUDA(cudaGetLastError());
+  }
+  const long long n4 = (long long)(nelem / 4);
+  const int blocks = (int)std::min<long long>((n4 + 255) / 256, (long long)st->num_sms * 8);
+  k_prefix_w<<<blocks, 256, 0, s>>>(ip.W0, ip.prefix_D, ip.prefix_Wb, ip.W, ip.Wsh[ip.cur], (long long)nelem, n,
+                                    ip.docs_reset, ip.W0, clip > 0.f ? ip.docs_sumsq : nullptr, clip);
+  st->launches++;
+  TTT_CUDA(cudaGetLastError());
+
+  // 3. O_j = Z_j·W_jᵀ over the padded chunks, then the rows of the documents back in place.
+  CUtensorMap tZk, tW;
+  TTT_TRY(map_bf16(&tZk, ip.docs_Z, f, Tp, 64, 128));
+  TTT_TRY(map_bf16(&tW, ip.prefix_Wb, f, (uint64_t)n * d, 64, 256));
+  GemmArgs gc{C, d, f, 0, 0, C, d, ip.docs_O, 0, (long long)C * d, d, 1.0f, ds};
+  TTT_TRY(gemm(st, tZk, tW, gc, n, s));
+  k_scatter_rows<<<gblocks, 256, 0, s>>>(ip.docs_O, O, ip.docs_rows, (long long)Tp, d);
+  st->launches++;
+  TTT_CUDA(cudaGetLastError());
+  return TTT_OK;
 }
 
 }  // namespace ttt

@@ -107,6 +107,12 @@ static void free_state(ttt_state* st) {
   dev_free(st->ip.Wf32_next);
   dev_free(st->ip.prefix_D);
   dev_free(st->ip.prefix_Wb);
+  dev_free(st->ip.docs_Z);
+  dev_free(st->ip.docs_V);
+  dev_free(st->ip.docs_O);
+  dev_free(st->ip.docs_rows);
+  dev_free(st->ip.docs_reset);
+  dev_free(st->ip.docs_sumsq);
   dev_free(st->ip.Wsh[0]);
   dev_free(st->ip.Wsh[1]);
   dev_free(st->ip.Wsh[2]);
@@ -358,6 +364,30 @@ ttt_status ttt_chunk_scan(ttt_state* st, const void* keys, const void* targets, 
                           void* out, float* loss_out, ttt_stream stream) {
   if (st == nullptr) return fail(TTT_ERR_INVALID_ARG, "state is NULL");
   return scan_impl(st, keys, targets, queries, T, out, loss_out, reinterpret_cast<cudaStream_t>(stream));
+}
+
+ttt_status ttt_chunk_scan_docs(ttt_state* st, const void* keys, const void* targets, int64_t T, void* out,
+                               const int64_t* doc_starts, int32_t ndocs, float clip_norm, ttt_stream stream) {
+  if (st == nullptr) return fail(TTT_ERR_INVALID_ARG, "state is NULL");
+  const ttt_config& c = st->cfg;
+  if (c.rule != TTT_RULE_INPLACE_HEBBIAN || c.io_dtype != TTT_BF16 || c.target_mode != 0)
+    return fail(TTT_ERR_UNSUPPORTED, "packed sequences run In-Place BF16 states with given targets");
+  if (T < 0 || T > (int64_t)INT32_MAX / 4) return fail(TTT_ERR_INVALID_ARG, "T out of range");
+  if (!(clip_norm >= 0.f)) return fail(TTT_ERR_INVALID_ARG, "clip_norm must be >= 0 (0: no clipping)");
+  if (T == 0) return TTT_OK;
+  if (doc_starts == nullptr || ndocs < 1) return fail(TTT_ERR_INVALID_ARG, "doc_starts must list at least one document");
+  if (doc_starts[0] != 0) return fail(TTT_ERR_INVALID_ARG, "the first document must start at token 0");
+  for (int32_t k = 1; k < ndocs; ++k)
+    if (doc_starts[k] <= doc_starts[k - 1])
+      return fail(TTT_ERR_INVALID_ARG, "doc_starts must increase strictly (entry %d)", (int)k);
+  if (doc_starts[ndocs - 1] >= T) return fail(TTT_ERR_INVALID_ARG, "every document must start below T");
+  if (keys == nullptr || targets == nullptr || out == nullptr || !aligned16(keys) || !aligned16(targets) ||
+      !aligned16(out))
+    return fail(TTT_ERR_INVALID_ARG, "keys, targets and out must be 16-byte aligned device pointers");
+  TTT_TRY(check_device(st));
+  return inplace_bf16_scan_docs(st, static_cast<const __nv_bfloat16*>(keys), static_cast<const __nv_bfloat16*>(targets),
+                                T, doc_starts, (int)ndocs, clip_norm, static_cast<__nv_bfloat16*>(out),
+                                reinterpret_cast<cudaStream_t>(stream));
 }
 
 ttt_status ttt_chunk_scan_host(ttt_state* st, const void* keys, const void* targets, const void* queries,

@@ -79,6 +79,20 @@ SR_TTT_GATE = LinearSpec("srttt_gate_B4_H16_T8192_b16", B=4, H=16, T=8192, b=16,
 WORKLOADS = {w.name: w for w in (INPLACE_FP32, LINEAR_GD, INPLACE_4B, INPLACE_128K_TARGET, SR_TTT_GATE)}
 
 
+def document_starts(T: int, n_docs: int, seed: int, min_len: int = 64) -> list[int]:
+    """First tokens of ``n_docs`` documents packed end to end in T tokens (0 first): the n_docs − 1
+    interior boundaries are drawn uniformly without replacement from the positions that leave
+    every document at least ``min_len`` tokens (a seeded draw; lengths then vary widely and
+    almost never fall on chunk boundaries, like packed pretraining text)."""
+    g = torch.Generator().manual_seed(seed)
+    cuts = set()
+    while len(cuts) < n_docs - 1:
+        c = int(torch.randint(min_len, T - min_len + 1, (1,), generator=g))
+        if all(abs(c - o) >= min_len for o in cuts):
+            cuts.add(c)
+    return [0] + sorted(cuts)
+
+
 def scaled(spec, **changes):
     """A variant of ``spec`` with some sizes changed (parity cases at oracle-friendly sizes)."""
     return replace(spec, **changes)

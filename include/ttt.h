@@ -30,7 +30,8 @@
  *    the row-major layout stated for it. The caller owns all such buffers; the library
  *    never frees or retains them beyond the call.
  *  - All work is enqueued on `stream` (a cudaStream_t; NULL is the legacy default
- *    stream). Calls that synchronise: ttt_state_poll(), ttt_chunk_scan_host() and
+ *    stream). Calls that synchronise: ttt_state_poll(), ttt_chunk_scan_host(),
+ *    ttt_chunk_scan_docs() (it uploads the document layout from host memory) and
  *    ttt_state_destroy() always; ttt_state_create(), the first ttt_chunk_scan() of an
  *    In-Place BF16 state (it builds and uploads its tile schedules) and a scan that must
  *    grow a state-owned scratch buffer (longer T than before, or the first host call) may,
@@ -145,6 +146,24 @@ ttt_status ttt_chunk_scan(ttt_state* st, const void* keys, const void* targets,
 ttt_status ttt_chunk_scan_host(ttt_state* st, const void* keys, const void* targets,
                                const void* queries, int64_t T, void* out, float* loss_out,
                                ttt_stream stream);
+
+/* Packed sequences for In-Place BF16 states with given targets (target_mode 0): `keys` Z
+ * (device, bf16 [T, d_key]) and `targets` V̂ (device, bf16 [T, d_val]) hold documents laid end
+ * to end; `doc_starts` (HOST, int64 [ndocs]) lists each document's first token: 0 first,
+ * strictly increasing, below T. Each document is scanned as if alone: the weight starts from
+ * the pretrained W0, its chunks are counted from its first token (its last chunk may be
+ * shorter: T need not be a multiple of chunk), and with clip_norm > 0 each chunk's delta
+ * η·V̂_cᵀ·Z_c is scaled to Frobenius norm clip_norm when its norm is larger (0: no clipping).
+ * Writes `out` (device, bf16 [T, d_val]); afterwards the state holds the last document's
+ * final weight. Runs in the context-parallel form (all chunk deltas, their norms, sums that
+ * restart at each document, all outputs), with state-owned scratch for the padded layout and
+ * the deltas (grown on demand). Errors: INVALID_ARG (a malformed doc_starts, negative or NaN
+ * clip_norm, misaligned buffers), UNSUPPORTED (other states), CUDA. Defined by "In-Place
+ * Test-Time Training", §6 and the implementation notes after it (the weight goes back to its
+ * pretrained value at each independent document; the Frobenius norm of the update delta is
+ * clipped). */
+ttt_status ttt_chunk_scan_docs(ttt_state* st, const void* keys, const void* targets, int64_t T, void* out,
+                               const int64_t* doc_starts, int32_t ndocs, float clip_norm, ttt_stream stream);
 
 /* Run the surprisal gate alone on a loss array `loss` (device, fp32 [batch, heads, T]),
  * advancing the state's τ, cache and token position exactly as a gated scan would.
