@@ -19,6 +19,9 @@ pages' order, with no blocking, fusion or reordering beyond the definitions:
 * :mod:`oracle.packed` — packed sequences: the weight reset to its pretrained value at every
   document start, and the update delta's Frobenius norm clipped (In-Place Test-Time
   Training, §6 and its implementation notes).
+* :mod:`oracle.inner` — the richer inner models of a TTT layer: TTT-Linear with LayerNorm
+  and residual, and TTT-MLP (TTT layers page: its two instances, the DeltaNet remark on
+  LayerNorm and residual, and the conclusion on TTT-MLP's memory I/O).
 
 Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline leg may
 import it. The product path (the C-ABI library and its Python binding) never does;
@@ -28,4 +31,4 @@ Every function here is pinned by ``tests/test_oracle_*.py`` to closed forms,
 hand-derived worked examples (``tests/golden/``), special cases and brute force.
 """
 
-from . import cache_attention, gate, inplace, linear, packed  # noqa: F401
+from . import cache_attention, gate, inner, inplace, linear, packed  # noqa: F401

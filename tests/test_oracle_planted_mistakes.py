@@ -97,6 +97,54 @@ MUTANTS = [
      [("return dW * (clip / n) if n > clip else dW", "return dW * (clip / n) if n < clip else dW")]),
     ("packed", "short last mini-batch divided by b instead of its own size",
      [("W = W - (eta / n) * (Kd[s, h, r].T @ R)", "W = W - (eta / b) * (Kd[s, h, r].T @ R)")]),
+    ("inner", "LayerNorm variance divided by D - 1",
+     [("var = ((Z - mu) ** 2).mean(axis=-1, keepdims=True)",
+       "var = ((Z - mu) ** 2).sum(axis=-1, keepdims=True) / (Z.shape[-1] - 1)")]),
+    ("inner", "LayerNorm without the mean subtracted",
+     [("zhat = (Z - mu) * rstd", "zhat = Z * rstd")]),
+    ("inner", "epsilon outside the square root",
+     [("rstd = 1.0 / np.sqrt(var + eps)", "rstd = 1.0 / (np.sqrt(var) + eps)")]),
+    ("inner", "gain and bias in the wrong order",
+     [("return gamma * zhat + beta, zhat, rstd", "return gamma * (zhat + beta), zhat, rstd")]),
+    ("inner", "LayerNorm backward without the normalised-input term",
+     [(" - zhat * (g * zhat).mean(axis=-1, keepdims=True))", ")")]),
+    ("inner", "LayerNorm backward without the mean term",
+     [("(g - g.mean(axis=-1, keepdims=True) - zhat", "(g - zhat")]),
+    ("inner", "gain not applied in the backward",
+     [("    g = dY * gamma\n", "    g = dY\n")]),
+    ("inner", "residual missing from the TTT-Linear loss",
+     [("        E = Ki + Y - Vi                                    # f(k) − v\n",
+       "        E = Y - Vi\n")]),
+    ("inner", "residual missing from the outputs",
+     [("O[:, s] = Qf[:, s] + layer_norm(Qf[:, s] @ W, gam, bet, eps)[0]",
+       "O[:, s] = layer_norm(Qf[:, s] @ W, gam, bet, eps)[0]")]),
+    ("inner", "TTT-Linear step with the wrong sign",
+     [("W = W - (eta / b) * (np.swapaxes(Ki, 1, 2) @ dZ)", "W = W + (eta / b) * (np.swapaxes(Ki, 1, 2) @ dZ)")]),
+    ("inner", "TTT-Linear outputs from the weight after the step",
+     [("        if Qf is not None:\n"
+       "            O[:, s] = Qf[:, s] + layer_norm(Qf[:, s] @ W, gam, bet, eps)[0]  # f(q; W_i)\n", ""),
+      ("        W = W - (eta / b) * (np.swapaxes(Ki, 1, 2) @ dZ)   # one gradient step on ℓ_i\n",
+       "        W = W - (eta / b) * (np.swapaxes(Ki, 1, 2) @ dZ)\n"
+       "        if Qf is not None:\n"
+       "            O[:, s] = Qf[:, s] + layer_norm(Qf[:, s] @ W, gam, bet, eps)[0]\n")]),
+    ("inner", "MLP first layer's gradient taken through the updated second layer",
+     [("        dH = (dZ @ np.swapaxes(W2, 1, 2)) * act_grad(Hpre)  # back through W2 and the activation\n"
+       "        dW1 = np.swapaxes(Ki, 1, 2) @ dH\n"
+       "        W1 = W1 - (eta / b) * dW1\n"
+       "        W2 = W2 - (eta / b) * dW2\n",
+       "        W2 = W2 - (eta / b) * dW2\n"
+       "        dH = (dZ @ np.swapaxes(W2, 1, 2)) * act_grad(Hpre)\n"
+       "        dW1 = np.swapaxes(Ki, 1, 2) @ dH\n"
+       "        W1 = W1 - (eta / b) * dW1\n")]),
+    ("inner", "GELU derivative without the density term",
+     [(" + x * np.exp(-0.5 * x * x) / np.sqrt(2.0 * np.pi)", "")]),
+    ("inner", "second layer's gradient from the pre-activation",
+     [("dW2 = np.swapaxes(A, 1, 2) @ dZ", "dW2 = np.swapaxes(Hpre, 1, 2) @ dZ")]),
+    ("inner", "MLP outputs without the activation",
+     [("O[:, s] = Qf[:, s] + layer_norm(act(Qf[:, s] @ W1) @ W2, gam, bet, eps)[0]",
+       "O[:, s] = Qf[:, s] + layer_norm((Qf[:, s] @ W1) @ W2, gam, bet, eps)[0]")]),
+    ("inner", "GELU from the wrong distribution scale",
+     [("return 0.5 * x * (1.0 + erf(x / np.sqrt(2.0)))", "return 0.5 * x * (1.0 + erf(x))")]),
 ]
 
 
@@ -132,7 +180,7 @@ def _failing_pins(module: str, impl: types.ModuleType) -> list[str]:
     return failed
 
 
-@pytest.mark.parametrize("module", ["inplace", "linear", "gate", "cache_attention", "packed"])
+@pytest.mark.parametrize("module", ["inplace", "linear", "gate", "cache_attention", "packed", "inner"])
 def test_unmutated_oracle_passes_every_pin(module):
     assert _failing_pins(module, _load(module, [])) == []
 
