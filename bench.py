@@ -7,8 +7,10 @@ batch with inputs resident in HBM. The K timed steps run back to back between tw
 events (the state is reset once before the warm-up; consecutive steps continue one scan, as
 successive calls do) and take their inputs from copies whose total is over three times the
 126 MB L2, so every step reads from HBM rather than from L2. The other four workloads
-(In-Place fp32, In-Place 4B-class, In-Place 128k with fused target, SR-TTT gate) are
-measured the same way and reported under "workloads".
+(In-Place fp32, In-Place 4B-class, In-Place 128k with fused target, SR-TTT gate), the two
+richer inner models at the TTT-Linear workload's shapes (LayerNorm TTT-Linear, TTT-MLP) and
+the further forms of the path (context-parallel In-Place, the cache read path, packed
+sequences) are measured the same way and reported under "workloads".
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--workload NAME]
                   [--only-main]
@@ -56,6 +58,14 @@ def load_peaks() -> dict:
 # --------------------------------------------------------------------------------------------
 
 def work(spec) -> dict:
+    if isinstance(spec, wl.InnerSpec):
+        # K, V, Q read and O written (bf16), the weights read and written once (fp32); the MLP's
+        # algorithmic flops outweigh its bytes at the measured peaks, the LayerNorm model's do not.
+        n = spec.B * spec.H * spec.T * spec.D
+        per_head = spec.D * spec.D if spec.model == "linear_ln" else 2 * spec.D * spec.hidden
+        byts = (2 + 2 * spec.with_queries) * n * 2 + 2 * spec.B * spec.H * per_head * 4
+        return {"tokens": spec.B * spec.T, "flops": spec.flops, "bytes": byts,
+                "bound": "hbm" if spec.model == "linear_ln" else "tensor"}
     if isinstance(spec, wl.LinearSpec):
         n = spec.B * spec.H * spec.T * spec.D
         io_b = 2
@@ -100,7 +110,15 @@ class Runner:
         self.spec = spec
         self.cwl = cwl
         self.device = device
-        if isinstance(spec, wl.LinearSpec):
+        if isinstance(spec, wl.InnerSpec):
+            x = wl.inner_inputs(spec, device=device)
+            cfg = cwl.config(spec.model, batch=spec.B, heads=spec.H, eta=spec.eta, ln_eps=spec.eps)
+            self.state = cwl.FastWeightState(cfg, x["W0"])
+            self.state.set_layernorm(x["gamma"], x["beta"])
+            args = dict(keys=x["K"], targets=x["V"], queries=x.get("Q"))
+            out = torch.empty_like(x["K"]) if spec.with_queries else None
+            loss = None
+        elif isinstance(spec, wl.LinearSpec):
             x = wl.linear_inputs(spec, device=device)
             cfg = cwl.config("linear", batch=spec.B, heads=spec.H, chunk=spec.b, eta=spec.eta,
                              gate_enable=int(spec.gate))
@@ -262,6 +280,8 @@ class ClockSampler:
 
 
 def dominant_kernel(spec) -> str:
+    if isinstance(spec, wl.InnerSpec):
+        return "k_inner_ln" if spec.model == "linear_ln" else "k_inner_mlp"
     if isinstance(spec, wl.LinearSpec):
         return "k_linear_b16" if spec.b == 16 else "k_linear_scan"
     return "k_f32_chunk" if spec.dtype == "f32" else "k_inplace_tc"
@@ -334,11 +354,33 @@ def cpu_baseline(spec, limit_s=12.0, prefix=False) -> dict:
     CPU time over the sample's wall time, i.e. how many of them were busy on average."""
     import numpy as np  # noqa: F401
     from oracle import gate as ogate
+    from oracle import inner as oinn
     from oracle import inplace as oinp
     from oracle import linear as olin
     cores = oracle_threads()
     t0, c0 = time.perf_counter(), time.process_time()
-    if isinstance(spec, wl.LinearSpec):
+    if isinstance(spec, wl.InnerSpec):
+        x = wl.inner_inputs(spec)
+        BH = spec.B * spec.H
+        K, V, Q = (x[k].reshape(BH, 1, spec.T, spec.D) for k in "KVQ")
+        g, be = x["gamma"], x["beta"]
+        done_heads = 0
+        t0, c0 = time.perf_counter(), time.process_time()
+        while done_heads < BH and time.perf_counter() - t0 < limit_s:
+            h = done_heads
+            hs = slice(h, h + 1)
+            gh, bh_ = g[h % spec.H:h % spec.H + 1], be[h % spec.H:h % spec.H + 1]
+            if spec.model == "linear_ln":
+                oinn.ttt_linear_ln_scan(K[hs], V[hs], Q[hs], x["W0"].reshape(BH, 1, spec.D, spec.D)[hs], gh, bh_,
+                                        spec.eta, spec.b, spec.eps)
+            else:
+                oinn.ttt_mlp_scan(K[hs], V[hs], Q[hs], x["W1"].reshape(BH, 1, spec.D, spec.hidden)[hs],
+                                  x["W2"].reshape(BH, 1, spec.hidden, spec.D)[hs], gh, bh_, spec.eta, spec.b, spec.eps)
+            done_heads += 1
+        dt = time.perf_counter() - t0
+        tokens = spec.T * done_heads / spec.H
+        sample = f"{done_heads} of {BH} (sequence, head) scans, one at a time"
+    elif isinstance(spec, wl.LinearSpec):
         x = wl.linear_inputs(spec)
         done_heads = 0
         BH = spec.B * spec.H
@@ -690,10 +732,10 @@ def bench_config(spec, world) -> dict:
 
 
 def spec_by_name(name):
-    for s in wl.WORKLOADS.values():
+    for s in list(wl.WORKLOADS.values()) + list(wl.INNER_WORKLOADS.values()):
         if s.name == name:
             return s
-    raise SystemExit(f"unknown workload {name}; choose from {list(wl.WORKLOADS)}")
+    raise SystemExit(f"unknown workload {name}; choose from {list(wl.WORKLOADS) + list(wl.INNER_WORKLOADS)}")
 
 
 def main():
@@ -703,7 +745,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--workload", default=MAIN)
-    ap.add_argument("--only-main", action="store_true", help="skip the other four workloads")
+    ap.add_argument("--only-main", action="store_true", help="skip the other workloads")
     ap.add_argument("--tokens", type=int, default=None,
                     help="run the named workload with this many tokens instead (same widths and chunk; a smaller "
                          "case for profilers, not a bench line)")
@@ -820,12 +862,12 @@ def main():
     del runner
     torch.cuda.empty_cache()
 
-    # The other four workloads, each a full measurement of its own (device time, roofline,
+    # The other workloads, each a full measurement of its own (device time, roofline,
     # end-to-end through the host-buffer call, oracle baseline on a bounded sample). The clock
     # sampler keeps running through them, so its samples cover the whole of the GPU's work.
     extra = {}
     if not a.only_main and world == 1:
-        for s in wl.WORKLOADS.values():
+        for s in list(wl.WORKLOADS.values()) + list(wl.INNER_WORKLOADS.values()):
             if s.name == spec.name:
                 continue
             try:
@@ -850,7 +892,7 @@ def main():
             extra[DOCS] = {"error": str(ex)}
     clk.__exit__(None, None, None)
     # The oracle baselines run after the sampler stops (the GPU idles meanwhile).
-    for s in wl.WORKLOADS.values():
+    for s in list(wl.WORKLOADS.values()) + list(wl.INNER_WORKLOADS.values()):
         if s.name in extra and "error" not in extra[s.name]:
             extra[s.name]["cpu_baseline"] = cpu_baseline(s, 6.0)
     if "error" not in extra.get(wl.INPLACE_4B.name + " (context-parallel form)", {"error": 1}):

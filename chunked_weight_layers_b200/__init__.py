@@ -67,12 +67,16 @@ def _stream(stream) -> int | None:
     return stream.cuda_stream or None
 
 
+RULES = {"inplace": abi.TTT_RULE_INPLACE_HEBBIAN, "linear": abi.TTT_RULE_LINEAR_GD,
+         "linear_ln": abi.TTT_RULE_LINEAR_LN_GD, "mlp": abi.TTT_RULE_MLP_GD}
+
+
 def config(rule: str, **fields) -> abi.ttt_config:
-    """A ttt_config with the library's defaults for ``rule`` ("inplace" or "linear"), then
-    ``fields`` applied (e.g. ``d_key=512, d_val=256, chunk=512, eta=0.01, io_dtype=0``)."""
+    """A ttt_config with the library's defaults for ``rule`` ("inplace", "linear", "linear_ln"
+    or "mlp"), then ``fields`` applied (e.g. ``d_key=512, d_val=256, chunk=512, eta=0.01``)."""
     lib = abi.load()
     cfg = abi.ttt_config()
-    r = abi.TTT_RULE_INPLACE_HEBBIAN if rule == "inplace" else abi.TTT_RULE_LINEAR_GD
+    r = RULES[rule]
     check(lib.ttt_config_init(ctypes.byref(cfg), r))
     for k, v in fields.items():
         if not hasattr(cfg, k):
@@ -88,6 +92,8 @@ def _layout(cfg: abi.ttt_config):
     io = torch.float32 if cfg.io_dtype == abi.TTT_F32 else torch.bfloat16
     bh = 1 if inplace else cfg.batch * cfg.heads
     nW = cfg.d_val * cfg.d_key if inplace else bh * cfg.d_key * cfg.d_key
+    if cfg.rule == abi.TTT_RULE_MLP_GD:
+        nW = bh * 2 * 64 * 256  # W1 [64, 256] then W2 [256, 64] per (sequence, head)
     cap = cfg.cache_capacity if (not inplace and cfg.gate_enable) else 1
     return inplace, io, bh, cfg.d_key, cfg.d_val, nW, cap
 
@@ -184,6 +190,13 @@ class FastWeightState:
     def set_weights(self, W, stream=None):
         check(self._lib.ttt_state_set_weights(self._h, _arg(W, "W", torch.float32, self._nW, _current_device()),
                                               _stream(stream)))
+
+    def set_layernorm(self, gamma, beta, stream=None):
+        """ttt_state_set_layernorm: the inner model's LayerNorm gain and bias, fp32 [heads, 64]."""
+        dev = _current_device()
+        n = self.cfg.heads * 64
+        check(self._lib.ttt_state_set_layernorm(self._h, _arg(gamma, "gamma", torch.float32, n, dev),
+                                                _arg(beta, "beta", torch.float32, n, dev), _stream(stream)))
 
     def cache_read(self, entries=None, counts=None, stream=None):
         dev = _current_device()

@@ -25,6 +25,8 @@ STATUS_NAMES = {0: "TTT_OK", 1: "TTT_ERR_INVALID_ARG", 2: "TTT_ERR_UNSUPPORTED",
 
 TTT_RULE_INPLACE_HEBBIAN = 0
 TTT_RULE_LINEAR_GD = 1
+TTT_RULE_LINEAR_LN_GD = 2
+TTT_RULE_MLP_GD = 3
 TTT_F32 = 0
 TTT_BF16 = 1
 
@@ -56,6 +58,7 @@ class ttt_config(ctypes.Structure):
         ("gate_ema_new", ctypes.c_float),
         ("gate_mean_num", ctypes.c_int32),
         ("gate_mean_den", ctypes.c_int32),
+        ("ln_eps", ctypes.c_float),
     ]
 
 
@@ -72,6 +75,7 @@ _SIGNATURES = {
     "ttt_state_reset": (_st, [_vp, _vp]),
     "ttt_state_get_weights": (_st, [_vp, _vp, _vp]),
     "ttt_state_set_weights": (_st, [_vp, _vp, _vp]),
+    "ttt_state_set_layernorm": (_st, [_vp, _vp, _vp, _vp]),
     "ttt_cache_read": (_st, [_vp, _vp, _vp, _vp]),
     "ttt_gate_read": (_st, [_vp, _vp, _vp, _vp]),
     "ttt_state_set_option": (_st, [_vp, ctypes.c_int32, ctypes.c_int64]),

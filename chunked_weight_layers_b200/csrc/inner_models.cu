@@ -1,0 +1,875 @@
+// Richer TTT inner models ("テスト時学習（Test-Time Training）とは", the TTT layers page: the
+// hidden state is itself a model trained by one self-supervised step per mini-batch; its two
+// instances are TTT-Linear and TTT-MLP, and by its DeltaNet remark the full TTT-Linear carries a
+// LayerNorm and a residual connection). Per (sequence, head) and inner mini-batch i of 16 tokens,
+// with f(x) = x + LN(g(x)), LN over the head's 64 values with per-head gain γ and bias β:
+//   O_i = f(Q_i; θ_i),   E_i = f(K_i; θ_i) − V_i,   L_t = ‖E_i[t]‖²,   θ_{i+1} = θ_i − η·∇ℓ_i(θ_i)
+// with ℓ_i = 1/(2b)·‖E_i‖²; g(x) = x·W (TTT-Linear with LayerNorm and residual) or
+// g(x) = GELU(x·W1)·W2 (TTT-MLP, hidden width 256).
+//
+// Design (B200), shared with the plain TTT-Linear scan: one CTA per (sequence, head), the weights
+// in mma accumulator registers for the whole scan, every product computed transposed so each
+// accumulator layout is directly the next mma's A operand, K/V/Q streamed by a TMA producer warp
+// through a ring of 64-token tiles (128-byte swizzle), outputs staged in shared memory and written
+// by TMA stores. The per-head chain of dependent steps bounds both kernels, as it bounds the plain
+// scan; what is new is LayerNorm, whose statistics span the 64 columns that the compute warps
+// split between them:
+//  * inside a warp, the eight lanes that share a token reduce by a butterfly reduce-scatter
+//    (seven shuffles for eight sums) and an all-gather, two-pass (mean, then the squared
+//    deviations from it);
+//  * across warps, the per-warp (sum, M2) pairs meet in shared memory behind one named barrier
+//    and are merged by the parallel-variance formula, so each step has one barrier for the
+//    forward statistics and one for the backward ones (Σg and Σg·ẑ, g = γ·E).
+// The weights and the update operand S = −(η/b)·∂ℓ/∂Z reach the tensor cores as bf16 hi + lo
+// pairs (x ≈ hi + lo to ~2^-17 relative, two mma per product): LayerNorm's 1/σ and the
+// recurrence amplify operand rounding, and with single bf16 operands the outputs drift to
+// ~1e-2 of their scale over 128 steps, against ~1e-5 with the pairs (measured on the CPU
+// against float64). The weights and every accumulation stay fp32.
+#include "common.cuh"
+#include "internal.h"
+
+namespace ttt {
+
+namespace {
+
+constexpr int kStagesI = 4;                   // 64-token tiles in flight
+constexpr int kTileTokI = 64;
+constexpr int kTileBytesI = kTileTokI * 128;  // 64 tokens x 64 bf16
+constexpr int kMB = 16;                       // inner mini-batch
+
+__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void ldsm4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm4_t(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+__device__ __forceinline__ float2 bf2_to_f2(uint32_t v) {
+  return __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&v));
+}
+
+// Two fp32 values as packed bf16 hi and lo words (x ≈ hi + lo).
+__device__ __forceinline__ void hilo2(float x, float y, uint32_t& hi, uint32_t& lo) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(x, y);
+  const float2 hf = __bfloat1622float2(h);
+  hi = *reinterpret_cast<uint32_t*>(&h);
+  lo = pack_bf16(x - hf.x, y - hf.y);
+}
+
+// A fragment (hi and lo) of a 16x16 slice of an accumulator-layout matrix from its two
+// 16x8 accumulator tiles c0 (k 0..7) and c1 (k 8..15).
+__device__ __forceinline__ void afrag_hilo(const float (&c0)[4], const float (&c1)[4], uint32_t (&hi)[4],
+                                           uint32_t (&lo)[4]) {
+  hilo2(c0[0], c0[1], hi[0], lo[0]);
+  hilo2(c0[2], c0[3], hi[1], lo[1]);
+  hilo2(c1[0], c1[1], hi[2], lo[2]);
+  hilo2(c1[2], c1[3], hi[3], lo[3]);
+}
+
+template <int kWarps>
+__device__ __forceinline__ void compute_sync() {
+  asm volatile("bar.sync 1, %0;" ::"n"(kWarps * 32));
+}
+
+// Butterfly reduce-scatter over the eight lanes that share lane & 3 (lane bits 2..4 = g): each
+// lane brings eight values, and lane g leaves with the sum of value g over the eight lanes.
+__device__ __forceinline__ float reduce_scatter8(const float (&v)[8], int g) {
+  const bool b2 = g & 4, b1 = g & 2, b0 = g & 1;
+  float a[4], c[2];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) a[i] = (b2 ? v[i + 4] : v[i]) + __shfl_xor_sync(0xffffffffu, b2 ? v[i] : v[i + 4], 16);
+#pragma unroll
+  for (int i = 0; i < 2; ++i) c[i] = (b1 ? a[i + 2] : a[i]) + __shfl_xor_sync(0xffffffffu, b1 ? a[i] : a[i + 2], 8);
+  return (b0 ? c[1] : c[0]) + __shfl_xor_sync(0xffffffffu, b0 ? c[0] : c[1], 4);
+}
+
+// The inverse: lane g holds value g; every lane of the eight leaves with all eight values.
+__device__ __forceinline__ void all_gather8(float x, float (&v)[8], int g) {
+  const bool b2 = g & 4, b1 = g & 2, b0 = g & 1;
+  const float y = __shfl_xor_sync(0xffffffffu, x, 4);
+  const float c0 = b0 ? y : x, c1 = b0 ? x : y;  // values (g & 6) + 0, 1
+  const float p0 = __shfl_xor_sync(0xffffffffu, c0, 8), p1 = __shfl_xor_sync(0xffffffffu, c1, 8);
+  float a[4];  // values (g & 4) + 0..3
+  a[0] = b1 ? p0 : c0;
+  a[1] = b1 ? p1 : c1;
+  a[2] = b1 ? c0 : p0;
+  a[3] = b1 ? c1 : p1;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float p = __shfl_xor_sync(0xffffffffu, a[i], 16);
+    v[i] = b2 ? p : a[i];
+    v[i + 4] = b2 ? a[i] : p;
+  }
+}
+
+// ============================ TTT-Linear with LayerNorm and residual ============================
+
+constexpr int kLnWarps = 4;                       // compute warps: sixteen columns of W each
+constexpr int kLnThreads = (kLnWarps + 1) * 32;   // + the TMA producer warp
+
+struct __align__(1024) LnSmem {
+  uint8_t K[kStagesI][kTileBytesI];
+  uint8_t V[kStagesI][kTileBytesI];
+  uint8_t Q[kStagesI][kTileBytesI];
+  uint8_t O[2][kTileBytesI];
+  float fwd[2][kMB][8];   // [k·W or q·W][token]: per-warp sums (warps 0..3), then per-warp M2
+  float bwd[kMB][8];      // [token]: per-warp Σg, then per-warp Σg·ẑ
+  float lossp[kMB][4];    // [token]: per-warp Σe²
+  uint64_t full[kStagesI];
+  uint64_t empty[kStagesI];
+  int abort;              // set by the producer when one of its waits ran out
+  int cabort[2];          // set by a compute warp whose wait for tile s ran out (index s & 1)
+};
+
+// Per-token mean and 1/sqrt(var + ε) from four warps' (sum, M2) over sixteen columns each.
+__device__ __forceinline__ void merge_stats(const float* p, float eps, float& mu, float& rstd) {
+  const float4 S = *reinterpret_cast<const float4*>(p);
+  const float4 M = *reinterpret_cast<const float4*>(p + 4);
+  mu = ((S.x + S.y) + (S.z + S.w)) * (1.f / 64.f);
+  const float d0 = S.x * (1.f / 16.f) - mu, d1 = S.y * (1.f / 16.f) - mu;
+  const float d2 = S.z * (1.f / 16.f) - mu, d3 = S.w * (1.f / 16.f) - mu;
+  const float m2 = ((M.x + M.y) + (M.z + M.w)) + 16.f * ((d0 * d0 + d1 * d1) + (d2 * d2 + d3 * d3));
+  rstd = rsqrtf(m2 * (1.f / 64.f) + eps);
+}
+
+template <bool HAS_Q, bool LOSS>
+__global__ void __launch_bounds__(kLnThreads, 1)
+    k_inner_ln(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+               const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
+               float* __restrict__ Wstate, const float* __restrict__ gamma, const float* __restrict__ beta,
+               float* __restrict__ loss, int T, int heads, float lr, float eps, const DevStatus status) {
+  extern __shared__ uint8_t smem_raw[];
+  LnSmem& sm = *reinterpret_cast<LnSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bh = blockIdx.x;
+  const int ntiles = (T + kTileTokI - 1) / kTileTokI;
+  const uint32_t stage_bytes = (HAS_Q ? 3u : 2u) * kTileBytesI;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStagesI; ++i) {
+      mbar_init(&sm.full[i], 1);
+      mbar_init(&sm.empty[i], kLnWarps);
+    }
+    sm.abort = 0;
+    sm.cabort[0] = sm.cabort[1] = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  if (warp == kLnWarps) {
+    // ---------------- producer: TMA loads of K, V, Q tiles ----------------
+    if (lane == 0) {
+      int issued = 0;
+      for (int s = 0; s < ntiles; ++s) {
+        const int slot = s % kStagesI;
+        if (s >= kStagesI && !mbar_wait(&sm.empty[slot], ((s / kStagesI) - 1) & 1, status, &sm.abort)) break;
+        mbar_arrive_expect_tx(&sm.full[slot], stage_bytes);
+        tma_load_3d(sm.K[slot], &tmK, &sm.full[slot], 0, s * kTileTokI, bh);
+        tma_load_3d(sm.V[slot], &tmV, &sm.full[slot], 0, s * kTileTokI, bh);
+        if (HAS_Q) tma_load_3d(sm.Q[slot], &tmQ, &sm.full[slot], 0, s * kTileTokI, bh);
+        issued = s + 1;
+      }
+      // Nothing may still be landing in shared memory when the CTA exits.
+      for (int s = issued - kStagesI; s < issued; ++s) {
+        if (s < 0) continue;
+        mbar_wait(&sm.full[s % kStagesI], (s / kStagesI) & 1, status, nullptr);
+      }
+    }
+    __syncthreads();
+    return;
+  }
+
+  // ---------------- compute warps ----------------
+  const int g = lane >> 2, q = lane & 3, mi = lane >> 3, ri = lane & 7;
+  const int col0 = 16 * warp;
+  float* Wg = Wstate + (size_t)bh * 64 * 64;
+  // Wᵀ slice in accumulator layout: acc[nt][e] = W[8nt + 2q + (e&1)][col0 + g + 8(e>>1)].
+  float acc[8][4];
+#pragma unroll
+  for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[nt][e] = Wg[(8 * nt + 2 * q + (e & 1)) * 64 + col0 + g + 8 * (e >> 1)];
+  const int h = bh % heads;
+  const float gam[2] = {gamma[h * 64 + col0 + g], gamma[h * 64 + col0 + g + 8]};
+  const float bet[2] = {beta[h * 64 + col0 + g], beta[h * 64 + col0 + g + 8]};
+  // Token (within the mini-batch) whose per-warp partial this lane publishes after a
+  // reduce-scatter of values indexed 4·kind + 2·nt + jj.
+  const int pub_tok = 8 * ((g >> 1) & 1) + 2 * q + (g & 1);
+
+  for (int s = 0; s < ntiles; ++s) {
+    const int slot = s % kStagesI;
+    // Every compute warp takes the same exit decision: the flag for tile s is only written
+    // before this barrier and only read after it.
+    if (!mbar_wait(&sm.full[slot], (s / kStagesI) & 1, status, nullptr)) sm.cabort[s & 1] = 1;
+    compute_sync<kLnWarps>();
+    if (*reinterpret_cast<volatile int*>(&sm.cabort[s & 1])) break;
+    const int ntok = min(kTileTokI, T - s * kTileTokI);
+    const uint32_t kbase = smem_u32(sm.K[slot]), vbase = smem_u32(sm.V[slot]), qbase = smem_u32(sm.Q[slot]);
+    uint8_t* obuf = sm.O[s & 1];
+
+    for (int r0 = 0; r0 < ntok; r0 += kMB) {
+      // ---- forward: Zᵀ = Wᵀ·Kᵀ and (queries) Pᵀ = Wᵀ·Qᵀ, all with the weight at the step's start
+      uint32_t whi[4][4], wlo[4][4];
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks) afrag_hilo(acc[2 * ks], acc[2 * ks + 1], whi[ks], wlo[ks]);
+      float z[2][4], o[2][4];
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        float z2[4] = {0.f, 0.f, 0.f, 0.f}, o2[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) z[nt][e] = o[nt][e] = 0.f;
+#pragma unroll
+        for (int ks = 0; ks < 4; ks += 2) {
+          const uint32_t off = swz128_bf16(r0 + 8 * nt + ri, 16 * ks + 8 * mi);
+          uint32_t kb[4];
+          ldsm4(kbase + off, kb);
+          mma_bf16(z[nt], whi[ks], kb[0], kb[1]);
+          mma_bf16(z2, wlo[ks], kb[0], kb[1]);
+          mma_bf16(z[nt], whi[ks + 1], kb[2], kb[3]);
+          mma_bf16(z2, wlo[ks + 1], kb[2], kb[3]);
+          if (HAS_Q) {
+            uint32_t qb[4];
+            ldsm4(qbase + off, qb);
+            mma_bf16(o[nt], whi[ks], qb[0], qb[1]);
+            mma_bf16(o2, wlo[ks], qb[0], qb[1]);
+            mma_bf16(o[nt], whi[ks + 1], qb[2], qb[3]);
+            mma_bf16(o2, wlo[ks + 1], qb[2], qb[3]);
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          z[nt][e] += z2[e];
+          o[nt][e] += o2[e];
+        }
+      }
+      // k − v (and q) at this thread's (column, token) positions of the Zᵀ layout.
+      float kv[2][4], qv[2][4];
+      {
+        const uint32_t off = swz128_bf16(r0 + 8 * (mi >> 1) + ri, col0 + 8 * (mi & 1));
+        uint32_t kr[4], vr[4];
+        ldsm4_t(kbase + off, kr);
+        ldsm4_t(vbase + off, vr);
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          const float2 k0 = bf2_to_f2(kr[2 * nt]), k1 = bf2_to_f2(kr[2 * nt + 1]);
+          const float2 v0 = bf2_to_f2(vr[2 * nt]), v1 = bf2_to_f2(vr[2 * nt + 1]);
+          kv[nt][0] = k0.x - v0.x;
+          kv[nt][1] = k0.y - v0.y;
+          kv[nt][2] = k1.x - v1.x;
+          kv[nt][3] = k1.y - v1.y;
+        }
+        if (HAS_Q) {
+          uint32_t qr[4];
+          ldsm4_t(qbase + off, qr);
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt) {
+            const float2 a = bf2_to_f2(qr[2 * nt]), b = bf2_to_f2(qr[2 * nt + 1]);
+            qv[nt][0] = a.x;
+            qv[nt][1] = a.y;
+            qv[nt][2] = b.x;
+            qv[nt][3] = b.y;
+          }
+        }
+      }
+
+      // ---- LayerNorm statistics: per warp two-pass over its sixteen columns, then merged
+      float v8[8], all[8];
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int jj = 0; jj < 2; ++jj) {
+          v8[2 * nt + jj] = z[nt][jj] + z[nt][jj + 2];
+          v8[4 + 2 * nt + jj] = o[nt][jj] + o[nt][jj + 2];
+        }
+      const float sw = reduce_scatter8(v8, g);
+      all_gather8(sw, all, g);
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int jj = 0; jj < 2; ++jj) {
+          const float mz = all[2 * nt + jj] * (1.f / 16.f), mo = all[4 + 2 * nt + jj] * (1.f / 16.f);
+          const float a = z[nt][jj] - mz, b = z[nt][jj + 2] - mz, c = o[nt][jj] - mo, d = o[nt][jj + 2] - mo;
+          v8[2 * nt + jj] = a * a + b * b;
+          v8[4 + 2 * nt + jj] = c * c + d * d;
+        }
+      const float m2w = reduce_scatter8(v8, g);
+      sm.fwd[g >> 2][pub_tok][warp] = sw;
+      sm.fwd[g >> 2][pub_tok][4 + warp] = m2w;
+      compute_sync<kLnWarps>();
+
+      float zh[2][4], ev[2][4], gg[2][4], rz[2][2];
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int jj = 0; jj < 2; ++jj) {
+          const int tok = 8 * nt + 2 * q + jj;
+          float mu, rstd;
+          merge_stats(sm.fwd[0][tok], eps, mu, rstd);
+          rz[nt][jj] = rstd;
+#pragma unroll
+          for (int hc = 0; hc < 2; ++hc) {
+            const int e = jj + 2 * hc;
+            zh[nt][e] = (z[nt][e] - mu) * rstd;
+            ev[nt][e] = fmaf(gam[hc], zh[nt][e], bet[hc]) + kv[nt][e];  // f(k) − v
+            gg[nt][e] = gam[hc] * ev[nt][e];
+          }
+          if (HAS_Q) {
+            merge_stats(sm.fwd[1][tok], eps, mu, rstd);
+#pragma unroll
+            for (int hc = 0; hc < 2; ++hc) {
+              const int e = jj + 2 * hc;
+              const float y = qv[nt][e] + fmaf(gam[hc], (o[nt][e] - mu) * rstd, bet[hc]);
+              *reinterpret_cast<__nv_bfloat16*>(obuf + swz128_bf16(r0 + tok, col0 + g + 8 * hc)) = __float2bfloat16_rn(y);
+            }
+          }
+        }
+
+      // ---- backward statistics: Σg and Σg·ẑ per token (and Σe² for the loss)
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int jj = 0; jj < 2; ++jj) {
+          v8[2 * nt + jj] = gg[nt][jj] + gg[nt][jj + 2];
+          v8[4 + 2 * nt + jj] = gg[nt][jj] * zh[nt][jj] + gg[nt][jj + 2] * zh[nt][jj + 2];
+        }
+      const float bw = reduce_scatter8(v8, g);
+      sm.bwd[pub_tok][4 * (g >> 2) + warp] = bw;
+      if (LOSS) {
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int jj = 0; jj < 2; ++jj) {
+            v8[2 * nt + jj] = ev[nt][jj] * ev[nt][jj] + ev[nt][jj + 2] * ev[nt][jj + 2];
+            v8[4 + 2 * nt + jj] = 0.f;
+          }
+        const float lw = reduce_scatter8(v8, g);
+        if (g < 4) sm.lossp[pub_tok][warp] = lw;
+      }
+      compute_sync<kLnWarps>();
+
+      // ---- dZ = rstd·(g − mean g − ẑ·mean(g·ẑ)); W ← W − (η/b)·Kᵀ·dZ
+      float dz[2][4];
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int jj = 0; jj < 2; ++jj) {
+          const int tok = 8 * nt + 2 * q + jj;
+          const float4 A = *reinterpret_cast<const float4*>(&sm.bwd[tok][0]);
+          const float4 B = *reinterpret_cast<const float4*>(&sm.bwd[tok][4]);
+          const float mg = ((A.x + A.y) + (A.z + A.w)) * (1.f / 64.f);
+          const float mgz = ((B.x + B.y) + (B.z + B.w)) * (1.f / 64.f);
+#pragma unroll
+          for (int hc = 0; hc < 2; ++hc) {
+            const int e = jj + 2 * hc;
+            dz[nt][e] = -lr * (rz[nt][jj] * (gg[nt][e] - mg - zh[nt][e] * mgz));
+          }
+          if (LOSS && warp == 0 && g == 0) {
+            const float4 L = *reinterpret_cast<const float4*>(&sm.lossp[tok][0]);
+            loss[(size_t)bh * T + (size_t)s * kTileTokI + r0 + tok] = (L.x + L.y) + (L.z + L.w);
+          }
+        }
+      uint32_t shi[4], slo[4];
+      afrag_hilo(dz[0], dz[1], shi, slo);
+#pragma unroll
+      for (int nt = 0; nt < 8; nt += 2) {
+        uint32_t kb[4];
+        ldsm4_t(kbase + swz128_bf16(r0 + 8 * (mi & 1) + ri, 8 * nt + 8 * (mi >> 1)), kb);
+        mma_bf16(acc[nt], shi, kb[0], kb[1]);
+        mma_bf16(acc[nt], slo, kb[0], kb[1]);
+        mma_bf16(acc[nt + 1], shi, kb[2], kb[3]);
+        mma_bf16(acc[nt + 1], slo, kb[2], kb[3]);
+      }
+    }
+    // End of the tile: its outputs are complete in shared memory.
+    if (HAS_Q) fence_proxy_async_smem();
+    compute_sync<kLnWarps>();
+    if (threadIdx.x == 0 && HAS_Q) {
+      tma_store_3d(&tmO, obuf, 0, s * kTileTokI, bh);
+      bulk_commit();
+      bulk_wait_read<1>();  // the other staging tile is free again
+    }
+    compute_sync<kLnWarps>();
+    if (lane == 0) mbar_arrive(&sm.empty[slot]);
+  }
+
+  if (threadIdx.x == 0 && HAS_Q) bulk_wait<0>();
+#pragma unroll
+  for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) Wg[(8 * nt + 2 * q + (e & 1)) * 64 + col0 + g + 8 * (e >> 1)] = acc[nt][e];
+  __syncthreads();
+}
+
+// ======================================== TTT-MLP ========================================
+//
+// Warp w of eight owns hidden units [32w, 32w+32): its slices of W1ᵀ (32 x 64) and W2ᵀ (64 x 32)
+// stay in accumulator registers (128 fp32 a thread). The second layer contracts over the hidden
+// units, so each warp's Zᵀ is a partial sum: the eight partials meet in shared memory (fp32), and
+// warp w finishes LayerNorm, the loss and the output rows of tokens 2w and 2w+1 with sixteen lanes
+// a token (four columns a lane), then publishes S = −(η/b)·∂ℓ/∂Z as bf16 hi and lo tiles that
+// every warp reads for its gradients. W2 takes part in both orientations (Z = A·W2 forward, S·W2ᵀ backward):
+// the backward's operand comes from the accumulators by movmatrix. No producer warp: the loads of
+// tile s + kStagesM go out from thread 0 as soon as every warp has finished tile s, which leaves
+// the register file to the eight compute warps.
+
+constexpr int kMlpWarps = 8;
+constexpr int kMlpThreads = kMlpWarps * 32;
+constexpr int kStagesM = 3;
+constexpr int kHid = 256;
+constexpr int kRedStride = 68;  // floats per token row of a partial Zᵀ (64 + 4: stores without bank conflicts)
+
+struct __align__(1024) MlpSmem {
+  uint8_t K[kStagesM][kTileBytesI];
+  uint8_t V[kStagesM][kTileBytesI];
+  uint8_t Q[kStagesM][kTileBytesI];
+  uint8_t O[2][kTileBytesI];
+  uint8_t S[2][kMB * 128];                 // −(η/b)·∂ℓ/∂Z [token][column] as bf16 hi and lo, 128-byte swizzle
+  float red[2][kMlpWarps][kMB][kRedStride];  // [keys or queries][warp][token][column]: partial Z
+  uint64_t full[kStagesM];
+  int cabort[2];
+};
+
+__device__ __forceinline__ uint32_t movm_t(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
+// GELU(x) = x·Φ(x) and its derivative Φ(x) + x·φ(x), through CUDA's erff and expf.
+__device__ __forceinline__ void gelu_and_grad(float x, float& y, float& dy) {
+  const float cdf = 0.5f * (1.f + erff(x * 0.70710678118654752f));
+  y = x * cdf;
+  dy = fmaf(x * 0.39894228040143268f, expf(-0.5f * x * x), cdf);
+}
+
+// Sum over the sixteen lanes that share lane >> 4.
+__device__ __forceinline__ float sum16(float x) {
+#pragma unroll
+  for (int m = 1; m < 16; m <<= 1) x += __shfl_xor_sync(0xffffffffu, x, m);
+  return x;
+}
+
+// LayerNorm of one token's four columns held by this lane (sixteen lanes hold the 64 columns).
+__device__ __forceinline__ void ln16(const float (&x)[4], float eps, float (&xh)[4], float& rstd) {
+  const float mu = sum16((x[0] + x[1]) + (x[2] + x[3])) * (1.f / 64.f);
+  float m2 = 0.f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float d = x[i] - mu;
+    m2 = fmaf(d, d, m2);
+  }
+  rstd = rsqrtf(sum16(m2) * (1.f / 64.f) + eps);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) xh[i] = (x[i] - mu) * rstd;
+}
+
+__device__ __forceinline__ void load4_bf16(const uint8_t* tile, int row, int col, float (&x)[4]) {
+  const uint2 u = *reinterpret_cast<const uint2*>(tile + swz128_bf16(row, col));
+  const float2 a = bf2_to_f2(u.x), b = bf2_to_f2(u.y);
+  x[0] = a.x;
+  x[1] = a.y;
+  x[2] = b.x;
+  x[3] = b.y;
+}
+
+__device__ __forceinline__ void store4_bf16(uint8_t* tile, int row, int col, const float (&x)[4]) {
+  *reinterpret_cast<uint2*>(tile + swz128_bf16(row, col)) = make_uint2(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]));
+}
+
+template <bool HAS_Q, bool LOSS>
+__global__ void __launch_bounds__(kMlpThreads, 1)
+    k_inner_mlp(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
+                float* __restrict__ Wstate, const float* __restrict__ gamma, const float* __restrict__ beta,
+                float* __restrict__ loss, int T, int heads, float lr, float eps, const DevStatus status) {
+  extern __shared__ uint8_t smem_raw[];
+  MlpSmem& sm = *reinterpret_cast<MlpSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, q = lane & 3, mi = lane >> 3, ri = lane & 7;
+  const int bh = blockIdx.x;
+  const int ntiles = (T + kTileTokI - 1) / kTileTokI;
+  const uint32_t stage_bytes = (HAS_Q ? 3u : 2u) * kTileBytesI;
+
+  auto issue = [&](int s) {
+    const int slot = s % kStagesM;
+    mbar_arrive_expect_tx(&sm.full[slot], stage_bytes);
+    tma_load_3d(sm.K[slot], &tmK, &sm.full[slot], 0, s * kTileTokI, bh);
+    tma_load_3d(sm.V[slot], &tmV, &sm.full[slot], 0, s * kTileTokI, bh);
+    if (HAS_Q) tma_load_3d(sm.Q[slot], &tmQ, &sm.full[slot], 0, s * kTileTokI, bh);
+  };
+  int issued = 0;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStagesM; ++i) mbar_init(&sm.full[i], 1);
+    sm.cabort[0] = sm.cabort[1] = 0;
+    fence_barrier_init();
+    for (; issued < kStagesM && issued < ntiles; ++issued) issue(issued);
+  }
+  __syncthreads();
+
+  // Per head: W1 [64][256] then W2 [256][64], row-major fp32.
+  float* W1g = Wstate + (size_t)bh * 2 * 64 * kHid;
+  float* W2g = W1g + 64 * kHid;
+  const int hid0 = 32 * warp;
+  // a1[mt][nt][e] = W1ᵀ[hid0 + 16mt + g + 8(e>>1)][8nt + 2q + (e&1)]
+  // a2[mt][nt][e] = W2ᵀ[16mt + g + 8(e>>1)][hid0 + 8nt + 2q + (e&1)]
+  float a1[2][8][4], a2[4][4][4];
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        a1[mt][nt][e] = W1g[(8 * nt + 2 * q + (e & 1)) * kHid + hid0 + 16 * mt + g + 8 * (e >> 1)];
+#pragma unroll
+  for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        a2[mt][nt][e] = W2g[(hid0 + 8 * nt + 2 * q + (e & 1)) * 64 + 16 * mt + g + 8 * (e >> 1)];
+
+  // LayerNorm stage: token 2·warp + (lane >> 4), columns c0 .. c0+3.
+  const int ltok = 2 * warp + (lane >> 4), c0 = 4 * (lane & 15);
+  const int h = bh % heads;
+  float gam[4], bet[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    gam[i] = gamma[h * 64 + c0 + i];
+    bet[i] = beta[h * 64 + c0 + i];
+  }
+  const uint32_t sbase[2] = {smem_u32(sm.S[0]), smem_u32(sm.S[1])};
+
+  int s = 0;
+  for (; s < ntiles; ++s) {
+    const int slot = s % kStagesM;
+    if (!mbar_wait(&sm.full[slot], (s / kStagesM) & 1, status, nullptr)) sm.cabort[s & 1] = 1;
+    compute_sync<kMlpWarps>();
+    if (*reinterpret_cast<volatile int*>(&sm.cabort[s & 1])) break;
+    const int ntok = min(kTileTokI, T - s * kTileTokI);
+    const uint8_t* Kt = sm.K[slot];
+    const uint8_t* Vt = sm.V[slot];
+    const uint8_t* Qt = sm.Q[slot];
+    const uint32_t kbase = smem_u32(Kt), qbase = smem_u32(Qt);
+    uint8_t* obuf = sm.O[s & 1];
+
+    for (int r0 = 0; r0 < ntok; r0 += kMB) {
+      // ---- first layer: Hᵀ = W1ᵀ·Kᵀ (and for the queries), hidden x tokens
+      float hk[2][2][4], hq[2][2][4];
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) hk[mt][nt][e] = hq[mt][nt][e] = 0.f;
+#pragma unroll
+      for (int ks = 0; ks < 4; ks += 2) {
+        uint32_t kb[2][4], qb[2][4];
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          const uint32_t off = swz128_bf16(r0 + 8 * nt + ri, 16 * ks + 8 * mi);
+          ldsm4(kbase + off, kb[nt]);
+          if (HAS_Q) ldsm4(qbase + off, qb[nt]);
+        }
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt) {
+          uint32_t whi[2][4], wlo[2][4];  // k-steps ks, ks + 1
+          afrag_hilo(a1[mt][2 * ks], a1[mt][2 * ks + 1], whi[0], wlo[0]);
+          afrag_hilo(a1[mt][2 * ks + 2], a1[mt][2 * ks + 3], whi[1], wlo[1]);
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int kk = 0; kk < 2; ++kk) {
+              mma_bf16(hk[mt][nt], whi[kk], kb[nt][2 * kk], kb[nt][2 * kk + 1]);
+              mma_bf16(hk[mt][nt], wlo[kk], kb[nt][2 * kk], kb[nt][2 * kk + 1]);
+              if (HAS_Q) {
+                mma_bf16(hq[mt][nt], whi[kk], qb[nt][2 * kk], qb[nt][2 * kk + 1]);
+                mma_bf16(hq[mt][nt], wlo[kk], qb[nt][2 * kk], qb[nt][2 * kk + 1]);
+              }
+            }
+        }
+      }
+      // ---- activation; A is kept as packed bf16 pairs in the accumulator layout (the B operand
+      // of the second layer's update) and GELU'(H) for the backward.
+      uint32_t ak[2][2][2], aq[2][2][2];
+      float dact[2][2][4];
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          float y[4], yq[4], dq;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            gelu_and_grad(hk[mt][nt][e], y[e], dact[mt][nt][e]);
+            if (HAS_Q) gelu_and_grad(hq[mt][nt][e], yq[e], dq);
+          }
+          ak[mt][nt][0] = pack_bf16(y[0], y[1]);
+          ak[mt][nt][1] = pack_bf16(y[2], y[3]);
+          if (HAS_Q) {
+            aq[mt][nt][0] = pack_bf16(yq[0], yq[1]);
+            aq[mt][nt][1] = pack_bf16(yq[2], yq[3]);
+          }
+        }
+      // ---- second layer, this warp's share: Zᵀ_w = W2ᵀ[:, slice]·Aᵀ[slice, :], columns x tokens.
+      // Aᵀ B fragments (hidden x tokens) by transposing the 8x8 blocks of the accumulator-layout A.
+      {
+        uint32_t bk[2][2][2], bq[2][2][2];  // [token n-tile][hidden k-step][half]
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int ks = 0; ks < 2; ++ks)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              bk[nt][ks][hh] = movm_t(ak[ks][nt][hh]);
+              if (HAS_Q) bq[nt][ks][hh] = movm_t(aq[ks][nt][hh]);
+            }
+#pragma unroll
+        for (int mt = 0; mt < 4; ++mt) {
+          uint32_t whi[2][4], wlo[2][4];  // hidden k-steps 0, 1
+          afrag_hilo(a2[mt][0], a2[mt][1], whi[0], wlo[0]);
+          afrag_hilo(a2[mt][2], a2[mt][3], whi[1], wlo[1]);
+#pragma unroll
+          for (int kind = 0; kind < (HAS_Q ? 2 : 1); ++kind) {
+            float* red = &sm.red[kind][warp][0][0];
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+              const uint32_t(&b)[2][2] = kind == 0 ? bk[nt] : bq[nt];
+              float zp[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+              for (int ks = 0; ks < 2; ++ks) {
+                mma_bf16(zp, whi[ks], b[ks][0], b[ks][1]);
+                mma_bf16(zp, wlo[ks], b[ks][0], b[ks][1]);
+              }
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                red[(8 * nt + 2 * q + (e & 1)) * kRedStride + 16 * mt + g + 8 * (e >> 1)] = zp[e];
+            }
+          }
+        }
+      }
+      compute_sync<kMlpWarps>();
+
+      // ---- LayerNorm, loss, outputs and S for tokens 2w, 2w+1
+      {
+        float z[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int p = 0; p < kMlpWarps; ++p) {
+          const float4 v = *reinterpret_cast<const float4*>(&sm.red[0][p][ltok][c0]);
+          z[0] += v.x;
+          z[1] += v.y;
+          z[2] += v.z;
+          z[3] += v.w;
+        }
+        float zh[4], rstd, kx[4], vx[4], ev[4], gg[4];
+        ln16(z, eps, zh, rstd);
+        load4_bf16(Kt, r0 + ltok, c0, kx);
+        load4_bf16(Vt, r0 + ltok, c0, vx);
+        float sg = 0.f, sgz = 0.f, se = 0.f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          ev[i] = fmaf(gam[i], zh[i], bet[i]) + (kx[i] - vx[i]);  // f(k) − v
+          gg[i] = gam[i] * ev[i];
+          sg += gg[i];
+          sgz = fmaf(gg[i], zh[i], sgz);
+          se = fmaf(ev[i], ev[i], se);
+        }
+        const float mg = sum16(sg) * (1.f / 64.f), mgz = sum16(sgz) * (1.f / 64.f);
+        float sv[4], sl[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          sv[i] = -lr * (rstd * (gg[i] - mg - zh[i] * mgz));
+          sl[i] = sv[i] - __bfloat162float(__float2bfloat16_rn(sv[i]));
+        }
+        store4_bf16(sm.S[0], ltok, c0, sv);  // rounds to the hi part
+        store4_bf16(sm.S[1], ltok, c0, sl);
+        if (LOSS) {
+          se = sum16(se);
+          if ((lane & 15) == 0) loss[(size_t)bh * T + (size_t)s * kTileTokI + r0 + ltok] = se;
+        }
+        if (HAS_Q) {
+          float zq[4] = {0.f, 0.f, 0.f, 0.f}, qh[4], qr, qx[4], y[4];
+#pragma unroll
+          for (int p = 0; p < kMlpWarps; ++p) {
+            const float4 v = *reinterpret_cast<const float4*>(&sm.red[1][p][ltok][c0]);
+            zq[0] += v.x;
+            zq[1] += v.y;
+            zq[2] += v.z;
+            zq[3] += v.w;
+          }
+          ln16(zq, eps, qh, qr);
+          load4_bf16(Qt, r0 + ltok, c0, qx);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) y[i] = qx[i] + fmaf(gam[i], qh[i], bet[i]);
+          store4_bf16(obuf, r0 + ltok, c0, y);
+        }
+      }
+      compute_sync<kMlpWarps>();
+
+      // ---- backward, every warp for its hidden slice; gradients at the step's starting weights
+      // dHᵀ = (W2[slice, :]·Sᵀ) ⊙ GELU'(H): W2 as the A operand, transposed from the W2ᵀ slice.
+      float dh[2][2][4];
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) dh[mt][nt][e] = 0.f;
+#pragma unroll
+      for (int ks = 0; ks < 4; ks += 2) {
+        uint32_t sb[2][2][4];  // Sᵀ B fragments (columns x tokens): [hi, lo][token n-tile]
+#pragma unroll
+        for (int p = 0; p < 2; ++p)
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt) ldsm4(sbase[p] + swz128_bf16(8 * nt + ri, 16 * ks + 8 * mi), sb[p][nt]);
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk) {
+          const int fk = ks + kk;  // 16-column k-step = W2ᵀ feature m-tile
+#pragma unroll
+          for (int mt = 0; mt < 2; ++mt) {
+            uint32_t w[4];
+            w[0] = movm_t(pack_bf16(a2[fk][2 * mt][0], a2[fk][2 * mt][1]));
+            w[1] = movm_t(pack_bf16(a2[fk][2 * mt + 1][0], a2[fk][2 * mt + 1][1]));
+            w[2] = movm_t(pack_bf16(a2[fk][2 * mt][2], a2[fk][2 * mt][3]));
+            w[3] = movm_t(pack_bf16(a2[fk][2 * mt + 1][2], a2[fk][2 * mt + 1][3]));
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+              for (int p = 0; p < 2; ++p) mma_bf16(dh[mt][nt], w, sb[p][nt][2 * kk], sb[p][nt][2 * kk + 1]);
+          }
+        }
+      }
+      // W1ᵀ += dHᵀ·K (S already carries −η/b).
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt) {
+        uint32_t da[4];
+        da[0] = pack_bf16(dh[mt][0][0] * dact[mt][0][0], dh[mt][0][1] * dact[mt][0][1]);
+        da[1] = pack_bf16(dh[mt][0][2] * dact[mt][0][2], dh[mt][0][3] * dact[mt][0][3]);
+        da[2] = pack_bf16(dh[mt][1][0] * dact[mt][1][0], dh[mt][1][1] * dact[mt][1][1]);
+        da[3] = pack_bf16(dh[mt][1][2] * dact[mt][1][2], dh[mt][1][3] * dact[mt][1][3]);
+#pragma unroll
+        for (int nt = 0; nt < 8; nt += 2) {
+          uint32_t kb[4];
+          ldsm4_t(kbase + swz128_bf16(r0 + 8 * (mi & 1) + ri, 8 * nt + 8 * (mi >> 1)), kb);
+          mma_bf16(a1[mt][nt], da, kb[0], kb[1]);
+          mma_bf16(a1[mt][nt + 1], da, kb[2], kb[3]);
+        }
+      }
+      // W2ᵀ += Sᵀ·A: Sᵀ as the A operand (columns x tokens), A (tokens x hidden) as B.
+#pragma unroll
+      for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+          uint32_t sa[4];
+          ldsm4_t(sbase[p] + swz128_bf16(8 * (mi >> 1) + ri, 16 * mt + 8 * (mi & 1)), sa);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) mma_bf16(a2[mt][j], sa, ak[j >> 1][0][j & 1], ak[j >> 1][1][j & 1]);
+        }
+    }
+    // End of the tile: its outputs are complete in shared memory and every warp is done with
+    // its inputs, so the slot takes tile s + kStagesM.
+    if (HAS_Q) fence_proxy_async_smem();
+    compute_sync<kMlpWarps>();
+    if (threadIdx.x == 0) {
+      if (HAS_Q) {
+        tma_store_3d(&tmO, obuf, 0, s * kTileTokI, bh);
+        bulk_commit();
+      }
+      if (issued < ntiles) issue(issued++);
+      if (HAS_Q) bulk_wait_read<1>();  // the other staging tile is free again
+    }
+  }
+  if (threadIdx.x == 0) {
+    if (HAS_Q) bulk_wait<0>();
+    // Nothing may still be landing in shared memory when the CTA exits (after an abort the
+    // tiles issued past the last one consumed).
+    for (int t = s; t < issued; ++t) mbar_wait(&sm.full[t % kStagesM], (t / kStagesM) & 1, status, nullptr);
+  }
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        W1g[(8 * nt + 2 * q + (e & 1)) * kHid + hid0 + 16 * mt + g + 8 * (e >> 1)] = a1[mt][nt][e];
+#pragma unroll
+  for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        W2g[(hid0 + 8 * nt + 2 * q + (e & 1)) * 64 + 16 * mt + g + 8 * (e >> 1)] = a2[mt][nt][e];
+  __syncthreads();
+}
+
+template <bool HAS_Q, bool LOSS>
+ttt_status launch_inner(ttt_state* st, const CUtensorMap* maps, float* loss, int T, cudaStream_t s) {
+  const ttt_config& c = st->cfg;
+  const bool mlp = c.rule == TTT_RULE_MLP_GD;
+  const size_t smem = (mlp ? sizeof(MlpSmem) : sizeof(LnSmem)) + 1024;
+  // One bit per instantiation whose shared-memory limit has been raised on this state's device.
+  const uint64_t bit = 1ull << (48 + 4 * mlp + 2 * HAS_Q + LOSS);
+  auto kernel = mlp ? k_inner_mlp<HAS_Q, LOSS> : k_inner_ln<HAS_Q, LOSS>;
+  if (!(st->lin.smem_set & bit)) {
+    TTT_CUDA(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    st->lin.smem_set |= bit;
+  }
+  const int grid = c.batch * c.heads;
+  const float lr = c.eta / (float)kMB;
+  kernel<<<grid, mlp ? kMlpThreads : kLnThreads, smem, s>>>(
+      maps[0], maps[1], maps[2], maps[3], st->lin.W, st->lin.ln_gamma, st->lin.ln_beta, loss, T, c.heads, lr,
+      c.ln_eps, DevStatus{st->status.dev, st->wait_limit_ns, st->status.dev + 1});
+  st->launches++;
+  TTT_CUDA(cudaGetLastError());
+  return TTT_OK;
+}
+
+}  // namespace
+
+ttt_status inner_scan(ttt_state* st, const __nv_bfloat16* K, const __nv_bfloat16* V, const __nv_bfloat16* Q,
+                      int64_t T, __nv_bfloat16* O, float* loss, cudaStream_t s) {
+  const ttt_config& c = st->cfg;
+  // [B·H, T, 64] bf16 views of K, V, Q and O, 64-token boxes with the 128-byte swizzle; the maps
+  // of the last few buffer sets are kept (encoding costs microseconds of host time).
+  const uint64_t dims[3] = {64, (uint64_t)T, (uint64_t)c.batch * c.heads};
+  const uint64_t strides[2] = {128, (uint64_t)T * 128};
+  const uint32_t box[3] = {64, (uint32_t)kTileTokI, 1};
+  LinearBuffers& lb = st->lin;
+  const bool has_q = Q != nullptr;
+  const void* key[4] = {K, V, Q, O};
+  LinearMapSet* ms = nullptr;
+  for (LinearMapSet& m : lb.map_sets)
+    if (m.T == T && m.key[0] == key[0] && m.key[1] == key[1] && m.key[2] == key[2] && m.key[3] == key[3]) ms = &m;
+  if (ms == nullptr) {
+    ms = &lb.map_sets[0];
+    for (LinearMapSet& m : lb.map_sets)
+      if (m.last_use < ms->last_use) ms = &m;
+    ms->T = -1;  // invalid until all four are encoded
+    for (int i = 0; i < 4; ++i) {
+      const void* base = key[i] != nullptr ? key[i] : key[0];
+      TTT_TRY(encode_tmap(&ms->maps[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box,
+                          CU_TENSOR_MAP_SWIZZLE_128B));
+      ms->key[i] = key[i];
+    }
+    ms->T = T;
+  }
+  ms->last_use = ++lb.map_clock;
+  if (has_q)
+    return loss ? launch_inner<true, true>(st, ms->maps, loss, (int)T, s)
+                : launch_inner<true, false>(st, ms->maps, loss, (int)T, s);
+  return loss ? launch_inner<false, true>(st, ms->maps, loss, (int)T, s)
+              : launch_inner<false, false>(st, ms->maps, loss, (int)T, s);
+}
+
+}  // namespace ttt

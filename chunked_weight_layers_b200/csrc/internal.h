@@ -85,8 +85,10 @@ struct LinearMapSet {
 };
 
 struct LinearBuffers {
-  float* W = nullptr;   // [B, H, D, D]
-  float* W0 = nullptr;  // [B, H, D, D]
+  float* W = nullptr;   // [B, H, D, D] (TTT-MLP: [B, H, 64·256 + 256·64], W1 then W2 per head)
+  float* W0 = nullptr;  // same shape
+  float* ln_gamma = nullptr;  // LayerNorm rules: [H, 64] gain and bias of the inner model's LN
+  float* ln_beta = nullptr;
   static constexpr int kMapSets = 8;
   LinearMapSet map_sets[kMapSets];
   uint64_t map_clock = 0;
@@ -162,6 +164,11 @@ void free_tc(ttt_state* st);
 ttt_status linear_scan(ttt_state* st, const __nv_bfloat16* K, const __nv_bfloat16* V,
                        const __nv_bfloat16* Q, int64_t T, __nv_bfloat16* O, float* loss,
                        cudaStream_t s);
+
+// TTT-Linear with LayerNorm and residual, or TTT-MLP: the scan over T tokens of every
+// (sequence, head), mini-batch 16.
+ttt_status inner_scan(ttt_state* st, const __nv_bfloat16* K, const __nv_bfloat16* V, const __nv_bfloat16* Q,
+                      int64_t T, __nv_bfloat16* O, float* loss, cudaStream_t s);
 
 // Residual-cache read path: out = o_ttt + clamp(α, 0, 1) ⊙ (attention over the visible entries).
 ttt_status cache_attention(const ttt_state* st, const __nv_bfloat16* Q, const __nv_bfloat16* K,

@@ -92,11 +92,24 @@ static ttt_status validate(const ttt_config* c) {
     }
     return TTT_OK;
   }
+  if (c->rule == TTT_RULE_LINEAR_LN_GD || c->rule == TTT_RULE_MLP_GD) {
+    const char* name = c->rule == TTT_RULE_MLP_GD ? "TTT-MLP" : "TTT-Linear with LayerNorm";
+    if (c->io_dtype != TTT_BF16) return fail(TTT_ERR_UNSUPPORTED, "%s: io_dtype must be BF16", name);
+    if (c->batch < 1 || c->heads < 1) return fail(TTT_ERR_INVALID_ARG, "%s: batch and heads must be positive", name);
+    if (c->d_key != 64 || c->d_val != 64)
+      return fail(TTT_ERR_UNSUPPORTED, "%s: head width must be 64 (d_key = d_val = 64)", name);
+    if (c->chunk != 16) return fail(TTT_ERR_UNSUPPORTED, "%s: inner mini-batch must be 16", name);
+    if (c->target_mode != 0) return fail(TTT_ERR_INVALID_ARG, "target_mode applies to In-Place only");
+    if (c->gate_enable) return fail(TTT_ERR_UNSUPPORTED, "the surprisal gate runs on TTT-Linear states");
+    if (!(c->ln_eps > 0.f)) return fail(TTT_ERR_INVALID_ARG, "%s: ln_eps must be positive", name);
+    return TTT_OK;
+  }
   return fail(TTT_ERR_INVALID_ARG, "unknown rule %d", c->rule);
 }
 
 static size_t weight_elems(const ttt_config& c) {
   if (c.rule == TTT_RULE_INPLACE_HEBBIAN) return (size_t)c.d_val * c.d_key;
+  if (c.rule == TTT_RULE_MLP_GD) return (size_t)c.batch * c.heads * 2 * 64 * 256;
   return (size_t)c.batch * c.heads * c.d_key * c.d_key;
 }
 
@@ -124,6 +137,8 @@ static void free_state(ttt_state* st) {
   dev_free(st->ip.Vhat[2]);
   dev_free(st->lin.W);
   dev_free(st->lin.W0);
+  dev_free(st->lin.ln_gamma);
+  dev_free(st->lin.ln_beta);
   dev_free(st->gate.tau);
   dev_free(st->gate.tau_set);
   dev_free(st->gate.entries);
@@ -215,6 +230,10 @@ static ttt_status create_impl(const ttt_config* cfg, const void* W0, const void*
     const size_t bh = (size_t)c.batch * c.heads;
     const int cap = c.gate_enable ? c.cache_capacity : 1;
     st->cfg.cache_capacity = cap;
+    if (r == TTT_OK && (c.rule == TTT_RULE_LINEAR_LN_GD || c.rule == TTT_RULE_MLP_GD)) {
+      guard(dev_alloc((void**)&st->lin.ln_gamma, (size_t)c.heads * 64 * 4, "LayerNorm gain")) &&
+          guard(dev_alloc((void**)&st->lin.ln_beta, (size_t)c.heads * 64 * 4, "LayerNorm bias"));
+    }
     if (r == TTT_OK) {
       guard(dev_alloc((void**)&st->gate.tau, bh * 4, "tau")) &&
           guard(dev_alloc((void**)&st->gate.tau_set, bh * 4, "tau_set")) &&
@@ -239,6 +258,14 @@ static ttt_status create_impl(const ttt_config* cfg, const void* W0, const void*
   }
   r = load_weights(st, W0dst, s);
   if (r == TTT_OK && c.rule == TTT_RULE_LINEAR_GD) r = gate_reset(st, s);
+  if (r == TTT_OK && st->lin.ln_gamma != nullptr) {
+    // γ = 1 (the bits of 1.0f), β = 0.
+    r = fill_i32(reinterpret_cast<int32_t*>(st->lin.ln_gamma), 0x3f800000, (size_t)c.heads * 64, s, st);
+    if (r == TTT_OK) {
+      e = cudaMemsetAsync(st->lin.ln_beta, 0, (size_t)c.heads * 64 * 4, s);
+      if (e != cudaSuccess) r = cuda_fail(e, "LayerNorm bias");
+    }
+  }
   if (r != TTT_OK) {
     free_state(st);
     return r;
@@ -296,6 +323,9 @@ static ttt_status scan_impl(ttt_state* st, const void* keys, const void* targets
   if (queries != nullptr && (!aligned16(queries) || !aligned16(out)))
     return fail(TTT_ERR_INVALID_ARG, "queries and out must be 16-byte aligned");
   if (loss != nullptr && !aligned16(loss)) return fail(TTT_ERR_INVALID_ARG, "loss_out must be 16-byte aligned");
+  if (c.rule != TTT_RULE_LINEAR_GD)
+    return inner_scan(st, static_cast<const __nv_bfloat16*>(keys), static_cast<const __nv_bfloat16*>(targets),
+                      static_cast<const __nv_bfloat16*>(queries), T, static_cast<__nv_bfloat16*>(out), loss, s);
   if (c.gate_enable) {
     if (loss == nullptr) return fail(TTT_ERR_INVALID_ARG, "the gate needs loss_out");
     if (T % c.gate_chunk != 0) return fail(TTT_ERR_INVALID_ARG, "T must be a multiple of gate_chunk with the gate on");
@@ -325,13 +355,13 @@ using namespace ttt;
 
 extern "C" {
 
-int32_t ttt_abi_version(void) { return 1; }
+int32_t ttt_abi_version(void) { return 2; }
 
 const char* ttt_last_error_string(void) { return ttt::g_last_error; }
 
 ttt_status ttt_config_init(ttt_config* cfg, int32_t rule) {
   if (cfg == nullptr) return fail(TTT_ERR_INVALID_ARG, "cfg is NULL");
-  if (rule != TTT_RULE_INPLACE_HEBBIAN && rule != TTT_RULE_LINEAR_GD) return fail(TTT_ERR_INVALID_ARG, "unknown rule %d", rule);
+  if (rule < TTT_RULE_INPLACE_HEBBIAN || rule > TTT_RULE_MLP_GD) return fail(TTT_ERR_INVALID_ARG, "unknown rule %d", rule);
   memset(cfg, 0, sizeof(*cfg));
   cfg->rule = rule;
   cfg->io_dtype = TTT_BF16;
@@ -339,7 +369,7 @@ ttt_status ttt_config_init(ttt_config* cfg, int32_t rule) {
   cfg->heads = 1;
   cfg->d_key = 64;
   cfg->d_val = 64;
-  cfg->chunk = rule == TTT_RULE_LINEAR_GD ? 16 : 1024;
+  cfg->chunk = rule == TTT_RULE_INPLACE_HEBBIAN ? 1024 : 16;
   cfg->eta = 1.0f;
   cfg->conv_taps = 3;
   cfg->gate_chunk = 64;
@@ -349,6 +379,7 @@ ttt_status ttt_config_init(ttt_config* cfg, int32_t rule) {
   cfg->gate_ema_new = 0.1f;
   cfg->gate_mean_num = 4;
   cfg->gate_mean_den = 5;
+  cfg->ln_eps = 1e-6f;
   return TTT_OK;
 }
 
@@ -476,9 +507,22 @@ ttt_status ttt_state_set_weights(ttt_state* st, const float* W, ttt_stream strea
   return load_weights(st, W, reinterpret_cast<cudaStream_t>(stream));
 }
 
+ttt_status ttt_state_set_layernorm(ttt_state* st, const float* gamma, const float* beta, ttt_stream stream) {
+  if (st == nullptr) return fail(TTT_ERR_INVALID_ARG, "state is NULL");
+  if (st->lin.ln_gamma == nullptr) return fail(TTT_ERR_UNSUPPORTED, "only the LayerNorm rules have a LayerNorm");
+  if (gamma == nullptr || beta == nullptr || !aligned16(gamma) || !aligned16(beta))
+    return fail(TTT_ERR_INVALID_ARG, "gamma and beta must be 16-byte aligned device pointers");
+  TTT_TRY(check_device(st));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t bytes = (size_t)st->cfg.heads * 64 * 4;
+  TTT_CUDA(cudaMemcpyAsync(st->lin.ln_gamma, gamma, bytes, cudaMemcpyDeviceToDevice, s));
+  TTT_CUDA(cudaMemcpyAsync(st->lin.ln_beta, beta, bytes, cudaMemcpyDeviceToDevice, s));
+  return TTT_OK;
+}
+
 ttt_status ttt_cache_read(const ttt_state* st, int32_t* entries, int32_t* counts, ttt_stream stream) {
   if (st == nullptr) return fail(TTT_ERR_INVALID_ARG, "state is NULL");
-  if (st->cfg.rule != TTT_RULE_LINEAR_GD) return fail(TTT_ERR_UNSUPPORTED, "In-Place states have no residual cache");
+  if (st->cfg.rule != TTT_RULE_LINEAR_GD) return fail(TTT_ERR_UNSUPPORTED, "only TTT-Linear states have a residual cache");
   TTT_TRY(check_device(st));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const size_t bh = (size_t)st->cfg.batch * st->cfg.heads;
@@ -490,7 +534,7 @@ ttt_status ttt_cache_read(const ttt_state* st, int32_t* entries, int32_t* counts
 
 ttt_status ttt_gate_read(const ttt_state* st, float* tau, int32_t* tau_set, ttt_stream stream) {
   if (st == nullptr) return fail(TTT_ERR_INVALID_ARG, "state is NULL");
-  if (st->cfg.rule != TTT_RULE_LINEAR_GD) return fail(TTT_ERR_UNSUPPORTED, "In-Place states have no gate");
+  if (st->cfg.rule != TTT_RULE_LINEAR_GD) return fail(TTT_ERR_UNSUPPORTED, "only TTT-Linear states have a gate");
   TTT_TRY(check_device(st));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const size_t bh = (size_t)st->cfg.batch * st->cfg.heads;

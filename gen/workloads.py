@@ -65,6 +65,35 @@ class LinearSpec:
         return per * self.D * self.D * self.T * self.B * self.H
 
 
+@dataclass(frozen=True)
+class InnerSpec:
+    """TTT-Linear with LayerNorm and residual ("linear_ln") or TTT-MLP ("mlp") over B sequences x
+    H heads of width 64, inner mini-batch b."""
+
+    name: str
+    model: str
+    B: int
+    H: int
+    T: int
+    b: int = 16
+    eta: float = 0.1
+    eps: float = 1e-6
+    with_queries: bool = True
+    seed: int = 1000
+    D: int = 64
+    hidden: int = 256
+
+    @property
+    def flops(self) -> float:
+        """Products per (token, head): LayerNorm TTT-Linear k·W, q·W and Kᵀ·dZ (2·D² each);
+        TTT-MLP two layers forward for keys and queries and three gradient products (2·D·Dh each)."""
+        if self.model == "linear_ln":
+            per = (6.0 if self.with_queries else 4.0) * self.D * self.D
+        else:
+            per = (14.0 if self.with_queries else 10.0) * self.D * self.hidden
+        return per * self.T * self.B * self.H
+
+
 # The five workloads, by what they are.
 INPLACE_FP32 = InplaceSpec("inplace_fp32_T2048_C512_d256_f512", T=2048, C=512, d=256, f=512,
                            eta=0.01, dtype="f32", seed=1001)
@@ -77,6 +106,12 @@ SR_TTT_GATE = LinearSpec("srttt_gate_B4_H16_T8192_b16", B=4, H=16, T=8192, b=16,
                          with_queries=False, needle_frac=0.01, gate=True, seed=1005)
 
 WORKLOADS = {w.name: w for w in (INPLACE_FP32, LINEAR_GD, INPLACE_4B, INPLACE_128K_TARGET, SR_TTT_GATE)}
+
+# The richer inner models at the TTT-Linear workload's shapes (the TTT layers page's two
+# instances, with LayerNorm and residual).
+LINEAR_LN = InnerSpec("ttt_linear_ln_B8_H12_T2048_b16", model="linear_ln", B=8, H=12, T=2048, seed=1007)
+MLP = InnerSpec("ttt_mlp_B8_H12_T2048_b16", model="mlp", B=8, H=12, T=2048, seed=1008)
+INNER_WORKLOADS = {w.name: w for w in (LINEAR_LN, MLP)}
 
 
 def document_starts(T: int, n_docs: int, seed: int, min_len: int = 64) -> list[int]:
@@ -189,4 +224,32 @@ def linear_inputs(spec: LinearSpec, device="cpu") -> dict:
         out["Q"] = (rng.normal("Q", shape, s, device) / 8.0).to(torch.bfloat16)
     eye = torch.eye(spec.D, dtype=torch.float32, device=device)
     out["W0"] = eye.expand(spec.B, spec.H, spec.D, spec.D).contiguous()
+    return out
+
+
+# ----------------------------------------------------------------------------------------------
+# Richer inner models
+# ----------------------------------------------------------------------------------------------
+
+def inner_inputs(spec: InnerSpec, device="cpu") -> dict:
+    """K, V (and Q) [B,H,T,64] bf16 ~ N(0,1)/8 as for TTT-Linear; LayerNorm gain 1 + 0.1·N(0,1)
+    and bias 0.1·N(0,1) per head [H, 64] fp32. LayerNorm TTT-Linear: W0 = I [B,H,64,64].
+    TTT-MLP: W1 ~ N(0,1) [B,H,64,256] (so k·W1 ~ N(0,1)) and W2 ~ N(0,1)/16 [B,H,256,64],
+    packed per (sequence, head) as W1 then W2."""
+    s, shape = spec.seed, (spec.B, spec.H, spec.T, spec.D)
+    out = {"eta": spec.eta, "eps": spec.eps}
+    out["K"] = (rng.normal("K", shape, s, device) / 8.0).to(torch.bfloat16)
+    out["V"] = (rng.normal("V", shape, s, device) / 8.0).to(torch.bfloat16)
+    if spec.with_queries:
+        out["Q"] = (rng.normal("Q", shape, s, device) / 8.0).to(torch.bfloat16)
+    out["gamma"] = (1.0 + 0.1 * rng.normal("ln_gamma", (spec.H, spec.D), s, device)).to(torch.float32)
+    out["beta"] = (0.1 * rng.normal("ln_beta", (spec.H, spec.D), s, device)).to(torch.float32)
+    if spec.model == "linear_ln":
+        eye = torch.eye(spec.D, dtype=torch.float32, device=device)
+        out["W0"] = eye.expand(spec.B, spec.H, spec.D, spec.D).contiguous()
+    else:
+        W1 = rng.normal("W1", (spec.B, spec.H, spec.D, spec.hidden), s, device).to(torch.float32)
+        W2 = (rng.normal("W2", (spec.B, spec.H, spec.hidden, spec.D), s, device) / 16.0).to(torch.float32)
+        out["W1"], out["W2"] = W1, W2
+        out["W0"] = torch.cat([W1.reshape(spec.B, spec.H, -1), W2.reshape(spec.B, spec.H, -1)], dim=2).contiguous()
     return out

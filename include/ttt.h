@@ -16,6 +16,15 @@
  *  (sequence, head), for each inner mini-batch i of b tokens: O_i = Q_i · W_i,
  *  R_i = K_i · W_i − V_i, L_t = ‖R_i[t]‖², W_{i+1} = W_i − (η/b) · K_iᵀ · R_i.
  *
+ *  Richer inner models (the TTT layers page: TTT-Linear and TTT-MLP are its two instances,
+ *  and by its DeltaNet remark the full TTT-Linear carries a LayerNorm and a residual
+ *  connection). The inner model is f(x) = x + LN(g(x)) with g(x) = x · W (rule
+ *  TTT_RULE_LINEAR_LN_GD) or g(x) = GELU(x · W1) · W2 (TTT_RULE_MLP_GD, hidden width 256,
+ *  GELU(x) = x·Φ(x)); LN normalises a token's 64 values by their mean and population variance
+ *  (ε under the square root) and applies the per-head gain γ and bias β, which the inner step
+ *  does not change. Per mini-batch of 16 tokens: O_i = f(Q_i; θ_i), E_i = f(K_i; θ_i) − V_i,
+ *  L_t = ‖E_i[t]‖², θ_{i+1} = θ_i − η · ∇ℓ_i(θ_i) with ℓ_i = ‖E_i‖² / (2·16).
+ *
  *  Surprisal gate ("SR-TTT: Surprisal-Aware Residual Test-Time Training", §2.1). Per
  *  (sequence, head) and chunk of 64 losses: p95 = 61st smallest; τ = p95 for the first
  *  chunk, else τ = fl32(fl32(0.9·τ) + fl32(0.1·p95)); the chunk passes if
@@ -68,7 +77,12 @@ typedef enum {
   TTT_ERR_DEVICE = 6       /* a device-side consistency check failed (from ttt_state_poll) */
 } ttt_status;
 
-typedef enum { TTT_RULE_INPLACE_HEBBIAN = 0, TTT_RULE_LINEAR_GD = 1 } ttt_rule;
+typedef enum {
+  TTT_RULE_INPLACE_HEBBIAN = 0,
+  TTT_RULE_LINEAR_GD = 1,     /* TTT-Linear: linear inner model, no normalisation */
+  TTT_RULE_LINEAR_LN_GD = 2,  /* TTT-Linear with LayerNorm and residual */
+  TTT_RULE_MLP_GD = 3         /* TTT-MLP: two-layer GELU MLP (hidden 256) with LayerNorm and residual */
+} ttt_rule;
 typedef enum { TTT_F32 = 0, TTT_BF16 = 1 } ttt_dtype;
 
 typedef struct {
@@ -95,6 +109,7 @@ typedef struct {
   float gate_ema_new;     /* weight on the chunk's percentile; 0.1f */
   int32_t gate_mean_num;  /* the mean test is S/gate_chunk >= (num/den)·τ; 4 */
   int32_t gate_mean_den;  /* 5 */
+  float ln_eps;           /* TTT_RULE_LINEAR_LN_GD and TTT_RULE_MLP_GD: LayerNorm ε; 1e-6 */
 } ttt_config;
 
 typedef struct ttt_state ttt_state; /* opaque; owns all of its device memory */
@@ -102,13 +117,19 @@ typedef struct ttt_state ttt_state; /* opaque; owns all of its device memory */
 /* ABI version of this header (incremented on any incompatible change). */
 int32_t ttt_abi_version(void);
 
-/* Fill *cfg with the defaults of `rule` (the values noted above, eta = 1, chunk 16 for
- * TTT-Linear, 1024 for In-Place, BF16). INVALID_ARG if cfg is NULL or rule unknown. */
+/* Fill *cfg with the defaults of `rule` (the values noted above, eta = 1, chunk 16 for the
+ * TTT-Linear and TTT-MLP rules, 1024 for In-Place, BF16). INVALID_ARG if cfg is NULL or rule
+ * unknown. The rules with LayerNorm and the MLP take only batch, heads, eta and ln_eps: head
+ * width 64, mini-batch 16, BF16 io, no gate (else UNSUPPORTED at ttt_state_create). */
 ttt_status ttt_config_init(ttt_config* cfg, int32_t rule);
 
 /* Create a scan state on the current device and copy the initial weights into it.
  *   W0       device. In-Place: fp32 [d_val, d_key] (Wdown, row-major).
- *                    TTT-Linear: fp32 [batch, heads, d_key, d_key], applied as x·W.
+ *                    TTT-Linear (with or without LayerNorm): fp32 [batch, heads, d_key, d_key],
+ *                    applied as x·W.
+ *                    TTT-MLP: fp32 [batch, heads, 64·256 + 256·64]: per (sequence, head) W1
+ *                    [64, 256] then W2 [256, 64], row-major, applied as GELU(x·W1)·W2.
+ *            The LayerNorm rules start with γ = 1 and β = 0 (ttt_state_set_layernorm).
  *   Wtarget  device, In-Place with target_mode 1 only (else NULL): bf16 [d_val, d_val],
  *            [in, out], V̂[t, j] = Σ_i conv[t, i]·Wtarget[i, j].
  *   convw    device, target_mode 1 only (else NULL): fp32 [d_val, conv_taps].
@@ -125,7 +146,8 @@ ttt_status ttt_state_create(const ttt_config* cfg, const void* W0, const void* W
  *   In-Place:   keys = Z [T, d_key]; targets = V̂ [T, d_val] (target_mode 0) or X0 [T, d_val]
  *               (target_mode 1); queries must be NULL; out = O [T, d_val] (required);
  *               loss_out must be NULL. T must be a multiple of chunk.
- *   TTT-Linear: keys = K, targets = V, queries = Q (or NULL), all [batch, heads, T, d_key];
+ *   TTT-Linear, TTT-MLP: keys = K, targets = V, queries = Q (or NULL), all
+ *               [batch, heads, T, d_key];
  *               out = O [batch, heads, T, d_key] (NULL iff queries is NULL);
  *               loss_out = L [batch, heads, T] fp32 (or NULL; required when the gate is
  *               enabled). T must be a multiple of chunk (and of gate_chunk with the gate).
@@ -189,6 +211,14 @@ ttt_status ttt_state_reset(ttt_state* st, ttt_stream stream);
  * it back resumes a scan exactly at a chunk boundary. */
 ttt_status ttt_state_get_weights(const ttt_state* st, float* W, ttt_stream stream);
 ttt_status ttt_state_set_weights(ttt_state* st, const float* W, ttt_stream stream);
+
+/* Set the LayerNorm gain and bias of the inner model (TTT_RULE_LINEAR_LN_GD and
+ * TTT_RULE_MLP_GD states; UNSUPPORTED otherwise): gamma and beta (device) fp32 [heads, 64],
+ * shared by every sequence. They are parameters of the outer model: the scan reads them and
+ * never updates them (copied; the caller keeps ownership). A state starts with γ = 1, β = 0.
+ * Defined by the TTT layers page (the full TTT-Linear's inner model carries a LayerNorm, which
+ * DeltaNet drops). */
+ttt_status ttt_state_set_layernorm(ttt_state* st, const float* gamma, const float* beta, ttt_stream stream);
 
 /* Copy out the residual cache: entries (device) int32 [batch, heads, cache_capacity, 3]
  * holding (sequence, head, t) with t counted from the last reset, unused entries -1;

@@ -46,6 +46,10 @@ def test_config_defaults(lib):
     assert abs(cfg.gate_pct - 0.95) < 1e-7 and cfg.gate_ema_old == ctypes.c_float(0.9).value
     assert cfg.gate_ema_new == ctypes.c_float(0.1).value
     assert (cfg.gate_mean_num, cfg.gate_mean_den) == (4, 5)
+    for rule in (abi.TTT_RULE_LINEAR_LN_GD, abi.TTT_RULE_MLP_GD):
+        assert lib.ttt_config_init(ctypes.byref(cfg), rule) == abi.TTT_OK
+        assert (cfg.rule, cfg.chunk, cfg.d_key, cfg.d_val, cfg.io_dtype) == (rule, 16, 64, 64, abi.TTT_BF16)
+        assert cfg.ln_eps == ctypes.c_float(1e-6).value
     assert lib.ttt_config_init(None, 0) == abi.TTT_ERR_INVALID_ARG
     assert lib.ttt_config_init(ctypes.byref(cfg), 7) == abi.TTT_ERR_INVALID_ARG
     assert b"unknown rule" in lib.ttt_last_error_string()
@@ -61,7 +65,7 @@ def test_host_argument_checks(lib):
     assert lib.ttt_surprisal_route(None, None, 0, None) == abi.TTT_ERR_INVALID_ARG
     assert lib.ttt_state_destroy(None) == abi.TTT_OK
     assert lib.ttt_state_launch_count(None) == 0
-    assert lib.ttt_abi_version() == 1
+    assert lib.ttt_abi_version() == 2
 
 
 def test_binding_refuses_without_library(tmp_path):
@@ -127,6 +131,12 @@ def test_binding_element_counts_follow_the_config(monkeypatch):
         # In-Place fp32 with the same widths.
         (dict(rule=0, io_dtype=0, batch=1, heads=1, d_key=512, d_val=256, chunk=128), 384,
          dict(keys=196608, targets=98304, out=98304), 131072, 1),
+        # TTT-Linear with LayerNorm, B=1, H=2, T=32: W [B,H,64,64].
+        (dict(rule=2, io_dtype=1, batch=1, heads=2, d_key=64, d_val=64, chunk=16), 32,
+         dict(keys=4096, targets=4096, queries=4096, out=4096, loss_out=64), 8192, 1),
+        # TTT-MLP, B=1, H=2: W1 [64, 256] and W2 [256, 64] per pair.
+        (dict(rule=3, io_dtype=1, batch=1, heads=2, d_key=64, d_val=64, chunk=16), 32,
+         dict(keys=4096, targets=4096, queries=4096, out=4096, loss_out=64), 65536, 1),
     ]
     for fields, T, want, nW, cap in cases:
         cfg = cwl.abi.ttt_config(**fields)

@@ -44,4 +44,4 @@ def test_plain_c_program_uses_the_abi(tmp_path):
                     str(src), "-L", libdir, "-lttt", f"-Wl,-rpath,{libdir}", "-o", str(exe)], check=True)
     out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
     assert out.returncode == 0, (out.returncode, out.stdout, out.stderr)
-    assert out.stdout.splitlines() == ["abi=1 chunk=1024 io=1 taps=3", "ok"]
+    assert out.stdout.splitlines() == ["abi=2 chunk=1024 io=1 taps=3", "ok"]
