@@ -22,6 +22,10 @@ Readings taken where the page prints no formula (the plainest ones the rest supp
   the mini-batch: θ_{i+1} = θ_i − η·∇ℓ_i(θ_i).
 * as for the plain TTT-Linear scan, the b outputs of mini-batch i are o_t = f(q_t; θ_i) and
   the per-token loss is L_t = ‖f(k_t; θ_i) − v_t‖².
+* per-token weights (``token_weights=True``, the TTT layer's mini-batch form in which each token
+  sees the gradient steps of the tokens before it and its own): output t of mini-batch i uses
+  θ_t = θ_i − (η/b)·Σ_{s ≤ t} ∇(½‖f(k_s; θ_i) − v_s‖²), every gradient taken at θ_i, so the
+  last token of the mini-batch sees θ_{i+1}; losses and the weight update are unchanged.
 
 The gradients are written out by the chain rule, one layer at a time; the pins check them
 against central differences of the loss.
@@ -80,7 +84,7 @@ def _check(Kd, b):
         raise ValueError("T must be a multiple of the inner mini-batch b")
 
 
-def ttt_linear_ln_scan(K, V, Q, W0, gamma, beta, eta: float, b: int, eps: float):
+def ttt_linear_ln_scan(K, V, Q, W0, gamma, beta, eta: float, b: int, eps: float, token_weights: bool = False):
     """TTT-Linear with LayerNorm and residual over every (sequence, head) of [B, H, T, D]
     inputs; W0 [B, H, D, D], gamma and beta [H, D].
 
@@ -98,18 +102,24 @@ def ttt_linear_ln_scan(K, V, Q, W0, gamma, beta, eta: float, b: int, eps: float)
     for i in range(T // b):
         s = slice(i * b, (i + 1) * b)
         Ki, Vi = Kf[:, s], Vf[:, s]
-        if Qf is not None:
+        if Qf is not None and not token_weights:
             O[:, s] = Qf[:, s] + layer_norm(Qf[:, s] @ W, gam, bet, eps)[0]  # f(q; W_i)
         Y, zhat, rstd = layer_norm(Ki @ W, gam, bet, eps)
         E = Ki + Y - Vi                                    # f(k) − v
         loss[:, s] = np.sum(E * E, axis=2)
         dZ = layer_norm_backward(E, zhat, rstd, gam)       # ∂(½‖f(k) − v‖²)/∂(k·W)
+        if Qf is not None and token_weights:
+            for j in range(b):                             # token j sees the steps of tokens 0..j
+                Wt = W - (eta / b) * (np.swapaxes(Ki[:, :j + 1], 1, 2) @ dZ[:, :j + 1])
+                t = i * b + j
+                O[:, t:t + 1] = Qf[:, t:t + 1] + layer_norm(Qf[:, t:t + 1] @ Wt, gam, bet, eps)[0]
         W = W - (eta / b) * (np.swapaxes(Ki, 1, 2) @ dZ)   # one gradient step on ℓ_i
     O = None if O is None else O.reshape(B, H, T, D)
     return O, W.reshape(B, H, D, D), loss.reshape(B, H, T)
 
 
-def ttt_mlp_scan(K, V, Q, W1_0, W2_0, gamma, beta, eta: float, b: int, eps: float, activation: str = "gelu"):
+def ttt_mlp_scan(K, V, Q, W1_0, W2_0, gamma, beta, eta: float, b: int, eps: float, activation: str = "gelu",
+                 token_weights: bool = False):
     """TTT-MLP over every (sequence, head) of [B, H, T, D] inputs; W1_0 [B, H, D, Dh],
     W2_0 [B, H, Dh, D], gamma and beta [H, D].
 
@@ -130,7 +140,7 @@ def ttt_mlp_scan(K, V, Q, W1_0, W2_0, gamma, beta, eta: float, b: int, eps: floa
     for i in range(T // b):
         s = slice(i * b, (i + 1) * b)
         Ki, Vi = Kf[:, s], Vf[:, s]
-        if Qf is not None:
+        if Qf is not None and not token_weights:
             O[:, s] = Qf[:, s] + layer_norm(act(Qf[:, s] @ W1) @ W2, gam, bet, eps)[0]
         Hpre = Ki @ W1                                     # hidden pre-activation [b, Dh]
         A = act(Hpre)
@@ -141,6 +151,12 @@ def ttt_mlp_scan(K, V, Q, W1_0, W2_0, gamma, beta, eta: float, b: int, eps: floa
         dW2 = np.swapaxes(A, 1, 2) @ dZ
         dH = (dZ @ np.swapaxes(W2, 1, 2)) * act_grad(Hpre)  # back through W2 and the activation
         dW1 = np.swapaxes(Ki, 1, 2) @ dH
+        if Qf is not None and token_weights:
+            for j in range(b):                             # token j sees the steps of tokens 0..j
+                W1t = W1 - (eta / b) * (np.swapaxes(Ki[:, :j + 1], 1, 2) @ dH[:, :j + 1])
+                W2t = W2 - (eta / b) * (np.swapaxes(A[:, :j + 1], 1, 2) @ dZ[:, :j + 1])
+                t = i * b + j
+                O[:, t:t + 1] = Qf[:, t:t + 1] + layer_norm(act(Qf[:, t:t + 1] @ W1t) @ W2t, gam, bet, eps)[0]
         W1 = W1 - (eta / b) * dW1
         W2 = W2 - (eta / b) * dW2
     O = None if O is None else O.reshape(B, H, T, D)

@@ -227,3 +227,64 @@ def test_outputs_and_losses_evaluate_the_same_model():
     np.testing.assert_allclose(np.sum((O - V) ** 2, axis=3), L, rtol=1e-12)
     assert abs(L[0, 0, :b].sum() - 2 * b * inner.inner_loss_mlp(K[0, 0, :b], V[0, 0, :b], W1[0, 0], W2[0, 0], g[0],
                                                                 be[0], 1e-5)) < 1e-10
+
+
+def _shifted_queries(Q, positions, sources):
+    """Q with the rows at ``positions`` replaced by the rows at ``sources``."""
+    Q2 = Q.copy()
+    Q2[..., positions, :] = Q[..., sources, :]
+    return Q2
+
+
+def test_token_weights_last_token_sees_the_next_minibatch_weight():
+    """With per-token weights the last token of mini-batch i has taken every step of it, so its
+    output is the output the plain scan gives a query equal to it at the first token of
+    mini-batch i + 1 (whose weight is θ_{i+1})."""
+    B, H, T, D, b = 1, 2, 24, 6, 4
+    K, V, Q = _rand((B, H, T, D), 67), _rand((B, H, T, D), 68), _rand((B, H, T, D), 69)
+    W0 = _rand((B, H, D, D), 70, 0.5)
+    W1, W2 = _rand((B, H, D, 4 * D), 71, 0.5), _rand((B, H, 4 * D, D), 72, 0.5)
+    g, be = _rand((H, D), 73) + 1.0, _rand((H, D), 74)
+    last = np.arange(b - 1, T - b, b)
+    Q2 = _shifted_queries(Q, last + 1, last)
+    O_tw = inner.ttt_linear_ln_scan(K, V, Q, W0, g, be, 0.3, b, 1e-4, token_weights=True)[0]
+    O_pl = inner.ttt_linear_ln_scan(K, V, Q2, W0, g, be, 0.3, b, 1e-4)[0]
+    np.testing.assert_allclose(O_tw[..., last, :], O_pl[..., last + 1, :], rtol=1e-11, atol=1e-11)
+    O_tw = inner.ttt_mlp_scan(K, V, Q, W1, W2, g, be, 0.3, b, 1e-4, token_weights=True)[0]
+    O_pl = inner.ttt_mlp_scan(K, V, Q2, W1, W2, g, be, 0.3, b, 1e-4)[0]
+    np.testing.assert_allclose(O_tw[..., last, :], O_pl[..., last + 1, :], rtol=1e-11, atol=1e-11)
+
+
+def test_token_weights_first_token_takes_only_its_own_step():
+    """The first token of a mini-batch sees θ_i − (η/b)·∇ of its own loss alone: the weight a
+    plain scan with mini-batch 1 and step η/b reaches after that one token."""
+    B, H, D, b, eta = 1, 2, 6, 4, 0.3
+    K, V, Q = _rand((B, H, b, D), 75), _rand((B, H, b, D), 76), _rand((B, H, b, D), 77)
+    W0 = _rand((B, H, D, D), 78, 0.5)
+    W1, W2 = _rand((B, H, D, 4 * D), 79, 0.5), _rand((B, H, 4 * D, D), 80, 0.5)
+    g, be = _rand((H, D), 81) + 1.0, _rand((H, D), 82)
+    # Two-token plain scans with mini-batch 1: token 0 steps, token 1 carries the query.
+    K2 = np.concatenate([K[..., :1, :], K[..., :1, :]], axis=2)
+    V2 = np.concatenate([V[..., :1, :], V[..., :1, :]], axis=2)
+    Q2 = np.concatenate([Q[..., :1, :], Q[..., :1, :]], axis=2)
+    O_tw = inner.ttt_linear_ln_scan(K, V, Q, W0, g, be, eta, b, 1e-4, token_weights=True)[0]
+    O_pl = inner.ttt_linear_ln_scan(K2, V2, Q2, W0, g, be, eta / b, 1, 1e-4)[0]
+    np.testing.assert_allclose(O_tw[..., 0, :], O_pl[..., 1, :], rtol=1e-11, atol=1e-11)
+    O_tw = inner.ttt_mlp_scan(K, V, Q, W1, W2, g, be, eta, b, 1e-4, token_weights=True)[0]
+    O_pl = inner.ttt_mlp_scan(K2, V2, Q2, W1, W2, g, be, eta / b, 1, 1e-4)[0]
+    np.testing.assert_allclose(O_tw[..., 0, :], O_pl[..., 1, :], rtol=1e-11, atol=1e-11)
+
+
+def test_token_weights_change_only_the_outputs():
+    """Losses and the final weights do not depend on how the outputs are taken; with mini-batch
+    1 the two forms differ by exactly one step (checked above), with larger ones the middle
+    tokens differ from both ends."""
+    B, H, T, D, b = 1, 1, 16, 5, 8
+    K, V, Q = _rand((B, H, T, D), 83), _rand((B, H, T, D), 84), _rand((B, H, T, D), 85)
+    W0 = _rand((B, H, D, D), 86, 0.5)
+    g, be = _rand((H, D), 87) + 1.0, _rand((H, D), 88)
+    Oa, Wa, La = inner.ttt_linear_ln_scan(K, V, Q, W0, g, be, 0.3, b, 1e-4)
+    Ob, Wb, Lb = inner.ttt_linear_ln_scan(K, V, Q, W0, g, be, 0.3, b, 1e-4, token_weights=True)
+    np.testing.assert_array_equal(Wa, Wb)
+    np.testing.assert_array_equal(La, Lb)
+    assert np.abs(Oa - Ob).max() > 1e-3

@@ -121,21 +121,18 @@ MUTANTS = [
     ("inner", "TTT-Linear step with the wrong sign",
      [("W = W - (eta / b) * (np.swapaxes(Ki, 1, 2) @ dZ)", "W = W + (eta / b) * (np.swapaxes(Ki, 1, 2) @ dZ)")]),
     ("inner", "TTT-Linear outputs from the weight after the step",
-     [("        if Qf is not None:\n"
+     [("        if Qf is not None and not token_weights:\n"
        "            O[:, s] = Qf[:, s] + layer_norm(Qf[:, s] @ W, gam, bet, eps)[0]  # f(q; W_i)\n", ""),
       ("        W = W - (eta / b) * (np.swapaxes(Ki, 1, 2) @ dZ)   # one gradient step on ℓ_i\n",
        "        W = W - (eta / b) * (np.swapaxes(Ki, 1, 2) @ dZ)\n"
-       "        if Qf is not None:\n"
+       "        if Qf is not None and not token_weights:\n"
        "            O[:, s] = Qf[:, s] + layer_norm(Qf[:, s] @ W, gam, bet, eps)[0]\n")]),
     ("inner", "MLP first layer's gradient taken through the updated second layer",
-     [("        dH = (dZ @ np.swapaxes(W2, 1, 2)) * act_grad(Hpre)  # back through W2 and the activation\n"
-       "        dW1 = np.swapaxes(Ki, 1, 2) @ dH\n"
-       "        W1 = W1 - (eta / b) * dW1\n"
-       "        W2 = W2 - (eta / b) * dW2\n",
+     [("        W1 = W1 - (eta / b) * dW1\n        W2 = W2 - (eta / b) * dW2\n",
+       "        W1 = W1 - (eta / b) * dW1\n"),
+      ("        dH = (dZ @ np.swapaxes(W2, 1, 2)) * act_grad(Hpre)  # back through W2 and the activation\n",
        "        W2 = W2 - (eta / b) * dW2\n"
-       "        dH = (dZ @ np.swapaxes(W2, 1, 2)) * act_grad(Hpre)\n"
-       "        dW1 = np.swapaxes(Ki, 1, 2) @ dH\n"
-       "        W1 = W1 - (eta / b) * dW1\n")]),
+       "        dH = (dZ @ np.swapaxes(W2, 1, 2)) * act_grad(Hpre)\n")]),
     ("inner", "GELU derivative without the density term",
      [(" + x * np.exp(-0.5 * x * x) / np.sqrt(2.0 * np.pi)", "")]),
     ("inner", "second layer's gradient from the pre-activation",
@@ -143,6 +140,14 @@ MUTANTS = [
     ("inner", "MLP outputs without the activation",
      [("O[:, s] = Qf[:, s] + layer_norm(act(Qf[:, s] @ W1) @ W2, gam, bet, eps)[0]",
        "O[:, s] = Qf[:, s] + layer_norm((Qf[:, s] @ W1) @ W2, gam, bet, eps)[0]")]),
+    ("inner", "per-token weights without the token's own step",
+     [("Wt = W - (eta / b) * (np.swapaxes(Ki[:, :j + 1], 1, 2) @ dZ[:, :j + 1])",
+       "Wt = W - (eta / b) * (np.swapaxes(Ki[:, :j], 1, 2) @ dZ[:, :j])")]),
+    ("inner", "per-token weights that see the next token's step",
+     [("Wt = W - (eta / b) * (np.swapaxes(Ki[:, :j + 1], 1, 2) @ dZ[:, :j + 1])",
+       "Wt = W - (eta / b) * (np.swapaxes(Ki[:, :j + 2], 1, 2) @ dZ[:, :j + 2])")]),
+    ("inner", "MLP per-token weights with the second layer left at the mini-batch's start",
+     [("W2t = W2 - (eta / b) * (np.swapaxes(A[:, :j + 1], 1, 2) @ dZ[:, :j + 1])", "W2t = W2")]),
     ("inner", "GELU from the wrong distribution scale",
      [("return 0.5 * x * (1.0 + erf(x / np.sqrt(2.0)))", "return 0.5 * x * (1.0 + erf(x))")]),
 ]
