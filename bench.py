@@ -112,7 +112,8 @@ class Runner:
         self.device = device
         if isinstance(spec, wl.InnerSpec):
             x = wl.inner_inputs(spec, device=device)
-            cfg = cwl.config(spec.model, batch=spec.B, heads=spec.H, eta=spec.eta, ln_eps=spec.eps)
+            cfg = cwl.config(spec.model, batch=spec.B, heads=spec.H, eta=spec.eta, ln_eps=spec.eps,
+                             token_weights=int(spec.token_weights))
             self.state = cwl.FastWeightState(cfg, x["W0"])
             self.state.set_layernorm(x["gamma"], x["beta"])
             args = dict(keys=x["K"], targets=x["V"], queries=x.get("Q"))
@@ -372,10 +373,11 @@ def cpu_baseline(spec, limit_s=12.0, prefix=False) -> dict:
             gh, bh_ = g[h % spec.H:h % spec.H + 1], be[h % spec.H:h % spec.H + 1]
             if spec.model == "linear_ln":
                 oinn.ttt_linear_ln_scan(K[hs], V[hs], Q[hs], x["W0"].reshape(BH, 1, spec.D, spec.D)[hs], gh, bh_,
-                                        spec.eta, spec.b, spec.eps)
+                                        spec.eta, spec.b, spec.eps, token_weights=spec.token_weights)
             else:
                 oinn.ttt_mlp_scan(K[hs], V[hs], Q[hs], x["W1"].reshape(BH, 1, spec.D, spec.hidden)[hs],
-                                  x["W2"].reshape(BH, 1, spec.hidden, spec.D)[hs], gh, bh_, spec.eta, spec.b, spec.eps)
+                                  x["W2"].reshape(BH, 1, spec.hidden, spec.D)[hs], gh, bh_, spec.eta, spec.b, spec.eps,
+                                  token_weights=spec.token_weights)
             done_heads += 1
         dt = time.perf_counter() - t0
         tokens = spec.T * done_heads / spec.H

@@ -59,6 +59,7 @@ class ttt_config(ctypes.Structure):
         ("gate_mean_num", ctypes.c_int32),
         ("gate_mean_den", ctypes.c_int32),
         ("ln_eps", ctypes.c_float),
+        ("token_weights", ctypes.c_int32),
     ]
 
 

@@ -134,6 +134,40 @@ struct __align__(1024) LnSmem {
   int cabort[2];          // set by a compute warp whose wait for tile s ran out (index s & 1)
 };
 
+// Per-warp LayerNorm statistics of the keys' (z) and, with QUERIES, the queries' (o) products
+// of a step (Zᵀ layout: this thread holds columns g, g+8 of tokens 8nt + 2q + jj): two-pass over
+// the warp's sixteen columns, published as (sum, M2) in fwd[kind][token][warp] and [4 + warp].
+// KEYS = false publishes the queries' statistics alone (the keys' slots are left untouched).
+template <bool QUERIES, bool KEYS = true>
+__device__ __forceinline__ void publish_stats(const float (&z)[2][4], const float (&o)[2][4],
+                                              float (*fwd)[kMB][8], int pub_tok, int warp, int g) {
+  float v8[8], all[8];
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+    for (int jj = 0; jj < 2; ++jj) {
+      v8[2 * nt + jj] = KEYS ? z[nt][jj] + z[nt][jj + 2] : 0.f;
+      v8[4 + 2 * nt + jj] = QUERIES ? o[nt][jj] + o[nt][jj + 2] : 0.f;
+    }
+  const float sw = reduce_scatter8(v8, g);
+  all_gather8(sw, all, g);
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+    for (int jj = 0; jj < 2; ++jj) {
+      const float mz = all[2 * nt + jj] * (1.f / 16.f), mo = all[4 + 2 * nt + jj] * (1.f / 16.f);
+      const float a = z[nt][jj] - mz, b = z[nt][jj + 2] - mz, c = o[nt][jj] - mo, d = o[nt][jj + 2] - mo;
+      v8[2 * nt + jj] = KEYS ? a * a + b * b : 0.f;
+      v8[4 + 2 * nt + jj] = QUERIES ? c * c + d * d : 0.f;
+    }
+  const float m2w = reduce_scatter8(v8, g);
+  const int kind = g >> 2;
+  if ((kind == 0 && KEYS) || (kind == 1 && QUERIES)) {
+    fwd[kind][pub_tok][warp] = sw;
+    fwd[kind][pub_tok][4 + warp] = m2w;
+  }
+}
+
 // Per-token mean and 1/sqrt(var + ε) from four warps' (sum, M2) over sixteen columns each.
 __device__ __forceinline__ void merge_stats(const float* p, float eps, float& mu, float& rstd) {
   const float4 S = *reinterpret_cast<const float4*>(p);
@@ -145,7 +179,33 @@ __device__ __forceinline__ void merge_stats(const float* p, float eps, float& mu
   rstd = rsqrtf(m2 * (1.f / 64.f) + eps);
 }
 
-template <bool HAS_Q, bool LOSS>
+// TW: per-token weights within the mini-batch. Token t's output uses
+// W_t = W_i + Σ_{s ≤ t} k_sᵀ·S_s (S = −(η/b)·∂ℓ/∂Z, every gradient at W_i), so
+// q_t·W_t = q_t·W_i + Σ_{s ≤ t} (q_t·k_s)·S_s: the query products of the forward pass plus
+// Sᵀ·Mᵀ with M = Q·Kᵀ masked to s ≤ t, added once S is known; the outputs' LayerNorm
+// statistics then take a third exchange.
+// Outputs q + γ·LN(o) + β of the step's sixteen tokens at this thread's two columns, from the
+// queries' merged statistics, into the swizzled staging tile.
+__device__ __forceinline__ void emit_outputs(const float (&o)[2][4], const float (&qv)[2][4], const float (*st)[8],
+                                             const float (&gam)[2], const float (&bet)[2], float eps, uint8_t* obuf,
+                                             int r0, int col0, int g, int q) {
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+    for (int jj = 0; jj < 2; ++jj) {
+      const int tok = 8 * nt + 2 * q + jj;
+      float mu, rstd;
+      merge_stats(st[tok], eps, mu, rstd);
+#pragma unroll
+      for (int hc = 0; hc < 2; ++hc) {
+        const int e = jj + 2 * hc;
+        const float y = qv[nt][e] + fmaf(gam[hc], (o[nt][e] - mu) * rstd, bet[hc]);
+        *reinterpret_cast<__nv_bfloat16*>(obuf + swz128_bf16(r0 + tok, col0 + g + 8 * hc)) = __float2bfloat16_rn(y);
+      }
+    }
+}
+
+template <bool HAS_Q, bool LOSS, bool TW>
 __global__ void __launch_bounds__(kLnThreads, 1)
     k_inner_ln(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
@@ -226,6 +286,14 @@ __global__ void __launch_bounds__(kLnThreads, 1)
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks) afrag_hilo(acc[2 * ks], acc[2 * ks + 1], whi[ks], wlo[ks]);
       float z[2][4], o[2][4];
+      // TW: M = Q·Kᵀ (tokens x tokens), mm[nt][e] = M[g + 8(e>>1)][8nt + 2q + (e&1)]; Q as the A
+      // operand, the K fragments of the forward product as B.
+      uint32_t qa[4][4];
+      float mm[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      if (TW) {
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) ldsm4(qbase + swz128_bf16(r0 + 8 * (mi & 1) + ri, 16 * ks + 8 * (mi >> 1)), qa[ks]);
+      }
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt) {
         float z2[4] = {0.f, 0.f, 0.f, 0.f}, o2[4] = {0.f, 0.f, 0.f, 0.f};
@@ -240,6 +308,10 @@ __global__ void __launch_bounds__(kLnThreads, 1)
           mma_bf16(z2, wlo[ks], kb[0], kb[1]);
           mma_bf16(z[nt], whi[ks + 1], kb[2], kb[3]);
           mma_bf16(z2, wlo[ks + 1], kb[2], kb[3]);
+          if (TW) {
+            mma_bf16(mm[nt], qa[ks], kb[0], kb[1]);
+            mma_bf16(mm[nt], qa[ks + 1], kb[2], kb[3]);
+          }
           if (HAS_Q) {
             uint32_t qb[4];
             ldsm4(qbase + off, qb);
@@ -285,29 +357,10 @@ __global__ void __launch_bounds__(kLnThreads, 1)
         }
       }
 
-      // ---- LayerNorm statistics: per warp two-pass over its sixteen columns, then merged
-      float v8[8], all[8];
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int jj = 0; jj < 2; ++jj) {
-          v8[2 * nt + jj] = z[nt][jj] + z[nt][jj + 2];
-          v8[4 + 2 * nt + jj] = o[nt][jj] + o[nt][jj + 2];
-        }
-      const float sw = reduce_scatter8(v8, g);
-      all_gather8(sw, all, g);
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int jj = 0; jj < 2; ++jj) {
-          const float mz = all[2 * nt + jj] * (1.f / 16.f), mo = all[4 + 2 * nt + jj] * (1.f / 16.f);
-          const float a = z[nt][jj] - mz, b = z[nt][jj + 2] - mz, c = o[nt][jj] - mo, d = o[nt][jj + 2] - mo;
-          v8[2 * nt + jj] = a * a + b * b;
-          v8[4 + 2 * nt + jj] = c * c + d * d;
-        }
-      const float m2w = reduce_scatter8(v8, g);
-      sm.fwd[g >> 2][pub_tok][warp] = sw;
-      sm.fwd[g >> 2][pub_tok][4 + warp] = m2w;
+      // ---- LayerNorm statistics: per warp two-pass over its sixteen columns, then merged. The
+      // queries' share here unless TW (their products are not complete before the backward).
+      constexpr bool kOutNow = HAS_Q && !TW;
+      publish_stats<kOutNow>(z, o, sm.fwd, pub_tok, warp, g);
       compute_sync<kLnWarps>();
 
       float zh[2][4], ev[2][4], gg[2][4], rz[2][2];
@@ -326,18 +379,11 @@ __global__ void __launch_bounds__(kLnThreads, 1)
             ev[nt][e] = fmaf(gam[hc], zh[nt][e], bet[hc]) + kv[nt][e];  // f(k) − v
             gg[nt][e] = gam[hc] * ev[nt][e];
           }
-          if (HAS_Q) {
-            merge_stats(sm.fwd[1][tok], eps, mu, rstd);
-#pragma unroll
-            for (int hc = 0; hc < 2; ++hc) {
-              const int e = jj + 2 * hc;
-              const float y = qv[nt][e] + fmaf(gam[hc], (o[nt][e] - mu) * rstd, bet[hc]);
-              *reinterpret_cast<__nv_bfloat16*>(obuf + swz128_bf16(r0 + tok, col0 + g + 8 * hc)) = __float2bfloat16_rn(y);
-            }
-          }
         }
+      if (kOutNow) emit_outputs(o, qv, sm.fwd[1], gam, bet, eps, obuf, r0, col0, g, q);
 
       // ---- backward statistics: Σg and Σg·ẑ per token (and Σe² for the loss)
+      float v8[8];
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
@@ -391,6 +437,28 @@ __global__ void __launch_bounds__(kLnThreads, 1)
         mma_bf16(acc[nt], slo, kb[0], kb[1]);
         mma_bf16(acc[nt + 1], shi, kb[2], kb[3]);
         mma_bf16(acc[nt + 1], slo, kb[2], kb[3]);
+      }
+      if (HAS_Q && TW) {
+        // Pᵀ += Sᵀ·Mᵀ, M masked to s ≤ t. The Mᵀ B fragment of token n-tile nt (t = 8nt + g)
+        // holds M[t][2q, 2q+1] and M[t][8 + 2q, 9 + 2q]: the accumulator values of row t.
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          const int t = 8 * nt + g;
+          const float m00 = 2 * q <= t ? mm[0][2 * nt] : 0.f, m01 = 2 * q + 1 <= t ? mm[0][2 * nt + 1] : 0.f;
+          const float m10 = 2 * q + 8 <= t ? mm[1][2 * nt] : 0.f, m11 = 2 * q + 9 <= t ? mm[1][2 * nt + 1] : 0.f;
+          uint32_t bh0, bl0, bh1, bl1;
+          hilo2(m00, m01, bh0, bl0);
+          hilo2(m10, m11, bh1, bl1);
+          float o2[4] = {0.f, 0.f, 0.f, 0.f};
+          mma_bf16(o[nt], shi, bh0, bh1);
+          mma_bf16(o2, shi, bl0, bl1);
+          mma_bf16(o2, slo, bh0, bh1);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) o[nt][e] += o2[e];
+        }
+        publish_stats<true, false>(z, o, sm.fwd, pub_tok, warp, g);
+        compute_sync<kLnWarps>();
+        emit_outputs(o, qv, sm.fwd[1], gam, bet, eps, obuf, r0, col0, g, q);
       }
     }
     // End of the tile: its outputs are complete in shared memory.
@@ -489,7 +557,13 @@ __device__ __forceinline__ void store4_bf16(uint8_t* tile, int row, int col, con
   *reinterpret_cast<uint2*>(tile + swz128_bf16(row, col)) = make_uint2(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]));
 }
 
-template <bool HAS_Q, bool LOSS>
+// TW: per-token weights within the mini-batch. With every gradient at the step's starting
+// weights, W1_t = W1_i + Σ_{s ≤ t} k_sᵀ·dH_s and W2_t = W2_i + Σ_{s ≤ t} a_sᵀ·S_s (dH and S carry
+// −η/b), so the queries' first layer is Q·W1_i + tril(Q·Kᵀ)·dH and their second layer
+// A_q·W2_i + tril(A_q·Aᵀ)·S. The second Gram matrix splits over the hidden slices like the
+// product itself, so each warp adds its slice's term to its partial Zᵀ; the queries' path runs
+// after the backward, and their LayerNorm behind a third barrier.
+template <bool HAS_Q, bool LOSS, bool TW>
 __global__ void __launch_bounds__(kMlpThreads, 1)
     k_inner_mlp(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                 const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
@@ -566,8 +640,12 @@ __global__ void __launch_bounds__(kMlpThreads, 1)
     uint8_t* obuf = sm.O[s & 1];
 
     for (int r0 = 0; r0 < ntok; r0 += kMB) {
+      constexpr bool kQNow = HAS_Q && !TW;  // the queries' path alongside the keys'
       // ---- first layer: Hᵀ = W1ᵀ·Kᵀ (and for the queries), hidden x tokens
       float hk[2][2][4], hq[2][2][4];
+      // TW: M = Q·Kᵀ, mm[nt][e] = M[g + 8(e>>1)][8nt + 2q + (e&1)] (Q as the A operand, the K
+      // fragments of the first layer as B).
+      float mm[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
       for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
@@ -582,6 +660,15 @@ __global__ void __launch_bounds__(kMlpThreads, 1)
           const uint32_t off = swz128_bf16(r0 + 8 * nt + ri, 16 * ks + 8 * mi);
           ldsm4(kbase + off, kb[nt]);
           if (HAS_Q) ldsm4(qbase + off, qb[nt]);
+        }
+        if (TW) {
+#pragma unroll
+          for (int kk = 0; kk < 2; ++kk) {
+            uint32_t qa[4];
+            ldsm4(qbase + swz128_bf16(r0 + 8 * (mi & 1) + ri, 16 * (ks + kk) + 8 * (mi >> 1)), qa);
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) mma_bf16(mm[nt], qa, kb[nt][2 * kk], kb[nt][2 * kk + 1]);
+          }
         }
 #pragma unroll
         for (int mt = 0; mt < 2; ++mt) {
@@ -613,11 +700,11 @@ __global__ void __launch_bounds__(kMlpThreads, 1)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             gelu_and_grad(hk[mt][nt][e], y[e], dact[mt][nt][e]);
-            if (HAS_Q) gelu_and_grad(hq[mt][nt][e], yq[e], dq);
+            if (kQNow) gelu_and_grad(hq[mt][nt][e], yq[e], dq);
           }
           ak[mt][nt][0] = pack_bf16(y[0], y[1]);
           ak[mt][nt][1] = pack_bf16(y[2], y[3]);
-          if (HAS_Q) {
+          if (kQNow) {
             aq[mt][nt][0] = pack_bf16(yq[0], yq[1]);
             aq[mt][nt][1] = pack_bf16(yq[2], yq[3]);
           }
@@ -633,7 +720,7 @@ __global__ void __launch_bounds__(kMlpThreads, 1)
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
               bk[nt][ks][hh] = movm_t(ak[ks][nt][hh]);
-              if (HAS_Q) bq[nt][ks][hh] = movm_t(aq[ks][nt][hh]);
+              if (kQNow) bq[nt][ks][hh] = movm_t(aq[ks][nt][hh]);
             }
 #pragma unroll
         for (int mt = 0; mt < 4; ++mt) {
@@ -641,7 +728,7 @@ __global__ void __launch_bounds__(kMlpThreads, 1)
           afrag_hilo(a2[mt][0], a2[mt][1], whi[0], wlo[0]);
           afrag_hilo(a2[mt][2], a2[mt][3], whi[1], wlo[1]);
 #pragma unroll
-          for (int kind = 0; kind < (HAS_Q ? 2 : 1); ++kind) {
+          for (int kind = 0; kind < (kQNow ? 2 : 1); ++kind) {
             float* red = &sm.red[kind][warp][0][0];
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt) {
@@ -698,23 +785,25 @@ __global__ void __launch_bounds__(kMlpThreads, 1)
           se = sum16(se);
           if ((lane & 15) == 0) loss[(size_t)bh * T + (size_t)s * kTileTokI + r0 + ltok] = se;
         }
-        if (HAS_Q) {
-          float zq[4] = {0.f, 0.f, 0.f, 0.f}, qh[4], qr, qx[4], y[4];
-#pragma unroll
-          for (int p = 0; p < kMlpWarps; ++p) {
-            const float4 v = *reinterpret_cast<const float4*>(&sm.red[1][p][ltok][c0]);
-            zq[0] += v.x;
-            zq[1] += v.y;
-            zq[2] += v.z;
-            zq[3] += v.w;
-          }
-          ln16(zq, eps, qh, qr);
-          load4_bf16(Qt, r0 + ltok, c0, qx);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) y[i] = qx[i] + fmaf(gam[i], qh[i], bet[i]);
-          store4_bf16(obuf, r0 + ltok, c0, y);
-        }
       }
+      // Outputs of tokens 2w, 2w+1: q + γ·LN(Σ partial Zᵀ of the queries) + β.
+      auto query_outputs = [&]() {
+        float zq[4] = {0.f, 0.f, 0.f, 0.f}, qh[4], qr, qx[4], y[4];
+#pragma unroll
+        for (int p = 0; p < kMlpWarps; ++p) {
+          const float4 v = *reinterpret_cast<const float4*>(&sm.red[1][p][ltok][c0]);
+          zq[0] += v.x;
+          zq[1] += v.y;
+          zq[2] += v.z;
+          zq[3] += v.w;
+        }
+        ln16(zq, eps, qh, qr);
+        load4_bf16(Qt, r0 + ltok, c0, qx);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) y[i] = qx[i] + fmaf(gam[i], qh[i], bet[i]);
+        store4_bf16(obuf, r0 + ltok, c0, y);
+      };
+      if (kQNow) query_outputs();
       compute_sync<kMlpWarps>();
 
       // ---- backward, every warp for its hidden slice; gradients at the step's starting weights
@@ -750,32 +839,124 @@ __global__ void __launch_bounds__(kMlpThreads, 1)
           }
         }
       }
-      // W1ᵀ += dHᵀ·K (S already carries −η/b).
+      // dHᵀ = dh ⊙ GELU'(H) as A fragments (hidden x tokens), S already carrying −η/b.
+      uint32_t da[2][4];
 #pragma unroll
       for (int mt = 0; mt < 2; ++mt) {
-        uint32_t da[4];
-        da[0] = pack_bf16(dh[mt][0][0] * dact[mt][0][0], dh[mt][0][1] * dact[mt][0][1]);
-        da[1] = pack_bf16(dh[mt][0][2] * dact[mt][0][2], dh[mt][0][3] * dact[mt][0][3]);
-        da[2] = pack_bf16(dh[mt][1][0] * dact[mt][1][0], dh[mt][1][1] * dact[mt][1][1]);
-        da[3] = pack_bf16(dh[mt][1][2] * dact[mt][1][2], dh[mt][1][3] * dact[mt][1][3]);
+        da[mt][0] = pack_bf16(dh[mt][0][0] * dact[mt][0][0], dh[mt][0][1] * dact[mt][0][1]);
+        da[mt][1] = pack_bf16(dh[mt][0][2] * dact[mt][0][2], dh[mt][0][3] * dact[mt][0][3]);
+        da[mt][2] = pack_bf16(dh[mt][1][0] * dact[mt][1][0], dh[mt][1][1] * dact[mt][1][1]);
+        da[mt][3] = pack_bf16(dh[mt][1][2] * dact[mt][1][2], dh[mt][1][3] * dact[mt][1][3]);
+      }
+      if (HAS_Q && TW) {
+        // Queries' first layer (from the forward pass): Hqᵀ += dHᵀ·Mᵀ with M masked to s ≤ t (the
+        // Mᵀ B fragment of token n-tile nt holds row t = 8nt + g of M).
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          const int t = 8 * nt + g;
+          const float m00 = 2 * q <= t ? mm[0][2 * nt] : 0.f, m01 = 2 * q + 1 <= t ? mm[0][2 * nt + 1] : 0.f;
+          const float m10 = 2 * q + 8 <= t ? mm[1][2 * nt] : 0.f, m11 = 2 * q + 9 <= t ? mm[1][2 * nt + 1] : 0.f;
+          uint32_t bh0, bl0, bh1, bl1;
+          hilo2(m00, m01, bh0, bl0);
+          hilo2(m10, m11, bh1, bl1);
+#pragma unroll
+          for (int mt = 0; mt < 2; ++mt) {
+            mma_bf16(hq[mt][nt], da[mt], bh0, bh1);
+            mma_bf16(hq[mt][nt], da[mt], bl0, bl1);
+          }
+        }
+      }
+      // W1ᵀ += dHᵀ·K.
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt) {
 #pragma unroll
         for (int nt = 0; nt < 8; nt += 2) {
           uint32_t kb[4];
           ldsm4_t(kbase + swz128_bf16(r0 + 8 * (mi & 1) + ri, 8 * nt + 8 * (mi >> 1)), kb);
-          mma_bf16(a1[mt][nt], da, kb[0], kb[1]);
-          mma_bf16(a1[mt][nt + 1], da, kb[2], kb[3]);
+          mma_bf16(a1[mt][nt], da[mt], kb[0], kb[1]);
+          mma_bf16(a1[mt][nt + 1], da[mt], kb[2], kb[3]);
         }
       }
-      // W2ᵀ += Sᵀ·A: Sᵀ as the A operand (columns x tokens), A (tokens x hidden) as B.
+      // TW: the queries' activation, their Gram matrix with the keys' over this warp's hidden
+      // slice, gw[nt][e] = G[g + 8(e>>1)][8nt + 2q + (e&1)] with G = A_q·Aᵀ, and its Mᵀ-style B
+      // fragments (masked to s ≤ t, hi and lo).
+      uint32_t gbh[2][2], gbl[2][2];
+      uint32_t bq[2][2][2];  // the queries' Aᵀ B fragments: [token n-tile][hidden k-step][half]
+      if (HAS_Q && TW) {
+        uint32_t bk[2][2][2];
 #pragma unroll
-      for (int mt = 0; mt < 4; ++mt)
+        for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-        for (int p = 0; p < 2; ++p) {
-          uint32_t sa[4];
-          ldsm4_t(sbase[p] + swz128_bf16(8 * (mi >> 1) + ri, 16 * mt + 8 * (mi & 1)), sa);
+          for (int nt = 0; nt < 2; ++nt) {
+            float yq[4], dq;
 #pragma unroll
-          for (int j = 0; j < 4; ++j) mma_bf16(a2[mt][j], sa, ak[j >> 1][0][j & 1], ak[j >> 1][1][j & 1]);
+            for (int e = 0; e < 4; ++e) gelu_and_grad(hq[mt][nt][e], yq[e], dq);
+            aq[mt][nt][0] = pack_bf16(yq[0], yq[1]);
+            aq[mt][nt][1] = pack_bf16(yq[2], yq[3]);
+          }
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int ks = 0; ks < 2; ++ks)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              bq[nt][ks][hh] = movm_t(aq[ks][nt][hh]);
+              bk[nt][ks][hh] = movm_t(ak[ks][nt][hh]);
+            }
+        float gw[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks) {
+          const uint32_t a[4] = {bq[0][ks][0], bq[1][ks][0], bq[0][ks][1], bq[1][ks][1]};  // A_q rows t
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt) mma_bf16(gw[nt], a, bk[nt][ks][0], bk[nt][ks][1]);
         }
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          const int t = 8 * nt + g;
+          const float g00 = 2 * q <= t ? gw[0][2 * nt] : 0.f, g01 = 2 * q + 1 <= t ? gw[0][2 * nt + 1] : 0.f;
+          const float g10 = 2 * q + 8 <= t ? gw[1][2 * nt] : 0.f, g11 = 2 * q + 9 <= t ? gw[1][2 * nt + 1] : 0.f;
+          hilo2(g00, g01, gbh[nt][0], gbl[nt][0]);
+          hilo2(g10, g11, gbh[nt][1], gbl[nt][1]);
+        }
+      }
+      // W2ᵀ += Sᵀ·A: Sᵀ as the A operand (columns x tokens), A (tokens x hidden) as B. With TW,
+      // each feature tile first gives the queries' partial Zᵀ from the W2 it holds before the
+      // update: W2ᵀ·Aqᵀ + Sᵀ·Gᵀ.
+#pragma unroll
+      for (int mt = 0; mt < 4; ++mt) {
+        uint32_t sa[2][4];
+#pragma unroll
+        for (int p = 0; p < 2; ++p) ldsm4_t(sbase[p] + swz128_bf16(8 * (mi >> 1) + ri, 16 * mt + 8 * (mi & 1)), sa[p]);
+        if (HAS_Q && TW) {
+          uint32_t whi[2][4], wlo[2][4];
+          afrag_hilo(a2[mt][0], a2[mt][1], whi[0], wlo[0]);
+          afrag_hilo(a2[mt][2], a2[mt][3], whi[1], wlo[1]);
+          float* red = &sm.red[1][warp][0][0];
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt) {
+            float zp[4] = {0.f, 0.f, 0.f, 0.f}, z2[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int ks = 0; ks < 2; ++ks) {
+              mma_bf16(zp, whi[ks], bq[nt][ks][0], bq[nt][ks][1]);
+              mma_bf16(z2, wlo[ks], bq[nt][ks][0], bq[nt][ks][1]);
+            }
+            mma_bf16(zp, sa[0], gbh[nt][0], gbh[nt][1]);
+            mma_bf16(z2, sa[0], gbl[nt][0], gbl[nt][1]);
+            mma_bf16(z2, sa[1], gbh[nt][0], gbh[nt][1]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              red[(8 * nt + 2 * q + (e & 1)) * kRedStride + 16 * mt + g + 8 * (e >> 1)] = zp[e] + z2[e];
+          }
+        }
+#pragma unroll
+        for (int p = 0; p < 2; ++p)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) mma_bf16(a2[mt][j], sa[p], ak[j >> 1][0][j & 1], ak[j >> 1][1][j & 1]);
+      }
+      if (HAS_Q && TW) {
+        compute_sync<kMlpWarps>();
+        query_outputs();
+      }
     }
     // End of the tile: its outputs are complete in shared memory and every warp is done with
     // its inputs, so the slot takes tile s + kStagesM.
@@ -813,14 +994,14 @@ __global__ void __launch_bounds__(kMlpThreads, 1)
   __syncthreads();
 }
 
-template <bool HAS_Q, bool LOSS>
+template <bool HAS_Q, bool LOSS, bool TW>
 ttt_status launch_inner(ttt_state* st, const CUtensorMap* maps, float* loss, int T, cudaStream_t s) {
   const ttt_config& c = st->cfg;
   const bool mlp = c.rule == TTT_RULE_MLP_GD;
   const size_t smem = (mlp ? sizeof(MlpSmem) : sizeof(LnSmem)) + 1024;
   // One bit per instantiation whose shared-memory limit has been raised on this state's device.
-  const uint64_t bit = 1ull << (48 + 4 * mlp + 2 * HAS_Q + LOSS);
-  auto kernel = mlp ? k_inner_mlp<HAS_Q, LOSS> : k_inner_ln<HAS_Q, LOSS>;
+  const uint64_t bit = 1ull << (48 + 8 * mlp + 4 * TW + 2 * HAS_Q + LOSS);
+  auto kernel = mlp ? k_inner_mlp<HAS_Q, LOSS, TW> : k_inner_ln<HAS_Q, LOSS, TW>;
   if (!(st->lin.smem_set & bit)) {
     TTT_CUDA(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
     st->lin.smem_set |= bit;
@@ -865,11 +1046,15 @@ ttt_status inner_scan(ttt_state* st, const __nv_bfloat16* K, const __nv_bfloat16
     ms->T = T;
   }
   ms->last_use = ++lb.map_clock;
+  // Per-token weights change only the outputs.
+  if (has_q && c.token_weights)
+    return loss ? launch_inner<true, true, true>(st, ms->maps, loss, (int)T, s)
+                : launch_inner<true, false, true>(st, ms->maps, loss, (int)T, s);
   if (has_q)
-    return loss ? launch_inner<true, true>(st, ms->maps, loss, (int)T, s)
-                : launch_inner<true, false>(st, ms->maps, loss, (int)T, s);
-  return loss ? launch_inner<false, true>(st, ms->maps, loss, (int)T, s)
-              : launch_inner<false, false>(st, ms->maps, loss, (int)T, s);
+    return loss ? launch_inner<true, true, false>(st, ms->maps, loss, (int)T, s)
+                : launch_inner<true, false, false>(st, ms->maps, loss, (int)T, s);
+  return loss ? launch_inner<false, true, false>(st, ms->maps, loss, (int)T, s)
+              : launch_inner<false, false, false>(st, ms->maps, loss, (int)T, s);
 }
 
 }  // namespace ttt

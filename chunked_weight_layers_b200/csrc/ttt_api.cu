@@ -49,6 +49,8 @@ static void dev_free(void* p) {
 }
 
 static ttt_status validate(const ttt_config* c) {
+  if (c->token_weights != 0 && c->rule != TTT_RULE_LINEAR_LN_GD && c->rule != TTT_RULE_MLP_GD)
+    return fail(TTT_ERR_UNSUPPORTED, "per-token weights apply to the LayerNorm inner models only");
   if (c->rule == TTT_RULE_INPLACE_HEBBIAN) {
     if (c->batch != 1 || c->heads != 1)
       return fail(TTT_ERR_UNSUPPORTED, "In-Place scan: batch and heads must be 1 (one Wdown state)");
@@ -102,6 +104,8 @@ static ttt_status validate(const ttt_config* c) {
     if (c->target_mode != 0) return fail(TTT_ERR_INVALID_ARG, "target_mode applies to In-Place only");
     if (c->gate_enable) return fail(TTT_ERR_UNSUPPORTED, "the surprisal gate runs on TTT-Linear states");
     if (!(c->ln_eps > 0.f)) return fail(TTT_ERR_INVALID_ARG, "%s: ln_eps must be positive", name);
+    if (c->token_weights != 0 && c->token_weights != 1)
+      return fail(TTT_ERR_INVALID_ARG, "token_weights must be 0 or 1");
     return TTT_OK;
   }
   return fail(TTT_ERR_INVALID_ARG, "unknown rule %d", c->rule);

@@ -82,10 +82,11 @@ class InnerSpec:
     seed: int = 1000
     D: int = 64
     hidden: int = 256
+    token_weights: bool = False   # outputs with per-token weights within the mini-batch
 
     @property
     def flops(self) -> float:
-        """Products per (token, head): LayerNorm TTT-Linear k·W, q·W and Kᵀ·dZ (2·D² each);
+        """Products per (token, head) (the per-token form's extra products are not counted): LayerNorm TTT-Linear k·W, q·W and Kᵀ·dZ (2·D² each);
         TTT-MLP two layers forward for keys and queries and three gradient products (2·D·Dh each)."""
         if self.model == "linear_ln":
             per = (6.0 if self.with_queries else 4.0) * self.D * self.D
@@ -111,7 +112,11 @@ WORKLOADS = {w.name: w for w in (INPLACE_FP32, LINEAR_GD, INPLACE_4B, INPLACE_12
 # instances, with LayerNorm and residual).
 LINEAR_LN = InnerSpec("ttt_linear_ln_B8_H12_T2048_b16", model="linear_ln", B=8, H=12, T=2048, seed=1007)
 MLP = InnerSpec("ttt_mlp_B8_H12_T2048_b16", model="mlp", B=8, H=12, T=2048, seed=1008)
-INNER_WORKLOADS = {w.name: w for w in (LINEAR_LN, MLP)}
+LINEAR_LN_TW = InnerSpec("ttt_linear_ln_B8_H12_T2048_b16_token_weights", model="linear_ln", B=8, H=12, T=2048,
+                         seed=1007, token_weights=True)
+MLP_TW = InnerSpec("ttt_mlp_B8_H12_T2048_b16_token_weights", model="mlp", B=8, H=12, T=2048, seed=1008,
+                   token_weights=True)
+INNER_WORKLOADS = {w.name: w for w in (LINEAR_LN, MLP, LINEAR_LN_TW, MLP_TW)}
 
 
 def document_starts(T: int, n_docs: int, seed: int, min_len: int = 64) -> list[int]:

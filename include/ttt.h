@@ -23,7 +23,9 @@
  *  GELU(x) = x·Φ(x)); LN normalises a token's 64 values by their mean and population variance
  *  (ε under the square root) and applies the per-head gain γ and bias β, which the inner step
  *  does not change. Per mini-batch of 16 tokens: O_i = f(Q_i; θ_i), E_i = f(K_i; θ_i) − V_i,
- *  L_t = ‖E_i[t]‖², θ_{i+1} = θ_i − η · ∇ℓ_i(θ_i) with ℓ_i = ‖E_i‖² / (2·16).
+ *  L_t = ‖E_i[t]‖², θ_{i+1} = θ_i − η · ∇ℓ_i(θ_i) with ℓ_i = ‖E_i‖² / (2·16). With per-token
+ *  weights (token_weights = 1, the TTT layer's mini-batch form) output t instead uses the
+ *  weights after the gradient steps of the mini-batch's tokens up to t, all taken at θ_i.
  *
  *  Surprisal gate ("SR-TTT: Surprisal-Aware Residual Test-Time Training", §2.1). Per
  *  (sequence, head) and chunk of 64 losses: p95 = 61st smallest; τ = p95 for the first
@@ -110,6 +112,11 @@ typedef struct {
   int32_t gate_mean_num;  /* the mean test is S/gate_chunk >= (num/den)·τ; 4 */
   int32_t gate_mean_den;  /* 5 */
   float ln_eps;           /* TTT_RULE_LINEAR_LN_GD and TTT_RULE_MLP_GD: LayerNorm ε; 1e-6 */
+  int32_t token_weights;  /* TTT_RULE_LINEAR_LN_GD and TTT_RULE_MLP_GD: 0 (default): the outputs of a
+                             mini-batch use its starting weights θ_i. 1: per-token weights, output t
+                             uses θ_i − (η/b)·Σ_{s ≤ t} ∇½‖f(k_s; θ_i) − v_s‖² over the mini-batch's
+                             tokens s up to t (the last token sees θ_{i+1}); losses and the weight
+                             update are unchanged. Other rules: must be 0. */
 } ttt_config;
 
 typedef struct ttt_state ttt_state; /* opaque; owns all of its device memory */

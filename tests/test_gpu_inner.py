@@ -23,15 +23,16 @@ def cwl():
     return cwl
 
 
-def make_state(cwl, spec, x):
-    cfg = cwl.config(spec.model, batch=spec.B, heads=spec.H, eta=spec.eta, ln_eps=spec.eps)
+def make_state(cwl, spec, x, token_weights=0):
+    cfg = cwl.config(spec.model, batch=spec.B, heads=spec.H, eta=spec.eta, ln_eps=spec.eps,
+                     token_weights=int(token_weights))
     st = cwl.FastWeightState(cfg, x["W0"])
     st.set_layernorm(x["gamma"], x["beta"])
     return st
 
 
-def run(cwl, spec, x, with_q=True, loss=True, splits=None):
-    st = make_state(cwl, spec, x)
+def run(cwl, spec, x, with_q=True, loss=True, splits=None, token_weights=False):
+    st = make_state(cwl, spec, x, token_weights)
     K, V = x["K"], x["V"]
     Q = x.get("Q") if with_q else None
     O = torch.full_like(K, float("nan")) if Q is not None else None
@@ -53,15 +54,15 @@ def run(cwl, spec, x, with_q=True, loss=True, splits=None):
     return O, W, L
 
 
-def oracle(spec, x, with_q=True):
+def oracle(spec, x, with_q=True, token_weights=False):
     cpu = {k: (v.cpu() if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
     Q = cpu.get("Q") if with_q else None
     if spec.model == "linear_ln":
         O, W, L = ora.ttt_linear_ln_scan(cpu["K"], cpu["V"], Q, cpu["W0"], cpu["gamma"], cpu["beta"], spec.eta,
-                                         spec.b, spec.eps)
+                                         spec.b, spec.eps, token_weights=token_weights)
         return O, W, L
     O, W1, W2, L = ora.ttt_mlp_scan(cpu["K"], cpu["V"], Q, cpu["W1"], cpu["W2"], cpu["gamma"], cpu["beta"],
-                                    spec.eta, spec.b, spec.eps)
+                                    spec.eta, spec.b, spec.eps, token_weights=token_weights)
     B, H = spec.B, spec.H
     return O, np.concatenate([W1.reshape(B, H, -1), W2.reshape(B, H, -1)], axis=2), L
 
@@ -178,3 +179,43 @@ def test_workload_full_size(cwl, model):
     print(f"{spec.name}: O {eo:.3e}  W {ew:.3e}  loss {el:.3e}")
     assert eo <= TOL and ew <= TOL and el <= TOL
     assert np.isfinite(to_np(O)).all()
+
+
+TW_MODELS = ["linear_ln", "mlp"]
+
+
+@pytest.mark.parametrize("model", TW_MODELS)
+@pytest.mark.parametrize("T", [208, 16])
+def test_token_weights_small_against_oracle(cwl, model, T):
+    """Per-token weights within the mini-batch: outputs against the oracle; losses and the final
+    weight equal the default form's bit for bit (only the outputs change)."""
+    spec = spec_of(model, B=2, H=3, T=T, seed=2600 + T)
+    x = workloads.inner_inputs(spec, device="cuda")
+    O, W, L = run(cwl, spec, x, token_weights=True)
+    Oref, Wref, Lref = oracle(spec, x, token_weights=True)
+    eo = rel_err(O, Oref)
+    print(f"{model} T={T} per-token weights: O {eo:.3e}")
+    assert eo <= TOL and max(weight_errs(spec, W, Wref)) <= TOL and rel_err(L, Lref) <= TOL
+    O0, W0_, L0 = run(cwl, spec, x)
+    assert torch.equal(W, W0_) and torch.equal(L, L0)
+    assert rel_err(O, to_np(O0)) > 1e-3
+
+
+@pytest.mark.parametrize("model", TW_MODELS)
+def test_token_weights_streaming(cwl, model):
+    spec = spec_of(model, B=1, H=2, T=192, seed=2700)
+    x = workloads.inner_inputs(spec, device="cuda")
+    O1, W1, L1 = run(cwl, spec, x, token_weights=True)
+    O2, W2, L2 = run(cwl, spec, x, splits=[(0, 48), (48, 192)], token_weights=True)
+    assert torch.equal(O1, O2) and torch.equal(W1, W2) and torch.equal(L1, L2)
+
+
+@pytest.mark.parametrize("model", TW_MODELS)
+def test_token_weights_workload_full_size(cwl, model):
+    spec = workloads.LINEAR_LN if model == "linear_ln" else workloads.MLP
+    x = workloads.inner_inputs(spec, device="cuda")
+    O, W, L = run(cwl, spec, x, token_weights=True)
+    Oref, Wref, Lref = oracle(spec, x, token_weights=True)
+    eo, ew, el = rel_err(O, Oref), max(weight_errs(spec, W, Wref)), rel_err(L, Lref)
+    print(f"{spec.name} per-token weights: O {eo:.3e}  W {ew:.3e}  loss {el:.3e}")
+    assert eo <= TOL and ew <= TOL and el <= TOL
