@@ -184,25 +184,43 @@ __device__ __forceinline__ void merge_stats(const float* p, float eps, float& mu
 // q_t·W_t = q_t·W_i + Σ_{s ≤ t} (q_t·k_s)·S_s: the query products of the forward pass plus
 // Sᵀ·Mᵀ with M = Q·Kᵀ masked to s ≤ t, added once S is known; the outputs' LayerNorm
 // statistics then take a third exchange.
-// Outputs q + γ·LN(o) + β of the step's sixteen tokens at this thread's two columns, from the
-// queries' merged statistics, into the swizzled staging tile.
-__device__ __forceinline__ void emit_outputs(const float (&o)[2][4], const float (&qv)[2][4], const float (*st)[8],
-                                             const float (&gam)[2], const float (&bet)[2], float eps, uint8_t* obuf,
-                                             int r0, int col0, int g, int q) {
+// Each lane merges the statistics it published (value g: kind g >> 2, token pub_tok) and the
+// eight lanes of a token group share them: mu[i], rs[i] for value i = 4·kind + 2·nt + jj.
+__device__ __forceinline__ void gather_stats(float (*fwd)[kMB][8], int pub_tok, int g, float eps, float (&mu)[8],
+                                             float (&rs)[8]) {
+  float m, r;
+  merge_stats(fwd[g >> 2][pub_tok], eps, m, r);
+  all_gather8(m, mu, g);
+  all_gather8(r, rs, g);
+}
+
+__device__ __forceinline__ void stsm4_t(uint32_t addr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3) {
+  asm volatile("stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(r0), "r"(r1),
+               "r"(r2), "r"(r3)
+               : "memory");
+}
+
+// Outputs q + γ·LN(o) + β of the step's sixteen tokens at this warp's sixteen columns, from the
+// queries' statistics (values 4..7 of mu, rs), into the swizzled staging tile by one transposing
+// stmatrix: matrix (nt, hc) holds tokens 8nt.. and columns col0 + 8hc.., its rows addressed by
+// lanes 8·(2nt + hc) + row (ofs_o = that lane's row and column offset).
+__device__ __forceinline__ void emit_outputs(const float (&o)[2][4], const float (&qv)[2][4], const float (&mu)[8],
+                                             const float (&rs)[8], const float (&gam)[2], const float (&bet)[2],
+                                             uint32_t obase, uint32_t ofs_o, int r0) {
+  uint32_t r[4];
 #pragma unroll
   for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-    for (int jj = 0; jj < 2; ++jj) {
-      const int tok = 8 * nt + 2 * q + jj;
-      float mu, rstd;
-      merge_stats(st[tok], eps, mu, rstd);
+    for (int hc = 0; hc < 2; ++hc) {
+      float y[2];
 #pragma unroll
-      for (int hc = 0; hc < 2; ++hc) {
-        const int e = jj + 2 * hc;
-        const float y = qv[nt][e] + fmaf(gam[hc], (o[nt][e] - mu) * rstd, bet[hc]);
-        *reinterpret_cast<__nv_bfloat16*>(obuf + swz128_bf16(r0 + tok, col0 + g + 8 * hc)) = __float2bfloat16_rn(y);
+      for (int jj = 0; jj < 2; ++jj) {
+        const int e = jj + 2 * hc, i = 4 + 2 * nt + jj;
+        y[jj] = qv[nt][e] + fmaf(gam[hc], (o[nt][e] - mu[i]) * rs[i], bet[hc]);
       }
+      r[2 * nt + hc] = pack_bf16(y[0], y[1]);
     }
+  stsm4_t(obase + ofs_o + (uint32_t)r0 * 128u, r[0], r[1], r[2], r[3]);
 }
 
 template <bool HAS_Q, bool LOSS, bool TW>
@@ -268,6 +286,7 @@ __global__ void __launch_bounds__(kLnThreads, 1)
   // Token (within the mini-batch) whose per-warp partial this lane publishes after a
   // reduce-scatter of values indexed 4·kind + 2·nt + jj.
   const int pub_tok = 8 * ((g >> 1) & 1) + 2 * q + (g & 1);
+  const uint32_t ofs_o = swz128_bf16(8 * (mi >> 1) + ri, col0 + 8 * (mi & 1));
 
   for (int s = 0; s < ntiles; ++s) {
     const int slot = s % kStagesI;
@@ -278,7 +297,7 @@ __global__ void __launch_bounds__(kLnThreads, 1)
     if (*reinterpret_cast<volatile int*>(&sm.cabort[s & 1])) break;
     const int ntok = min(kTileTokI, T - s * kTileTokI);
     const uint32_t kbase = smem_u32(sm.K[slot]), vbase = smem_u32(sm.V[slot]), qbase = smem_u32(sm.Q[slot]);
-    uint8_t* obuf = sm.O[s & 1];
+    const uint32_t obase = smem_u32(sm.O[s & 1]);
 
     for (int r0 = 0; r0 < ntok; r0 += kMB) {
       // ---- forward: Zᵀ = Wᵀ·Kᵀ and (queries) Pᵀ = Wᵀ·Qᵀ, all with the weight at the step's start
@@ -363,24 +382,22 @@ __global__ void __launch_bounds__(kLnThreads, 1)
       publish_stats<kOutNow>(z, o, sm.fwd, pub_tok, warp, g);
       compute_sync<kLnWarps>();
 
-      float zh[2][4], ev[2][4], gg[2][4], rz[2][2];
+      float zh[2][4], ev[2][4], gg[2][4], mu[8], rs[8];
+      gather_stats(sm.fwd, pub_tok, g, eps, mu, rs);
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
         for (int jj = 0; jj < 2; ++jj) {
-          const int tok = 8 * nt + 2 * q + jj;
-          float mu, rstd;
-          merge_stats(sm.fwd[0][tok], eps, mu, rstd);
-          rz[nt][jj] = rstd;
+          const int i = 2 * nt + jj;
 #pragma unroll
           for (int hc = 0; hc < 2; ++hc) {
             const int e = jj + 2 * hc;
-            zh[nt][e] = (z[nt][e] - mu) * rstd;
+            zh[nt][e] = (z[nt][e] - mu[i]) * rs[i];
             ev[nt][e] = fmaf(gam[hc], zh[nt][e], bet[hc]) + kv[nt][e];  // f(k) − v
             gg[nt][e] = gam[hc] * ev[nt][e];
           }
         }
-      if (kOutNow) emit_outputs(o, qv, sm.fwd[1], gam, bet, eps, obuf, r0, col0, g, q);
+      if (kOutNow) emit_outputs(o, qv, mu, rs, gam, bet, obase, ofs_o, r0);
 
       // ---- backward statistics: Σg and Σg·ẑ per token (and Σe² for the loss)
       float v8[8];
@@ -406,27 +423,28 @@ __global__ void __launch_bounds__(kLnThreads, 1)
       }
       compute_sync<kLnWarps>();
 
-      // ---- dZ = rstd·(g − mean g − ẑ·mean(g·ẑ)); W ← W − (η/b)·Kᵀ·dZ
-      float dz[2][4];
+      // ---- dZ = rstd·(g − mean g − ẑ·mean(g·ẑ)); W ← W − (η/b)·Kᵀ·dZ. Each lane sums the
+      // four warps' partials of the value it published; the token group shares the means.
+      float dz[2][4], bm[8];
+      {
+        const float4 A = *reinterpret_cast<const float4*>(&sm.bwd[pub_tok][4 * (g >> 2)]);
+        all_gather8(((A.x + A.y) + (A.z + A.w)) * (1.f / 64.f), bm, g);
+      }
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
         for (int jj = 0; jj < 2; ++jj) {
-          const int tok = 8 * nt + 2 * q + jj;
-          const float4 A = *reinterpret_cast<const float4*>(&sm.bwd[tok][0]);
-          const float4 B = *reinterpret_cast<const float4*>(&sm.bwd[tok][4]);
-          const float mg = ((A.x + A.y) + (A.z + A.w)) * (1.f / 64.f);
-          const float mgz = ((B.x + B.y) + (B.z + B.w)) * (1.f / 64.f);
+          const int i = 2 * nt + jj;
 #pragma unroll
           for (int hc = 0; hc < 2; ++hc) {
             const int e = jj + 2 * hc;
-            dz[nt][e] = -lr * (rz[nt][jj] * (gg[nt][e] - mg - zh[nt][e] * mgz));
-          }
-          if (LOSS && warp == 0 && g == 0) {
-            const float4 L = *reinterpret_cast<const float4*>(&sm.lossp[tok][0]);
-            loss[(size_t)bh * T + (size_t)s * kTileTokI + r0 + tok] = (L.x + L.y) + (L.z + L.w);
+            dz[nt][e] = -lr * (rs[i] * (gg[nt][e] - bm[i] - zh[nt][e] * bm[4 + i]));
           }
         }
+      if (LOSS && warp == 0) {
+        const float4 L = *reinterpret_cast<const float4*>(&sm.lossp[pub_tok][0]);
+        if (g < 4) loss[(size_t)bh * T + (size_t)s * kTileTokI + r0 + pub_tok] = (L.x + L.y) + (L.z + L.w);
+      }
       uint32_t shi[4], slo[4];
       afrag_hilo(dz[0], dz[1], shi, slo);
 #pragma unroll
@@ -458,14 +476,15 @@ __global__ void __launch_bounds__(kLnThreads, 1)
         }
         publish_stats<true, false>(z, o, sm.fwd, pub_tok, warp, g);
         compute_sync<kLnWarps>();
-        emit_outputs(o, qv, sm.fwd[1], gam, bet, eps, obuf, r0, col0, g, q);
+        gather_stats(sm.fwd, pub_tok, g, eps, mu, rs);
+        emit_outputs(o, qv, mu, rs, gam, bet, obase, ofs_o, r0);
       }
     }
     // End of the tile: its outputs are complete in shared memory.
     if (HAS_Q) fence_proxy_async_smem();
     compute_sync<kLnWarps>();
     if (threadIdx.x == 0 && HAS_Q) {
-      tma_store_3d(&tmO, obuf, 0, s * kTileTokI, bh);
+      tma_store_3d(&tmO, sm.O[s & 1], 0, s * kTileTokI, bh);
       bulk_commit();
       bulk_wait_read<1>();  // the other staging tile is free again
     }
