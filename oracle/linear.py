@@ -13,6 +13,11 @@ is ℓ_i(W) = 1/(2b)·‖K_i·W − V_i‖²_F, so one gradient step is
 W ← W − (η/b)·K_iᵀ(K_i·W − V_i); the b outputs of mini-batch i all use the W in effect at
 its start (O_i = Q_i·W_i); there is no LayerNorm or residual inside the inner model; the
 per-token loss (SR-TTT §2.1, inner-loop forward pass) is L_t = ‖k_t·W_i − v_t‖².
+
+Per-token weights (``token_weights=True``; the same page: with mini-batch 1 the rule is the
+delta rule, in which each token trains before the next is read): output t of mini-batch i uses
+W_t = W_i − (η/b)·Σ_{s ≤ t} k_sᵀ(k_s·W_i − v_s), the gradients of the mini-batch's tokens up
+to t, all at W_i; the last token sees W_{i+1}. Losses and the update are unchanged.
 """
 
 from __future__ import annotations
@@ -22,7 +27,7 @@ import numpy as np
 from ._util import f64
 
 
-def ttt_linear_scan(K, V, Q, W0, eta: float, b: int):
+def ttt_linear_scan(K, V, Q, W0, eta: float, b: int, token_weights: bool = False):
     """Scan every (sequence, head) of [B, H, T, D] inputs.
 
     Returns (O [B,H,T,D] or None when Q is None, W_final [B,H,D,D], loss [B,H,T]).
@@ -42,9 +47,13 @@ def ttt_linear_scan(K, V, Q, W0, eta: float, b: int):
     for i in range(T // b):
         s = slice(i * b, (i + 1) * b)
         Ki, Vi = Kf[:, s], Vf[:, s]
-        if Qf is not None:
+        if Qf is not None and not token_weights:
             O[:, s] = Qf[:, s] @ W                       # output with W_i (start of mini-batch)
         R = Ki @ W - Vi                                  # residual of the inner model
+        if Qf is not None and token_weights:
+            for j in range(b):                           # token j sees the steps of tokens 0..j
+                t = i * b + j
+                O[:, t:t + 1] = Qf[:, t:t + 1] @ (W - (eta / b) * (np.swapaxes(Ki[:, :j + 1], 1, 2) @ R[:, :j + 1]))
         loss[:, s] = np.sum(R * R, axis=2)               # L_t = ‖k_t W_i − v_t‖²
         W = W - (eta / b) * (np.swapaxes(Ki, 1, 2) @ R)  # one gradient step on ℓ_i
     O = None if O is None else O.reshape(B, H, T, D)

@@ -28,6 +28,7 @@ from __future__ import annotations
 
 import numpy as np
 
+from . import inner
 from ._util import f64
 
 
@@ -63,7 +64,7 @@ def inplace_scan_docs(Z, Vhat, W0, eta: float, C: int, doc_starts, clip=None):
     return O, W
 
 
-def ttt_linear_scan_docs(K, V, Q, W0, eta: float, b: int, doc_starts):
+def ttt_linear_scan_docs(K, V, Q, W0, eta: float, b: int, doc_starts, token_weights: bool = False):
     """TTT-Linear over packed sequences; ``doc_starts[s]`` lists sequence s's document starts.
 
     K, V, Q [B, H, T, D] (Q may be None), W0 [B, H, D, D]. Returns (O or None, W after each
@@ -84,10 +85,59 @@ def ttt_linear_scan_docs(K, V, Q, W0, eta: float, b: int, doc_starts):
                 for i0 in range(a, e, b):
                     r = slice(i0, min(i0 + b, e))
                     n = r.stop - r.start                 # b, or fewer for the last mini-batch
-                    if Qd is not None:
+                    if Qd is not None and not token_weights:
                         O[s, h, r] = Qd[s, h, r] @ W     # outputs with the mini-batch's start W
                     R = Kd[s, h, r] @ W - Vd[s, h, r]
                     loss[s, h, r] = np.sum(R * R, axis=1)
+                    if Qd is not None and token_weights:  # token j sees the steps of tokens 0..j
+                        for j in range(n):
+                            Wt = W - (eta / n) * (Kd[s, h, i0:i0 + j + 1].T @ R[:j + 1])
+                            O[s, h, i0 + j] = Qd[s, h, i0 + j] @ Wt
                     W = W - (eta / n) * (Kd[s, h, r].T @ R)
             Wout[s, h] = W
     return O, Wout, loss
+
+
+def inner_scan_docs(model: str, K, V, Q, W0, gamma, beta, eta: float, b: int, eps: float, doc_starts,
+                    token_weights: bool = False):
+    """The richer inner models (``model`` "linear_ln" or "mlp", oracle.inner) over packed
+    sequences, by the same reading: every document of sequence s (``doc_starts[s]``) restarts
+    every head from W0 (LayerNorm TTT-Linear: [B,H,D,D]; TTT-MLP: the pair (W1 [B,H,D,Dh],
+    W2 [B,H,Dh,D])), mini-batches count from its first token, and a last mini-batch of n < b
+    tokens takes the step of its own loss (one step of the inner scan with mini-batch n).
+
+    Returns (O or None, the weights after each sequence's last document, loss [B, H, T])."""
+    Kd, Vd = f64(K), f64(V)
+    Qd = None if Q is None else f64(Q)
+    B, H, T, D = Kd.shape
+    mlp = model == "mlp"
+    W0s = (f64(W0[0]), f64(W0[1])) if mlp else f64(W0)
+    O = None if Qd is None else np.empty((B, H, T, D))
+    loss = np.empty((B, H, T))
+    Wout = ([np.empty_like(W0s[0]), np.empty_like(W0s[1])] if mlp else np.empty_like(W0s))
+    for s in range(B):
+        docs = _documents(doc_starts[s], T)
+        for h in range(H):
+            g, be = f64(gamma)[h:h + 1], f64(beta)[h:h + 1]
+            for a, e in docs:
+                W = (W0s[0][s, h], W0s[1][s, h]) if mlp else W0s[s, h]   # document boundary: θ ← θ0
+                for i0 in range(a, e, b):
+                    r = slice(i0, min(i0 + b, e))
+                    n = r.stop - r.start
+                    one = lambda x: None if x is None else x[s, h, r][None, None]  # noqa: E731
+                    if mlp:
+                        o, W1n, W2n, l = inner.ttt_mlp_scan(one(Kd), one(Vd), one(Qd), W[0][None, None], W[1][None, None],
+                                                            g, be, eta, n, eps, token_weights=token_weights)
+                        W = (W1n[0, 0], W2n[0, 0])
+                    else:
+                        o, Wn, l = inner.ttt_linear_ln_scan(one(Kd), one(Vd), one(Qd), W[None, None], g, be, eta, n, eps,
+                                                            token_weights=token_weights)
+                        W = Wn[0, 0]
+                    if O is not None:
+                        O[s, h, r] = o[0, 0]
+                    loss[s, h, r] = l[0, 0]
+            if mlp:
+                Wout[0][s, h], Wout[1][s, h] = W
+            else:
+                Wout[s, h] = W
+    return O, (tuple(Wout) if mlp else Wout), loss

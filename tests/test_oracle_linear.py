@@ -121,3 +121,23 @@ def test_heads_are_independent():
     np.testing.assert_array_equal(O[1, 0], O1[0, 0])
     np.testing.assert_array_equal(W[1, 0], W1[0, 0])
     np.testing.assert_array_equal(L[1, 0], L1[0, 0])
+
+
+def test_token_weights_last_and_first_token():
+    """Per-token weights: the last token of a mini-batch gives the plain scan's output at the next
+    mini-batch's first token (weight W_{i+1}); the first token the output of a plain scan with
+    mini-batch 1 and step η/b after that token alone (the delta rule's step)."""
+    T, D, b, eta = 24, 5, 4, 0.4
+    K, V, Q, W0 = _rand((T, D), 30), _rand((T, D), 31), _rand((T, D), 32), _rand((D, D), 33)
+    O_tw, W_tw, L_tw = linear.ttt_linear_scan(_single(K), _single(V), _single(Q), _single(W0), eta, b,
+                                              token_weights=True)
+    last = np.arange(b - 1, T - b, b)
+    Q2 = Q.copy()
+    Q2[last + 1] = Q[last]
+    O_pl, W_pl, L_pl = linear.ttt_linear_scan(_single(K), _single(V), _single(Q2), _single(W0), eta, b)
+    np.testing.assert_allclose(O_tw[0, 0, last], O_pl[0, 0, last + 1], rtol=1e-12, atol=1e-12)
+    np.testing.assert_array_equal(W_tw, W_pl)
+    np.testing.assert_array_equal(L_tw, L_pl)
+    K2, V2, Q3 = (np.stack([x[0], x[0]]) for x in (K, V, Q))
+    O_one = linear.ttt_linear_scan(_single(K2), _single(V2), _single(Q3), _single(W0), eta / b, 1)[0]
+    np.testing.assert_allclose(O_tw[0, 0, 0], O_one[0, 0, 1], rtol=1e-12, atol=1e-12)

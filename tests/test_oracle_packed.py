@@ -111,3 +111,71 @@ def test_rejects_bad_document_starts():
     for starts in ([], [1], [0, 0], [0, 5, 3], [0, 8]):
         with pytest.raises(ValueError):
             packed.inplace_scan_docs(Z, V, W0, 0.1, 4, starts)
+
+
+def test_linear_token_weights_per_document():
+    """Per-token weights over packed sequences: one document of whole mini-batches equals the
+    per-token scan, and the final weight and losses do not depend on the outputs' form."""
+    B, H, T, D, b, eta = 1, 2, 32, 4, 8, 0.3
+    K, V, Q = _rand((B, H, T, D), 40, 0.5), _rand((B, H, T, D), 41, 0.5), _rand((B, H, T, D), 42)
+    W0 = _rand((B, H, D, D), 43, 0.3)
+    O, W, L = packed.ttt_linear_scan_docs(K, V, Q, W0, eta, b, [[0]], token_weights=True)
+    O_r, W_r, L_r = linear.ttt_linear_scan(K, V, Q, W0, eta, b, token_weights=True)
+    for got, want in ((O, O_r), (W, W_r), (L, L_r)):
+        np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
+    O2, W2, L2 = packed.ttt_linear_scan_docs(K, V, Q, W0, eta, b, [[0, 13]], token_weights=True)
+    O3, W3, L3 = packed.ttt_linear_scan_docs(K, V, Q, W0, eta, b, [[0, 13]])
+    np.testing.assert_array_equal(W2, W3)
+    np.testing.assert_array_equal(L2, L3)
+    # The first document's 5-token last mini-batch: the per-token scan with b = 5 from the weight
+    # after its first 8 tokens.
+    _, W8, _ = linear.ttt_linear_scan(K[:, :, :8], V[:, :, :8], Q[:, :, :8], W0, eta, b)
+    O5 = linear.ttt_linear_scan(K[:, :, 8:13], V[:, :, 8:13], Q[:, :, 8:13], W8, eta, 5, token_weights=True)[0]
+    np.testing.assert_allclose(O2[:, :, 8:13], O5, rtol=0, atol=1e-12)
+
+
+def test_layernorm_model_per_document():
+    _inner_per_document("linear_ln")
+
+
+def test_mlp_model_per_document():
+    _inner_per_document("mlp")
+
+
+def _inner_per_document(model):
+    """The LayerNorm and MLP models over packed sequences: one document of whole mini-batches is
+    the inner scan; every document restarts from the pretrained weights; a short last mini-batch
+    is one step of the inner scan with mini-batch n."""
+    from oracle import inner
+    B, H, T, D, b, eta, eps = 2, 2, 40, 4, 8, 0.3, 1e-3
+    K, V, Q = _rand((B, H, T, D), 44, 0.5), _rand((B, H, T, D), 45, 0.5), _rand((B, H, T, D), 46)
+    g, be = _rand((H, D), 47) + 1.0, _rand((H, D), 48)
+    if model == "mlp":
+        W0 = (_rand((B, H, D, 4 * D), 49, 0.5), _rand((B, H, 4 * D, D), 50, 0.5))
+        scan = lambda k, v, q, w, bb: inner.ttt_mlp_scan(k, v, q, w[0], w[1], g, be, eta, bb, eps)  # noqa: E731
+        weights = lambda r: (r[1], r[2])  # noqa: E731
+    else:
+        W0 = _rand((B, H, D, D), 49, 0.5)
+        scan = lambda k, v, q, w, bb: inner.ttt_linear_ln_scan(k, v, q, w, g, be, eta, bb, eps)  # noqa: E731
+        weights = lambda r: r[1]  # noqa: E731
+    O, W, L = packed.inner_scan_docs(model, K, V, Q, W0, g, be, eta, b, eps, [[0], [0]])
+    ref = scan(K, V, Q, W0, b)
+    np.testing.assert_allclose(O, ref[0], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(L, ref[-1], rtol=0, atol=1e-12)
+    # Sequence 1 as two documents, [0, 24) and [24, 40): 24 = 3 mini-batches, then 16 = 2.
+    O, W, L = packed.inner_scan_docs(model, K, V, Q, W0, g, be, eta, b, eps, [[0], [0, 24]])
+    sl = lambda x, a, e: x[1:2, :, a:e]  # noqa: E731
+    w1 = (W0[0][1:2], W0[1][1:2]) if model == "mlp" else W0[1:2]
+    r1 = scan(sl(K, 0, 24), sl(V, 0, 24), sl(Q, 0, 24), w1, b)
+    r2 = scan(sl(K, 24, 40), sl(V, 24, 40), sl(Q, 24, 40), w1, b)
+    np.testing.assert_allclose(O[1:2, :, :24], r1[0], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(O[1:2, :, 24:], r2[0], rtol=0, atol=1e-12)
+    # A 13-token document with b = 8: one full mini-batch, then one step with mini-batch 5.
+    O, W, L = packed.inner_scan_docs(model, K[:, :, :13], V[:, :, :13], Q[:, :, :13], W0, g, be, eta, b, eps,
+                                     [[0], [0]])
+    full = scan(K[:, :, :8], V[:, :, :8], Q[:, :, :8], W0, b)
+    tail = scan(K[:, :, 8:13], V[:, :, 8:13], Q[:, :, 8:13], weights(full), 5)
+    np.testing.assert_allclose(O[:, :, 8:13], tail[0], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(L[:, :, 8:13], tail[-1], rtol=0, atol=1e-12)
+    for got, want in zip(W if model == "mlp" else (W,), weights(tail) if model == "mlp" else (weights(tail),)):
+        np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)

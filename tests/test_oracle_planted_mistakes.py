@@ -46,13 +46,25 @@ MUTANTS = [
     ("linear", "transposed gradient",
      [("W = W - (eta / b) * (np.swapaxes(Ki, 1, 2) @ R)", "W = W - (eta / b) * (np.swapaxes(R, 1, 2) @ Ki)")]),
     ("linear", "outputs from the weight after the mini-batch's update",
-     [("        if Qf is not None:\n"
+     [("        if Qf is not None and not token_weights:\n"
        "            O[:, s] = Qf[:, s] @ W                       # output with W_i (start of mini-batch)\n",
        ""),
       ("        W = W - (eta / b) * (np.swapaxes(Ki, 1, 2) @ R)  # one gradient step on ℓ_i\n",
        "        W = W - (eta / b) * (np.swapaxes(Ki, 1, 2) @ R)\n"
-       "        if Qf is not None:\n"
+       "        if Qf is not None and not token_weights:\n"
        "            O[:, s] = Qf[:, s] @ W\n")]),
+    ("linear", "per-token weights without the token's own step",
+     [("(np.swapaxes(Ki[:, :j + 1], 1, 2) @ R[:, :j + 1])", "(np.swapaxes(Ki[:, :j], 1, 2) @ R[:, :j])")]),
+    ("packed", "per-document per-token weights from the wrong step size",
+     [("Wt = W - (eta / n) * (Kd[s, h, i0:i0 + j + 1].T @ R[:j + 1])", "Wt = W - (eta / b) * (Kd[s, h, i0:i0 + j + 1].T @ R[:j + 1])")]),
+    ("packed", "LayerNorm and MLP documents not restarted from the pretrained weights",
+     [("                W = (W0s[0][s, h], W0s[1][s, h]) if mlp else W0s[s, h]   # document boundary: θ ← θ0\n",
+       "                W = W if a > 0 else ((W0s[0][s, h], W0s[1][s, h]) if mlp else W0s[s, h])\n")]),
+    ("packed", "short last LayerNorm or MLP mini-batch stepped as a full one",
+     [("                                                            g, be, eta, n, eps, token_weights=token_weights)",
+       "                                                            g, be, eta * n / b, n, eps, token_weights=token_weights)"),
+      ("        o, Wn, l = inner.ttt_linear_ln_scan(one(Kd), one(Vd), one(Qd), W[None, None], g, be, eta, n, eps,",
+       "        o, Wn, l = inner.ttt_linear_ln_scan(one(Kd), one(Vd), one(Qd), W[None, None], g, be, eta * n / b, n, eps,")]),
     ("linear", "loss not squared per element",
      [("loss[:, s] = np.sum(R * R, axis=2)", "loss[:, s] = np.sum(R, axis=2) ** 2")]),
     ("gate", "percentile one rank too high",
