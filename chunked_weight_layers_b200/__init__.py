@@ -157,6 +157,24 @@ class FastWeightState:
                                             ctypes.cast(starts, ctypes.c_void_p), len(doc_starts),
                                             float(clip or 0.0), _stream(stream)))
 
+    def chunk_scan_packed(self, keys, targets, doc_starts, queries=None, out=None, loss_out=None, T=None,
+                          stream=None):
+        """ttt_chunk_scan_packed (the TTT-Linear family): ``doc_starts[b]`` lists sequence b's
+        document starts (ints, 0 first); every document is scanned from the pretrained weights.
+        Synchronises the stream (the layout goes up from host memory)."""
+        import ctypes
+        if T is None:
+            T = keys.shape[-2]
+        if len(doc_starts) != self.cfg.batch:
+            raise ValueError(f"doc_starts must hold one list per sequence ({self.cfg.batch})")
+        flat = [int(a) for seq in doc_starts for a in seq]
+        starts = (ctypes.c_int64 * len(flat))(*flat)
+        counts = (ctypes.c_int32 * len(doc_starts))(*[len(seq) for seq in doc_starts])
+        check(self._lib.ttt_chunk_scan_packed(self._h, *self._scan_args(keys, targets, queries, out, loss_out, T,
+                                                                        _current_device()),
+                                              ctypes.cast(starts, ctypes.c_void_p), ctypes.cast(counts, ctypes.c_void_p),
+                                              _stream(stream)))
+
     def surprisal_route(self, loss, T=None, stream=None):
         if T is None:
             T = loss.shape[-1]

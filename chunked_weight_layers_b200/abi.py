@@ -72,6 +72,7 @@ _SIGNATURES = {
     "ttt_chunk_scan": (_st, [_vp, _vp, _vp, _vp, ctypes.c_int64, _vp, _vp, _vp]),
     "ttt_chunk_scan_host": (_st, [_vp, _vp, _vp, _vp, ctypes.c_int64, _vp, _vp, _vp]),
     "ttt_chunk_scan_docs": (_st, [_vp, _vp, _vp, ctypes.c_int64, _vp, _vp, ctypes.c_int32, ctypes.c_float, _vp]),
+    "ttt_chunk_scan_packed": (_st, [_vp, _vp, _vp, _vp, ctypes.c_int64, _vp, _vp, _vp, _vp, _vp]),
     "ttt_surprisal_route": (_st, [_vp, _vp, ctypes.c_int64, _vp]),
     "ttt_state_reset": (_st, [_vp, _vp]),
     "ttt_state_get_weights": (_st, [_vp, _vp, _vp]),

@@ -25,6 +25,9 @@
 // recurrence amplify operand rounding, and with single bf16 operands the outputs drift to
 // ~1e-2 of their scale over 128 steps, against ~1e-5 with the pairs (measured on the CPU
 // against float64). The weights and every accumulation stay fp32.
+#include <algorithm>
+#include <vector>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -115,6 +118,19 @@ __device__ __forceinline__ void all_gather8(float x, float (&v)[8], int g) {
   }
 }
 
+// Arguments of one scan launch (both kernels).
+struct InnerArgs {
+  float* W;            // [B·H] per-head weights, fp32, updated in place
+  const float* W0;     // the pretrained weights (packed sequences reset to them)
+  const float* gamma;  // LayerNorm gain and bias [H, 64]
+  const float* beta;
+  float* loss;         // [B·H, T] or null
+  const int2* steps;   // packed sequences: per (sequence, mini-batch) {reset to W0 first, real tokens}; or null
+  int T, heads, nsteps;  // nsteps: entries of steps a sequence
+  float eta, eps;
+  DevStatus status;
+};
+
 // ============================ TTT-Linear with LayerNorm and residual ============================
 
 constexpr int kLnWarps = 4;                       // compute warps: sixteen columns of W each
@@ -179,11 +195,6 @@ __device__ __forceinline__ void merge_stats(const float* p, float eps, float& mu
   rstd = rsqrtf(m2 * (1.f / 64.f) + eps);
 }
 
-// TW: per-token weights within the mini-batch. Token t's output uses
-// W_t = W_i + Σ_{s ≤ t} k_sᵀ·S_s (S = −(η/b)·∂ℓ/∂Z, every gradient at W_i), so
-// q_t·W_t = q_t·W_i + Σ_{s ≤ t} (q_t·k_s)·S_s: the query products of the forward pass plus
-// Sᵀ·Mᵀ with M = Q·Kᵀ masked to s ≤ t, added once S is known; the outputs' LayerNorm
-// statistics then take a third exchange.
 // Each lane merges the statistics it published (value g: kind g >> 2, token pub_tok) and the
 // eight lanes of a token group share them: mu[i], rs[i] for value i = 4·kind + 2·nt + jj.
 __device__ __forceinline__ void gather_stats(float (*fwd)[kMB][8], int pub_tok, int g, float eps, float (&mu)[8],
@@ -223,16 +234,34 @@ __device__ __forceinline__ void emit_outputs(const float (&o)[2][4], const float
   stsm4_t(obase + ofs_o + (uint32_t)r0 * 128u, r[0], r[1], r[2], r[3]);
 }
 
-template <bool HAS_Q, bool LOSS, bool TW>
+// Plain outputs (no LayerNorm, no residual) into the staging tile, as in emit_outputs.
+__device__ __forceinline__ void emit_plain(const float (&o)[2][4], uint32_t obase, uint32_t ofs_o, int r0) {
+  stsm4_t(obase + ofs_o + (uint32_t)r0 * 128u, pack_bf16(o[0][0], o[0][1]), pack_bf16(o[0][2], o[0][3]),
+          pack_bf16(o[1][0], o[1][1]), pack_bf16(o[1][2], o[1][3]));
+}
+
+// LN = true: TTT-Linear with LayerNorm and residual; LN = false: the plain TTT-Linear rule
+// (f(x) = x·W), run by this kernel for per-token weights and packed sequences.
+//
+// TW: per-token weights within the mini-batch. Token t's output uses
+// W_t = W_i + Σ_{s ≤ t} k_sᵀ·S_s (S = −(η/n)·∂ℓ/∂Z, every gradient at W_i), so
+// q_t·W_t = q_t·W_i + Σ_{s ≤ t} (q_t·k_s)·S_s: the query products of the forward pass plus
+// Sᵀ·Mᵀ with M = Q·Kᵀ masked to s ≤ t, added once S is known; with LayerNorm the outputs'
+// statistics then take a third exchange.
+//
+// Packed sequences (a.steps set): each (sequence, mini-batch) entry says whether the weight
+// goes back to W0 before it (a document's first mini-batch) and how many of its 16 tokens are
+// real (a document's last mini-batch may be shorter; the rest are zero padding): padded
+// tokens contribute no gradient and the step is η/n for n real tokens.
+template <bool HAS_Q, bool LOSS, bool TW, bool LN>
 __global__ void __launch_bounds__(kLnThreads, 1)
     k_inner_ln(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-               const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
-               float* __restrict__ Wstate, const float* __restrict__ gamma, const float* __restrict__ beta,
-               float* __restrict__ loss, int T, int heads, float lr, float eps, const DevStatus status) {
+               const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO, const InnerArgs a) {
   extern __shared__ uint8_t smem_raw[];
   LnSmem& sm = *reinterpret_cast<LnSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bh = blockIdx.x;
+  const int T = a.T;
   const int ntiles = (T + kTileTokI - 1) / kTileTokI;
   const uint32_t stage_bytes = (HAS_Q ? 3u : 2u) * kTileBytesI;
 
@@ -253,7 +282,7 @@ __global__ void __launch_bounds__(kLnThreads, 1)
       int issued = 0;
       for (int s = 0; s < ntiles; ++s) {
         const int slot = s % kStagesI;
-        if (s >= kStagesI && !mbar_wait(&sm.empty[slot], ((s / kStagesI) - 1) & 1, status, &sm.abort)) break;
+        if (s >= kStagesI && !mbar_wait(&sm.empty[slot], ((s / kStagesI) - 1) & 1, a.status, &sm.abort)) break;
         mbar_arrive_expect_tx(&sm.full[slot], stage_bytes);
         tma_load_3d(sm.K[slot], &tmK, &sm.full[slot], 0, s * kTileTokI, bh);
         tma_load_3d(sm.V[slot], &tmV, &sm.full[slot], 0, s * kTileTokI, bh);
@@ -263,7 +292,7 @@ __global__ void __launch_bounds__(kLnThreads, 1)
       // Nothing may still be landing in shared memory when the CTA exits.
       for (int s = issued - kStagesI; s < issued; ++s) {
         if (s < 0) continue;
-        mbar_wait(&sm.full[s % kStagesI], (s / kStagesI) & 1, status, nullptr);
+        mbar_wait(&sm.full[s % kStagesI], (s / kStagesI) & 1, a.status, nullptr);
       }
     }
     __syncthreads();
@@ -273,16 +302,26 @@ __global__ void __launch_bounds__(kLnThreads, 1)
   // ---------------- compute warps ----------------
   const int g = lane >> 2, q = lane & 3, mi = lane >> 3, ri = lane & 7;
   const int col0 = 16 * warp;
-  float* Wg = Wstate + (size_t)bh * 64 * 64;
+  float* Wg = a.W + (size_t)bh * 64 * 64;
+  const float* W0g = a.W0 + (size_t)bh * 64 * 64;
   // Wᵀ slice in accumulator layout: acc[nt][e] = W[8nt + 2q + (e&1)][col0 + g + 8(e>>1)].
   float acc[8][4];
+  auto load_w = [&](const float* src) {
 #pragma unroll
-  for (int nt = 0; nt < 8; ++nt)
+    for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
-    for (int e = 0; e < 4; ++e) acc[nt][e] = Wg[(8 * nt + 2 * q + (e & 1)) * 64 + col0 + g + 8 * (e >> 1)];
-  const int h = bh % heads;
-  const float gam[2] = {gamma[h * 64 + col0 + g], gamma[h * 64 + col0 + g + 8]};
-  const float bet[2] = {beta[h * 64 + col0 + g], beta[h * 64 + col0 + g + 8]};
+      for (int e = 0; e < 4; ++e) acc[nt][e] = src[(8 * nt + 2 * q + (e & 1)) * 64 + col0 + g + 8 * (e >> 1)];
+  };
+  load_w(Wg);
+  const int h = bh % a.heads;
+  float gam[2] = {1.f, 1.f}, bet[2] = {0.f, 0.f};
+  if (LN) {
+    gam[0] = a.gamma[h * 64 + col0 + g];
+    gam[1] = a.gamma[h * 64 + col0 + g + 8];
+    bet[0] = a.beta[h * 64 + col0 + g];
+    bet[1] = a.beta[h * 64 + col0 + g + 8];
+  }
+  const int2* steps = a.steps == nullptr ? nullptr : a.steps + (size_t)(bh / a.heads) * a.nsteps;
   // Token (within the mini-batch) whose per-warp partial this lane publishes after a
   // reduce-scatter of values indexed 4·kind + 2·nt + jj.
   const int pub_tok = 8 * ((g >> 1) & 1) + 2 * q + (g & 1);
@@ -292,7 +331,7 @@ __global__ void __launch_bounds__(kLnThreads, 1)
     const int slot = s % kStagesI;
     // Every compute warp takes the same exit decision: the flag for tile s is only written
     // before this barrier and only read after it.
-    if (!mbar_wait(&sm.full[slot], (s / kStagesI) & 1, status, nullptr)) sm.cabort[s & 1] = 1;
+    if (!mbar_wait(&sm.full[slot], (s / kStagesI) & 1, a.status, nullptr)) sm.cabort[s & 1] = 1;
     compute_sync<kLnWarps>();
     if (*reinterpret_cast<volatile int*>(&sm.cabort[s & 1])) break;
     const int ntok = min(kTileTokI, T - s * kTileTokI);
@@ -300,6 +339,13 @@ __global__ void __launch_bounds__(kLnThreads, 1)
     const uint32_t obase = smem_u32(sm.O[s & 1]);
 
     for (int r0 = 0; r0 < ntok; r0 += kMB) {
+      int nval = kMB;  // real tokens of this mini-batch
+      if (steps != nullptr) {
+        const int2 e = steps[s * (kTileTokI / kMB) + r0 / kMB];
+        if (e.x) load_w(W0g);  // a document starts: the pretrained weight
+        nval = e.y;
+      }
+      const float lr = a.eta / (float)max(nval, 1);
       // ---- forward: Zᵀ = Wᵀ·Kᵀ and (queries) Pᵀ = Wᵀ·Qᵀ, all with the weight at the step's start
       uint32_t whi[4][4], wlo[4][4];
 #pragma unroll
@@ -346,12 +392,13 @@ __global__ void __launch_bounds__(kLnThreads, 1)
           o[nt][e] += o2[e];
         }
       }
-      // k − v (and q) at this thread's (column, token) positions of the Zᵀ layout.
+      // k − v with LayerNorm's residual, −v without (and q for the residual of the outputs) at
+      // this thread's (column, token) positions of the Zᵀ layout.
       float kv[2][4], qv[2][4];
       {
         const uint32_t off = swz128_bf16(r0 + 8 * (mi >> 1) + ri, col0 + 8 * (mi & 1));
-        uint32_t kr[4], vr[4];
-        ldsm4_t(kbase + off, kr);
+        uint32_t kr[4] = {0u, 0u, 0u, 0u}, vr[4];
+        if (LN) ldsm4_t(kbase + off, kr);
         ldsm4_t(vbase + off, vr);
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
@@ -362,54 +409,63 @@ __global__ void __launch_bounds__(kLnThreads, 1)
           kv[nt][2] = k1.x - v1.x;
           kv[nt][3] = k1.y - v1.y;
         }
-        if (HAS_Q) {
+        if (HAS_Q && LN) {
           uint32_t qr[4];
           ldsm4_t(qbase + off, qr);
 #pragma unroll
           for (int nt = 0; nt < 2; ++nt) {
-            const float2 a = bf2_to_f2(qr[2 * nt]), b = bf2_to_f2(qr[2 * nt + 1]);
-            qv[nt][0] = a.x;
-            qv[nt][1] = a.y;
-            qv[nt][2] = b.x;
-            qv[nt][3] = b.y;
+            const float2 p = bf2_to_f2(qr[2 * nt]), r = bf2_to_f2(qr[2 * nt + 1]);
+            qv[nt][0] = p.x;
+            qv[nt][1] = p.y;
+            qv[nt][2] = r.x;
+            qv[nt][3] = r.y;
           }
         }
       }
 
-      // ---- LayerNorm statistics: per warp two-pass over its sixteen columns, then merged. The
-      // queries' share here unless TW (their products are not complete before the backward).
+      // The queries' outputs now, unless TW (their products are not complete before the backward).
       constexpr bool kOutNow = HAS_Q && !TW;
-      publish_stats<kOutNow>(z, o, sm.fwd, pub_tok, warp, g);
-      compute_sync<kLnWarps>();
-
       float zh[2][4], ev[2][4], gg[2][4], mu[8], rs[8];
-      gather_stats(sm.fwd, pub_tok, g, eps, mu, rs);
+      if (LN) {
+        // ---- LayerNorm statistics: per warp two-pass over its sixteen columns, then merged
+        publish_stats<kOutNow>(z, o, sm.fwd, pub_tok, warp, g);
+        compute_sync<kLnWarps>();
+        gather_stats(sm.fwd, pub_tok, g, a.eps, mu, rs);
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
+        for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-        for (int jj = 0; jj < 2; ++jj) {
-          const int i = 2 * nt + jj;
+          for (int jj = 0; jj < 2; ++jj) {
+            const int i = 2 * nt + jj;
 #pragma unroll
-          for (int hc = 0; hc < 2; ++hc) {
-            const int e = jj + 2 * hc;
-            zh[nt][e] = (z[nt][e] - mu[i]) * rs[i];
-            ev[nt][e] = fmaf(gam[hc], zh[nt][e], bet[hc]) + kv[nt][e];  // f(k) − v
-            gg[nt][e] = gam[hc] * ev[nt][e];
+            for (int hc = 0; hc < 2; ++hc) {
+              const int e = jj + 2 * hc;
+              zh[nt][e] = (z[nt][e] - mu[i]) * rs[i];
+              ev[nt][e] = fmaf(gam[hc], zh[nt][e], bet[hc]) + kv[nt][e];  // f(k) − v
+              gg[nt][e] = gam[hc] * ev[nt][e];
+            }
           }
-        }
-      if (kOutNow) emit_outputs(o, qv, mu, rs, gam, bet, obase, ofs_o, r0);
+        if (kOutNow) emit_outputs(o, qv, mu, rs, gam, bet, obase, ofs_o, r0);
+      } else {
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) gg[nt][e] = ev[nt][e] = z[nt][e] + kv[nt][e];  // k·W − v
+        if (kOutNow) emit_plain(o, obase, ofs_o, r0);
+      }
 
-      // ---- backward statistics: Σg and Σg·ẑ per token (and Σe² for the loss)
+      // ---- backward statistics: Σg and Σg·ẑ per token (LayerNorm), Σe² for the loss
       float v8[8];
+      if (LN) {
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
+        for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-        for (int jj = 0; jj < 2; ++jj) {
-          v8[2 * nt + jj] = gg[nt][jj] + gg[nt][jj + 2];
-          v8[4 + 2 * nt + jj] = gg[nt][jj] * zh[nt][jj] + gg[nt][jj + 2] * zh[nt][jj + 2];
-        }
-      const float bw = reduce_scatter8(v8, g);
-      sm.bwd[pub_tok][4 * (g >> 2) + warp] = bw;
+          for (int jj = 0; jj < 2; ++jj) {
+            v8[2 * nt + jj] = gg[nt][jj] + gg[nt][jj + 2];
+            v8[4 + 2 * nt + jj] = gg[nt][jj] * zh[nt][jj] + gg[nt][jj + 2] * zh[nt][jj + 2];
+          }
+        const float bw = reduce_scatter8(v8, g);
+        sm.bwd[pub_tok][4 * (g >> 2) + warp] = bw;
+      }
       if (LOSS) {
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt)
@@ -421,12 +477,13 @@ __global__ void __launch_bounds__(kLnThreads, 1)
         const float lw = reduce_scatter8(v8, g);
         if (g < 4) sm.lossp[pub_tok][warp] = lw;
       }
-      compute_sync<kLnWarps>();
+      if (LN || LOSS) compute_sync<kLnWarps>();
 
-      // ---- dZ = rstd·(g − mean g − ẑ·mean(g·ẑ)); W ← W − (η/b)·Kᵀ·dZ. Each lane sums the
-      // four warps' partials of the value it published; the token group shares the means.
+      // ---- dZ (LayerNorm: rstd·(g − mean g − ẑ·mean(g·ẑ)); plain: the residual), zero for
+      // padding tokens; W ← W − (η/n)·Kᵀ·dZ. Each lane sums the four warps' partials of the
+      // value it published; the token group shares the means.
       float dz[2][4], bm[8];
-      {
+      if (LN) {
         const float4 A = *reinterpret_cast<const float4*>(&sm.bwd[pub_tok][4 * (g >> 2)]);
         all_gather8(((A.x + A.y) + (A.z + A.w)) * (1.f / 64.f), bm, g);
       }
@@ -435,15 +492,17 @@ __global__ void __launch_bounds__(kLnThreads, 1)
 #pragma unroll
         for (int jj = 0; jj < 2; ++jj) {
           const int i = 2 * nt + jj;
+          const bool real = 8 * nt + 2 * q + jj < nval;
 #pragma unroll
           for (int hc = 0; hc < 2; ++hc) {
             const int e = jj + 2 * hc;
-            dz[nt][e] = -lr * (rs[i] * (gg[nt][e] - bm[i] - zh[nt][e] * bm[4 + i]));
+            const float d = LN ? rs[i] * (gg[nt][e] - bm[i] - zh[nt][e] * bm[4 + i]) : gg[nt][e];
+            dz[nt][e] = real ? -lr * d : 0.f;
           }
         }
       if (LOSS && warp == 0) {
         const float4 L = *reinterpret_cast<const float4*>(&sm.lossp[pub_tok][0]);
-        if (g < 4) loss[(size_t)bh * T + (size_t)s * kTileTokI + r0 + pub_tok] = (L.x + L.y) + (L.z + L.w);
+        if (g < 4) a.loss[(size_t)bh * T + (size_t)s * kTileTokI + r0 + pub_tok] = (L.x + L.y) + (L.z + L.w);
       }
       uint32_t shi[4], slo[4];
       afrag_hilo(dz[0], dz[1], shi, slo);
@@ -474,10 +533,14 @@ __global__ void __launch_bounds__(kLnThreads, 1)
 #pragma unroll
           for (int e = 0; e < 4; ++e) o[nt][e] += o2[e];
         }
-        publish_stats<true, false>(z, o, sm.fwd, pub_tok, warp, g);
-        compute_sync<kLnWarps>();
-        gather_stats(sm.fwd, pub_tok, g, eps, mu, rs);
-        emit_outputs(o, qv, mu, rs, gam, bet, obase, ofs_o, r0);
+        if (LN) {
+          publish_stats<true, false>(z, o, sm.fwd, pub_tok, warp, g);
+          compute_sync<kLnWarps>();
+          gather_stats(sm.fwd, pub_tok, g, a.eps, mu, rs);
+          emit_outputs(o, qv, mu, rs, gam, bet, obase, ofs_o, r0);
+        } else {
+          emit_plain(o, obase, ofs_o, r0);
+        }
       }
     }
     // End of the tile: its outputs are complete in shared memory.
@@ -586,13 +649,14 @@ template <bool HAS_Q, bool LOSS, bool TW>
 __global__ void __launch_bounds__(kMlpThreads, 1)
     k_inner_mlp(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                 const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
-                float* __restrict__ Wstate, const float* __restrict__ gamma, const float* __restrict__ beta,
-                float* __restrict__ loss, int T, int heads, float lr, float eps, const DevStatus status) {
+                const InnerArgs a) {
   extern __shared__ uint8_t smem_raw[];
   MlpSmem& sm = *reinterpret_cast<MlpSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, q = lane & 3, mi = lane >> 3, ri = lane & 7;
   const int bh = blockIdx.x;
+  const int T = a.T;
+  const float eps = a.eps;
   const int ntiles = (T + kTileTokI - 1) / kTileTokI;
   const uint32_t stage_bytes = (HAS_Q ? 3u : 2u) * kTileBytesI;
 
@@ -613,42 +677,47 @@ __global__ void __launch_bounds__(kMlpThreads, 1)
   __syncthreads();
 
   // Per head: W1 [64][256] then W2 [256][64], row-major fp32.
-  float* W1g = Wstate + (size_t)bh * 2 * 64 * kHid;
+  float* W1g = a.W + (size_t)bh * 2 * 64 * kHid;
   float* W2g = W1g + 64 * kHid;
+  const float* W10 = a.W0 + (size_t)bh * 2 * 64 * kHid;
   const int hid0 = 32 * warp;
   // a1[mt][nt][e] = W1ᵀ[hid0 + 16mt + g + 8(e>>1)][8nt + 2q + (e&1)]
   // a2[mt][nt][e] = W2ᵀ[16mt + g + 8(e>>1)][hid0 + 8nt + 2q + (e&1)]
   float a1[2][8][4], a2[4][4][4];
+  auto load_w = [&](const float* w1, const float* w2) {
 #pragma unroll
-  for (int mt = 0; mt < 2; ++mt)
+    for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-    for (int nt = 0; nt < 8; ++nt)
+      for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
-      for (int e = 0; e < 4; ++e)
-        a1[mt][nt][e] = W1g[(8 * nt + 2 * q + (e & 1)) * kHid + hid0 + 16 * mt + g + 8 * (e >> 1)];
+        for (int e = 0; e < 4; ++e)
+          a1[mt][nt][e] = w1[(8 * nt + 2 * q + (e & 1)) * kHid + hid0 + 16 * mt + g + 8 * (e >> 1)];
 #pragma unroll
-  for (int mt = 0; mt < 4; ++mt)
+    for (int mt = 0; mt < 4; ++mt)
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt)
+      for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-      for (int e = 0; e < 4; ++e)
-        a2[mt][nt][e] = W2g[(hid0 + 8 * nt + 2 * q + (e & 1)) * 64 + 16 * mt + g + 8 * (e >> 1)];
+        for (int e = 0; e < 4; ++e)
+          a2[mt][nt][e] = w2[(hid0 + 8 * nt + 2 * q + (e & 1)) * 64 + 16 * mt + g + 8 * (e >> 1)];
+  };
+  load_w(W1g, W2g);
+  const int2* steps = a.steps == nullptr ? nullptr : a.steps + (size_t)(bh / a.heads) * a.nsteps;
 
   // LayerNorm stage: token 2·warp + (lane >> 4), columns c0 .. c0+3.
   const int ltok = 2 * warp + (lane >> 4), c0 = 4 * (lane & 15);
-  const int h = bh % heads;
+  const int h = bh % a.heads;
   float gam[4], bet[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    gam[i] = gamma[h * 64 + c0 + i];
-    bet[i] = beta[h * 64 + c0 + i];
+    gam[i] = a.gamma[h * 64 + c0 + i];
+    bet[i] = a.beta[h * 64 + c0 + i];
   }
   const uint32_t sbase[2] = {smem_u32(sm.S[0]), smem_u32(sm.S[1])};
 
   int s = 0;
   for (; s < ntiles; ++s) {
     const int slot = s % kStagesM;
-    if (!mbar_wait(&sm.full[slot], (s / kStagesM) & 1, status, nullptr)) sm.cabort[s & 1] = 1;
+    if (!mbar_wait(&sm.full[slot], (s / kStagesM) & 1, a.status, nullptr)) sm.cabort[s & 1] = 1;
     compute_sync<kMlpWarps>();
     if (*reinterpret_cast<volatile int*>(&sm.cabort[s & 1])) break;
     const int ntok = min(kTileTokI, T - s * kTileTokI);
@@ -659,6 +728,13 @@ __global__ void __launch_bounds__(kMlpThreads, 1)
     uint8_t* obuf = sm.O[s & 1];
 
     for (int r0 = 0; r0 < ntok; r0 += kMB) {
+      int nval = kMB;  // real tokens of this mini-batch (packed sequences: see k_inner_ln)
+      if (steps != nullptr) {
+        const int2 e = steps[s * (kTileTokI / kMB) + r0 / kMB];
+        if (e.x) load_w(W10, W10 + 64 * kHid);  // a document starts: the pretrained weights
+        nval = e.y;
+      }
+      const float lr = a.eta / (float)max(nval, 1);
       constexpr bool kQNow = HAS_Q && !TW;  // the queries' path alongside the keys'
       // ---- first layer: Hᵀ = W1ᵀ·Kᵀ (and for the queries), hidden x tokens
       float hk[2][2][4], hq[2][2][4];
@@ -795,14 +871,14 @@ __global__ void __launch_bounds__(kMlpThreads, 1)
         float sv[4], sl[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          sv[i] = -lr * (rstd * (gg[i] - mg - zh[i] * mgz));
+          sv[i] = ltok < nval ? -lr * (rstd * (gg[i] - mg - zh[i] * mgz)) : 0.f;  // padding: no gradient
           sl[i] = sv[i] - __bfloat162float(__float2bfloat16_rn(sv[i]));
         }
         store4_bf16(sm.S[0], ltok, c0, sv);  // rounds to the hi part
         store4_bf16(sm.S[1], ltok, c0, sl);
         if (LOSS) {
           se = sum16(se);
-          if ((lane & 15) == 0) loss[(size_t)bh * T + (size_t)s * kTileTokI + r0 + ltok] = se;
+          if ((lane & 15) == 0) a.loss[(size_t)bh * T + (size_t)s * kTileTokI + r0 + ltok] = se;
         }
       }
       // Outputs of tokens 2w, 2w+1: q + γ·LN(Σ partial Zᵀ of the queries) + β.
@@ -994,7 +1070,7 @@ __global__ void __launch_bounds__(kMlpThreads, 1)
     if (HAS_Q) bulk_wait<0>();
     // Nothing may still be landing in shared memory when the CTA exits (after an abort the
     // tiles issued past the last one consumed).
-    for (int t = s; t < issued; ++t) mbar_wait(&sm.full[t % kStagesM], (t / kStagesM) & 1, status, nullptr);
+    for (int t = s; t < issued; ++t) mbar_wait(&sm.full[t % kStagesM], (t / kStagesM) & 1, a.status, nullptr);
   }
 #pragma unroll
   for (int mt = 0; mt < 2; ++mt)
@@ -1014,22 +1090,22 @@ __global__ void __launch_bounds__(kMlpThreads, 1)
 }
 
 template <bool HAS_Q, bool LOSS, bool TW>
-ttt_status launch_inner(ttt_state* st, const CUtensorMap* maps, float* loss, int T, cudaStream_t s) {
+ttt_status launch_inner(ttt_state* st, const CUtensorMap* maps, float* loss, int T, const int2* steps,
+                        cudaStream_t s) {
   const ttt_config& c = st->cfg;
-  const bool mlp = c.rule == TTT_RULE_MLP_GD;
+  const bool mlp = c.rule == TTT_RULE_MLP_GD, ln = c.rule == TTT_RULE_LINEAR_LN_GD;
   const size_t smem = (mlp ? sizeof(MlpSmem) : sizeof(LnSmem)) + 1024;
   // One bit per instantiation whose shared-memory limit has been raised on this state's device.
-  const uint64_t bit = 1ull << (48 + 8 * mlp + 4 * TW + 2 * HAS_Q + LOSS);
-  auto kernel = mlp ? k_inner_mlp<HAS_Q, LOSS, TW> : k_inner_ln<HAS_Q, LOSS, TW>;
+  const uint64_t bit = 1ull << (40 + 8 * (mlp ? 2 : ln ? 1 : 0) + 4 * TW + 2 * HAS_Q + LOSS);
+  auto kernel = mlp ? k_inner_mlp<HAS_Q, LOSS, TW> : ln ? k_inner_ln<HAS_Q, LOSS, TW, true> : k_inner_ln<HAS_Q, LOSS, TW, false>;
   if (!(st->lin.smem_set & bit)) {
     TTT_CUDA(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
     st->lin.smem_set |= bit;
   }
   const int grid = c.batch * c.heads;
-  const float lr = c.eta / (float)kMB;
-  kernel<<<grid, mlp ? kMlpThreads : kLnThreads, smem, s>>>(
-      maps[0], maps[1], maps[2], maps[3], st->lin.W, st->lin.ln_gamma, st->lin.ln_beta, loss, T, c.heads, lr,
-      c.ln_eps, DevStatus{st->status.dev, st->wait_limit_ns, st->status.dev + 1});
+  InnerArgs a{st->lin.W, st->lin.W0, st->lin.ln_gamma, st->lin.ln_beta, loss, steps, T, c.heads, T / kMB,
+              c.eta, c.ln_eps, DevStatus{st->status.dev, st->wait_limit_ns, st->status.dev + 1}};
+  kernel<<<grid, mlp ? kMlpThreads : kLnThreads, smem, s>>>(maps[0], maps[1], maps[2], maps[3], a);
   st->launches++;
   TTT_CUDA(cudaGetLastError());
   return TTT_OK;
@@ -1037,8 +1113,9 @@ ttt_status launch_inner(ttt_state* st, const CUtensorMap* maps, float* loss, int
 
 }  // namespace
 
-ttt_status inner_scan(ttt_state* st, const __nv_bfloat16* K, const __nv_bfloat16* V, const __nv_bfloat16* Q,
-                      int64_t T, __nv_bfloat16* O, float* loss, cudaStream_t s) {
+// One launch over [B·H, T, 64] buffers (T a multiple of 16 when steps is set).
+static ttt_status inner_launch(ttt_state* st, const __nv_bfloat16* K, const __nv_bfloat16* V, const __nv_bfloat16* Q,
+                               int64_t T, __nv_bfloat16* O, float* loss, const int2* steps, cudaStream_t s) {
   const ttt_config& c = st->cfg;
   // [B·H, T, 64] bf16 views of K, V, Q and O, 64-token boxes with the 128-byte swizzle; the maps
   // of the last few buffer sets are kept (encoding costs microseconds of host time).
@@ -1067,13 +1144,146 @@ ttt_status inner_scan(ttt_state* st, const __nv_bfloat16* K, const __nv_bfloat16
   ms->last_use = ++lb.map_clock;
   // Per-token weights change only the outputs.
   if (has_q && c.token_weights)
-    return loss ? launch_inner<true, true, true>(st, ms->maps, loss, (int)T, s)
-                : launch_inner<true, false, true>(st, ms->maps, loss, (int)T, s);
+    return loss ? launch_inner<true, true, true>(st, ms->maps, loss, (int)T, steps, s)
+                : launch_inner<true, false, true>(st, ms->maps, loss, (int)T, steps, s);
   if (has_q)
-    return loss ? launch_inner<true, true, false>(st, ms->maps, loss, (int)T, s)
-                : launch_inner<true, false, false>(st, ms->maps, loss, (int)T, s);
-  return loss ? launch_inner<false, true, false>(st, ms->maps, loss, (int)T, s)
-              : launch_inner<false, false, false>(st, ms->maps, loss, (int)T, s);
+    return loss ? launch_inner<true, true, false>(st, ms->maps, loss, (int)T, steps, s)
+                : launch_inner<true, false, false>(st, ms->maps, loss, (int)T, steps, s);
+  return loss ? launch_inner<false, true, false>(st, ms->maps, loss, (int)T, steps, s)
+              : launch_inner<false, false, false>(st, ms->maps, loss, (int)T, steps, s);
+}
+
+ttt_status inner_scan(ttt_state* st, const __nv_bfloat16* K, const __nv_bfloat16* V, const __nv_bfloat16* Q,
+                      int64_t T, __nv_bfloat16* O, float* loss, cudaStream_t s) {
+  return inner_launch(st, K, V, Q, T, O, loss, nullptr, s);
+}
+
+namespace {
+
+// Row r of the padded [B·H, Tp, 64] layout takes input row rows[b·Tp + t] of its (sequence, head)
+// (zero where that is -1). One thread a 16-byte vector.
+__global__ void k_gather_heads(const __nv_bfloat16* __restrict__ src, __nv_bfloat16* __restrict__ dst,
+                               const int32_t* __restrict__ rows, int H, int T, int Tp, long long nrows) {
+  const long long n = nrows * 8;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const long long r = i >> 3;
+    const int c = (int)(i & 7);
+    const long long bh = r / Tp;
+    const int tp = (int)(r % Tp);
+    const int32_t from = rows[(bh / H) * Tp + tp];
+    uint4 x = make_uint4(0u, 0u, 0u, 0u);
+    if (from >= 0) x = reinterpret_cast<const uint4*>(src + (bh * T + from) * 64)[c];
+    reinterpret_cast<uint4*>(dst + r * 64)[c] = x;
+  }
+}
+
+// The inverse for the outputs (bf16 rows) and the losses (one float a row); padding rows are
+// dropped.
+__global__ void k_scatter_heads(const __nv_bfloat16* __restrict__ srcO, __nv_bfloat16* __restrict__ dstO,
+                                const float* __restrict__ srcL, float* __restrict__ dstL,
+                                const int32_t* __restrict__ rows, int H, int T, int Tp, long long nrows) {
+  const long long n = nrows * 8;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const long long r = i >> 3;
+    const int c = (int)(i & 7);
+    const long long bh = r / Tp;
+    const int tp = (int)(r % Tp);
+    const int32_t to = rows[(bh / H) * Tp + tp];
+    if (to < 0) continue;
+    if (srcO != nullptr) reinterpret_cast<uint4*>(dstO + (bh * T + to) * 64)[c] = reinterpret_cast<const uint4*>(srcO + r * 64)[c];
+    if (srcL != nullptr && c == 0) dstL[bh * T + to] = srcL[r];
+  }
+}
+
+int grid_for(long long n) {
+  const long long b = (n + 255) / 256;
+  return (int)(b < 148 * 16 ? (b < 1 ? 1 : b) : 148 * 16);
+}
+
+}  // namespace
+
+void free_packed(ttt_state* st) {
+  LinearBuffers& lb = st->lin;
+  for (auto*& p : lb.pk) {
+    if (p != nullptr) cudaFree(p);
+    p = nullptr;
+  }
+  if (lb.pk_loss != nullptr) cudaFree(lb.pk_loss);
+  if (lb.pk_rows != nullptr) cudaFree(lb.pk_rows);
+  if (lb.pk_steps != nullptr) cudaFree(lb.pk_steps);
+  lb.pk_loss = nullptr;
+  lb.pk_rows = nullptr;
+  lb.pk_steps = nullptr;
+  lb.pk_cap = lb.pk_map_cap = 0;
+}
+
+ttt_status inner_scan_packed(ttt_state* st, const __nv_bfloat16* K, const __nv_bfloat16* V, const __nv_bfloat16* Q,
+                             int64_t T, __nv_bfloat16* O, float* loss, const int64_t* doc_starts,
+                             const int32_t* docs_per_seq, cudaStream_t s) {
+  const ttt_config& c = st->cfg;
+  const int B = c.batch, H = c.heads;
+  // Layout: every document padded to whole mini-batches; the sequences padded to the longest.
+  std::vector<int64_t> padded(B, 0);
+  int64_t off = 0;
+  for (int b = 0; b < B; ++b) {
+    for (int k = 0; k < docs_per_seq[b]; ++k) {
+      const int64_t a = doc_starts[off + k], e = k + 1 < docs_per_seq[b] ? doc_starts[off + k + 1] : T;
+      padded[b] += (e - a + kMB - 1) / kMB * kMB;
+    }
+    off += docs_per_seq[b];
+  }
+  int64_t Tp = kMB;
+  for (int64_t p : padded) Tp = std::max(Tp, p);
+  if (Tp > (int64_t)INT32_MAX / 4) return fail(TTT_ERR_UNSUPPORTED, "packed layout too long");
+  const int64_t nsteps = Tp / kMB;
+  std::vector<int32_t> rows((size_t)(B * Tp), -1);
+  std::vector<int2> steps((size_t)(B * nsteps), make_int2(0, 0));
+  off = 0;
+  for (int b = 0; b < B; ++b) {
+    int64_t p = 0;
+    for (int k = 0; k < docs_per_seq[b]; ++k) {
+      const int64_t a = doc_starts[off + k], e = k + 1 < docs_per_seq[b] ? doc_starts[off + k + 1] : T;
+      for (int64_t t0 = a; t0 < e; t0 += kMB, p += kMB) {
+        const int n = (int)std::min<int64_t>(kMB, e - t0);
+        steps[(size_t)(b * nsteps + p / kMB)] = make_int2(t0 == a ? 1 : 0, n);
+        for (int j = 0; j < n; ++j) rows[(size_t)(b * Tp + p + j)] = (int32_t)(t0 + j);
+      }
+    }
+    off += docs_per_seq[b];
+  }
+  // Scratch, grown on demand.
+  LinearBuffers& lb = st->lin;
+  const int64_t nrows = (int64_t)B * H * Tp;
+  if (nrows > lb.pk_cap || B * Tp > lb.pk_map_cap) {
+    free_packed(st);
+    const size_t rb = (size_t)nrows * 128;
+    for (auto*& p : lb.pk) TTT_CUDA(cudaMalloc(reinterpret_cast<void**>(&p), rb));
+    TTT_CUDA(cudaMalloc(reinterpret_cast<void**>(&lb.pk_loss), (size_t)nrows * 4));
+    TTT_CUDA(cudaMalloc(reinterpret_cast<void**>(&lb.pk_rows), (size_t)(B * Tp) * 4));
+    TTT_CUDA(cudaMalloc(reinterpret_cast<void**>(&lb.pk_steps), (size_t)(B * nsteps) * sizeof(int2)));
+    lb.pk_cap = nrows;
+    lb.pk_map_cap = B * Tp;
+  }
+  TTT_CUDA(cudaMemcpyAsync(lb.pk_rows, rows.data(), rows.size() * 4, cudaMemcpyHostToDevice, s));
+  TTT_CUDA(cudaMemcpyAsync(lb.pk_steps, steps.data(), steps.size() * sizeof(int2), cudaMemcpyHostToDevice, s));
+  const int gb = grid_for(nrows * 8);
+  k_gather_heads<<<gb, 256, 0, s>>>(K, lb.pk[0], lb.pk_rows, H, (int)T, (int)Tp, nrows);
+  k_gather_heads<<<gb, 256, 0, s>>>(V, lb.pk[1], lb.pk_rows, H, (int)T, (int)Tp, nrows);
+  st->launches += 2;
+  if (Q != nullptr) {
+    k_gather_heads<<<gb, 256, 0, s>>>(Q, lb.pk[2], lb.pk_rows, H, (int)T, (int)Tp, nrows);
+    st->launches++;
+  }
+  TTT_CUDA(cudaGetLastError());
+  TTT_TRY(inner_launch(st, lb.pk[0], lb.pk[1], Q != nullptr ? lb.pk[2] : nullptr, Tp, Q != nullptr ? lb.pk[3] : nullptr,
+                       loss != nullptr ? lb.pk_loss : nullptr, lb.pk_steps, s));
+  if (O != nullptr || loss != nullptr) {
+    k_scatter_heads<<<gb, 256, 0, s>>>(O != nullptr ? lb.pk[3] : nullptr, O, loss != nullptr ? lb.pk_loss : nullptr, loss,
+                                       lb.pk_rows, H, (int)T, (int)Tp, nrows);
+    st->launches++;
+    TTT_CUDA(cudaGetLastError());
+  }
+  return TTT_OK;
 }
 
 }  // namespace ttt

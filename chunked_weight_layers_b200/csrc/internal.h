@@ -97,6 +97,16 @@ struct LinearBuffers {
   // Inner mini-batches per chunk of the b = 16 scan (TTT_OPT_LINEAR_CHUNK): 1 = one step at a
   // time, 2 or 4 = the chunked form; 0 = the library's choice (1).
   int form = 0;
+  // Packed sequences (ttt_chunk_scan_packed): K, V, Q, O with every document padded to whole
+  // mini-batches [B, H, Tp, 64], the losses [B, H, Tp], the padded row -> input token map
+  // [B, Tp] (-1: padding) and the per-(sequence, mini-batch) {reset, real tokens} table,
+  // grown on demand.
+  __nv_bfloat16* pk[4] = {nullptr, nullptr, nullptr, nullptr};
+  float* pk_loss = nullptr;
+  int32_t* pk_rows = nullptr;
+  int2* pk_steps = nullptr;
+  int64_t pk_cap = 0;      // rows of pk[] (B·H·Tp)
+  int64_t pk_map_cap = 0;  // entries of pk_rows (B·Tp)
 };
 
 struct GateBuffers {
@@ -165,10 +175,18 @@ ttt_status linear_scan(ttt_state* st, const __nv_bfloat16* K, const __nv_bfloat1
                        const __nv_bfloat16* Q, int64_t T, __nv_bfloat16* O, float* loss,
                        cudaStream_t s);
 
-// TTT-Linear with LayerNorm and residual, or TTT-MLP: the scan over T tokens of every
-// (sequence, head), mini-batch 16.
+// TTT-Linear with LayerNorm and residual, TTT-MLP, or the plain TTT-Linear rule with per-token
+// weights: the scan over T tokens of every (sequence, head), mini-batch 16.
 ttt_status inner_scan(ttt_state* st, const __nv_bfloat16* K, const __nv_bfloat16* V, const __nv_bfloat16* Q,
                       int64_t T, __nv_bfloat16* O, float* loss, cudaStream_t s);
+
+// The same over packed sequences: sequence b holds docs_per_seq[b] documents laid end to end
+// whose first tokens are the next docs_per_seq[b] entries of doc_starts (host memory); each is
+// scanned from W0 with mini-batches counted from its first token.
+ttt_status inner_scan_packed(ttt_state* st, const __nv_bfloat16* K, const __nv_bfloat16* V, const __nv_bfloat16* Q,
+                             int64_t T, __nv_bfloat16* O, float* loss, const int64_t* doc_starts,
+                             const int32_t* docs_per_seq, cudaStream_t s);
+void free_packed(ttt_state* st);
 
 // Residual-cache read path: out = o_ttt + clamp(α, 0, 1) ⊙ (attention over the visible entries).
 ttt_status cache_attention(const ttt_state* st, const __nv_bfloat16* Q, const __nv_bfloat16* K,

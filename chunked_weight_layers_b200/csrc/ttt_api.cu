@@ -49,8 +49,11 @@ static void dev_free(void* p) {
 }
 
 static ttt_status validate(const ttt_config* c) {
-  if (c->token_weights != 0 && c->rule != TTT_RULE_LINEAR_LN_GD && c->rule != TTT_RULE_MLP_GD)
-    return fail(TTT_ERR_UNSUPPORTED, "per-token weights apply to the LayerNorm inner models only");
+  if (c->token_weights != 0 && c->token_weights != 1) return fail(TTT_ERR_INVALID_ARG, "token_weights must be 0 or 1");
+  if (c->token_weights && c->rule == TTT_RULE_INPLACE_HEBBIAN)
+    return fail(TTT_ERR_UNSUPPORTED, "per-token weights apply to the TTT-Linear family");
+  if (c->token_weights && c->rule == TTT_RULE_LINEAR_GD && (c->chunk != 16 || c->gate_enable))
+    return fail(TTT_ERR_UNSUPPORTED, "TTT-Linear per-token weights: mini-batch 16, no gate");
   if (c->rule == TTT_RULE_INPLACE_HEBBIAN) {
     if (c->batch != 1 || c->heads != 1)
       return fail(TTT_ERR_UNSUPPORTED, "In-Place scan: batch and heads must be 1 (one Wdown state)");
@@ -104,8 +107,6 @@ static ttt_status validate(const ttt_config* c) {
     if (c->target_mode != 0) return fail(TTT_ERR_INVALID_ARG, "target_mode applies to In-Place only");
     if (c->gate_enable) return fail(TTT_ERR_UNSUPPORTED, "the surprisal gate runs on TTT-Linear states");
     if (!(c->ln_eps > 0.f)) return fail(TTT_ERR_INVALID_ARG, "%s: ln_eps must be positive", name);
-    if (c->token_weights != 0 && c->token_weights != 1)
-      return fail(TTT_ERR_INVALID_ARG, "token_weights must be 0 or 1");
     return TTT_OK;
   }
   return fail(TTT_ERR_INVALID_ARG, "unknown rule %d", c->rule);
@@ -143,6 +144,7 @@ static void free_state(ttt_state* st) {
   dev_free(st->lin.W0);
   dev_free(st->lin.ln_gamma);
   dev_free(st->lin.ln_beta);
+  free_packed(st);
   dev_free(st->gate.tau);
   dev_free(st->gate.tau_set);
   dev_free(st->gate.entries);
@@ -327,7 +329,7 @@ static ttt_status scan_impl(ttt_state* st, const void* keys, const void* targets
   if (queries != nullptr && (!aligned16(queries) || !aligned16(out)))
     return fail(TTT_ERR_INVALID_ARG, "queries and out must be 16-byte aligned");
   if (loss != nullptr && !aligned16(loss)) return fail(TTT_ERR_INVALID_ARG, "loss_out must be 16-byte aligned");
-  if (c.rule != TTT_RULE_LINEAR_GD)
+  if (c.rule != TTT_RULE_LINEAR_GD || c.token_weights)
     return inner_scan(st, static_cast<const __nv_bfloat16*>(keys), static_cast<const __nv_bfloat16*>(targets),
                       static_cast<const __nv_bfloat16*>(queries), T, static_cast<__nv_bfloat16*>(out), loss, s);
   if (c.gate_enable) {
@@ -423,6 +425,42 @@ ttt_status ttt_chunk_scan_docs(ttt_state* st, const void* keys, const void* targ
   return inplace_bf16_scan_docs(st, static_cast<const __nv_bfloat16*>(keys), static_cast<const __nv_bfloat16*>(targets),
                                 T, doc_starts, (int)ndocs, clip_norm, static_cast<__nv_bfloat16*>(out),
                                 reinterpret_cast<cudaStream_t>(stream));
+}
+
+ttt_status ttt_chunk_scan_packed(ttt_state* st, const void* keys, const void* targets, const void* queries, int64_t T,
+                                 void* out, float* loss_out, const int64_t* doc_starts, const int32_t* docs_per_seq,
+                                 ttt_stream stream) {
+  if (st == nullptr) return fail(TTT_ERR_INVALID_ARG, "state is NULL");
+  const ttt_config& c = st->cfg;
+  if (c.rule == TTT_RULE_INPLACE_HEBBIAN)
+    return fail(TTT_ERR_UNSUPPORTED, "In-Place states take packed sequences through ttt_chunk_scan_docs");
+  if (c.chunk != 16 || c.gate_enable)
+    return fail(TTT_ERR_UNSUPPORTED, "packed sequences: mini-batch 16, no gate");
+  if (T < 0 || T > (int64_t)INT32_MAX / 4) return fail(TTT_ERR_INVALID_ARG, "T out of range");
+  if (T == 0) return TTT_OK;
+  if (doc_starts == nullptr || docs_per_seq == nullptr)
+    return fail(TTT_ERR_INVALID_ARG, "doc_starts and docs_per_seq are required (host memory)");
+  int64_t off = 0;
+  for (int b = 0; b < c.batch; ++b) {
+    const int32_t n = docs_per_seq[b];
+    if (n < 1) return fail(TTT_ERR_INVALID_ARG, "sequence %d lists no document", b);
+    if (doc_starts[off] != 0) return fail(TTT_ERR_INVALID_ARG, "sequence %d: the first document must start at 0", b);
+    for (int32_t k = 1; k < n; ++k)
+      if (doc_starts[off + k] <= doc_starts[off + k - 1])
+        return fail(TTT_ERR_INVALID_ARG, "sequence %d: document starts must increase strictly", b);
+    if (doc_starts[off + n - 1] >= T) return fail(TTT_ERR_INVALID_ARG, "sequence %d: every document must start below T", b);
+    off += n;
+  }
+  if ((queries == nullptr) != (out == nullptr))
+    return fail(TTT_ERR_INVALID_ARG, "out must be given exactly when queries are");
+  const void* p[5] = {keys, targets, queries, out, loss_out};
+  for (int i = 0; i < 5; ++i)
+    if ((i < 2 && p[i] == nullptr) || (p[i] != nullptr && !aligned16(p[i])))
+      return fail(TTT_ERR_INVALID_ARG, "keys and targets (and queries, out, loss_out when given) must be 16-byte aligned device pointers");
+  TTT_TRY(check_device(st));
+  return inner_scan_packed(st, static_cast<const __nv_bfloat16*>(keys), static_cast<const __nv_bfloat16*>(targets),
+                           static_cast<const __nv_bfloat16*>(queries), T, static_cast<__nv_bfloat16*>(out), loss_out,
+                           doc_starts, docs_per_seq, reinterpret_cast<cudaStream_t>(stream));
 }
 
 ttt_status ttt_chunk_scan_host(ttt_state* st, const void* keys, const void* targets, const void* queries,

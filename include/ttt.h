@@ -112,11 +112,12 @@ typedef struct {
   int32_t gate_mean_num;  /* the mean test is S/gate_chunk >= (num/den)·τ; 4 */
   int32_t gate_mean_den;  /* 5 */
   float ln_eps;           /* TTT_RULE_LINEAR_LN_GD and TTT_RULE_MLP_GD: LayerNorm ε; 1e-6 */
-  int32_t token_weights;  /* TTT_RULE_LINEAR_LN_GD and TTT_RULE_MLP_GD: 0 (default): the outputs of a
+  int32_t token_weights;  /* TTT-Linear family: 0 (default): the outputs of a
                              mini-batch use its starting weights θ_i. 1: per-token weights, output t
                              uses θ_i − (η/b)·Σ_{s ≤ t} ∇½‖f(k_s; θ_i) − v_s‖² over the mini-batch's
                              tokens s up to t (the last token sees θ_{i+1}); losses and the weight
-                             update are unchanged. Other rules: must be 0. */
+                             update are unchanged. Also TTT_RULE_LINEAR_GD with mini-batch 16 and no
+                             gate (the dual form of the plain rule). In-Place: must be 0. */
 } ttt_config;
 
 typedef struct ttt_state ttt_state; /* opaque; owns all of its device memory */
@@ -193,6 +194,27 @@ ttt_status ttt_chunk_scan_host(ttt_state* st, const void* keys, const void* targ
  * clipped). */
 ttt_status ttt_chunk_scan_docs(ttt_state* st, const void* keys, const void* targets, int64_t T, void* out,
                                const int64_t* doc_starts, int32_t ndocs, float clip_norm, ttt_stream stream);
+
+/* Packed sequences for the TTT-Linear family (plain, LayerNorm and MLP rules; mini-batch 16, no
+ * gate): sequence b of the batch holds docs_per_seq[b] documents laid end to end, whose first
+ * tokens are the next docs_per_seq[b] entries of doc_starts (host memory, sequence after
+ * sequence; each sequence's list starts at 0, increases strictly and stays below T). Each
+ * document is scanned as if alone: the weights of every head start from the pretrained W0,
+ * mini-batches are counted from its first token, and its last mini-batch may be shorter: with
+ * b' < 16 tokens it takes the step of its own loss (η/b' for the plain rule). T need not be a
+ * multiple of 16. keys, targets, queries (or NULL), out (NULL iff queries is NULL) and loss_out
+ * (or NULL) are laid out as for ttt_chunk_scan, [batch, heads, T, ...]; afterwards the state holds
+ * each sequence's last document's final weights. Per-token weights (token_weights = 1) apply
+ * within every mini-batch. Runs one scan launch over a padded copy (state-owned scratch grown
+ * on demand, with gather and scatter launches around it) and synchronises (the layout goes up
+ * from host memory). Errors: INVALID_ARG (malformed document lists, misaligned buffers),
+ * UNSUPPORTED (In-Place states, other mini-batches, the gate), CUDA. Defined by "In-Place
+ * Test-Time Training", §6 and the notes after it (the weights go back to their pretrained value
+ * at each independent document) and the TTT layers page (the hidden state is the inner model's
+ * weight, so a new sequence starts it afresh). */
+ttt_status ttt_chunk_scan_packed(ttt_state* st, const void* keys, const void* targets, const void* queries, int64_t T,
+                                 void* out, float* loss_out, const int64_t* doc_starts, const int32_t* docs_per_seq,
+                                 ttt_stream stream);
 
 /* Run the surprisal gate alone on a loss array `loss` (device, fp32 [batch, heads, T]),
  * advancing the state's τ, cache and token position exactly as a gated scan would.
