@@ -614,6 +614,97 @@ def cpu_baseline_docs(limit_s) -> dict:
             "kind": "oracle", "sample": f"{chunks} chunk(s) of {spec.C} tokens (one document, clipped)", "seconds": dt}
 
 
+PACKED = wl.LINEAR_GD.name + " packed (4 documents per sequence)"
+PACKED_SEED, PACKED_N = 1009, 4
+
+
+def packed_starts(spec):
+    """Seeded ragged document starts of every sequence (at least 16 tokens a document)."""
+    return [wl.document_starts(spec.T, PACKED_N, PACKED_SEED + b, min_len=16) for b in range(spec.B)]
+
+
+def measure_packed(steps, warmup, peaks, device):
+    """ttt_chunk_scan_packed on the TTT-Linear workload: every sequence as four documents of seeded
+    ragged lengths, each scanned from W0 with its own mini-batches (a shorter last one). The
+    scan runs in the LayerNorm kernel's plain mode over a padded copy, with gather and scatter
+    launches around it; work counts the real tokens."""
+    import chunked_weight_layers_b200 as cwl
+    spec = wl.LINEAR_GD
+    starts = packed_starts(spec)
+    x = wl.linear_inputs(spec, device=device)
+    cfg = cwl.config("linear", batch=spec.B, heads=spec.H, chunk=spec.b, eta=spec.eta)
+    st = cwl.FastWeightState(cfg, x["W0"])
+    O = torch.empty_like(x["K"])
+    w = work(spec)
+    for _ in range(warmup):
+        st.chunk_scan_packed(x["K"], x["V"], starts, queries=x["Q"], out=O)
+    torch.cuda.synchronize()
+    n0 = st.launch_count()
+    stream = torch.cuda.current_stream()
+    times = []
+    for _ in range(steps):  # the call synchronises (its layout goes up from host memory): time each
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        st.chunk_scan_packed(x["K"], x["V"], starts, queries=x["Q"], out=O)
+        e1.record(stream)
+        e1.synchronize()
+        times.append(e0.elapsed_time(e1))
+    st.poll()
+    launches = (st.launch_count() - n0) / steps
+    ms = sum(times) / steps
+    achieved = w["bytes"] / (ms * 1e-3) / 1e9
+    hk, hv, hq = (x[k].cpu().pin_memory() for k in "KVQ")
+    ho = torch.empty(O.shape, dtype=O.dtype).pin_memory()
+    dk, dv, dq = torch.empty_like(x["K"]), torch.empty_like(x["V"]), torch.empty_like(x["Q"])
+    e2e = []
+    for _ in range(3):
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        dq.copy_(hq, non_blocking=True)
+        st.chunk_scan_packed(dk, dv, starts, queries=dq, out=O)
+        ho.copy_(O, non_blocking=True)
+        torch.cuda.synchronize()
+        e2e.append((time.perf_counter() - t0) * 1e3)
+    e2e_ms = statistics.median(e2e)
+    out = {"workload": PACKED, "doc_starts": starts, "ms_per_step": ms, "ms_median": statistics.median(times),
+           "tokens_per_s": w["tokens"] / (ms * 1e-3), "tflops": w["flops"] / (ms * 1e-3) / 1e12,
+           "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                        "frac": achieved / peaks["hbm_gbs"], "traffic": None, "peak_source": peaks["source"],
+                        "kernel": "k_inner_ln (plain mode)"},
+           "gpu_launches_per_step": launches, "times_ms": times,
+           "l2": "each call timed alone (it synchronises to upload its layout); its 100 MB of inputs are gathered into a padded copy",
+           "e2e": {"value": w["tokens"] / (e2e_ms * 1e-3), "unit": "tokens/s",
+                   "h2d_bytes_per_step": 3 * hk.numel() * 2, "d2h_bytes_per_step": ho.numel() * 2,
+                   "ms_per_step": e2e_ms}}
+    st.close()
+    del x, O, dk, dv, dq
+    torch.cuda.empty_cache()
+    return out
+
+
+def cpu_baseline_packed(limit_s) -> dict:
+    """The oracle's packed TTT-Linear scan, one (sequence, head) at a time, within the limit."""
+    from oracle import packed as opk
+    spec = wl.LINEAR_GD
+    starts = packed_starts(spec)
+    x = wl.linear_inputs(spec)
+    cores = oracle_threads()
+    t0, c0 = time.perf_counter(), time.process_time()
+    done = 0
+    while done < spec.B * spec.H and time.perf_counter() - t0 < limit_s:
+        b, h = divmod(done, spec.H)
+        sl = (slice(b, b + 1), slice(h, h + 1))
+        opk.ttt_linear_scan_docs(x["K"][sl], x["V"][sl], x["Q"][sl], x["W0"][sl], spec.eta, spec.b, [starts[b]])
+        done += 1
+    dt = time.perf_counter() - t0
+    busy = (time.process_time() - c0) / dt if dt > 0 else 0.0
+    return {"value": spec.T * done / spec.H / dt, "unit": "tokens/s", "cores": cores, "busy_threads": round(busy, 2),
+            "kind": "oracle", "sample": f"{done} of {spec.B * spec.H} (sequence, head) scans, one at a time",
+            "seconds": dt}
+
+
 def cpu_baseline_cache_read(limit_s) -> dict:
     """The oracle's read path (attention over the visible entries, α fusion) on (sequence, head)
     pairs of the gate workload's cache, one at a time, within the time limit."""
@@ -892,6 +983,10 @@ def main():
             extra[DOCS] = measure_docs(max(3, min(a.steps, 5)), 2, peaks, device)
         except Exception as ex:
             extra[DOCS] = {"error": str(ex)}
+        try:
+            extra[PACKED] = measure_packed(max(5, min(a.steps, 20)), 3, peaks, device)
+        except Exception as ex:
+            extra[PACKED] = {"error": str(ex)}
     clk.__exit__(None, None, None)
     # The oracle baselines run after the sampler stops (the GPU idles meanwhile).
     for s in list(wl.WORKLOADS.values()) + list(wl.INNER_WORKLOADS.values()):
@@ -904,6 +999,8 @@ def main():
         extra[CACHE_READ]["cpu_baseline"] = cpu_baseline_cache_read(6.0)
     if "error" not in extra.get(DOCS, {"error": 1}):
         extra[DOCS]["cpu_baseline"] = cpu_baseline_docs(6.0)
+    if "error" not in extra.get(PACKED, {"error": 1}):
+        extra[PACKED]["cpu_baseline"] = cpu_baseline_packed(6.0)
 
     if rank == 0:
         rl = roofline(spec, w, ms, peaks, traffic_per_launch(spec), timed_ms=total_ms)
