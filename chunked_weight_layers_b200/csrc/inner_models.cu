@@ -129,6 +129,7 @@ struct InnerArgs {
   int T, heads, nsteps;  // nsteps: entries of steps a sequence
   float eta, eps;
   DevStatus status;
+  int stall_tile;      // fault injection (tests): this 64-token tile is never loaded (-1: none)
 };
 
 // ============================ TTT-Linear with LayerNorm and residual ============================
@@ -283,15 +284,17 @@ __global__ void __launch_bounds__(kLnThreads, 1)
       for (int s = 0; s < ntiles; ++s) {
         const int slot = s % kStagesI;
         if (s >= kStagesI && !mbar_wait(&sm.empty[slot], ((s / kStagesI) - 1) & 1, a.status, &sm.abort)) break;
-        mbar_arrive_expect_tx(&sm.full[slot], stage_bytes);
-        tma_load_3d(sm.K[slot], &tmK, &sm.full[slot], 0, s * kTileTokI, bh);
-        tma_load_3d(sm.V[slot], &tmV, &sm.full[slot], 0, s * kTileTokI, bh);
-        if (HAS_Q) tma_load_3d(sm.Q[slot], &tmQ, &sm.full[slot], 0, s * kTileTokI, bh);
+        if (s != a.stall_tile) {
+          mbar_arrive_expect_tx(&sm.full[slot], stage_bytes);
+          tma_load_3d(sm.K[slot], &tmK, &sm.full[slot], 0, s * kTileTokI, bh);
+          tma_load_3d(sm.V[slot], &tmV, &sm.full[slot], 0, s * kTileTokI, bh);
+          if (HAS_Q) tma_load_3d(sm.Q[slot], &tmQ, &sm.full[slot], 0, s * kTileTokI, bh);
+        }
         issued = s + 1;
       }
       // Nothing may still be landing in shared memory when the CTA exits.
       for (int s = issued - kStagesI; s < issued; ++s) {
-        if (s < 0) continue;
+        if (s < 0 || s == a.stall_tile) continue;
         mbar_wait(&sm.full[s % kStagesI], (s / kStagesI) & 1, a.status, nullptr);
       }
     }
@@ -661,6 +664,7 @@ __global__ void __launch_bounds__(kMlpThreads, 1)
   const uint32_t stage_bytes = (HAS_Q ? 3u : 2u) * kTileBytesI;
 
   auto issue = [&](int s) {
+    if (s == a.stall_tile) return;
     const int slot = s % kStagesM;
     mbar_arrive_expect_tx(&sm.full[slot], stage_bytes);
     tma_load_3d(sm.K[slot], &tmK, &sm.full[slot], 0, s * kTileTokI, bh);
@@ -1070,7 +1074,8 @@ __global__ void __launch_bounds__(kMlpThreads, 1)
     if (HAS_Q) bulk_wait<0>();
     // Nothing may still be landing in shared memory when the CTA exits (after an abort the
     // tiles issued past the last one consumed).
-    for (int t = s; t < issued; ++t) mbar_wait(&sm.full[t % kStagesM], (t / kStagesM) & 1, a.status, nullptr);
+    for (int t = s; t < issued; ++t)
+      if (t != a.stall_tile) mbar_wait(&sm.full[t % kStagesM], (t / kStagesM) & 1, a.status, nullptr);
   }
 #pragma unroll
   for (int mt = 0; mt < 2; ++mt)
@@ -1103,8 +1108,14 @@ ttt_status launch_inner(ttt_state* st, const CUtensorMap* maps, float* loss, int
     st->lin.smem_set |= bit;
   }
   const int grid = c.batch * c.heads;
+  // Fault injection (tests): the second 64-token tile is never loaded, so the waits for it run out.
+  int stall_tile = -1;
+  if (st->inject_stall && T > kTileTokI) {
+    stall_tile = 1;
+    st->inject_stall = 0;
+  }
   InnerArgs a{st->lin.W, st->lin.W0, st->lin.ln_gamma, st->lin.ln_beta, loss, steps, T, c.heads, T / kMB,
-              c.eta, c.ln_eps, DevStatus{st->status.dev, st->wait_limit_ns, st->status.dev + 1}};
+              c.eta, c.ln_eps, DevStatus{st->status.dev, st->wait_limit_ns, st->status.dev + 1}, stall_tile};
   kernel<<<grid, mlp ? kMlpThreads : kLnThreads, smem, s>>>(maps[0], maps[1], maps[2], maps[3], a);
   st->launches++;
   TTT_CUDA(cudaGetLastError());

@@ -219,3 +219,43 @@ def test_token_weights_workload_full_size(cwl, model):
     eo, ew, el = rel_err(O, Oref), max(weight_errs(spec, W, Wref)), rel_err(L, Lref)
     print(f"{spec.name} per-token weights: O {eo:.3e}  W {ew:.3e}  loss {el:.3e}")
     assert eo <= TOL and ew <= TOL and el <= TOL
+
+
+@pytest.mark.parametrize("model", MODELS)
+def test_reset_rescan_and_weight_roundtrip(cwl, model):
+    """reset() returns every head to W0 (a rescan repeats the first scan bit for bit); get/set of
+    the weights resumes a scan exactly at a mini-batch boundary; T = 0 is a no-op."""
+    spec = spec_of(model, B=2, H=2, T=192, seed=2800)
+    x = workloads.inner_inputs(spec, device="cuda")
+    st = make_state(cwl, spec, x)
+    K, V, Q = x["K"], x["V"], x["Q"]
+
+    def call(a, e):
+        O = torch.empty_like(K[:, :, a:e])
+        L = torch.empty(K.shape[0], K.shape[1], e - a, device="cuda")
+        st.chunk_scan(K[:, :, a:e].contiguous(), V[:, :, a:e].contiguous(), Q[:, :, a:e].contiguous(), out=O,
+                      loss_out=L, T=e - a)
+        return O, L
+
+    O1, L1 = call(0, 192)
+    W1 = torch.empty_like(x["W0"])
+    st.get_weights(W1)
+    st.reset()
+    O2, L2 = call(0, 192)
+    assert torch.equal(O1, O2) and torch.equal(L1, L2)
+    st.reset()
+    call(0, 96)
+    Wmid = torch.empty_like(x["W0"])
+    st.get_weights(Wmid)
+    st.reset()
+    st.set_weights(Wmid)
+    O3, L3 = call(96, 192)
+    W3 = torch.empty_like(x["W0"])
+    st.get_weights(W3)
+    torch.cuda.synchronize()
+    assert torch.equal(O3, O1[:, :, 96:]) and torch.equal(L3, L1[:, :, 96:]) and torch.equal(W3, W1)
+    st.chunk_scan(K, V, Q, out=torch.empty_like(K), T=0)
+    W4 = torch.empty_like(x["W0"])
+    st.get_weights(W4)
+    torch.cuda.synchronize()
+    assert torch.equal(W4, W1)

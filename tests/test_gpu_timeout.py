@@ -116,3 +116,48 @@ def test_option_ranges(cwl):
         assert e.value.status == abi.TTT_ERR_INVALID_ARG
     st.set_option(abi.TTT_OPT_WAIT_LIMIT_NS, 2_000_000_000)
     st.set_option(abi.TTT_OPT_INJECT_STALL, 0)
+
+
+@pytest.mark.parametrize("model", ["linear_ln", "mlp"])
+def test_inner_model_scan_wait_runs_out(cwl, model):
+    """The LayerNorm TTT-Linear and TTT-MLP scans never get their second 64-token tile: their
+    waits give up, TTT_ERR_TIMEOUT is reported, and a reset state then scans like a fresh one
+    (bit for bit) and like the oracle."""
+    from chunked_weight_layers_b200 import abi
+    from oracle import inner as oinn
+    base = workloads.LINEAR_LN if model == "linear_ln" else workloads.MLP
+    spec = workloads.scaled(base, B=1, H=3, T=256, seed=406)
+    x = workloads.inner_inputs(spec, device="cuda")
+    cfg = cwl.config(model, batch=1, heads=3, eta=spec.eta, ln_eps=spec.eps)
+
+    def make():
+        st = cwl.FastWeightState(cfg, x["W0"])
+        st.set_layernorm(x["gamma"], x["beta"])
+        return st
+
+    def scan(st):
+        O = torch.empty_like(x["K"])
+        L = torch.empty((1, 3, spec.T), device="cuda")
+        st.chunk_scan(x["K"], x["V"], x["Q"], out=O, loss_out=L)
+        W = torch.empty_like(x["W0"])
+        st.get_weights(W)
+        return O, W, L
+
+    st = make()
+    st.set_option(abi.TTT_OPT_WAIT_LIMIT_NS, LIMIT_NS)
+    st.set_option(abi.TTT_OPT_INJECT_STALL, 1)
+    scan(st)
+    _expect_timeout(st)
+    st.reset()
+    O, W, L = scan(st)  # the injection was used up: this scan runs normally
+    st.poll()
+    O2, W2, L2 = scan(make())
+    torch.cuda.synchronize()
+    assert torch.equal(O, O2) and torch.equal(W, W2) and torch.equal(L, L2)
+    c = {k: v.cpu() for k, v in x.items() if isinstance(v, torch.Tensor)}
+    if model == "linear_ln":
+        Oref = oinn.ttt_linear_ln_scan(c["K"], c["V"], c["Q"], c["W0"], c["gamma"], c["beta"], spec.eta, 16, spec.eps)[0]
+    else:
+        Oref = oinn.ttt_mlp_scan(c["K"], c["V"], c["Q"], c["W1"], c["W2"], c["gamma"], c["beta"], spec.eta, 16,
+                                 spec.eps)[0]
+    assert rel_err(O, Oref) <= 2e-2
