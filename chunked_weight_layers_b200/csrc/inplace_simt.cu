@@ -20,14 +20,17 @@ namespace {
 constexpr int BM = 32, BN = 64, BK = 32, NT = 256;
 
 struct SgemmSmem {
-  float As[BK][BM + 4];
-  float Bs[BK][BN + 4];
+  float As[2][BK][BM + 4];
+  float Bs[2][BK][BN + 4];
 };
 
 // One tile of C[M,N] = A[M,K]·B[K,N] (UPDATE = false) or C = Cin + eta·A·B (UPDATE = true),
 // where A is stored K-contiguous (A_KC, as [M,K]) or M-contiguous (as [K,M]) and B is stored
 // K-contiguous (B_KC, as [N,K]) or N-contiguous (as [K,N]). Every output accumulates its
-// products in increasing k with fmaf, so results do not depend on the tiling.
+// products in increasing k with fmaf, so results do not depend on the tiling. The k slices go
+// through two shared-memory buffers: the global loads of slice s + 1 are issued into registers
+// before slice s is computed and stored to the other buffer after it, so their latency hides
+// behind the arithmetic and each slice takes one barrier.
 template <bool A_KC, bool B_KC, bool UPDATE>
 __device__ __forceinline__ void sgemm_tile(SgemmSmem& sm, const float* __restrict__ A, const float* __restrict__ B,
                                            const float* __restrict__ Cin, float* __restrict__ Cout, int M, int N,
@@ -35,44 +38,74 @@ __device__ __forceinline__ void sgemm_tile(SgemmSmem& sm, const float* __restric
   const int tid = threadIdx.x;
   const int tx = tid % 16, ty = tid / 16;
   float acc[2][4] = {};
-  for (int k0 = 0; k0 < K; k0 += BK) {
-    // Stage A as As[k][m] (32 x 32: four elements a thread).
+  float ra[4], rb[8];  // this thread's share of the next slice
+  // Slice k0 of A (32 x 32: four elements a thread) and B (32 x 64: eight) into registers.
+  auto fetch = [&](int k0) {
     if (A_KC) {
       const int r = tid / 8, kq = (tid % 8) * 4;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int m = m0 + r, k = k0 + kq + j;
-        sm.As[kq + j][r] = (m < M && k < K) ? A[(size_t)m * lda + k] : 0.f;
+        ra[j] = (m < M && k < K) ? A[(size_t)m * lda + k] : 0.f;
       }
     } else {
       const int kk = tid / 8, mq = (tid % 8) * 4;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int m = m0 + mq + j, k = k0 + kk;
-        sm.As[kk][mq + j] = (m < M && k < K) ? A[(size_t)k * lda + m] : 0.f;
+        ra[j] = (m < M && k < K) ? A[(size_t)k * lda + m] : 0.f;
       }
     }
-    // Stage B as Bs[k][n] (32 x 64: eight elements a thread).
     if (B_KC) {
       const int r = tid / 4, kq = (tid % 4) * 8;
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         const int n = n0 + r, k = k0 + kq + j;
-        sm.Bs[kq + j][r] = (n < N && k < K) ? B[(size_t)n * ldb + k] : 0.f;
+        rb[j] = (n < N && k < K) ? B[(size_t)n * ldb + k] : 0.f;
       }
     } else {
       const int kk = tid / 8, nq = (tid % 8) * 8;
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         const int n = n0 + nq + j, k = k0 + kk;
-        sm.Bs[kk][nq + j] = (n < N && k < K) ? B[(size_t)k * ldb + n] : 0.f;
+        rb[j] = (n < N && k < K) ? B[(size_t)k * ldb + n] : 0.f;
       }
     }
-    __syncthreads();
+  };
+  // The registers into buffer b as As[b][k][m] and Bs[b][k][n].
+  auto stash = [&](int b) {
+    if (A_KC) {
+      const int r = tid / 8, kq = (tid % 8) * 4;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) sm.As[b][kq + j][r] = ra[j];
+    } else {
+      const int kk = tid / 8, mq = (tid % 8) * 4;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) sm.As[b][kk][mq + j] = ra[j];
+    }
+    if (B_KC) {
+      const int r = tid / 4, kq = (tid % 4) * 8;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) sm.Bs[b][kq + j][r] = rb[j];
+    } else {
+      const int kk = tid / 8, nq = (tid % 8) * 8;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) sm.Bs[b][kk][nq + j] = rb[j];
+    }
+  };
+  fetch(0);
+  stash(0);
+  __syncthreads();
+  int buf = 0;
+  for (int k0 = 0; k0 < K; k0 += BK) {
+    const bool more = k0 + BK < K;
+    if (more) fetch(k0 + BK);
+    // The products of a slice stop at K (its zero-filled tail is not run).
     const int kend = min(BK, K - k0);
+#pragma unroll 8
     for (int k = 0; k < kend; ++k) {
-      const float2 a = *reinterpret_cast<const float2*>(&sm.As[k][ty * 2]);
-      const float4 b = *reinterpret_cast<const float4*>(&sm.Bs[k][tx * 4]);
+      const float2 a = *reinterpret_cast<const float2*>(&sm.As[buf][k][ty * 2]);
+      const float4 b = *reinterpret_cast<const float4*>(&sm.Bs[buf][k][tx * 4]);
       const float av[2] = {a.x, a.y};
       const float bv[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
@@ -80,7 +113,9 @@ __device__ __forceinline__ void sgemm_tile(SgemmSmem& sm, const float* __restric
 #pragma unroll
         for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
     }
-    __syncthreads();
+    if (more) stash(buf ^ 1);
+    __syncthreads();  // buffer buf ^ 1 is complete; buffer buf is free for slice k0 + 2·BK
+    buf ^= 1;
   }
 #pragma unroll
   for (int i = 0; i < 2; ++i) {
