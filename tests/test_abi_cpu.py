@@ -63,6 +63,8 @@ def test_host_argument_checks(lib):
     assert lib.ttt_state_create(None, None, None, None, None, None) == abi.TTT_ERR_INVALID_ARG
     assert lib.ttt_chunk_scan(None, None, None, None, 0, None, None, None) == abi.TTT_ERR_INVALID_ARG
     assert lib.ttt_surprisal_route(None, None, 0, None) == abi.TTT_ERR_INVALID_ARG
+    assert lib.ttt_chunk_scan_packed(None, None, None, None, 0, None, None, None, None, None) == abi.TTT_ERR_INVALID_ARG
+    assert lib.ttt_state_set_layernorm(None, None, None, None) == abi.TTT_ERR_INVALID_ARG
     assert lib.ttt_state_destroy(None) == abi.TTT_OK
     assert lib.ttt_state_launch_count(None) == 0
     assert lib.ttt_abi_version() == 2
