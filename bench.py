@@ -308,6 +308,32 @@ def traffic_per_launch(spec):
     return rec["bytes_per_launch"] * rec.get("launches_per_step", 1)
 
 
+def recorded_traffic(key, chunks=None):
+    """DRAM bytes per step of a further form's dominant kernel from the committed ncu record
+    ``key`` (kernel@line): per padded chunk times ``chunks`` when the record was captured on a
+    smaller case, else its bytes per launch times launches per step; None when there is no
+    record or the kernel's source changed since the capture."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(p):
+        return None
+    rec = json.load(open(p)).get(key)
+    if rec is None:
+        return None
+    src = os.path.join(ROOT, rec["source"])
+    if not os.path.exists(src) or not hashlib.sha256(open(src, "rb").read()).hexdigest().startswith(rec["sha256_prefix"]):
+        return None
+    if "bytes_per_chunk" in rec:
+        return None if chunks is None else rec["bytes_per_chunk"] * chunks
+    return rec["bytes_per_launch"] * rec.get("launches_per_step", 1)
+
+
+def padded_chunks(T, C, starts):
+    """Chunks of a packed layout with every document padded to whole chunks."""
+    ends = starts[1:] + [T]
+    return sum(-(-(e - a) // C) for a, e in zip(starts, ends))
+
+
 SUSTAINED_MS = 50.0  # a timed region at least this long runs in the power-capped regime
 
 
@@ -435,7 +461,9 @@ def measure(spec, steps, warmup, peaks, device, with_e2e, cpu_limit_s=None, pref
     rl = roofline(spec, w, ms, peaks, traffic_per_launch(spec), timed_ms=total)
     rl["kernel"] = "k_gemm_tc" if prefix else dominant_kernel(spec)
     if prefix:
-        rl["traffic"] = None  # no ncu capture of this form is recorded
+        # The two GEMM launches of a step, from a capture on fewer chunks (every chunk moves the
+        # same data).
+        rl["traffic"] = recorded_traffic(f"k_gemm_tc@{spec.name} (context-parallel form)", spec.T // spec.C)
     out = {"workload": spec.name + (" (context-parallel form)" if prefix else ""), "ms_per_step": ms, "ms_median": statistics.median(times),
            "tokens_per_s": w["tokens"] / (ms * 1e-3), "tflops": w["flops"] / (ms * 1e-3) / 1e12,
            "roofline": rl, "gpu_launches_per_step": launches / max(1, steps), "times_ms": times,
@@ -516,15 +544,35 @@ def measure_cache_read(steps, warmup, peaks, device):
     st.poll()
     ms = e0.elapsed_time(e1) / steps
     achieved = w["bytes"] / (ms * 1e-3) / 1e9
+    # End to end: the call's inputs (queries, keys, values, the scan's outputs, α) from pinned host
+    # memory, the call, its outputs back.
+    hin = [t.cpu().pin_memory() for t in (x["Q"], x["K"], x["V"], O, alpha)]
+    din = [torch.empty_like(t) for t in (x["Q"], x["K"], x["V"], O, alpha)]
+    hout = torch.empty(O.shape, dtype=O.dtype).pin_memory()
+    dout = torch.empty_like(O)
+    e2e = []
+    for _ in range(3):
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        for d, h in zip(din, hin):
+            d.copy_(h, non_blocking=True)
+        st.cache_attention(din[0], din[1], din[2], din[3], din[4], out=dout)
+        hout.copy_(dout, non_blocking=True)
+        torch.cuda.synchronize()
+        e2e.append((time.perf_counter() - t0) * 1e3)
+    e2e_ms = statistics.median(e2e)
     out = {"workload": CACHE_READ, "ms_per_step": ms, "tokens_per_s": w["tokens"] / (ms * 1e-3),
            "tflops": w["flops"] / (ms * 1e-3) / 1e12,
            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                        "frac": achieved / peaks["hbm_gbs"], "traffic": None, "peak_source": peaks["source"],
-                        "kernel": "k_cache_attn",
+                        "frac": achieved / peaks["hbm_gbs"], "traffic": recorded_traffic("k_cache_attn@" + CACHE_READ),
+                        "peak_source": peaks["source"], "kernel": "k_cache_attn",
                         "tensor_frac": w["flops"] / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"]},
            "gpu_launches_per_step": 1.0, "host_ms_per_step": host_ms,
            "l2": f"inputs larger than L2: {n_sets} copies of the call's queries and outputs taken in turn",
-           "e2e": None, "e2e_note": "the read path has no host-buffer entry point"}
+           "e2e": {"value": w["tokens"] / (e2e_ms * 1e-3), "unit": "tokens/s",
+                   "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in hin),
+                   "d2h_bytes_per_step": hout.numel() * hout.element_size(), "ms_per_step": e2e_ms,
+                   "note": "through ttt_cache_attention with its inputs copied from pinned host memory"}}
     st.close()
     torch.cuda.empty_cache()
     return out
@@ -581,8 +629,9 @@ def measure_docs(steps, warmup, peaks, device):
     out = {"workload": DOCS, "doc_starts": starts, "clip_norm": DOCS_CLIP, "ms_per_step": ms,
            "ms_median": statistics.median(times), "tokens_per_s": w["tokens"] / (ms * 1e-3), "tflops": tf,
            "roofline": {"bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                        "frac": tf / peaks["bf16_tflops"], "traffic": None, "peak_source": peaks["source"],
-                        "kernel": "k_gemm_tc",
+                        "frac": tf / peaks["bf16_tflops"],
+                        "traffic": recorded_traffic("k_gemm_tc@" + DOCS, padded_chunks(spec.T, spec.C, starts)),
+                        "peak_source": peaks["source"], "kernel": "k_gemm_tc",
                         "peak_kind": "burst (each call timed alone: it synchronises to upload its layout)"},
            "gpu_launches_per_step": launches, "times_ms": times,
            "l2": "inputs larger than L2 (the 4B-class Z alone is 637 MB)",
@@ -671,8 +720,8 @@ def measure_packed(steps, warmup, peaks, device):
     out = {"workload": PACKED, "doc_starts": starts, "ms_per_step": ms, "ms_median": statistics.median(times),
            "tokens_per_s": w["tokens"] / (ms * 1e-3), "tflops": w["flops"] / (ms * 1e-3) / 1e12,
            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                        "frac": achieved / peaks["hbm_gbs"], "traffic": None, "peak_source": peaks["source"],
-                        "kernel": "k_inner_ln (plain mode)"},
+                        "frac": achieved / peaks["hbm_gbs"], "traffic": recorded_traffic("k_inner_ln@" + PACKED),
+                        "peak_source": peaks["source"], "kernel": "k_inner_ln (plain mode)"},
            "gpu_launches_per_step": launches, "times_ms": times,
            "l2": "each call timed alone (it synchronises to upload its layout); its 100 MB of inputs are gathered into a padded copy",
            "e2e": {"value": w["tokens"] / (e2e_ms * 1e-3), "unit": "tokens/s",
@@ -816,6 +865,40 @@ def run_row_sharded(spec, a, world, rank, local, peaks):
         dist.destroy_process_group()
 
 
+def profile_form(form, spec, device, calls):
+    """``calls`` calls of a further form (for profilers): the packed In-Place scan on the In-Place
+    workload ``spec`` (its seeded document layout for spec.T tokens), the cache read path on the
+    gate workload's cache, or packed TTT-Linear on the TTT-Linear workload."""
+    import chunked_weight_layers_b200 as cwl
+    if form == "docs":
+        starts = wl.document_starts(spec.T, DOCS_N, DOCS_SEED)
+        x = wl.inplace_inputs(spec, device=device)
+        st = cwl.FastWeightState(cwl.config("inplace", io_dtype=1, d_key=spec.f, d_val=spec.d, chunk=spec.C,
+                                            eta=spec.eta), x["W0"])
+        O = torch.empty((spec.T, spec.d), device=device, dtype=torch.bfloat16)
+        for _ in range(calls):
+            st.chunk_scan_docs(x["Z"], x["Vhat"], starts, clip=DOCS_CLIP, out=O)
+        print(f"profiled {spec.name} packed: {calls} calls, {padded_chunks(spec.T, spec.C, starts)} padded chunks")
+    elif form == "cache_read":
+        spec_c, x, st, O, alpha = _cache_read_setup(device)
+        out = torch.empty_like(O)
+        for _ in range(calls):
+            st.cache_attention(x["Q"], x["K"], x["V"], O, alpha, out=out)
+        print(f"profiled {CACHE_READ}: {calls} calls")
+    else:
+        spec_p = wl.LINEAR_GD
+        starts = packed_starts(spec_p)
+        x = wl.linear_inputs(spec_p, device=device)
+        st = cwl.FastWeightState(cwl.config("linear", batch=spec_p.B, heads=spec_p.H, chunk=spec_p.b, eta=spec_p.eta),
+                                 x["W0"])
+        O = torch.empty_like(x["K"])
+        for _ in range(calls):
+            st.chunk_scan_packed(x["K"], x["V"], starts, queries=x["Q"], out=O)
+        print(f"profiled {PACKED}: {calls} calls")
+    torch.cuda.synchronize()
+    st.poll()
+
+
 def bench_config(spec, world) -> dict:
     """The workload description both arms report."""
     return {"workload": spec.name, "B": getattr(spec, "B", 1), "H": getattr(spec, "H", 1), "T": spec.T,
@@ -846,6 +929,9 @@ def main():
                     help="with N ranks: 'replicas' (default) runs an independent copy of the workload per rank "
                          "(weak scaling); 'rows' splits one In-Place layer's Wdown rows over the ranks and "
                          "all-gathers the output columns each step (strong scaling; In-Place workloads)")
+    ap.add_argument("--form", choices=["scan", "prefix", "docs", "cache_read", "packed"], default="scan",
+                    help="with --profile: the further form to run (the context-parallel In-Place scan, the packed "
+                         "In-Place scan or packed TTT-Linear on the named workload's inputs, the cache read path)")
     ap.add_argument("--profile", type=int, default=None, metavar="N",
                     help="for profilers: build the named workload, run one warm-up step and N more steps, print "
                          "nothing else (no timing, no end-to-end pass, no oracle)")
@@ -890,13 +976,17 @@ def main():
         torch.cuda.set_device(local)
         from chunked_weight_layers_b200 import build
         build.build()
-        runner = Runner(spec, torch.device("cuda", local))
-        runner.state.reset()
-        for k in range(1 + a.profile):
-            runner.step(k)
-        torch.cuda.synchronize()
-        runner.state.poll()
-        print(f"profiled {spec.name}: 1 + {a.profile} steps, {runner.state.launch_count()} library launches")
+        device = torch.device("cuda", local)
+        if a.form in ("scan", "prefix"):
+            runner = Runner(spec, device, prefix=a.form == "prefix")
+            runner.state.reset()
+            for k in range(1 + a.profile):
+                runner.step(k)
+            torch.cuda.synchronize()
+            runner.state.poll()
+            print(f"profiled {spec.name} ({a.form}): 1 + {a.profile} steps, {runner.state.launch_count()} library launches")
+            return
+        profile_form(a.form, spec, device, 1 + a.profile)
         return
 
     if a.warmup < 3:
