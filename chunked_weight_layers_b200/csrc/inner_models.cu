@@ -781,8 +781,10 @@ __global__ void __launch_bounds__(kMlpThreads, 1)
               mma_bf16(hk[mt][nt], whi[kk], kb[nt][2 * kk], kb[nt][2 * kk + 1]);
               mma_bf16(hk[mt][nt], wlo[kk], kb[nt][2 * kk], kb[nt][2 * kk + 1]);
               if (HAS_Q) {
+                // The queries' products feed only the outputs (no recurrence amplifies their
+                // rounding): the bf16 weights alone, except with TW, whose corrections follow.
                 mma_bf16(hq[mt][nt], whi[kk], qb[nt][2 * kk], qb[nt][2 * kk + 1]);
-                mma_bf16(hq[mt][nt], wlo[kk], qb[nt][2 * kk], qb[nt][2 * kk + 1]);
+                if (TW) mma_bf16(hq[mt][nt], wlo[kk], qb[nt][2 * kk], qb[nt][2 * kk + 1]);
               }
             }
         }
@@ -836,7 +838,7 @@ __global__ void __launch_bounds__(kMlpThreads, 1)
 #pragma unroll
               for (int ks = 0; ks < 2; ++ks) {
                 mma_bf16(zp, whi[ks], b[ks][0], b[ks][1]);
-                mma_bf16(zp, wlo[ks], b[ks][0], b[ks][1]);
+                if (kind == 0) mma_bf16(zp, wlo[ks], b[ks][0], b[ks][1]);  // queries: bf16 weights alone
               }
 #pragma unroll
               for (int e = 0; e < 4; ++e)
