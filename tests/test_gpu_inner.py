@@ -259,3 +259,13 @@ def test_reset_rescan_and_weight_roundtrip(cwl, model):
     st.get_weights(W4)
     torch.cuda.synchronize()
     assert torch.equal(W4, W1)
+
+
+@pytest.mark.parametrize("model", MODELS)
+def test_more_heads_than_sms(cwl, model):
+    """160 (sequence, head) pairs, one CTA each: more than the 148 SMs hold at once."""
+    spec = spec_of(model, B=10, H=16, T=48, seed=2900)
+    x = workloads.inner_inputs(spec, device="cuda")
+    O, W, L = run(cwl, spec, x)
+    Oref, Wref, Lref = oracle(spec, x)
+    assert rel_err(O, Oref) <= TOL and max(weight_errs(spec, W, Wref)) <= TOL and rel_err(L, Lref) <= TOL
