@@ -79,8 +79,9 @@ __global__ void __launch_bounds__(kThreadsCA) k_cache_attn(const __nv_bfloat16* 
                                                            const __nv_bfloat16* __restrict__ V,
                                                            const __nv_bfloat16* O_ttt, const float* __restrict__ alpha,
                                                            const int32_t* __restrict__ entries,
-                                                           const int32_t* __restrict__ counts, int T, int heads,
-                                                           int capacity, __nv_bfloat16* out) {
+                                                           const int32_t* __restrict__ counts,
+                                                           const int64_t* __restrict__ tokens, int T, int heads,
+                                                           int capacity, __nv_bfloat16* out, const DevStatus status) {
   extern __shared__ uint8_t smem_raw[];
   CacheAttnSmem& sm =
       *reinterpret_cast<CacheAttnSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -91,6 +92,10 @@ __global__ void __launch_bounds__(kThreadsCA) k_cache_attn(const __nv_bfloat16* 
   const size_t base = (size_t)bh * T * 64;
   const int32_t* E = entries + (size_t)bh * capacity * 3;
   const int n = min(counts[2 * bh], capacity);
+  // The cache holds positions of the tokens gated since the reset, which the caller's arrays
+  // must span exactly (positions past T are skipped below whatever the outcome).
+  if (blockIdx.x == 0 && threadIdx.x == 0 && tokens[bh] != (int64_t)T)
+    record_status(status, kDevInvalidArg, kSiteCacheLength | (bh & 0xFFFF));
 
   // Entries a block at token t0 sees: those of tokens before its gate chunk (a prefix of the
   // cache, which holds its tokens in increasing order).
@@ -285,8 +290,9 @@ ttt_status cache_attention(const ttt_state* st, const __nv_bfloat16* Q, const __
   TTT_CUDA(cudaFuncSetAttribute(k_cache_attn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   const int nblk = (int)((T + kQBlk - 1) / kQBlk);
   const dim3 grid((unsigned)((nblk + kQPerCta - 1) / kQPerCta), (unsigned)BH);
-  k_cache_attn<<<grid, kThreadsCA, smem, s>>>(Q, K, V, O_ttt, alpha, st->gate.entries, st->gate.counts, (int)T,
-                                             c.heads, c.cache_capacity, out);
+  k_cache_attn<<<grid, kThreadsCA, smem, s>>>(Q, K, V, O_ttt, alpha, st->gate.entries, st->gate.counts,
+                                             st->gate.tokens, (int)T, c.heads, c.cache_capacity, out,
+                                             DevStatus{st->status.dev, st->wait_limit_ns, st->status.dev + 1});
   TTT_CUDA(cudaGetLastError());
   return TTT_OK;
 }

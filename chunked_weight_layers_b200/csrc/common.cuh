@@ -9,6 +9,8 @@
 namespace ttt {
 
 // Status codes written by kernels (same values as ttt_status).
+constexpr int kDevInvalidArg = 1;
+constexpr int kDevUnsupported = 2;
 constexpr int kDevTimeout = 5;
 constexpr int kDevCheck = 6;
 
@@ -28,6 +30,11 @@ struct DevStatus {
 // counter in global memory (detail: the low bits of its word address).
 constexpr int kSiteMbarrier = 0x10000;
 constexpr int kSiteCounter = 0x20000;
+// Argument checks that only the device can make, because the count they compare against lives
+// on the device: the gate's token position would pass 2^31 − 1; the cache read's T is not the
+// number of tokens gated since the reset (detail: the (sequence, head) index, low 16 bits).
+constexpr int kSiteTokenLimit = 0x40000;
+constexpr int kSiteCacheLength = 0x50000;
 
 __device__ __forceinline__ void record_status(int* status, int code) {
   if (status != nullptr) atomicCAS(status, 0, code);

@@ -43,12 +43,14 @@ struct __align__(16) GateSmem {
   float tau_carry;
   int tau_set;
   int routed;
+  long long tokens;  // tokens gated since reset before this call
 };
 
 __global__ void __launch_bounds__(kGateThreads)
     k_gate(const float* __restrict__ loss, int T, int heads, int rank, float ema_old, float ema_new, double lhs_scale,
            double rhs_scale, float* __restrict__ tau_state, int32_t* __restrict__ tau_set_state,
-           int32_t* __restrict__ entries, int32_t* __restrict__ counts, int capacity, int64_t t_offset) {
+           int32_t* __restrict__ entries, int32_t* __restrict__ counts, int capacity, int64_t* __restrict__ tokens,
+           int* status) {
   __shared__ GateSmem sm;
   const int bh = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -57,8 +59,10 @@ __global__ void __launch_bounds__(kGateThreads)
     sm.tau_carry = tau_state[bh];
     sm.tau_set = tau_set_state[bh];
     sm.routed = counts[2 * bh + 0];
+    sm.tokens = tokens[bh];
   }
   __syncthreads();
+  const long long t_offset = sm.tokens;
 
   for (int b0 = 0; b0 < T; b0 += kBlockTok) {
     const int ntok = min(kBlockTok, T - b0);
@@ -141,6 +145,9 @@ __global__ void __launch_bounds__(kGateThreads)
     tau_set_state[bh] = sm.tau_set;
     counts[2 * bh + 0] = sm.routed;
     counts[2 * bh + 1] = sm.routed > capacity ? sm.routed - capacity : 0;
+    tokens[bh] = t_offset + T;
+    if (t_offset + T > 0x7FFFFFFFll)
+      record_status(DevStatus{status, 0, status + 1}, kDevUnsupported, kSiteTokenLimit | (bh & 0xFFFF));
   }
 }
 
@@ -163,7 +170,8 @@ ttt_status gate_route(ttt_state* st, const float* loss, int64_t T, cudaStream_t 
   const double rhs = (double)c.gate_mean_num * kChunk;
   k_gate<<<c.batch * c.heads, kGateThreads, 0, s>>>(loss, (int)T, c.heads, rank, c.gate_ema_old, c.gate_ema_new, lhs,
                                                     rhs, st->gate.tau, st->gate.tau_set, st->gate.entries,
-                                                    st->gate.counts, c.cache_capacity, st->gate.t_offset);
+                                                    st->gate.counts, c.cache_capacity, st->gate.tokens,
+                                                    st->status.dev);
   st->launches++;
   TTT_CUDA(cudaGetLastError());
   st->gate.t_offset += T;

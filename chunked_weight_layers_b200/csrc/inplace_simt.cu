@@ -3,8 +3,8 @@
 // weight from before the chunk, then W_{c+1} = W_c + η·V̂_cᵀ·Z_c (§2).
 //
 // Both steps are small GEMMs (0.13 GFLOP per chunk each), independent of each other within a
-// chunk: one launch per chunk runs the tiles of both (the update writes a second weight
-// buffer, swapped after the launch).
+// chunk: one launch per chunk runs the tiles of both (the update writes the other of two weight
+// buffers; the scan alternates between them and leaves the weight in the first).
 // Tensor cores are not used here: TF32 would miss the 1e-4 tolerance of this workload and
 // the exact-integer checks, and the work is far too small to be throughput-bound.
 #include "common.cuh"
@@ -152,17 +152,14 @@ __global__ void __launch_bounds__(NT) k_f32_chunk(const float* __restrict__ Z, c
 
 }  // namespace
 
-ttt_status inplace_f32_chunk(ttt_state* st, const float* Z, const float* Vhat, float* O, int C, cudaStream_t s) {
+ttt_status inplace_f32_chunk(ttt_state* st, const float* Z, const float* Vhat, const float* W, float* Wn, float* O,
+                             int C, cudaStream_t s) {
   const int d = st->cfg.d_val, f = st->cfg.d_key;
   const int apply_tn = (d + BN - 1) / BN;
   const int tiles = ((C + BM - 1) / BM) * apply_tn + ((d + BM - 1) / BM) * ((f + BN - 1) / BN);
-  k_f32_chunk<<<tiles, NT, 0, s>>>(Z, Vhat, st->ip.W, st->ip.Wf32_next, O, C, d, f, st->cfg.eta, apply_tn);
+  k_f32_chunk<<<tiles, NT, 0, s>>>(Z, Vhat, W, Wn, O, C, d, f, st->cfg.eta, apply_tn);
   st->launches++;
   TTT_CUDA(cudaGetLastError());
-  // The weight after this chunk is in the second buffer: swap the two.
-  float* w = st->ip.W;
-  st->ip.W = st->ip.Wf32_next;
-  st->ip.Wf32_next = w;
   return TTT_OK;
 }
 

@@ -98,6 +98,7 @@ struct __align__(1024) TCSmem {
   uint64_t dep_ok[kDepSlots], dep_free[kDepSlots];
   uint32_t tmem_base;
   int abort;
+  int cur0;         // the bf16 copy of W that round 0 applies with
   int eflag[2][2];  // per column half: a wait of sub-tile e ran out (index e & 1)
   int tflag[2][2];  // per column half: the accumulator wait of tile t ran out (index t & 1)
 };
@@ -126,7 +127,12 @@ struct TCArgs {
   // round r − 1's UPDATE tiles of its block, an UPDATE tile of round r for round r − 2's APPLY
   // tiles of its block. Null counters: one round, no waits.
   int rounds;
+  // The bf16 copy round 0 applies with: ring[0] when ring is set, else cur0. With ring set the
+  // last CTA to finish adds `advance` to ring[0] (mod 3) once every CTA has read it, counting
+  // finished CTAs in ring[1] (left at 0 again), so no index lives on the host between calls.
   int cur0;
+  int* ring;
+  int advance;
   int nbd;
   int* upd_done;
   int* app_done;
@@ -407,6 +413,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       mbar_init(&sm.dep_free[i], 1);
     }
     sm.abort = 0;
+    sm.cur0 = args.ring != nullptr ? __ldcg(args.ring) : args.cur0;
     sm.eflag[0][0] = sm.eflag[0][1] = sm.eflag[1][0] = sm.eflag[1][1] = 0;
     sm.tflag[0][0] = sm.tflag[0][1] = sm.tflag[1][0] = sm.tflag[1][1] = 0;
     fence_barrier_init();
@@ -434,7 +441,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         const int chunk = args.chunk + rnd;
         const int r0 = row0_of(m);
         const int b0 = n * BN + rank * (BN / 2);  // first B column (N) this CTA loads
-        const CUtensorMap* wk = pick3(tmWk0, tmWk1, tmWk2, (args.cur0 + rnd) % 3);
+        const CUtensorMap* wk = pick3(tmWk0, tmWk1, tmWk2, (sm.cur0 + rnd) % 3);
         if (args.upd_done != nullptr) {
           // The dependency warp has seen this tile's inputs published by other CTAs.
           const int slot = (int)(dep_u % kDepSlots);
@@ -625,7 +632,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     for_tiles([&](int rnd, int32_t tc) -> bool {
       const int type = tile_type(tc), m = tile_m(tc), n = tile_n(tc);
       const int r0 = row0_of(m);
-      const CUtensorMap* ws = pick3(tmWs0, tmWs1, tmWs2, (args.cur0 + rnd + 1) % 3);
+      const CUtensorMap* ws = pick3(tmWs0, tmWs1, tmWs2, (sm.cur0 + rnd + 1) % 3);
       const int acc = tcount & 1;
       bool ok = mbar_wait(&sm.tfull[acc], (tcount >> 1) & 1, args.status, nullptr);
       ok = __all_sync(0xffffffffu, ok);
@@ -755,6 +762,14 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   if constexpr (PAIR) cluster_sync();
   tc_fence_after();
   if (warp == 1) tmem_dealloc<PAIR>(tmem, kTmemCols);
+  if (args.ring != nullptr && threadIdx.x == 0) {
+    // This CTA read ring[0] before its first barrier.
+    __threadfence();
+    if (atomicAdd(args.ring + 1, 1) == (int)gridDim.x - 1) {
+      args.ring[0] = (sm.cur0 + args.advance) % 3;
+      args.ring[1] = 0;
+    }
+  }
 }
 
 // Depthwise future-tap convolution of X0 for the fused target:
@@ -1055,7 +1070,9 @@ ttt_status inplace_bf16_scan(ttt_state* st, const __nv_bfloat16* Z, const __nv_b
     }
     a.rotate = list_rotation(r->lists[plan]);
     a.rounds = rounds;
-    a.cur0 = st->ip.cur;
+    a.cur0 = 0;
+    a.ring = st->ip.ring;
+    a.advance = plan == 1 ? 0 : rounds;  // plan 1 holds TARGET tiles alone
     a.nbd = (d + BN - 1) / BN;
     a.upd_done = counters;
     a.app_done = counters ? counters + (size_t)rounds * a.nbd : nullptr;
@@ -1084,7 +1101,6 @@ ttt_status inplace_bf16_scan(ttt_state* st, const __nv_bfloat16* Z, const __nv_b
                       &tmWs[0], &tmWs[1], &tmWs[2], &a};
     TTT_TRY(launch_tc(r->pair, r->grid[0], true, params, s));
     st->launches++;
-    st->ip.cur = (st->ip.cur + nchunks) % 3;
     return TTT_OK;
   };
   const int nbd = (d + BN - 1) / BN;
@@ -1125,7 +1141,6 @@ ttt_status inplace_bf16_scan(ttt_state* st, const __nv_bfloat16* Z, const __nv_b
     const bool last = ch + 1 == nchunks;
     const int plan = last ? 2 : 0;
     TTT_TRY(launch(plan, args_for(plan, ch, ch + 1, 1, nullptr), tmVm_buf[ch % 3]));
-    st->ip.cur = (st->ip.cur + 1) % 3;  // the bf16 copy written by this launch holds W_{c+1}
   }
   return TTT_OK;
 }
@@ -1183,6 +1198,8 @@ ttt_status target_values_into(const __nv_bfloat16* X0, const float* convw, const
   a.stall_round = -1;
   a.rounds = 1;
   a.cur0 = 0;
+  a.ring = nullptr;
+  a.advance = 0;
   a.nbd = 0;
   a.upd_done = nullptr;
   a.app_done = nullptr;

@@ -47,7 +47,10 @@ struct InplaceBuffers {
   // writes the next; three so that an update never overwrites the copy that the chunk
   // before is still applying with when chunks overlap in one launch.
   __nv_bfloat16* Wsh[3] = {nullptr, nullptr, nullptr};
-  int cur = 0;                   // index of the bf16 copy that holds the current W
+  // Device words {index of the bf16 copy that holds the current W, CTAs of the running scan
+  // launch that have finished}: the scan kernel reads the index and its last CTA advances it,
+  // so the host holds no per-call state and a captured call replays correctly.
+  int* ring = nullptr;
   __nv_bfloat16* Wtarget = nullptr;  // [d, d]
   float* convw = nullptr;        // [d, taps]
   // Targets of a chunk [C, d] (fused target): chunk c's are produced while chunk c − 1 runs and
@@ -114,7 +117,11 @@ struct GateBuffers {
   int32_t* tau_set = nullptr; // [B, H]
   int32_t* entries = nullptr; // [B, H, cap, 3]
   int32_t* counts = nullptr;  // [B, H, 2]
-  int64_t t_offset = 0;       // tokens gated since the last reset (host-side counter)
+  // Tokens gated since the last reset, per (sequence, head) on the device: the gating kernels
+  // read it and advance it. t_offset counts the same through the calls made on the host; it
+  // only gives early errors, since it misses the replays of a captured call.
+  int64_t* tokens = nullptr;  // [B, H]
+  int64_t t_offset = 0;
 };
 
 struct HostStaging {
@@ -148,8 +155,8 @@ size_t io_size(int dtype);
 // ---- kernel launchers (each returns TTT_OK or TTT_ERR_CUDA after the launch) ----------
 
 // In-Place, fp32 SIMT: one chunk of the scan (apply with W, then W += η·V̂ᵀZ).
-ttt_status inplace_f32_chunk(ttt_state* st, const float* Z, const float* Vhat, float* O, int C,
-                             cudaStream_t s);
+ttt_status inplace_f32_chunk(ttt_state* st, const float* Z, const float* Vhat, const float* W, float* Wn, float* O,
+                             int C, cudaStream_t s);
 
 // In-Place, bf16 tensor cores: the whole scan over T tokens.
 ttt_status inplace_bf16_scan(ttt_state* st, const __nv_bfloat16* Z, const __nv_bfloat16* targets,

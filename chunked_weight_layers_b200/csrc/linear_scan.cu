@@ -516,6 +516,7 @@ struct __align__(1024) B16Smem {
   int g_tau_set;
   int g_routed;
   int gate_turn;
+  long long g_tokens;  // tokens gated since reset before this call
 };
 
 // The surprisal gate's state and constants for the scan that runs it in its own warps.
@@ -527,7 +528,7 @@ struct GateArgs {
   int capacity, rank, heads;
   float ema_old, ema_new;
   double lhs, rhs;    // pass ⇔ lhs·S ≥ rhs·τ
-  int64_t t_offset;   // tokens gated since reset before this call
+  int64_t* tokens;    // [B·H] tokens gated since reset, advanced by this call's T
 };
 
 // Warp-uniform bounded wait: false (with abort set) if the phase did not complete in time.
@@ -699,6 +700,7 @@ __global__ void __launch_bounds__(b16_threads<true>(), 1)
       sm.g_tau = ga.tau[bh];
       sm.g_tau_set = ga.tau_set[bh];
       sm.g_routed = ga.counts[2 * bh];
+      sm.g_tokens = ga.tokens[bh];
     }
     __syncwarp();
     for (int t = w; t < ntiles; t += kGateWarps) {
@@ -715,13 +717,14 @@ __global__ void __launch_bounds__(b16_threads<true>(), 1)
       float tau = *reinterpret_cast<volatile float*>(&sm.g_tau);
       const bool set = *reinterpret_cast<volatile int*>(&sm.g_tau_set) != 0;
       const int routed = *reinterpret_cast<volatile int*>(&sm.g_routed);
+      const long long tok0 = *reinterpret_cast<volatile long long*>(&sm.g_tokens);
       tau = tau_next(tau, set, p, ga.ema_old, ga.ema_new);
       const bool pass = ga.lhs * S >= ga.rhs * (double)tau;
       const bool f0 = pass && v0 > tau, f1 = pass && v1 > tau;
       const unsigned m0 = __ballot_sync(0xffffffffu, f0), m1 = __ballot_sync(0xffffffffu, f1);
       const unsigned below = (1u << lane) - 1u;
       const int pos0 = routed + __popc(m0 & below), pos1 = routed + __popc(m0) + __popc(m1 & below);
-      const int tok = (int)(ga.t_offset + (int64_t)t * kTileTok) + lane;
+      const int tok = (int)(tok0 + (long long)t * kTileTok) + lane;
       if (f0 && pos0 < ga.capacity) {
         E[3 * pos0 + 0] = seq;
         E[3 * pos0 + 1] = head;
@@ -750,6 +753,9 @@ __global__ void __launch_bounds__(b16_threads<true>(), 1)
       ga.tau_set[bh] = sm.g_tau_set;
       ga.counts[2 * bh + 0] = routed;
       ga.counts[2 * bh + 1] = routed > ga.capacity ? routed - ga.capacity : 0;
+      const long long tokens = sm.g_tokens + (long long)ntiles * kTileTok;
+      ga.tokens[bh] = tokens;
+      if (tokens > 0x7FFFFFFFll) record_status(status, kDevUnsupported, kSiteTokenLimit | (bh & 0xFFFF));
     }
     return;
   }
@@ -1209,7 +1215,7 @@ ttt_status launch_b16(ttt_state* st, const CUtensorMap& tk, const CUtensorMap& t
   if (c.gate_enable) {
     ga = GateArgs{st->gate.tau, st->gate.tau_set, st->gate.entries, st->gate.counts, c.cache_capacity,
                   gate_rank(c), c.heads, c.gate_ema_old, c.gate_ema_new, (double)c.gate_mean_den,
-                  (double)c.gate_mean_num * kTileTok, st->gate.t_offset};
+                  (double)c.gate_mean_num * kTileTok, st->gate.tokens};
     const ttt_status r = has_q ? launch_b16_impl<true, true, true>(st, tk, tv, tq, to, loss, T, ga, s)
                                : launch_b16_impl<false, true, true>(st, tk, tv, tq, to, loss, T, ga, s);
     if (r != TTT_OK) return r;

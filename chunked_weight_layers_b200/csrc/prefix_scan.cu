@@ -189,11 +189,18 @@ __global__ void __launch_bounds__(kGThreads, 1)
 // its bf16 copy. Four consecutive elements a thread; the sum over the chunks runs in chunk
 // order. Packed sequences: where reset[j] is set the sum restarts from Wreset (a document's
 // first chunk), and with sumsq given s_i = clip / ‖D_i‖_F when that norm exceeds clip (else
-// 1, as without sumsq: the plain form's sums are bit for bit those of W + D).
+// 1, as without sumsq: the plain form's sums are bit for bit those of W + D). The final bf16
+// copy goes to the state's current copy, whose index the device holds (ring[0]).
+struct BfCopies {
+  __nv_bfloat16* w[3];
+  const int* ring;
+};
+
 __global__ void k_prefix_w(const float* W0, const float* __restrict__ D, __nv_bfloat16* __restrict__ Wb, float* Wout,
-                           __nv_bfloat16* __restrict__ Wcopy, long long nelem, int n, const int32_t* __restrict__ reset,
+                           const BfCopies copies, long long nelem, int n, const int32_t* __restrict__ reset,
                            const float* __restrict__ Wreset, const double* __restrict__ sumsq, float clip) {
   const long long n4 = nelem / 4;
+  __nv_bfloat16* Wcopy = copies.w[*copies.ring];
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (long long)gridDim.x * blockDim.x) {
     float4 acc = reinterpret_cast<const float4*>(W0)[i];
     for (int j = 0; j < n; ++j) {
@@ -320,8 +327,9 @@ ttt_status inplace_bf16_scan_prefix(ttt_state* st, const __nv_bfloat16* Z, const
   // 2. Exclusive prefix sums: the weight each chunk applies with, and the final weight.
   const long long n4 = (long long)(nelem / 4);
   const int blocks = (int)std::min<long long>((n4 + 255) / 256, (long long)st->num_sms * 8);
-  k_prefix_w<<<blocks, 256, 0, s>>>(ip.W, ip.prefix_D, ip.prefix_Wb, ip.W, ip.Wsh[ip.cur], (long long)nelem, n,
-                                    nullptr, nullptr, nullptr, 0.f);
+  k_prefix_w<<<blocks, 256, 0, s>>>(ip.W, ip.prefix_D, ip.prefix_Wb, ip.W,
+                                    BfCopies{{ip.Wsh[0], ip.Wsh[1], ip.Wsh[2]}, ip.ring}, (long long)nelem, n, nullptr,
+                                    nullptr, nullptr, 0.f);
   st->launches++;
   TTT_CUDA(cudaGetLastError());
 
@@ -419,7 +427,8 @@ ttt_status inplace_bf16_scan_docs(ttt_state* st, const __nv_bfloat16* Z, const _
   }
   const long long n4 = (long long)(nelem / 4);
   const int blocks = (int)std::min<long long>((n4 + 255) / 256, (long long)st->num_sms * 8);
-  k_prefix_w<<<blocks, 256, 0, s>>>(ip.W0, ip.prefix_D, ip.prefix_Wb, ip.W, ip.Wsh[ip.cur], (long long)nelem, n,
+  k_prefix_w<<<blocks, 256, 0, s>>>(ip.W0, ip.prefix_D, ip.prefix_Wb, ip.W,
+                                    BfCopies{{ip.Wsh[0], ip.Wsh[1], ip.Wsh[2]}, ip.ring}, (long long)nelem, n,
                                     ip.docs_reset, ip.W0, clip > 0.f ? ip.docs_sumsq : nullptr, clip);
   st->launches++;
   TTT_CUDA(cudaGetLastError());

@@ -5,6 +5,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include "common.cuh"
 #include "internal.h"
 
 namespace ttt {
@@ -134,6 +135,7 @@ static void free_state(ttt_state* st) {
   dev_free(st->ip.Wsh[0]);
   dev_free(st->ip.Wsh[1]);
   dev_free(st->ip.Wsh[2]);
+  dev_free(st->ip.ring);
   dev_free(st->ip.Wtarget);
   dev_free(st->ip.convw);
   free_tc(st);
@@ -149,6 +151,7 @@ static void free_state(ttt_state* st) {
   dev_free(st->gate.tau_set);
   dev_free(st->gate.entries);
   dev_free(st->gate.counts);
+  dev_free(st->gate.tokens);
   for (int i = 0; i < 5; ++i) dev_free(st->staging.buf[i]);
   if (st->status.host != nullptr) cudaFreeHost(st->status.host);
   delete st;
@@ -160,6 +163,7 @@ static ttt_status gate_reset(ttt_state* st, cudaStream_t s) {
   TTT_CUDA(cudaMemsetAsync(st->gate.tau, 0, bh * sizeof(float), s));
   TTT_CUDA(cudaMemsetAsync(st->gate.tau_set, 0, bh * sizeof(int32_t), s));
   TTT_CUDA(cudaMemsetAsync(st->gate.counts, 0, bh * 2 * sizeof(int32_t), s));
+  TTT_CUDA(cudaMemsetAsync(st->gate.tokens, 0, bh * sizeof(int64_t), s));
   TTT_TRY(fill_i32(st->gate.entries, -1, bh * (size_t)c.cache_capacity * 3, s, st));
   st->gate.t_offset = 0;
   return TTT_OK;
@@ -170,7 +174,7 @@ static ttt_status load_weights(ttt_state* st, const float* W, cudaStream_t s) {
   if (st->cfg.rule == TTT_RULE_INPLACE_HEBBIAN) {
     TTT_CUDA(cudaMemcpyAsync(st->ip.W, W, n * sizeof(float), cudaMemcpyDeviceToDevice, s));
     if (st->cfg.io_dtype == TTT_BF16) {
-      st->ip.cur = 0;
+      TTT_CUDA(cudaMemsetAsync(st->ip.ring, 0, 2 * sizeof(int), s));
       TTT_TRY(f32_to_bf16(st->ip.W, st->ip.Wsh[0], n, s, st));
     }
   } else {
@@ -221,7 +225,8 @@ static ttt_status create_impl(const ttt_config* cfg, const void* W0, const void*
     if (r == TTT_OK && c.io_dtype == TTT_BF16) {
       guard(dev_alloc((void**)&st->ip.Wsh[0], nW * 2, "W bf16 copy")) &&
           guard(dev_alloc((void**)&st->ip.Wsh[1], nW * 2, "W bf16 copy")) &&
-          guard(dev_alloc((void**)&st->ip.Wsh[2], nW * 2, "W bf16 copy"));
+          guard(dev_alloc((void**)&st->ip.Wsh[2], nW * 2, "W bf16 copy")) &&
+          guard(dev_alloc((void**)&st->ip.ring, 2 * sizeof(int), "bf16 copy index"));
     }
     if (r == TTT_OK && target) {
       const size_t dd = (size_t)c.d_val * c.d_val;
@@ -244,7 +249,8 @@ static ttt_status create_impl(const ttt_config* cfg, const void* W0, const void*
       guard(dev_alloc((void**)&st->gate.tau, bh * 4, "tau")) &&
           guard(dev_alloc((void**)&st->gate.tau_set, bh * 4, "tau_set")) &&
           guard(dev_alloc((void**)&st->gate.entries, bh * (size_t)cap * 3 * 4, "cache")) &&
-          guard(dev_alloc((void**)&st->gate.counts, bh * 2 * 4, "cache counts"));
+          guard(dev_alloc((void**)&st->gate.counts, bh * 2 * 4, "cache counts")) &&
+          guard(dev_alloc((void**)&st->gate.tokens, bh * sizeof(int64_t), "token positions"));
     }
   }
   if (r != TTT_OK) {
@@ -313,8 +319,15 @@ static ttt_status scan_impl(ttt_state* st, const void* keys, const void* targets
       const float* Z = static_cast<const float*>(keys);
       const float* V = static_cast<const float*>(targets);
       float* O = static_cast<float*>(out);
-      for (int64_t t0 = 0; t0 < T; t0 += c.chunk)
-        TTT_TRY(inplace_f32_chunk(st, Z + t0 * c.d_key, V + t0 * c.d_val, O + t0 * c.d_val, c.chunk, s));
+      // Chunk j reads buffer j mod 2 and writes the other; after an odd number of chunks the
+      // weight goes back to ip.W, so that every call starts and ends with it there.
+      float* buf[2] = {st->ip.W, st->ip.Wf32_next};
+      int64_t j = 0;
+      for (int64_t t0 = 0; t0 < T; t0 += c.chunk, ++j)
+        TTT_TRY(inplace_f32_chunk(st, Z + t0 * c.d_key, V + t0 * c.d_val, buf[j & 1], buf[(j + 1) & 1],
+                                  O + t0 * c.d_val, c.chunk, s));
+      if (j & 1)
+        TTT_CUDA(cudaMemcpyAsync(st->ip.W, st->ip.Wf32_next, weight_elems(c) * sizeof(float), cudaMemcpyDeviceToDevice, s));
       return TTT_OK;
     }
     if (st->ip.prefix_form)
@@ -512,8 +525,11 @@ ttt_status ttt_cache_attention(const ttt_state* st, const void* queries, const v
   if (st == nullptr) return fail(TTT_ERR_INVALID_ARG, "state is NULL");
   if (st->cfg.rule != TTT_RULE_LINEAR_GD || !st->cfg.gate_enable)
     return fail(TTT_ERR_UNSUPPORTED, "the cache read path needs a TTT-Linear state with the gate enabled");
-  if (T <= 0 || T != st->gate.t_offset)
-    return fail(TTT_ERR_INVALID_ARG, "T=%lld must equal the tokens scanned since the last reset (%lld)",
+  // T must equal the tokens gated since the reset. That count lives on the device (the kernel
+  // checks it and reports a mismatch through ttt_state_poll); the host's count misses replays of
+  // captured calls, so it can only show that T is too small.
+  if (T <= 0 || T < st->gate.t_offset)
+    return fail(TTT_ERR_INVALID_ARG, "T=%lld must equal the tokens scanned since the last reset (at least %lld)",
                 (long long)T, (long long)st->gate.t_offset);
   const void* p[6] = {queries, keys, values, o_ttt, alpha, out};
   for (const void* x : p)
@@ -595,8 +611,14 @@ ttt_status ttt_state_poll(ttt_state* st) {
   if (v == 0) return TTT_OK;
   if (v == TTT_ERR_TIMEOUT)
     return fail(TTT_ERR_TIMEOUT, "a bounded device-side wait ran out (%s 0x%x)",
-                (site & 0x30000) == 0x20000 ? "progress counter at word" : "mbarrier at shared offset",
+                (site & 0xF0000) == kSiteCounter ? "progress counter at word" : "mbarrier at shared offset",
                 site & 0xFFFF);
+  if ((site & 0xF0000) == kSiteTokenLimit)
+    return fail(TTT_ERR_UNSUPPORTED, "the gate's token position passed 2^31 - 1 (sequence-head %d; reset the state)",
+                site & 0xFFFF);
+  if ((site & 0xF0000) == kSiteCacheLength)
+    return fail(TTT_ERR_INVALID_ARG, "the cache read's T is not the number of tokens gated since the last reset "
+                "(sequence-head %d)", site & 0xFFFF);
   return fail(TTT_ERR_DEVICE, "a device-side check failed (code %d)", v);
 }
 

@@ -48,14 +48,21 @@
  *    grow a state-owned scratch buffer (longer T than before, or the first host call) may,
  *    through cudaMalloc, cudaFree and cudaMemcpy. Steady-state scans of unchanged sizes
  *    enqueue only.
+ *  - Everything a call reads and advances from one call to the next (the weights, the index
+ *    of the In-Place bf16 weight copy in use, the gate's threshold, cache and token position)
+ *    lives in device memory, and the fp32 In-Place weight ends every call in the same buffer.
+ *    So a steady-state scan (ttt_chunk_scan, ttt_surprisal_route, ttt_cache_attention,
+ *    ttt_state_reset) can be captured into a CUDA graph once and replayed any number of
+ *    times, each replay continuing the state where the last left it, with the caller copying
+ *    each segment's inputs into the captured buffers before the replay.
  *  - A call returns TTT_OK or an error status and never aborts the process. The message
  *    of the last error on the calling thread is returned by ttt_last_error_string().
  *  - Every call that takes a state must be made with the state's device current
  *    (else INVALID_ARG). Calls on one state must not run concurrently from several host
  *    threads; different states are independent.
  *  - Failures detected on the device (a bounded wait that ran out, a failed device-side
- *    check) are recorded in the state's status word and returned by the next call of
- *    ttt_state_poll().
+ *    check, an argument check against a count that only the device holds) are recorded in
+ *    the state's status word and returned by the next call of ttt_state_poll().
  */
 #ifndef TTT_H_
 #define TTT_H_
@@ -220,7 +227,8 @@ ttt_status ttt_chunk_scan_packed(ttt_state* st, const void* keys, const void* ta
  * advancing the state's τ, cache and token position exactly as a gated scan would.
  * TTT-Linear states only; T must be a multiple of gate_chunk. The token position (stored
  * in the cache as int32) may not pass 2^31 − 1 between resets: a gated call that would take
- * it there (this one or ttt_chunk_scan with the gate on) returns UNSUPPORTED. Defined by
+ * it there (this one or ttt_chunk_scan with the gate on) returns UNSUPPORTED, or, when only
+ * the device's count shows it (replays of a captured call), the next ttt_state_poll does. Defined by
  * "SR-TTT: Surprisal-Aware Residual Test-Time Training", §2.1 (the loss gate's two
  * conditions and the residual cache). */
 ttt_status ttt_surprisal_route(ttt_state* st, const float* loss, int64_t T, ttt_stream stream);
@@ -274,8 +282,10 @@ ttt_status ttt_gate_read(const ttt_state* st, float* tau, int32_t* tau_set, ttt_
  * values of an entry are the scanned K and V rows of its token. A query that sees no entry adds
  * nothing (out = o_ttt).
  *   queries, keys, values, o_ttt  device bf16 [batch, heads, T, 64]: the Q, K and V of all T
- *            tokens scanned since the last reset (T must equal that count) and the scan's
- *            outputs.
+ *            tokens scanned since the last reset (T must equal that count: a T below the
+ *            count of the calls made on the host returns INVALID_ARG; any other mismatch is
+ *            found by the kernel, which holds the count, and the next ttt_state_poll returns
+ *            INVALID_ARG) and the scan's outputs.
  *   alpha    device fp32 [heads, 64].
  *   out      device bf16 [batch, heads, T, 64]; may be o_ttt itself (updated in place).
  * TTT-Linear states with the gate, cache_capacity ≤ 256. The cache is read as the gate left it
@@ -362,9 +372,12 @@ typedef enum {
 ttt_status ttt_state_set_option(ttt_state* st, int32_t option, int64_t value);
 
 /* Synchronise the device and return the first device-side failure recorded since the
- * last poll (TTT_ERR_TIMEOUT or TTT_ERR_DEVICE), or TTT_OK; clears the record. For a timeout,
- * ttt_last_error_string() names the wait that ran out: an mbarrier (by its shared-memory
- * offset in the kernel's layout) or a progress counter (by the low bits of its address). */
+ * last poll, or TTT_OK; clears the record. TTT_ERR_TIMEOUT: a bounded wait ran out, and
+ * ttt_last_error_string() names it: an mbarrier (by its shared-memory offset in the
+ * kernel's layout) or a progress counter (by the low bits of its address). INVALID_ARG: the
+ * T given to ttt_cache_attention was not the count of tokens gated since the reset.
+ * UNSUPPORTED: the gate's token position passed 2^31 − 1. TTT_ERR_DEVICE: another
+ * device-side check failed. The message names the (sequence, head) of the last two. */
 ttt_status ttt_state_poll(ttt_state* st);
 
 /* Number of kernels this state has launched since creation. */

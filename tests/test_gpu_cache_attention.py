@@ -124,6 +124,15 @@ def test_read_path_rejects_bad_arguments(cwl):
         st.cache_attention(x["Q"][:, :, :128].contiguous(), x["K"][:, :, :128].contiguous(),
                            x["V"][:, :, :128].contiguous(), O[:, :, :128].contiguous(), alpha, T=128)
     assert e.value.status == abi.TTT_ERR_INVALID_ARG
+    # A T beyond the tokens gated is caught on the device, which holds the count (the host's
+    # misses replays of captured calls): the call returns and ttt_state_poll reports it once.
+    two = {k: torch.cat([x[k], x[k]], dim=2).contiguous() for k in ("Q", "K", "V")}
+    O2 = torch.cat([O, O], dim=2).contiguous()
+    st.cache_attention(two["Q"], two["K"], two["V"], O2, alpha, out=torch.empty_like(O2), T=2 * spec.T)
+    with pytest.raises(TTTError) as e:
+        st.poll()
+    assert e.value.status == abi.TTT_ERR_INVALID_ARG
+    st.poll()
     W0 = torch.eye(64, device="cuda").expand(1, 2, 64, 64).contiguous()
     no_gate = cwl.FastWeightState(cwl.config("linear", batch=1, heads=2, chunk=16), W0)
     with pytest.raises(TTTError) as e:
