@@ -124,9 +124,18 @@ struct GateBuffers {
   int64_t t_offset = 0;
 };
 
+// ttt_chunk_scan_host: two sets of device buffers for one segment of tokens (keys, targets,
+// queries, out, loss), so that a segment's copies in and out overlap the scan of its
+// neighbours, and the copy streams and events of that pipeline (created on first use).
 struct HostStaging {
-  void* buf[5] = {nullptr, nullptr, nullptr, nullptr, nullptr};
-  size_t bytes[5] = {0, 0, 0, 0, 0};
+  void* buf[2][5] = {};
+  size_t bytes[2][5] = {};
+  cudaStream_t copy_in = nullptr;
+  cudaStream_t copy_out = nullptr;
+  cudaEvent_t entry = nullptr;
+  cudaEvent_t in_done[2] = {nullptr, nullptr};    // a set's inputs are on the device
+  cudaEvent_t scan_done[2] = {nullptr, nullptr};  // a set's scan ended: inputs free, outputs ready
+  cudaEvent_t out_done[2] = {nullptr, nullptr};   // a set's outputs are back in host memory
 };
 
 }  // namespace ttt

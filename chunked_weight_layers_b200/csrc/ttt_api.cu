@@ -5,6 +5,8 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <numeric>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -152,7 +154,15 @@ static void free_state(ttt_state* st) {
   dev_free(st->gate.entries);
   dev_free(st->gate.counts);
   dev_free(st->gate.tokens);
-  for (int i = 0; i < 5; ++i) dev_free(st->staging.buf[i]);
+  HostStaging& hs = st->staging;
+  for (int j = 0; j < 2; ++j)
+    for (int i = 0; i < 5; ++i) dev_free(hs.buf[j][i]);
+  cudaEvent_t* evs[] = {&hs.entry, &hs.in_done[0], &hs.in_done[1], &hs.scan_done[0], &hs.scan_done[1],
+                        &hs.out_done[0], &hs.out_done[1]};
+  for (cudaEvent_t* e : evs)
+    if (*e != nullptr) cudaEventDestroy(*e);
+  if (hs.copy_in != nullptr) cudaStreamDestroy(hs.copy_in);
+  if (hs.copy_out != nullptr) cudaStreamDestroy(hs.copy_out);
   if (st->status.host != nullptr) cudaFreeHost(st->status.host);
   delete st;
 }
@@ -358,13 +368,63 @@ static ttt_status scan_impl(ttt_state* st, const void* keys, const void* targets
   return TTT_OK;
 }
 
-static ttt_status ensure_staging(ttt_state* st, int i, size_t bytes) {
-  if (st->staging.bytes[i] >= bytes) return TTT_OK;
-  dev_free(st->staging.buf[i]);
-  st->staging.buf[i] = nullptr;
-  st->staging.bytes[i] = 0;
-  TTT_TRY(dev_alloc(&st->staging.buf[i], bytes, "host-call staging buffer"));
-  st->staging.bytes[i] = bytes;
+static ttt_status ensure_staging(ttt_state* st, int set, int i, size_t bytes) {
+  HostStaging& hs = st->staging;
+  if (hs.bytes[set][i] >= bytes) return TTT_OK;
+  dev_free(hs.buf[set][i]);
+  hs.buf[set][i] = nullptr;
+  hs.bytes[set][i] = 0;
+  TTT_TRY(dev_alloc(&hs.buf[set][i], bytes, "host-call staging buffer"));
+  hs.bytes[set][i] = bytes;
+  return TTT_OK;
+}
+
+static ttt_status ensure_pipeline(ttt_state* st) {
+  HostStaging& hs = st->staging;
+  if (hs.copy_out != nullptr) return TTT_OK;
+  cudaEvent_t* evs[] = {&hs.entry, &hs.in_done[0], &hs.in_done[1], &hs.scan_done[0], &hs.scan_done[1],
+                        &hs.out_done[0], &hs.out_done[1]};
+  for (cudaEvent_t* e : evs)
+    if (*e == nullptr) TTT_CUDA(cudaEventCreateWithFlags(e, cudaEventDisableTiming));
+  if (hs.copy_in == nullptr) TTT_CUDA(cudaStreamCreateWithFlags(&hs.copy_in, cudaStreamNonBlocking));
+  TTT_CUDA(cudaStreamCreateWithFlags(&hs.copy_out, cudaStreamNonBlocking));
+  return TTT_OK;
+}
+
+// Tokens of one segment of a host call: about a quarter of T (a few segments keep the copies
+// of one busy while the scan of another runs), in whole units of what a call may end on (the
+// chunk; the gate's 64-token chunk when the gate is on). The whole call where a call boundary
+// would change the result (the fused target's taps past the call end, pad mode 1), and for the
+// TTT-Linear family when it copies back less than a fifth of what it copies in: a segment of
+// [batch, heads, T, 64] tensors is a strided copy, which measured ~15 % slower over PCIe than
+// a plain one, more than overlapping the small copy back (the losses alone) gains.
+static int64_t host_segment(const ttt_config& c, int64_t T, size_t in_bytes, size_t out_bytes) {
+  if (c.rule == TTT_RULE_INPLACE_HEBBIAN && c.target_mode == 1 && c.conv_pad_mode == 1) return T;
+  if (c.rule != TTT_RULE_INPLACE_HEBBIAN && 5 * out_bytes < in_bytes) return T;
+  int64_t unit = c.chunk;
+  if (c.gate_enable) unit = unit * c.gate_chunk / std::gcd<int64_t>(unit, c.gate_chunk);
+  int64_t seg = (T / 4 + unit - 1) / unit * unit;
+  return seg < unit ? unit : (seg > T ? T : seg);
+}
+
+// Rows of `rows` [.., T, width] blocks (width bytes a token) between host and device memory for
+// tokens [t0, t0 + n): the device side is the dense segment [.., n, width].
+static ttt_status copy_segment(void* dst, const void* src, size_t width, int64_t T, int64_t t0, int64_t n,
+                               size_t rows, bool to_device, cudaStream_t s) {
+  if (n == T || rows == 1) {  // one contiguous range
+    const size_t off = t0 * width, bytes = rows * n * width;
+    if (to_device)
+      TTT_CUDA(cudaMemcpyAsync(dst, static_cast<const uint8_t*>(src) + off, bytes, cudaMemcpyHostToDevice, s));
+    else
+      TTT_CUDA(cudaMemcpyAsync(static_cast<uint8_t*>(dst) + off, src, bytes, cudaMemcpyDeviceToHost, s));
+    return TTT_OK;
+  }
+  if (to_device)
+    TTT_CUDA(cudaMemcpy2DAsync(dst, n * width, static_cast<const uint8_t*>(src) + t0 * width, T * width, n * width,
+                               rows, cudaMemcpyHostToDevice, s));
+  else
+    TTT_CUDA(cudaMemcpy2DAsync(static_cast<uint8_t*>(dst) + t0 * width, T * width, src, n * width, n * width, rows,
+                               cudaMemcpyDeviceToHost, s));
   return TTT_OK;
 }
 
@@ -484,27 +544,68 @@ ttt_status ttt_chunk_scan_host(ttt_state* st, const void* keys, const void* targ
   if (T < 0 || T % c.chunk != 0) return fail(TTT_ERR_INVALID_ARG, "T must be a non-negative multiple of the chunk");
   if (T == 0) return TTT_OK;
   if (keys == nullptr || targets == nullptr) return fail(TTT_ERR_INVALID_ARG, "keys and targets are required");
-  const size_t es = io_size(c.io_dtype);
-  const size_t bh = (size_t)c.batch * c.heads;
-  const size_t kb = bh * T * c.d_key * es;
-  const size_t vb = bh * T * c.d_val * es;
-  const size_t ob = c.rule == TTT_RULE_INPLACE_HEBBIAN ? T * c.d_val * es : bh * T * c.d_key * es;
-  const size_t lb = bh * T * sizeof(float);
   TTT_TRY(check_device(st));
-  TTT_TRY(ensure_staging(st, 0, kb));
-  TTT_TRY(ensure_staging(st, 1, vb));
-  if (queries != nullptr) TTT_TRY(ensure_staging(st, 2, kb));
-  if (out != nullptr) TTT_TRY(ensure_staging(st, 3, ob));
-  if (loss_out != nullptr) TTT_TRY(ensure_staging(st, 4, lb));
-  TTT_CUDA(cudaMemcpyAsync(st->staging.buf[0], keys, kb, cudaMemcpyHostToDevice, s));
-  TTT_CUDA(cudaMemcpyAsync(st->staging.buf[1], targets, vb, cudaMemcpyHostToDevice, s));
-  if (queries != nullptr) TTT_CUDA(cudaMemcpyAsync(st->staging.buf[2], queries, kb, cudaMemcpyHostToDevice, s));
-  TTT_TRY(scan_impl(st, st->staging.buf[0], st->staging.buf[1], queries ? st->staging.buf[2] : nullptr, T,
-                    out ? st->staging.buf[3] : nullptr, loss_out ? static_cast<float*>(st->staging.buf[4]) : nullptr,
-                    s));
-  if (out != nullptr) TTT_CUDA(cudaMemcpyAsync(out, st->staging.buf[3], ob, cudaMemcpyDeviceToHost, s));
-  if (loss_out != nullptr) TTT_CUDA(cudaMemcpyAsync(loss_out, st->staging.buf[4], lb, cudaMemcpyDeviceToHost, s));
-  TTT_CUDA(cudaStreamSynchronize(s));
+  // Per token: bytes of a key, target and output row, over `rows` blocks of T tokens each
+  // (In-Place: one [T, width] block; the TTT-Linear family: one block per (sequence, head)).
+  const size_t es = io_size(c.io_dtype);
+  const bool inplace = c.rule == TTT_RULE_INPLACE_HEBBIAN;
+  const size_t rows = inplace ? 1 : (size_t)c.batch * c.heads;
+  const size_t kw = (size_t)c.d_key * es, vw = (size_t)c.d_val * es, ow = (inplace ? c.d_val : c.d_key) * es;
+  const size_t lw = sizeof(float);
+  const void* hin[3] = {keys, targets, queries};
+  void* hout[2] = {out, loss_out};
+  const size_t win[3] = {kw, vw, kw}, wout[2] = {ow, lw};
+  size_t in_bytes = 0, out_bytes = 0;
+  for (int i = 0; i < 3; ++i) in_bytes += hin[i] != nullptr ? win[i] : 0;
+  for (int i = 0; i < 2; ++i) out_bytes += hout[i] != nullptr ? wout[i] : 0;
+  const int64_t seg = host_segment(c, T, in_bytes, out_bytes);
+  for (int j = 0; j < (seg < T ? 2 : 1); ++j) {
+    for (int i = 0; i < 3; ++i)
+      if (hin[i] != nullptr) TTT_TRY(ensure_staging(st, j, i, rows * seg * win[i]));
+    for (int i = 0; i < 2; ++i)
+      if (hout[i] != nullptr) TTT_TRY(ensure_staging(st, j, 3 + i, rows * seg * wout[i]));
+  }
+  TTT_TRY(ensure_pipeline(st));
+  HostStaging& hs = st->staging;
+  // Segment k uses buffer set k mod 2. Its inputs go up on the copy-in stream once the scan of
+  // segment k - 2 (the set's last reader) has ended; its scan runs on the caller's stream once
+  // they are there and segment k - 2's outputs (the set's last contents) are back; its outputs
+  // go down on the copy-out stream once its scan has ended. Each segment continues the scan
+  // exactly as a separate call would.
+  TTT_CUDA(cudaEventRecord(hs.entry, s));
+  TTT_CUDA(cudaStreamWaitEvent(hs.copy_in, hs.entry, 0));
+  TTT_CUDA(cudaStreamWaitEvent(hs.copy_out, hs.entry, 0));
+  ttt_status r = TTT_OK;
+  int k = 0;
+  for (int64_t t0 = 0; t0 < T && r == TTT_OK; t0 += seg, ++k) {
+    const int j = k & 1;
+    const int64_t n = std::min<int64_t>(seg, T - t0);
+    void** b = hs.buf[j];
+    auto step = [&]() -> ttt_status {
+      if (k >= 2) TTT_CUDA(cudaStreamWaitEvent(hs.copy_in, hs.scan_done[j], 0));
+      for (int i = 0; i < 3; ++i)
+        if (hin[i] != nullptr) TTT_TRY(copy_segment(b[i], hin[i], win[i], T, t0, n, rows, true, hs.copy_in));
+      TTT_CUDA(cudaEventRecord(hs.in_done[j], hs.copy_in));
+      TTT_CUDA(cudaStreamWaitEvent(s, hs.in_done[j], 0));
+      if (k >= 2) TTT_CUDA(cudaStreamWaitEvent(s, hs.out_done[j], 0));
+      TTT_TRY(scan_impl(st, b[0], b[1], queries ? b[2] : nullptr, n, out ? b[3] : nullptr,
+                        loss_out ? static_cast<float*>(b[4]) : nullptr, s));
+      TTT_CUDA(cudaEventRecord(hs.scan_done[j], s));
+      TTT_CUDA(cudaStreamWaitEvent(hs.copy_out, hs.scan_done[j], 0));
+      for (int i = 0; i < 2; ++i)
+        if (hout[i] != nullptr) TTT_TRY(copy_segment(hout[i], b[3 + i], wout[i], T, t0, n, rows, false, hs.copy_out));
+      TTT_CUDA(cudaEventRecord(hs.out_done[j], hs.copy_out));
+      return TTT_OK;
+    };
+    r = step();
+  }
+  // Whatever happened, nothing of this call is left in flight when it returns.
+  const cudaError_t e1 = cudaStreamSynchronize(hs.copy_in), e2 = cudaStreamSynchronize(s),
+                    e3 = cudaStreamSynchronize(hs.copy_out);
+  if (r != TTT_OK) return r;
+  if (e1 != cudaSuccess) return cuda_fail(e1, "copy-in stream");
+  if (e2 != cudaSuccess) return cuda_fail(e2, "scan stream");
+  if (e3 != cudaSuccess) return cuda_fail(e3, "copy-out stream");
   return TTT_OK;
 }
 

@@ -177,9 +177,17 @@ ttt_status ttt_chunk_scan(ttt_state* st, const void* keys, const void* targets,
                           const void* queries, int64_t T, void* out, float* loss_out,
                           ttt_stream stream);
 
-/* ttt_chunk_scan with HOST buffers of the same shapes: copies the inputs to device
- * staging buffers owned by the state (grown on demand), runs the scan, copies the outputs
- * back and synchronises `stream`. Host buffers should be pinned for full speed. */
+/* ttt_chunk_scan with HOST buffers of the same shapes, returning when the outputs are in
+ * host memory. T is cut into segments of about T/4 tokens (whole chunks; whole gate chunks
+ * with the gate; one segment for the fused target in conv_pad_mode 1, whose taps reach past
+ * the call's end, and for the TTT-Linear family when the outputs are less than a fifth of the
+ * inputs), each scanned as a separate ttt_chunk_scan call would be, so the results are those
+ * of one call. A segment's inputs are copied to one of two sets of device staging
+ * buffers owned by the state (grown on demand) on a copy stream of the state's, its scan runs
+ * on `stream`, its outputs come back on a second copy stream: the copies of neighbouring
+ * segments overlap each scan, in both directions at once. All three streams are synchronised
+ * before the call returns, on errors too. Host buffers should be pinned: copies from or to
+ * pageable memory do not overlap. */
 ttt_status ttt_chunk_scan_host(ttt_state* st, const void* keys, const void* targets,
                                const void* queries, int64_t T, void* out, float* loss_out,
                                ttt_stream stream);
