@@ -66,14 +66,15 @@ def target_conv(X0, convw, C: int, pad_mode: int = 0):
     """Depthwise future-tap convolution conv[t, i] = Σ_k w[i, k]·X0[t + k, i], k = 0..taps-1.
 
     A tap that would read past the boundary contributes zero; the boundary is the end of
-    token t's chunk (pad_mode 0) or the end of the sequence (pad_mode 1).
+    token t's chunk (pad_mode 0) or the end of the sequence (pad_mode 1), and never lies past
+    the sequence's end (a shorter last chunk has no tokens beyond T).
     """
     X = f64(X0)
     w = f64(convw)
     T, d = X.shape
     taps = w.shape[1]
     t = np.arange(T)
-    end = (t // C + 1) * C if pad_mode == 0 else np.full(T, T)
+    end = np.minimum((t // C + 1) * C, T) if pad_mode == 0 else np.full(T, T)
     out = np.zeros((T, d))
     for k in range(taps):
         src = t + k

@@ -22,13 +22,17 @@ Readings taken where the pages leave it open (a CUDA path must apply the same on
   1/(2b')·‖K·W − V‖², i.e. W ← W − (η/b')·Kᵀ(K·W − V);
 * clipping acts on each chunk's delta ΔW_c = η·V̂_cᵀ·Z_c on its own: if ‖ΔW_c‖_F exceeds the
   threshold, ΔW_c is scaled to that norm; the threshold is a parameter (None: no clipping).
+* with the target made inside the scan (V̂ = Conv1D(X0)·Wtarget, §4), each document's targets
+  are its own: the future taps stop at the document's end as they stop at the sequence's end
+  (and, in pad mode 0, at the end of each of its chunks, counted from its first token), so a
+  document's targets read nothing of the next document.
 """
 
 from __future__ import annotations
 
 import numpy as np
 
-from . import inner
+from . import inner, inplace
 from ._util import f64
 
 
@@ -62,6 +66,18 @@ def inplace_scan_docs(Z, Vhat, W0, eta: float, C: int, doc_starts, clip=None):
             O[rows] = Zd[rows] @ W.T                     # apply first
             W = W + clip_delta(eta * (Vd[rows].T @ Zd[rows]), clip)   # then update
     return O, W
+
+
+def inplace_scan_docs_target(Z, X0, convw, Wtarget, W0, eta: float, C: int, doc_starts, pad_mode: int = 0,
+                             clip=None):
+    """inplace_scan_docs with each document's targets V̂ = Conv1D(X0)·Wtarget computed from
+    that document alone (X0 [T, d], convw [d, taps], Wtarget [d, d])."""
+    X = f64(X0)
+    T = X.shape[0]
+    V = np.empty((T, f64(Wtarget).shape[1]))
+    for a, e in _documents(doc_starts, T):
+        V[a:e] = inplace.target_values(X[a:e], convw, Wtarget, C, pad_mode)
+    return inplace_scan_docs(Z, V, W0, eta, C, doc_starts, clip)
 
 
 def ttt_linear_scan_docs(K, V, Q, W0, eta: float, b: int, doc_starts, token_weights: bool = False):

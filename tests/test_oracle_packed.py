@@ -179,3 +179,49 @@ def _inner_per_document(model):
     np.testing.assert_allclose(L[:, :, 8:13], tail[-1], rtol=0, atol=1e-12)
     for got, want in zip(W if model == "mlp" else (W,), weights(tail) if model == "mlp" else (weights(tail),)):
         np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
+
+
+def _target_inputs(T, C, d, f, seed):
+    Z, X0 = _rand((T, f), seed), _rand((T, d), seed + 1)
+    w, Wt, W0 = _rand((d, 3), seed + 2, 0.6), _rand((d, d), seed + 3, 0.3), _rand((d, f), seed + 4, 0.1)
+    return Z, X0, w, Wt, W0
+
+
+def test_fused_target_one_document_is_the_fused_target_scan():
+    """One document: the scan with the targets Conv1D(X0)·Wtarget of the whole sequence (both
+    padding modes)."""
+    T, C, d, f, eta = 96, 32, 5, 7, 0.05
+    Z, X0, w, Wt, W0 = _target_inputs(T, C, d, f, 30)
+    for pad_mode in (0, 1):
+        O, W = packed.inplace_scan_docs_target(Z, X0, w, Wt, W0, eta, C, [0], pad_mode)
+        O_ref, W_ref = inplace.inplace_scan(Z, inplace.target_values(X0, w, Wt, C, pad_mode), W0, eta, C)
+        np.testing.assert_allclose(O, O_ref, rtol=0, atol=1e-13)
+        np.testing.assert_allclose(W, W_ref, rtol=0, atol=1e-13)
+
+
+def test_fused_target_documents_read_only_their_own_rows():
+    for pad_mode in (0, 1):
+        _documents_read_only_their_own_rows(pad_mode)
+
+
+def _documents_read_only_their_own_rows(pad_mode):
+    """Documents of 64 (two whole chunks: its last taps sit right before the next document),
+    37 and 59 tokens: each document's outputs are those of the same call on that document
+    alone, and changing another document's X0 changes none of them."""
+    T, C, d, f, eta = 160, 32, 4, 6, 0.08
+    Z, X0, w, Wt, W0 = _target_inputs(T, C, d, f, 40)
+    starts = [0, 64, 101]
+    O, W = packed.inplace_scan_docs_target(Z, X0, w, Wt, W0, eta, C, starts, pad_mode)
+    bounds = list(zip(starts, starts[1:] + [T]))
+    for a, e in bounds:
+        O_doc, W_doc = packed.inplace_scan_docs_target(Z[a:e], X0[a:e], w, Wt, W0, eta, C, [0], pad_mode)
+        np.testing.assert_allclose(O[a:e], O_doc, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(W, W_doc, rtol=0, atol=1e-13)
+    for k, (a, e) in enumerate(bounds):
+        X1 = X0.copy()
+        X1[a:e] += 5.0
+        O1, _ = packed.inplace_scan_docs_target(Z, X1, w, Wt, W0, eta, C, starts, pad_mode)
+        for j, (a2, e2) in enumerate(bounds):
+            if j != k:
+                np.testing.assert_array_equal(O1[a2:e2], O[a2:e2])
+        assert not np.allclose(O1[a:e], O[a:e])

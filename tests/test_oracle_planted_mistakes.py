@@ -34,7 +34,7 @@ MUTANTS = [
     ("inplace", "convolution tap shifted by one token",
      [("        src = t + k\n", "        src = t + k + 1\n")]),
     ("inplace", "convolution ignores the chunk boundary",
-     [("end = (t // C + 1) * C if pad_mode == 0 else np.full(T, T)", "end = np.full(T, T)")]),
+     [("end = np.minimum((t // C + 1) * C, T) if pad_mode == 0 else np.full(T, T)", "end = np.full(T, T)")]),
     ("inplace", "convolution weights of the wrong tap",
      [("out[ok] += X[src[ok]] * w[:, k]", "out[ok] += X[src[ok]] * w[:, taps - 1 - k]")]),
     ("linear", "wrong sign of the gradient step",
@@ -100,6 +100,12 @@ MUTANTS = [
        "kc, vc, gc = Vd[bi, hi, ts], Kd[bi, hi, ts], ts // gate_chunk")]),
     ("cache_attention", "query of the previous token",
      [("s = (kc[visible] @ Qd[bi, hi, t]) * scale", "s = (kc[visible] @ Qd[bi, hi, t - 1]) * scale")]),
+    ("packed", "fused targets of a document computed over the whole packed sequence",
+     [("V[a:e] = inplace.target_values(X[a:e], convw, Wtarget, C, pad_mode)",
+       "V[a:e] = inplace.target_values(X, convw, Wtarget, C, pad_mode)[a:e]")]),
+    ("packed", "fused targets of packed documents always padded at chunk ends",
+     [("V[a:e] = inplace.target_values(X[a:e], convw, Wtarget, C, pad_mode)",
+       "V[a:e] = inplace.target_values(X[a:e], convw, Wtarget, C, 0)")]),
     ("packed", "In-Place weight not reset at a document start",
      [("        W = W0d.copy()                                   # document boundary: pretrained weight\n",
        "")]),
