@@ -75,6 +75,13 @@ struct InplaceBuffers {
   double* docs_sumsq = nullptr;
   int64_t docs_rows_cap = 0;
   int docs_chunks_cap = 0;
+  // With the target made in the scan: the padded layout's conv rows and targets [Tp, d_val]
+  // and the target tiles' schedule, grown on demand.
+  __nv_bfloat16* docs_conv = nullptr;
+  __nv_bfloat16* docs_T = nullptr;
+  int32_t* docs_plan = nullptr;
+  int64_t docs_target_cap = 0;
+  int64_t docs_plan_cap = 0;
 };
 
 // Tensor maps of one scan's K, V, Q, O (encoding them costs microseconds of host time, so the
@@ -164,6 +171,13 @@ size_t io_size(int dtype);
 // ---- kernel launchers (each returns TTT_OK or TTT_ERR_CUDA after the launch) ----------
 
 // In-Place, fp32 SIMT: one chunk of the scan (apply with W, then W += η·V̂ᵀZ).
+// Targets V̂ = Conv1D(X0)·Wtarget for T tokens (T a multiple of 128) into `out`, with the
+// caller's scratch for the conv rows [T, d] and the tile schedule (target_values_plan_ints).
+int target_values_plan_ints(int T, int d, int num_sms);
+ttt_status target_values_into(const __nv_bfloat16* X0, const float* convw, const __nv_bfloat16* Wtarget, int T, int d,
+                              int C, int taps, int pad_mode, __nv_bfloat16* conv_scratch, int32_t* plan_scratch,
+                              __nv_bfloat16* out, int32_t* status, int num_sms, cudaStream_t s);
+
 ttt_status inplace_f32_chunk(ttt_state* st, const float* Z, const float* Vhat, const float* W, float* Wn, float* O,
                              int C, cudaStream_t s);
 

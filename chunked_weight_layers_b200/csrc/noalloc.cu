@@ -29,11 +29,6 @@
 
 namespace ttt {
 
-int target_values_plan_ints(int T, int d, int num_sms);
-ttt_status target_values_into(const __nv_bfloat16* X0, const float* convw, const __nv_bfloat16* Wtarget, int T, int d,
-                              int C, int taps, int pad_mode, __nv_bfloat16* conv_scratch, int32_t* plan_scratch,
-                              __nv_bfloat16* out, int32_t* status, int num_sms, cudaStream_t s);
-
 namespace {
 
 constexpr size_t kMaxConvElems = (size_t)1 << 22;  // T·d ≤ 4,194,304 (8 MB of bf16 conv rows)

@@ -361,11 +361,18 @@ ttt_status inplace_bf16_scan_docs(ttt_state* st, const __nv_bfloat16* Z, const _
   const size_t nelem = (size_t)d * f;
   InplaceBuffers& ip = st->ip;
   // Padded layout: every document starts a chunk and fills its last chunk with zero rows (a
-  // zero row of Z and V̂ adds nothing to the delta, and its output row is dropped).
+  // zero row of Z and V̂ adds nothing to the delta, and its output row is dropped). With the
+  // target made here (`targets` is X0), the targets come from the padded X0: in pad mode 0 the
+  // taps stop at each chunk end, which the layout aligns with the documents; in pad mode 1 they
+  // stop only at the end of the layout, so each document is followed by at least taps − 1 zero
+  // rows (one more chunk of padding where its last chunk has fewer spare rows), which its last
+  // tokens' taps read instead of the next document.
+  const bool target = c.target_mode == 1;
+  const int64_t tail = target && c.conv_pad_mode == 1 ? c.conv_taps - 1 : 0;
   std::vector<int32_t> rows, reset;
   for (int k = 0; k < ndocs; ++k) {
     const int64_t a = doc_starts[k], e = k + 1 < ndocs ? doc_starts[k + 1] : T;
-    const int64_t nch = (e - a + C - 1) / C;
+    const int64_t nch = (e - a + tail + C - 1) / C;
     for (int64_t j = 0; j < nch; ++j) {
       reset.push_back(j == 0 ? 1 : 0);
       for (int r = 0; r < C; ++r) {
@@ -378,6 +385,7 @@ ttt_status inplace_bf16_scan_docs(ttt_state* st, const __nv_bfloat16* Z, const _
   const int64_t Tp = (int64_t)n * C;
   if (Tp > (int64_t)INT32_MAX / 2) return fail(TTT_ERR_UNSUPPORTED, "padded length too large");
   if (ip.docs_rows_cap < Tp) {
+    ip.docs_rows_cap = 0;  // until every buffer below has its new size
     TTT_TRY(grow(&ip.docs_Z, (size_t)Tp * f));
     TTT_TRY(grow(&ip.docs_V, (size_t)Tp * d));
     TTT_TRY(grow(&ip.docs_O, (size_t)Tp * d));
@@ -385,6 +393,7 @@ ttt_status inplace_bf16_scan_docs(ttt_state* st, const __nv_bfloat16* Z, const _
     ip.docs_rows_cap = Tp;
   }
   if (ip.docs_chunks_cap < n) {
+    ip.docs_chunks_cap = 0;
     TTT_TRY(grow(&ip.docs_reset, (size_t)n));
     TTT_TRY(grow(&ip.docs_sumsq, (size_t)n));
     ip.docs_chunks_cap = n;
@@ -408,10 +417,29 @@ ttt_status inplace_bf16_scan_docs(ttt_state* st, const __nv_bfloat16* Z, const _
   k_gather_rows<<<gblocks, 256, 0, s>>>(Vhat, ip.docs_V, ip.docs_rows, (long long)Tp, d);
   st->launches += 2;
   TTT_CUDA(cudaGetLastError());
+  const __nv_bfloat16* Vp = ip.docs_V;  // the padded targets
+  if (target) {
+    const int64_t plan = target_values_plan_ints((int)Tp, d, st->num_sms);
+    if (ip.docs_target_cap < Tp) {
+      ip.docs_target_cap = 0;
+      TTT_TRY(grow(&ip.docs_conv, (size_t)Tp * d));
+      TTT_TRY(grow(&ip.docs_T, (size_t)Tp * d));
+      ip.docs_target_cap = Tp;
+    }
+    if (ip.docs_plan_cap < plan) {
+      ip.docs_plan_cap = 0;
+      TTT_TRY(grow(&ip.docs_plan, (size_t)plan));
+      ip.docs_plan_cap = plan;
+    }
+    TTT_TRY(target_values_into(ip.docs_V, ip.convw, ip.Wtarget, (int)Tp, d, C, c.conv_taps, c.conv_pad_mode,
+                               ip.docs_conv, ip.docs_plan, ip.docs_T, st->status.dev, st->num_sms, s));
+    st->launches += 3;
+    Vp = ip.docs_T;
+  }
 
   // 1. D_j = η·V̂_jᵀ·Z_j over the padded chunks.
   CUtensorMap tV, tZm;
-  TTT_TRY(map_bf16(&tV, ip.docs_V, d, Tp, 64, 64));
+  TTT_TRY(map_bf16(&tV, Vp, d, Tp, 64, 64));
   TTT_TRY(map_bf16(&tZm, ip.docs_Z, f, Tp, 64, 64));
   GemmArgs ga{d, f, C, 1, 1, C, C, ip.prefix_D, 1, (long long)nelem, f, c.eta, ds};
   TTT_TRY(gemm(st, tV, tZm, ga, n, s));

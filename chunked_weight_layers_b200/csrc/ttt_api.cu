@@ -134,6 +134,9 @@ static void free_state(ttt_state* st) {
   dev_free(st->ip.docs_rows);
   dev_free(st->ip.docs_reset);
   dev_free(st->ip.docs_sumsq);
+  dev_free(st->ip.docs_conv);
+  dev_free(st->ip.docs_T);
+  dev_free(st->ip.docs_plan);
   dev_free(st->ip.Wsh[0]);
   dev_free(st->ip.Wsh[1]);
   dev_free(st->ip.Wsh[2]);
@@ -480,8 +483,8 @@ ttt_status ttt_chunk_scan_docs(ttt_state* st, const void* keys, const void* targ
                                const int64_t* doc_starts, int32_t ndocs, float clip_norm, ttt_stream stream) {
   if (st == nullptr) return fail(TTT_ERR_INVALID_ARG, "state is NULL");
   const ttt_config& c = st->cfg;
-  if (c.rule != TTT_RULE_INPLACE_HEBBIAN || c.io_dtype != TTT_BF16 || c.target_mode != 0)
-    return fail(TTT_ERR_UNSUPPORTED, "packed sequences run In-Place BF16 states with given targets");
+  if (c.rule != TTT_RULE_INPLACE_HEBBIAN || c.io_dtype != TTT_BF16)
+    return fail(TTT_ERR_UNSUPPORTED, "packed sequences of this call run In-Place BF16 states");
   if (T < 0 || T > (int64_t)INT32_MAX / 4) return fail(TTT_ERR_INVALID_ARG, "T out of range");
   if (!(clip_norm >= 0.f)) return fail(TTT_ERR_INVALID_ARG, "clip_norm must be >= 0 (0: no clipping)");
   if (T == 0) return TTT_OK;

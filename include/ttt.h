@@ -192,13 +192,16 @@ ttt_status ttt_chunk_scan_host(ttt_state* st, const void* keys, const void* targ
                                const void* queries, int64_t T, void* out, float* loss_out,
                                ttt_stream stream);
 
-/* Packed sequences for In-Place BF16 states with given targets (target_mode 0): `keys` Z
- * (device, bf16 [T, d_key]) and `targets` V̂ (device, bf16 [T, d_val]) hold documents laid end
+/* Packed sequences for In-Place BF16 states: `keys` Z (device, bf16 [T, d_key]) and `targets`
+ * (device, bf16 [T, d_val]: V̂ with target_mode 0, X0 with target_mode 1) hold documents laid end
  * to end; `doc_starts` (HOST, int64 [ndocs]) lists each document's first token: 0 first,
  * strictly increasing, below T. Each document is scanned as if alone: the weight starts from
  * the pretrained W0, its chunks are counted from its first token (its last chunk may be
  * shorter: T need not be a multiple of chunk), and with clip_norm > 0 each chunk's delta
  * η·V̂_cᵀ·Z_c is scaled to Frobenius norm clip_norm when its norm is larger (0: no clipping).
+ * With target_mode 1 each document's targets Conv1D(X0)·Wtarget are made from its own rows:
+ * the taps stop at its end (and in conv_pad_mode 0 at the end of each of its chunks, counted
+ * from its first token).
  * Writes `out` (device, bf16 [T, d_val]); afterwards the state holds the last document's
  * final weight. Runs in the context-parallel form (all chunk deltas, their norms, sums that
  * restart at each document, all outputs), with state-owned scratch for the padded layout and

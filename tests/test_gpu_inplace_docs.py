@@ -118,6 +118,60 @@ def test_rejects_bad_arguments(cwl):
     assert e.value.status == abi.TTT_ERR_UNSUPPORTED
 
 
+def _target_state(cwl, x, C, eta, pad_mode):
+    d, f = x["W0"].shape
+    cfg = cwl.config("inplace", io_dtype=1, d_key=f, d_val=d, chunk=C, eta=eta, target_mode=1,
+                     conv_pad_mode=pad_mode)
+    return cwl.FastWeightState(cfg, x["W0"], x["Wtarget"], x["convw"])
+
+
+def _run(st, Z, targets, doc_starts, clip=None):
+    O = torch.full((Z.shape[0], st.cfg.d_val), float("nan"), device="cuda", dtype=torch.bfloat16)
+    st.chunk_scan_docs(Z, targets, doc_starts, clip=clip, out=O)
+    W = torch.empty((st.cfg.d_val, st.cfg.d_key), device="cuda")
+    st.get_weights(W)
+    torch.cuda.synchronize()
+    st.poll()
+    return O, W
+
+
+@pytest.mark.parametrize("pad_mode", [0, 1])
+@pytest.mark.parametrize("clip", [None, 0.04])
+def test_fused_target_documents_against_oracle(cwl, pad_mode, clip):
+    """The target made inside the scan from X0, per document: documents of 256 tokens (whole
+    chunks: in pad mode 1 its last taps would reach the next document without the extra
+    padding), 44, 211 and 189 tokens, with and without clipping, against the oracle."""
+    spec = workloads.scaled(workloads.INPLACE_128K_TARGET, T=700, C=128, d=256, f=384, seed=91 + pad_mode)
+    x = workloads.inplace_inputs(spec, device="cuda")
+    starts = [0, 256, 300, 511]
+    c = {k: x[k].cpu() for k in ("Z", "X0", "convw", "Wtarget", "W0")}
+    O_ref, W_ref = opk.inplace_scan_docs_target(c["Z"], c["X0"], c["convw"], c["Wtarget"], c["W0"], spec.eta, spec.C,
+                                                starts, pad_mode, clip)
+    O, W = _run(_target_state(cwl, x, spec.C, spec.eta, pad_mode), x["Z"], x["X0"], starts, clip)
+    eo, ew = rel_err(O, O_ref), rel_err(W, W_ref)
+    print(f"packed fused target pad {pad_mode} clip {clip}: O {eo:.3e}  W {ew:.3e}")
+    assert eo <= TOL and ew <= TOL
+
+
+@pytest.mark.parametrize("pad_mode", [0, 1])
+def test_fused_target_one_document_equals_given_targets(cwl, pad_mode):
+    """One document of whole chunks: the targets made inside the call are those of
+    ttt_target_values_noalloc (the same kernels) and the scan then equals the packed scan with
+    those targets given, bit for bit."""
+    from chunked_weight_layers_b200 import abi
+    spec = workloads.scaled(workloads.INPLACE_128K_TARGET, T=512, C=128, d=256, f=384, seed=95)
+    x = workloads.inplace_inputs(spec, device="cuda")
+    V = torch.empty((spec.T, spec.d), device="cuda", dtype=torch.bfloat16)
+    lib = abi.load()
+    r = lib.ttt_target_values_noalloc(x["X0"].data_ptr(), x["convw"].data_ptr(), x["Wtarget"].data_ptr(), spec.T,
+                                      spec.d, spec.C, 3, pad_mode, V.data_ptr(), None,
+                                      torch.cuda.current_stream().cuda_stream or None)
+    assert r == abi.TTT_OK
+    O1, W1 = _run(_target_state(cwl, x, spec.C, spec.eta, pad_mode), x["Z"], x["X0"], [0])
+    O2, W2 = _run(new_state(cwl, x["W0"], spec.C, spec.eta), x["Z"], V, [0])
+    assert torch.equal(O1, O2) and torch.equal(W1, W2)
+
+
 ROWS = [0, 1, 127, 128, 1000, 2047, 2048, 2559]
 
 
