@@ -146,3 +146,20 @@ def test_inplace_f32(cwl):
     cfg = cwl.config("inplace", io_dtype=0, d_key=spec.f, d_val=spec.d, chunk=spec.C, eta=spec.eta)
     _assert_same(*_both_paths(lambda: cwl.FastWeightState(cfg, x["W0"]), (x["Z"], x["Vhat"], None),
                               ((spec.T, spec.d), torch.float32), None, _weights(x["W0"])))
+
+
+def test_pageable_host_buffers(cwl):
+    """Host buffers that are not pinned: the copies do not overlap, the results are the same."""
+    spec = workloads.scaled(workloads.LINEAR_GD, B=2, H=2, T=16 * 11, seed=529)
+    x = workloads.linear_inputs(spec, device="cuda")
+    cfg = cwl.config("linear", batch=spec.B, heads=spec.H, chunk=16, eta=spec.eta)
+    shape = (spec.B, spec.H, spec.T)
+    st_d = cwl.FastWeightState(cfg, x["W0"])
+    O_d, L_d = torch.empty(shape + (64,), device="cuda", dtype=torch.bfloat16), torch.empty(shape, device="cuda")
+    st_d.chunk_scan(x["K"], x["V"], x["Q"], out=O_d, loss_out=L_d)
+    st_h = cwl.FastWeightState(cfg, x["W0"])
+    O_h, L_h = torch.empty(shape + (64,), dtype=torch.bfloat16), torch.empty(shape)
+    st_h.chunk_scan_host(x["K"].cpu(), x["V"].cpu(), x["Q"].cpu(), out=O_h, loss_out=L_h)
+    torch.cuda.synchronize()
+    assert torch.equal(O_d.cpu(), O_h) and torch.equal(L_d.cpu(), L_h)
+    assert torch.equal(_weights(x["W0"])(st_d)[0], _weights(x["W0"])(st_h)[0])
