@@ -71,6 +71,15 @@ RULES = {"inplace": abi.TTT_RULE_INPLACE_HEBBIAN, "linear": abi.TTT_RULE_LINEAR_
          "linear_ln": abi.TTT_RULE_LINEAR_LN_GD, "mlp": abi.TTT_RULE_MLP_GD}
 
 
+def add_f32(y, x, alpha: float = 1.0, stream=None):
+    """ttt_add_f32: y ← y + alpha·x for fp32 device tensors of the same size; returns y."""
+    dev = _current_device()
+    n = y.numel()
+    check(abi.load().ttt_add_f32(_arg(y, "y", torch.float32, n, dev), _arg(x, "x", torch.float32, n, dev),
+                                 float(alpha), n, _stream(stream)))
+    return y
+
+
 def config(rule: str, **fields) -> abi.ttt_config:
     """A ttt_config with the library's defaults for ``rule`` ("inplace", "linear", "linear_ln"
     or "mlp"), then ``fields`` applied (e.g. ``d_key=512, d_val=256, chunk=512, eta=0.01``)."""

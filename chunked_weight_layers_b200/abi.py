@@ -77,6 +77,7 @@ _SIGNATURES = {
     "ttt_state_reset": (_st, [_vp, _vp]),
     "ttt_state_get_weights": (_st, [_vp, _vp, _vp]),
     "ttt_state_set_weights": (_st, [_vp, _vp, _vp]),
+    "ttt_add_f32": (_st, [_vp, _vp, ctypes.c_float, ctypes.c_int64, _vp]),
     "ttt_state_set_layernorm": (_st, [_vp, _vp, _vp, _vp]),
     "ttt_cache_read": (_st, [_vp, _vp, _vp, _vp]),
     "ttt_gate_read": (_st, [_vp, _vp, _vp, _vp]),

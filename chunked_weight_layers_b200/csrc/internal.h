@@ -178,6 +178,9 @@ ttt_status target_values_into(const __nv_bfloat16* X0, const float* convw, const
                               int C, int taps, int pad_mode, __nv_bfloat16* conv_scratch, int32_t* plan_scratch,
                               __nv_bfloat16* out, int32_t* status, int num_sms, cudaStream_t s);
 
+// y ← y + alpha·x over n fp32 elements (device), on stream s.
+ttt_status add_f32(float* y, const float* x, float alpha, size_t n, int num_sms, cudaStream_t s);
+
 ttt_status inplace_f32_chunk(ttt_state* st, const float* Z, const float* Vhat, const float* W, float* Wn, float* O,
                              int C, cudaStream_t s);
 

@@ -663,6 +663,16 @@ ttt_status ttt_state_get_weights(const ttt_state* st, float* W, ttt_stream strea
   return TTT_OK;
 }
 
+ttt_status ttt_add_f32(float* y, const float* x, float alpha, int64_t n, ttt_stream stream) {
+  if (n < 0) return fail(TTT_ERR_INVALID_ARG, "n must be non-negative");
+  if (n == 0) return TTT_OK;
+  if (y == nullptr || x == nullptr) return fail(TTT_ERR_INVALID_ARG, "y and x must be device pointers");
+  int dev = 0, sms = 0;
+  TTT_CUDA(cudaGetDevice(&dev));
+  TTT_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  return add_f32(y, x, alpha, (size_t)n, sms, reinterpret_cast<cudaStream_t>(stream));
+}
+
 ttt_status ttt_state_set_weights(ttt_state* st, const float* W, ttt_stream stream) {
   if (st == nullptr || W == nullptr || !aligned16(W)) return fail(TTT_ERR_INVALID_ARG, "state and an aligned W are required");
   TTT_TRY(check_device(st));

@@ -21,6 +21,27 @@ __global__ void k_f32_to_bf16(const float* __restrict__ src, __nv_bfloat16* __re
   }
 }
 
+// y ← y + alpha·x, four elements a thread where both are 16-byte aligned, else one.
+__global__ void k_add_f32(float* __restrict__ y, const float* __restrict__ x, float alpha, size_t n) {
+  const size_t stride = (size_t)gridDim.x * blockDim.x;
+  const size_t i0 = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (((reinterpret_cast<uintptr_t>(y) | reinterpret_cast<uintptr_t>(x)) & 15u) == 0) {
+    const size_t n4 = n / 4;
+    for (size_t i = i0; i < n4; i += stride) {
+      float4 a = reinterpret_cast<float4*>(y)[i];
+      const float4 b = reinterpret_cast<const float4*>(x)[i];
+      a.x = fmaf(alpha, b.x, a.x);
+      a.y = fmaf(alpha, b.y, a.y);
+      a.z = fmaf(alpha, b.z, a.z);
+      a.w = fmaf(alpha, b.w, a.w);
+      reinterpret_cast<float4*>(y)[i] = a;
+    }
+    for (size_t i = n4 * 4 + i0; i < n; i += stride) y[i] = fmaf(alpha, x[i], y[i]);
+  } else {
+    for (size_t i = i0; i < n; i += stride) y[i] = fmaf(alpha, x[i], y[i]);
+  }
+}
+
 __global__ void k_fill_i32(int32_t* dst, int32_t v, size_t n) {
   const size_t stride = (size_t)gridDim.x * blockDim.x;
   for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) dst[i] = v;
@@ -37,6 +58,16 @@ ttt_status f32_to_bf16(const float* src, __nv_bfloat16* dst, size_t n, cudaStrea
   if (n == 0) return TTT_OK;
   k_f32_to_bf16<<<grid_for((n + 3) / 4, 256, st), 256, 0, s>>>(src, dst, n);
   st->launches++;
+  TTT_CUDA(cudaGetLastError());
+  return TTT_OK;
+}
+
+ttt_status add_f32(float* y, const float* x, float alpha, size_t n, int num_sms, cudaStream_t s) {
+  if (n == 0) return TTT_OK;
+  size_t blocks = (n / 4 + 255) / 256 + 1;
+  const size_t cap = (size_t)(num_sms > 0 ? num_sms : 148) * 8;
+  if (blocks > cap) blocks = cap;
+  k_add_f32<<<(int)blocks, 256, 0, s>>>(y, x, alpha, n);
   TTT_CUDA(cudaGetLastError());
   return TTT_OK;
 }

@@ -260,6 +260,15 @@ ttt_status ttt_state_reset(ttt_state* st, ttt_stream stream);
 ttt_status ttt_state_get_weights(const ttt_state* st, float* W, ttt_stream stream);
 ttt_status ttt_state_set_weights(ttt_state* st, const float* W, ttt_stream stream);
 
+/* y ← y + alpha·x over n fp32 elements (device buffers of the current device; y and x may
+ * not overlap unless equal), enqueued on `stream`. The context-parallel form across devices
+ * combines weights with it: the In-Place update η·V̂ᵀ·Z does not depend on W, so the weight a
+ * device's first chunk starts from is the weight before the sequence plus the sums of the
+ * deltas of the devices before it ("In-Place Test-Time Training", §6, context parallelism: an
+ * exclusive prefix sum of the chunk deltas). Errors: INVALID_ARG (NULL with n > 0, n < 0),
+ * CUDA. */
+ttt_status ttt_add_f32(float* y, const float* x, float alpha, int64_t n, ttt_stream stream);
+
 /* Set the LayerNorm gain and bias of the inner model (TTT_RULE_LINEAR_LN_GD and
  * TTT_RULE_MLP_GD states; UNSUPPORTED otherwise): gamma and beta (device) fp32 [heads, 64],
  * shared by every sequence. They are parameters of the outer model: the scan reads them and

@@ -139,3 +139,82 @@ def test_inplace_rows_shard_across_two_gloo_ranks():
             p.join(timeout=120)
             assert p.exitcode == 0
         assert out[0] is True and out[1] is True
+
+
+class _OracleWholeState(_OracleState):
+    """The oracle's scan of the whole weight, with set_weights (the calls SequenceShardedInplace
+    makes)."""
+
+    def chunk_scan(self, Z, Vhat, out, T):
+        from oracle import inplace
+        O, W = inplace.inplace_scan(Z[:T].numpy(), Vhat[:T].numpy(), self.W.numpy(), self.cfg.eta, self.cfg.chunk)
+        out.copy_(torch.from_numpy(O))
+        self.W = torch.from_numpy(W)
+
+    def set_weights(self, W):
+        self.W = W.clone()
+
+
+def _add(y, x, alpha):
+    y.add_(x, alpha=alpha)
+    return y
+
+
+def _sequence_worker(rank, world, port, out):
+    """Each rank runs SequenceShardedInplace (the product's host logic: a first scan from zero
+    for the rank's delta sum, the all-gather, the rank's start and end weights) over the oracle's
+    scan, on its own run of chunks; the outputs of all ranks in token order and the final weight
+    must be the single-process scan's, over two calls in a row."""
+    import numpy as np
+    import chunked_weight_layers_b200 as cwl
+    from chunked_weight_layers_b200.dist import SequenceShardedInplace
+    from oracle import inplace
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        rng = np.random.default_rng(11)
+        C, d, f, eta = 32, 7, 9, 0.05
+        calls = [96 * world, 32 * world]  # tokens of each call: 3 chunks a rank, then 1
+        T = sum(calls)
+        Z, V, W0 = rng.standard_normal((T, f)), rng.standard_normal((T, d)), 0.1 * rng.standard_normal((d, f))
+        cfg = cwl.abi.ttt_config()
+        cfg.rule, cfg.io_dtype, cfg.d_key, cfg.d_val, cfg.chunk, cfg.eta = 0, 0, f, d, C, eta
+        layer = SequenceShardedInplace(cfg, torch.from_numpy(W0), make_state=_OracleWholeState, add=_add)
+        Zt, Vt = torch.from_numpy(Z), torch.from_numpy(V)
+        mine, t0 = [], 0
+        for n in calls:
+            a, b = shard_range(n // C, rank, world)
+            sl = slice(t0 + a * C, t0 + b * C)
+            mine.append((sl, layer.scan(Zt[sl], Vt[sl])))
+            t0 += n
+        O_ref, W_ref = inplace.inplace_scan(Z, V, W0, cfg.eta, C)
+        ok = all(np.allclose(o.numpy(), O_ref[sl], rtol=0, atol=1e-12) for sl, o in mine)
+        ok = ok and np.allclose(layer.get_weights().numpy(), W_ref, rtol=0, atol=1e-12)
+        # Without the exchange every rank after the first would start from W0.
+        if rank > 0:
+            O_alone, _ = inplace.inplace_scan(Z[mine[0][0]], V[mine[0][0]], W0, cfg.eta, C)
+            ok = ok and not np.allclose(O_alone, mine[0][1].numpy())
+        layer.reset()
+        ok = ok and np.array_equal(layer.get_weights().numpy(), W0)
+        out[rank] = bool(ok)
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_inplace_sequence_shards_across_gloo_ranks(world):
+    """The context-parallel form across ranks: each rank scans its own chunks of the sequence and
+    the ranks exchange their delta sums once a call; the outputs in token order and the final
+    weight equal the single-process scan (to float64 rounding)."""
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as m:
+        out = m.dict()
+        port = _free_port()
+        procs = [ctx.Process(target=_sequence_worker, args=(r, world, port, out)) for r in range(world)]
+        for p in procs:
+            p.start()
+        for p in procs:
+            p.join(timeout=120)
+            assert p.exitcode == 0
+        assert all(out[r] is True for r in range(world))
