@@ -799,17 +799,20 @@ def cpu_baseline_cache_read(limit_s) -> dict:
 
 
 def run_row_sharded(spec, a, world, rank, local, peaks):
-    """One In-Place layer split over the ranks by Wdown rows (RowShardedInplace): every rank holds
-    the whole Z and V̂ (same seed) and its rows of W; a step is one scan of the T tokens on every
-    rank plus the all-gather of the output columns. Strong scaling: value = T / the slowest
-    rank's time per step."""
+    """One In-Place layer split over the ranks, strong scaling: value = T / the slowest rank's
+    time per step. ``--shard rows`` (RowShardedInplace): every rank holds the whole Z and V̂
+    (same seed) and its rows of W; a step is one scan of the T tokens plus the all-gather of the
+    output columns. ``--shard sequence`` (SequenceShardedInplace, the context-parallel form
+    across devices): every rank holds its own run of whole chunks of Z and V̂ and the whole W; a
+    step is its two scans of those chunks plus the all-gather of the ranks' delta sums, and its
+    outputs stay on the rank."""
     import datetime
 
     import torch.distributed as dist
     from chunked_weight_layers_b200 import build
-    from chunked_weight_layers_b200.dist import RowShardedInplace, max_over_ranks
+    from chunked_weight_layers_b200.dist import RowShardedInplace, SequenceShardedInplace, max_over_ranks, shard_range
     if not isinstance(spec, wl.InplaceSpec) or spec.target or spec.dtype != "bf16":
-        raise SystemExit("--shard rows takes an In-Place bf16 workload with given targets")
+        raise SystemExit(f"--shard {a.shard} takes an In-Place bf16 workload with given targets")
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
     if world > 1:
@@ -821,7 +824,12 @@ def run_row_sharded(spec, a, world, rank, local, peaks):
     import chunked_weight_layers_b200 as cwl
     x = wl.inplace_inputs(spec, device=device)
     cfg = cwl.config("inplace", io_dtype=1, d_key=spec.f, d_val=spec.d, chunk=spec.C, eta=spec.eta)
-    layer = RowShardedInplace(cfg, x["W0"])
+    if a.shard == "rows":
+        layer = RowShardedInplace(cfg, x["W0"])
+    else:
+        c0, c1 = shard_range(spec.T // spec.C, rank, world)
+        x["Z"], x["Vhat"] = x["Z"][c0 * spec.C:c1 * spec.C].contiguous(), x["Vhat"][c0 * spec.C:c1 * spec.C].contiguous()
+        layer = SequenceShardedInplace(cfg, x["W0"])
     for _ in range(a.warmup):
         layer.scan(x["Z"], x["Vhat"])
     torch.cuda.synchronize()
@@ -848,7 +856,7 @@ def run_row_sharded(spec, a, world, rank, local, peaks):
     w = work(spec)
     # End to end: inputs copied from pinned host memory, the sharded scan, the gathered output read back.
     hZ, hV = x["Z"].cpu().pin_memory(), x["Vhat"].cpu().pin_memory()
-    hO = torch.empty((spec.T, spec.d), dtype=torch.bfloat16).pin_memory()
+    hO = torch.empty((x["Z"].shape[0] if a.shard == "sequence" else spec.T, spec.d), dtype=torch.bfloat16).pin_memory()
     t = []
     for k in range(3):
         torch.cuda.synchronize()
@@ -868,7 +876,7 @@ def run_row_sharded(spec, a, world, rank, local, peaks):
             "metric": METRIC, "value": w["tokens"] / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world,
             "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "strong",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": dict(bench_config(spec, world), parallelism=f"rows{world}",
+            "config": dict(bench_config(spec, world), parallelism=f"{'rows' if a.shard == 'rows' else 'sequence'}{world}",
                            l2="inputs larger than L2 (one step moves over 1 GB)"),
             "tflops": w["flops"] / (ms * 1e-3) / 1e12, "roofline": rl,
             "e2e": {"value": w["tokens"] / (e2e_ms * 1e-3), "unit": "tokens/s",
@@ -942,10 +950,12 @@ def main():
     ap.add_argument("--tokens", type=int, default=None,
                     help="run the named workload with this many tokens instead (same widths and chunk; a smaller "
                          "case for profilers, not a bench line)")
-    ap.add_argument("--shard", choices=["replicas", "rows"], default="replicas",
+    ap.add_argument("--shard", choices=["replicas", "rows", "sequence"], default="replicas",
                     help="with N ranks: 'replicas' (default) runs an independent copy of the workload per rank "
                          "(weak scaling); 'rows' splits one In-Place layer's Wdown rows over the ranks and "
-                         "all-gathers the output columns each step (strong scaling; In-Place workloads)")
+                         "all-gathers the output columns each step; 'sequence' gives each rank its own chunks of the "
+                         "sequence and all-gathers the ranks' delta sums each step (strong scaling; In-Place "
+                         "workloads)")
     ap.add_argument("--form", choices=["scan", "prefix", "docs", "cache_read", "packed"], default="scan",
                     help="with --profile: the further form to run (the context-parallel In-Place scan, the packed "
                          "In-Place scan or packed TTT-Linear on the named workload's inputs, the cache read path)")
@@ -1008,7 +1018,7 @@ def main():
 
     if a.warmup < 3:
         a.warmup = 3
-    if a.shard == "rows":
+    if a.shard in ("rows", "sequence"):
         run_row_sharded(spec, a, world, rank, local, peaks)
         return
     torch.cuda.set_device(local)
