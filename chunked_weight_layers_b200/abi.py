@@ -35,6 +35,7 @@ TTT_OPT_WAIT_LIMIT_NS = 2
 TTT_OPT_INJECT_STALL = 3
 TTT_OPT_INPLACE_PREFIX = 4
 TTT_OPT_SM_PAIR = 5
+TTT_OPT_GATE_TOKENS = 6
 
 
 class ttt_config(ctypes.Structure):

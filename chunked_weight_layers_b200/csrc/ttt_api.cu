@@ -6,6 +6,7 @@
 #include <string.h>
 
 #include <numeric>
+#include <vector>
 
 #include "common.cuh"
 #include "internal.h"
@@ -767,6 +768,18 @@ ttt_status ttt_state_set_option(ttt_state* st, int32_t option, int64_t value) {
       if (value != 0 && value != 1) return fail(TTT_ERR_INVALID_ARG, "TTT_OPT_INJECT_STALL must be 0 or 1");
       st->inject_stall = (int)value;
       return TTT_OK;
+    case TTT_OPT_GATE_TOKENS: {
+      if (st->cfg.rule == TTT_RULE_INPLACE_HEBBIAN || st->gate.tokens == nullptr)
+        return fail(TTT_ERR_UNSUPPORTED, "TTT_OPT_GATE_TOKENS applies to TTT-Linear states");
+      if (value < 0 || value > (int64_t)INT32_MAX)
+        return fail(TTT_ERR_INVALID_ARG, "TTT_OPT_GATE_TOKENS must lie in [0, 2^31 - 1]");
+      TTT_TRY(check_device(st));
+      const size_t bh = (size_t)st->cfg.batch * st->cfg.heads;
+      std::vector<int64_t> v(bh, value);
+      TTT_CUDA(cudaDeviceSynchronize());
+      TTT_CUDA(cudaMemcpy(st->gate.tokens, v.data(), bh * sizeof(int64_t), cudaMemcpyHostToDevice));
+      return TTT_OK;
+    }
     default:
       return fail(TTT_ERR_INVALID_ARG, "unknown option %d", option);
   }

@@ -384,7 +384,13 @@ typedef enum {
    * always uses single SMs. Both give the same results up to the order of fp32 additions
    * inside the tensor cores. Changing it rebuilds the state's tile schedules on the next scan
    * (the call synchronises the device). Other states ignore it. */
-  TTT_OPT_SM_PAIR = 5
+  TTT_OPT_SM_PAIR = 5,
+  /* Tests of the device-side check of the gate's token position: sets the count of tokens
+   * gated since the reset, held on the device per (sequence, head), to `value` for every
+   * (sequence, head), leaving the host's own count alone, as replays of a captured call do.
+   * Range [0, 2^31 − 1]; synchronises the device. TTT-Linear states only (UNSUPPORTED
+   * otherwise). */
+  TTT_OPT_GATE_TOKENS = 6
 } ttt_option;
 
 /* Set option `option` of state `st` to `value`. Takes effect from the next call that

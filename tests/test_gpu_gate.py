@@ -223,3 +223,49 @@ def test_percentile_ranks_and_nans_bit_exact(cwl, pct):
     ref = ogate.GateState(B, H, 256)
     ogate.surprisal_route(L, ref, pct=pct)
     assert_same_as_oracle(*read_gate(st, B, H, 256), ref)
+
+
+def test_token_position_is_kept_and_checked_on_the_device(cwl):
+    """The gate's token position lives on the device (so replays of captured calls advance it):
+    set there to 1000, a scan's routed positions are those of a fresh state plus 1000, and the
+    cache read then wants T = 1256 (found on the device: the host counted 256); set near 2^31,
+    a scan that passes 2^31 - 1 is reported by ttt_state_poll."""
+    from chunked_weight_layers_b200 import TTTError, abi
+    spec = workloads.scaled(workloads.SR_TTT_GATE, B=1, H=2, T=256, with_queries=True, seed=531)
+    x = workloads.linear_inputs(spec, device="cuda")
+    cfg = cwl.config("linear", batch=1, heads=2, chunk=16, eta=spec.eta, gate_enable=1)
+
+    def run(base):
+        st = cwl.FastWeightState(cfg, x["W0"])
+        if base is not None:
+            st.set_option(abi.TTT_OPT_GATE_TOKENS, base)
+        O = torch.empty_like(x["K"])
+        st.chunk_scan(x["K"], x["V"], x["Q"], out=O, loss_out=torch.empty((1, 2, spec.T), device="cuda"))
+        E = torch.empty((1, 2, 256, 3), device="cuda", dtype=torch.int32)
+        C = torch.empty((1, 2, 2), device="cuda", dtype=torch.int32)
+        st.cache_read(E, C)
+        torch.cuda.synchronize()
+        return st, O, E.cpu(), C.cpu()
+
+    st0, _, E0, C0 = run(None)
+    st0.poll()
+    st1, O1, E1, C1 = run(1000)
+    st1.poll()
+    assert torch.equal(C0, C1)
+    valid = E0[..., 2] >= 0
+    assert torch.equal(E1[..., 2][valid], E0[..., 2][valid] + 1000)
+    assert torch.equal(E1[..., :2], E0[..., :2])
+    alpha = torch.full((2, 64), 0.5, device="cuda")
+    st1.cache_attention(x["Q"], x["K"], x["V"], O1, alpha, out=torch.empty_like(O1))
+    with pytest.raises(TTTError) as e:
+        st1.poll()
+    assert e.value.status == abi.TTT_ERR_INVALID_ARG
+    st2, _, _, _ = run(2**31 - 64)
+    with pytest.raises(TTTError) as e:
+        st2.poll()
+    assert e.value.status == abi.TTT_ERR_UNSUPPORTED
+    st2.poll()  # the record was cleared
+    with pytest.raises(TTTError) as e:
+        cwl.FastWeightState(cwl.config("inplace", io_dtype=1, d_key=128, d_val=128, chunk=128),
+                            torch.zeros((128, 128), device="cuda")).set_option(abi.TTT_OPT_GATE_TOKENS, 5)
+    assert e.value.status == abi.TTT_ERR_UNSUPPORTED
