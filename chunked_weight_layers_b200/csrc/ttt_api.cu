@@ -8,6 +8,8 @@
 #include <numeric>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -432,6 +434,15 @@ static ttt_status copy_segment(void* dst, const void* src, size_t width, int64_t
   return TTT_OK;
 }
 
+// A named NVTX range around each call that enqueues a scan, so a timeline tool shows the
+// library's calls beside their kernels (no cost without such a tool attached).
+struct CallRange {
+  explicit CallRange(const char* name) { nvtxRangePushA(name); }
+  ~CallRange() { nvtxRangePop(); }
+  CallRange(const CallRange&) = delete;
+  CallRange& operator=(const CallRange&) = delete;
+};
+
 }  // namespace ttt
 
 using namespace ttt;
@@ -476,12 +487,14 @@ ttt_status ttt_state_create(const ttt_config* cfg, const void* W0, const void* W
 
 ttt_status ttt_chunk_scan(ttt_state* st, const void* keys, const void* targets, const void* queries, int64_t T,
                           void* out, float* loss_out, ttt_stream stream) {
+  const CallRange range("ttt_chunk_scan");
   if (st == nullptr) return fail(TTT_ERR_INVALID_ARG, "state is NULL");
   return scan_impl(st, keys, targets, queries, T, out, loss_out, reinterpret_cast<cudaStream_t>(stream));
 }
 
 ttt_status ttt_chunk_scan_docs(ttt_state* st, const void* keys, const void* targets, int64_t T, void* out,
                                const int64_t* doc_starts, int32_t ndocs, float clip_norm, ttt_stream stream) {
+  const CallRange range("ttt_chunk_scan_docs");
   if (st == nullptr) return fail(TTT_ERR_INVALID_ARG, "state is NULL");
   const ttt_config& c = st->cfg;
   if (c.rule != TTT_RULE_INPLACE_HEBBIAN || c.io_dtype != TTT_BF16)
@@ -507,6 +520,7 @@ ttt_status ttt_chunk_scan_docs(ttt_state* st, const void* keys, const void* targ
 ttt_status ttt_chunk_scan_packed(ttt_state* st, const void* keys, const void* targets, const void* queries, int64_t T,
                                  void* out, float* loss_out, const int64_t* doc_starts, const int32_t* docs_per_seq,
                                  ttt_stream stream) {
+  const CallRange range("ttt_chunk_scan_packed");
   if (st == nullptr) return fail(TTT_ERR_INVALID_ARG, "state is NULL");
   const ttt_config& c = st->cfg;
   if (c.rule == TTT_RULE_INPLACE_HEBBIAN)
@@ -542,6 +556,7 @@ ttt_status ttt_chunk_scan_packed(ttt_state* st, const void* keys, const void* ta
 
 ttt_status ttt_chunk_scan_host(ttt_state* st, const void* keys, const void* targets, const void* queries,
                                int64_t T, void* out, float* loss_out, ttt_stream stream) {
+  const CallRange range("ttt_chunk_scan_host");
   if (st == nullptr) return fail(TTT_ERR_INVALID_ARG, "state is NULL");
   const ttt_config& c = st->cfg;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -614,6 +629,7 @@ ttt_status ttt_chunk_scan_host(ttt_state* st, const void* keys, const void* targ
 }
 
 ttt_status ttt_surprisal_route(ttt_state* st, const float* loss, int64_t T, ttt_stream stream) {
+  const CallRange range("ttt_surprisal_route");
   if (st == nullptr) return fail(TTT_ERR_INVALID_ARG, "state is NULL");
   if (st->cfg.rule != TTT_RULE_LINEAR_GD) return fail(TTT_ERR_UNSUPPORTED, "the surprisal gate runs on TTT-Linear states");
   if (!st->cfg.gate_enable) return fail(TTT_ERR_INVALID_ARG, "the state was created with gate_enable = 0");
@@ -627,6 +643,7 @@ ttt_status ttt_surprisal_route(ttt_state* st, const float* loss, int64_t T, ttt_
 
 ttt_status ttt_cache_attention(const ttt_state* st, const void* queries, const void* keys, const void* values,
                                const void* o_ttt, const float* alpha, int64_t T, void* out, ttt_stream stream) {
+  const CallRange range("ttt_cache_attention");
   if (st == nullptr) return fail(TTT_ERR_INVALID_ARG, "state is NULL");
   if (st->cfg.rule != TTT_RULE_LINEAR_GD || !st->cfg.gate_enable)
     return fail(TTT_ERR_UNSUPPORTED, "the cache read path needs a TTT-Linear state with the gate enabled");
@@ -647,6 +664,7 @@ ttt_status ttt_cache_attention(const ttt_state* st, const void* queries, const v
 }
 
 ttt_status ttt_state_reset(ttt_state* st, ttt_stream stream) {
+  const CallRange range("ttt_state_reset");
   if (st == nullptr) return fail(TTT_ERR_INVALID_ARG, "state is NULL");
   TTT_TRY(check_device(st));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
