@@ -401,9 +401,9 @@ static ttt_status ensure_pipeline(ttt_state* st) {
 // of one busy while the scan of another runs), in whole units of what a call may end on (the
 // chunk; the gate's 64-token chunk when the gate is on). The whole call where a call boundary
 // would change the result (the fused target's taps past the call end, pad mode 1), and for the
-// TTT-Linear family when it copies back less than a fifth of what it copies in: a segment of
-// [batch, heads, T, 64] tensors is a strided copy, which measured ~15 % slower over PCIe than
-// a plain one, more than overlapping the small copy back (the losses alone) gains.
+// TTT-Linear family when it copies back less than a fifth of what it copies in: its scan is
+// short next to the copies, so with only the losses coming back there is almost nothing for
+// the segments to overlap, and each segment costs launches and strided copies of its own.
 static int64_t host_segment(const ttt_config& c, int64_t T, size_t in_bytes, size_t out_bytes) {
   if (c.rule == TTT_RULE_INPLACE_HEBBIAN && c.target_mode == 1 && c.conv_pad_mode == 1) return T;
   if (c.rule != TTT_RULE_INPLACE_HEBBIAN && 5 * out_bytes < in_bytes) return T;
